@@ -1,0 +1,174 @@
+"""CPU oracle for the NVFP4 quantize / fake-quantize path -- TEST INFRASTRUCTURE ONLY.
+
+Thin numpy/ctypes wrapper around ``nvfp4_oracle.c`` (plain scalar C, fp32 IEEE with one
+rounding per operation).  Only the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import this package; the GPU library never uses it and
+shares no code with it.
+
+Tensors are passed as numpy arrays of raw bits: bf16 as ``uint16``, packed nibbles,
+and E4M3 scale bytes as ``uint8``.  Sources cited in the C file: fp4_optimization.py
+(VideoX-Fun) for the quantize / dequantize math, and the verl ``linear.py`` tutorial
+for the fake-quant, STE, sibling fusion and activation observers.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from .build import build_oracle
+
+_LIB = None
+
+STATIC_MINMAX = 0
+EMA = 1
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        # NVFP4_ORACLE_LIB points at another build of the same source; the mutation test
+        # uses it to check that the pins reject deliberately broken copies of the oracle.
+        path = os.environ.get("NVFP4_ORACLE_LIB") or build_oracle()
+        lib = ctypes.CDLL(path)
+        u16p = ctypes.POINTER(ctypes.c_uint16)
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        i64 = ctypes.c_int64
+        f32 = ctypes.c_float
+        lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16_to_f32.restype = f32
+        lib.oracle_f32_to_bf16.argtypes = [f32]
+        lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_decode.restype = f32
+        lib.oracle_e4m3_encode.argtypes = [f32]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_e2m1_round_index.argtypes = [f32]
+        lib.oracle_e2m1_round_index.restype = ctypes.c_int
+        lib.oracle_e2m1_lut.argtypes = [ctypes.c_int]
+        lib.oracle_e2m1_lut.restype = f32
+        lib.oracle_amax.argtypes = [u16p, i64]
+        lib.oracle_amax.restype = f32
+        lib.oracle_amax_multi.argtypes = [ctypes.POINTER(u16p), ctypes.POINTER(i64), ctypes.c_int]
+        lib.oracle_amax_multi.restype = f32
+        lib.oracle_global_scale.argtypes = [f32]
+        lib.oracle_global_scale.restype = f32
+        lib.oracle_quantize.argtypes = [u16p, i64, i64, f32, u8p, u8p]
+        lib.oracle_quantize.restype = None
+        lib.oracle_dequantize.argtypes = [u8p, u8p, f32, i64, i64, u16p]
+        lib.oracle_dequantize.restype = None
+        lib.oracle_fake_quant.argtypes = [u16p, i64, i64, f32, u16p]
+        lib.oracle_fake_quant.restype = ctypes.c_int
+        lib.oracle_observer_update.argtypes = [f32, f32, ctypes.c_int, ctypes.c_double]
+        lib.oracle_observer_update.restype = f32
+        _LIB = lib
+    return _LIB
+
+
+def _u16(a):
+    a = np.ascontiguousarray(a, dtype=np.uint16)
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16))
+
+
+def _u8(a):
+    a = np.ascontiguousarray(a, dtype=np.uint8)
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
+
+
+def f32(v) -> float:
+    """Round a Python number to the nearest fp32 and return it as a Python float."""
+    return float(np.float32(v))
+
+
+# ---- scalar codecs ------------------------------------------------------------------
+
+def bf16_to_f32(bits):
+    bits = np.asarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16(values):
+    """Round fp32 values to bf16 bits, one at a time through the oracle."""
+    v = np.asarray(values, dtype=np.float32).ravel()
+    lib = _lib()
+    out = np.array([lib.oracle_f32_to_bf16(float(x)) for x in v], dtype=np.uint16)
+    return out.reshape(np.shape(values))
+
+
+def e4m3_decode(codes):
+    lib = _lib()
+    c = np.asarray(codes, dtype=np.uint8).ravel()
+    return np.array([lib.oracle_e4m3_decode(int(x)) for x in c], dtype=np.float32).reshape(np.shape(codes))
+
+
+def e4m3_encode(values):
+    lib = _lib()
+    v = np.asarray(values, dtype=np.float32).ravel()
+    return np.array([lib.oracle_e4m3_encode(float(x)) for x in v], dtype=np.uint8).reshape(np.shape(values))
+
+
+def e2m1_round_index(values):
+    lib = _lib()
+    v = np.asarray(values, dtype=np.float32).ravel()
+    return np.array([lib.oracle_e2m1_round_index(float(x)) for x in v], dtype=np.int32).reshape(np.shape(values))
+
+
+def e2m1_lut(code: int) -> float:
+    return _lib().oracle_e2m1_lut(int(code))
+
+
+# ---- the method -----------------------------------------------------------------------
+
+def amax(x_bits) -> float:
+    a, p = _u16(x_bits)
+    return _lib().oracle_amax(p, a.size)
+
+
+def amax_multi(xs_bits) -> float:
+    arrs = [_u16(x) for x in xs_bits]
+    u16p = ctypes.POINTER(ctypes.c_uint16)
+    ptrs = (u16p * len(arrs))(*[p for _, p in arrs])
+    ns = (ctypes.c_int64 * len(arrs))(*[a.size for a, _ in arrs])
+    return _lib().oracle_amax_multi(ptrs, ns, len(arrs))
+
+
+def global_scale(amax_value: float) -> float:
+    return _lib().oracle_global_scale(f32(amax_value))
+
+
+def quantize(x_bits, global_scale_value: float):
+    """x_bits: uint16 [M, N] (N % 16 == 0).  Returns (packed [M, N/2], scales [M, N/16])."""
+    a, p = _u16(x_bits)
+    M, N = a.shape
+    packed = np.empty((M, N // 2), dtype=np.uint8)
+    scales = np.empty((M, N // 16), dtype=np.uint8)
+    _lib().oracle_quantize(p, M, N, f32(global_scale_value),
+                           packed.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+                           scales.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    return packed, scales
+
+
+def dequantize(packed, scales, global_scale_value: float, M: int, N: int):
+    pk, pp = _u8(packed)
+    sc, sp = _u8(scales)
+    y = np.empty((M, N), dtype=np.uint16)
+    _lib().oracle_dequantize(pp, sp, f32(global_scale_value), M, N,
+                             y.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)))
+    return y
+
+
+def fake_quant(x_bits, amax_value: float):
+    a, p = _u16(x_bits)
+    M, N = a.shape
+    y = np.empty((M, N), dtype=np.uint16)
+    rc = _lib().oracle_fake_quant(p, M, N, f32(amax_value), y.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)))
+    if rc != 0:
+        raise MemoryError("oracle_fake_quant could not allocate its temporaries")
+    return y
+
+
+def observer_update(state: float, cur: float, kind: int, decay: float = 0.01) -> float:
+    return _lib().oracle_observer_update(f32(state), f32(cur), int(kind), float(decay))
+
+
+def library_path() -> str:
+    return os.path.abspath(build_oracle())
