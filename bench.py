@@ -1,0 +1,379 @@
+#!/usr/bin/env python
+"""Throughput of the NVFP4 quantize / fake-quant hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+One step is one pass of the whole path over one batch: the activation observer
+(global amax + EMA update; with N > 1 ranks the amax is MAX-all-reduced over NCCL
+first, as a data-parallel QAT step does), fake-quant with the observed amax, quantize
+to packed E2M1 codes + E4M3 scales, and dequantize back to bf16.  Every rank owns its
+own bf16 [65536, 8192] activation (1 GiB, N(0,1)), so the work per GPU is fixed
+(weak scaling).  ``value`` is the algorithmic bytes of all ranks' steps divided by the
+slowest rank's device time, in GB/s.
+
+Rank 0 prints one JSON line.  The native arm also reports the dominant kernel's
+roofline, the CPU oracle's throughput on a bounded sample (cpu_baseline), an
+end-to-end figure with host buffers (e2e), the SM clocks seen during the timed region
+and the number of library kernels launched.  ``--impl reference`` times the CPU oracle
+instead (the reference arm), on a bounded sample of the same workload.
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 fake-quant/quantize GB/s and fraction of B200 HBM roofline"
+UNIT = "GB/s"
+# Algorithmic (minimal) bytes per element of each kernel of the step.
+KERNEL_BYTES = {"amax": 2.0, "fake_quant": 4.0, "quantize": 2.0 + 0.5 + 1.0 / 16, "dequantize": 0.5 + 1.0 / 16 + 2.0}
+STEP_BYTES = sum(KERNEL_BYTES.values())  # 11.125 bytes per element
+FALLBACK_HBM_GBS = 6650.0
+CSRC = os.path.join(ROOT, "qat_nvfp4_b200", "csrc")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["native", "reference"], default="native")
+    p.add_argument("--rows", type=int, default=65536)
+    p.add_argument("--cols", type=int, default=8192)
+    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--cpu-rows", type=int, default=2048, help="rows of the oracle sample (cpu_baseline)")
+    p.add_argument("--skip-e2e", action="store_true")
+    p.add_argument("--skip-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def workload_config(args, world):
+    return {
+        "workload": f"bf16 activation {args.rows}x{args.cols} ~ N(0,1) per GPU; step = EMA(0.01) observer amax"
+                    f"{' + NCCL MAX all-reduce' if world > 1 else ''} -> fake-quant -> quantize -> dequantize",
+        "shape": [args.rows, args.cols],
+        "bytes_per_elem_per_step": STEP_BYTES,
+        "l2": "inputs larger than L2 (1 GiB per GPU vs 126 MB), no flush" if args.rows * args.cols * 2 > (256 << 20)
+              else "inputs smaller than 2x L2: L2-warm figures",
+        "parallelism": f"dp{world}",
+    }
+
+
+def source_digest():
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(CSRC)):
+        with open(os.path.join(CSRC, fn), "rb") as f:
+            h.update(fn.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, burst copy)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback (earlier measurement on this pool)"
+
+
+def stored_traffic(kernel, numel):
+    """dram bytes per launch from the committed ncu summary, scaled to `numel` elements,
+    or None if there is none or the kernel sources changed since it was taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)[kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    if t.get("source_sha256") != source_digest():
+        return None
+    return t["dram_bytes_per_elem"] * numel
+
+
+# ---------------------------------------------------------------------------------------
+# Clocks during the timed region (NVML, polled from a thread).
+
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index, period_s=0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 - report, never fail the bench on telemetry
+            self.nvml, self.error = None, str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def _sample(self):
+        try:
+            self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.handle, self.nvml.NVML_CLOCK_SM))
+            mask = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+            self.reasons |= {n for n, b in self.REASONS.items() if mask & b}
+        except Exception:  # noqa: BLE001
+            pass
+
+    def start(self):
+        if self.nvml:
+            self._sample()
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self.nvml and self._thread:
+            self._stop.set()
+            self._thread.join()
+            self._sample()
+
+    def summary(self):
+        if not self.nvml:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "")}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------------
+# The CPU oracle step (cpu_baseline and the reference arm).
+
+def oracle_step(x_bits, state=-1.0):
+    import oracle
+    a = oracle.amax(x_bits)
+    s = oracle.observer_update(state, a, oracle.EMA, 0.01)
+    oracle.fake_quant(x_bits, s)
+    gs = oracle.global_scale(s)
+    packed, scales = oracle.quantize(x_bits, gs)
+    oracle.dequantize(packed, scales, gs, *x_bits.shape)
+    return s
+
+
+def time_oracle(x_bits, repeats=1):
+    t0 = time.perf_counter()
+    for _ in range(repeats):
+        oracle_step(x_bits)
+    return (time.perf_counter() - t0) / repeats
+
+
+# ---------------------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from qat_nvfp4_b200 import synthetic
+    cols = args.cols
+    # size the sample so that warm-up + steps end in about two minutes
+    probe = synthetic.activation_normal((16, cols), seed=12)
+    per_row = time_oracle(probe) / 16
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    rows = int(max(8, min(args.rows, budget / per_row)))
+    x = synthetic.activation_normal((rows, cols), seed=12)
+    for _ in range(args.warmup):
+        oracle_step(x)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(x)
+    elapsed = time.perf_counter() - t0
+    value = STEP_BYTES * rows * cols * args.steps / elapsed / 1e9
+    sample = (f"first {rows} of {args.rows} rows x {cols} (one oracle step per timed step: amax, EMA observer, "
+              f"fake-quant, quantize, dequantize), single thread")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(args, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    from qat_nvfp4_b200 import nvfp4 as nv
+    from qat_nvfp4_b200 import synthetic
+
+    M, N = args.rows, args.cols
+    numel = M * N
+    x = synthetic.activation_normal_device((M, N), seed=5 + 7 + 1000 * rank, device=dev)
+    y = torch.empty_like(x)
+    y2 = torch.empty_like(x)
+    packed = torch.empty((M, N // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((M, N // 16), dtype=torch.uint8, device=dev)
+    gs = torch.empty(1, dtype=torch.float32, device=dev)
+    cur = torch.empty(1, dtype=torch.float32, device=dev)
+    state = torch.full((1,), -1.0, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    stages = ["amax", "fake_quant", "quantize", "dequantize"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        if world == 1:
+            nv.nvfp4_observe_amax(x, state, kind="minmax", decay=0.01, cur_out=cur)
+        else:
+            nv.nvfp4_amax(x, out=cur)
+            dist.all_reduce(cur, op=dist.ReduceOp.MAX)
+            nv.nvfp4_observer_update(state, cur, kind="minmax", decay=0.01)
+        mark(1)
+        nv.nvfp4_fake_quant(x, state, out=y)
+        mark(2)
+        nv.nvfp4_quantize(x, state, packed, scales, gs)
+        mark(3)
+        nv.nvfp4_dequantize(packed, scales, gs, out=y2)
+        mark(4)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return t.item()
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier()
+    launches0 = nv.nvfp4_kernel_launch_count()
+    sampler.start()
+    start.record(stream)
+    for k in range(args.steps):
+        step(events[k])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.stop()
+    launches = nv.nvfp4_kernel_launch_count() - launches0
+    barrier()
+    elapsed_ms = max_over_ranks(start.elapsed_time(end))
+    stage_ms = {s: statistics.fmean(events[k][i].elapsed_time(events[k][i + 1]) for k in range(args.steps))
+                for i, s in enumerate(stages)}
+    stage_ms = {s: max_over_ranks(v) for s, v in stage_ms.items()}
+
+    value = world * args.steps * numel * STEP_BYTES / (elapsed_ms / 1e3) / 1e9
+    peak, peak_src = hbm_peak()
+    kernels = {s: {"ms": stage_ms[s], "GB/s": numel * KERNEL_BYTES[s] / (stage_ms[s] / 1e3) / 1e9,
+                   "bytes_per_elem": KERNEL_BYTES[s]} for s in stages}
+    for s in stages:
+        kernels[s]["frac_of_hbm_peak"] = kernels[s]["GB/s"] / peak
+    fq = kernels["fake_quant"]
+    roofline = {"bound": "hbm", "kernel": "fake_quant_kernel", "achieved": fq["GB/s"], "peak": peak,
+                "unit": "GB/s", "frac": fq["GB/s"] / peak, "traffic": stored_traffic("fake_quant", numel),
+                "algorithmic_bytes_per_launch": numel * KERNEL_BYTES["fake_quant"], "peak_source": peak_src}
+
+    # ---- end to end with host buffers: H2D of x, the step, D2H of every output ----
+    e2e = None
+    if not args.skip_e2e:
+        x_h = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+        x_h.copy_(x)
+        outs = [(y, torch.empty_like(y, device="cpu", pin_memory=True)),
+                (y2, torch.empty_like(y2, device="cpu", pin_memory=True)),
+                (packed, torch.empty_like(packed, device="cpu", pin_memory=True)),
+                (scales, torch.empty_like(scales, device="cpu", pin_memory=True)),
+                (gs, torch.empty_like(gs, device="cpu", pin_memory=True)),
+                (state, torch.empty_like(state, device="cpu", pin_memory=True))]
+
+        def e2e_step():
+            x.copy_(x_h, non_blocking=True)
+            step()
+            for d, h in outs:
+                h.copy_(d, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+        d2h = sum(d.numel() * d.element_size() for d, _ in outs)
+        e2e = {"value": world * args.e2e_steps * numel * STEP_BYTES / (e2e_ms / 1e3) / 1e9, "unit": UNIT,
+               "h2d_bytes_per_step": numel * 2, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "ms_per_step": e2e_ms / args.e2e_steps}
+
+    # ---- the CPU oracle on a bounded sample (rank 0, one GPU only) ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        rows = min(args.cpu_rows, M)
+        sample = x[:rows].contiguous().view(torch.int16).cpu().numpy().view("uint16")
+        t = time_oracle(sample)
+        cpu = {"value": STEP_BYTES * rows * N / t / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"first {rows} of {M} rows x {N}: one oracle step (amax, EMA observer, fake-quant, "
+                         f"quantize, dequantize), single thread, {t:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(args, world), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches, "clocks": sampler.summary(), "kernels": kernels,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.cols % 16 or args.rows < 1:
+        raise SystemExit("--cols must be a multiple of 16 and --rows positive")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,167 @@
+/*
+ * nvfp4.h -- C ABI of libnvfp4.so: NVFP4 two-level block quantization and QAT
+ * fake-quantization on NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages), cited by title and section:
+ *   [FP4OPT]  VideoX-Fun, videox_fun/utils/fp4_optimization.py -- constants block,
+ *             _float4_round, quantize_weight_to_float4, dequantize_weight_from_float4.
+ *   [QATLIN]  verl code tutorial, "linear.py" (verl.utils.qat.linear) -- section 1 (Triton
+ *             FP4 fake-quant kernel), section 2 (straight-through estimator), section 4
+ *             (weight fake-quant with sibling fusion), section 5 (activation observers).
+ *
+ * Data model shared by every call:
+ *   - x is a bf16 tensor [M, N], row-major and contiguous (the last dimension is the
+ *     input-feature / hidden dimension).  Blocks are 16 consecutive elements of a row,
+ *     so N must be a multiple of 16 for the block calls.
+ *   - packed is uint8 [M, N/2], row-major: byte j of a row holds element 2j in its low
+ *     nibble and element 2j+1 in its high nibble.  A nibble is an E2M1 code,
+ *     magnitude index | sign << 3, magnitudes (0, 0.5, 1, 1.5, 2, 3, 4, 6).
+ *   - scales is uint8 [M, N/16], row-major: one E4M3 (float8_e4m3fn) byte per block, in
+ *     plain row order (not a swizzled GEMM layout).
+ *   - amax, global scale and observer state are single fp32 values in device memory.
+ *     global_scale = 2688 / max(amax, 1e-12) is the ENCODE scale of [FP4OPT].
+ *
+ * Conventions:
+ *   - Every pointer argument is DEVICE memory owned by the caller, except the arrays of
+ *     pointers and sizes passed to the *_multi / *_siblings calls, which are HOST arrays
+ *     read before the call returns.  The library allocates nothing and keeps no pointer.
+ *   - Every call is asynchronous and ordered on `stream` (NULL = the legacy default
+ *     stream).  It validates its arguments on the host first and returns an error code
+ *     with nothing launched; otherwise it enqueues its work and returns NVFP4_OK, or
+ *     NVFP4_ERR_CUDA if a launch failed (cudaGetLastError).  No call throws.
+ *   - Alignment: bf16 tensors 32 bytes, packed 8 bytes, fp32 scalars 4 bytes, scales 1.
+ *   - Results are bit-exact: every fp32 operation of the pages' formulas is one IEEE
+ *     round-to-nearest-even (no fast-math, no contraction of the formulas).
+ *   - Non-finite inputs are outside the method's domain; their outputs are unspecified.
+ *   - The calls are thread-safe; calls on different streams may run concurrently when
+ *     they touch disjoint outputs.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so this header needs no CUDA include. */
+typedef struct CUstream_st* nvfp4_stream_t;
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_NULL = 1,    /* a required pointer is NULL */
+    NVFP4_ERR_SHAPE = 2,   /* negative size, N % 16 != 0, or a size that overflows */
+    NVFP4_ERR_ALIGN = 3,   /* a pointer is not aligned as the conventions require */
+    NVFP4_ERR_ARG = 4,     /* any other invalid argument (kind, decay, k, overlap) */
+    NVFP4_ERR_CUDA = 5,    /* the CUDA runtime reported an error */
+    NVFP4_ERR_TIMEOUT = 6  /* a bounded device-side wait gave up */
+} nvfp4_status;
+
+typedef enum {
+    NVFP4_OBS_STATIC_MINMAX = 0, /* state = max(state, amax)            */
+    NVFP4_OBS_EMA = 1            /* state = (1-d)*state + d*amax ("minmax") */
+} nvfp4_observer;
+
+/* Largest number of tensors in one *_multi / *_siblings call. */
+#define NVFP4_MAX_SIBLINGS 16
+
+/* Global amax: *d_amax = max |x_i| over `numel` bf16 values, exactly (the bf16 maximum
+ * widened to fp32; no clamp -- the 1e-12 clamp is applied where the scale is formed).
+ * numel == 0 writes 0.  [FP4OPT] quantize_weight_to_float4 (global_amax = x.abs().amax());
+ * [QATLIN] section 4 (weight.abs().max()).
+ *   x       bf16 [numel], 32-byte aligned (may be NULL when numel == 0)
+ *   d_amax  fp32 out
+ * Enqueues a 4-byte memset and one kernel. */
+nvfp4_status nvfp4_amax(const void* x, int64_t numel, float* d_amax, nvfp4_stream_t stream);
+
+/* Fused-siblings amax: *d_amax = max over the k tensors of max |x|, so that layers fused
+ * into one GEMM (q/k/v) share one global scale.  [QATLIN] section 4
+ * (max(stack([m.weight.abs().max() for m in [self] + siblings]))).
+ *   xs      HOST array of k device pointers to bf16 data, each 32-byte aligned
+ *   numels  HOST array of k element counts (any >= 0)
+ *   k       1 .. NVFP4_MAX_SIBLINGS
+ *   d_amax  fp32 out
+ * Enqueues a 4-byte memset and one kernel over all k tensors. */
+nvfp4_status nvfp4_amax_multi(const void* const* xs, const int64_t* numels, int k, float* d_amax,
+                              nvfp4_stream_t stream);
+
+/* Activation observer step on an amax already computed (and, in data-parallel
+ * training, already MAX-reduced across ranks).  [QATLIN] section 5
+ * (_update_input_global_scale).  With s = *d_state and c = *d_cur_amax:
+ *   s < 0 (the -1 "not yet observed" buffer)  ->  s = c
+ *   NVFP4_OBS_STATIC_MINMAX                   ->  s = max(s, c)
+ *   NVFP4_OBS_EMA                             ->  s = fl(fl(k1 * s) + fl(k0 * c)),
+ *                                                  k0 = (float)decay, k1 = (float)(1 - decay)
+ * decay (EMA only) must be finite and in [0, 1]; 1 - decay is formed in double.
+ *   d_state     fp32 in/out     d_cur_amax  fp32 in
+ * Enqueues one single-thread kernel. */
+nvfp4_status nvfp4_observer_update(float* d_state, const float* d_cur_amax, nvfp4_observer kind,
+                                   double decay, nvfp4_stream_t stream);
+
+/* nvfp4_amax into d_cur_amax followed by nvfp4_observer_update: one observed activation
+ * on one GPU.  [QATLIN] section 5.  Fake-quantizing the activation with d_state as its
+ * amax afterwards uses the updated state.
+ *   x           bf16 [numel], 32-byte aligned
+ *   d_state     fp32 in/out     d_cur_amax  fp32 out (this step's amax)
+ * Enqueues a memset and two kernels. */
+nvfp4_status nvfp4_observe_amax(const void* x, int64_t numel, float* d_state, nvfp4_observer kind,
+                                double decay, float* d_cur_amax, nvfp4_stream_t stream);
+
+/* Quantize: bf16 [M, N] -> packed E2M1 codes [M, N/2] + E4M3 block scales [M, N/16] (+ the
+ * fp32 global scale).  [FP4OPT] quantize_weight_to_float4, with the amax given:
+ *   gs    = 2688 / max(*d_amax, 1e-12)
+ *   byte  = E4M3_rne_satfinite((block_amax / 6) * gs)
+ *   bs    = max(E4M3(byte) / gs, 1e-12)              (the dequantized block scale)
+ *   code  = E2M1 index of clamp(x / bs, -6, 6), ties to the even index, | 8 if < 0
+ *   x         bf16 [M, N], N % 16 == 0, 32-byte aligned
+ *   d_amax    fp32 in: the tensor's (or the siblings', or the observer's) amax
+ *   packed    uint8 out [M, N/2], 8-byte aligned
+ *   scales    uint8 out [M, N/16]
+ *   d_global_scale  fp32 out, may be NULL
+ * Enqueues one kernel. */
+nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
+                            uint8_t* scales, float* d_global_scale, nvfp4_stream_t stream);
+
+/* Dequantize: y = bf16_rne(LUT[code] * (E4M3(byte) / gs)), no clamp on this side.
+ * [FP4OPT] dequantize_weight_from_float4.
+ *   packed  uint8 [M, N/2], 8-byte aligned     scales  uint8 [M, N/16]
+ *   d_global_scale  fp32 in (as written by nvfp4_quantize)
+ *   y       bf16 out [M, N], 32-byte aligned
+ * Enqueues one kernel. */
+nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* scales, const float* d_global_scale,
+                              int64_t M, int64_t N, void* y, nvfp4_stream_t stream);
+
+/* Fake-quantize, bf16 -> bf16: y = dequantize(quantize(x)) bit for bit, in one pass with
+ * no codes written to memory -- the forward of the straight-through estimator ([QATLIN]
+ * sections 1 and 2; formulas of [FP4OPT]).  The STE backward is the identity and has no
+ * kernel.
+ *   x, y    bf16 [M, N], N % 16 == 0, 32-byte aligned; y == x (in place) is allowed,
+ *           any other overlap is NVFP4_ERR_ARG
+ *   d_amax  fp32 in
+ * Enqueues one kernel. */
+nvfp4_status nvfp4_fake_quant(const void* x, void* y, int64_t M, int64_t N, const float* d_amax,
+                              nvfp4_stream_t stream);
+
+/* Fused siblings: the shared amax of k tensors, then each one fake-quantized with it.
+ * [QATLIN] section 4 (fusion mode) followed by sections 1-2.
+ *   xs, ys  HOST arrays of k device pointers (bf16, 32-byte aligned; ys[j] == xs[j] allowed)
+ *   Ms, Ns  HOST arrays of k sizes, each Ns[j] % 16 == 0
+ *   k       1 .. NVFP4_MAX_SIBLINGS
+ *   d_shared_amax  fp32 out: the shared amax that was used
+ * Enqueues a memset and two kernels (one amax launch and one fake-quant launch over all
+ * k tensors). */
+nvfp4_status nvfp4_fake_quant_siblings(int k, const void* const* xs, void* const* ys, const int64_t* Ms,
+                                       const int64_t* Ns, float* d_shared_amax, nvfp4_stream_t stream);
+
+/* Human-readable name of a status code (a static string). */
+const char* nvfp4_status_string(nvfp4_status status);
+
+/* Number of kernels this library has launched in this process (memsets not counted). */
+uint64_t nvfp4_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */

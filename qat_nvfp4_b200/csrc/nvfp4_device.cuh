@@ -1,0 +1,212 @@
+// nvfp4_device.cuh -- device-side building blocks of the NVFP4 kernels (sm_100a).
+//
+// Everything here works on one 16-element block held by one thread: eight 32-bit words,
+// word i holding elements 2i (low half) and 2i+1 (high half) as bf16.  The arithmetic
+// follows fp4_optimization.py (VideoX-Fun), quantize_weight_to_float4 and
+// dequantize_weight_from_float4, with every fp32 operation a single IEEE
+// round-to-nearest-even (explicit __f*_rn intrinsics, so nothing is contracted).
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace nvfp4 {
+
+constexpr int kBlockElems = 16;     // NVFP4 block: 16 elements along the row
+constexpr int kBlockBytesIn = 32;   // one block of bf16
+constexpr int kBlockBytesPacked = 8;
+
+// clamp(min=1e-12) of an fp32 tensor: the fp32 nearest to 1e-12 (0x2B8CBCCC).
+constexpr float kTinyClamp = 1e-12f;
+// FLOAT8_E4M3_MAX * FLOAT4_MAX = 448 * 6.
+constexpr float kGlobalNumerator = 2688.0f;
+
+// ---------------------------------------------------------------------------------------
+// Global memory access.  32-byte vector accesses are native on sm_100.  The loads are
+// volatile asm so that the order written in the kernels (all loads of an unrolled group
+// first, then the math and the stores) is the order issued.
+
+__device__ __forceinline__ void ld_b256(const void* p, uint32_t (&w)[8]) {
+    asm volatile("ld.global.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]),
+                   "=r"(w[7])
+                 : "l"(p));
+}
+
+// Read-only variant (the data is not written by the same kernel).
+__device__ __forceinline__ void ld_b256_ro(const void* p, uint32_t (&w)[8]) {
+    asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]),
+                   "=r"(w[7])
+                 : "l"(p));
+}
+
+__device__ __forceinline__ void ld_b64_ro(const void* p, uint32_t& a, uint32_t& b) {
+    asm volatile("ld.global.nc.v2.b32 {%0,%1}, [%2];" : "=r"(a), "=r"(b) : "l"(p));
+}
+
+__device__ __forceinline__ uint32_t ld_u8_ro(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.u8 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_b256(void* p, const uint32_t (&w)[8]) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_b64(void* p, uint32_t a, uint32_t b) {
+    asm volatile("st.global.v2.b32 [%0], {%1,%2};" ::"l"(p), "r"(a), "r"(b) : "memory");
+}
+
+__device__ __forceinline__ void st_u8(void* p, uint32_t v) {
+    asm volatile("st.global.u8 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// ---------------------------------------------------------------------------------------
+// bf16 pairs
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// max(|a|, |b|) per bf16 lane (the sign of the result is the xor of the signs; callers
+// only use the magnitude).
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Exact block amax: the largest |x| of the 16 bf16 values, widened to fp32.
+__device__ __forceinline__ float block_amax(const uint32_t (&w)[8]) {
+    uint32_t m = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(w[0], w[1]), absmax_bf16x2(w[2], w[3])),
+                               absmax_bf16x2(absmax_bf16x2(w[4], w[5]), absmax_bf16x2(w[6], w[7])));
+    return fmaxf(fabsf(bf16_lo(m)), fabsf(bf16_hi(m)));
+}
+
+// ---------------------------------------------------------------------------------------
+// Format conversions (hardware cvt, checked against the CPU oracle by the parity tests)
+
+// fp32 -> E4M3 byte, round to nearest even, finite overflow saturated to +-448.
+__device__ __forceinline__ uint32_t e4m3_rne_satfinite(float v) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+    return r & 0xFFu;  // the second source lands in the low byte
+}
+
+// E4M3 byte -> fp32 (exact: every E4M3 value is an f16 value).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(code & 0xFFu)));
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+
+// Two fp32 values -> one byte of E2M1 codes (lo in bits 3:0, hi in bits 7:4), round to
+// nearest even onto {0, 0.5, 1, 1.5, 2, 3, 4, 6}, saturating beyond 6.  Nearest-even
+// on this grid is the pages' rule: ties go to the even magnitude index.  The sign bit
+// follows the sign of the value, including -0.0, so callers pass +0.0 for a zero.
+__device__ __forceinline__ uint32_t e2m1x2_rne(float lo, float hi) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(hi), "f"(lo));
+    return r;
+}
+
+// One byte of two E2M1 codes -> f16x2 (bits 3:0 -> low half), exact.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(r) : "r"(byte));
+    return r;
+}
+
+// ---------------------------------------------------------------------------------------
+// Scales
+
+// global_scale = 2688 / max(amax, 1e-12), one IEEE division.
+__device__ __forceinline__ float global_scale_of(float amax) {
+    return __fdiv_rn(kGlobalNumerator, fmaxf(amax, kTinyClamp));
+}
+
+// Everything the element loop needs about a block whose scale byte is `code`, given the
+// global scale gs.  There are only 127 finite non-negative E4M3 bytes, so each CTA builds
+// this table once instead of dividing per block:
+//   x = sq  = max(E4M3(code) / gs, 1e-12)   the dequantized block scale of the encode side
+//   y = rcp = the correctly rounded 1 / sq
+//   z = sd  = E4M3(code) / gs               the decode-side scale (no clamp)
+//   w = lim = 2^64 if sq < 2^16, else 0      (see encode_block: the fast-quotient guard)
+__device__ __forceinline__ float4 scale_entry(uint32_t code, float gs) {
+    float dec = (code == 0x7Fu) ? 448.0f : e4m3_to_f32(code);  // 0x7F (NaN) is never produced
+    float sd = __fdiv_rn(dec, gs);
+    float sq = fmaxf(sd, kTinyClamp);
+    float rcp = __frcp_rn(sq);
+    float lim = (sq < 65536.0f) ? 18446744073709551616.0f : 0.0f;
+    return make_float4(sq, rcp, sd, lim);
+}
+
+// ---------------------------------------------------------------------------------------
+// Element quotient x / sq.
+//
+// Only the E2M1 index of fl(x / sq) and whether fl(x / sq) is negative matter.  The
+// fast path forms the quotient from the per-block reciprocal with one refinement step
+// (Markstein's theorem: with y = RN(1/b) and q within one ulp of a/b, the residual
+// r = a - b*q is exact in an FMA and RN(q + r*y) = RN(a/b), as long as nothing
+// underflows or overflows).  encode_block takes it only when sq < 2^16 and
+// block_amax / sq < 2^64: then every quotient that can sit on or near an E2M1 boundary
+// (0.125 .. 8) has normal-range operands and residual, so its index is exact, every
+// other quotient stays on the same side of 0.25 and of zero, and x = +-0 gives +0.
+// Blocks outside the guard (enormous or saturated block scales, where a quotient may
+// underflow to a signed zero or overflow) take the IEEE division instead.
+__device__ __forceinline__ float quot_fast(float x, float sq, float rcp) {
+    float q0 = __fmul_rn(x, rcp);
+    float r = __fmaf_rn(-q0, sq, x);
+    return __fmaf_rn(r, rcp, q0);
+}
+
+// The pages' steps literally: IEEE division, clamp to [-6, 6], and +0.0 so that a zero
+// quotient of either sign encodes as code 0 (the sign bit is set only for q < 0).
+__device__ __forceinline__ float quot_exact(float x, float sq) {
+    float q = __fdiv_rn(x, sq);
+    q = fminf(fmaxf(q, -6.0f), 6.0f);
+    return __fadd_rn(q, 0.0f);
+}
+
+// Quantize one block: returns its E4M3 scale byte; codes[i] receives the byte of E2M1
+// codes of elements 2i (bits 3:0) and 2i+1 (bits 7:4); sd the decode-side scale.
+__device__ __forceinline__ uint32_t encode_block(const uint32_t (&w)[8], float gs, const float4* tab,
+                                                 uint32_t (&codes)[8], float& sd) {
+    const float b = block_amax(w);
+    const float v = __fmul_rn(__fdiv_rn(b, 6.0f), gs);
+    const uint32_t s8 = e4m3_rne_satfinite(v);
+    const float4 t = tab[s8 & 0x7Fu];  // s8 <= 0x7F always (v >= 0 or NaN); the mask only bounds the read
+    sd = t.z;
+    if (__fmul_rn(b, t.y) < t.w) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            codes[i] = e2m1x2_rne(quot_fast(bf16_lo(w[i]), t.x, t.y), quot_fast(bf16_hi(w[i]), t.x, t.y));
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            codes[i] = e2m1x2_rne(quot_exact(bf16_lo(w[i]), t.x), quot_exact(bf16_hi(w[i]), t.x));
+    }
+    return s8;
+}
+
+// Pack four code bytes into one little-endian word.
+__device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return a | (b << 8) | (c << 16) | (d << 24);
+}
+
+// Dequantize a byte of two codes: bf16_rne(LUT[code] * sd) for both, as one bf16x2 word.
+__device__ __forceinline__ uint32_t decode_pair(uint32_t code_byte, float sd) {
+    const uint32_t h2 = e2m1x2_to_f16x2(code_byte);
+    const float lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+    const float hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
+    __nv_bfloat162 r = __floats2bfloat162_rn(__fmul_rn(lo, sd), __fmul_rn(hi, sd));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+}  // namespace nvfp4

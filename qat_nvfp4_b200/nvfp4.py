@@ -1,0 +1,282 @@
+"""Python binding of libnvfp4.so (the C ABI in include/nvfp4.h).
+
+Argument marshalling only: each function checks dtypes, devices and contiguity, allocates
+outputs with torch when the caller does not pass them, and hands raw device pointers and
+the current CUDA stream to the library.  Every step of the computation runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback, and importing this module
+raises if the library has not been built (``python -m qat_nvfp4_b200.build``).
+
+Sources (web pages): fp4_optimization.py (VideoX-Fun) -- quantize_weight_to_float4,
+dequantize_weight_from_float4; the verl ``linear.py`` tutorial -- section 2 (the
+straight-through estimator), section 4 (sibling fusion), section 5 (observers).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Sequence
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build the CUDA library first "
+        "(python -m qat_nvfp4_b200.build, or __graft_entry__.build()).")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+MAX_SIBLINGS = 16
+STATIC_MINMAX = 0
+EMA = 1
+OBSERVERS = {"static_minmax": STATIC_MINMAX, "minmax": EMA, "ema": EMA}
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_status = ctypes.c_int
+
+
+def _sig(name, args, res=_status):
+    fn = getattr(_lib, name)
+    fn.argtypes = args
+    fn.restype = res
+    return fn
+
+
+_c_amax = _sig("nvfp4_amax", [_vp, _i64, _vp, _vp])
+_c_amax_multi = _sig("nvfp4_amax_multi", [ctypes.POINTER(_vp), ctypes.POINTER(_i64), ctypes.c_int, _vp, _vp])
+_c_observer_update = _sig("nvfp4_observer_update", [_vp, _vp, ctypes.c_int, ctypes.c_double, _vp])
+_c_observe_amax = _sig("nvfp4_observe_amax", [_vp, _i64, _vp, ctypes.c_int, ctypes.c_double, _vp, _vp])
+_c_quantize = _sig("nvfp4_quantize", [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp])
+_c_dequantize = _sig("nvfp4_dequantize", [_vp, _vp, _vp, _i64, _i64, _vp, _vp])
+_c_fake_quant = _sig("nvfp4_fake_quant", [_vp, _vp, _i64, _i64, _vp, _vp])
+_c_fake_quant_siblings = _sig("nvfp4_fake_quant_siblings",
+                              [ctypes.c_int, ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_i64),
+                               ctypes.POINTER(_i64), _vp, _vp])
+_c_status_string = _sig("nvfp4_status_string", [ctypes.c_int], ctypes.c_char_p)
+_c_launch_count = _sig("nvfp4_kernel_launch_count", [], ctypes.c_uint64)
+
+
+class NVFP4Error(RuntimeError):
+    """A libnvfp4 call returned a non-OK status."""
+
+
+def nvfp4_status_string(status: int) -> str:
+    return _c_status_string(int(status)).decode()
+
+
+def nvfp4_kernel_launch_count() -> int:
+    """Kernels launched by libnvfp4 in this process."""
+    return int(_c_launch_count())
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise NVFP4Error(f"{what}: {nvfp4_status_string(status)}")
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise RuntimeError(f"{name} must be a CUDA tensor (libnvfp4 has no CPU path)")
+    if dtype is not None and t.dtype != dtype:
+        raise RuntimeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise RuntimeError(f"{name} must be contiguous")
+    return t
+
+
+def _scalar(t: torch.Tensor, name: str):
+    _cuda(t, name, torch.float32)
+    if t.numel() != 1:
+        raise RuntimeError(f"{name} must hold exactly one fp32 value")
+    return t
+
+
+def _matrix(x: torch.Tensor, name: str = "x"):
+    _cuda(x, name, torch.bfloat16)
+    if x.dim() < 1:
+        raise RuntimeError(f"{name} must have at least one dimension")
+    N = x.shape[-1]
+    M = x.numel() // N if N else 0
+    if N % 16:
+        raise RuntimeError(f"{name}: the last dimension ({N}) must be a multiple of 16")
+    return M, N
+
+
+def nvfp4_amax(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Exact max |x| of a bf16 tensor, as a 1-element fp32 CUDA tensor."""
+    _cuda(x, "x", torch.bfloat16)
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _scalar(out, "out")
+    with torch.cuda.device(x.device):
+        _check(_c_amax(x.data_ptr(), x.numel(), out.data_ptr(), _stream(x.device)), "nvfp4_amax")
+    return out
+
+
+def nvfp4_amax_multi(xs: Sequence[torch.Tensor], out: torch.Tensor | None = None) -> torch.Tensor:
+    """Shared amax of fused sibling tensors (max over all of them)."""
+    xs = list(xs)
+    if not 1 <= len(xs) <= MAX_SIBLINGS:
+        raise RuntimeError(f"between 1 and {MAX_SIBLINGS} tensors")
+    for i, t in enumerate(xs):
+        _cuda(t, f"xs[{i}]", torch.bfloat16)
+        if t.device != xs[0].device:
+            raise RuntimeError("all siblings must be on one device")
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=xs[0].device)
+    _scalar(out, "out")
+    k = len(xs)
+    ptrs = (_vp * k)(*[t.data_ptr() for t in xs])
+    ns = (_i64 * k)(*[t.numel() for t in xs])
+    with torch.cuda.device(xs[0].device):
+        _check(_c_amax_multi(ptrs, ns, k, out.data_ptr(), _stream(xs[0].device)), "nvfp4_amax_multi")
+    return out
+
+
+def _kind(kind) -> int:
+    if isinstance(kind, str):
+        if kind not in OBSERVERS:
+            raise RuntimeError(f"unknown observer {kind!r}; one of {sorted(OBSERVERS)}")
+        return OBSERVERS[kind]
+    return int(kind)
+
+
+def nvfp4_observer_update(state: torch.Tensor, cur_amax: torch.Tensor, kind="static_minmax",
+                          decay: float = 0.01) -> torch.Tensor:
+    """One observer step on an already computed (and already all-reduced) amax; in place."""
+    _scalar(state, "state")
+    _scalar(cur_amax, "cur_amax")
+    with torch.cuda.device(state.device):
+        _check(_c_observer_update(state.data_ptr(), cur_amax.data_ptr(), _kind(kind), float(decay),
+                                  _stream(state.device)), "nvfp4_observer_update")
+    return state
+
+
+def nvfp4_observe_amax(x: torch.Tensor, state: torch.Tensor, kind="static_minmax", decay: float = 0.01,
+                       cur_out: torch.Tensor | None = None) -> torch.Tensor:
+    """amax of x, then the observer step on ``state`` (in place); returns this step's amax."""
+    _cuda(x, "x", torch.bfloat16)
+    _scalar(state, "state")
+    if cur_out is None:
+        cur_out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _scalar(cur_out, "cur_out")
+    with torch.cuda.device(x.device):
+        _check(_c_observe_amax(x.data_ptr(), x.numel(), state.data_ptr(), _kind(kind), float(decay),
+                               cur_out.data_ptr(), _stream(x.device)), "nvfp4_observe_amax")
+    return cur_out
+
+
+def nvfp4_quantize(x: torch.Tensor, amax: torch.Tensor, packed: torch.Tensor | None = None,
+                   scales: torch.Tensor | None = None, global_scale: torch.Tensor | None = None):
+    """bf16 [..., N] -> (packed uint8 [..., N/2], E4M3 scale bytes uint8 [..., N/16],
+    global scale fp32 [1]).  ``amax`` is the tensor's (or siblings', or observer's) amax."""
+    M, N = _matrix(x)
+    _scalar(amax, "amax")
+    lead = tuple(x.shape[:-1])
+    if packed is None:
+        packed = torch.empty(lead + (N // 2,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(lead + (N // 16,), dtype=torch.uint8, device=x.device)
+    if global_scale is None:
+        global_scale = torch.empty(1, dtype=torch.float32, device=x.device)
+    _cuda(packed, "packed", torch.uint8)
+    _cuda(scales, "scales", torch.uint8)
+    _scalar(global_scale, "global_scale")
+    if packed.numel() != M * N // 2 or scales.numel() != M * N // 16:
+        raise RuntimeError("packed / scales have the wrong number of elements")
+    with torch.cuda.device(x.device):
+        _check(_c_quantize(x.data_ptr(), M, N, amax.data_ptr(), packed.data_ptr(), scales.data_ptr(),
+                           global_scale.data_ptr(), _stream(x.device)), "nvfp4_quantize")
+    return packed, scales, global_scale
+
+
+def nvfp4_dequantize(packed: torch.Tensor, scales: torch.Tensor, global_scale: torch.Tensor,
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    """(packed [..., N/2], scales [..., N/16], global scale) -> bf16 [..., N]."""
+    _cuda(packed, "packed", torch.uint8)
+    _cuda(scales, "scales", torch.uint8)
+    _scalar(global_scale, "global_scale")
+    N = packed.shape[-1] * 2
+    M = packed.numel() // (N // 2) if N else 0
+    if scales.numel() != M * N // 16:
+        raise RuntimeError("scales has the wrong number of elements")
+    if out is None:
+        out = torch.empty(tuple(packed.shape[:-1]) + (N,), dtype=torch.bfloat16, device=packed.device)
+    _cuda(out, "out", torch.bfloat16)
+    if out.numel() != M * N:
+        raise RuntimeError("out has the wrong number of elements")
+    with torch.cuda.device(packed.device):
+        _check(_c_dequantize(packed.data_ptr(), scales.data_ptr(), global_scale.data_ptr(), M, N,
+                             out.data_ptr(), _stream(packed.device)), "nvfp4_dequantize")
+    return out
+
+
+def nvfp4_fake_quant(x: torch.Tensor, amax: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 -> bf16 fake-quantization (dequantize(quantize(x)) in one pass).  ``out`` may be x."""
+    M, N = _matrix(x)
+    _scalar(amax, "amax")
+    if out is None:
+        out = torch.empty_like(x)
+    _cuda(out, "out", torch.bfloat16)
+    if out.numel() != x.numel():
+        raise RuntimeError("out has the wrong number of elements")
+    with torch.cuda.device(x.device):
+        _check(_c_fake_quant(x.data_ptr(), out.data_ptr(), M, N, amax.data_ptr(), _stream(x.device)),
+               "nvfp4_fake_quant")
+    return out
+
+
+def nvfp4_fake_quant_siblings(xs: Sequence[torch.Tensor], outs: Sequence[torch.Tensor] | None = None,
+                              amax_out: torch.Tensor | None = None):
+    """Shared amax of the siblings, then each fake-quantized with it.  Returns (outs, amax)."""
+    xs = list(xs)
+    k = len(xs)
+    if not 1 <= k <= MAX_SIBLINGS:
+        raise RuntimeError(f"between 1 and {MAX_SIBLINGS} tensors")
+    shapes = [_matrix(t, f"xs[{i}]") for i, t in enumerate(xs)]
+    dev = xs[0].device
+    if any(t.device != dev for t in xs):
+        raise RuntimeError("all siblings must be on one device")
+    outs = [torch.empty_like(t) for t in xs] if outs is None else list(outs)
+    if len(outs) != k:
+        raise RuntimeError("outs must match xs")
+    for i, (o, t) in enumerate(zip(outs, xs)):
+        _cuda(o, f"outs[{i}]", torch.bfloat16)
+        if o.numel() != t.numel() or o.device != dev:
+            raise RuntimeError(f"outs[{i}] does not match xs[{i}]")
+    if amax_out is None:
+        amax_out = torch.empty(1, dtype=torch.float32, device=dev)
+    _scalar(amax_out, "amax_out")
+    xp = (_vp * k)(*[t.data_ptr() for t in xs])
+    yp = (_vp * k)(*[t.data_ptr() for t in outs])
+    Ms = (_i64 * k)(*[m for m, _ in shapes])
+    Ns = (_i64 * k)(*[n for _, n in shapes])
+    with torch.cuda.device(dev):
+        _check(_c_fake_quant_siblings(k, xp, yp, Ms, Ns, amax_out.data_ptr(), _stream(dev)),
+               "nvfp4_fake_quant_siblings")
+    return outs, amax_out
+
+
+class FakeQuantSTE(torch.autograd.Function):
+    """NVFP4 fake-quant forward with the straight-through backward (the gradient passes
+    unchanged): the verl linear.py tutorial, section 2 (STEFP4QuantTriton)."""
+
+    @staticmethod
+    def forward(ctx, x, amax):
+        return nvfp4_fake_quant(x.contiguous(), amax)
+
+    @staticmethod
+    def backward(ctx, grad_output):
+        return grad_output, None
+
+
+def fake_quant_ste(x: torch.Tensor, amax: torch.Tensor) -> torch.Tensor:
+    return FakeQuantSTE.apply(x, amax)

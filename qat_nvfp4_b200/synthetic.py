@@ -2,10 +2,14 @@
 activations, fused q/k/v siblings, an activation size sweep).
 
 This module only draws numbers: it holds none of the quantization arithmetic, and both
-the GPU tests and the CPU oracle take their inputs from it.  Every generator draws fp32
-values with numpy's PCG64 (``default_rng(seed)``) and rounds them to bf16 with torch's
-CPU cast (round to nearest, ties to even).  bf16 tensors are returned as numpy
-``uint16`` bit patterns.
+the GPU tests and the CPU oracle take their inputs from it.  The host generators draw
+fp32 values with numpy's PCG64 and round them to bf16 with torch's CPU cast (round to
+nearest, ties to even); bf16 tensors are returned as numpy ``uint16`` bit patterns.
+``activation_normal_device`` draws on the GPU instead (the benchmark's 1 GiB input).
+
+Large draws are split into fixed chunks of 2^22 values, each with its own child stream of
+``SeedSequence(seed)`` and filled on a thread pool; the values depend only on the seed and
+the shape, not on the number of threads.
 
 Workloads (all bf16, row-major, blocks of 16 along the last dimension):
   * ``weight_with_grid_blocks``  256x1024 weight ~ N(0, 0.02) with 1% of its blocks
@@ -19,6 +23,9 @@ Workloads (all bf16, row-major, blocks of 16 along the last dimension):
   * ``activation_normal``        N(0, 1) activations of any shape (the size sweep).
 """
 from __future__ import annotations
+
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 import torch
@@ -34,6 +41,32 @@ GRID_MAGNITUDES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
 GRID_MIDPOINTS = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
 
 _CHUNK = 1 << 24
+_DRAW_CHUNK = 1 << 22
+
+
+def _streams(seed: int):
+    """(bulk, misc): the child sequence for chunked bulk draws and a generator for the
+    small draws (positions, choices) of one workload."""
+    bulk, misc = np.random.SeedSequence(seed).spawn(2)
+    return bulk, np.random.default_rng(misc)
+
+
+def _chunked(bulk: np.random.SeedSequence, n: int, fill) -> np.ndarray:
+    """n fp32 values, chunk c drawn by fill(rng_c, out_chunk) from child stream c."""
+    out = np.empty(n, dtype=np.float32)
+    nchunks = (n + _DRAW_CHUNK - 1) // _DRAW_CHUNK
+    children = bulk.spawn(nchunks)
+
+    def work(c):
+        fill(np.random.default_rng(children[c]), out[c * _DRAW_CHUNK:(c + 1) * _DRAW_CHUNK])
+
+    if nchunks <= 1:
+        for c in range(nchunks):
+            work(c)
+    else:
+        with ThreadPoolExecutor(max_workers=min(nchunks, os.cpu_count() or 1)) as pool:
+            list(pool.map(work, range(nchunks)))
+    return out
 
 
 def to_bf16_bits(values_f32: np.ndarray) -> np.ndarray:
@@ -51,17 +84,18 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
 
 
-def _normal_f32(rng: np.random.Generator, shape, std: float) -> np.ndarray:
-    x = rng.standard_normal(size=shape, dtype=np.float32)
-    if std != 1.0:
-        x *= np.float32(std)
-    return x
+def _normal_f32(bulk: np.random.SeedSequence, shape, std: float) -> np.ndarray:
+    def fill(rng, out):
+        rng.standard_normal(out=out, dtype=np.float32)
+        if std != 1.0:
+            out *= np.float32(std)
+    return _chunked(bulk, int(np.prod(shape)), fill).reshape(shape)
 
 
 def activation_normal(shape, seed: int) -> np.ndarray:
     """N(0, 1) bf16 activations (the size sweep)."""
-    rng = np.random.default_rng(seed)
-    return to_bf16_bits(_normal_f32(rng, shape, 1.0))
+    bulk, _ = _streams(seed)
+    return to_bf16_bits(_normal_f32(bulk, shape, 1.0))
 
 
 def sweep_seed(size_index: int) -> int:
@@ -71,8 +105,8 @@ def sweep_seed(size_index: int) -> int:
 def weight_with_outliers(shape=(4096, 4096), seed: int = 2, std: float = 0.02,
                          outlier_fraction: float = 0.001, outlier_gain: float = 50.0) -> np.ndarray:
     """N(0, std) weight with a fraction of random positions multiplied by ``outlier_gain``."""
-    rng = np.random.default_rng(seed)
-    x = _normal_f32(rng, shape, std)
+    bulk, rng = _streams(seed)
+    x = _normal_f32(bulk, shape, std)
     n = x.size
     k = int(round(n * outlier_fraction))
     pos = rng.choice(n, size=k, replace=False)
@@ -83,24 +117,26 @@ def weight_with_outliers(shape=(4096, 4096), seed: int = 2, std: float = 0.02,
 
 def activation_student_t(step: int, shape=(8192, 4096), seed: int = 3, scale: float = 0.5) -> np.ndarray:
     """One step's W4A4 activations: scale * Student-t(df=3), seed + step."""
-    rng = np.random.default_rng(seed + step)
-    x = rng.standard_t(3, size=shape).astype(np.float32)
-    x *= np.float32(scale)
-    return to_bf16_bits(x)
+    bulk, _ = _streams(seed + step)
+
+    def fill(rng, out):
+        out[:] = rng.standard_t(3, size=out.size)
+        out *= np.float32(scale)
+    return to_bf16_bits(_chunked(bulk, int(np.prod(shape)), fill).reshape(shape))
 
 
 def large_weight(shape=(14336, 4096), seed: int = 103, std: float = 0.02) -> np.ndarray:
     """The MLP-sized weight fake-quantized next to the W4A4 activations."""
-    rng = np.random.default_rng(seed)
-    return to_bf16_bits(_normal_f32(rng, shape, std))
+    bulk, _ = _streams(seed)
+    return to_bf16_bits(_normal_f32(bulk, shape, std))
 
 
 def qkv_siblings(seed: int = 4, hidden: int = 4096, kv_rows: int = 1024, std: float = 0.02,
                  multipliers=(1.0, 2.0, 0.5)):
     """Fused q/k/v sibling weights with different spreads; returns [q, k, v] bf16 bits."""
-    rng = np.random.default_rng(seed)
     shapes = [(hidden, hidden), (kv_rows, hidden), (kv_rows, hidden)]
-    return [to_bf16_bits(_normal_f32(rng, s, std * m)) for s, m in zip(shapes, multipliers)]
+    children = np.random.SeedSequence(seed).spawn(len(shapes))
+    return [to_bf16_bits(_normal_f32(c, s, std * m)) for c, s, m in zip(children, shapes, multipliers)]
 
 
 def weight_with_grid_blocks(seed: int = 1, shape=(256, 1024), std: float = 0.02,
@@ -121,8 +157,8 @@ def weight_with_grid_blocks(seed: int = 1, shape=(256, 1024), std: float = 0.02,
     """
     rows, cols = shape
     nb_row = cols // 16
-    rng = np.random.default_rng(seed)
-    x = _normal_f32(rng, shape, std)
+    bulk, rng = _streams(seed)
+    x = _normal_f32(bulk, shape, std)
     if float(np.abs(x).max()) >= 0.375:
         raise ValueError("a Gaussian sample reached the pinned amax 0.375; choose another seed")
     total = rows * nb_row
@@ -151,3 +187,18 @@ def weight_with_grid_blocks(seed: int = 1, shape=(256, 1024), std: float = 0.02,
         blocks.append({"row": r, "block": b, "j": j, "elements": elems})
     x[0, zero_block * 16:(zero_block + 1) * 16] = 0.0
     return to_bf16_bits(x), blocks
+
+
+def activation_normal_device(shape, seed: int, device) -> torch.Tensor:
+    """N(0, 1) bf16 activations drawn on the GPU with torch's seeded CUDA generator (fp32
+    draws rounded to bf16 by torch's cast), for workloads too large to draw on the host
+    quickly.  Deterministic for a given seed, shape and device type."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    flat = out.view(-1)
+    step = 1 << 26
+    for s in range(0, flat.numel(), step):
+        n = min(step, flat.numel() - s)
+        flat[s:s + n] = torch.randn(n, generator=gen, dtype=torch.float32, device=device).to(torch.bfloat16)
+    return out

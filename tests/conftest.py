@@ -9,6 +9,15 @@ if ROOT not in sys.path:
 
 GOLDEN = os.path.join(ROOT, "tests", "golden")
 
+# Build the two native libraries in-tree if they are missing or stale (nvcc and gcc
+# cross-compile without a GPU).  The CUDA library is never replaced by a fallback: if it
+# cannot be built, importing the binding fails.
+from oracle.build import build_oracle  # noqa: E402
+from qat_nvfp4_b200.build import build_library  # noqa: E402
+
+build_oracle()
+build_library()
+
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")

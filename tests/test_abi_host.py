@@ -1,0 +1,151 @@
+"""Host-side checks of the C ABI that need no GPU: every symbol the header declares is
+exported, and every argument error is reported before anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from qat_nvfp4_b200.build import INCLUDE, LIB
+
+NVFP4_OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_ARG, ERR_CUDA = 0, 1, 2, 3, 4, 5
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(INCLUDE):
+        if fn.endswith(".h"):
+            with open(os.path.join(INCLUDE, fn)) as f:
+                text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+            names |= set(re.findall(r"\b(nvfp4_\w+)\s*\(", text))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return ctypes.CDLL(LIB)
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for required in ["nvfp4_amax", "nvfp4_amax_multi", "nvfp4_observer_update", "nvfp4_observe_amax",
+                     "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fake_quant", "nvfp4_fake_quant_siblings",
+                     "nvfp4_status_string", "nvfp4_kernel_launch_count"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (nvfp4_\w+)", out))
+    for name in declared_symbols():
+        assert name in exported, f"{name} declared but not exported"
+        assert getattr(lib, name) is not None
+    # nothing else with the prefix leaks out
+    assert exported <= set(declared_symbols())
+
+
+def test_status_strings(lib):
+    lib.nvfp4_status_string.restype = ctypes.c_char_p
+    for code in range(7):
+        assert lib.nvfp4_status_string(code).startswith(b"NVFP4_")
+    assert b"unknown" in lib.nvfp4_status_string(99)
+
+
+# Fake device addresses: validation must reject them before any CUDA call, so they are
+# never dereferenced.
+A32 = 0x7F0000000000  # 32-byte aligned
+A8 = A32 + 8          # 8-byte aligned only
+ODD = A32 + 2         # bf16 aligned only
+
+
+def _call(lib, name, *args):
+    fn = getattr(lib, name)
+    fn.restype = ctypes.c_int
+    return fn(*args)
+
+
+def _i(v):
+    return ctypes.c_int64(v)
+
+
+def _p(v):
+    return ctypes.c_void_p(v)
+
+
+def test_validation_errors_launch_nothing(lib):
+    lib.nvfp4_kernel_launch_count.restype = ctypes.c_uint64
+    before = lib.nvfp4_kernel_launch_count()
+    S = _p(0)  # default stream
+    amax, gs = _p(A32 + 64), _p(A32 + 128)
+    cases = [
+        # fake_quant
+        (ERR_SHAPE, "nvfp4_fake_quant", _p(A32), _p(A32 + 4096), _i(4), _i(24), amax, S),
+        (ERR_SHAPE, "nvfp4_fake_quant", _p(A32), _p(A32 + 4096), _i(-1), _i(16), amax, S),
+        (ERR_SHAPE, "nvfp4_fake_quant", _p(A32), _p(A32 + 4096), _i(1 << 40), _i(1 << 40), amax, S),
+        (ERR_NULL, "nvfp4_fake_quant", _p(0), _p(A32 + 4096), _i(4), _i(16), amax, S),
+        (ERR_NULL, "nvfp4_fake_quant", _p(A32), _p(A32 + 4096), _i(4), _i(16), _p(0), S),
+        (ERR_ALIGN, "nvfp4_fake_quant", _p(ODD), _p(A32 + 4096), _i(4), _i(16), amax, S),
+        (ERR_ALIGN, "nvfp4_fake_quant", _p(A32), _p(A32 + 4096), _i(4), _i(16), _p(A32 + 2), S),
+        (ERR_ARG, "nvfp4_fake_quant", _p(A32), _p(A32 + 32), _i(4), _i(16), amax, S),  # partial overlap
+        # quantize
+        (ERR_SHAPE, "nvfp4_quantize", _p(A32), _i(2), _i(8), amax, _p(A32), _p(A32), gs, S),
+        (ERR_NULL, "nvfp4_quantize", _p(A32), _i(2), _i(16), amax, _p(0), _p(A32), gs, S),
+        (ERR_NULL, "nvfp4_quantize", _p(A32), _i(2), _i(16), amax, _p(A32), _p(0), gs, S),
+        (ERR_ALIGN, "nvfp4_quantize", _p(A32), _i(2), _i(16), amax, _p(A32 + 4), _p(A32), gs, S),
+        (ERR_ALIGN, "nvfp4_quantize", _p(A8), _i(2), _i(16), amax, _p(A32), _p(A32), gs, S),
+        # dequantize
+        (ERR_NULL, "nvfp4_dequantize", _p(A32), _p(A32), _p(0), _i(2), _i(16), _p(A32), S),
+        (ERR_ALIGN, "nvfp4_dequantize", _p(A32), _p(A32), gs, _i(2), _i(16), _p(A8), S),
+        (ERR_SHAPE, "nvfp4_dequantize", _p(A32), _p(A32), gs, _i(2), _i(17), _p(A32), S),
+        # amax
+        (ERR_NULL, "nvfp4_amax", _p(A32), _i(16), _p(0), S),
+        (ERR_NULL, "nvfp4_amax", _p(0), _i(16), amax, S),
+        (ERR_SHAPE, "nvfp4_amax", _p(A32), _i(-5), amax, S),
+        (ERR_ALIGN, "nvfp4_amax", _p(A8), _i(16), amax, S),
+        (ERR_ALIGN, "nvfp4_amax", _p(A32), _i(16), _p(A32 + 1), S),
+    ]
+    for expect, name, *args in cases:
+        assert _call(lib, name, *args) == expect, (name, expect)
+
+    # observers: unknown kind, bad decay
+    lib.nvfp4_observer_update.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_double,
+                                          ctypes.c_void_p]
+    assert _call(lib, "nvfp4_observer_update", A32, A32 + 4, 7, 0.01, None) == ERR_ARG
+    assert _call(lib, "nvfp4_observer_update", A32, A32 + 4, 1, float("nan"), None) == ERR_ARG
+    assert _call(lib, "nvfp4_observer_update", A32, A32 + 4, 1, 1.5, None) == ERR_ARG
+    assert _call(lib, "nvfp4_observer_update", None, A32 + 4, 0, 0.01, None) == ERR_NULL
+    assert _call(lib, "nvfp4_observer_update", A32 + 1, A32 + 4, 0, 0.01, None) == ERR_ALIGN
+    lib.nvfp4_observe_amax.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int,
+                                       ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p]
+    assert _call(lib, "nvfp4_observe_amax", A32, 16, A32 + 64, 3, 0.01, A32 + 68, None) == ERR_ARG
+    assert _call(lib, "nvfp4_observe_amax", A32, 16, A32 + 64, 0, 0.01, None, None) == ERR_NULL
+
+    # lists: k out of range, null arrays, bad member
+    VP = ctypes.c_void_p
+    xs = (VP * 2)(A32, A32 + 1024)
+    ns = (ctypes.c_int64 * 2)(32, 48)
+    assert _call(lib, "nvfp4_amax_multi", xs, ns, 0, amax, S) == ERR_ARG
+    assert _call(lib, "nvfp4_amax_multi", xs, ns, 17, amax, S) == ERR_ARG
+    assert _call(lib, "nvfp4_amax_multi", None, ns, 2, amax, S) == ERR_NULL
+    bad = (VP * 2)(A32, A8)
+    assert _call(lib, "nvfp4_amax_multi", bad, ns, 2, amax, S) == ERR_ALIGN
+    Ms = (ctypes.c_int64 * 2)(2, 3)
+    Ns = (ctypes.c_int64 * 2)(16, 24)
+    assert _call(lib, "nvfp4_fake_quant_siblings", ctypes.c_int(2), xs, xs, Ms, Ns, amax, S) == ERR_SHAPE
+    Ns2 = (ctypes.c_int64 * 2)(16, 32)
+    assert _call(lib, "nvfp4_fake_quant_siblings", ctypes.c_int(2), xs, xs, Ms, Ns2, _p(0), S) == ERR_NULL
+    assert _call(lib, "nvfp4_fake_quant_siblings", ctypes.c_int(0), xs, xs, Ms, Ns2, amax, S) == ERR_ARG
+
+    assert lib.nvfp4_kernel_launch_count() == before
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    from qat_nvfp4_b200 import nvfp4
+    x = torch.zeros(4, 16, dtype=torch.bfloat16)
+    amax = torch.ones(1)
+    for call in (lambda: nvfp4.nvfp4_fake_quant(x, amax), lambda: nvfp4.nvfp4_amax(x),
+                 lambda: nvfp4.nvfp4_quantize(x, amax)):
+        with pytest.raises(RuntimeError, match="CUDA tensor"):
+            call()
