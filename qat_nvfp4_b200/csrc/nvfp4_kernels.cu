@@ -2,9 +2,9 @@
 //
 // All kernels are HBM-bound streams over 16-element blocks, one block per thread: a
 // warp covers 32 consecutive blocks, so every 32-byte vector access of a warp is one
-// contiguous kilobyte.  Grids are persistent: as many CTAs as fit on the SMs at once
-// (occupancy x SM count), each thread walking the blocks with a grid-sized stride and
-// issuing the loads of U blocks before any math, to keep enough bytes in flight.
+// contiguous kilobyte.  Each CTA streams a contiguous chunk, issuing the loads of U
+// blocks per thread before any math; grids oversubscribe the SMs so that the hardware
+// scheduler keeps them full (see stream_blocks and the launch-shape knobs).
 //
 // Sources: fp4_optimization.py (VideoX-Fun), quantize_weight_to_float4 and
 // dequantize_weight_from_float4 for the math; the verl linear.py tutorial, sections 1,
@@ -25,10 +25,59 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int kThreads = 256;  // the dequantize table relies on 256
-constexpr int kUnrollAmax = 4;
-constexpr int kUnrollEncode = 2;
-constexpr int kUnrollDecode = 2;
+// Launch shape.  Each is a compile-time constant; the defaults are the values measured
+// best on B200 (the sweep is summarised under profiles/).
+//   NVFP4_U_*     blocks each thread loads before it does any math
+//   NVFP4_GRID_*  CTAs launched, as a multiple of the CTAs resident on the GPU at once
+//                 (0: one CTA per kThreads x U blocks).  Oversubscribing lets each CTA
+//                 stream one contiguous chunk while the hardware scheduler keeps every
+//                 SM full, which keeps DRAM accesses local; a persistent grid-stride loop
+//                 spreads the warps over the whole tensor instead.
+#ifndef NVFP4_THREADS
+#define NVFP4_THREADS 256
+#endif
+#ifndef NVFP4_U_AMAX
+#define NVFP4_U_AMAX 4
+#endif
+#ifndef NVFP4_U_FQ
+#define NVFP4_U_FQ 2
+#endif
+#ifndef NVFP4_U_Q
+#define NVFP4_U_Q 1
+#endif
+#ifndef NVFP4_U_DEC
+#define NVFP4_U_DEC 2
+#endif
+#ifndef NVFP4_GRID_AMAX
+#define NVFP4_GRID_AMAX 16
+#endif
+#ifndef NVFP4_GRID_FQ
+#define NVFP4_GRID_FQ 32
+#endif
+#ifndef NVFP4_GRID_Q
+#define NVFP4_GRID_Q 16
+#endif
+#ifndef NVFP4_GRID_DEC
+#define NVFP4_GRID_DEC 64
+#endif
+// 1: register double buffering -- the loads of the next group of blocks are issued
+// before the current group is processed, so every thread always has loads in flight.
+#ifndef NVFP4_PIPE_FQ
+#define NVFP4_PIPE_FQ 0
+#endif
+#ifndef NVFP4_PIPE_Q
+#define NVFP4_PIPE_Q 0
+#endif
+#ifndef NVFP4_PIPE_DEC
+#define NVFP4_PIPE_DEC 0
+#endif
+
+constexpr int kThreads = NVFP4_THREADS;
+constexpr int kUnrollAmax = NVFP4_U_AMAX;
+constexpr int kUnrollFq = NVFP4_U_FQ;
+constexpr int kUnrollQ = NVFP4_U_Q;
+constexpr int kUnrollDecode = NVFP4_U_DEC;
+static_assert(kThreads % 32 == 0 && kThreads <= 1024, "CTA size");
 
 std::atomic<uint64_t> g_launches{0};
 
@@ -50,38 +99,113 @@ struct FqList {
 };
 
 // ---------------------------------------------------------------------------------------
+// The streaming schedule shared by the kernels.  Blocks are handed out so that a warp
+// always touches 32 consecutive blocks (one contiguous kilobyte of bf16).
+//   NVFP4_SCHED 1: CTA c owns one contiguous chunk of ceil(nblk / grid) blocks (rounded
+//                  up to whole steps) and walks it kThreads x U blocks per step.
+//   NVFP4_SCHED 0: grid-stride -- thread t owns blocks t, t + S, t + 2S, ... (S = threads
+//                  in the grid), U of them per step.
+// load(bi, slot) issues the loads of block bi; work(bi, slot) consumes them.  Without
+// pipelining a step issues U loads and then does the U blocks' work; with pipelining the
+// next step's loads are issued before this step's work.
+#ifndef NVFP4_SCHED
+#define NVFP4_SCHED 0
+#endif
+
+template <int U, bool kPipe, class Slot, class Load, class Work>
+__device__ __forceinline__ void stream_blocks(int64_t nblk, Load load, Work work) {
+#if NVFP4_SCHED == 1
+    const int64_t ustride = blockDim.x;
+    const int64_t step = (int64_t)blockDim.x * U;
+    const int64_t per_cta = (nblk + gridDim.x - 1) / gridDim.x;
+    const int64_t chunk = (per_cta + step - 1) / step * step;
+    const int64_t beg = (int64_t)blockIdx.x * chunk;
+    const int64_t end = beg + chunk < nblk ? beg + chunk : nblk;
+    int64_t base = beg + threadIdx.x;
+#else
+    const int64_t ustride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t step = ustride * U;
+    const int64_t end = nblk;
+    int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+#endif
+    if constexpr (!kPipe) {
+        for (; base < end; base += step) {
+            Slot sl[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (base + u * ustride < end) load(base + u * ustride, sl[u]);
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (base + u * ustride < end) work(base + u * ustride, sl[u]);
+        }
+    } else {
+        Slot nxt[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (base + u * ustride < end) load(base + u * ustride, nxt[u]);
+        while (base < end) {
+            Slot cur[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) cur[u] = nxt[u];
+            const int64_t cb = base;
+            base += step;
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (base + u * ustride < end) load(base + u * ustride, nxt[u]);
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (cb + u * ustride < end) work(cb + u * ustride, cur[u]);
+        }
+    }
+}
+
+struct Block32 {
+    uint32_t w[8];
+};
+
+struct FqSlot {
+    uint32_t w[8];
+    uint8_t* y;
+};
+
+struct PackedSlot {
+    uint32_t p0, p1, s;
+};
+
+// ---------------------------------------------------------------------------------------
 // Global amax.  Each thread keeps a running bf16x2 |max|; the CTA reduces it and
 // publishes it with one atomicMax on the fp32 bits (non-negative floats order like
 // their bit patterns), so the result is exact and independent of scheduling.  The
 // destination is zeroed by a memset enqueued just before the launch.
 
+__device__ __forceinline__ float cta_max(float f) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) f = fmaxf(f, __shfl_xor_sync(0xFFFFFFFFu, f, o));
+    __shared__ float warp_max[32];
+    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = f;
+    __syncthreads();
+    f = (threadIdx.x < kThreads / 32) ? warp_max[threadIdx.x] : 0.0f;
+    if (threadIdx.x < 32) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) f = fmaxf(f, __shfl_xor_sync(0xFFFFFFFFu, f, o));
+    }
+    return f;  // valid in thread 0
+}
+
 __global__ void __launch_bounds__(kThreads) amax_kernel(AmaxList L, int64_t total_units, unsigned* out) {
     uint32_t m = 0;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < total_units;
-         base += stride * kUnrollAmax) {
-        uint32_t w[kUnrollAmax][8];
-#pragma unroll
-        for (int u = 0; u < kUnrollAmax; ++u) {
-            const int64_t unit = base + u * stride;
-            if (unit < total_units) {
-                int j = 0;
-                while (j + 1 < L.k && unit >= L.full_end[j]) ++j;
-                const int64_t local = unit - (j ? L.full_end[j - 1] : 0);
-                ld_b256_ro(L.ptr[j] + local * kBlockBytesIn, w[u]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) w[u][i] = 0;
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kUnrollAmax; ++u) {
-            m = absmax_bf16x2(m, absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(w[u][0], w[u][1]),
-                                                             absmax_bf16x2(w[u][2], w[u][3])),
-                                               absmax_bf16x2(absmax_bf16x2(w[u][4], w[u][5]),
-                                                             absmax_bf16x2(w[u][6], w[u][7]))));
-        }
-    }
+    stream_blocks<kUnrollAmax, false, Block32>(
+        total_units,
+        [&](int64_t unit, Block32& b) {
+            int j = 0;
+            while (j + 1 < L.k && unit >= L.full_end[j]) ++j;
+            const int64_t local = unit - (j ? L.full_end[j - 1] : 0);
+            ld_b256_ro(L.ptr[j] + local * kBlockBytesIn, b.w);
+        },
+        [&](int64_t, Block32& b) {
+            m = absmax_bf16x2(m, absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(b.w[0], b.w[1]), absmax_bf16x2(b.w[2], b.w[3])),
+                                               absmax_bf16x2(absmax_bf16x2(b.w[4], b.w[5]), absmax_bf16x2(b.w[6], b.w[7]))));
+        });
     float f = fmaxf(fabsf(bf16_lo(m)), fabsf(bf16_hi(m)));
     // The ragged tails (numel % 16 elements per tensor): one lane of the first warp each.
     if (blockIdx.x == 0 && threadIdx.x < (unsigned)L.k) {
@@ -91,17 +215,8 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(AmaxList L, int64_t tota
         for (int64_t e = full * kBlockElems; e < L.numel[j]; ++e)
             f = fmaxf(f, fabsf(__uint_as_float((uint32_t)p[e] << 16)));
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) f = fmaxf(f, __shfl_xor_sync(0xFFFFFFFFu, f, o));
-    __shared__ float warp_max[kThreads / 32];
-    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = f;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        f = threadIdx.x < kThreads / 32 ? warp_max[threadIdx.x] : 0.0f;
-#pragma unroll
-        for (int o = 4; o > 0; o >>= 1) f = fmaxf(f, __shfl_xor_sync(0xFFFFFFFFu, f, o));
-        if (threadIdx.x == 0) atomicMax(out, __float_as_uint(f));
-    }
+    f = cta_max(f);
+    if (threadIdx.x == 0) atomicMax(out, __float_as_uint(f));
 }
 
 // ---------------------------------------------------------------------------------------
@@ -123,7 +238,7 @@ __global__ void observer_kernel(float* state, const float* cur, int kind, float 
 
 __device__ __forceinline__ float build_scale_table(float4* tab, const float* d_amax) {
     const float gs = global_scale_of(__ldg(d_amax));
-    if (threadIdx.x < 128) tab[threadIdx.x] = scale_entry(threadIdx.x, gs);
+    for (int i = threadIdx.x; i < 128; i += blockDim.x) tab[i] = scale_entry(i, gs);
     __syncthreads();
     return gs;
 }
@@ -137,27 +252,15 @@ __global__ void __launch_bounds__(kThreads)
     __shared__ float4 tab[128];
     const float gs = build_scale_table(tab, d_amax);
     if (d_gs != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *d_gs = gs;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < nblk;
-         base += stride * kUnrollEncode) {
-        uint32_t w[kUnrollEncode][8];
-#pragma unroll
-        for (int u = 0; u < kUnrollEncode; ++u) {
-            const int64_t bi = base + u * stride;
-            if (bi < nblk) ld_b256_ro(x + bi * kBlockBytesIn, w[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < kUnrollEncode; ++u) {
-            const int64_t bi = base + u * stride;
-            if (bi < nblk) {
-                uint32_t c[8];
-                float sd;
-                const uint32_t s8 = encode_block(w[u], gs, tab, c, sd);
-                st_b64(packed + bi * kBlockBytesPacked, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
-                st_u8(scales + bi, s8);
-            }
-        }
-    }
+    stream_blocks<kUnrollQ, NVFP4_PIPE_Q != 0, Block32>(
+        nblk, [&](int64_t bi, Block32& b) { ld_b256_ro(x + bi * kBlockBytesIn, b.w); },
+        [&](int64_t bi, Block32& b) {
+            uint32_t c[8];
+            float sd;
+            const uint32_t s8 = encode_block(b.w, gs, tab, c, sd);
+            st_b64(packed + bi * kBlockBytesPacked, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
+            st_u8(scales + bi, s8);
+        });
 }
 
 // ---------------------------------------------------------------------------------------
@@ -183,34 +286,22 @@ template <bool kMulti>
 __global__ void __launch_bounds__(kThreads) fake_quant_kernel(FqList L, int64_t nblk, const float* d_amax) {
     __shared__ float4 tab[128];
     const float gs = build_scale_table(tab, d_amax);
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < nblk;
-         base += stride * kUnrollEncode) {
-        uint32_t w[kUnrollEncode][8];
-        uint8_t* yp[kUnrollEncode];
+    stream_blocks<kUnrollFq, NVFP4_PIPE_FQ != 0, FqSlot>(
+        nblk,
+        [&](int64_t bi, FqSlot& sl) {
+            const uint8_t* xp;
+            locate_fq<kMulti>(L, bi, xp, sl.y);
+            ld_b256(xp, sl.w);
+        },
+        [&](int64_t, FqSlot& sl) {
+            uint32_t c[8];
+            float sd;
+            encode_block(sl.w, gs, tab, c, sd);
+            uint32_t o[8];
 #pragma unroll
-        for (int u = 0; u < kUnrollEncode; ++u) {
-            const int64_t bi = base + u * stride;
-            if (bi < nblk) {
-                const uint8_t* xp;
-                locate_fq<kMulti>(L, bi, xp, yp[u]);
-                ld_b256(xp, w[u]);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kUnrollEncode; ++u) {
-            const int64_t bi = base + u * stride;
-            if (bi < nblk) {
-                uint32_t c[8];
-                float sd;
-                encode_block(w[u], gs, tab, c, sd);
-                uint32_t o[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
-                st_b256(yp[u], o);
-            }
-        }
-    }
+            for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
+            st_b256(sl.y, o);
+        });
 }
 
 // ---------------------------------------------------------------------------------------
@@ -219,38 +310,26 @@ __global__ void __launch_bounds__(kThreads) fake_quant_kernel(FqList L, int64_t 
 __global__ void __launch_bounds__(kThreads)
     dequantize_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
                       const float* __restrict__ d_gs, uint8_t* __restrict__ y, int64_t nblk) {
-    // sd for every possible scale byte (kThreads == 256 fills it in one step).
-    __shared__ float tab_sd[256];
+    __shared__ float tab_sd[256];  // sd for every possible scale byte
     const float gs = __ldg(d_gs);
-    tab_sd[threadIdx.x] = __fdiv_rn(e4m3_to_f32(threadIdx.x), gs);
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) tab_sd[i] = __fdiv_rn(e4m3_to_f32(i), gs);
     __syncthreads();
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < nblk;
-         base += stride * kUnrollDecode) {
-        uint32_t p[kUnrollDecode][2], s[kUnrollDecode];
+    stream_blocks<kUnrollDecode, NVFP4_PIPE_DEC != 0, PackedSlot>(
+        nblk,
+        [&](int64_t bi, PackedSlot& sl) {
+            ld_b64_ro(packed + bi * kBlockBytesPacked, sl.p0, sl.p1);
+            sl.s = ld_u8_ro(scales + bi);
+        },
+        [&](int64_t bi, PackedSlot& sl) {
+            const float sd = tab_sd[sl.s & 0xFFu];
+            uint32_t o[8];
 #pragma unroll
-        for (int u = 0; u < kUnrollDecode; ++u) {
-            const int64_t bi = base + u * stride;
-            if (bi < nblk) {
-                ld_b64_ro(packed + bi * kBlockBytesPacked, p[u][0], p[u][1]);
-                s[u] = ld_u8_ro(scales + bi);
+            for (int i = 0; i < 4; ++i) {
+                o[i] = decode_pair((sl.p0 >> (8 * i)) & 0xFFu, sd);
+                o[4 + i] = decode_pair((sl.p1 >> (8 * i)) & 0xFFu, sd);
             }
-        }
-#pragma unroll
-        for (int u = 0; u < kUnrollDecode; ++u) {
-            const int64_t bi = base + u * stride;
-            if (bi < nblk) {
-                const float sd = tab_sd[s[u] & 0xFFu];
-                uint32_t o[8];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    o[i] = decode_pair((p[u][0] >> (8 * i)) & 0xFFu, sd);
-                    o[4 + i] = decode_pair((p[u][1] >> (8 * i)) & 0xFFu, sd);
-                }
-                st_b256(y + bi * kBlockBytesIn, o);
-            }
-        }
-    }
+            st_b256(y + bi * kBlockBytesIn, o);
+        });
 }
 
 // ---------------------------------------------------------------------------------------
@@ -301,18 +380,19 @@ nvfp4_status occupancy(const void* fn, int* out) {
     return NVFP4_OK;
 }
 
-// Persistent grid: min(CTAs needed for `items` work items at `per_thread` each, CTAs
-// resident on the whole GPU).
-nvfp4_status grid_for(const void* fn, int64_t items, int per_thread, int* grid) {
+// Grid: min(CTAs needed for `items` work items at `per_thread` each, `mult` times the
+// CTAs resident on the whole GPU at once; mult == 0 means no cap).
+nvfp4_status grid_for(const void* fn, int64_t items, int per_thread, int mult, int* grid) {
     int sms = 0, occ = 0;
     nvfp4_status st = sm_count(&sms);
     if (st != NVFP4_OK) return st;
     st = occupancy(fn, &occ);
     if (st != NVFP4_OK) return st;
     const int64_t per_cta = (int64_t)kThreads * per_thread;
-    int64_t need = (items + per_cta - 1) / per_cta;
-    int64_t cap = (int64_t)sms * occ;
+    const int64_t need = (items + per_cta - 1) / per_cta;
+    const int64_t cap = mult > 0 ? (int64_t)sms * occ * mult : need;
     int64_t g = need < cap ? need : cap;
+    if (g > 0x7FFFFFFF) g = 0x7FFFFFFF;
     *grid = (int)(g < 1 ? 1 : g);
     return NVFP4_OK;
 }
@@ -347,7 +427,7 @@ nvfp4_status launch_amax(const AmaxList& L, float* d_amax, nvfp4_stream_t stream
     if (cudaMemsetAsync(d_amax, 0, sizeof(float), cs(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
     const int64_t units = L.full_end[L.k - 1];
     int grid = 1;
-    nvfp4_status st = grid_for(reinterpret_cast<const void*>(&amax_kernel), units, kUnrollAmax, &grid);
+    nvfp4_status st = grid_for(reinterpret_cast<const void*>(&amax_kernel), units, kUnrollAmax, NVFP4_GRID_AMAX, &grid);
     if (st != NVFP4_OK) return st;
     amax_kernel<<<grid, kThreads, 0, cs(stream)>>>(L, units, reinterpret_cast<unsigned*>(d_amax));
     return after_launch();
@@ -462,7 +542,7 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const
     const int64_t nblk = numel / kBlockElems;
     if (nblk == 0 && d_global_scale == nullptr) return NVFP4_OK;
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&quantize_kernel), nblk, kUnrollEncode, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&quantize_kernel), nblk, kUnrollQ, NVFP4_GRID_Q, &grid);
     if (st != NVFP4_OK) return st;
     quantize_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), nblk, d_amax, packed, scales,
                                                        d_global_scale);
@@ -481,7 +561,7 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* sc
     const int64_t nblk = numel / kBlockElems;
     if (nblk == 0) return NVFP4_OK;
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&dequantize_kernel), nblk, kUnrollDecode, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&dequantize_kernel), nblk, kUnrollDecode, NVFP4_GRID_DEC, &grid);
     if (st != NVFP4_OK) return st;
     dequantize_kernel<<<grid, kThreads, 0, cs(stream)>>>(packed, scales, d_global_scale, static_cast<uint8_t*>(y), nblk);
     return after_launch();
@@ -506,7 +586,7 @@ NVFP4_API nvfp4_status nvfp4_fake_quant(const void* x, void* y, int64_t M, int64
     L.y[0] = static_cast<uint8_t*>(y);
     L.blk_end[0] = nblk;
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<false>), nblk, kUnrollEncode, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<false>), nblk, kUnrollFq, NVFP4_GRID_FQ, &grid);
     if (st != NVFP4_OK) return st;
     fake_quant_kernel<false><<<grid, kThreads, 0, cs(stream)>>>(L, nblk, d_amax);
     return after_launch();
@@ -543,7 +623,7 @@ NVFP4_API nvfp4_status nvfp4_fake_quant_siblings(int k, const void* const* xs, v
     const int64_t nblk = acc;
     if (nblk == 0) return NVFP4_OK;
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<true>), nblk, kUnrollEncode, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<true>), nblk, kUnrollFq, NVFP4_GRID_FQ, &grid);
     if (st != NVFP4_OK) return st;
     fake_quant_kernel<true><<<grid, kThreads, 0, cs(stream)>>>(F, nblk, d_shared_amax);
     return after_launch();
