@@ -240,6 +240,7 @@ def run_native(args):
     gs = torch.empty(1, dtype=torch.float32, device=dev)
     cur = torch.empty(1, dtype=torch.float32, device=dev)
     state = torch.full((1,), -1.0, dtype=torch.float32, device=dev)
+    ws = nv.new_workspace(dev)
     stream = torch.cuda.current_stream(dev)
 
     stages = ["amax", "fake_quant", "quantize", "dequantize"]
@@ -250,9 +251,9 @@ def run_native(args):
                 ev[i].record(stream)
         mark(0)
         if world == 1:
-            nv.nvfp4_observe_amax(x, state, kind="minmax", decay=0.01, cur_out=cur)
+            nv.nvfp4_observe_amax(x, state, kind="minmax", decay=0.01, cur_out=cur, workspace=ws)
         else:
-            nv.nvfp4_amax(x, out=cur)
+            nv.nvfp4_amax(x, out=cur, workspace=ws)
             dist.all_reduce(cur, op=dist.ReduceOp.MAX)
             nv.nvfp4_observer_update(state, cur, kind="minmax", decay=0.01)
         mark(1)

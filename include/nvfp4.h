@@ -108,6 +108,29 @@ nvfp4_status nvfp4_observer_update(float* d_state, const float* d_cur_amax, nvfp
 nvfp4_status nvfp4_observe_amax(const void* x, int64_t numel, float* d_state, nvfp4_observer kind,
                                 double decay, float* d_cur_amax, nvfp4_stream_t stream);
 
+/* ---- single-launch variants with a workspace --------------------------------------- */
+
+/* A workspace is NVFP4_WORKSPACE_BYTES of caller-owned device memory, 16-byte aligned,
+ * zero-filled by the caller once before its first use (cudaMemset).  A call that uses it
+ * leaves it zero-filled again when its kernel completes, so it can be reused by every
+ * later call on the same stream without another memset.  Two calls that may run at the
+ * same time (different streams) need two workspaces.  If a call reports NVFP4_ERR_CUDA
+ * the workspace contents are undefined and must be zero-filled again. */
+#define NVFP4_WORKSPACE_BYTES 256
+
+/* nvfp4_amax in one kernel launch (no memset): the last CTA to finish publishes the
+ * result.  Same result, arguments and errors as nvfp4_amax, plus
+ *   d_workspace  NVFP4_WORKSPACE_BYTES, 16-byte aligned, zero-filled (see above). */
+nvfp4_status nvfp4_amax_ws(const void* x, int64_t numel, float* d_amax, void* d_workspace, nvfp4_stream_t stream);
+
+/* nvfp4_observe_amax in one kernel launch: the amax and the observer step of [QATLIN]
+ * section 5, applied by the last CTA to finish.  Same results, arguments and errors as
+ * nvfp4_observe_amax, plus d_workspace as for nvfp4_amax_ws. */
+nvfp4_status nvfp4_observe_amax_ws(const void* x, int64_t numel, float* d_state, nvfp4_observer kind,
+                                   double decay, float* d_cur_amax, void* d_workspace, nvfp4_stream_t stream);
+
+/* ---- block quantization ------------------------------------------------------------- */
+
 /* Quantize: bf16 [M, N] -> packed E2M1 codes [M, N/2] + E4M3 block scales [M, N/16] (+ the
  * fp32 global scale).  [FP4OPT] quantize_weight_to_float4, with the amax given:
  *   gs    = 2688 / max(*d_amax, 1e-12)

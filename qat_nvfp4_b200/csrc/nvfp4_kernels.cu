@@ -192,7 +192,9 @@ __device__ __forceinline__ float cta_max(float f) {
     return f;  // valid in thread 0
 }
 
-__global__ void __launch_bounds__(kThreads) amax_kernel(AmaxList L, int64_t total_units, unsigned* out) {
+// This thread's share of max |x| over a tensor list: its blocks, plus (first lanes of
+// CTA 0) the ragged tails of numel % 16 elements.
+__device__ __forceinline__ float thread_amax(const AmaxList& L, int64_t total_units) {
     uint32_t m = 0;
     stream_blocks<kUnrollAmax, false, Block32>(
         total_units,
@@ -207,7 +209,6 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(AmaxList L, int64_t tota
                                                absmax_bf16x2(absmax_bf16x2(b.w[4], b.w[5]), absmax_bf16x2(b.w[6], b.w[7]))));
         });
     float f = fmaxf(fabsf(bf16_lo(m)), fabsf(bf16_hi(m)));
-    // The ragged tails (numel % 16 elements per tensor): one lane of the first warp each.
     if (blockIdx.x == 0 && threadIdx.x < (unsigned)L.k) {
         const int j = threadIdx.x;
         const int64_t full = L.full_end[j] - (j ? L.full_end[j - 1] : 0);
@@ -215,21 +216,63 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(AmaxList L, int64_t tota
         for (int64_t e = full * kBlockElems; e < L.numel[j]; ++e)
             f = fmaxf(f, fabsf(__uint_as_float((uint32_t)p[e] << 16)));
     }
-    f = cta_max(f);
+    return f;
+}
+
+__global__ void __launch_bounds__(kThreads) amax_kernel(AmaxList L, int64_t total_units, unsigned* out) {
+    const float f = cta_max(thread_amax(L, total_units));
     if (threadIdx.x == 0) atomicMax(out, __float_as_uint(f));
 }
 
-// ---------------------------------------------------------------------------------------
-// Observer update: one thread (verl linear.py tutorial, section 5).
+// Observer step (verl linear.py tutorial, section 5): a negative state is unset and takes
+// the current amax; static_minmax keeps the running max; the EMA ("minmax") mixes
+// fl(keep * s) + fl(take * c) with keep = fl(1 - decay), take = fl(decay).
+__device__ __forceinline__ float observer_step(float s, float c, int kind, float keep, float take) {
+    if (s < 0.0f) return c;
+    if (kind == NVFP4_OBS_STATIC_MINMAX) return fmaxf(s, c);
+    return __fadd_rn(__fmul_rn(keep, s), __fmul_rn(take, c));
+}
 
 __global__ void observer_kernel(float* state, const float* cur, int kind, float keep, float take) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        float s = *state;
-        const float c = *cur;
-        if (s < 0.0f) s = c;
-        else if (kind == NVFP4_OBS_STATIC_MINMAX) s = fmaxf(s, c);
-        else s = __fadd_rn(__fmul_rn(keep, s), __fmul_rn(take, c));
-        *state = s;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *state = observer_step(*state, *cur, kind, keep, take);
+}
+
+// ---------------------------------------------------------------------------------------
+// Single-launch amax (and observer step) with a workspace.  Every CTA folds its maximum
+// into ws->acc with atomicMax and then counts itself in ws->arrived; the CTA that
+// arrives last has seen every other CTA's atomicMax land (each CTA fences between its
+// two atomics), so it publishes the amax, applies the observer step if asked, and puts
+// the workspace back to zero for the next call.  No CTA ever waits for another.
+
+struct Workspace {
+    unsigned acc;      // running max |x| as fp32 bits
+    unsigned arrived;  // CTAs finished so far
+    unsigned pad[62];
+};
+static_assert(sizeof(Workspace) == 256, "NVFP4_WORKSPACE_BYTES");
+
+__device__ __forceinline__ bool last_to_arrive(Workspace* ws, float cta_amax) {
+    __shared__ bool last;
+    if (threadIdx.x == 0) {
+        atomicMax(&ws->acc, __float_as_uint(cta_amax));
+        __threadfence();
+        last = atomicAdd(&ws->arrived, 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    return last;
+}
+
+template <bool kObserve>
+__global__ void __launch_bounds__(kThreads)
+    amax_ws_kernel(AmaxList L, int64_t total_units, Workspace* ws, float* out, float* state, int kind, float keep,
+                   float take) {
+    const float f = cta_max(thread_amax(L, total_units));
+    if (last_to_arrive(ws, f) && threadIdx.x == 0) {
+        __threadfence();
+        const float a = __uint_as_float(atomicExch(&ws->acc, 0u));
+        atomicExch(&ws->arrived, 0u);
+        *out = a;
+        if (kObserve) *state = observer_step(*state, a, kind, keep, take);
     }
 }
 
@@ -433,6 +476,24 @@ nvfp4_status launch_amax(const AmaxList& L, float* d_amax, nvfp4_stream_t stream
     return after_launch();
 }
 
+// One launch: amax (and the observer step when state != nullptr) through a workspace.
+nvfp4_status launch_amax_ws(const AmaxList& L, float* d_amax, void* d_ws, float* state, int kind, float keep, float take,
+                            nvfp4_stream_t stream) {
+    const int64_t units = L.full_end[L.k - 1];
+    Workspace* ws = static_cast<Workspace*>(d_ws);
+    int grid = 1;
+    if (state == nullptr) {
+        nvfp4_status st = grid_for(reinterpret_cast<const void*>(&amax_ws_kernel<false>), units, kUnrollAmax, NVFP4_GRID_AMAX, &grid);
+        if (st != NVFP4_OK) return st;
+        amax_ws_kernel<false><<<grid, kThreads, 0, cs(stream)>>>(L, units, ws, d_amax, nullptr, 0, 0.f, 0.f);
+    } else {
+        nvfp4_status st = grid_for(reinterpret_cast<const void*>(&amax_ws_kernel<true>), units, kUnrollAmax, NVFP4_GRID_AMAX, &grid);
+        if (st != NVFP4_OK) return st;
+        amax_ws_kernel<true><<<grid, kThreads, 0, cs(stream)>>>(L, units, ws, d_amax, state, kind, keep, take);
+    }
+    return after_launch();
+}
+
 nvfp4_status build_amax_list(const void* const* xs, const int64_t* numels, int k, AmaxList* L) {
     if (k < 1 || k > NVFP4_MAX_SIBLINGS) return NVFP4_ERR_ARG;
     if (xs == nullptr || numels == nullptr) return NVFP4_ERR_NULL;
@@ -528,6 +589,33 @@ NVFP4_API nvfp4_status nvfp4_observe_amax(const void* x, int64_t numel, float* d
     if (st != NVFP4_OK) return st;
     observer_kernel<<<1, 32, 0, cs(stream)>>>(d_state, d_cur_amax, (int)kind, keep, take);
     return after_launch();
+}
+
+NVFP4_API nvfp4_status nvfp4_amax_ws(const void* x, int64_t numel, float* d_amax, void* d_workspace,
+                                     nvfp4_stream_t stream) {
+    if (d_amax == nullptr || d_workspace == nullptr) return NVFP4_ERR_NULL;
+    if (!aligned(d_amax, 4) || !aligned(d_workspace, 16)) return NVFP4_ERR_ALIGN;
+    AmaxList L;
+    const void* xs[1] = {x};
+    const int64_t ns[1] = {numel};
+    nvfp4_status st = build_amax_list(xs, ns, 1, &L);
+    if (st != NVFP4_OK) return st;
+    return launch_amax_ws(L, d_amax, d_workspace, nullptr, 0, 0.f, 0.f, stream);
+}
+
+NVFP4_API nvfp4_status nvfp4_observe_amax_ws(const void* x, int64_t numel, float* d_state, nvfp4_observer kind,
+                                             double decay, float* d_cur_amax, void* d_workspace, nvfp4_stream_t stream) {
+    if (d_state == nullptr || d_cur_amax == nullptr || d_workspace == nullptr) return NVFP4_ERR_NULL;
+    if (!aligned(d_state, 4) || !aligned(d_cur_amax, 4) || !aligned(d_workspace, 16)) return NVFP4_ERR_ALIGN;
+    float keep = 0.f, take = 0.f;
+    nvfp4_status st = check_observer(kind, decay, &keep, &take);
+    if (st != NVFP4_OK) return st;
+    AmaxList L;
+    const void* xs[1] = {x};
+    const int64_t ns[1] = {numel};
+    st = build_amax_list(xs, ns, 1, &L);
+    if (st != NVFP4_OK) return st;
+    return launch_amax_ws(L, d_cur_amax, d_workspace, d_state, (int)kind, keep, take, stream);
 }
 
 NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,

@@ -28,6 +28,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 MAX_SIBLINGS = 16
+WORKSPACE_BYTES = 256
 STATIC_MINMAX = 0
 EMA = 1
 OBSERVERS = {"static_minmax": STATIC_MINMAX, "minmax": EMA, "ema": EMA}
@@ -48,6 +49,8 @@ _c_amax = _sig("nvfp4_amax", [_vp, _i64, _vp, _vp])
 _c_amax_multi = _sig("nvfp4_amax_multi", [ctypes.POINTER(_vp), ctypes.POINTER(_i64), ctypes.c_int, _vp, _vp])
 _c_observer_update = _sig("nvfp4_observer_update", [_vp, _vp, ctypes.c_int, ctypes.c_double, _vp])
 _c_observe_amax = _sig("nvfp4_observe_amax", [_vp, _i64, _vp, ctypes.c_int, ctypes.c_double, _vp, _vp])
+_c_amax_ws = _sig("nvfp4_amax_ws", [_vp, _i64, _vp, _vp, _vp])
+_c_observe_amax_ws = _sig("nvfp4_observe_amax_ws", [_vp, _i64, _vp, ctypes.c_int, ctypes.c_double, _vp, _vp, _vp])
 _c_quantize = _sig("nvfp4_quantize", [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp])
 _c_dequantize = _sig("nvfp4_dequantize", [_vp, _vp, _vp, _i64, _i64, _vp, _vp])
 _c_fake_quant = _sig("nvfp4_fake_quant", [_vp, _vp, _i64, _i64, _vp, _vp])
@@ -110,14 +113,33 @@ def _matrix(x: torch.Tensor, name: str = "x"):
     return M, N
 
 
-def nvfp4_amax(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
-    """Exact max |x| of a bf16 tensor, as a 1-element fp32 CUDA tensor."""
+def new_workspace(device) -> torch.Tensor:
+    """A zero-filled workspace for the single-launch calls (one per stream in flight)."""
+    return torch.zeros(WORKSPACE_BYTES, dtype=torch.uint8, device=device)
+
+
+def _workspace(ws: torch.Tensor, device):
+    _cuda(ws, "workspace", torch.uint8)
+    if ws.numel() < WORKSPACE_BYTES or ws.device != device:
+        raise RuntimeError(f"workspace must hold {WORKSPACE_BYTES} bytes on {device}")
+    return ws
+
+
+def nvfp4_amax(x: torch.Tensor, out: torch.Tensor | None = None,
+               workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Exact max |x| of a bf16 tensor, as a 1-element fp32 CUDA tensor.  With a workspace
+    (see new_workspace) it is one kernel launch instead of a memset and a kernel."""
     _cuda(x, "x", torch.bfloat16)
     if out is None:
         out = torch.empty(1, dtype=torch.float32, device=x.device)
     _scalar(out, "out")
     with torch.cuda.device(x.device):
-        _check(_c_amax(x.data_ptr(), x.numel(), out.data_ptr(), _stream(x.device)), "nvfp4_amax")
+        if workspace is None:
+            _check(_c_amax(x.data_ptr(), x.numel(), out.data_ptr(), _stream(x.device)), "nvfp4_amax")
+        else:
+            _workspace(workspace, x.device)
+            _check(_c_amax_ws(x.data_ptr(), x.numel(), out.data_ptr(), workspace.data_ptr(), _stream(x.device)),
+                   "nvfp4_amax_ws")
     return out
 
 
@@ -161,16 +183,23 @@ def nvfp4_observer_update(state: torch.Tensor, cur_amax: torch.Tensor, kind="sta
 
 
 def nvfp4_observe_amax(x: torch.Tensor, state: torch.Tensor, kind="static_minmax", decay: float = 0.01,
-                       cur_out: torch.Tensor | None = None) -> torch.Tensor:
-    """amax of x, then the observer step on ``state`` (in place); returns this step's amax."""
+                       cur_out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """amax of x, then the observer step on ``state`` (in place); returns this step's amax.
+    With a workspace it is one kernel launch."""
     _cuda(x, "x", torch.bfloat16)
     _scalar(state, "state")
     if cur_out is None:
         cur_out = torch.empty(1, dtype=torch.float32, device=x.device)
     _scalar(cur_out, "cur_out")
     with torch.cuda.device(x.device):
-        _check(_c_observe_amax(x.data_ptr(), x.numel(), state.data_ptr(), _kind(kind), float(decay),
-                               cur_out.data_ptr(), _stream(x.device)), "nvfp4_observe_amax")
+        if workspace is None:
+            _check(_c_observe_amax(x.data_ptr(), x.numel(), state.data_ptr(), _kind(kind), float(decay),
+                                   cur_out.data_ptr(), _stream(x.device)), "nvfp4_observe_amax")
+        else:
+            _workspace(workspace, x.device)
+            _check(_c_observe_amax_ws(x.data_ptr(), x.numel(), state.data_ptr(), _kind(kind), float(decay),
+                                      cur_out.data_ptr(), workspace.data_ptr(), _stream(x.device)),
+                   "nvfp4_observe_amax_ws")
     return cur_out
 
 

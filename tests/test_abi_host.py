@@ -137,6 +137,15 @@ def test_validation_errors_launch_nothing(lib):
     assert _call(lib, "nvfp4_fake_quant_siblings", ctypes.c_int(2), xs, xs, Ms, Ns2, _p(0), S) == ERR_NULL
     assert _call(lib, "nvfp4_fake_quant_siblings", ctypes.c_int(0), xs, xs, Ms, Ns2, amax, S) == ERR_ARG
 
+    # workspace variants: null or misaligned workspace
+    assert _call(lib, "nvfp4_amax_ws", _p(A32), _i(16), amax, _p(0), S) == ERR_NULL
+    assert _call(lib, "nvfp4_amax_ws", _p(A32), _i(16), amax, _p(A32 + 8), S) == ERR_ALIGN
+    assert _call(lib, "nvfp4_amax_ws", _p(A8), _i(16), amax, _p(A32), S) == ERR_ALIGN
+    lib.nvfp4_observe_amax_ws.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int,
+                                          ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    assert _call(lib, "nvfp4_observe_amax_ws", A32, 16, A32 + 64, 1, 0.01, A32 + 68, None, None) == ERR_NULL
+    assert _call(lib, "nvfp4_observe_amax_ws", A32, 16, A32 + 64, 1, -0.5, A32 + 68, A32, None) == ERR_ARG
+
     assert lib.nvfp4_kernel_launch_count() == before
 
 

@@ -342,3 +342,37 @@ def test_dequantize_arbitrary_scale_bytes():
     gs = np.float32(7168.0)
     got = nv.nvfp4_dequantize(u8_to_dev(packed), u8_to_dev(scales), scalar(float(gs)))
     assert_equal_bits(bits(got), oracle_dequantize_rows(packed, scales, float(gs)), "arbitrary bytes")
+
+
+# ---- single-launch calls with a workspace ----------------------------------------------------
+
+@pytest.mark.parametrize("numel", [0, 5, 16, 4099, 1 << 20, 8192 * 4096 + 3])
+def test_amax_with_workspace(numel):
+    rng = np.random.default_rng(numel + 1)
+    x = synthetic.to_bf16_bits(rng.standard_t(3, numel).astype(np.float32))
+    xd = to_dev(x)
+    ws = nv.new_workspace("cuda")
+    for _ in range(3):  # the workspace is reusable call after call
+        got = nv.nvfp4_amax(xd, workspace=ws)
+        assert f32_bits(got) == f32_bits(oracle.amax(x))
+        torch.cuda.synchronize()
+        assert not ws.any().item(), "workspace not returned to zero"
+
+
+def test_observe_with_workspace_16_steps():
+    """The single-launch observer matches the oracle (and so the memset+two-kernel path)
+    step for step, for both observer kinds, on the 8192x4096 Student-t activations."""
+    ws = nv.new_workspace("cuda")
+    for name, kind in (("static_minmax", oracle.STATIC_MINMAX), ("minmax", oracle.EMA)):
+        sd, s = scalar(-1.0), -1.0
+        before = nv.nvfp4_kernel_launch_count()
+        for step in range(16):
+            x = synthetic.activation_student_t(step)
+            cur_d = nv.nvfp4_observe_amax(to_dev(x), sd, kind=name, decay=0.01, workspace=ws)
+            cur = oracle.amax(x)
+            s = oracle.observer_update(s, cur, kind, 0.01)
+            assert f32_bits(cur_d) == f32_bits(cur), f"{name} step {step}: amax"
+            assert f32_bits(sd) == f32_bits(s), f"{name} step {step}: state"
+        assert nv.nvfp4_kernel_launch_count() - before == 16  # one launch per step
+        torch.cuda.synchronize()
+        assert not ws.any().item()
