@@ -24,7 +24,9 @@
  * Conventions:
  *   - Every pointer argument is DEVICE memory owned by the caller, except the arrays of
  *     pointers and sizes passed to the *_multi / *_siblings calls, which are HOST arrays
- *     read before the call returns.  The library allocates nothing and keeps no pointer.
+ *     read before the call returns.  The library allocates nothing at run time and keeps
+ *     no pointer to caller memory (nvfp4_observe_amax_noalloc uses a small static device
+ *     array of the library instead).
  *   - Every call is asynchronous and ordered on `stream` (NULL = the legacy default
  *     stream).  It validates its arguments on the host first and returns an error code
  *     with nothing launched; otherwise it enqueues its work and returns NVFP4_OK, or
@@ -128,6 +130,34 @@ nvfp4_status nvfp4_amax_ws(const void* x, int64_t numel, float* d_amax, void* d_
  * nvfp4_observe_amax, plus d_workspace as for nvfp4_amax_ws. */
 nvfp4_status nvfp4_observe_amax_ws(const void* x, int64_t numel, float* d_state, nvfp4_observer kind,
                                    double decay, float* d_cur_amax, void* d_workspace, nvfp4_stream_t stream);
+
+/* ---- no-allocation variant ------------------------------------------------------------ */
+
+/* Bytes of device memory the library reserves, on every GPU where it is loaded and until
+ * the process exits, for nvfp4_observe_amax_noalloc. */
+#define NVFP4_NOALLOC_SCRATCH_BYTES 256
+
+/* nvfp4_observe_amax_ws without a workspace argument, for callers that cannot allocate
+ * device memory where they call it: code that runs inside a memory plan fixed in advance
+ * (an inference-engine plugin with a pre-sized arena, a framework op that may only use
+ * the buffers it is handed) or a loop that must never enter an allocator.  The pages
+ * have no counterpart; this is a convenience of this library.
+ *   - Scratch: a static device array of NVFP4_NOALLOC_SCRATCH_BYTES inside the library.
+ *     The kernel needs one 256-byte workspace whatever the size of x, so no input is too
+ *     large for it (sizes beyond the library-wide limit are NVFP4_ERR_SHAPE as for every
+ *     call); if a build ever needed more scratch than the array holds the call would
+ *     return NVFP4_ERR_ARG.
+ *   - Nothing is allocated: no cudaMalloc / cudaFree, no allocating library routine.
+ *   - The first call on each device looks up that device's copy of the array
+ *     (cudaGetSymbolAddress, with the device current); make that first call before any
+ *     stream capture.
+ *   - Every call on a device shares the one array: each call clears it (a memset on
+ *     `stream`) before its kernel, and calls that overlap on the GPU (different streams)
+ *     race with each other.  Use nvfp4_observe_amax_ws with one workspace per stream for
+ *     concurrent calls.
+ * Arguments, results and other errors are those of nvfp4_observe_amax. */
+nvfp4_status nvfp4_observe_amax_noalloc(const void* x, int64_t numel, float* d_state, nvfp4_observer kind,
+                                        double decay, float* d_cur_amax, nvfp4_stream_t stream);
 
 /* ---- block quantization ------------------------------------------------------------- */
 

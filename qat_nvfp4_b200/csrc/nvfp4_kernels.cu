@@ -618,6 +618,56 @@ NVFP4_API nvfp4_status nvfp4_observe_amax_ws(const void* x, int64_t numel, float
     return launch_amax_ws(L, d_cur_amax, d_workspace, d_state, (int)kind, keep, take, stream);
 }
 
+// ---------------------------------------------------------------------------------------
+// Observer step without a caller-provided workspace.  For callers that cannot allocate
+// device memory on this path (code running inside a memory plan fixed in advance, such as
+// an engine plugin with a pre-sized arena, or a loop that must never enter an allocator),
+// the workspace lives in a static device array of this library instead: every GPU that
+// loads the library holds these bytes until the process exits.
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NVFP4_NOALLOC_SCRATCH_BYTES];
+
+namespace nvfp4 {
+namespace {
+void* g_noalloc_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+}  // namespace
+}  // namespace nvfp4
+
+NVFP4_API nvfp4_status nvfp4_observe_amax_noalloc(const void* x, int64_t numel, float* d_state, nvfp4_observer kind,
+                                                  double decay, float* d_cur_amax, nvfp4_stream_t stream) {
+    if (d_state == nullptr || d_cur_amax == nullptr) return NVFP4_ERR_NULL;
+    if (!aligned(d_state, 4) || !aligned(d_cur_amax, 4)) return NVFP4_ERR_ALIGN;
+    float keep = 0.f, take = 0.f;
+    nvfp4_status st = check_observer(kind, decay, &keep, &take);
+    if (st != NVFP4_OK) return st;
+    AmaxList L;
+    const void* xs[1] = {x};
+    const int64_t ns[1] = {numel};
+    st = build_amax_list(xs, ns, 1, &L);
+    if (st != NVFP4_OK) return st;
+    // The kernel needs one workspace whatever the size of x; refuse if that ever exceeded
+    // the static array.
+    const size_t need = sizeof(Workspace);
+    if (need > sizeof(g_noalloc_scratch)) return NVFP4_ERR_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_CUDA;
+    void* scratch = nullptr;
+    {
+        // First call on a device: look up this device's copy of the array (with the device
+        // current).  Later calls reuse the address.
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (g_noalloc_ptr[dev] == nullptr) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return NVFP4_ERR_CUDA;
+            g_noalloc_ptr[dev] = p;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    // The array keeps whatever the previous call left; the kernel needs it zeroed.
+    if (cudaMemsetAsync(scratch, 0, need, cs(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
+    return launch_amax_ws(L, d_cur_amax, scratch, d_state, (int)kind, keep, take, stream);
+}
+
 NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
                                       uint8_t* scales, float* d_global_scale, nvfp4_stream_t stream) {
     int64_t numel = 0;
