@@ -131,6 +131,43 @@ nvfp4_status nvfp4_amax_ws(const void* x, int64_t numel, float* d_amax, void* d_
 nvfp4_status nvfp4_observe_amax_ws(const void* x, int64_t numel, float* d_state, nvfp4_observer kind,
                                    double decay, float* d_cur_amax, void* d_workspace, nvfp4_stream_t stream);
 
+/* ---- fused amax -> fake-quant --------------------------------------------------------- */
+
+/* Fake-quantize x with its own global amax in one pass over HBM when x fits in L2: a
+ * cooperative kernel reduces max |x| (keeping x in L2), meets at a grid barrier, then
+ * fake-quantizes x from L2.  Above twice the L2 size it enqueues the single-launch amax
+ * and the fake-quant kernel instead.  Bit-identical to nvfp4_amax + nvfp4_fake_quant.
+ * [QATLIN] sections 1, 2 and 4 with the formulas of [FP4OPT].
+ *   x, y         bf16 [M, N] as for nvfp4_fake_quant (y == x allowed)
+ *   d_amax       fp32 out: the amax that was used
+ *   d_workspace  as for nvfp4_amax_ws
+ * The barrier's wait is bounded (2 s); if it ever gives up, y is left unfinished and the
+ * workspace records NVFP4_ERR_TIMEOUT for nvfp4_workspace_check.
+ * Enqueues one cooperative kernel (or two kernels). */
+nvfp4_status nvfp4_fake_quant_fused(const void* x, void* y, int64_t M, int64_t N, float* d_amax, void* d_workspace,
+                                    nvfp4_stream_t stream);
+
+/* One W4A4 activation step in one pass: amax of x, the observer step of [QATLIN]
+ * section 5 on *d_state, and fake-quant of x with the updated state -- the fused form of
+ * nvfp4_observe_amax followed by nvfp4_fake_quant (bit-identical).  Arguments as for
+ * nvfp4_observe_amax and nvfp4_fake_quant_fused; d_cur_amax receives this step's amax. */
+nvfp4_status nvfp4_observe_fake_quant(const void* x, void* y, int64_t M, int64_t N, float* d_state,
+                                      nvfp4_observer kind, double decay, float* d_cur_amax, void* d_workspace,
+                                      nvfp4_stream_t stream);
+
+/* Waits for `stream`, then reports whether a bounded device-side wait of an earlier call
+ * that used this workspace gave up: NVFP4_OK if not, NVFP4_ERR_TIMEOUT if one did (the
+ * workspace is then zero-filled again so that it can be reused). */
+nvfp4_status nvfp4_workspace_check(void* d_workspace, nvfp4_stream_t stream);
+
+/* Self-test of the bounded wait: runs the fused kernel of nvfp4_fake_quant_fused with a
+ * barrier that can never complete (one arrival more than the grid has) and a wait limit
+ * of timeout_us microseconds (1 .. 100000).  Every CTA gives up, records
+ * NVFP4_ERR_TIMEOUT in the workspace and returns; nvfp4_workspace_check then reports it.
+ * y is not written.  Arguments otherwise as for nvfp4_fake_quant_fused (M*N > 0). */
+nvfp4_status nvfp4_selftest_barrier_timeout(const void* x, void* y, int64_t M, int64_t N, float* d_amax,
+                                            void* d_workspace, uint32_t timeout_us, nvfp4_stream_t stream);
+
 /* ---- no-allocation variant ------------------------------------------------------------ */
 
 /* Bytes of device memory the library reserves, on every GPU where it is loaded and until

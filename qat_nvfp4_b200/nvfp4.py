@@ -51,6 +51,12 @@ _c_observer_update = _sig("nvfp4_observer_update", [_vp, _vp, ctypes.c_int, ctyp
 _c_observe_amax = _sig("nvfp4_observe_amax", [_vp, _i64, _vp, ctypes.c_int, ctypes.c_double, _vp, _vp])
 _c_amax_ws = _sig("nvfp4_amax_ws", [_vp, _i64, _vp, _vp, _vp])
 _c_observe_amax_ws = _sig("nvfp4_observe_amax_ws", [_vp, _i64, _vp, ctypes.c_int, ctypes.c_double, _vp, _vp, _vp])
+_c_fake_quant_fused = _sig("nvfp4_fake_quant_fused", [_vp, _vp, _i64, _i64, _vp, _vp, _vp])
+_c_observe_fake_quant = _sig("nvfp4_observe_fake_quant",
+                             [_vp, _vp, _i64, _i64, _vp, ctypes.c_int, ctypes.c_double, _vp, _vp, _vp])
+_c_workspace_check = _sig("nvfp4_workspace_check", [_vp, _vp])
+_c_selftest_barrier_timeout = _sig("nvfp4_selftest_barrier_timeout",
+                                   [_vp, _vp, _i64, _i64, _vp, _vp, ctypes.c_uint32, _vp])
 _c_quantize = _sig("nvfp4_quantize", [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp])
 _c_dequantize = _sig("nvfp4_dequantize", [_vp, _vp, _vp, _i64, _i64, _vp, _vp])
 _c_fake_quant = _sig("nvfp4_fake_quant", [_vp, _vp, _i64, _i64, _vp, _vp])
@@ -292,6 +298,65 @@ def nvfp4_fake_quant_siblings(xs: Sequence[torch.Tensor], outs: Sequence[torch.T
         _check(_c_fake_quant_siblings(k, xp, yp, Ms, Ns, amax_out.data_ptr(), _stream(dev)),
                "nvfp4_fake_quant_siblings")
     return outs, amax_out
+
+
+def nvfp4_fake_quant_fused(x: torch.Tensor, out: torch.Tensor | None = None, amax_out: torch.Tensor | None = None,
+                           workspace: torch.Tensor | None = None):
+    """Fake-quantize x with its own amax in one pass (one cooperative kernel when x fits in
+    L2).  Returns (y, amax).  ``out`` may be x."""
+    M, N = _matrix(x)
+    out = torch.empty_like(x) if out is None else out
+    _cuda(out, "out", torch.bfloat16)
+    if out.numel() != x.numel():
+        raise RuntimeError("out has the wrong number of elements")
+    amax_out = torch.empty(1, dtype=torch.float32, device=x.device) if amax_out is None else amax_out
+    _scalar(amax_out, "amax_out")
+    workspace = new_workspace(x.device) if workspace is None else _workspace(workspace, x.device)
+    with torch.cuda.device(x.device):
+        _check(_c_fake_quant_fused(x.data_ptr(), out.data_ptr(), M, N, amax_out.data_ptr(), workspace.data_ptr(),
+                                   _stream(x.device)), "nvfp4_fake_quant_fused")
+    return out, amax_out
+
+
+def nvfp4_observe_fake_quant(x: torch.Tensor, state: torch.Tensor, kind="static_minmax", decay: float = 0.01,
+                             out: torch.Tensor | None = None, cur_out: torch.Tensor | None = None,
+                             workspace: torch.Tensor | None = None):
+    """One W4A4 activation step in one pass: amax of x, observer step on ``state`` (in
+    place), fake-quant with the updated state.  Returns (y, this step's amax)."""
+    M, N = _matrix(x)
+    _scalar(state, "state")
+    out = torch.empty_like(x) if out is None else out
+    _cuda(out, "out", torch.bfloat16)
+    if out.numel() != x.numel():
+        raise RuntimeError("out has the wrong number of elements")
+    cur_out = torch.empty(1, dtype=torch.float32, device=x.device) if cur_out is None else cur_out
+    _scalar(cur_out, "cur_out")
+    workspace = new_workspace(x.device) if workspace is None else _workspace(workspace, x.device)
+    with torch.cuda.device(x.device):
+        _check(_c_observe_fake_quant(x.data_ptr(), out.data_ptr(), M, N, state.data_ptr(), _kind(kind), float(decay),
+                                     cur_out.data_ptr(), workspace.data_ptr(), _stream(x.device)),
+               "nvfp4_observe_fake_quant")
+    return out, cur_out
+
+
+def nvfp4_workspace_check(workspace: torch.Tensor) -> int:
+    """Wait for the current stream; return 0 if no bounded device wait gave up since the
+    last check, else the status code (NVFP4_ERR_TIMEOUT = 6), re-zeroing the workspace."""
+    _workspace(workspace, workspace.device)
+    with torch.cuda.device(workspace.device):
+        return int(_c_workspace_check(workspace.data_ptr(), _stream(workspace.device)))
+
+
+def nvfp4_selftest_barrier_timeout(x: torch.Tensor, workspace: torch.Tensor, timeout_us: int = 2000) -> int:
+    """Run the fused kernel with a barrier that cannot complete and a short wait limit (a
+    test of the bounded wait); returns the launch status."""
+    M, N = _matrix(x)
+    _workspace(workspace, x.device)
+    y = torch.empty_like(x)
+    amax = torch.empty(1, dtype=torch.float32, device=x.device)
+    with torch.cuda.device(x.device):
+        return int(_c_selftest_barrier_timeout(x.data_ptr(), y.data_ptr(), M, N, amax.data_ptr(),
+                                               workspace.data_ptr(), int(timeout_us), _stream(x.device)))
 
 
 class FakeQuantSTE(torch.autograd.Function):

@@ -146,6 +146,22 @@ def test_validation_errors_launch_nothing(lib):
     assert _call(lib, "nvfp4_observe_amax_ws", A32, 16, A32 + 64, 1, 0.01, A32 + 68, None, None) == ERR_NULL
     assert _call(lib, "nvfp4_observe_amax_ws", A32, 16, A32 + 64, 1, -0.5, A32 + 68, A32, None) == ERR_ARG
 
+    # fused calls
+    assert _call(lib, "nvfp4_fake_quant_fused", _p(A32), _p(A32 + 4096), _i(4), _i(24), amax, _p(A32 + 512), S) == ERR_SHAPE
+    assert _call(lib, "nvfp4_fake_quant_fused", _p(A32), _p(A32 + 4096), _i(4), _i(16), amax, _p(0), S) == ERR_NULL
+    assert _call(lib, "nvfp4_fake_quant_fused", _p(A32), _p(A32 + 32), _i(4), _i(16), amax, _p(A32 + 512), S) == ERR_ARG
+    assert _call(lib, "nvfp4_fake_quant_fused", _p(A8), _p(A32 + 4096), _i(4), _i(16), amax, _p(A32 + 512), S) == ERR_ALIGN
+    lib.nvfp4_observe_fake_quant.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                             ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_void_p,
+                                             ctypes.c_void_p, ctypes.c_void_p]
+    assert _call(lib, "nvfp4_observe_fake_quant", A32, A32 + 4096, 4, 16, None, 1, 0.01, A32 + 64, A32 + 512, None) == ERR_NULL
+    assert _call(lib, "nvfp4_observe_fake_quant", A32, A32 + 4096, 4, 16, A32 + 68, 9, 0.01, A32 + 64, A32 + 512, None) == ERR_ARG
+    lib.nvfp4_selftest_barrier_timeout.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint32, ctypes.c_void_p]
+    assert _call(lib, "nvfp4_selftest_barrier_timeout", A32, A32 + 4096, 4, 16, A32 + 64, A32 + 512, 0, None) == ERR_ARG
+    assert _call(lib, "nvfp4_selftest_barrier_timeout", A32, A32 + 4096, 4, 16, A32 + 64, A32 + 512, 10**6, None) == ERR_ARG
+    assert _call(lib, "nvfp4_workspace_check", _p(0), S) == ERR_NULL
+
     assert lib.nvfp4_kernel_launch_count() == before
 
 

@@ -1,0 +1,71 @@
+"""The fused amax -> fake-quant calls against the oracle (0 ULP), on both of their paths
+(one cooperative kernel when x fits in L2, the amax + fake-quant pair above that), and
+the bounded wait of the fused kernel's grid barrier."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from qat_nvfp4_b200 import synthetic
+from nvfp4_testutil import assert_equal_bits, bits, f32_bits, oracle_fake_quant_rows, sample_rows, scalar, to_dev
+
+pytestmark = pytest.mark.gpu
+
+nv = pytest.importorskip("qat_nvfp4_b200.nvfp4")
+
+
+@pytest.mark.parametrize("shape", [(1, 16), (37, 48), (1024, 1024), (4096, 4096), (8192, 4096), (16384, 8192)])
+def test_fake_quant_fused_matches_oracle(shape):
+    M, N = shape
+    x = synthetic.activation_normal(shape, 50 + M)
+    xd = to_dev(x)
+    ws = nv.new_workspace("cuda")
+    for _ in range(2):  # twice: the workspace must come back clean
+        y, a = nv.nvfp4_fake_quant_fused(xd, workspace=ws)
+        want_a = oracle.amax(x)
+        assert f32_bits(a) == f32_bits(want_a)
+        rows = slice(None) if M * N <= 4096 * 4096 else sample_rows(M, 48, seed=M)
+        assert_equal_bits(bits(y)[rows], oracle_fake_quant_rows(x[rows], want_a), f"{M}x{N} fused")
+    assert nv.nvfp4_workspace_check(ws) == 0
+    assert not ws.any().item()
+
+
+def test_fake_quant_fused_in_place_and_weight():
+    x = synthetic.weight_with_outliers()
+    xd = to_dev(x)
+    ws = nv.new_workspace("cuda")
+    y, a = nv.nvfp4_fake_quant_fused(xd, out=xd, workspace=ws)
+    assert y.data_ptr() == xd.data_ptr()
+    assert_equal_bits(bits(xd), oracle_fake_quant_rows(x, oracle.amax(x)), "in place")
+
+
+def test_observe_fake_quant_16_steps():
+    """The W4A4 activation step in one call, for both observers, 16 steps."""
+    ws = nv.new_workspace("cuda")
+    for name, kind in (("static_minmax", oracle.STATIC_MINMAX), ("minmax", oracle.EMA)):
+        sd, s = scalar(-1.0), -1.0
+        for step in range(16):
+            x = synthetic.activation_student_t(step)
+            y, cur = nv.nvfp4_observe_fake_quant(to_dev(x), sd, kind=name, decay=0.01, workspace=ws)
+            c = oracle.amax(x)
+            s = oracle.observer_update(s, c, kind, 0.01)
+            assert f32_bits(cur) == f32_bits(c), f"{name} step {step}: amax"
+            assert f32_bits(sd) == f32_bits(s), f"{name} step {step}: state"
+            rows = sample_rows(x.shape[0], 24, seed=step)
+            assert_equal_bits(bits(y)[rows], oracle_fake_quant_rows(x[rows], s), f"{name} step {step}")
+    assert nv.nvfp4_workspace_check(ws) == 0
+
+
+def test_barrier_wait_gives_up_and_context_stays_usable():
+    """A barrier nothing can complete: every CTA gives up after 2 ms, the workspace
+    records NVFP4_ERR_TIMEOUT, the check reports it and re-zeroes the workspace, and the
+    next fused call on the same workspace is correct."""
+    x = synthetic.activation_normal((2048, 2048), 77)
+    xd = to_dev(x)
+    ws = nv.new_workspace("cuda")
+    assert nv.nvfp4_selftest_barrier_timeout(xd, ws, timeout_us=2000) == 0
+    assert nv.nvfp4_workspace_check(ws) == 6  # NVFP4_ERR_TIMEOUT
+    assert not ws.any().item()
+    assert nv.nvfp4_workspace_check(ws) == 0
+    y, a = nv.nvfp4_fake_quant_fused(xd, workspace=ws)
+    assert_equal_bits(bits(y), oracle_fake_quant_rows(x, oracle.amax(x)), "after a timeout")
