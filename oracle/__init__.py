@@ -135,12 +135,18 @@ def global_scale(amax_value: float) -> float:
     return _lib().oracle_global_scale(f32(amax_value))
 
 
+def padded_blocks(N: int) -> int:
+    """Blocks per row: ceil(N / 16) (rows are zero-padded to a multiple of 16)."""
+    return (N + 15) // 16
+
+
 def quantize(x_bits, global_scale_value: float):
-    """x_bits: uint16 [M, N] (N % 16 == 0).  Returns (packed [M, N/2], scales [M, N/16])."""
+    """x_bits: uint16 [M, N].  Returns (packed [M, 8*B], scales [M, B]), B = ceil(N/16)."""
     a, p = _u16(x_bits)
     M, N = a.shape
-    packed = np.empty((M, N // 2), dtype=np.uint8)
-    scales = np.empty((M, N // 16), dtype=np.uint8)
+    B = padded_blocks(N)
+    packed = np.empty((M, 8 * B), dtype=np.uint8)
+    scales = np.empty((M, B), dtype=np.uint8)
     _lib().oracle_quantize(p, M, N, f32(global_scale_value),
                            packed.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
                            scales.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))

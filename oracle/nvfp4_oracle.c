@@ -168,8 +168,10 @@ ORACLE_API float oracle_global_scale(float amax) {
     return numerator / a;
 }
 
-/* [FP4OPT] quantize_weight_to_float4 for a row-major [M, N] bf16 tensor with
- * N % 16 == 0, given its per-tensor global_scale.  Per 16-element block along the row:
+/* [FP4OPT] quantize_weight_to_float4 for a row-major [M, N] bf16 tensor, given its
+ * per-tensor global_scale.  When N % 16 != 0 each row is first padded on the right with
+ * zeros to P = 16 * ceil(N / 16) columns (the page's `pad = (-features) % block_size`
+ * branch), and the padded row is quantized.  Per 16-element block along the row:
  *   block_amax      = max |x|
  *   block_scale_fp8 = E4M3((block_amax / 6) * global_scale)
  *   block_scale     = max(float(block_scale_fp8) / global_scale, 1e-12)
@@ -177,13 +179,17 @@ ORACLE_API float oracle_global_scale(float amax) {
  *   idx             = _float4_round(|scaled|)
  *   code            = idx + 8 if scaled < 0 else idx
  *   packed[j]       = code[2j] | code[2j+1] << 4
- * packed is [M, N/2] bytes, scales is [M, N/16] E4M3 bytes, both row-major. */
+ * packed is [M, P/2] bytes, scales is [M, P/16] E4M3 bytes, both row-major. */
 ORACLE_API void oracle_quantize(const uint16_t* x, int64_t M, int64_t N, float global_scale,
                                 uint8_t* packed, uint8_t* scales) {
-    int64_t nblk = N / FLOAT4_BLOCK;
+    int64_t nblk = (N + FLOAT4_BLOCK - 1) / FLOAT4_BLOCK;
+    int64_t P = nblk * FLOAT4_BLOCK;
+    uint16_t* row = (uint16_t*)calloc((size_t)(P ? P : 1), sizeof(uint16_t)); /* zero padding */
+    if (!row) return;
     for (int64_t r = 0; r < M; ++r) {
+        memcpy(row, x + r * N, (size_t)N * sizeof(uint16_t));
         for (int64_t b = 0; b < nblk; ++b) {
-            const uint16_t* xb = x + r * N + b * FLOAT4_BLOCK;
+            const uint16_t* xb = row + b * FLOAT4_BLOCK;
             float block_amax = 0.0f;
             for (int i = 0; i < FLOAT4_BLOCK; ++i) {
                 float v = fabsf(oracle_bf16_to_f32(xb[i]));
@@ -204,22 +210,26 @@ ORACLE_API void oracle_quantize(const uint16_t* x, int64_t M, int64_t N, float g
                 int idx = oracle_e2m1_round_index(fabsf(scaled));
                 code[i] = (uint8_t)(scaled < 0.0f ? idx + 8 : idx);
             }
-            uint8_t* pb = packed + r * (N / 2) + b * (FLOAT4_BLOCK / 2);
+            uint8_t* pb = packed + r * (P / 2) + b * (FLOAT4_BLOCK / 2);
             for (int j = 0; j < FLOAT4_BLOCK / 2; ++j)
                 pb[j] = (uint8_t)(code[2 * j] | (code[2 * j + 1] << 4));
         }
     }
+    free(row);
 }
 
 /* [FP4OPT] dequantize_weight_from_float4: split each byte into (low, high) nibbles,
  * look the codes up in FLOAT4_LUT, multiply by float(block_scale_fp8) / global_scale
- * (no clamp on this side) and round the fp32 product to bf16. */
+ * (no clamp on this side) and round the fp32 product to bf16.  packed / scales hold the
+ * P = 16 * ceil(N / 16) padded columns; the result is cropped to the first N (the page's
+ * `[:, :shape[1]]`). */
 ORACLE_API void oracle_dequantize(const uint8_t* packed, const uint8_t* scales, float global_scale,
                                   int64_t M, int64_t N, uint16_t* y) {
-    int64_t nblk = N / FLOAT4_BLOCK;
+    int64_t nblk = (N + FLOAT4_BLOCK - 1) / FLOAT4_BLOCK;
+    int64_t P = nblk * FLOAT4_BLOCK;
     for (int64_t r = 0; r < M; ++r) {
         for (int64_t c = 0; c < N; ++c) {
-            uint8_t byte = packed[r * (N / 2) + c / 2];
+            uint8_t byte = packed[r * (P / 2) + c / 2];
             int code = (c % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
             float value = oracle_e2m1_lut(code);
             float block_scale = oracle_e4m3_decode(scales[r * nblk + c / FLOAT4_BLOCK]) / global_scale;
@@ -235,7 +245,8 @@ ORACLE_API void oracle_dequantize(const uint8_t* packed, const uint8_t* scales, 
  * -1 if the temporaries cannot be allocated. */
 ORACLE_API int oracle_fake_quant(const uint16_t* x, int64_t M, int64_t N, float amax, uint16_t* y) {
     float gs = oracle_global_scale(amax);
-    size_t npacked = (size_t)M * (size_t)(N / 2), nscale = (size_t)M * (size_t)(N / FLOAT4_BLOCK);
+    int64_t nblk = (N + FLOAT4_BLOCK - 1) / FLOAT4_BLOCK;
+    size_t npacked = (size_t)M * (size_t)(nblk * 8), nscale = (size_t)M * (size_t)nblk;
     uint8_t* packed = (uint8_t*)malloc(npacked ? npacked : 1);
     uint8_t* scales = (uint8_t*)malloc(nscale ? nscale : 1);
     if (!packed || !scales) { free(packed); free(scales); return -1; }

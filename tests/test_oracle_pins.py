@@ -382,3 +382,32 @@ def test_observer_ema_closed_forms():
     for _ in range(100):
         s = oracle.observer_update(s, 0.0, oracle.EMA)
     assert abs(s - float(keep) ** 100) <= 100 * 2.0 ** -24 * float(keep) ** 100
+
+
+# ---- rows whose length is not a multiple of 16 --------------------------------------------
+
+@pytest.mark.parametrize("N", [1, 5, 15, 17, 20, 33, 1000])
+def test_padding_is_zero_padding_then_crop(N):
+    """fp4_optimization.py pads the feature dimension with zeros up to a multiple of 16
+    and crops after dequantizing: quantizing an N-column tensor must give exactly the
+    bytes of the explicitly zero-padded tensor (pinned above), and dequantizing must give
+    the first N columns of the padded result."""
+    rng = np.random.default_rng(N)
+    M = 7
+    x = synthetic.to_bf16_bits(rng.standard_normal((M, N)).astype(np.float32))
+    P = 16 * ((N + 15) // 16)
+    xp = np.zeros((M, P), dtype=np.uint16)
+    xp[:, :N] = x
+    a = oracle.amax(x)
+    assert a == oracle.amax(xp)
+    gs = oracle.global_scale(a)
+    packed, scales = oracle.quantize(x, gs)
+    packed_p, scales_p = oracle.quantize(xp, gs)
+    np.testing.assert_array_equal(packed, packed_p)
+    np.testing.assert_array_equal(scales, scales_p)
+    y = oracle.dequantize(packed, scales, gs, M, N)
+    np.testing.assert_array_equal(y, oracle.dequantize(packed_p, scales_p, gs, M, P)[:, :N])
+    np.testing.assert_array_equal(oracle.fake_quant(x, a), y)
+    # the padded positions hold code 0
+    codes = _unpack(packed)
+    assert not codes[:, N:].any()
