@@ -11,12 +11,15 @@
  *
  * Data model shared by every call:
  *   - x is a bf16 tensor [M, N], row-major and contiguous (the last dimension is the
- *     input-feature / hidden dimension).  Blocks are 16 consecutive elements of a row,
- *     so N must be a multiple of 16 for the block calls.
- *   - packed is uint8 [M, N/2], row-major: byte j of a row holds element 2j in its low
+ *     input-feature / hidden dimension).  Blocks are 16 consecutive elements of a row.
+ *     Any N >= 0 is accepted: as in [FP4OPT] quantize_weight_to_float4, a row whose
+ *     length is not a multiple of 16 is padded on the right with zeros to
+ *     P = 16 * ceil(N / 16) columns before it is quantized, and dequantize / fake-quant
+ *     return the first N columns.  (P == N when N % 16 == 0, the fast path.)
+ *   - packed is uint8 [M, P/2], row-major: byte j of a row holds element 2j in its low
  *     nibble and element 2j+1 in its high nibble.  A nibble is an E2M1 code,
  *     magnitude index | sign << 3, magnitudes (0, 0.5, 1, 1.5, 2, 3, 4, 6).
- *   - scales is uint8 [M, N/16], row-major: one E4M3 (float8_e4m3fn) byte per block, in
+ *   - scales is uint8 [M, P/16], row-major: one E4M3 (float8_e4m3fn) byte per block, in
  *     plain row order (not a swizzled GEMM layout).
  *   - amax, global scale and observer state are single fp32 values in device memory.
  *     global_scale = 2688 / max(amax, 1e-12) is the ENCODE scale of [FP4OPT].
@@ -53,7 +56,7 @@ typedef struct CUstream_st* nvfp4_stream_t;
 typedef enum {
     NVFP4_OK = 0,
     NVFP4_ERR_NULL = 1,    /* a required pointer is NULL */
-    NVFP4_ERR_SHAPE = 2,   /* negative size, N % 16 != 0, or a size that overflows */
+    NVFP4_ERR_SHAPE = 2,   /* negative size, or a size that overflows */
     NVFP4_ERR_ALIGN = 3,   /* a pointer is not aligned as the conventions require */
     NVFP4_ERR_ARG = 4,     /* any other invalid argument (kind, decay, k, overlap) */
     NVFP4_ERR_CUDA = 5,    /* the CUDA runtime reported an error */
@@ -136,7 +139,8 @@ nvfp4_status nvfp4_observe_amax_ws(const void* x, int64_t numel, float* d_state,
 /* Fake-quantize x with its own global amax in one pass over HBM when x fits in L2: a
  * cooperative kernel reduces max |x| (keeping x in L2), meets at a grid barrier, then
  * fake-quantizes x from L2.  Above twice the L2 size it enqueues the single-launch amax
- * and the fake-quant kernel instead.  Bit-identical to nvfp4_amax + nvfp4_fake_quant.
+ * and the fake-quant kernel instead (as it does for N % 16 != 0).  Bit-identical to
+ * nvfp4_amax + nvfp4_fake_quant.
  * [QATLIN] sections 1, 2 and 4 with the formulas of [FP4OPT].
  *   x, y         bf16 [M, N] as for nvfp4_fake_quant (y == x allowed)
  *   d_amax       fp32 out: the amax that was used
@@ -164,7 +168,8 @@ nvfp4_status nvfp4_workspace_check(void* d_workspace, nvfp4_stream_t stream);
  * barrier that can never complete (one arrival more than the grid has) and a wait limit
  * of timeout_us microseconds (1 .. 100000).  Every CTA gives up, records
  * NVFP4_ERR_TIMEOUT in the workspace and returns; nvfp4_workspace_check then reports it.
- * y is not written.  Arguments otherwise as for nvfp4_fake_quant_fused (M*N > 0). */
+ * y is not written.  Arguments otherwise as for nvfp4_fake_quant_fused (M*N > 0,
+ * N % 16 == 0, else NVFP4_ERR_SHAPE). */
 nvfp4_status nvfp4_selftest_barrier_timeout(const void* x, void* y, int64_t M, int64_t N, float* d_amax,
                                             void* d_workspace, uint32_t timeout_us, nvfp4_stream_t stream);
 
@@ -204,10 +209,10 @@ nvfp4_status nvfp4_observe_amax_noalloc(const void* x, int64_t numel, float* d_s
  *   byte  = E4M3_rne_satfinite((block_amax / 6) * gs)
  *   bs    = max(E4M3(byte) / gs, 1e-12)              (the dequantized block scale)
  *   code  = E2M1 index of clamp(x / bs, -6, 6), ties to the even index, | 8 if < 0
- *   x         bf16 [M, N], N % 16 == 0, 32-byte aligned
+ *   x         bf16 [M, N], 32-byte aligned
  *   d_amax    fp32 in: the tensor's (or the siblings', or the observer's) amax
- *   packed    uint8 out [M, N/2], 8-byte aligned
- *   scales    uint8 out [M, N/16]
+ *   packed    uint8 out [M, P/2], 8-byte aligned (P = 16 * ceil(N / 16))
+ *   scales    uint8 out [M, P/16]
  *   d_global_scale  fp32 out, may be NULL
  * Enqueues one kernel. */
 nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
@@ -215,9 +220,9 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const float* d_
 
 /* Dequantize: y = bf16_rne(LUT[code] * (E4M3(byte) / gs)), no clamp on this side.
  * [FP4OPT] dequantize_weight_from_float4.
- *   packed  uint8 [M, N/2], 8-byte aligned     scales  uint8 [M, N/16]
+ *   packed  uint8 [M, P/2], 8-byte aligned     scales  uint8 [M, P/16]
  *   d_global_scale  fp32 in (as written by nvfp4_quantize)
- *   y       bf16 out [M, N], 32-byte aligned
+ *   y       bf16 out [M, N], 32-byte aligned (the padding columns are not written)
  * Enqueues one kernel. */
 nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* scales, const float* d_global_scale,
                               int64_t M, int64_t N, void* y, nvfp4_stream_t stream);
@@ -226,7 +231,7 @@ nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* scales, cons
  * no codes written to memory -- the forward of the straight-through estimator ([QATLIN]
  * sections 1 and 2; formulas of [FP4OPT]).  The STE backward is the identity and has no
  * kernel.
- *   x, y    bf16 [M, N], N % 16 == 0, 32-byte aligned; y == x (in place) is allowed,
+ *   x, y    bf16 [M, N], 32-byte aligned; y == x (in place) is allowed,
  *           any other overlap is NVFP4_ERR_ARG
  *   d_amax  fp32 in
  * Enqueues one kernel. */
@@ -236,7 +241,7 @@ nvfp4_status nvfp4_fake_quant(const void* x, void* y, int64_t M, int64_t N, cons
 /* Fused siblings: the shared amax of k tensors, then each one fake-quantized with it.
  * [QATLIN] section 4 (fusion mode) followed by sections 1-2.
  *   xs, ys  HOST arrays of k device pointers (bf16, 32-byte aligned; ys[j] == xs[j] allowed)
- *   Ms, Ns  HOST arrays of k sizes, each Ns[j] % 16 == 0
+ *   Ms, Ns  HOST arrays of k sizes (members with N % 16 != 0 get one launch each)
  *   k       1 .. NVFP4_MAX_SIBLINGS
  *   d_shared_amax  fp32 out: the shared amax that was used
  * Enqueues a memset and two kernels (one amax launch and one fake-quant launch over all

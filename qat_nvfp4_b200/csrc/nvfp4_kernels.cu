@@ -481,6 +481,120 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ---------------------------------------------------------------------------------------
+// Rows whose length N is not a multiple of 16.  fp4_optimization.py pads such rows on the
+// right with zeros to P = 16 * ceil(N / 16) columns before quantizing, and crops the
+// dequantized rows back to N.  Block g = r * nb + b (nb = P / 16) covers columns
+// [16b, min(16b + 16, N)) of row r; columns past N read as +0.0, and only the N real
+// columns are ever written.  Rows are not 32-byte aligned here, so elements move two
+// bytes at a time; packed and scales keep the padded layout ([M, P/2] and [M, P/16]),
+// which makes their offsets g * 8 and g exactly as in the aligned kernels.
+
+struct Ragged {
+    int64_t N;      // real columns
+    int64_t nb;     // blocks per row, ceil(N / 16)
+    int64_t total;  // M * nb
+};
+
+__device__ __forceinline__ int64_t ragged_offset(const Ragged& R, int64_t g, int& n) {
+    const int64_t r = g / R.nb, b = g - r * R.nb;
+    const int64_t c0 = b * kBlockElems;
+    n = (int)(R.N - c0 < kBlockElems ? R.N - c0 : kBlockElems);
+    return r * R.N + c0;
+}
+
+__device__ __forceinline__ void ld_ragged(const uint16_t* p, int n, uint32_t (&w)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t lo = (2 * i < n) ? (uint32_t)p[2 * i] : 0u;
+        const uint32_t hi = (2 * i + 1 < n) ? (uint32_t)p[2 * i + 1] : 0u;
+        w[i] = lo | (hi << 16);
+    }
+}
+
+__device__ __forceinline__ void st_ragged(uint16_t* p, int n, const uint32_t (&o)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        if (2 * i < n) p[2 * i] = (uint16_t)(o[i] & 0xFFFFu);
+        if (2 * i + 1 < n) p[2 * i + 1] = (uint16_t)(o[i] >> 16);
+    }
+}
+
+struct RaggedSlot {
+    uint32_t w[8];
+    int64_t off;
+    int n;
+};
+
+__global__ void __launch_bounds__(kThreads)
+    quantize_ragged_kernel(const uint16_t* __restrict__ x, Ragged R, const float* __restrict__ d_amax,
+                           uint8_t* __restrict__ packed, uint8_t* __restrict__ scales, float* __restrict__ d_gs) {
+    __shared__ float4 tab[128];
+    const float gs = build_scale_table(tab, d_amax);
+    if (d_gs != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *d_gs = gs;
+    stream_blocks<1, false, RaggedSlot>(
+        R.total,
+        [&](int64_t g, RaggedSlot& sl) {
+            sl.off = ragged_offset(R, g, sl.n);
+            ld_ragged(x + sl.off, sl.n, sl.w);
+        },
+        [&](int64_t g, RaggedSlot& sl) {
+            uint32_t c[8];
+            float sd;
+            const uint32_t s8 = encode_block(sl.w, gs, tab, c, sd);
+            st_b64(packed + g * kBlockBytesPacked, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
+            st_u8(scales + g, s8);
+        });
+}
+
+__global__ void __launch_bounds__(kThreads)
+    fake_quant_ragged_kernel(const uint16_t* x, uint16_t* y, Ragged R, const float* d_amax) {
+    __shared__ float4 tab[128];
+    const float gs = build_scale_table(tab, d_amax);
+    stream_blocks<1, false, RaggedSlot>(
+        R.total,
+        [&](int64_t g, RaggedSlot& sl) {
+            sl.off = ragged_offset(R, g, sl.n);
+            ld_ragged(x + sl.off, sl.n, sl.w);
+        },
+        [&](int64_t, RaggedSlot& sl) {
+            uint32_t c[8];
+            float sd;
+            encode_block(sl.w, gs, tab, c, sd);
+            uint32_t o[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
+            st_ragged(y + sl.off, sl.n, o);
+        });
+}
+
+__global__ void __launch_bounds__(kThreads)
+    dequantize_ragged_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
+                             const float* __restrict__ d_gs, uint16_t* __restrict__ y, Ragged R) {
+    __shared__ float tab_sd[256];
+    const float gs = __ldg(d_gs);
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) tab_sd[i] = __fdiv_rn(e4m3_to_f32(i), gs);
+    __syncthreads();
+    stream_blocks<1, false, PackedSlot>(
+        R.total,
+        [&](int64_t g, PackedSlot& sl) {
+            ld_b64_ro(packed + g * kBlockBytesPacked, sl.p0, sl.p1);
+            sl.s = ld_u8_ro(scales + g);
+        },
+        [&](int64_t g, PackedSlot& sl) {
+            const float sd = tab_sd[sl.s & 0xFFu];
+            uint32_t o[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                o[i] = decode_pair((sl.p0 >> (8 * i)) & 0xFFu, sd);
+                o[4 + i] = decode_pair((sl.p1 >> (8 * i)) & 0xFFu, sd);
+            }
+            int n;
+            const int64_t off = ragged_offset(R, g, n);
+            st_ragged(y + off, n, o);
+        });
+}
+
+// ---------------------------------------------------------------------------------------
 // Host side: device properties, grid sizing, validation.
 
 constexpr int kMaxDevices = 64;
@@ -556,11 +670,35 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 // int64 overflow.
 constexpr int64_t kMaxElems = (int64_t)1 << 60;
 
+cudaStream_t cs(nvfp4_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Any M, N >= 0 whose padded size fits; rows with N % 16 != 0 take the ragged kernels.
 nvfp4_status check_matrix(int64_t M, int64_t N, int64_t* numel) {
-    if (M < 0 || N < 0 || N % kBlockElems != 0) return NVFP4_ERR_SHAPE;
-    if (N != 0 && M > kMaxElems / N) return NVFP4_ERR_SHAPE;
+    if (M < 0 || N < 0) return NVFP4_ERR_SHAPE;
+    const int64_t P = (N + kBlockElems - 1) / kBlockElems * kBlockElems;
+    if (P != 0 && M > kMaxElems / P) return NVFP4_ERR_SHAPE;
     *numel = M * N;
     return NVFP4_OK;
+}
+
+Ragged ragged_of(int64_t M, int64_t N) {
+    Ragged R;
+    R.N = N;
+    R.nb = (N + kBlockElems - 1) / kBlockElems;
+    R.total = M * R.nb;
+    return R;
+}
+
+// Ragged launches shared by the entry points (arguments already validated).
+nvfp4_status launch_fq_ragged(const void* x, void* y, int64_t M, int64_t N, const float* d_amax, nvfp4_stream_t stream) {
+    const Ragged R = ragged_of(M, N);
+    if (R.total == 0) return NVFP4_OK;
+    int grid = 1;
+    nvfp4_status st = grid_for(reinterpret_cast<const void*>(&fake_quant_ragged_kernel), R.total, 1, NVFP4_GRID_FQ, &grid);
+    if (st != NVFP4_OK) return st;
+    fake_quant_ragged_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint16_t*>(x), static_cast<uint16_t*>(y),
+                                                                R, d_amax);
+    return after_launch();
 }
 
 bool overlap(const void* a, const void* b, int64_t bytes) {
@@ -568,7 +706,6 @@ bool overlap(const void* a, const void* b, int64_t bytes) {
     return pa < pb + (uintptr_t)bytes && pb < pa + (uintptr_t)bytes;
 }
 
-cudaStream_t cs(nvfp4_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
 // Enqueue memset + amax kernel over an already validated list.
 nvfp4_status launch_amax(const AmaxList& L, float* d_amax, nvfp4_stream_t stream) {
@@ -830,8 +967,19 @@ static nvfp4_status fused_common(const void* x, void* y, int64_t M, int64_t N, f
 
 // Fake-quant one tensor with its own amax (or the observer's), choosing between the fused
 // kernel (x fits in L2) and the amax + fake-quant pair.
-static nvfp4_status fake_quant_auto(const void* x, void* y, int64_t nblk, void* d_ws, float* d_amax_out, float* state,
-                                    int kind, float keep, float take, nvfp4_stream_t stream) {
+static nvfp4_status fake_quant_auto(const void* x, void* y, int64_t M, int64_t N, void* d_ws, float* d_amax_out,
+                                    float* state, int kind, float keep, float take, nvfp4_stream_t stream) {
+    if (N % kBlockElems != 0) {  // ragged rows: single-launch amax, then the ragged fake-quant
+        AmaxList L;
+        const void* xs[1] = {x};
+        const int64_t ns[1] = {M * N};
+        nvfp4_status st = build_amax_list(xs, ns, 1, &L);
+        if (st != NVFP4_OK) return st;
+        st = launch_amax_ws(L, d_amax_out, d_ws, state, kind, keep, take, stream);
+        if (st != NVFP4_OK) return st;
+        return launch_fq_ragged(x, y, M, N, state ? state : d_amax_out, stream);
+    }
+    const int64_t nblk = M * N / kBlockElems;
     int64_t l2 = 0;
     nvfp4_status st = l2_bytes(&l2);
     if (st != NVFP4_OK) return st;
@@ -864,7 +1012,8 @@ NVFP4_API nvfp4_status nvfp4_fake_quant_fused(const void* x, void* y, int64_t M,
     int64_t nblk = 0;
     nvfp4_status st = fused_common(x, y, M, N, d_amax, d_workspace, &nblk);
     if (st != NVFP4_OK) return st;
-    return fake_quant_auto(x, y, nblk, d_workspace, d_amax, nullptr, 0, 0.f, 0.f, stream);
+    (void)nblk;
+    return fake_quant_auto(x, y, M, N, d_workspace, d_amax, nullptr, 0, 0.f, 0.f, stream);
 }
 
 NVFP4_API nvfp4_status nvfp4_observe_fake_quant(const void* x, void* y, int64_t M, int64_t N, float* d_state,
@@ -878,7 +1027,8 @@ NVFP4_API nvfp4_status nvfp4_observe_fake_quant(const void* x, void* y, int64_t 
     int64_t nblk = 0;
     st = fused_common(x, y, M, N, d_cur_amax, d_workspace, &nblk);
     if (st != NVFP4_OK) return st;
-    return fake_quant_auto(x, y, nblk, d_workspace, d_cur_amax, d_state, (int)kind, keep, take, stream);
+    (void)nblk;
+    return fake_quant_auto(x, y, M, N, d_workspace, d_cur_amax, d_state, (int)kind, keep, take, stream);
 }
 
 NVFP4_API nvfp4_status nvfp4_workspace_check(void* d_workspace, nvfp4_stream_t stream) {
@@ -900,6 +1050,7 @@ NVFP4_API nvfp4_status nvfp4_selftest_barrier_timeout(const void* x, void* y, in
     int64_t nblk = 0;
     nvfp4_status st = fused_common(x, y, M, N, d_amax, d_workspace, &nblk);
     if (st != NVFP4_OK) return st;
+    if (N % kBlockElems != 0) return NVFP4_ERR_SHAPE;
     if (nblk == 0 || timeout_us == 0 || timeout_us > 100000) return NVFP4_ERR_ARG;
     // One arrival more than the grid has: nothing ever completes the barrier.
     return launch_fused(static_cast<const uint8_t*>(x), static_cast<uint8_t*>(y), nblk, d_workspace, d_amax, nullptr,
@@ -915,6 +1066,15 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const
     if (numel > 0 && (x == nullptr || packed == nullptr || scales == nullptr)) return NVFP4_ERR_NULL;
     if (!aligned(d_amax, 4) || (d_global_scale && !aligned(d_global_scale, 4))) return NVFP4_ERR_ALIGN;
     if (numel > 0 && (!aligned(x, 32) || !aligned(packed, 8))) return NVFP4_ERR_ALIGN;
+    if (N % kBlockElems != 0) {
+        const Ragged R = ragged_of(M, N);
+        int grid = 1;
+        st = grid_for(reinterpret_cast<const void*>(&quantize_ragged_kernel), R.total, 1, NVFP4_GRID_Q, &grid);
+        if (st != NVFP4_OK) return st;
+        quantize_ragged_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint16_t*>(x), R, d_amax, packed,
+                                                                  scales, d_global_scale);
+        return after_launch();
+    }
     const int64_t nblk = numel / kBlockElems;
     if (nblk == 0 && d_global_scale == nullptr) return NVFP4_OK;
     int grid = 1;
@@ -934,6 +1094,16 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* sc
     if (numel > 0 && (packed == nullptr || scales == nullptr || y == nullptr)) return NVFP4_ERR_NULL;
     if (!aligned(d_global_scale, 4)) return NVFP4_ERR_ALIGN;
     if (numel > 0 && (!aligned(packed, 8) || !aligned(y, 32))) return NVFP4_ERR_ALIGN;
+    if (N % kBlockElems != 0) {
+        const Ragged R = ragged_of(M, N);
+        if (R.total == 0) return NVFP4_OK;
+        int grid = 1;
+        st = grid_for(reinterpret_cast<const void*>(&dequantize_ragged_kernel), R.total, 1, NVFP4_GRID_DEC, &grid);
+        if (st != NVFP4_OK) return st;
+        dequantize_ragged_kernel<<<grid, kThreads, 0, cs(stream)>>>(packed, scales, d_global_scale,
+                                                                    static_cast<uint16_t*>(y), R);
+        return after_launch();
+    }
     const int64_t nblk = numel / kBlockElems;
     if (nblk == 0) return NVFP4_OK;
     int grid = 1;
@@ -953,6 +1123,7 @@ NVFP4_API nvfp4_status nvfp4_fake_quant(const void* x, void* y, int64_t M, int64
     if (!aligned(d_amax, 4)) return NVFP4_ERR_ALIGN;
     if (numel > 0 && (!aligned(x, 32) || !aligned(y, 32))) return NVFP4_ERR_ALIGN;
     if (x != y && numel > 0 && overlap(x, y, numel * 2)) return NVFP4_ERR_ARG;
+    if (N % kBlockElems != 0) return launch_fq_ragged(x, y, M, N, d_amax, stream);
     const int64_t nblk = numel / kBlockElems;
     if (nblk == 0) return NVFP4_OK;
     FqList L;
@@ -996,6 +1167,16 @@ NVFP4_API nvfp4_status nvfp4_fake_quant_siblings(int k, const void* const* xs, v
     if (st != NVFP4_OK) return st;
     st = launch_amax(L, d_shared_amax, stream);
     if (st != NVFP4_OK) return st;
+    bool all_aligned = true;
+    for (int j = 0; j < k; ++j) all_aligned = all_aligned && (Ns[j] % kBlockElems == 0);
+    if (!all_aligned) {  // one launch per member, each with the shared amax
+        for (int j = 0; j < k; ++j) {
+            st = Ns[j] % kBlockElems ? launch_fq_ragged(xs[j], ys[j], Ms[j], Ns[j], d_shared_amax, stream)
+                                     : nvfp4_fake_quant(xs[j], ys[j], Ms[j], Ns[j], d_shared_amax, stream);
+            if (st != NVFP4_OK) return st;
+        }
+        return NVFP4_OK;
+    }
     const int64_t nblk = acc;
     if (nblk == 0) return NVFP4_OK;
     int grid = 1;

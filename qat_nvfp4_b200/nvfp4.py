@@ -13,6 +13,7 @@ straight-through estimator), section 4 (sibling fusion), section 5 (observers).
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from typing import Sequence
 
@@ -109,14 +110,17 @@ def _scalar(t: torch.Tensor, name: str):
 
 
 def _matrix(x: torch.Tensor, name: str = "x"):
+    """(M, N) of a bf16 tensor seen as [M, N] rows along its last dimension."""
     _cuda(x, name, torch.bfloat16)
     if x.dim() < 1:
         raise RuntimeError(f"{name} must have at least one dimension")
     N = x.shape[-1]
-    M = x.numel() // N if N else 0
-    if N % 16:
-        raise RuntimeError(f"{name}: the last dimension ({N}) must be a multiple of 16")
-    return M, N
+    return math.prod(x.shape[:-1]), N
+
+
+def padded_blocks(N: int) -> int:
+    """Blocks per row: rows are zero-padded to 16 * ceil(N / 16) columns."""
+    return (N + 15) // 16
 
 
 def new_workspace(device) -> torch.Tensor:
@@ -215,17 +219,18 @@ def nvfp4_quantize(x: torch.Tensor, amax: torch.Tensor, packed: torch.Tensor | N
     global scale fp32 [1]).  ``amax`` is the tensor's (or siblings', or observer's) amax."""
     M, N = _matrix(x)
     _scalar(amax, "amax")
+    B = padded_blocks(N)
     lead = tuple(x.shape[:-1])
     if packed is None:
-        packed = torch.empty(lead + (N // 2,), dtype=torch.uint8, device=x.device)
+        packed = torch.empty(lead + (8 * B,), dtype=torch.uint8, device=x.device)
     if scales is None:
-        scales = torch.empty(lead + (N // 16,), dtype=torch.uint8, device=x.device)
+        scales = torch.empty(lead + (B,), dtype=torch.uint8, device=x.device)
     if global_scale is None:
         global_scale = torch.empty(1, dtype=torch.float32, device=x.device)
     _cuda(packed, "packed", torch.uint8)
     _cuda(scales, "scales", torch.uint8)
     _scalar(global_scale, "global_scale")
-    if packed.numel() != M * N // 2 or scales.numel() != M * N // 16:
+    if packed.numel() != M * 8 * B or scales.numel() != M * B:
         raise RuntimeError("packed / scales have the wrong number of elements")
     with torch.cuda.device(x.device):
         _check(_c_quantize(x.data_ptr(), M, N, amax.data_ptr(), packed.data_ptr(), scales.data_ptr(),
@@ -234,14 +239,19 @@ def nvfp4_quantize(x: torch.Tensor, amax: torch.Tensor, packed: torch.Tensor | N
 
 
 def nvfp4_dequantize(packed: torch.Tensor, scales: torch.Tensor, global_scale: torch.Tensor,
-                     out: torch.Tensor | None = None) -> torch.Tensor:
-    """(packed [..., N/2], scales [..., N/16], global scale) -> bf16 [..., N]."""
+                     out: torch.Tensor | None = None, n_cols: int | None = None) -> torch.Tensor:
+    """(packed [..., P/2], scales [..., P/16], global scale) -> bf16 [..., N].  ``n_cols``
+    is the unpadded row length N (default P, the padded length), as the page keeps the
+    original shape next to the packed weight."""
     _cuda(packed, "packed", torch.uint8)
     _cuda(scales, "scales", torch.uint8)
     _scalar(global_scale, "global_scale")
-    N = packed.shape[-1] * 2
-    M = packed.numel() // (N // 2) if N else 0
-    if scales.numel() != M * N // 16:
+    P = packed.shape[-1] * 2
+    N = P if n_cols is None else int(n_cols)
+    if padded_blocks(N) * 16 != P:
+        raise RuntimeError(f"n_cols={N} does not match packed rows of {P // 2} bytes")
+    M = math.prod(packed.shape[:-1])
+    if scales.numel() != M * (P // 16):
         raise RuntimeError("scales has the wrong number of elements")
     if out is None:
         out = torch.empty(tuple(packed.shape[:-1]) + (N,), dtype=torch.bfloat16, device=packed.device)

@@ -60,8 +60,9 @@ def oracle_quantize_rows(x_bits, gs, threads=8):
     import oracle
     from concurrent.futures import ThreadPoolExecutor
     M, N = x_bits.shape
-    packed = np.empty((M, N // 2), dtype=np.uint8)
-    scales = np.empty((M, N // 16), dtype=np.uint8)
+    B = (N + 15) // 16  # rows are zero-padded to 16 * B columns
+    packed = np.empty((M, 8 * B), dtype=np.uint8)
+    scales = np.empty((M, B), dtype=np.uint8)
 
     def work(rr):
         r0, r1 = rr
@@ -86,11 +87,11 @@ def oracle_fake_quant_rows(x_bits, amax, threads=8):
     return y
 
 
-def oracle_dequantize_rows(packed, scales, gs, threads=8):
+def oracle_dequantize_rows(packed, scales, gs, threads=8, n_cols=None):
     import oracle
     from concurrent.futures import ThreadPoolExecutor
     M = packed.shape[0]
-    N = packed.shape[1] * 2
+    N = packed.shape[1] * 2 if n_cols is None else n_cols
     y = np.empty((M, N), dtype=np.uint16)
 
     def work(rr):

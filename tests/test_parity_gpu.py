@@ -39,8 +39,8 @@ def _full_check(x_bits, amax_value=None, what=""):
     packed, scales = oracle_quantize_rows(x_bits, gs)
     assert_equal_bits(u8(scales_d), scales, f"{what}: scale bytes")
     assert_equal_bits(u8(packed_d), packed, f"{what}: packed codes")
-    y_d = nv.nvfp4_dequantize(packed_d, scales_d, gs_d)
-    y = oracle_dequantize_rows(packed, scales, gs)
+    y_d = nv.nvfp4_dequantize(packed_d, scales_d, gs_d, n_cols=N)
+    y = oracle_dequantize_rows(packed, scales, gs, n_cols=N)
     assert_equal_bits(bits(y_d), y, f"{what}: dequantize")
     fq_d = nv.nvfp4_fake_quant(xd, amax_d)
     assert_equal_bits(bits(fq_d), y, f"{what}: fake-quant == dequantize(quantize)")
@@ -376,3 +376,37 @@ def test_observe_with_workspace_16_steps():
         assert nv.nvfp4_kernel_launch_count() - before == 16  # one launch per step
         torch.cuda.synchronize()
         assert not ws.any().item()
+
+
+# ---- rows whose length is not a multiple of 16 (zero padding, crop) -----------------------
+
+@pytest.mark.parametrize("M,N", [(1, 1), (5, 15), (3, 20), (17, 1000), (255, 4097), (64, 8191), (2, 33), (4096, 1000)])
+def test_ragged_rows(M, N):
+    rng = np.random.default_rng(M * 131 + N)
+    x = synthetic.to_bf16_bits(rng.standard_t(3, (M, N)).astype(np.float32))
+    packed, scales, y = _full_check(x, what=f"{M}x{N} ragged")
+    assert packed.shape == (M, 8 * ((N + 15) // 16))
+    # in place, the fused call (its ragged path) and the observer step in one call
+    xd = to_dev(x)
+    a = oracle.amax(x)
+    nv.nvfp4_fake_quant(xd, scalar(a), out=xd)
+    assert_equal_bits(bits(xd), y, f"{M}x{N} ragged in place")
+    y2, a2 = nv.nvfp4_fake_quant_fused(to_dev(x))
+    assert f32_bits(a2) == f32_bits(a)
+    assert_equal_bits(bits(y2), y, f"{M}x{N} ragged fused")
+    st = scalar(-1.0)
+    y3, c3 = nv.nvfp4_observe_fake_quant(to_dev(x), st, kind="minmax")
+    assert f32_bits(st) == f32_bits(a)
+    assert_equal_bits(bits(y3), y, f"{M}x{N} ragged observe")
+
+
+def test_siblings_with_ragged_members():
+    rng = np.random.default_rng(61)
+    shapes = [(64, 4096), (16, 1000), (7, 33)]
+    xs = [synthetic.to_bf16_bits(rng.standard_normal(s).astype(np.float32) * np.float32(m))
+          for s, m in zip(shapes, (1.0, 3.0, 0.5))]
+    outs, shared = nv.nvfp4_fake_quant_siblings([to_dev(t) for t in xs])
+    a = oracle.amax_multi(xs)
+    assert f32_bits(shared) == f32_bits(a)
+    for t, o in zip(xs, outs):
+        assert_equal_bits(bits(o), oracle_fake_quant_rows(t, a), f"{t.shape} sibling")
