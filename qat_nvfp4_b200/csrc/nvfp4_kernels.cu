@@ -485,9 +485,16 @@ __global__ void __launch_bounds__(kThreads)
 // right with zeros to P = 16 * ceil(N / 16) columns before quantizing, and crops the
 // dequantized rows back to N.  Block g = r * nb + b (nb = P / 16) covers columns
 // [16b, min(16b + 16, N)) of row r; columns past N read as +0.0, and only the N real
-// columns are ever written.  Rows are not 32-byte aligned here, so elements move two
-// bytes at a time; packed and scales keep the padded layout ([M, P/2] and [M, P/16]),
-// which makes their offsets g * 8 and g exactly as in the aligned kernels.
+// columns are ever written.  packed and scales keep the padded layout ([M, P/2] and
+// [M, P/16]), so their offsets are g * 8 and g exactly as in the aligned kernels.
+//
+// Rows are not 32-byte aligned here, but the real elements of consecutive blocks are
+// consecutive in memory.  So a CTA takes a tile of kThreads consecutive blocks, stages the
+// tile's element range through shared memory with 16-byte vector accesses (only the one
+// 16-byte chunk that crosses the end of the tensor moves two bytes at a time), gives each
+// thread its block from there, and writes bf16 results back the same way -- whole
+// 16-byte chunks inside its range, two-byte stores for the bytes it owns in the two edge
+// chunks it shares with the neighbouring tiles.
 
 struct Ragged {
     int64_t N;      // real columns
@@ -495,103 +502,252 @@ struct Ragged {
     int64_t total;  // M * nb
 };
 
+// First element and real length of block g (32-bit division whenever the sizes allow).
 __device__ __forceinline__ int64_t ragged_offset(const Ragged& R, int64_t g, int& n) {
-    const int64_t r = g / R.nb, b = g - r * R.nb;
+    int64_t r;
+    if (R.total <= 0xFFFFFFFFll) r = (int64_t)((uint32_t)g / (uint32_t)R.nb);
+    else r = g / R.nb;
+    const int64_t b = g - r * R.nb;
     const int64_t c0 = b * kBlockElems;
     n = (int)(R.N - c0 < kBlockElems ? R.N - c0 : kBlockElems);
     return r * R.N + c0;
 }
 
-__device__ __forceinline__ void ld_ragged(const uint16_t* p, int n, uint32_t (&w)[8]) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const uint32_t lo = (2 * i < n) ? (uint32_t)p[2 * i] : 0u;
-        const uint32_t hi = (2 * i + 1 < n) ? (uint32_t)p[2 * i + 1] : 0u;
-        w[i] = lo | (hi << 16);
+// Blocks per thread in one tile, and bytes of staging per CTA: kRaggedTile blocks of at
+// most 32 bytes, plus the 16-byte rounding at the start of the range.
+constexpr int kRaggedU = 4;
+constexpr int kRaggedTile = kThreads * kRaggedU;
+constexpr int kStageBytes = kRaggedTile * kBlockBytesIn + 64;
+
+// The stage holds 16-byte chunk k of the tile's byte range at chunk position
+// k ^ ((k >> 3) & 1).  Lanes whose blocks sit two chunks apart then read eight different
+// bank groups in each quarter-warp phase of a 128-bit shared load (without the swizzle
+// lanes l and l + 4 would collide).
+__device__ __forceinline__ int chunk_pos(int k) { return k ^ ((k >> 3) & 1); }
+__device__ __forceinline__ int stage_addr(int64_t byte) {
+    const int b = (int)byte;
+    return b ^ ((b >> 3) & 16);  // == chunk_pos(b >> 4) * 16 + (b & 15)
+}
+
+// Byte range [B0, B1) of the tile that starts at block g0 (both even).
+__device__ __forceinline__ void tile_range(const Ragged& R, int64_t g0, int64_t& B0, int64_t& B1) {
+    const int64_t g1 = (g0 + kRaggedTile < R.total ? g0 + kRaggedTile : R.total) - 1;
+    int n0, n1;
+    B0 = 2 * ragged_offset(R, g0, n0);
+    B1 = 2 * (ragged_offset(R, g1, n1) + n1);
+}
+
+// Issue the copies that fill a stage with the 16-byte chunks covering [B0, B1) (chunk k
+// of the range, starting at A0 = B0 rounded down to 16, goes to chunk position
+// chunk_pos(k)).  Whole chunks go global -> shared as asynchronous 16-byte copies
+// (cp.async.cg, through L2, so they see writes of other CTAs); the chunk that crosses the
+// end of the tensor, if any, moves two bytes at a time and never reads past total_bytes.
+// The caller waits for the copies (cp.async.wait_all) and syncs the CTA.
+__device__ __forceinline__ void stage_issue(const uint8_t* src, int64_t B0, int64_t B1, int64_t total_bytes,
+                                            uint8_t* stage) {
+    const int64_t A0 = B0 & ~(int64_t)15;
+    const int nch = (int)((B1 - A0 + 15) >> 4);
+    for (int k = threadIdx.x; k < nch; k += blockDim.x) {
+        const int64_t a = A0 + 16 * (int64_t)k;
+        if (a + 16 <= total_bytes) {
+            const unsigned dst = (unsigned)__cvta_generic_to_shared(stage + 16 * chunk_pos(k));
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src + a) : "memory");
+        } else {
+            uint16_t* st16 = reinterpret_cast<uint16_t*>(stage + 16 * chunk_pos(k));
+            const uint16_t* s16 = reinterpret_cast<const uint16_t*>(src + a);
+            for (int i = 0; i < 8; ++i) st16[i] = (a + 2 * i + 2 <= total_bytes) ? s16[i] : (uint16_t)0;
+        }
     }
 }
 
-__device__ __forceinline__ void st_ragged(uint16_t* p, int n, const uint32_t (&o)[8]) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        if (2 * i < n) p[2 * i] = (uint16_t)(o[i] & 0xFFFFu);
-        if (2 * i + 1 < n) p[2 * i + 1] = (uint16_t)(o[i] >> 16);
+// dst[b] = stage byte (b - A0) for every byte b in [B0, B1): whole 16-byte chunks inside
+// the range as one vector store, the two shared edge chunks two bytes at a time.
+__device__ __forceinline__ void stage_out(uint8_t* dst, int64_t B0, int64_t B1, const uint8_t* stage) {
+    const int64_t A0 = B0 & ~(int64_t)15;
+    const int nch = (int)((B1 - A0 + 15) >> 4);
+    for (int k = threadIdx.x; k < nch; k += blockDim.x) {
+        const int64_t a = A0 + 16 * (int64_t)k;
+        if (a >= B0 && a + 16 <= B1) {
+            const uint4 v = *reinterpret_cast<const uint4*>(stage + 16 * chunk_pos(k));
+            asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(dst + a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                         : "memory");
+        } else {
+            const int64_t lo = a > B0 ? a : B0, hi = a + 16 < B1 ? a + 16 : B1;
+            for (int64_t b = lo; b < hi; b += 2)
+                *reinterpret_cast<uint16_t*>(dst + b) = *reinterpret_cast<const uint16_t*>(stage + stage_addr(b - A0));
+        }
     }
 }
 
-struct RaggedSlot {
-    uint32_t w[8];
-    int64_t off;
-    int n;
-};
+// This thread's block (n real elements starting at stage byte X, X even) as eight bf16x2
+// words, zeros past n: the three 16-byte chunks that cover it are read whole, then
+// shifted down by X & 15 bytes with selects and a funnel shift.
+__device__ __forceinline__ void block_from_stage(const uint8_t* stage, int64_t X, int n, uint32_t (&w)[8]) {
+    const int k0 = (int)(X >> 4);
+    const int sh = (int)(X & 15);
+    uint32_t c[12];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        const uint4 v = *reinterpret_cast<const uint4*>(stage + 16 * chunk_pos(k0 + j));
+        c[4 * j] = v.x;
+        c[4 * j + 1] = v.y;
+        c[4 * j + 2] = v.z;
+        c[4 * j + 3] = v.w;
+    }
+    const int s4 = sh >> 2;
+    uint32_t t[10], u[9];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) t[i] = (s4 & 2) ? c[i + 2] : c[i];
+#pragma unroll
+    for (int i = 0; i < 9; ++i) u[i] = (s4 & 1) ? t[i + 1] : t[i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t v = (sh & 2) ? __funnelshift_r(u[i], u[i + 1], 16) : u[i];
+        if (2 * i + 1 >= n) v &= 0x0000FFFFu;  // the row's padding reads as +0.0
+        if (2 * i >= n) v = 0u;
+        w[i] = v;
+    }
+}
+
+// Write this thread's n output elements back to stage byte X: 32-bit stores on 4-byte
+// boundaries, 16-bit stores for a leading or trailing half word.
+__device__ __forceinline__ void block_to_stage(uint8_t* stage, int64_t X, int n, const uint32_t (&o)[8]) {
+    if ((X & 2) == 0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (2 * i + 1 < n) *reinterpret_cast<uint32_t*>(stage + stage_addr(X + 4 * i)) = o[i];
+            else if (2 * i < n) *reinterpret_cast<uint16_t*>(stage + stage_addr(X + 4 * i)) = (uint16_t)(o[i] & 0xFFFFu);
+        }
+    } else {
+        *reinterpret_cast<uint16_t*>(stage + stage_addr(X)) = (uint16_t)(o[0] & 0xFFFFu);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t next = i < 7 ? o[i + 1] : 0u;
+            const uint32_t v = (o[i] >> 16) | (next << 16);  // elements 2i+1, 2i+2
+            if (2 * i + 2 < n) *reinterpret_cast<uint32_t*>(stage + stage_addr(X + 4 * i + 2)) = v;
+            else if (2 * i + 1 < n) *reinterpret_cast<uint16_t*>(stage + stage_addr(X + 4 * i + 2)) = (uint16_t)(v & 0xFFFFu);
+        }
+    }
+}
+
+// The tiles of this CTA: tile starts g0 = blockIdx.x * tile, + gridDim.x * tile, ...
+// Each tile is staged, processed by work(g0, B0, B1, stage) between CTA barriers, and the
+// stage reused.  (A two-stage version that prefetched the next tile measured no faster:
+// the ragged kernels are bound by their per-element index and shift work, not by load
+// latency.)
+template <class Work>
+__device__ __forceinline__ void ragged_tiles(const uint8_t* src, const Ragged& R, uint8_t* stage, Work work) {
+    const int64_t total_bytes = 2 * (R.total / R.nb) * R.N;
+    for (int64_t g0 = (int64_t)blockIdx.x * kRaggedTile; g0 < R.total; g0 += (int64_t)gridDim.x * kRaggedTile) {
+        int64_t B0, B1;
+        tile_range(R, g0, B0, B1);
+        stage_issue(src, B0, B1, total_bytes, stage);
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncthreads();
+        work(g0, B0, B1, stage);
+        __syncthreads();
+    }
+}
 
 __global__ void __launch_bounds__(kThreads)
-    quantize_ragged_kernel(const uint16_t* __restrict__ x, Ragged R, const float* __restrict__ d_amax,
+    quantize_ragged_kernel(const uint8_t* __restrict__ x, Ragged R, const float* __restrict__ d_amax,
                            uint8_t* __restrict__ packed, uint8_t* __restrict__ scales, float* __restrict__ d_gs) {
     __shared__ float4 tab[128];
+    extern __shared__ __align__(16) uint8_t stage[];
     const float gs = build_scale_table(tab, d_amax);
     if (d_gs != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *d_gs = gs;
-    stream_blocks<1, false, RaggedSlot>(
-        R.total,
-        [&](int64_t g, RaggedSlot& sl) {
-            sl.off = ragged_offset(R, g, sl.n);
-            ld_ragged(x + sl.off, sl.n, sl.w);
-        },
-        [&](int64_t g, RaggedSlot& sl) {
-            uint32_t c[8];
-            float sd;
-            const uint32_t s8 = encode_block(sl.w, gs, tab, c, sd);
-            st_b64(packed + g * kBlockBytesPacked, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
-            st_u8(scales + g, s8);
-        });
+    ragged_tiles(x, R, stage, [&](int64_t g0, int64_t B0, int64_t, uint8_t* stage) {
+        const int64_t A0 = B0 & ~(int64_t)15;
+#pragma unroll
+        for (int u = 0; u < kRaggedU; ++u) {
+            const int64_t g = g0 + u * kThreads + threadIdx.x;
+            if (g < R.total) {
+                int n;
+                const int64_t e = ragged_offset(R, g, n);
+                uint32_t w[8];
+                block_from_stage(stage, 2 * e - A0, n, w);
+                uint32_t c[8];
+                float sd;
+                const uint32_t s8 = encode_block(w, gs, tab, c, sd);
+                st_b64(packed + g * kBlockBytesPacked, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
+                st_u8(scales + g, s8);
+            }
+        }
+    });
 }
 
 __global__ void __launch_bounds__(kThreads)
-    fake_quant_ragged_kernel(const uint16_t* x, uint16_t* y, Ragged R, const float* d_amax) {
+    fake_quant_ragged_kernel(const uint8_t* x, uint8_t* y, Ragged R, const float* d_amax) {
     __shared__ float4 tab[128];
+    extern __shared__ __align__(16) uint8_t stage[];
     const float gs = build_scale_table(tab, d_amax);
-    stream_blocks<1, false, RaggedSlot>(
-        R.total,
-        [&](int64_t g, RaggedSlot& sl) {
-            sl.off = ragged_offset(R, g, sl.n);
-            ld_ragged(x + sl.off, sl.n, sl.w);
-        },
-        [&](int64_t, RaggedSlot& sl) {
-            uint32_t c[8];
-            float sd;
-            encode_block(sl.w, gs, tab, c, sd);
-            uint32_t o[8];
+    // y may be x: the copies read through L2, and a tile's bytes are read before any CTA
+    // writes them (each CTA writes only its own tile's bytes, after reading them).
+    ragged_tiles(x, R, stage, [&](int64_t g0, int64_t B0, int64_t B1, uint8_t* stage) {
+        const int64_t A0 = B0 & ~(int64_t)15;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
-            st_ragged(y + sl.off, sl.n, o);
-        });
+        for (int u = 0; u < kRaggedU; ++u) {
+            const int64_t g = g0 + u * kThreads + threadIdx.x;
+            if (g < R.total) {
+                int n;
+                const int64_t e = ragged_offset(R, g, n);
+                uint32_t w[8];
+                block_from_stage(stage, 2 * e - A0, n, w);
+                uint32_t c[8];
+                float sd;
+                encode_block(w, gs, tab, c, sd);
+                uint32_t o[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
+                block_to_stage(stage, 2 * e - A0, n, o);  // each thread rewrites only its own elements
+            }
+        }
+        __syncthreads();
+        stage_out(y, B0, B1, stage);
+    });
 }
 
 __global__ void __launch_bounds__(kThreads)
     dequantize_ragged_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
-                             const float* __restrict__ d_gs, uint16_t* __restrict__ y, Ragged R) {
+                             const float* __restrict__ d_gs, uint8_t* __restrict__ y, Ragged R) {
     __shared__ float tab_sd[256];
+    extern __shared__ __align__(16) uint8_t stage[];  // one stage: only the outputs are staged
     const float gs = __ldg(d_gs);
     for (int i = threadIdx.x; i < 256; i += blockDim.x) tab_sd[i] = __fdiv_rn(e4m3_to_f32(i), gs);
     __syncthreads();
-    stream_blocks<1, false, PackedSlot>(
-        R.total,
-        [&](int64_t g, PackedSlot& sl) {
-            ld_b64_ro(packed + g * kBlockBytesPacked, sl.p0, sl.p1);
-            sl.s = ld_u8_ro(scales + g);
-        },
-        [&](int64_t g, PackedSlot& sl) {
-            const float sd = tab_sd[sl.s & 0xFFu];
-            uint32_t o[8];
+    for (int64_t g0 = (int64_t)blockIdx.x * kRaggedTile; g0 < R.total; g0 += (int64_t)gridDim.x * kRaggedTile) {
+        int64_t B0, B1;
+        tile_range(R, g0, B0, B1);
+        const int64_t A0 = B0 & ~(int64_t)15;
+        uint32_t p[kRaggedU][2], sb[kRaggedU];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                o[i] = decode_pair((sl.p0 >> (8 * i)) & 0xFFu, sd);
-                o[4 + i] = decode_pair((sl.p1 >> (8 * i)) & 0xFFu, sd);
+        for (int u = 0; u < kRaggedU; ++u) {
+            const int64_t g = g0 + u * kThreads + threadIdx.x;
+            if (g < R.total) {
+                ld_b64_ro(packed + g * kBlockBytesPacked, p[u][0], p[u][1]);
+                sb[u] = ld_u8_ro(scales + g);
             }
-            int n;
-            const int64_t off = ragged_offset(R, g, n);
-            st_ragged(y + off, n, o);
-        });
+        }
+#pragma unroll
+        for (int u = 0; u < kRaggedU; ++u) {
+            const int64_t g = g0 + u * kThreads + threadIdx.x;
+            if (g < R.total) {
+                const float sd = tab_sd[sb[u] & 0xFFu];
+                uint32_t o[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    o[i] = decode_pair((p[u][0] >> (8 * i)) & 0xFFu, sd);
+                    o[4 + i] = decode_pair((p[u][1] >> (8 * i)) & 0xFFu, sd);
+                }
+                int n;
+                const int64_t e = ragged_offset(R, g, n);
+                block_to_stage(stage, 2 * e - A0, n, o);
+            }
+        }
+        __syncthreads();
+        stage_out(y, B0, B1, stage);
+        __syncthreads();
+    }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -615,7 +771,8 @@ nvfp4_status sm_count(int* out) {
     return NVFP4_OK;
 }
 
-// Resident CTAs per SM for a kernel, cached per device (the kernels are fixed, so a
+// Resident CTAs per SM for a kernel launched with `smem` bytes of dynamic shared memory,
+// cached per device (each kernel is always launched with the same shared memory, so a
 // small table keyed by the kernel's address suffices).
 struct OccEntry {
     const void* fn;
@@ -625,7 +782,7 @@ struct OccEntry {
 OccEntry g_occ[64];
 int g_occ_n = 0;
 
-nvfp4_status occupancy(const void* fn, int* out) {
+nvfp4_status occupancy(const void* fn, int* out, size_t smem = 0) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mu);
@@ -635,7 +792,7 @@ nvfp4_status occupancy(const void* fn, int* out) {
             return NVFP4_OK;
         }
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kThreads, 0) != cudaSuccess || n <= 0)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kThreads, smem) != cudaSuccess || n <= 0)
         return NVFP4_ERR_CUDA;
     if (g_occ_n < 64) g_occ[g_occ_n++] = OccEntry{fn, dev, n};
     *out = n;
@@ -644,11 +801,11 @@ nvfp4_status occupancy(const void* fn, int* out) {
 
 // Grid: min(CTAs needed for `items` work items at `per_thread` each, `mult` times the
 // CTAs resident on the whole GPU at once; mult == 0 means no cap).
-nvfp4_status grid_for(const void* fn, int64_t items, int per_thread, int mult, int* grid) {
+nvfp4_status grid_for(const void* fn, int64_t items, int per_thread, int mult, int* grid, size_t smem = 0) {
     int sms = 0, occ = 0;
     nvfp4_status st = sm_count(&sms);
     if (st != NVFP4_OK) return st;
-    st = occupancy(fn, &occ);
+    st = occupancy(fn, &occ, smem);
     if (st != NVFP4_OK) return st;
     const int64_t per_cta = (int64_t)kThreads * per_thread;
     const int64_t need = (items + per_cta - 1) / per_cta;
@@ -689,14 +846,27 @@ Ragged ragged_of(int64_t M, int64_t N) {
     return R;
 }
 
+// The ragged kernels stage kStageBytes of dynamic shared memory per CTA; above the
+// default 48 KB a kernel must opt in once per device.
+template <class K>
+nvfp4_status ragged_smem_optin(K* kernel, int bytes) {
+    if (bytes <= 48 * 1024) return NVFP4_OK;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
+               ? NVFP4_OK
+               : NVFP4_ERR_CUDA;
+}
+
 // Ragged launches shared by the entry points (arguments already validated).
 nvfp4_status launch_fq_ragged(const void* x, void* y, int64_t M, int64_t N, const float* d_amax, nvfp4_stream_t stream) {
     const Ragged R = ragged_of(M, N);
     if (R.total == 0) return NVFP4_OK;
     int grid = 1;
-    nvfp4_status st = grid_for(reinterpret_cast<const void*>(&fake_quant_ragged_kernel), R.total, 1, NVFP4_GRID_FQ, &grid);
+    nvfp4_status st = ragged_smem_optin(fake_quant_ragged_kernel, kStageBytes);
     if (st != NVFP4_OK) return st;
-    fake_quant_ragged_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint16_t*>(x), static_cast<uint16_t*>(y),
+    st = grid_for(reinterpret_cast<const void*>(&fake_quant_ragged_kernel), R.total, kRaggedU, NVFP4_GRID_FQ, &grid,
+                  kStageBytes);
+    if (st != NVFP4_OK) return st;
+    fake_quant_ragged_kernel<<<grid, kThreads, kStageBytes, cs(stream)>>>(static_cast<const uint8_t*>(x), static_cast<uint8_t*>(y),
                                                                 R, d_amax);
     return after_launch();
 }
@@ -1069,9 +1239,12 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const
     if (N % kBlockElems != 0) {
         const Ragged R = ragged_of(M, N);
         int grid = 1;
-        st = grid_for(reinterpret_cast<const void*>(&quantize_ragged_kernel), R.total, 1, NVFP4_GRID_Q, &grid);
+        st = ragged_smem_optin(quantize_ragged_kernel, kStageBytes);
         if (st != NVFP4_OK) return st;
-        quantize_ragged_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint16_t*>(x), R, d_amax, packed,
+        st = grid_for(reinterpret_cast<const void*>(&quantize_ragged_kernel), R.total, kRaggedU, NVFP4_GRID_Q, &grid,
+                      kStageBytes);
+        if (st != NVFP4_OK) return st;
+        quantize_ragged_kernel<<<grid, kThreads, kStageBytes, cs(stream)>>>(static_cast<const uint8_t*>(x), R, d_amax, packed,
                                                                   scales, d_global_scale);
         return after_launch();
     }
@@ -1098,10 +1271,12 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* sc
         const Ragged R = ragged_of(M, N);
         if (R.total == 0) return NVFP4_OK;
         int grid = 1;
-        st = grid_for(reinterpret_cast<const void*>(&dequantize_ragged_kernel), R.total, 1, NVFP4_GRID_DEC, &grid);
+        st = ragged_smem_optin(dequantize_ragged_kernel, kStageBytes);
         if (st != NVFP4_OK) return st;
-        dequantize_ragged_kernel<<<grid, kThreads, 0, cs(stream)>>>(packed, scales, d_global_scale,
-                                                                    static_cast<uint16_t*>(y), R);
+        st = grid_for(reinterpret_cast<const void*>(&dequantize_ragged_kernel), R.total, kRaggedU, NVFP4_GRID_DEC, &grid, kStageBytes);
+        if (st != NVFP4_OK) return st;
+        dequantize_ragged_kernel<<<grid, kThreads, kStageBytes, cs(stream)>>>(packed, scales, d_global_scale,
+                                                                    static_cast<uint8_t*>(y), R);
         return after_launch();
     }
     const int64_t nblk = numel / kBlockElems;

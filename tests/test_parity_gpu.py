@@ -410,3 +410,27 @@ def test_siblings_with_ragged_members():
     assert f32_bits(shared) == f32_bits(a)
     for t, o in zip(xs, outs):
         assert_equal_bits(bits(o), oracle_fake_quant_rows(t, a), f"{t.shape} sibling")
+
+
+@pytest.mark.parametrize("M,N", [(3, 20), (255, 4097), (1000, 33)])
+def test_ragged_outputs_stay_inside_their_tensor(M, N):
+    """Guard bands of 0xA5 bytes around y: the staged edge writes of the ragged kernels
+    touch no byte outside the M*N outputs."""
+    rng = np.random.default_rng(M + 7 * N)
+    x = synthetic.to_bf16_bits(rng.standard_normal((M, N)).astype(np.float32))
+    xd = to_dev(x)
+    a = nv.nvfp4_amax(xd)
+    pad = 64  # elements (128 bytes, keeps y 32-byte aligned)
+    buf = torch.full((pad + M * N + pad,), 0, dtype=torch.int16, device="cuda")
+    buf.view(torch.uint8).fill_(0xA5)
+    y = buf[pad:pad + M * N].view(torch.bfloat16).view(M, N)
+    nv.nvfp4_fake_quant(xd, a, out=y)
+    p, s, gs = nv.nvfp4_quantize(xd, a)
+    want = oracle_fake_quant_rows(x, a.item())
+    for what in ("fake-quant", "dequantize"):
+        head = buf[:pad].view(torch.uint8).cpu().numpy()
+        tail = buf[pad + M * N:].view(torch.uint8).cpu().numpy()
+        assert (head == 0xA5).all() and (tail == 0xA5).all(), f"{what} wrote outside y"
+        assert_equal_bits(bits(y), want, what)
+        buf.view(torch.uint8).fill_(0xA5)
+        nv.nvfp4_dequantize(p, s, gs, out=y, n_cols=N)
