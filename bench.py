@@ -53,6 +53,9 @@ def parse_args():
     p.add_argument("--cpu-rows", type=int, default=2048, help="rows of the oracle sample (cpu_baseline)")
     p.add_argument("--skip-e2e", action="store_true")
     p.add_argument("--skip-cpu-baseline", action="store_true")
+    p.add_argument("--sweep", metavar="OUT_JSON", default=None,
+                   help="instead of the one-line step benchmark, time each kernel on every workload size "
+                        "(L2 flushed before each rep), print a table and write it as JSON to OUT_JSON")
     return p.parse_args()
 
 
@@ -368,8 +371,90 @@ def run_native(args):
     return 0
 
 
+def run_sweep(args):
+    """Per-kernel GB/s on every workload shape: the activation size sweep 1024^2 .. 65536x8192,
+    the 256x1024 and 4096x4096 weights, the 8192x4096 activations and 14336x4096 weight,
+    and the q/k/v siblings.  Each rep is preceded by a read of a 512 MB buffer, so no input
+    starts in L2 and no dirty line is left behind; CUDA events, median of the reps."""
+    import torch
+    from qat_nvfp4_b200 import nvfp4 as nv
+    from qat_nvfp4_b200 import synthetic
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, peak_src = hbm_peak()
+    flush = torch.ones(512 << 20, dtype=torch.uint8, device=dev)
+    ws = nv.new_workspace(dev)
+    reps = 15
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.sum(dtype=torch.int32)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1))
+        return sorted(ts)[len(ts) // 2] / 1e3
+
+    shapes = [("activation sweep", s) for s in synthetic.SWEEP_SHAPES]
+    shapes += [("grid-block weight", (256, 1024)), ("outlier weight", (4096, 4096)),
+               ("W4A4 activation", (8192, 4096)), ("MLP weight", (14336, 4096))]
+    rows = []
+    for name, (M, N) in shapes:
+        x = synthetic.activation_normal_device((M, N), 99, dev)
+        n = M * N
+        amax = nv.nvfp4_amax(x)
+        y = torch.empty_like(x)
+        packed, scales, gs = nv.nvfp4_quantize(x, amax)
+        t = {
+            "amax": (2.0, timed(lambda: nv.nvfp4_amax(x, out=amax, workspace=ws))),
+            "fake_quant": (4.0, timed(lambda: nv.nvfp4_fake_quant(x, amax, out=y))),
+            "fake_quant_with_own_amax": (4.0, timed(lambda: nv.nvfp4_fake_quant_fused(x, out=y, amax_out=amax,
+                                                                                      workspace=ws))),
+            "quantize": (2.5625, timed(lambda: nv.nvfp4_quantize(x, amax, packed, scales, gs))),
+            "dequantize": (2.5625, timed(lambda: nv.nvfp4_dequantize(packed, scales, gs, out=y))),
+        }
+        rec = {"workload": name, "shape": [M, N], "bytes": 2 * n}
+        for k, (bpe, sec) in t.items():
+            rec[k] = {"us": sec * 1e6, "GB/s": n * bpe / sec / 1e9, "frac": n * bpe / sec / 1e9 / peak}
+        rows.append(rec)
+        del x, y, packed, scales
+    # the q/k/v siblings: shared amax + fake-quant of all three in one call
+    qkv = [synthetic.activation_normal_device(s, 98, dev) for s in ((4096, 4096), (1024, 4096), (1024, 4096))]
+    outs = [torch.empty_like(t) for t in qkv]
+    n = sum(t.numel() for t in qkv)
+    amax = torch.empty(1, dtype=torch.float32, device=dev)
+    sec = timed(lambda: nv.nvfp4_fake_quant_siblings(qkv, outs, amax))
+    rows.append({"workload": "q/k/v siblings (shared amax + fake-quant, 2 + 4 bytes/elem)", "shape": [6144, 4096],
+                 "bytes": 2 * n, "siblings": {"us": sec * 1e6, "GB/s": n * 6.0 / sec / 1e9,
+                                               "frac": n * 6.0 / sec / 1e9 / peak}})
+
+    cols = ["amax", "fake_quant", "fake_quant_with_own_amax", "quantize", "dequantize"]
+    print(f"peak {peak:.1f} GB/s ({peak_src}); GB/s of algorithmic bytes (frac of peak); L2 flushed by a read")
+    print("| workload | shape | " + " | ".join(cols) + " |")
+    print("|---|---|" + "---|" * len(cols))
+    for r in rows:
+        if "siblings" in r:
+            v = r["siblings"]
+            print(f"| {r['workload']} | {r['shape'][0]}x{r['shape'][1]} | " + " | ".join(
+                [f"{v['GB/s']:.0f} ({v['frac']:.2f})"] + [""] * (len(cols) - 1)) + " |")
+            continue
+        print(f"| {r['workload']} | {r['shape'][0]}x{r['shape'][1]} | " + " | ".join(
+            f"{r[c]['GB/s']:.0f} ({r[c]['frac']:.2f})" for c in cols) + " |")
+    with open(args.sweep, "w") as f:
+        json.dump({"peak_gbs": peak, "peak_source": peak_src, "rows": rows}, f, indent=1)
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.sweep:
+        return run_sweep(args)
     if args.cols < 1 or args.rows < 1:
         raise SystemExit("--rows and --cols must be positive")
     if args.impl == "reference":

@@ -17,6 +17,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "nvfp4.h"
 #include "nvfp4_device.cuh"
@@ -56,7 +57,7 @@ namespace {
 #define NVFP4_GRID_FQ 32
 #endif
 #ifndef NVFP4_GRID_Q
-#define NVFP4_GRID_Q 16
+#define NVFP4_GRID_Q 8
 #endif
 #ifndef NVFP4_GRID_DEC
 #define NVFP4_GRID_DEC 64
@@ -113,8 +114,10 @@ struct FqList {
 #define NVFP4_SCHED 0
 #endif
 
-template <int kSched, int U, bool kPipe, class Slot, class Load, class Work>
-__device__ __forceinline__ void stream_sched(int64_t nblk, Load load, Work work) {
+struct NoPrologue {};  // marks the plain loop (no prologue to overlap)
+
+template <int kSched, int U, bool kPipe, class Slot, class Load, class Work, class Pro>
+__device__ __forceinline__ void stream_sched(int64_t nblk, Load load, Work work, Pro pro) {
     int64_t ustride, step, end, base;
     if constexpr (kSched == 1) {
         ustride = blockDim.x;
@@ -130,7 +133,7 @@ __device__ __forceinline__ void stream_sched(int64_t nblk, Load load, Work work)
         end = nblk;
         base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     }
-    if constexpr (!kPipe) {
+    if constexpr (std::is_same<Pro, NoPrologue>::value) {
         for (; base < end; base += step) {
             Slot sl[U];
 #pragma unroll
@@ -141,29 +144,57 @@ __device__ __forceinline__ void stream_sched(int64_t nblk, Load load, Work work)
                 if (base + u * ustride < end) work(base + u * ustride, sl[u]);
         }
     } else {
-        Slot nxt[U];
+        // The first group's loads go out before the prologue (the per-CTA scale table and its
+        // barrier, run by every thread), so that the table is built under the load latency.
+        Slot cur[U];
 #pragma unroll
         for (int u = 0; u < U; ++u)
-            if (base + u * ustride < end) load(base + u * ustride, nxt[u]);
-        while (base < end) {
-            Slot cur[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) cur[u] = nxt[u];
-            const int64_t cb = base;
-            base += step;
+            if (base + u * ustride < end) load(base + u * ustride, cur[u]);
+        pro();
+        if constexpr (!kPipe) {
 #pragma unroll
             for (int u = 0; u < U; ++u)
-                if (base + u * ustride < end) load(base + u * ustride, nxt[u]);
+                if (base + u * ustride < end) work(base + u * ustride, cur[u]);
+            for (base += step; base < end; base += step) {
+                Slot sl[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u)
-                if (cb + u * ustride < end) work(cb + u * ustride, cur[u]);
+                for (int u = 0; u < U; ++u)
+                    if (base + u * ustride < end) load(base + u * ustride, sl[u]);
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (base + u * ustride < end) work(base + u * ustride, sl[u]);
+            }
+        } else {
+            while (base < end) {
+                Slot nxt[U];
+                const int64_t cb = base;
+                base += step;
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (base + u * ustride < end) load(base + u * ustride, nxt[u]);
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (cb + u * ustride < end) work(cb + u * ustride, cur[u]);
+#pragma unroll
+                for (int u = 0; u < U; ++u) cur[u] = nxt[u];
+            }
         }
     }
 }
 
+template <int kSched, int U, bool kPipe, class Slot, class Load, class Work>
+__device__ __forceinline__ void stream_sched(int64_t nblk, Load load, Work work) {
+    stream_sched<kSched, U, kPipe, Slot>(nblk, load, work, NoPrologue{});
+}
+
+template <int U, bool kPipe, class Slot, class Load, class Work, class Pro>
+__device__ __forceinline__ void stream_blocks(int64_t nblk, Load load, Work work, Pro pro) {
+    stream_sched<NVFP4_SCHED, U, kPipe, Slot>(nblk, load, work, pro);
+}
+
 template <int U, bool kPipe, class Slot, class Load, class Work>
 __device__ __forceinline__ void stream_blocks(int64_t nblk, Load load, Work work) {
-    stream_sched<NVFP4_SCHED, U, kPipe, Slot>(nblk, load, work);
+    stream_sched<NVFP4_SCHED, U, kPipe, Slot>(nblk, load, work, NoPrologue{});
 }
 
 struct Block32 {
@@ -302,8 +333,7 @@ __global__ void __launch_bounds__(kThreads)
     quantize_kernel(const uint8_t* __restrict__ x, int64_t nblk, const float* __restrict__ d_amax,
                     uint8_t* __restrict__ packed, uint8_t* __restrict__ scales, float* __restrict__ d_gs) {
     __shared__ float4 tab[128];
-    const float gs = build_scale_table(tab, d_amax);
-    if (d_gs != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *d_gs = gs;
+    float gs = 0.0f;
     stream_blocks<kUnrollQ, NVFP4_PIPE_Q != 0, Block32>(
         nblk, [&](int64_t bi, Block32& b) { ld_b256_ro(x + bi * kBlockBytesIn, b.w); },
         [&](int64_t bi, Block32& b) {
@@ -312,6 +342,10 @@ __global__ void __launch_bounds__(kThreads)
             const uint32_t s8 = encode_block(b.w, gs, tab, c, sd);
             st_b64(packed + bi * kBlockBytesPacked, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
             st_u8(scales + bi, s8);
+        },
+        [&] {
+            gs = build_scale_table(tab, d_amax);
+            if (d_gs != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *d_gs = gs;
         });
 }
 
@@ -337,7 +371,7 @@ __device__ __forceinline__ void locate_fq(const FqList& L, int64_t bi, const uin
 template <bool kMulti>
 __global__ void __launch_bounds__(kThreads) fake_quant_kernel(FqList L, int64_t nblk, const float* d_amax) {
     __shared__ float4 tab[128];
-    const float gs = build_scale_table(tab, d_amax);
+    float gs = 0.0f;
     stream_blocks<kUnrollFq, NVFP4_PIPE_FQ != 0, FqSlot>(
         nblk,
         [&](int64_t bi, FqSlot& sl) {
@@ -353,7 +387,8 @@ __global__ void __launch_bounds__(kThreads) fake_quant_kernel(FqList L, int64_t 
 #pragma unroll
             for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
             st_b256(sl.y, o);
-        });
+        },
+        [&] { gs = build_scale_table(tab, d_amax); });
 }
 
 // ---------------------------------------------------------------------------------------
@@ -459,9 +494,6 @@ __global__ void __launch_bounds__(kThreads)
     dequantize_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
                       const float* __restrict__ d_gs, uint8_t* __restrict__ y, int64_t nblk) {
     __shared__ float tab_sd[256];  // sd for every possible scale byte
-    const float gs = __ldg(d_gs);
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) tab_sd[i] = __fdiv_rn(e4m3_to_f32(i), gs);
-    __syncthreads();
     stream_blocks<kUnrollDecode, NVFP4_PIPE_DEC != 0, PackedSlot>(
         nblk,
         [&](int64_t bi, PackedSlot& sl) {
@@ -477,6 +509,11 @@ __global__ void __launch_bounds__(kThreads)
                 o[4 + i] = decode_pair((sl.p1 >> (8 * i)) & 0xFFu, sd);
             }
             st_b256(y + bi * kBlockBytesIn, o);
+        },
+        [&] {
+            const float gs = __ldg(d_gs);
+            for (int i = threadIdx.x; i < 256; i += blockDim.x) tab_sd[i] = __fdiv_rn(e4m3_to_f32(i), gs);
+            __syncthreads();
         });
 }
 
