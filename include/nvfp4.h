@@ -218,6 +218,21 @@ nvfp4_status nvfp4_observe_amax_noalloc(const void* x, int64_t numel, float* d_s
 nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
                             uint8_t* scales, float* d_global_scale, nvfp4_stream_t stream);
 
+/* nvfp4_quantize writing the block scales in the layout of the sm_100 block-scaled
+ * tensor-core GEMM (NVFP4 operands with 16-element E4M3 scale vectors), so that packed
+ * and scales_mma can be handed to such a GEMM as they are (with 1 / global_scale as the
+ * operand's per-tensor decode factor).  Not on the pages, which store the plain layout;
+ * codes, packed bytes and scale values are those of nvfp4_quantize.
+ *   scales_mma  uint8 out, R128 * C4 bytes, 16-byte aligned, R128 = 128 * ceil(M / 128),
+ *               C4 = 4 * ceil(B / 4), B = ceil(N / 16) blocks per row.  The [R128, C4]
+ *               scale matrix (zero past M rows and B columns) is stored as 128 x 4 tiles,
+ *               tile (tr, tc) at byte 512 * (tr * C4 / 4 + tc), and inside a tile the
+ *               scale of row r, column c at (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4.
+ * Other arguments and errors as for nvfp4_quantize.  Enqueues a memset of scales_mma when
+ * there is padding, and one kernel. */
+nvfp4_status nvfp4_quantize_mma(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
+                                uint8_t* scales_mma, float* d_global_scale, nvfp4_stream_t stream);
+
 /* Dequantize: y = bf16_rne(LUT[code] * (E4M3(byte) / gs)), no clamp on this side.
  * [FP4OPT] dequantize_weight_from_float4.
  *   packed  uint8 [M, P/2], 8-byte aligned     scales  uint8 [M, P/16]

@@ -327,11 +327,34 @@ __device__ __forceinline__ float build_scale_table(float4* tab, const float* d_a
 }
 
 // ---------------------------------------------------------------------------------------
+// Scale layouts.  Row-major: the byte of block (r, c) is at r * nb + c.  The block-scaled
+// tensor-core layout (the one cuBLAS documents for 1-D block scaling factors): the
+// [rows, nb] scale matrix, zero-padded to multiples of 128 rows and 4 columns, is cut into
+// 128 x 4 tiles stored one after another (tile row-major over (r / 128, c / 4)), and inside
+// a tile byte (r, c) sits at (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4).
+
+__device__ __forceinline__ int64_t mma_scale_offset(int64_t r, int64_t c, int64_t ncb) {
+    return ((r >> 7) * ncb + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
+}
+
+// Where the scale byte of block g goes (nb blocks per row; ncb = ceil(nb / 4) tiles per
+// tile-row).  kMma == false is the plain row-major layout.
+template <bool kMma>
+__device__ __forceinline__ int64_t scale_offset(int64_t g, int64_t nb, int64_t ncb, bool small) {
+    if (!kMma) return g;
+    const int64_t r = small ? (int64_t)((uint32_t)g / (uint32_t)nb) : g / nb;
+    return mma_scale_offset(r, g - r * nb, ncb);
+}
+
+// ---------------------------------------------------------------------------------------
 // Quantize: bf16 blocks -> 8 bytes of codes + 1 scale byte.
 
+template <bool kMma>
 __global__ void __launch_bounds__(kThreads)
     quantize_kernel(const uint8_t* __restrict__ x, int64_t nblk, const float* __restrict__ d_amax,
-                    uint8_t* __restrict__ packed, uint8_t* __restrict__ scales, float* __restrict__ d_gs) {
+                    uint8_t* __restrict__ packed, uint8_t* __restrict__ scales, float* __restrict__ d_gs, int64_t nb,
+                    int64_t ncb) {
+    const bool small = nblk <= 0xFFFFFFFFll;
     __shared__ float4 tab[128];
     float gs = 0.0f;
     stream_blocks<kUnrollQ, NVFP4_PIPE_Q != 0, Block32>(
@@ -341,7 +364,7 @@ __global__ void __launch_bounds__(kThreads)
             float sd;
             const uint32_t s8 = encode_block(b.w, gs, tab, c, sd);
             st_b64(packed + bi * kBlockBytesPacked, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
-            st_u8(scales + bi, s8);
+            st_u8(scales + scale_offset<kMma>(bi, nb, ncb, small), s8);
         },
         [&] {
             gs = build_scale_table(tab, d_amax);
@@ -686,9 +709,12 @@ __device__ __forceinline__ void ragged_tiles(const uint8_t* src, const Ragged& R
     }
 }
 
+template <bool kMma>
 __global__ void __launch_bounds__(kThreads)
     quantize_ragged_kernel(const uint8_t* __restrict__ x, Ragged R, const float* __restrict__ d_amax,
-                           uint8_t* __restrict__ packed, uint8_t* __restrict__ scales, float* __restrict__ d_gs) {
+                           uint8_t* __restrict__ packed, uint8_t* __restrict__ scales, float* __restrict__ d_gs,
+                           int64_t ncb) {
+    const bool small = R.total <= 0xFFFFFFFFll;
     __shared__ float4 tab[128];
     extern __shared__ __align__(16) uint8_t stage[];
     const float gs = build_scale_table(tab, d_amax);
@@ -707,7 +733,7 @@ __global__ void __launch_bounds__(kThreads)
                 float sd;
                 const uint32_t s8 = encode_block(w, gs, tab, c, sd);
                 st_b64(packed + g * kBlockBytesPacked, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
-                st_u8(scales + g, s8);
+                st_u8(scales + scale_offset<kMma>(g, R.nb, ncb, small), s8);
             }
         }
     });
@@ -1264,8 +1290,9 @@ NVFP4_API nvfp4_status nvfp4_selftest_barrier_timeout(const void* x, void* y, in
                         0, 0.f, 0.f, 1u, (uint64_t)timeout_us * 1000ull, stream);
 }
 
-NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
-                                      uint8_t* scales, float* d_global_scale, nvfp4_stream_t stream) {
+template <bool kMma>
+static nvfp4_status quantize_impl(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
+                                  uint8_t* scales, float* d_global_scale, nvfp4_stream_t stream) {
     int64_t numel = 0;
     nvfp4_status st = check_matrix(M, N, &numel);
     if (st != NVFP4_OK) return st;
@@ -1273,26 +1300,44 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const
     if (numel > 0 && (x == nullptr || packed == nullptr || scales == nullptr)) return NVFP4_ERR_NULL;
     if (!aligned(d_amax, 4) || (d_global_scale && !aligned(d_global_scale, 4))) return NVFP4_ERR_ALIGN;
     if (numel > 0 && (!aligned(x, 32) || !aligned(packed, 8))) return NVFP4_ERR_ALIGN;
+    const Ragged R = ragged_of(M, N);
+    const int64_t ncb = (R.nb + 3) / 4;
+    if (kMma && numel > 0) {
+        // The tile padding (rows past M, columns past nb) must read as zero scales.
+        const int64_t rows_p = (M + 127) / 128 * 128;
+        if (rows_p != M || ncb * 4 != R.nb)
+            if (cudaMemsetAsync(scales, 0, (size_t)(rows_p * ncb * 4), cs(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
+    }
     if (N % kBlockElems != 0) {
-        const Ragged R = ragged_of(M, N);
         int grid = 1;
-        st = ragged_smem_optin(quantize_ragged_kernel, kStageBytes);
+        st = ragged_smem_optin(quantize_ragged_kernel<kMma>, kStageBytes);
         if (st != NVFP4_OK) return st;
-        st = grid_for(reinterpret_cast<const void*>(&quantize_ragged_kernel), R.total, kRaggedU, NVFP4_GRID_Q, &grid,
-                      kStageBytes);
+        st = grid_for(reinterpret_cast<const void*>(&quantize_ragged_kernel<kMma>), R.total, kRaggedU, NVFP4_GRID_Q,
+                      &grid, kStageBytes);
         if (st != NVFP4_OK) return st;
-        quantize_ragged_kernel<<<grid, kThreads, kStageBytes, cs(stream)>>>(static_cast<const uint8_t*>(x), R, d_amax, packed,
-                                                                  scales, d_global_scale);
+        quantize_ragged_kernel<kMma><<<grid, kThreads, kStageBytes, cs(stream)>>>(
+            static_cast<const uint8_t*>(x), R, d_amax, packed, scales, d_global_scale, ncb);
         return after_launch();
     }
     const int64_t nblk = numel / kBlockElems;
     if (nblk == 0 && d_global_scale == nullptr) return NVFP4_OK;
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&quantize_kernel), nblk, kUnrollQ, NVFP4_GRID_Q, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&quantize_kernel<kMma>), nblk, kUnrollQ, NVFP4_GRID_Q, &grid);
     if (st != NVFP4_OK) return st;
-    quantize_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), nblk, d_amax, packed, scales,
-                                                       d_global_scale);
+    quantize_kernel<kMma><<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), nblk, d_amax, packed,
+                                                             scales, d_global_scale, R.nb > 0 ? R.nb : 1, ncb);
     return after_launch();
+}
+
+NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
+                                      uint8_t* scales, float* d_global_scale, nvfp4_stream_t stream) {
+    return quantize_impl<false>(x, M, N, d_amax, packed, scales, d_global_scale, stream);
+}
+
+NVFP4_API nvfp4_status nvfp4_quantize_mma(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
+                                          uint8_t* scales_mma, float* d_global_scale, nvfp4_stream_t stream) {
+    if (M > 0 && N > 0 && scales_mma != nullptr && !aligned(scales_mma, 16)) return NVFP4_ERR_ALIGN;
+    return quantize_impl<true>(x, M, N, d_amax, packed, scales_mma, d_global_scale, stream);
 }
 
 NVFP4_API nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* scales, const float* d_global_scale,

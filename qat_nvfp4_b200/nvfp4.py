@@ -59,6 +59,7 @@ _c_workspace_check = _sig("nvfp4_workspace_check", [_vp, _vp])
 _c_selftest_barrier_timeout = _sig("nvfp4_selftest_barrier_timeout",
                                    [_vp, _vp, _i64, _i64, _vp, _vp, ctypes.c_uint32, _vp])
 _c_quantize = _sig("nvfp4_quantize", [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp])
+_c_quantize_mma = _sig("nvfp4_quantize_mma", [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp])
 _c_dequantize = _sig("nvfp4_dequantize", [_vp, _vp, _vp, _i64, _i64, _vp, _vp])
 _c_fake_quant = _sig("nvfp4_fake_quant", [_vp, _vp, _i64, _i64, _vp, _vp])
 _c_fake_quant_siblings = _sig("nvfp4_fake_quant_siblings",
@@ -236,6 +237,37 @@ def nvfp4_quantize(x: torch.Tensor, amax: torch.Tensor, packed: torch.Tensor | N
         _check(_c_quantize(x.data_ptr(), M, N, amax.data_ptr(), packed.data_ptr(), scales.data_ptr(),
                            global_scale.data_ptr(), _stream(x.device)), "nvfp4_quantize")
     return packed, scales, global_scale
+
+
+def mma_scale_bytes(M: int, N: int) -> int:
+    """Bytes of the tensor-core scale layout for an [M, N] tensor: 128 * ceil(M / 128)
+    rows by 4 * ceil(B / 4) columns, B = ceil(N / 16)."""
+    return (M + 127) // 128 * 128 * ((padded_blocks(N) + 3) // 4 * 4)
+
+
+def nvfp4_quantize_mma(x: torch.Tensor, amax: torch.Tensor, packed: torch.Tensor | None = None,
+                       scales_mma: torch.Tensor | None = None, global_scale: torch.Tensor | None = None):
+    """nvfp4_quantize with the block scales written in the block-scaled tensor-core GEMM
+    layout (128 x 4 tiles).  Returns (packed [..., 8*B], scales_mma uint8 [mma_scale_bytes],
+    global scale fp32 [1]); the GEMM's per-tensor decode factor is 1 / global scale."""
+    M, N = _matrix(x)
+    _scalar(amax, "amax")
+    B = padded_blocks(N)
+    if packed is None:
+        packed = torch.empty(tuple(x.shape[:-1]) + (8 * B,), dtype=torch.uint8, device=x.device)
+    if scales_mma is None:
+        scales_mma = torch.empty(mma_scale_bytes(M, N), dtype=torch.uint8, device=x.device)
+    if global_scale is None:
+        global_scale = torch.empty(1, dtype=torch.float32, device=x.device)
+    _cuda(packed, "packed", torch.uint8)
+    _cuda(scales_mma, "scales_mma", torch.uint8)
+    _scalar(global_scale, "global_scale")
+    if packed.numel() != M * 8 * B or scales_mma.numel() != mma_scale_bytes(M, N):
+        raise RuntimeError("packed / scales_mma have the wrong number of elements")
+    with torch.cuda.device(x.device):
+        _check(_c_quantize_mma(x.data_ptr(), M, N, amax.data_ptr(), packed.data_ptr(), scales_mma.data_ptr(),
+                               global_scale.data_ptr(), _stream(x.device)), "nvfp4_quantize_mma")
+    return packed, scales_mma, global_scale
 
 
 def nvfp4_dequantize(packed: torch.Tensor, scales: torch.Tensor, global_scale: torch.Tensor,
