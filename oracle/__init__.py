@@ -58,6 +58,12 @@ def _lib():
         lib.oracle_dequantize.restype = None
         lib.oracle_fake_quant.argtypes = [u16p, i64, i64, f32, u16p]
         lib.oracle_fake_quant.restype = ctypes.c_int
+        lib.oracle_quantize_bs.argtypes = [u16p, i64, i64, i64, f32, u8p, u8p]
+        lib.oracle_quantize_bs.restype = ctypes.c_int
+        lib.oracle_dequantize_bs.argtypes = [u8p, u8p, f32, i64, i64, i64, u16p]
+        lib.oracle_dequantize_bs.restype = ctypes.c_int
+        lib.oracle_fake_quant_bs.argtypes = [u16p, i64, i64, i64, f32, u16p]
+        lib.oracle_fake_quant_bs.restype = ctypes.c_int
         lib.oracle_observer_update.argtypes = [f32, f32, ctypes.c_int, ctypes.c_double]
         lib.oracle_observer_update.restype = f32
         _LIB = lib
@@ -135,40 +141,46 @@ def global_scale(amax_value: float) -> float:
     return _lib().oracle_global_scale(f32(amax_value))
 
 
-def padded_blocks(N: int) -> int:
-    """Blocks per row: ceil(N / 16) (rows are zero-padded to a multiple of 16)."""
-    return (N + 15) // 16
+def padded_blocks(N: int, block: int = 16) -> int:
+    """Blocks per row: ceil(N / block) (rows are zero-padded to a multiple of block)."""
+    return (N + block - 1) // block
 
 
-def quantize(x_bits, global_scale_value: float):
-    """x_bits: uint16 [M, N].  Returns (packed [M, 8*B], scales [M, B]), B = ceil(N/16)."""
+def quantize(x_bits, global_scale_value: float, block: int = 16):
+    """x_bits: uint16 [M, N].  Returns (packed [M, B*block/2], scales [M, B]),
+    B = ceil(N / block)."""
     a, p = _u16(x_bits)
     M, N = a.shape
-    B = padded_blocks(N)
-    packed = np.empty((M, 8 * B), dtype=np.uint8)
+    B = padded_blocks(N, block)
+    packed = np.empty((M, B * block // 2), dtype=np.uint8)
     scales = np.empty((M, B), dtype=np.uint8)
-    _lib().oracle_quantize(p, M, N, f32(global_scale_value),
-                           packed.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
-                           scales.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    rc = _lib().oracle_quantize_bs(p, M, N, block, f32(global_scale_value),
+                                   packed.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+                                   scales.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    if rc != 0:
+        raise ValueError(f"oracle_quantize_bs failed (block {block})")
     return packed, scales
 
 
-def dequantize(packed, scales, global_scale_value: float, M: int, N: int):
+def dequantize(packed, scales, global_scale_value: float, M: int, N: int, block: int = 16):
     pk, pp = _u8(packed)
     sc, sp = _u8(scales)
     y = np.empty((M, N), dtype=np.uint16)
-    _lib().oracle_dequantize(pp, sp, f32(global_scale_value), M, N,
-                             y.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)))
+    rc = _lib().oracle_dequantize_bs(pp, sp, f32(global_scale_value), M, N, block,
+                                     y.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)))
+    if rc != 0:
+        raise ValueError(f"oracle_dequantize_bs failed (block {block})")
     return y
 
 
-def fake_quant(x_bits, amax_value: float):
+def fake_quant(x_bits, amax_value: float, block: int = 16):
     a, p = _u16(x_bits)
     M, N = a.shape
     y = np.empty((M, N), dtype=np.uint16)
-    rc = _lib().oracle_fake_quant(p, M, N, f32(amax_value), y.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)))
+    rc = _lib().oracle_fake_quant_bs(p, M, N, block, f32(amax_value),
+                                     y.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)))
     if rc != 0:
-        raise MemoryError("oracle_fake_quant could not allocate its temporaries")
+        raise ValueError(f"oracle_fake_quant_bs failed (block {block})")
     return y
 
 

@@ -168,10 +168,12 @@ ORACLE_API float oracle_global_scale(float amax) {
     return numerator / a;
 }
 
-/* [FP4OPT] quantize_weight_to_float4 for a row-major [M, N] bf16 tensor, given its
- * per-tensor global_scale.  When N % 16 != 0 each row is first padded on the right with
- * zeros to P = 16 * ceil(N / 16) columns (the page's `pad = (-features) % block_size`
- * branch), and the padded row is quantized.  Per 16-element block along the row:
+/* [FP4OPT] quantize_weight_to_float4(tensor, block_size) for a row-major [M, N] bf16
+ * tensor, given its per-tensor global_scale and the block size B (16 for NVFP4; the page's
+ * function takes the block size as an argument, and 32 is accepted here as well).  When
+ * N % B != 0 each row is first padded on the right with zeros to P = B * ceil(N / B)
+ * columns (the page's `pad = (-features) % block_size` branch), and the padded row is
+ * quantized.  Per block of B elements along the row:
  *   block_amax      = max |x|
  *   block_scale_fp8 = E4M3((block_amax / 6) * global_scale)
  *   block_scale     = max(float(block_scale_fp8) / global_scale, 1e-12)
@@ -179,19 +181,25 @@ ORACLE_API float oracle_global_scale(float amax) {
  *   idx             = _float4_round(|scaled|)
  *   code            = idx + 8 if scaled < 0 else idx
  *   packed[j]       = code[2j] | code[2j+1] << 4
- * packed is [M, P/2] bytes, scales is [M, P/16] E4M3 bytes, both row-major. */
-ORACLE_API void oracle_quantize(const uint16_t* x, int64_t M, int64_t N, float global_scale,
-                                uint8_t* packed, uint8_t* scales) {
-    int64_t nblk = (N + FLOAT4_BLOCK - 1) / FLOAT4_BLOCK;
-    int64_t P = nblk * FLOAT4_BLOCK;
+ * packed is [M, P/2] bytes, scales is [M, P/B] E4M3 bytes, both row-major.  Returns -1
+ * for an unsupported block size or if the row buffer cannot be allocated, else 0. */
+#define MAX_BLOCK 32
+
+static int block_ok(int64_t B) { return B == 16 || B == 32; }
+
+ORACLE_API int oracle_quantize_bs(const uint16_t* x, int64_t M, int64_t N, int64_t B, float global_scale,
+                                  uint8_t* packed, uint8_t* scales) {
+    if (!block_ok(B)) return -1;
+    int64_t nblk = (N + B - 1) / B;
+    int64_t P = nblk * B;
     uint16_t* row = (uint16_t*)calloc((size_t)(P ? P : 1), sizeof(uint16_t)); /* zero padding */
-    if (!row) return;
+    if (!row) return -1;
     for (int64_t r = 0; r < M; ++r) {
         memcpy(row, x + r * N, (size_t)N * sizeof(uint16_t));
         for (int64_t b = 0; b < nblk; ++b) {
-            const uint16_t* xb = row + b * FLOAT4_BLOCK;
+            const uint16_t* xb = row + b * B;
             float block_amax = 0.0f;
-            for (int i = 0; i < FLOAT4_BLOCK; ++i) {
+            for (int i = 0; i < B; ++i) {
                 float v = fabsf(oracle_bf16_to_f32(xb[i]));
                 if (v > block_amax) block_amax = v;
             }
@@ -202,59 +210,79 @@ ORACLE_API void oracle_quantize(const uint16_t* x, int64_t M, int64_t N, float g
             if (block_scale < TINY_CLAMP) block_scale = TINY_CLAMP;
             scales[r * nblk + b] = s8;
 
-            uint8_t code[FLOAT4_BLOCK];
-            for (int i = 0; i < FLOAT4_BLOCK; ++i) {
+            uint8_t code[MAX_BLOCK];
+            for (int i = 0; i < B; ++i) {
                 float scaled = oracle_bf16_to_f32(xb[i]) / block_scale;
                 if (scaled < -FLOAT4_MAX) scaled = -FLOAT4_MAX;
                 if (scaled > FLOAT4_MAX) scaled = FLOAT4_MAX;
                 int idx = oracle_e2m1_round_index(fabsf(scaled));
                 code[i] = (uint8_t)(scaled < 0.0f ? idx + 8 : idx);
             }
-            uint8_t* pb = packed + r * (P / 2) + b * (FLOAT4_BLOCK / 2);
-            for (int j = 0; j < FLOAT4_BLOCK / 2; ++j)
+            uint8_t* pb = packed + r * (P / 2) + b * (B / 2);
+            for (int j = 0; j < B / 2; ++j)
                 pb[j] = (uint8_t)(code[2 * j] | (code[2 * j + 1] << 4));
         }
     }
     free(row);
+    return 0;
+}
+
+/* The NVFP4 block size of 16. */
+ORACLE_API void oracle_quantize(const uint16_t* x, int64_t M, int64_t N, float global_scale,
+                                uint8_t* packed, uint8_t* scales) {
+    oracle_quantize_bs(x, M, N, FLOAT4_BLOCK, global_scale, packed, scales);
 }
 
 /* [FP4OPT] dequantize_weight_from_float4: split each byte into (low, high) nibbles,
  * look the codes up in FLOAT4_LUT, multiply by float(block_scale_fp8) / global_scale
  * (no clamp on this side) and round the fp32 product to bf16.  packed / scales hold the
- * P = 16 * ceil(N / 16) padded columns; the result is cropped to the first N (the page's
- * `[:, :shape[1]]`). */
-ORACLE_API void oracle_dequantize(const uint8_t* packed, const uint8_t* scales, float global_scale,
-                                  int64_t M, int64_t N, uint16_t* y) {
-    int64_t nblk = (N + FLOAT4_BLOCK - 1) / FLOAT4_BLOCK;
-    int64_t P = nblk * FLOAT4_BLOCK;
+ * P = B * ceil(N / B) padded columns; the result is cropped to the first N (the page's
+ * `[:, :shape[1]]`).  Returns -1 for an unsupported block size, else 0. */
+ORACLE_API int oracle_dequantize_bs(const uint8_t* packed, const uint8_t* scales, float global_scale,
+                                    int64_t M, int64_t N, int64_t B, uint16_t* y) {
+    if (!block_ok(B)) return -1;
+    int64_t nblk = (N + B - 1) / B;
+    int64_t P = nblk * B;
     for (int64_t r = 0; r < M; ++r) {
         for (int64_t c = 0; c < N; ++c) {
             uint8_t byte = packed[r * (P / 2) + c / 2];
             int code = (c % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
             float value = oracle_e2m1_lut(code);
-            float block_scale = oracle_e4m3_decode(scales[r * nblk + c / FLOAT4_BLOCK]) / global_scale;
+            float block_scale = oracle_e4m3_decode(scales[r * nblk + c / B]) / global_scale;
             float out = value * block_scale;
             y[r * N + c] = oracle_f32_to_bf16(out);
         }
     }
+    return 0;
+}
+
+ORACLE_API void oracle_dequantize(const uint8_t* packed, const uint8_t* scales, float global_scale,
+                                  int64_t M, int64_t N, uint16_t* y) {
+    oracle_dequantize_bs(packed, scales, global_scale, M, N, FLOAT4_BLOCK, y);
 }
 
 /* Fake-quantization, bf16 -> bf16: dequantize(quantize(x)) with the per-tensor scale
- * derived from `amax` ([QATLIN] section 2 forward, with [FP4OPT]'s formulas).  The
- * straight-through backward is the identity and needs no oracle.  Returns 0 on success,
- * -1 if the temporaries cannot be allocated. */
-ORACLE_API int oracle_fake_quant(const uint16_t* x, int64_t M, int64_t N, float amax, uint16_t* y) {
+ * derived from `amax` ([QATLIN] section 2 forward, with [FP4OPT]'s formulas) and blocks of
+ * B elements.  The straight-through backward is the identity and needs no oracle.
+ * Returns 0 on success, -1 for an unsupported block size or if the temporaries cannot be
+ * allocated. */
+ORACLE_API int oracle_fake_quant_bs(const uint16_t* x, int64_t M, int64_t N, int64_t B, float amax, uint16_t* y) {
+    if (!block_ok(B)) return -1;
     float gs = oracle_global_scale(amax);
-    int64_t nblk = (N + FLOAT4_BLOCK - 1) / FLOAT4_BLOCK;
-    size_t npacked = (size_t)M * (size_t)(nblk * 8), nscale = (size_t)M * (size_t)nblk;
+    int64_t nblk = (N + B - 1) / B;
+    size_t npacked = (size_t)M * (size_t)(nblk * B / 2), nscale = (size_t)M * (size_t)nblk;
     uint8_t* packed = (uint8_t*)malloc(npacked ? npacked : 1);
     uint8_t* scales = (uint8_t*)malloc(nscale ? nscale : 1);
     if (!packed || !scales) { free(packed); free(scales); return -1; }
-    oracle_quantize(x, M, N, gs, packed, scales);
-    oracle_dequantize(packed, scales, gs, M, N, y);
+    int rc = oracle_quantize_bs(x, M, N, B, gs, packed, scales);
+    if (rc == 0) rc = oracle_dequantize_bs(packed, scales, gs, M, N, B, y);
     free(packed);
     free(scales);
-    return 0;
+    return rc;
+}
+
+ORACLE_API int oracle_fake_quant(const uint16_t* x, int64_t M, int64_t N, float amax, uint16_t* y) {
+    return oracle_fake_quant_bs(x, M, N, FLOAT4_BLOCK, amax, y);
 }
 
 /* [QATLIN] section 5, one observer step given the current amax `cur` (after any

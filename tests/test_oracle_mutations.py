@@ -48,6 +48,8 @@ MUTATIONS = [
      "float v = oracle_bf16_to_f32(xb[i]);"),
     ("e4m3 exponent bias", "ldexp((double)(8 + m), e - 10)", "ldexp((double)(8 + m), e - 11)"),
     ("e2m1 lut sign", "return (code & 8) ? -m : m;", "return m;"),
+    ("block size ignored", "const uint16_t* xb = row + b * B;\n            float block_amax = 0.0f;\n            for (int i = 0; i < B; ++i) {",
+     "const uint16_t* xb = row + b * B;\n            float block_amax = 0.0f;\n            for (int i = 0; i < 16; ++i) {"),
 ]
 
 

@@ -220,15 +220,16 @@ def test_worked_examples(golden_dir):
         gs = oracle.global_scale(amax)
         if "global_scale" in case:
             assert gs == case["global_scale"], case["name"]
-        packed, scales = oracle.quantize(x, gs)
+        block = case.get("block", 16)
+        packed, scales = oracle.quantize(x, gs, block)
         assert list(scales.ravel()) == case["scales"], case["name"]
         assert list(_unpack(packed).ravel()) == case["codes"], case["name"]
         assert list(packed.ravel()) == case["packed"], case["name"]
-        y = oracle.dequantize(packed, scales, gs, M, N)
+        y = oracle.dequantize(packed, scales, gs, M, N, block)
         expect = _bf16_bits(np.array(case["dequant"], dtype=np.float32).reshape(M, N))
         np.testing.assert_array_equal(y, expect, err_msg=case["name"])
         # fake-quant is dequantize(quantize(x)) bit for bit
-        np.testing.assert_array_equal(oracle.fake_quant(x, amax), expect, err_msg=case["name"])
+        np.testing.assert_array_equal(oracle.fake_quant(x, amax, block), expect, err_msg=case["name"])
 
 
 def _grid_block_expectations(block):
@@ -411,3 +412,52 @@ def test_padding_is_zero_padding_then_crop(N):
     # the padded positions hold code 0
     codes = _unpack(packed)
     assert not codes[:, N:].any()
+
+
+def test_block_32_equals_block_16_when_both_halves_share_their_amax():
+    """With block 32 each block's scale comes from its 32-element amax; when the two
+    16-element halves of every 32-block have the same amax, the scales and therefore all
+    codes coincide with those of blocks of 16 (every other 16-block scale byte)."""
+    rng = np.random.default_rng(32)
+    M, N = 24, 256
+    v = rng.standard_normal((M, N // 32, 2, 16)).astype(np.float32)
+    peak = np.abs(v).max(axis=(2, 3))
+    v[:, :, 0, 0] = peak * np.sign(v[:, :, 0, 0] + 0.5)  # both halves hold the block's max
+    v[:, :, 1, 3] = peak
+    x = synthetic.to_bf16_bits(v.reshape(M, N))
+    a = oracle.amax(x)
+    gs = oracle.global_scale(a)
+    p16, s16 = oracle.quantize(x, gs, 16)
+    p32, s32 = oracle.quantize(x, gs, 32)
+    np.testing.assert_array_equal(s16[:, 0::2], s16[:, 1::2])
+    np.testing.assert_array_equal(s32, s16[:, 0::2])
+    np.testing.assert_array_equal(p32, p16)
+    np.testing.assert_array_equal(oracle.fake_quant(x, a, 32), oracle.fake_quant(x, a, 16))
+
+
+@pytest.mark.parametrize("N", [20, 33, 1000])
+def test_block_32_padding(N):
+    rng = np.random.default_rng(N + 32)
+    x = synthetic.to_bf16_bits(rng.standard_normal((5, N)).astype(np.float32))
+    P = 32 * ((N + 31) // 32)
+    xp = np.zeros((5, P), dtype=np.uint16)
+    xp[:, :N] = x
+    gs = oracle.global_scale(oracle.amax(x))
+    np.testing.assert_array_equal(np.concatenate(oracle.quantize(x, gs, 32), axis=1),
+                                  np.concatenate(oracle.quantize(xp, gs, 32), axis=1))
+    packed, scales = oracle.quantize(x, gs, 32)
+    np.testing.assert_array_equal(oracle.dequantize(packed, scales, gs, 5, N, 32),
+                                  oracle.dequantize(packed, scales, gs, 5, P, 32)[:, :N])
+
+
+def test_block_32_scale_is_the_larger_half_scale():
+    """The E4M3 scale byte is non-decreasing in the block amax (E4M3 codes of non-negative
+    values order like the values), so a 32-block's byte is the larger of its two
+    16-halves' bytes, for any input."""
+    rng = np.random.default_rng(3232)
+    x = synthetic.to_bf16_bits(rng.standard_t(3, (64, 512)).astype(np.float32)
+                               * np.exp2(rng.integers(-6, 6, (64, 1))).astype(np.float32))
+    gs = oracle.global_scale(oracle.amax(x))
+    _, s16 = oracle.quantize(x, gs, 16)
+    _, s32 = oracle.quantize(x, gs, 32)
+    np.testing.assert_array_equal(s32, np.maximum(s16[:, 0::2], s16[:, 1::2]))
