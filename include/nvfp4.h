@@ -264,6 +264,28 @@ nvfp4_status nvfp4_fake_quant(const void* x, void* y, int64_t M, int64_t N, cons
 nvfp4_status nvfp4_fake_quant_siblings(int k, const void* const* xs, void* const* ys, const int64_t* Ms,
                                        const int64_t* Ns, float* d_shared_amax, nvfp4_stream_t stream);
 
+/* ---- blocks of 16 or 32 elements ---------------------------------------------------- */
+
+/* The three block calls with the block length as an argument, as [FP4OPT]
+ * quantize_weight_to_float4 takes it (block_size): block is 16 (NVFP4; the same as the
+ * calls above) or 32, anything else is NVFP4_ERR_ARG.  Every formula, the E4M3 scale byte
+ * and the 1e-12 clamps are unchanged; only the block length L = block is:
+ *   block amax over L consecutive elements of a row, P = L * ceil(N / L) padded columns,
+ *   packed uint8 [M, P/2] (byte j of a row: element 2j low nibble, 2j+1 high nibble),
+ *   scales uint8 [M, P/L] in plain row order.
+ * Alignment: bf16 tensors 32 bytes, packed L/2 bytes (16 for block 32), scalars 4.
+ * The tensor-core scale layout (nvfp4_quantize_mma) and the fused / observer / sibling
+ * calls exist for block 16 only; for block 32 compose nvfp4_amax (or
+ * nvfp4_observe_amax) with the calls below.  Enqueue one kernel each. */
+nvfp4_status nvfp4_quantize_bs(const void* x, int64_t M, int64_t N, int block, const float* d_amax,
+                               uint8_t* packed, uint8_t* scales, float* d_global_scale, nvfp4_stream_t stream);
+
+nvfp4_status nvfp4_dequantize_bs(const uint8_t* packed, const uint8_t* scales, const float* d_global_scale,
+                                 int64_t M, int64_t N, int block, void* y, nvfp4_stream_t stream);
+
+nvfp4_status nvfp4_fake_quant_bs(const void* x, void* y, int64_t M, int64_t N, int block, const float* d_amax,
+                                 nvfp4_stream_t stream);
+
 /* Human-readable name of a status code (a static string). */
 const char* nvfp4_status_string(nvfp4_status status);
 

@@ -100,6 +100,14 @@ __device__ __forceinline__ void st_b64(void* p, uint32_t a, uint32_t b) {
     asm volatile("st.global.v2.b32 [%0], {%1,%2};" ::"l"(p), "r"(a), "r"(b) : "memory");
 }
 
+__device__ __forceinline__ void st_b128(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ void ld_b128_ro(const void* p, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
+    asm volatile("ld.global.nc.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "l"(p));
+}
+
 __device__ __forceinline__ void st_u8(void* p, uint32_t v) {
     asm volatile("st.global.u8 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -118,11 +126,38 @@ __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
     return d;
 }
 
-// Exact block amax: the largest |x| of the 16 bf16 values, widened to fp32.
-__device__ __forceinline__ float block_amax(const uint32_t (&w)[8]) {
-    uint32_t m = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(w[0], w[1]), absmax_bf16x2(w[2], w[3])),
-                               absmax_bf16x2(absmax_bf16x2(w[4], w[5]), absmax_bf16x2(w[6], w[7])));
-    return fmaxf(fabsf(bf16_lo(m)), fabsf(bf16_hi(m)));
+// Exact block amax: the largest |x| of the block's bf16 values (kW words of two),
+// widened to fp32.
+template <int kW>
+__device__ __forceinline__ float block_amax(const uint32_t (&w)[kW]) {
+    uint32_t m[kW];
+#pragma unroll
+    for (int i = 0; i < kW; ++i) m[i] = w[i];
+#pragma unroll
+    for (int step = 1; step < kW; step *= 2)
+#pragma unroll
+        for (int i = 0; i + step < kW; i += 2 * step) m[i] = absmax_bf16x2(m[i], m[i + step]);
+    return fmaxf(fabsf(bf16_lo(m[0])), fabsf(bf16_hi(m[0])));
+}
+
+// 32-byte-granular block loads and stores for blocks of 16 (kW = 8) or 32 (kW = 16)
+// elements.
+template <int kW>
+__device__ __forceinline__ void ld_block(const uint8_t* p, uint32_t (&w)[kW]) {
+#pragma unroll
+    for (int h = 0; h < kW / 8; ++h) ld_b256(p + 32 * h, *reinterpret_cast<uint32_t(*)[8]>(&w[8 * h]));
+}
+
+template <int kW>
+__device__ __forceinline__ void ld_block_ro(const uint8_t* p, uint32_t (&w)[kW]) {
+#pragma unroll
+    for (int h = 0; h < kW / 8; ++h) ld_b256_ro(p + 32 * h, *reinterpret_cast<uint32_t(*)[8]>(&w[8 * h]));
+}
+
+template <int kW>
+__device__ __forceinline__ void st_block(uint8_t* p, const uint32_t (&w)[kW]) {
+#pragma unroll
+    for (int h = 0; h < kW / 8; ++h) st_b256(p + 32 * h, *reinterpret_cast<const uint32_t(*)[8]>(&w[8 * h]));
 }
 
 // ---------------------------------------------------------------------------------------
@@ -212,10 +247,12 @@ __device__ __forceinline__ float quot_exact(float x, float sq) {
     return __fadd_rn(q, 0.0f);
 }
 
-// Quantize one block: returns its E4M3 scale byte; codes[i] receives the byte of E2M1
-// codes of elements 2i (bits 3:0) and 2i+1 (bits 7:4); sd the decode-side scale.
-__device__ __forceinline__ uint32_t encode_block(const uint32_t (&w)[8], float gs, const float4* tab,
-                                                 uint32_t (&codes)[8], float& sd) {
+// Quantize one block of 2 * kW elements: returns its E4M3 scale byte; codes[i] receives
+// the byte of E2M1 codes of elements 2i (bits 3:0) and 2i+1 (bits 7:4); sd the
+// decode-side scale.
+template <int kW>
+__device__ __forceinline__ uint32_t encode_block(const uint32_t (&w)[kW], float gs, const float4* tab,
+                                                 uint32_t (&codes)[kW], float& sd) {
     const float b = block_amax(w);
     const float v = __fmul_rn(__fdiv_rn(b, 6.0f), gs);
     const uint32_t s8 = e4m3_rne_satfinite(v);
@@ -223,11 +260,11 @@ __device__ __forceinline__ uint32_t encode_block(const uint32_t (&w)[8], float g
     sd = t.z;
     if (__fmul_rn(b, t.y) < t.w) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < kW; ++i)
             codes[i] = e2m1x2_rne(quot_fast(bf16_lo(w[i]), t.x, t.y), quot_fast(bf16_hi(w[i]), t.x, t.y));
     } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < kW; ++i)
             codes[i] = e2m1x2_rne(quot_exact(bf16_lo(w[i]), t.x), quot_exact(bf16_hi(w[i]), t.x));
     }
     return s8;

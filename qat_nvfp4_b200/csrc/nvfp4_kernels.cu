@@ -197,18 +197,57 @@ __device__ __forceinline__ void stream_blocks(int64_t nblk, Load load, Work work
     stream_sched<NVFP4_SCHED, U, kPipe, Slot>(nblk, load, work, NoPrologue{});
 }
 
-struct Block32 {
-    uint32_t w[8];
+// Per-thread staging of one block of 2 * kW elements (kW = 8: NVFP4's 16; kW = 16: 32).
+template <int kW>
+struct BlockW {
+    uint32_t w[kW];
 };
+using Block32 = BlockW<8>;
 
+template <int kW>
 struct FqSlot {
-    uint32_t w[8];
+    uint32_t w[kW];
     uint8_t* y;
 };
 
+template <int kW>
 struct PackedSlot {
-    uint32_t p0, p1, s;
+    uint32_t p[kW / 4];  // kW bytes of codes
+    uint32_t s;          // scale byte
 };
+
+// Blocks per thread and step for blocks of kW words: the same bytes in flight per thread
+// for both block sizes.
+template <int kW>
+__host__ __device__ constexpr int unroll_for(int u16) {
+    return kW == 8 ? u16 : (u16 / 2 > 0 ? u16 / 2 : 1);
+}
+
+// The packed codes of one block: kW bytes.
+template <int kW>
+__device__ __forceinline__ void st_codes(uint8_t* p, const uint32_t (&c)[kW]) {
+    if constexpr (kW == 8) {
+        st_b64(p, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
+    } else {
+        st_b128(p, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]), pack4(c[8], c[9], c[10], c[11]),
+                pack4(c[12], c[13], c[14], c[15]));
+    }
+}
+
+template <int kW>
+__device__ __forceinline__ void ld_codes_ro(const uint8_t* p, uint32_t (&w)[kW / 4]) {
+    if constexpr (kW == 8) ld_b64_ro(p, w[0], w[1]);
+    else ld_b128_ro(p, w[0], w[1], w[2], w[3]);
+}
+
+// bf16 outputs of one block from its code bytes and decode scale.
+template <int kW>
+__device__ __forceinline__ void decode_codes(const uint32_t (&p)[kW / 4], float sd, uint32_t (&o)[kW]) {
+#pragma unroll
+    for (int j = 0; j < kW / 4; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[4 * j + i] = decode_pair((p[j] >> (8 * i)) & 0xFFu, sd);
+}
 
 // ---------------------------------------------------------------------------------------
 // Global amax.  Each thread keeps a running bf16x2 |max|; the CTA reduces it and
@@ -349,7 +388,7 @@ __device__ __forceinline__ int64_t scale_offset(int64_t g, int64_t nb, int64_t n
 // ---------------------------------------------------------------------------------------
 // Quantize: bf16 blocks -> 8 bytes of codes + 1 scale byte.
 
-template <bool kMma>
+template <bool kMma, int kW>
 __global__ void __launch_bounds__(kThreads)
     quantize_kernel(const uint8_t* __restrict__ x, int64_t nblk, const float* __restrict__ d_amax,
                     uint8_t* __restrict__ packed, uint8_t* __restrict__ scales, float* __restrict__ d_gs, int64_t nb,
@@ -357,13 +396,13 @@ __global__ void __launch_bounds__(kThreads)
     const bool small = nblk <= 0xFFFFFFFFll;
     __shared__ float4 tab[128];
     float gs = 0.0f;
-    stream_blocks<kUnrollQ, NVFP4_PIPE_Q != 0, Block32>(
-        nblk, [&](int64_t bi, Block32& b) { ld_b256_ro(x + bi * kBlockBytesIn, b.w); },
-        [&](int64_t bi, Block32& b) {
-            uint32_t c[8];
+    stream_blocks<unroll_for<kW>(kUnrollQ), NVFP4_PIPE_Q != 0, BlockW<kW>>(
+        nblk, [&](int64_t bi, BlockW<kW>& b) { ld_block_ro(x + bi * (4 * kW), b.w); },
+        [&](int64_t bi, BlockW<kW>& b) {
+            uint32_t c[kW];
             float sd;
             const uint32_t s8 = encode_block(b.w, gs, tab, c, sd);
-            st_b64(packed + bi * kBlockBytesPacked, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
+            st_codes<kW>(packed + bi * kW, c);
             st_u8(scales + scale_offset<kMma>(bi, nb, ncb, small), s8);
         },
         [&] {
@@ -377,39 +416,39 @@ __global__ void __launch_bounds__(kThreads)
 // same buffer (each thread reads a block before it writes the same block), so the
 // loads use the coherent path.
 
-template <bool kMulti>
+template <bool kMulti, int kW>
 __device__ __forceinline__ void locate_fq(const FqList& L, int64_t bi, const uint8_t*& xp, uint8_t*& yp) {
     if (!kMulti) {
-        xp = L.x[0] + bi * kBlockBytesIn;
-        yp = L.y[0] + bi * kBlockBytesIn;
+        xp = L.x[0] + bi * (4 * kW);
+        yp = L.y[0] + bi * (4 * kW);
     } else {
         int j = 0;
         while (j + 1 < L.k && bi >= L.blk_end[j]) ++j;
         const int64_t local = bi - (j ? L.blk_end[j - 1] : 0);
-        xp = L.x[j] + local * kBlockBytesIn;
-        yp = L.y[j] + local * kBlockBytesIn;
+        xp = L.x[j] + local * (4 * kW);
+        yp = L.y[j] + local * (4 * kW);
     }
 }
 
-template <bool kMulti>
+template <bool kMulti, int kW>
 __global__ void __launch_bounds__(kThreads) fake_quant_kernel(FqList L, int64_t nblk, const float* d_amax) {
     __shared__ float4 tab[128];
     float gs = 0.0f;
-    stream_blocks<kUnrollFq, NVFP4_PIPE_FQ != 0, FqSlot>(
+    stream_blocks<unroll_for<kW>(kUnrollFq), NVFP4_PIPE_FQ != 0, FqSlot<kW>>(
         nblk,
-        [&](int64_t bi, FqSlot& sl) {
+        [&](int64_t bi, FqSlot<kW>& sl) {
             const uint8_t* xp;
-            locate_fq<kMulti>(L, bi, xp, sl.y);
-            ld_b256(xp, sl.w);
+            locate_fq<kMulti, kW>(L, bi, xp, sl.y);
+            ld_block(xp, sl.w);
         },
-        [&](int64_t, FqSlot& sl) {
-            uint32_t c[8];
+        [&](int64_t, FqSlot<kW>& sl) {
+            uint32_t c[kW];
             float sd;
             encode_block(sl.w, gs, tab, c, sd);
-            uint32_t o[8];
+            uint32_t o[kW];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
-            st_b256(sl.y, o);
+            for (int i = 0; i < kW; ++i) o[i] = decode_pair(c[i], sd);
+            st_block(sl.y, o);
         },
         [&] { gs = build_scale_table(tab, d_amax); });
 }
@@ -513,25 +552,21 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads)
 // ---------------------------------------------------------------------------------------
 // Dequantize: 8 bytes of codes + 1 scale byte -> bf16 block.
 
+template <int kW>
 __global__ void __launch_bounds__(kThreads)
     dequantize_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
                       const float* __restrict__ d_gs, uint8_t* __restrict__ y, int64_t nblk) {
     __shared__ float tab_sd[256];  // sd for every possible scale byte
-    stream_blocks<kUnrollDecode, NVFP4_PIPE_DEC != 0, PackedSlot>(
+    stream_blocks<unroll_for<kW>(kUnrollDecode), NVFP4_PIPE_DEC != 0, PackedSlot<kW>>(
         nblk,
-        [&](int64_t bi, PackedSlot& sl) {
-            ld_b64_ro(packed + bi * kBlockBytesPacked, sl.p0, sl.p1);
+        [&](int64_t bi, PackedSlot<kW>& sl) {
+            ld_codes_ro<kW>(packed + bi * kW, sl.p);
             sl.s = ld_u8_ro(scales + bi);
         },
-        [&](int64_t bi, PackedSlot& sl) {
-            const float sd = tab_sd[sl.s & 0xFFu];
-            uint32_t o[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                o[i] = decode_pair((sl.p0 >> (8 * i)) & 0xFFu, sd);
-                o[4 + i] = decode_pair((sl.p1 >> (8 * i)) & 0xFFu, sd);
-            }
-            st_b256(y + bi * kBlockBytesIn, o);
+        [&](int64_t bi, PackedSlot<kW>& sl) {
+            uint32_t o[kW];
+            decode_codes<kW>(sl.p, tab_sd[sl.s & 0xFFu], o);
+            st_block(y + bi * (4 * kW), o);
         },
         [&] {
             const float gs = __ldg(d_gs);
@@ -562,22 +597,33 @@ struct Ragged {
     int64_t total;  // M * nb
 };
 
-// First element and real length of block g (32-bit division whenever the sizes allow).
+// First element and real length of block g of 2 * kW elements (32-bit division whenever
+// the sizes allow).
+template <int kW>
 __device__ __forceinline__ int64_t ragged_offset(const Ragged& R, int64_t g, int& n) {
+    constexpr int kE = 2 * kW;
     int64_t r;
     if (R.total <= 0xFFFFFFFFll) r = (int64_t)((uint32_t)g / (uint32_t)R.nb);
     else r = g / R.nb;
     const int64_t b = g - r * R.nb;
-    const int64_t c0 = b * kBlockElems;
-    n = (int)(R.N - c0 < kBlockElems ? R.N - c0 : kBlockElems);
+    const int64_t c0 = b * kE;
+    n = (int)(R.N - c0 < kE ? R.N - c0 : kE);
     return r * R.N + c0;
 }
 
-// Blocks per thread in one tile, and bytes of staging per CTA: kRaggedTile blocks of at
-// most 32 bytes, plus the 16-byte rounding at the start of the range.
-constexpr int kRaggedU = 4;
-constexpr int kRaggedTile = kThreads * kRaggedU;
-constexpr int kStageBytes = kRaggedTile * kBlockBytesIn + 64;
+// Blocks per thread in one tile and blocks per tile (4 blocks of 16 or 2 of 32 per
+// thread), and bytes of staging per CTA: one tile of full blocks (32 KB for both block
+// sizes) plus the 16-byte rounding at the start of the range.
+template <int kW>
+__host__ __device__ constexpr int ragged_u() {
+    return kW == 8 ? 4 : 2;
+}
+template <int kW>
+__host__ __device__ constexpr int ragged_tile() {
+    return kThreads * ragged_u<kW>();
+}
+constexpr int kStageBytes = ragged_tile<8>() * 32 + 64;
+static_assert(ragged_tile<16>() * 64 + 64 == kStageBytes, "both block sizes stage the same bytes");
 
 // The stage holds 16-byte chunk k of the tile's byte range at chunk position
 // k ^ ((k >> 3) & 1).  Lanes whose blocks sit two chunks apart then read eight different
@@ -590,11 +636,12 @@ __device__ __forceinline__ int stage_addr(int64_t byte) {
 }
 
 // Byte range [B0, B1) of the tile that starts at block g0 (both even).
+template <int kW>
 __device__ __forceinline__ void tile_range(const Ragged& R, int64_t g0, int64_t& B0, int64_t& B1) {
-    const int64_t g1 = (g0 + kRaggedTile < R.total ? g0 + kRaggedTile : R.total) - 1;
+    const int64_t g1 = (g0 + ragged_tile<kW>() < R.total ? g0 + ragged_tile<kW>() : R.total) - 1;
     int n0, n1;
-    B0 = 2 * ragged_offset(R, g0, n0);
-    B1 = 2 * (ragged_offset(R, g1, n1) + n1);
+    B0 = 2 * ragged_offset<kW>(R, g0, n0);
+    B1 = 2 * (ragged_offset<kW>(R, g1, n1) + n1);
 }
 
 // Issue the copies that fill a stage with the 16-byte chunks covering [B0, B1) (chunk k
@@ -639,15 +686,17 @@ __device__ __forceinline__ void stage_out(uint8_t* dst, int64_t B0, int64_t B1, 
     }
 }
 
-// This thread's block (n real elements starting at stage byte X, X even) as eight bf16x2
-// words, zeros past n: the three 16-byte chunks that cover it are read whole, then
+// This thread's block (n real elements starting at stage byte X, X even) as kW bf16x2
+// words, zeros past n: the kW / 4 + 1 16-byte chunks that cover it are read whole, then
 // shifted down by X & 15 bytes with selects and a funnel shift.
-__device__ __forceinline__ void block_from_stage(const uint8_t* stage, int64_t X, int n, uint32_t (&w)[8]) {
+template <int kW>
+__device__ __forceinline__ void block_from_stage(const uint8_t* stage, int64_t X, int n, uint32_t (&w)[kW]) {
+    constexpr int kChunks = kW / 4 + 1;
     const int k0 = (int)(X >> 4);
     const int sh = (int)(X & 15);
-    uint32_t c[12];
+    uint32_t c[4 * kChunks];
 #pragma unroll
-    for (int j = 0; j < 3; ++j) {
+    for (int j = 0; j < kChunks; ++j) {
         const uint4 v = *reinterpret_cast<const uint4*>(stage + 16 * chunk_pos(k0 + j));
         c[4 * j] = v.x;
         c[4 * j + 1] = v.y;
@@ -655,13 +704,13 @@ __device__ __forceinline__ void block_from_stage(const uint8_t* stage, int64_t X
         c[4 * j + 3] = v.w;
     }
     const int s4 = sh >> 2;
-    uint32_t t[10], u[9];
+    uint32_t t[kW + 2], u[kW + 1];
 #pragma unroll
-    for (int i = 0; i < 10; ++i) t[i] = (s4 & 2) ? c[i + 2] : c[i];
+    for (int i = 0; i < kW + 2; ++i) t[i] = (s4 & 2) ? c[i + 2] : c[i];
 #pragma unroll
-    for (int i = 0; i < 9; ++i) u[i] = (s4 & 1) ? t[i + 1] : t[i];
+    for (int i = 0; i < kW + 1; ++i) u[i] = (s4 & 1) ? t[i + 1] : t[i];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kW; ++i) {
         uint32_t v = (sh & 2) ? __funnelshift_r(u[i], u[i + 1], 16) : u[i];
         if (2 * i + 1 >= n) v &= 0x0000FFFFu;  // the row's padding reads as +0.0
         if (2 * i >= n) v = 0u;
@@ -671,18 +720,19 @@ __device__ __forceinline__ void block_from_stage(const uint8_t* stage, int64_t X
 
 // Write this thread's n output elements back to stage byte X: 32-bit stores on 4-byte
 // boundaries, 16-bit stores for a leading or trailing half word.
-__device__ __forceinline__ void block_to_stage(uint8_t* stage, int64_t X, int n, const uint32_t (&o)[8]) {
+template <int kW>
+__device__ __forceinline__ void block_to_stage(uint8_t* stage, int64_t X, int n, const uint32_t (&o)[kW]) {
     if ((X & 2) == 0) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < kW; ++i) {
             if (2 * i + 1 < n) *reinterpret_cast<uint32_t*>(stage + stage_addr(X + 4 * i)) = o[i];
             else if (2 * i < n) *reinterpret_cast<uint16_t*>(stage + stage_addr(X + 4 * i)) = (uint16_t)(o[i] & 0xFFFFu);
         }
     } else {
         *reinterpret_cast<uint16_t*>(stage + stage_addr(X)) = (uint16_t)(o[0] & 0xFFFFu);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t next = i < 7 ? o[i + 1] : 0u;
+        for (int i = 0; i < kW; ++i) {
+            const uint32_t next = i < kW - 1 ? o[i + 1] : 0u;
             const uint32_t v = (o[i] >> 16) | (next << 16);  // elements 2i+1, 2i+2
             if (2 * i + 2 < n) *reinterpret_cast<uint32_t*>(stage + stage_addr(X + 4 * i + 2)) = v;
             else if (2 * i + 1 < n) *reinterpret_cast<uint16_t*>(stage + stage_addr(X + 4 * i + 2)) = (uint16_t)(v & 0xFFFFu);
@@ -695,12 +745,13 @@ __device__ __forceinline__ void block_to_stage(uint8_t* stage, int64_t X, int n,
 // stage reused.  (A two-stage version that prefetched the next tile measured no faster:
 // the ragged kernels are bound by their per-element index and shift work, not by load
 // latency.)
-template <class Work>
+template <int kW, class Work>
 __device__ __forceinline__ void ragged_tiles(const uint8_t* src, const Ragged& R, uint8_t* stage, Work work) {
+    constexpr int kTile = ragged_tile<kW>();
     const int64_t total_bytes = 2 * (R.total / R.nb) * R.N;
-    for (int64_t g0 = (int64_t)blockIdx.x * kRaggedTile; g0 < R.total; g0 += (int64_t)gridDim.x * kRaggedTile) {
+    for (int64_t g0 = (int64_t)blockIdx.x * kTile; g0 < R.total; g0 += (int64_t)gridDim.x * kTile) {
         int64_t B0, B1;
-        tile_range(R, g0, B0, B1);
+        tile_range<kW>(R, g0, B0, B1);
         stage_issue(src, B0, B1, total_bytes, stage);
         asm volatile("cp.async.wait_all;" ::: "memory");
         __syncthreads();
@@ -709,7 +760,7 @@ __device__ __forceinline__ void ragged_tiles(const uint8_t* src, const Ragged& R
     }
 }
 
-template <bool kMma>
+template <bool kMma, int kW>
 __global__ void __launch_bounds__(kThreads)
     quantize_ragged_kernel(const uint8_t* __restrict__ x, Ragged R, const float* __restrict__ d_amax,
                            uint8_t* __restrict__ packed, uint8_t* __restrict__ scales, float* __restrict__ d_gs,
@@ -719,26 +770,27 @@ __global__ void __launch_bounds__(kThreads)
     extern __shared__ __align__(16) uint8_t stage[];
     const float gs = build_scale_table(tab, d_amax);
     if (d_gs != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *d_gs = gs;
-    ragged_tiles(x, R, stage, [&](int64_t g0, int64_t B0, int64_t, uint8_t* stage) {
+    ragged_tiles<kW>(x, R, stage, [&](int64_t g0, int64_t B0, int64_t, uint8_t* stage) {
         const int64_t A0 = B0 & ~(int64_t)15;
 #pragma unroll
-        for (int u = 0; u < kRaggedU; ++u) {
+        for (int u = 0; u < ragged_u<kW>(); ++u) {
             const int64_t g = g0 + u * kThreads + threadIdx.x;
             if (g < R.total) {
                 int n;
-                const int64_t e = ragged_offset(R, g, n);
-                uint32_t w[8];
+                const int64_t e = ragged_offset<kW>(R, g, n);
+                uint32_t w[kW];
                 block_from_stage(stage, 2 * e - A0, n, w);
-                uint32_t c[8];
+                uint32_t c[kW];
                 float sd;
                 const uint32_t s8 = encode_block(w, gs, tab, c, sd);
-                st_b64(packed + g * kBlockBytesPacked, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
+                st_codes<kW>(packed + g * kW, c);
                 st_u8(scales + scale_offset<kMma>(g, R.nb, ncb, small), s8);
             }
         }
     });
 }
 
+template <int kW>
 __global__ void __launch_bounds__(kThreads)
     fake_quant_ragged_kernel(const uint8_t* x, uint8_t* y, Ragged R, const float* d_amax) {
     __shared__ float4 tab[128];
@@ -746,22 +798,22 @@ __global__ void __launch_bounds__(kThreads)
     const float gs = build_scale_table(tab, d_amax);
     // y may be x: the copies read through L2, and a tile's bytes are read before any CTA
     // writes them (each CTA writes only its own tile's bytes, after reading them).
-    ragged_tiles(x, R, stage, [&](int64_t g0, int64_t B0, int64_t B1, uint8_t* stage) {
+    ragged_tiles<kW>(x, R, stage, [&](int64_t g0, int64_t B0, int64_t B1, uint8_t* stage) {
         const int64_t A0 = B0 & ~(int64_t)15;
 #pragma unroll
-        for (int u = 0; u < kRaggedU; ++u) {
+        for (int u = 0; u < ragged_u<kW>(); ++u) {
             const int64_t g = g0 + u * kThreads + threadIdx.x;
             if (g < R.total) {
                 int n;
-                const int64_t e = ragged_offset(R, g, n);
-                uint32_t w[8];
+                const int64_t e = ragged_offset<kW>(R, g, n);
+                uint32_t w[kW];
                 block_from_stage(stage, 2 * e - A0, n, w);
-                uint32_t c[8];
+                uint32_t c[kW];
                 float sd;
                 encode_block(w, gs, tab, c, sd);
-                uint32_t o[8];
+                uint32_t o[kW];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
+                for (int i = 0; i < kW; ++i) o[i] = decode_pair(c[i], sd);
                 block_to_stage(stage, 2 * e - A0, n, o);  // each thread rewrites only its own elements
             }
         }
@@ -770,6 +822,7 @@ __global__ void __launch_bounds__(kThreads)
     });
 }
 
+template <int kW>
 __global__ void __launch_bounds__(kThreads)
     dequantize_ragged_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
                              const float* __restrict__ d_gs, uint8_t* __restrict__ y, Ragged R) {
@@ -778,32 +831,29 @@ __global__ void __launch_bounds__(kThreads)
     const float gs = __ldg(d_gs);
     for (int i = threadIdx.x; i < 256; i += blockDim.x) tab_sd[i] = __fdiv_rn(e4m3_to_f32(i), gs);
     __syncthreads();
-    for (int64_t g0 = (int64_t)blockIdx.x * kRaggedTile; g0 < R.total; g0 += (int64_t)gridDim.x * kRaggedTile) {
+    constexpr int kU = ragged_u<kW>();
+    constexpr int kTile = ragged_tile<kW>();
+    for (int64_t g0 = (int64_t)blockIdx.x * kTile; g0 < R.total; g0 += (int64_t)gridDim.x * kTile) {
         int64_t B0, B1;
-        tile_range(R, g0, B0, B1);
+        tile_range<kW>(R, g0, B0, B1);
         const int64_t A0 = B0 & ~(int64_t)15;
-        uint32_t p[kRaggedU][2], sb[kRaggedU];
+        uint32_t p[kU][kW / 4], sb[kU];
 #pragma unroll
-        for (int u = 0; u < kRaggedU; ++u) {
+        for (int u = 0; u < kU; ++u) {
             const int64_t g = g0 + u * kThreads + threadIdx.x;
             if (g < R.total) {
-                ld_b64_ro(packed + g * kBlockBytesPacked, p[u][0], p[u][1]);
+                ld_codes_ro<kW>(packed + g * kW, p[u]);
                 sb[u] = ld_u8_ro(scales + g);
             }
         }
 #pragma unroll
-        for (int u = 0; u < kRaggedU; ++u) {
+        for (int u = 0; u < kU; ++u) {
             const int64_t g = g0 + u * kThreads + threadIdx.x;
             if (g < R.total) {
-                const float sd = tab_sd[sb[u] & 0xFFu];
-                uint32_t o[8];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    o[i] = decode_pair((p[u][0] >> (8 * i)) & 0xFFu, sd);
-                    o[4 + i] = decode_pair((p[u][1] >> (8 * i)) & 0xFFu, sd);
-                }
+                uint32_t o[kW];
+                decode_codes<kW>(p[u], tab_sd[sb[u] & 0xFFu], o);
                 int n;
-                const int64_t e = ragged_offset(R, g, n);
+                const int64_t e = ragged_offset<kW>(R, g, n);
                 block_to_stage(stage, 2 * e - A0, n, o);
             }
         }
@@ -892,19 +942,20 @@ constexpr int64_t kMaxElems = (int64_t)1 << 60;
 
 cudaStream_t cs(nvfp4_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
-// Any M, N >= 0 whose padded size fits; rows with N % 16 != 0 take the ragged kernels.
-nvfp4_status check_matrix(int64_t M, int64_t N, int64_t* numel) {
+// Any M, N >= 0 whose padded size fits; rows with N % block != 0 take the ragged kernels.
+nvfp4_status check_matrix(int64_t M, int64_t N, int64_t* numel, int64_t block = kBlockElems) {
     if (M < 0 || N < 0) return NVFP4_ERR_SHAPE;
-    const int64_t P = (N + kBlockElems - 1) / kBlockElems * kBlockElems;
+    if (N > kMaxElems) return NVFP4_ERR_SHAPE;
+    const int64_t P = (N + block - 1) / block * block;
     if (P != 0 && M > kMaxElems / P) return NVFP4_ERR_SHAPE;
     *numel = M * N;
     return NVFP4_OK;
 }
 
-Ragged ragged_of(int64_t M, int64_t N) {
+Ragged ragged_of(int64_t M, int64_t N, int64_t block = kBlockElems) {
     Ragged R;
     R.N = N;
-    R.nb = (N + kBlockElems - 1) / kBlockElems;
+    R.nb = (N + block - 1) / block;
     R.total = M * R.nb;
     return R;
 }
@@ -920,19 +971,23 @@ nvfp4_status ragged_smem_optin(K* kernel, int bytes) {
 }
 
 // Ragged launches shared by the entry points (arguments already validated).
+template <int kW>
 nvfp4_status launch_fq_ragged(const void* x, void* y, int64_t M, int64_t N, const float* d_amax, nvfp4_stream_t stream) {
-    const Ragged R = ragged_of(M, N);
+    const Ragged R = ragged_of(M, N, 2 * kW);
     if (R.total == 0) return NVFP4_OK;
     int grid = 1;
-    nvfp4_status st = ragged_smem_optin(fake_quant_ragged_kernel, kStageBytes);
+    nvfp4_status st = ragged_smem_optin(fake_quant_ragged_kernel<kW>, kStageBytes);
     if (st != NVFP4_OK) return st;
-    st = grid_for(reinterpret_cast<const void*>(&fake_quant_ragged_kernel), R.total, kRaggedU, NVFP4_GRID_FQ, &grid,
-                  kStageBytes);
+    st = grid_for(reinterpret_cast<const void*>(&fake_quant_ragged_kernel<kW>), R.total, ragged_u<kW>(), NVFP4_GRID_FQ,
+                  &grid, kStageBytes);
     if (st != NVFP4_OK) return st;
-    fake_quant_ragged_kernel<<<grid, kThreads, kStageBytes, cs(stream)>>>(static_cast<const uint8_t*>(x), static_cast<uint8_t*>(y),
-                                                                R, d_amax);
+    fake_quant_ragged_kernel<kW><<<grid, kThreads, kStageBytes, cs(stream)>>>(static_cast<const uint8_t*>(x),
+                                                                            static_cast<uint8_t*>(y), R, d_amax);
     return after_launch();
 }
+
+// Words (bf16 pairs) per block for an accepted block size, 0 otherwise.
+int words_of_block(int block) { return block == 16 ? 8 : (block == 32 ? 16 : 0); }
 
 bool overlap(const void* a, const void* b, int64_t bytes) {
     const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
@@ -1210,7 +1265,7 @@ static nvfp4_status fake_quant_auto(const void* x, void* y, int64_t M, int64_t N
         if (st != NVFP4_OK) return st;
         st = launch_amax_ws(L, d_amax_out, d_ws, state, kind, keep, take, stream);
         if (st != NVFP4_OK) return st;
-        return launch_fq_ragged(x, y, M, N, state ? state : d_amax_out, stream);
+        return launch_fq_ragged<8>(x, y, M, N, state ? state : d_amax_out, stream);
     }
     const int64_t nblk = M * N / kBlockElems;
     int64_t l2 = 0;
@@ -1234,9 +1289,9 @@ static nvfp4_status fake_quant_auto(const void* x, void* y, int64_t M, int64_t N
     F.y[0] = static_cast<uint8_t*>(y);
     F.blk_end[0] = nblk;
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<false>), nblk, kUnrollFq, NVFP4_GRID_FQ, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<false, 8>), nblk, kUnrollFq, NVFP4_GRID_FQ, &grid);
     if (st != NVFP4_OK) return st;
-    fake_quant_kernel<false><<<grid, kThreads, 0, cs(stream)>>>(F, nblk, state ? state : d_amax_out);
+    fake_quant_kernel<false, 8><<<grid, kThreads, 0, cs(stream)>>>(F, nblk, state ? state : d_amax_out);
     return after_launch();
 }
 
@@ -1290,17 +1345,18 @@ NVFP4_API nvfp4_status nvfp4_selftest_barrier_timeout(const void* x, void* y, in
                         0, 0.f, 0.f, 1u, (uint64_t)timeout_us * 1000ull, stream);
 }
 
-template <bool kMma>
+template <bool kMma, int kW>
 static nvfp4_status quantize_impl(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
                                   uint8_t* scales, float* d_global_scale, nvfp4_stream_t stream) {
+    constexpr int kE = 2 * kW;
     int64_t numel = 0;
-    nvfp4_status st = check_matrix(M, N, &numel);
+    nvfp4_status st = check_matrix(M, N, &numel, kE);
     if (st != NVFP4_OK) return st;
     if (d_amax == nullptr) return NVFP4_ERR_NULL;
     if (numel > 0 && (x == nullptr || packed == nullptr || scales == nullptr)) return NVFP4_ERR_NULL;
     if (!aligned(d_amax, 4) || (d_global_scale && !aligned(d_global_scale, 4))) return NVFP4_ERR_ALIGN;
-    if (numel > 0 && (!aligned(x, 32) || !aligned(packed, 8))) return NVFP4_ERR_ALIGN;
-    const Ragged R = ragged_of(M, N);
+    if (numel > 0 && (!aligned(x, 32) || !aligned(packed, kW))) return NVFP4_ERR_ALIGN;
+    const Ragged R = ragged_of(M, N, kE);
     const int64_t ncb = (R.nb + 3) / 4;
     if (kMma && numel > 0) {
         // The tile padding (rows past M, columns past nb) must read as zero scales.
@@ -1308,80 +1364,77 @@ static nvfp4_status quantize_impl(const void* x, int64_t M, int64_t N, const flo
         if (rows_p != M || ncb * 4 != R.nb)
             if (cudaMemsetAsync(scales, 0, (size_t)(rows_p * ncb * 4), cs(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
     }
-    if (N % kBlockElems != 0) {
+    if (N % kE != 0) {
         int grid = 1;
-        st = ragged_smem_optin(quantize_ragged_kernel<kMma>, kStageBytes);
+        st = ragged_smem_optin(quantize_ragged_kernel<kMma, kW>, kStageBytes);
         if (st != NVFP4_OK) return st;
-        st = grid_for(reinterpret_cast<const void*>(&quantize_ragged_kernel<kMma>), R.total, kRaggedU, NVFP4_GRID_Q,
-                      &grid, kStageBytes);
+        st = grid_for(reinterpret_cast<const void*>(&quantize_ragged_kernel<kMma, kW>), R.total, ragged_u<kW>(),
+                      NVFP4_GRID_Q, &grid, kStageBytes);
         if (st != NVFP4_OK) return st;
-        quantize_ragged_kernel<kMma><<<grid, kThreads, kStageBytes, cs(stream)>>>(
+        quantize_ragged_kernel<kMma, kW><<<grid, kThreads, kStageBytes, cs(stream)>>>(
             static_cast<const uint8_t*>(x), R, d_amax, packed, scales, d_global_scale, ncb);
         return after_launch();
     }
-    const int64_t nblk = numel / kBlockElems;
+    const int64_t nblk = numel / kE;
     if (nblk == 0 && d_global_scale == nullptr) return NVFP4_OK;
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&quantize_kernel<kMma>), nblk, kUnrollQ, NVFP4_GRID_Q, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&quantize_kernel<kMma, kW>), nblk, unroll_for<kW>(kUnrollQ),
+                  NVFP4_GRID_Q, &grid);
     if (st != NVFP4_OK) return st;
-    quantize_kernel<kMma><<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), nblk, d_amax, packed,
-                                                             scales, d_global_scale, R.nb > 0 ? R.nb : 1, ncb);
+    quantize_kernel<kMma, kW><<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), nblk, d_amax, packed,
+                                                                 scales, d_global_scale, R.nb > 0 ? R.nb : 1, ncb);
     return after_launch();
 }
 
-NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
-                                      uint8_t* scales, float* d_global_scale, nvfp4_stream_t stream) {
-    return quantize_impl<false>(x, M, N, d_amax, packed, scales, d_global_scale, stream);
-}
-
-NVFP4_API nvfp4_status nvfp4_quantize_mma(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
-                                          uint8_t* scales_mma, float* d_global_scale, nvfp4_stream_t stream) {
-    if (M > 0 && N > 0 && scales_mma != nullptr && !aligned(scales_mma, 16)) return NVFP4_ERR_ALIGN;
-    return quantize_impl<true>(x, M, N, d_amax, packed, scales_mma, d_global_scale, stream);
-}
-
-NVFP4_API nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* scales, const float* d_global_scale,
-                                        int64_t M, int64_t N, void* y, nvfp4_stream_t stream) {
+template <int kW>
+static nvfp4_status dequantize_impl(const uint8_t* packed, const uint8_t* scales, const float* d_global_scale,
+                                    int64_t M, int64_t N, void* y, nvfp4_stream_t stream) {
+    constexpr int kE = 2 * kW;
     int64_t numel = 0;
-    nvfp4_status st = check_matrix(M, N, &numel);
+    nvfp4_status st = check_matrix(M, N, &numel, kE);
     if (st != NVFP4_OK) return st;
     if (d_global_scale == nullptr) return NVFP4_ERR_NULL;
     if (numel > 0 && (packed == nullptr || scales == nullptr || y == nullptr)) return NVFP4_ERR_NULL;
     if (!aligned(d_global_scale, 4)) return NVFP4_ERR_ALIGN;
-    if (numel > 0 && (!aligned(packed, 8) || !aligned(y, 32))) return NVFP4_ERR_ALIGN;
-    if (N % kBlockElems != 0) {
-        const Ragged R = ragged_of(M, N);
+    if (numel > 0 && (!aligned(packed, kW) || !aligned(y, 32))) return NVFP4_ERR_ALIGN;
+    if (N % kE != 0) {
+        const Ragged R = ragged_of(M, N, kE);
         if (R.total == 0) return NVFP4_OK;
         int grid = 1;
-        st = ragged_smem_optin(dequantize_ragged_kernel, kStageBytes);
+        st = ragged_smem_optin(dequantize_ragged_kernel<kW>, kStageBytes);
         if (st != NVFP4_OK) return st;
-        st = grid_for(reinterpret_cast<const void*>(&dequantize_ragged_kernel), R.total, kRaggedU, NVFP4_GRID_DEC, &grid, kStageBytes);
+        st = grid_for(reinterpret_cast<const void*>(&dequantize_ragged_kernel<kW>), R.total, ragged_u<kW>(),
+                      NVFP4_GRID_DEC, &grid, kStageBytes);
         if (st != NVFP4_OK) return st;
-        dequantize_ragged_kernel<<<grid, kThreads, kStageBytes, cs(stream)>>>(packed, scales, d_global_scale,
-                                                                    static_cast<uint8_t*>(y), R);
+        dequantize_ragged_kernel<kW><<<grid, kThreads, kStageBytes, cs(stream)>>>(packed, scales, d_global_scale,
+                                                                                static_cast<uint8_t*>(y), R);
         return after_launch();
     }
-    const int64_t nblk = numel / kBlockElems;
+    const int64_t nblk = numel / kE;
     if (nblk == 0) return NVFP4_OK;
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&dequantize_kernel), nblk, kUnrollDecode, NVFP4_GRID_DEC, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&dequantize_kernel<kW>), nblk, unroll_for<kW>(kUnrollDecode),
+                  NVFP4_GRID_DEC, &grid);
     if (st != NVFP4_OK) return st;
-    dequantize_kernel<<<grid, kThreads, 0, cs(stream)>>>(packed, scales, d_global_scale, static_cast<uint8_t*>(y), nblk);
+    dequantize_kernel<kW><<<grid, kThreads, 0, cs(stream)>>>(packed, scales, d_global_scale, static_cast<uint8_t*>(y),
+                                                             nblk);
     return after_launch();
 }
 
-NVFP4_API nvfp4_status nvfp4_fake_quant(const void* x, void* y, int64_t M, int64_t N, const float* d_amax,
-                                        nvfp4_stream_t stream) {
+template <int kW>
+static nvfp4_status fake_quant_impl(const void* x, void* y, int64_t M, int64_t N, const float* d_amax,
+                                    nvfp4_stream_t stream) {
+    constexpr int kE = 2 * kW;
     int64_t numel = 0;
-    nvfp4_status st = check_matrix(M, N, &numel);
+    nvfp4_status st = check_matrix(M, N, &numel, kE);
     if (st != NVFP4_OK) return st;
     if (d_amax == nullptr) return NVFP4_ERR_NULL;
     if (numel > 0 && (x == nullptr || y == nullptr)) return NVFP4_ERR_NULL;
     if (!aligned(d_amax, 4)) return NVFP4_ERR_ALIGN;
     if (numel > 0 && (!aligned(x, 32) || !aligned(y, 32))) return NVFP4_ERR_ALIGN;
     if (x != y && numel > 0 && overlap(x, y, numel * 2)) return NVFP4_ERR_ARG;
-    if (N % kBlockElems != 0) return launch_fq_ragged(x, y, M, N, d_amax, stream);
-    const int64_t nblk = numel / kBlockElems;
+    if (N % kE != 0) return launch_fq_ragged<kW>(x, y, M, N, d_amax, stream);
+    const int64_t nblk = numel / kE;
     if (nblk == 0) return NVFP4_OK;
     FqList L;
     std::memset(&L, 0, sizeof(L));
@@ -1390,10 +1443,59 @@ NVFP4_API nvfp4_status nvfp4_fake_quant(const void* x, void* y, int64_t M, int64
     L.y[0] = static_cast<uint8_t*>(y);
     L.blk_end[0] = nblk;
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<false>), nblk, kUnrollFq, NVFP4_GRID_FQ, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<false, kW>), nblk, unroll_for<kW>(kUnrollFq),
+                  NVFP4_GRID_FQ, &grid);
     if (st != NVFP4_OK) return st;
-    fake_quant_kernel<false><<<grid, kThreads, 0, cs(stream)>>>(L, nblk, d_amax);
+    fake_quant_kernel<false, kW><<<grid, kThreads, 0, cs(stream)>>>(L, nblk, d_amax);
     return after_launch();
+}
+
+NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
+                                      uint8_t* scales, float* d_global_scale, nvfp4_stream_t stream) {
+    return quantize_impl<false, 8>(x, M, N, d_amax, packed, scales, d_global_scale, stream);
+}
+
+NVFP4_API nvfp4_status nvfp4_quantize_mma(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
+                                          uint8_t* scales_mma, float* d_global_scale, nvfp4_stream_t stream) {
+    if (M > 0 && N > 0 && scales_mma != nullptr && !aligned(scales_mma, 16)) return NVFP4_ERR_ALIGN;
+    return quantize_impl<true, 8>(x, M, N, d_amax, packed, scales_mma, d_global_scale, stream);
+}
+
+NVFP4_API nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* scales, const float* d_global_scale,
+                                        int64_t M, int64_t N, void* y, nvfp4_stream_t stream) {
+    return dequantize_impl<8>(packed, scales, d_global_scale, M, N, y, stream);
+}
+
+NVFP4_API nvfp4_status nvfp4_fake_quant(const void* x, void* y, int64_t M, int64_t N, const float* d_amax,
+                                        nvfp4_stream_t stream) {
+    return fake_quant_impl<8>(x, y, M, N, d_amax, stream);
+}
+
+NVFP4_API nvfp4_status nvfp4_quantize_bs(const void* x, int64_t M, int64_t N, int block, const float* d_amax,
+                                         uint8_t* packed, uint8_t* scales, float* d_global_scale, nvfp4_stream_t stream) {
+    switch (words_of_block(block)) {
+        case 8: return quantize_impl<false, 8>(x, M, N, d_amax, packed, scales, d_global_scale, stream);
+        case 16: return quantize_impl<false, 16>(x, M, N, d_amax, packed, scales, d_global_scale, stream);
+        default: return NVFP4_ERR_ARG;
+    }
+}
+
+NVFP4_API nvfp4_status nvfp4_dequantize_bs(const uint8_t* packed, const uint8_t* scales, const float* d_global_scale,
+                                           int64_t M, int64_t N, int block, void* y, nvfp4_stream_t stream) {
+    switch (words_of_block(block)) {
+        case 8: return dequantize_impl<8>(packed, scales, d_global_scale, M, N, y, stream);
+        case 16: return dequantize_impl<16>(packed, scales, d_global_scale, M, N, y, stream);
+        default: return NVFP4_ERR_ARG;
+    }
+}
+
+NVFP4_API nvfp4_status nvfp4_fake_quant_bs(const void* x, void* y, int64_t M, int64_t N, int block,
+                                           const float* d_amax, nvfp4_stream_t stream) {
+    switch (words_of_block(block)) {
+        case 8: return fake_quant_impl<8>(x, y, M, N, d_amax, stream);
+        case 16: return fake_quant_impl<16>(x, y, M, N, d_amax, stream);
+        default: return NVFP4_ERR_ARG;
+    }
 }
 
 NVFP4_API nvfp4_status nvfp4_fake_quant_siblings(int k, const void* const* xs, void* const* ys, const int64_t* Ms,
@@ -1428,8 +1530,8 @@ NVFP4_API nvfp4_status nvfp4_fake_quant_siblings(int k, const void* const* xs, v
     for (int j = 0; j < k; ++j) all_aligned = all_aligned && (Ns[j] % kBlockElems == 0);
     if (!all_aligned) {  // one launch per member, each with the shared amax
         for (int j = 0; j < k; ++j) {
-            st = Ns[j] % kBlockElems ? launch_fq_ragged(xs[j], ys[j], Ms[j], Ns[j], d_shared_amax, stream)
-                                     : nvfp4_fake_quant(xs[j], ys[j], Ms[j], Ns[j], d_shared_amax, stream);
+            st = Ns[j] % kBlockElems ? launch_fq_ragged<8>(xs[j], ys[j], Ms[j], Ns[j], d_shared_amax, stream)
+                                     : fake_quant_impl<8>(xs[j], ys[j], Ms[j], Ns[j], d_shared_amax, stream);
             if (st != NVFP4_OK) return st;
         }
         return NVFP4_OK;
@@ -1437,8 +1539,8 @@ NVFP4_API nvfp4_status nvfp4_fake_quant_siblings(int k, const void* const* xs, v
     const int64_t nblk = acc;
     if (nblk == 0) return NVFP4_OK;
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<true>), nblk, kUnrollFq, NVFP4_GRID_FQ, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<true, 8>), nblk, kUnrollFq, NVFP4_GRID_FQ, &grid);
     if (st != NVFP4_OK) return st;
-    fake_quant_kernel<true><<<grid, kThreads, 0, cs(stream)>>>(F, nblk, d_shared_amax);
+    fake_quant_kernel<true, 8><<<grid, kThreads, 0, cs(stream)>>>(F, nblk, d_shared_amax);
     return after_launch();
 }

@@ -62,6 +62,9 @@ _c_quantize = _sig("nvfp4_quantize", [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp])
 _c_quantize_mma = _sig("nvfp4_quantize_mma", [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp])
 _c_dequantize = _sig("nvfp4_dequantize", [_vp, _vp, _vp, _i64, _i64, _vp, _vp])
 _c_fake_quant = _sig("nvfp4_fake_quant", [_vp, _vp, _i64, _i64, _vp, _vp])
+_c_quantize_bs = _sig("nvfp4_quantize_bs", [_vp, _i64, _i64, ctypes.c_int, _vp, _vp, _vp, _vp, _vp])
+_c_dequantize_bs = _sig("nvfp4_dequantize_bs", [_vp, _vp, _vp, _i64, _i64, ctypes.c_int, _vp, _vp])
+_c_fake_quant_bs = _sig("nvfp4_fake_quant_bs", [_vp, _vp, _i64, _i64, ctypes.c_int, _vp, _vp])
 _c_fake_quant_siblings = _sig("nvfp4_fake_quant_siblings",
                               [ctypes.c_int, ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_i64),
                                ctypes.POINTER(_i64), _vp, _vp])
@@ -119,9 +122,18 @@ def _matrix(x: torch.Tensor, name: str = "x"):
     return math.prod(x.shape[:-1]), N
 
 
-def padded_blocks(N: int) -> int:
-    """Blocks per row: rows are zero-padded to 16 * ceil(N / 16) columns."""
-    return (N + 15) // 16
+BLOCK_SIZES = (16, 32)
+
+
+def padded_blocks(N: int, block: int = 16) -> int:
+    """Blocks per row: rows are zero-padded to block * ceil(N / block) columns."""
+    return (N + block - 1) // block
+
+
+def _block(block) -> int:
+    if block not in BLOCK_SIZES:
+        raise ValueError(f"block must be one of {BLOCK_SIZES}, got {block!r}")
+    return int(block)
 
 
 def new_workspace(device) -> torch.Tensor:
@@ -215,15 +227,18 @@ def nvfp4_observe_amax(x: torch.Tensor, state: torch.Tensor, kind="static_minmax
 
 
 def nvfp4_quantize(x: torch.Tensor, amax: torch.Tensor, packed: torch.Tensor | None = None,
-                   scales: torch.Tensor | None = None, global_scale: torch.Tensor | None = None):
-    """bf16 [..., N] -> (packed uint8 [..., N/2], E4M3 scale bytes uint8 [..., N/16],
-    global scale fp32 [1]).  ``amax`` is the tensor's (or siblings', or observer's) amax."""
+                   scales: torch.Tensor | None = None, global_scale: torch.Tensor | None = None,
+                   block: int = 16):
+    """bf16 [..., N] -> (packed uint8 [..., P/2], E4M3 scale bytes uint8 [..., P/block],
+    global scale fp32 [1]), P = block * ceil(N / block).  ``amax`` is the tensor's (or
+    siblings', or observer's) amax; ``block`` is 16 (NVFP4) or 32."""
+    block = _block(block)
     M, N = _matrix(x)
     _scalar(amax, "amax")
-    B = padded_blocks(N)
+    B = padded_blocks(N, block)
     lead = tuple(x.shape[:-1])
     if packed is None:
-        packed = torch.empty(lead + (8 * B,), dtype=torch.uint8, device=x.device)
+        packed = torch.empty(lead + (block // 2 * B,), dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty(lead + (B,), dtype=torch.uint8, device=x.device)
     if global_scale is None:
@@ -231,11 +246,16 @@ def nvfp4_quantize(x: torch.Tensor, amax: torch.Tensor, packed: torch.Tensor | N
     _cuda(packed, "packed", torch.uint8)
     _cuda(scales, "scales", torch.uint8)
     _scalar(global_scale, "global_scale")
-    if packed.numel() != M * 8 * B or scales.numel() != M * B:
+    if packed.numel() != M * block // 2 * B or scales.numel() != M * B:
         raise RuntimeError("packed / scales have the wrong number of elements")
     with torch.cuda.device(x.device):
-        _check(_c_quantize(x.data_ptr(), M, N, amax.data_ptr(), packed.data_ptr(), scales.data_ptr(),
-                           global_scale.data_ptr(), _stream(x.device)), "nvfp4_quantize")
+        if block == 16:
+            st = _c_quantize(x.data_ptr(), M, N, amax.data_ptr(), packed.data_ptr(), scales.data_ptr(),
+                             global_scale.data_ptr(), _stream(x.device))
+        else:
+            st = _c_quantize_bs(x.data_ptr(), M, N, block, amax.data_ptr(), packed.data_ptr(), scales.data_ptr(),
+                                global_scale.data_ptr(), _stream(x.device))
+        _check(st, "nvfp4_quantize")
     return packed, scales, global_scale
 
 
@@ -271,19 +291,20 @@ def nvfp4_quantize_mma(x: torch.Tensor, amax: torch.Tensor, packed: torch.Tensor
 
 
 def nvfp4_dequantize(packed: torch.Tensor, scales: torch.Tensor, global_scale: torch.Tensor,
-                     out: torch.Tensor | None = None, n_cols: int | None = None) -> torch.Tensor:
-    """(packed [..., P/2], scales [..., P/16], global scale) -> bf16 [..., N].  ``n_cols``
+                     out: torch.Tensor | None = None, n_cols: int | None = None, block: int = 16) -> torch.Tensor:
+    """(packed [..., P/2], scales [..., P/block], global scale) -> bf16 [..., N].  ``n_cols``
     is the unpadded row length N (default P, the padded length), as the page keeps the
     original shape next to the packed weight."""
+    block = _block(block)
     _cuda(packed, "packed", torch.uint8)
     _cuda(scales, "scales", torch.uint8)
     _scalar(global_scale, "global_scale")
     P = packed.shape[-1] * 2
     N = P if n_cols is None else int(n_cols)
-    if padded_blocks(N) * 16 != P:
+    if padded_blocks(N, block) * block != P:
         raise RuntimeError(f"n_cols={N} does not match packed rows of {P // 2} bytes")
     M = math.prod(packed.shape[:-1])
-    if scales.numel() != M * (P // 16):
+    if scales.numel() != M * (P // block):
         raise RuntimeError("scales has the wrong number of elements")
     if out is None:
         out = torch.empty(tuple(packed.shape[:-1]) + (N,), dtype=torch.bfloat16, device=packed.device)
@@ -291,13 +312,21 @@ def nvfp4_dequantize(packed: torch.Tensor, scales: torch.Tensor, global_scale: t
     if out.numel() != M * N:
         raise RuntimeError("out has the wrong number of elements")
     with torch.cuda.device(packed.device):
-        _check(_c_dequantize(packed.data_ptr(), scales.data_ptr(), global_scale.data_ptr(), M, N,
-                             out.data_ptr(), _stream(packed.device)), "nvfp4_dequantize")
+        if block == 16:
+            st = _c_dequantize(packed.data_ptr(), scales.data_ptr(), global_scale.data_ptr(), M, N,
+                               out.data_ptr(), _stream(packed.device))
+        else:
+            st = _c_dequantize_bs(packed.data_ptr(), scales.data_ptr(), global_scale.data_ptr(), M, N, block,
+                                  out.data_ptr(), _stream(packed.device))
+        _check(st, "nvfp4_dequantize")
     return out
 
 
-def nvfp4_fake_quant(x: torch.Tensor, amax: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
-    """bf16 -> bf16 fake-quantization (dequantize(quantize(x)) in one pass).  ``out`` may be x."""
+def nvfp4_fake_quant(x: torch.Tensor, amax: torch.Tensor, out: torch.Tensor | None = None,
+                     block: int = 16) -> torch.Tensor:
+    """bf16 -> bf16 fake-quantization (dequantize(quantize(x)) in one pass).  ``out`` may be x;
+    ``block`` is 16 (NVFP4) or 32."""
+    block = _block(block)
     M, N = _matrix(x)
     _scalar(amax, "amax")
     if out is None:
@@ -306,8 +335,11 @@ def nvfp4_fake_quant(x: torch.Tensor, amax: torch.Tensor, out: torch.Tensor | No
     if out.numel() != x.numel():
         raise RuntimeError("out has the wrong number of elements")
     with torch.cuda.device(x.device):
-        _check(_c_fake_quant(x.data_ptr(), out.data_ptr(), M, N, amax.data_ptr(), _stream(x.device)),
-               "nvfp4_fake_quant")
+        if block == 16:
+            st = _c_fake_quant(x.data_ptr(), out.data_ptr(), M, N, amax.data_ptr(), _stream(x.device))
+        else:
+            st = _c_fake_quant_bs(x.data_ptr(), out.data_ptr(), M, N, block, amax.data_ptr(), _stream(x.device))
+        _check(st, "nvfp4_fake_quant")
     return out
 
 
@@ -406,13 +438,13 @@ class FakeQuantSTE(torch.autograd.Function):
     unchanged): the verl linear.py tutorial, section 2 (STEFP4QuantTriton)."""
 
     @staticmethod
-    def forward(ctx, x, amax):
-        return nvfp4_fake_quant(x.contiguous(), amax)
+    def forward(ctx, x, amax, block=16):
+        return nvfp4_fake_quant(x.contiguous(), amax, block=block)
 
     @staticmethod
     def backward(ctx, grad_output):
-        return grad_output, None
+        return grad_output, None, None
 
 
-def fake_quant_ste(x: torch.Tensor, amax: torch.Tensor) -> torch.Tensor:
-    return FakeQuantSTE.apply(x, amax)
+def fake_quant_ste(x: torch.Tensor, amax: torch.Tensor, block: int = 16) -> torch.Tensor:
+    return FakeQuantSTE.apply(x, amax, block)

@@ -56,24 +56,24 @@ def _row_chunks(M, parts):
     return [(r, min(M, r + step)) for r in range(0, M, step)]
 
 
-def oracle_quantize_rows(x_bits, gs, threads=8):
+def oracle_quantize_rows(x_bits, gs, threads=8, block=16):
     import oracle
     from concurrent.futures import ThreadPoolExecutor
     M, N = x_bits.shape
-    B = (N + 15) // 16  # rows are zero-padded to 16 * B columns
-    packed = np.empty((M, 8 * B), dtype=np.uint8)
+    B = (N + block - 1) // block  # rows are zero-padded to block * B columns
+    packed = np.empty((M, block // 2 * B), dtype=np.uint8)
     scales = np.empty((M, B), dtype=np.uint8)
 
     def work(rr):
         r0, r1 = rr
-        p, s = oracle.quantize(x_bits[r0:r1], gs)
+        p, s = oracle.quantize(x_bits[r0:r1], gs, block)
         packed[r0:r1], scales[r0:r1] = p, s
     with ThreadPoolExecutor(threads) as pool:
         list(pool.map(work, _row_chunks(M, threads * 2)))
     return packed, scales
 
 
-def oracle_fake_quant_rows(x_bits, amax, threads=8):
+def oracle_fake_quant_rows(x_bits, amax, threads=8, block=16):
     import oracle
     from concurrent.futures import ThreadPoolExecutor
     M, N = x_bits.shape
@@ -81,13 +81,13 @@ def oracle_fake_quant_rows(x_bits, amax, threads=8):
 
     def work(rr):
         r0, r1 = rr
-        y[r0:r1] = oracle.fake_quant(x_bits[r0:r1], amax)
+        y[r0:r1] = oracle.fake_quant(x_bits[r0:r1], amax, block)
     with ThreadPoolExecutor(threads) as pool:
         list(pool.map(work, _row_chunks(M, threads * 2)))
     return y
 
 
-def oracle_dequantize_rows(packed, scales, gs, threads=8, n_cols=None):
+def oracle_dequantize_rows(packed, scales, gs, threads=8, n_cols=None, block=16):
     import oracle
     from concurrent.futures import ThreadPoolExecutor
     M = packed.shape[0]
@@ -96,7 +96,7 @@ def oracle_dequantize_rows(packed, scales, gs, threads=8, n_cols=None):
 
     def work(rr):
         r0, r1 = rr
-        y[r0:r1] = oracle.dequantize(packed[r0:r1], scales[r0:r1], gs, r1 - r0, N)
+        y[r0:r1] = oracle.dequantize(packed[r0:r1], scales[r0:r1], gs, r1 - r0, N, block)
     with ThreadPoolExecutor(threads) as pool:
         list(pool.map(work, _row_chunks(M, threads * 2)))
     return y

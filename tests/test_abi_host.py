@@ -31,6 +31,7 @@ def test_header_declares_the_entry_points():
     names = declared_symbols()
     for required in ["nvfp4_amax", "nvfp4_amax_multi", "nvfp4_observer_update", "nvfp4_observe_amax",
                      "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fake_quant", "nvfp4_fake_quant_siblings",
+                     "nvfp4_quantize_bs", "nvfp4_dequantize_bs", "nvfp4_fake_quant_bs",
                      "nvfp4_status_string", "nvfp4_kernel_launch_count"]:
         assert required in names
 
@@ -73,6 +74,10 @@ def _p(v):
     return ctypes.c_void_p(v)
 
 
+def _c(v):
+    return ctypes.c_int(v)
+
+
 def _gpu_visible():
     try:
         import torch
@@ -111,6 +116,16 @@ def test_validation_errors_launch_nothing(lib):
         (ERR_NULL, "nvfp4_dequantize", _p(A32), _p(A32), _p(0), _i(2), _i(16), _p(A32), S),
         (ERR_ALIGN, "nvfp4_dequantize", _p(A32), _p(A32), gs, _i(2), _i(16), _p(A8), S),
         (ERR_SHAPE, "nvfp4_dequantize", _p(A32), _p(A32), gs, _i(-2), _i(17), _p(A32), S),
+        # block-size variants: only 16 and 32; block 32 wants 16-byte aligned codes
+        (ERR_ARG, "nvfp4_quantize_bs", _p(A32), _i(2), _i(64), _c(64), amax, _p(A32), _p(A32), gs, S),
+        (ERR_ARG, "nvfp4_quantize_bs", _p(A32), _i(2), _i(64), _c(0), amax, _p(A32), _p(A32), gs, S),
+        (ERR_ARG, "nvfp4_fake_quant_bs", _p(A32), _p(A32 + 4096), _i(2), _i(64), _c(8), amax, S),
+        (ERR_ARG, "nvfp4_dequantize_bs", _p(A32), _p(A32), gs, _i(2), _i(64), _c(-32), _p(A32), S),
+        (ERR_ALIGN, "nvfp4_quantize_bs", _p(A32), _i(2), _i(64), _c(32), amax, _p(A8), _p(A32), gs, S),
+        (ERR_ALIGN, "nvfp4_dequantize_bs", _p(A8), _p(A32), gs, _i(2), _i(64), _c(32), _p(A32), S),
+        (ERR_SHAPE, "nvfp4_quantize_bs", _p(A32), _i(1 << 56), _i(33), _c(32), amax, _p(A32), _p(A32), gs, S),
+        (ERR_SHAPE, "nvfp4_fake_quant_bs", _p(A32), _p(A32 + 4096), _i(2), _i(-32), _c(32), amax, S),
+        (ERR_NULL, "nvfp4_fake_quant_bs", _p(A32), _p(A32 + 4096), _i(2), _i(64), _c(32), _p(0), S),
         # amax
         (ERR_NULL, "nvfp4_amax", _p(A32), _i(16), _p(0), S),
         (ERR_NULL, "nvfp4_amax", _p(0), _i(16), amax, S),

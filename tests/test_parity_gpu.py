@@ -51,7 +51,7 @@ def _full_check(x_bits, amax_value=None, what=""):
 
 def test_worked_examples_gpu(golden_dir):
     with open(os.path.join(golden_dir, "worked_examples.json")) as f:
-        cases = json.load(f)["cases"]
+        cases = [c for c in json.load(f)["cases"] if c.get("block", 16) == 16]  # block 32: its own file
     for case in cases:
         M, N = case["rows"], case["cols"]
         x = synthetic.to_bf16_bits(np.array(case["x"], dtype=np.float32).reshape(M, N))
