@@ -443,6 +443,7 @@ def run_sweep(args):
         amax = nv.nvfp4_amax(x)
         y = torch.empty_like(x)
         packed, scales, gs = nv.nvfp4_quantize(x, amax)
+        packed32, scales32, _ = nv.nvfp4_quantize(x, amax, block=32)
         scales_mma = torch.empty(nv.mma_scale_bytes(M, N), dtype=torch.uint8, device=dev)
         t = {
             "amax": (2.0, timed(lambda: nv.nvfp4_amax(x, out=amax, workspace=ws))),
@@ -452,12 +453,17 @@ def run_sweep(args):
             "quantize": (2.5625, timed(lambda: nv.nvfp4_quantize(x, amax, packed, scales, gs))),
             "quantize_mma": (2.5625, timed(lambda: nv.nvfp4_quantize_mma(x, amax, packed, scales_mma, gs))),
             "dequantize": (2.5625, timed(lambda: nv.nvfp4_dequantize(packed, scales, gs, out=y))),
+            # blocks of 32: 1/32 of a scale byte per element
+            "fake_quant_b32": (4.0, timed(lambda: nv.nvfp4_fake_quant(x, amax, out=y, block=32))),
+            "quantize_b32": (2.53125, timed(lambda: nv.nvfp4_quantize(x, amax, packed32, scales32, gs, block=32))),
+            "dequantize_b32": (2.53125, timed(lambda: nv.nvfp4_dequantize(packed32, scales32, gs, out=y,
+                                                                          block=32))),
         }
         rec = {"workload": name, "shape": [M, N], "bytes": 2 * n}
         for k, (bpe, sec) in t.items():
             rec[k] = {"us": sec * 1e6, "GB/s": n * bpe / sec / 1e9, "frac": n * bpe / sec / 1e9 / peak}
         rows.append(rec)
-        del x, y, packed, scales, scales_mma
+        del x, y, packed, scales, scales_mma, packed32, scales32
     # the q/k/v siblings: shared amax + fake-quant of all three in one call
     qkv = [synthetic.activation_normal_device(s, 98, dev) for s in ((4096, 4096), (1024, 4096), (1024, 4096))]
     outs = [torch.empty_like(t) for t in qkv]
@@ -468,7 +474,8 @@ def run_sweep(args):
                  "bytes": 2 * n, "siblings": {"us": sec * 1e6, "GB/s": n * 6.0 / sec / 1e9,
                                                "frac": n * 6.0 / sec / 1e9 / peak}})
 
-    cols = ["amax", "fake_quant", "fake_quant_with_own_amax", "quantize", "quantize_mma", "dequantize"]
+    cols = ["amax", "fake_quant", "fake_quant_with_own_amax", "quantize", "quantize_mma", "dequantize",
+            "fake_quant_b32", "quantize_b32", "dequantize_b32"]
     print(f"peak {peak:.1f} GB/s ({peak_src}); GB/s of algorithmic bytes (frac of peak); L2 flushed by a read")
     print("| workload | shape | " + " | ".join(cols) + " |")
     print("|---|---|" + "---|" * len(cols))

@@ -184,6 +184,33 @@ def fake_quant(x_bits, amax_value: float, block: int = 16):
     return y
 
 
+def bf16_to_f64(bits) -> np.ndarray:
+    """bf16 bit patterns -> float64 values (exact: bf16 is the top half of an fp32)."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def w4a16_linear(x_bits, packed, scales, global_scale_value: float, n_out: int, block: int = 16,
+                 bias_bits=None):
+    """The forward of a Linear layer whose weight is stored packed ([FP4OPT]
+    _float4_autocast_forward): for the duration of one forward the packed weight is replaced
+    by dequantize_weight_from_float4(...) in bf16, and the layer's own forward
+    y = x W^T (+ bias) runs on it.
+
+    x_bits: uint16 [M, K] (bf16 activations); packed / scales: the weight [n_out, K] as
+    quantize() returns it; bias_bits: optional uint16 [n_out].  Returns float64 [M, n_out]:
+    the exact products (a product of two bf16 values is exact in float64) summed by a
+    library float64 matmul, before the forward's rounding of its output to bf16.  Rows are
+    independent, so the caller may pass any subset of activation rows."""
+    x = bf16_to_f64(x_bits)
+    M, K = x.shape
+    w = bf16_to_f64(dequantize(packed, scales, global_scale_value, n_out, K, block))
+    y = x @ w.T
+    if bias_bits is not None:
+        y = y + bf16_to_f64(np.asarray(bias_bits).reshape(1, n_out))
+    return y
+
+
 def observer_update(state: float, cur: float, kind: int, decay: float = 0.01) -> float:
     return _lib().oracle_observer_update(f32(state), f32(cur), int(kind), float(decay))
 

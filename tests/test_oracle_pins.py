@@ -461,3 +461,78 @@ def test_block_32_scale_is_the_larger_half_scale():
     _, s16 = oracle.quantize(x, gs, 16)
     _, s32 = oracle.quantize(x, gs, 32)
     np.testing.assert_array_equal(s32, np.maximum(s16[:, 0::2], s16[:, 1::2]))
+
+
+# ---- the packed-weight linear forward (W4A16) -----------------------------------------------
+
+def _packed_weight(n_out, K, seed):
+    rng = np.random.default_rng(seed)
+    w = synthetic.to_bf16_bits((rng.standard_normal((n_out, K)) * 0.02).astype(np.float32))
+    gs = oracle.global_scale(oracle.amax(w))
+    packed, scales = oracle.quantize(w, gs)
+    return packed, scales, gs
+
+
+def test_linear_one_hot_rows_select_weight_columns():
+    """x = rows of the identity: y[m, n] = W[n, m] with W the dequantized weight, exactly.
+    A transposed operand or a misread block would break it (the weight is not square)."""
+    n_out, K = 48, 64
+    packed, scales, gs = _packed_weight(n_out, K, 70)
+    w = oracle.bf16_to_f64(oracle.dequantize(packed, scales, gs, n_out, K))
+    x = _bf16_bits(np.eye(K, dtype=np.float32))
+    y = oracle.w4a16_linear(x, packed, scales, gs, n_out)
+    assert y.shape == (K, n_out)
+    assert np.array_equal(y, w.T)
+
+
+def test_linear_brute_force_exact_rationals():
+    """Tiny case by exact rational arithmetic (Fractions of the bf16 values): the float64
+    result is the exact sum to within float64 rounding."""
+    from fractions import Fraction
+    n_out, K, M = 5, 32, 3
+    packed, scales, gs = _packed_weight(n_out, K, 71)
+    wb = oracle.dequantize(packed, scales, gs, n_out, K)
+    rng = np.random.default_rng(72)
+    xb = _bf16_bits(rng.standard_normal((M, K)))
+    bb = _bf16_bits(rng.standard_normal(n_out))
+    fr = lambda b: Fraction(float(np.uint32(int(b) << 16).view(np.float32)))
+    y = oracle.w4a16_linear(xb, packed, scales, gs, n_out, bias_bits=bb)
+    for m in range(M):
+        for n in range(n_out):
+            exact = sum(fr(xb[m, k]) * fr(wb[n, k]) for k in range(K)) + fr(bb[n])
+            assert abs(Fraction(y[m, n]) - exact) <= abs(exact) * Fraction(1, 2 ** 48) + Fraction(1, 2 ** 120)
+
+
+def test_linear_zero_activations_give_the_bias():
+    n_out, K = 40, 32
+    packed, scales, gs = _packed_weight(n_out, K, 73)
+    bias = _bf16_bits(np.linspace(-3, 3, n_out))
+    y = oracle.w4a16_linear(np.zeros((4, K), dtype=np.uint16), packed, scales, gs, n_out, bias_bits=bias)
+    assert np.array_equal(y, np.broadcast_to(oracle.bf16_to_f64(bias), (4, n_out)))
+
+
+def test_linear_uses_the_dequantized_weight():
+    """A weight whose every block is 6*S followed by E2M1 grid points times S (S = 2^-j,
+    amax 0.375 so the global scale is 7168 and every block scale is exact) survives
+    quantize -> dequantize exactly, so the forward on the packed weight equals the plain
+    product with the original bf16 weight."""
+    rng = np.random.default_rng(75)
+    n_out, K = 24, 128
+    mags = np.asarray(synthetic.GRID_MAGNITUDES, dtype=np.float64)
+    S = 2.0 ** -rng.integers(4, 8, size=(n_out, K // 16, 1))
+    vals = mags[rng.integers(0, len(mags), size=(n_out, K // 16, 16))] * rng.choice([-1.0, 1.0], size=(n_out, K // 16, 16))
+    vals[vals == 0] = 0.0  # -0.0 encodes as +0 (the code's sign is set only below zero)
+    vals[:, :, 0] = 6.0
+    S[0, 0, 0] = 2.0 ** -4  # its first element is the tensor amax 0.375
+    w = _bf16_bits((vals * S).reshape(n_out, K))
+    a = oracle.amax(w)
+    assert a == 0.375
+    gs = oracle.global_scale(a)
+    packed, scales = oracle.quantize(w, gs)
+    assert np.array_equal(oracle.dequantize(packed, scales, gs, n_out, K), w)
+    x = _bf16_bits(rng.standard_normal((6, K)))
+    y = oracle.w4a16_linear(x, packed, scales, gs, n_out)
+    assert np.array_equal(y, oracle.bf16_to_f64(x) @ oracle.bf16_to_f64(w).T)
+    # scaling x by a power of two scales y exactly
+    x4 = _bf16_bits(oracle.bf16_to_f64(x) * 4.0)
+    assert np.array_equal(oracle.w4a16_linear(x4, packed, scales, gs, n_out), 4.0 * y)
