@@ -286,6 +286,35 @@ nvfp4_status nvfp4_dequantize_bs(const uint8_t* packed, const uint8_t* scales, c
 nvfp4_status nvfp4_fake_quant_bs(const void* x, void* y, int64_t M, int64_t N, int block, const float* d_amax,
                                  nvfp4_stream_t stream);
 
+/* ---- forward of a Linear layer on a packed weight (W4A16) ---------------------------- */
+
+/* y = x . W^T (+ bias), W the bf16 weight that dequantize_weight_from_float4 rebuilds from
+ * (packed, scales, global scale): [FP4OPT] _float4_autocast_forward, which unpacks the
+ * weight for one forward and runs the layer's bf16 forward on it.  One kernel on the
+ * tensor cores (bf16 x bf16, fp32 accumulation, output rounded to bf16 once; the bias is
+ * added to the fp32 sum before that rounding); the decoded weight is built tile by tile in
+ * shared memory and never written to device memory.  Each weight element is decoded
+ * exactly as nvfp4_dequantize does; the sum is not bit-reproducible against another GEMM
+ * (the accumulation order of the tensor cores is not IEEE sequential), see the tests for
+ * the bound used.
+ *   x       bf16 [M, K] row-major, 16-byte aligned
+ *   K       > 0, a multiple of 16 (the packed layout of a weight whose rows need no padding)
+ *   packed  uint8 [N, K/2], 8-byte aligned; scales uint8 [N, K/16]: nvfp4_quantize's output
+ *           for the weight [N, K]
+ *   d_global_scale  fp32: the weight's encode global scale
+ *   bias    bf16 [N] or NULL
+ *   y       bf16 out [M, N] row-major, 2-byte aligned (16-byte aligned with N % 8 == 0 is
+ *           faster); must not overlap the inputs
+ *   d_workspace  a workspace as above: a bounded wait inside the kernel that runs out
+ *           records NVFP4_ERR_TIMEOUT there (nvfp4_workspace_check), the kernel stops and y is
+ *           unspecified.  The call does not otherwise use it.
+ * Errors: NVFP4_ERR_SHAPE (K not a positive multiple of 16, sizes past the 32-bit tensor-map
+ * limits), NVFP4_ERR_NULL, NVFP4_ERR_ALIGN, NVFP4_ERR_ARG (tensor map rejected).  M == 0 or
+ * N == 0 launches nothing.  Enqueues one kernel. */
+nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* packed, const uint8_t* scales,
+                                const float* d_global_scale, int64_t N, const void* bias, void* y,
+                                void* d_workspace, nvfp4_stream_t stream);
+
 /* Human-readable name of a status code (a static string). */
 const char* nvfp4_status_string(nvfp4_status status);
 

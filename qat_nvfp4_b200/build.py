@@ -14,8 +14,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libnvfp4.so")
-SOURCES = [os.path.join(CSRC, "nvfp4_kernels.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, "nvfp4_device.cuh"), os.path.join(INCLUDE, "nvfp4.h")]
+SOURCES = [os.path.join(CSRC, "nvfp4_kernels.cu"), os.path.join(CSRC, "nvfp4_w4a16.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, "nvfp4_device.cuh"), os.path.join(CSRC, "nvfp4_runtime.h"),
+                  os.path.join(INCLUDE, "nvfp4.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

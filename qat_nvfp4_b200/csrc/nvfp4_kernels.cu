@@ -21,6 +21,7 @@
 
 #include "nvfp4.h"
 #include "nvfp4_device.cuh"
+#include "nvfp4_runtime.h"
 
 #define NVFP4_API extern "C" __attribute__((visibility("default")))
 
@@ -321,14 +322,6 @@ __global__ void observer_kernel(float* state, const float* cur, int kind, float 
 // two atomics), so it publishes the amax, applies the observer step if asked, and puts
 // the workspace back to zero for the next call.  No CTA ever waits for another.
 
-struct Workspace {
-    unsigned acc;       // running max |x| as fp32 bits
-    unsigned arrived;   // CTAs that have finished their share of the amax
-    unsigned departed;  // CTAs that have left the grid barrier (fused kernel)
-    unsigned error;     // NVFP4_ERR_TIMEOUT once a bounded wait gave up
-    unsigned pad[60];
-};
-static_assert(sizeof(Workspace) == 256, "NVFP4_WORKSPACE_BYTES");
 
 __device__ __forceinline__ bool last_to_arrive(Workspace* ws, float cta_amax) {
     __shared__ bool last;
@@ -930,7 +923,7 @@ nvfp4_status grid_for(const void* fn, int64_t items, int per_thread, int mult, i
 }
 
 nvfp4_status after_launch() {
-    g_launches.fetch_add(1, std::memory_order_relaxed);
+    note_launch();
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
@@ -1101,6 +1094,10 @@ NVFP4_API const char* nvfp4_status_string(nvfp4_status status) {
     }
     return "NVFP4 status: unknown code";
 }
+
+namespace nvfp4 {
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace nvfp4
 
 NVFP4_API uint64_t nvfp4_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 

@@ -31,7 +31,7 @@ def test_header_declares_the_entry_points():
     names = declared_symbols()
     for required in ["nvfp4_amax", "nvfp4_amax_multi", "nvfp4_observer_update", "nvfp4_observe_amax",
                      "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fake_quant", "nvfp4_fake_quant_siblings",
-                     "nvfp4_quantize_bs", "nvfp4_dequantize_bs", "nvfp4_fake_quant_bs",
+                     "nvfp4_quantize_bs", "nvfp4_dequantize_bs", "nvfp4_fake_quant_bs", "nvfp4_w4a16_linear",
                      "nvfp4_status_string", "nvfp4_kernel_launch_count"]:
         assert required in names
 
@@ -126,6 +126,22 @@ def test_validation_errors_launch_nothing(lib):
         (ERR_SHAPE, "nvfp4_quantize_bs", _p(A32), _i(1 << 56), _i(33), _c(32), amax, _p(A32), _p(A32), gs, S),
         (ERR_SHAPE, "nvfp4_fake_quant_bs", _p(A32), _p(A32 + 4096), _i(2), _i(-32), _c(32), amax, S),
         (ERR_NULL, "nvfp4_fake_quant_bs", _p(A32), _p(A32 + 4096), _i(2), _i(64), _c(32), _p(0), S),
+        # W4A16 linear: x, M, K, packed, scales, gs, N, bias, y, workspace
+        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(24), _p(A32), _p(A32), gs, _i(8), _p(0), _p(A32),
+         _p(A32), S),
+        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(0), _p(A32), _p(A32), gs, _i(8), _p(0), _p(A32),
+         _p(A32), S),
+        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(-1), _i(64), _p(A32), _p(A32), gs, _i(8), _p(0), _p(A32),
+         _p(A32), S),
+        (ERR_NULL, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(A32), _p(A32), gs, _i(8), _p(0), _p(A32),
+         _p(0), S),
+        (ERR_NULL, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(0), _p(A32), gs, _i(8), _p(0), _p(A32),
+         _p(A32), S),
+        (ERR_ALIGN, "nvfp4_w4a16_linear", _p(A8), _i(4), _i(64), _p(A32), _p(A32), gs, _i(8), _p(0), _p(A32),
+         _p(A32), S),
+        (ERR_ALIGN, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(A32 + 4), _p(A32), gs, _i(8), _p(0), _p(A32),
+         _p(A32), S),
+        (NVFP4_OK, "nvfp4_w4a16_linear", _p(0), _i(0), _i(64), _p(0), _p(0), gs, _i(8), _p(0), _p(0), _p(A32), S),
         # amax
         (ERR_NULL, "nvfp4_amax", _p(A32), _i(16), _p(0), S),
         (ERR_NULL, "nvfp4_amax", _p(0), _i(16), amax, S),

@@ -1,0 +1,127 @@
+"""Parity of the tensor-core W4A16 linear (nvfp4_w4a16_linear) with the oracle's forward of
+a Linear layer on a packed weight (fp4_optimization.py, _float4_autocast_forward).
+
+The weight the kernel multiplies by is decoded exactly as nvfp4_dequantize does (checked
+bit for bit elsewhere); what is not bit-reproducible is the fp32 sum inside the tensor
+cores.  Bound per output element, with exact = the oracle's float64 result and
+mag = sum_k |x_k| |w_k| (+ |bias|):
+
+    |y - exact| <= 2^-8 |exact| + (1 + 2^-8) K 2^-23 mag
+
+(every bf16 x bf16 product is exact in fp32; an fp32 sum of K terms in any order, rounded
+or truncated, is within K 2^-23 mag of the exact sum; rounding the result to bf16 adds at
+most half an ulp, 2^-8 relative.)  Shapes span several tiles in both dimensions with
+ragged edges in M, N and K, the single-tile and single-row cases, and the pages' MLP
+weight (14336 x 4096) under 4096 tokens on sampled rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from qat_nvfp4_b200 import synthetic
+from nvfp4_testutil import bits, sample_rows, to_dev, u8
+
+pytestmark = pytest.mark.gpu
+
+nv = pytest.importorskip("qat_nvfp4_b200.nvfp4")
+
+
+def _weight(n_out, K, seed, std=0.02):
+    rng = np.random.default_rng(seed)
+    w = synthetic.to_bf16_bits((rng.standard_normal((n_out, K)) * std).astype(np.float32))
+    wd = to_dev(w)
+    packed, scales, gs = nv.nvfp4_quantize(wd, nv.nvfp4_amax(wd))
+    return packed, scales, gs
+
+
+def _assert_within_bound(y_bits, x_bits, packed, scales, gs, bias_bits, what):
+    """y_bits: uint16 [R, N] for the activation rows x_bits [R, K]."""
+    pk, sc = u8(packed), u8(scales)
+    n_out, K = pk.shape[0], x_bits.shape[1]
+    g = float(gs.item())
+    exact = oracle.w4a16_linear(x_bits, pk, sc, g, n_out, bias_bits=bias_bits)
+    w = oracle.bf16_to_f64(oracle.dequantize(pk, sc, g, n_out, K))
+    mag = np.abs(oracle.bf16_to_f64(x_bits)) @ np.abs(w).T
+    if bias_bits is not None:
+        mag = mag + np.abs(oracle.bf16_to_f64(bias_bits))[None, :]
+    tol = 2.0 ** -8 * np.abs(exact) + (1 + 2.0 ** -8) * K * 2.0 ** -23 * mag
+    got = oracle.bf16_to_f64(y_bits)
+    err = np.abs(got - exact)
+    bad = np.argwhere(err > tol)
+    assert bad.size == 0, (f"{what}: {len(bad)} elements outside the bound, first {bad[:3].tolist()}: "
+                           f"got {got[tuple(bad[0])]}, exact {exact[tuple(bad[0])]}, tol {tol[tuple(bad[0])]}")
+    return exact
+
+
+@pytest.mark.parametrize("M,K,N,with_bias", [
+    (128, 64, 128, False),     # one tile, one stage
+    (128, 1024, 256, True),    # 16 stages, two output tiles
+    (300, 1040, 200, True),    # ragged M, N and K (K % 64 == 16)
+    (37, 48, 24, False),       # K below one stage
+    (5, 16, 13, True),         # N odd: element stores
+    (1, 4096, 4096, False),    # one token
+    (513, 2048, 1000, True),
+])
+def test_linear_matches_oracle(M, K, N, with_bias):
+    rng = np.random.default_rng(M * 7 + K * 3 + N)
+    x = synthetic.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    packed, scales, gs = _weight(N, K, M + K + N)
+    bias = synthetic.to_bf16_bits(rng.standard_normal(N).astype(np.float32)) if with_bias else None
+    ws = nv.new_workspace("cuda")
+    y = nv.nvfp4_w4a16_linear(to_dev(x), packed, scales, gs, bias=to_dev(bias) if with_bias else None,
+                              workspace=ws)
+    torch.cuda.synchronize()
+    assert nv.nvfp4_workspace_check(ws) == 0
+    assert tuple(y.shape) == (M, N)
+    _assert_within_bound(bits(y), x, packed, scales, gs, bias, f"{M}x{K} . {N}x{K}^T")
+
+
+def test_linear_agrees_with_a_library_gemm_on_the_dequantized_weight():
+    """Same inputs through nvfp4_dequantize + torch's bf16 linear (cuBLAS): both are within
+    the bound of the exact result, and they differ by at most one bf16 ulp almost
+    everywhere."""
+    M, K, N = 1024, 4096, 2048
+    rng = np.random.default_rng(5)
+    x = to_dev(synthetic.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32)))
+    packed, scales, gs = _weight(N, K, 6)
+    bias = to_dev(synthetic.to_bf16_bits(rng.standard_normal(N).astype(np.float32)))
+    ours = nv.nvfp4_w4a16_linear(x, packed, scales, gs, bias=bias)
+    w = nv.nvfp4_dequantize(packed, scales, gs)
+    ref = torch.nn.functional.linear(x, w, bias)
+    rows = sample_rows(M, 32, seed=1)
+    _assert_within_bound(bits(ours)[rows], bits(x)[rows], packed, scales, gs, bits(bias), "ours")
+    _assert_within_bound(bits(ref)[rows], bits(x)[rows], packed, scales, gs, bits(bias), "cuBLAS")
+    d = (ours.float() - ref.float()).abs()
+    ulp = torch.finfo(torch.bfloat16).eps * ref.float().abs().clamp_min(1e-30)
+    assert (d <= ulp).float().mean().item() > 0.99
+
+
+def test_mlp_weight_4096_tokens_sampled_rows():
+    """The pages' MLP weight 14336 x 4096 N(0, 0.02) under 4096 tokens of N(0, 1)."""
+    M, K, N = 4096, 4096, 14336
+    x = synthetic.activation_normal_device((M, K), 31, "cuda")
+    w = synthetic.activation_normal_device((N, K), 32, "cuda") * 0.02
+    packed, scales, gs = nv.nvfp4_quantize(w, nv.nvfp4_amax(w))
+    y = nv.nvfp4_w4a16_linear(x, packed, scales, gs)
+    rows = sample_rows(M, 24, seed=3)
+    _assert_within_bound(bits(y)[rows], bits(x)[rows], packed, scales, gs, None, "MLP 4096 tokens")
+
+
+def test_out_parameter_and_leading_dimensions():
+    rng = np.random.default_rng(9)
+    x = to_dev(synthetic.to_bf16_bits(rng.standard_normal((2, 3, 256)).astype(np.float32)))
+    packed, scales, gs = _weight(64, 256, 10)
+    out = torch.full((2, 3, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    y = nv.nvfp4_w4a16_linear(x, packed, scales, gs, out=out)
+    assert y.data_ptr() == out.data_ptr()
+    _assert_within_bound(bits(y).reshape(6, 64), bits(x).reshape(6, 256), packed, scales, gs, None, "3-D x")
+
+
+def test_empty_rows_launch_nothing():
+    packed, scales, gs = _weight(32, 64, 11)
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    before = nv.nvfp4_kernel_launch_count()
+    y = nv.nvfp4_w4a16_linear(x, packed, scales, gs, workspace=nv.new_workspace("cuda"))
+    assert tuple(y.shape) == (0, 32)
+    assert nv.nvfp4_kernel_launch_count() == before
