@@ -288,19 +288,35 @@ nvfp4_status nvfp4_fake_quant_bs(const void* x, void* y, int64_t M, int64_t N, i
 
 /* ---- forward of a Linear layer on a packed weight (W4A16) ---------------------------- */
 
+/* The weight's operand form: the packed weight cut into 128-row x 64-column tiles, one
+ * contiguous 4608-byte record per tile, so that the linear kernel fetches a tile with one
+ * bulk copy.  Not on the pages, which keep the plain layout; the same bytes, reordered
+ * once when the weight is converted (as [FP4OPT] convert_model_weight_to_float4 packs each
+ * weight once).  Record (tn, tk), KT = ceil(K / 64), starts at byte (tn * KT + tk) * 4608:
+ *   bytes [0, 4096)     row r (0..127) at 32 r: the code bytes of columns 64 tk .. 64 tk + 63
+ *                       of weight row 128 tn + r (element 2j in the low nibble of byte j)
+ *   bytes [4096, 4608)  row r at 4096 + 4 r: the scale bytes of those columns' 4 blocks
+ * Rows past N and columns past K are code 0 / scale byte 0 (they decode to +0).
+ * nvfp4_w4a16_tiled_bytes returns the size, ceil(N / 128) * KT * 4608, or -1 if (N, K) is
+ * not accepted (K a positive multiple of 16, N >= 0). */
+int64_t nvfp4_w4a16_tiled_bytes(int64_t N, int64_t K);
+
+/* packed [N, K/2] (8-byte aligned) + scales [N, K/16] (nvfp4_quantize's output for a
+ * weight [N, K]) -> tiled (nvfp4_w4a16_tiled_bytes(N, K) bytes, 16-byte aligned), every
+ * byte written.  Errors: NVFP4_ERR_SHAPE, NVFP4_ERR_NULL, NVFP4_ERR_ALIGN.  One kernel. */
+nvfp4_status nvfp4_w4a16_pack(const uint8_t* packed, const uint8_t* scales, int64_t N, int64_t K,
+                              uint8_t* tiled, nvfp4_stream_t stream);
+
 /* y = x . W^T (+ bias), W the bf16 weight that dequantize_weight_from_float4 rebuilds from
- * (packed, scales, global scale): [FP4OPT] _float4_autocast_forward, which unpacks the
- * weight for one forward and runs the layer's bf16 forward on it.  One kernel on the
- * tensor cores (bf16 x bf16, fp32 accumulation, output rounded to bf16 once; the bias is
- * added to the fp32 sum before that rounding); the decoded weight is built tile by tile in
- * shared memory and never written to device memory.  Each weight element is decoded
- * exactly as nvfp4_dequantize does; the sum is not bit-reproducible against another GEMM
- * (the accumulation order of the tensor cores is not IEEE sequential), see the tests for
- * the bound used.
- *   x       bf16 [M, K] row-major, 16-byte aligned
- *   K       > 0, a multiple of 16 (the packed layout of a weight whose rows need no padding)
- *   packed  uint8 [N, K/2], 8-byte aligned; scales uint8 [N, K/16]: nvfp4_quantize's output
- *           for the weight [N, K]
+ * the packed weight: [FP4OPT] _float4_autocast_forward, which unpacks the weight for one
+ * forward and runs the layer's bf16 forward on it.  One kernel on the tensor cores (bf16 x
+ * bf16, fp32 accumulation, output rounded to bf16 once; the bias is added to the fp32 sum
+ * before that rounding); the decoded weight is built tile by tile in shared memory and
+ * never written to device memory.  Each weight element is decoded exactly as
+ * nvfp4_dequantize does; the sum is not bit-reproducible against another GEMM (the order
+ * in which the tensor cores accumulate is not sequential IEEE), the tests state the bound.
+ *   x       bf16 [M, K] row-major, 16-byte aligned; K a positive multiple of 16
+ *   tiled   the weight [N, K] in operand form (nvfp4_w4a16_pack), 16-byte aligned
  *   d_global_scale  fp32: the weight's encode global scale
  *   bias    bf16 [N] or NULL
  *   y       bf16 out [M, N] row-major, 2-byte aligned (16-byte aligned with N % 8 == 0 is
@@ -308,10 +324,10 @@ nvfp4_status nvfp4_fake_quant_bs(const void* x, void* y, int64_t M, int64_t N, i
  *   d_workspace  a workspace as above: a bounded wait inside the kernel that runs out
  *           records NVFP4_ERR_TIMEOUT there (nvfp4_workspace_check), the kernel stops and y is
  *           unspecified.  The call does not otherwise use it.
- * Errors: NVFP4_ERR_SHAPE (K not a positive multiple of 16, sizes past the 32-bit tensor-map
- * limits), NVFP4_ERR_NULL, NVFP4_ERR_ALIGN, NVFP4_ERR_ARG (tensor map rejected).  M == 0 or
- * N == 0 launches nothing.  Enqueues one kernel. */
-nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* packed, const uint8_t* scales,
+ * Errors: NVFP4_ERR_SHAPE (K, sizes past the 32-bit tensor-map limits), NVFP4_ERR_NULL,
+ * NVFP4_ERR_ALIGN, NVFP4_ERR_ARG (tensor map rejected).  M == 0 or N == 0 launches nothing.
+ * Enqueues one kernel. */
+nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* tiled,
                                 const float* d_global_scale, int64_t N, const void* bias, void* y,
                                 void* d_workspace, nvfp4_stream_t stream);
 

@@ -5,14 +5,16 @@
 // own bf16 forward runs on it).
 //
 // One kernel on the sm_100a tensor cores (tcgen05, kind::f16, bf16 operands, fp32
-// accumulator in tensor memory).  The bf16 weight is never written to HBM: producer warps
-// decode each 128 x 64 weight tile from its packed codes and E4M3 scale bytes straight into
-// the shared-memory operand layout (128-byte swizzle, K-major) with the same arithmetic as
-// nvfp4_dequantize, bf16_rn(fl(LUT[code] * fl(E4M3(byte) / gs))), while a TMA warp streams
-// the activation tile and one thread issues the MMAs.
+// accumulators in tensor memory).  The bf16 weight is never written to HBM.  The weight is
+// read in a tile-major copy of its packed form (nvfp4_w4a16_pack: one contiguous 4608-byte
+// record per 128-row x 64-column tile, codes then scale bytes), so each pipeline stage
+// fetches its weight tile with one bulk copy; producer warps decode it in shared memory into
+// the MMA operand layout (128-byte swizzle, K-major) with the same arithmetic as
+// nvfp4_dequantize, bf16_rn(fl(LUT[code] * fl(E4M3(byte) / gs))).  A CTA computes a
+// 256 x 128 output tile as two 128 x 128 accumulators that share each decoded weight tile.
 //
 //   warps 0-7  decode weight tiles into the ring, then the epilogue (TMEM -> bf16 -> y)
-//   warp 8     TMA loads of activation tiles (one elected thread)
+//   warp 8     TMA load of the activation tile + bulk copy of the weight record per stage
 //   warp 9     TMEM allocation, MMA issue (one elected thread), TMEM release
 //
 // Every wait on an mbarrier is bounded (kWaitLimitNs of %globaltimer); a wait that runs
@@ -36,29 +38,35 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int kBM = 128;                  // rows of x per tile (MMA M)
+constexpr int kBM = 256;                  // rows of x per tile: two MMAs of M = 128
+constexpr int kMmaM = 128;
 constexpr int kBN = 128;                  // weight rows (output features) per tile (MMA N)
 constexpr int kBK = 64;                   // K per stage: 64 bf16 = one 128-byte swizzle row
 constexpr int kUmmaK = 16;                // K of one kind::f16 MMA
-constexpr int kRing = 6;                  // stages in the shared-memory ring
+constexpr int kRing = 4;                  // stages in the shared-memory ring
 constexpr int kDecodeWarps = 8;
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kGemmThreads = 320;
-constexpr int kTileABytes = kBM * kBK * 2;  // 16 KB
-constexpr int kTileBBytes = kBN * kBK * 2;  // 16 KB
-constexpr int kTmemCols = kBN;              // fp32 accumulator: 128 lanes x kBN columns
-constexpr int kPrefetch = 4;                // weight stages a decode thread keeps in flight
+constexpr int kTileABytes = kBM * kBK * 2;   // 32 KB
+constexpr int kTileBBytes = kBN * kBK * 2;   // 16 KB
+constexpr int kRecCodes = kBN * kBK / 2;     // 4096 bytes of E2M1 codes per weight tile
+constexpr int kRecBytes = kRecCodes + kBN * (kBK / kBlockElems);  // + 512 scale bytes = 4608
+constexpr int kStageBytes = kTileABytes + kTileBBytes + kRecBytes;
+constexpr int kTmemCols = 2 * kBN;           // two fp32 accumulators of 128 lanes x kBN columns
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 static_assert(kBK * 2 == 128, "one swizzle row per tile row");
 static_assert(kDecodeWarps * 32 == 2 * kBN, "two decode threads per weight row");
 static_assert(kGemmThreads == 32 * (kDecodeWarps + 2), "warp roles");
+static_assert(kRecBytes % 16 == 0, "bulk copy size");
+static_assert((kTileABytes + kTileBBytes) % 1024 == 0, "operand tiles stay 1024-byte aligned");
 
-// Shared memory: the ring (1024-byte aligned tiles), then the barriers and tables.
+// Shared memory: the ring (activation and decoded weight tiles 1024-byte aligned, then the
+// weight records), then the barriers and the table.
 struct GemmShared {
-    uint64_t full_a[kRing];   // TMA bytes of the activation tile landed
-    uint64_t full_b[kRing];   // the decode warps wrote the weight tile
+    uint64_t full[kRing];     // activation tile and weight record landed (TMA bytes)
+    uint64_t decoded[kRing];  // the decode warps wrote the weight tile
     uint64_t empty[kRing];    // the MMAs that read the stage completed
     uint64_t accum;           // every MMA of the tile completed
     uint64_t drain;           // used only when stopping early
@@ -66,8 +74,9 @@ struct GemmShared {
     uint32_t abort;
     float sd[256];            // decode scale for every E4M3 byte: fl(E4M3(b) / gs)
 };
-constexpr int kRingBytes = kRing * (kTileABytes + kTileBBytes);
+constexpr int kRingBytes = kRing * kStageBytes;
 constexpr int kGemmSmemBytes = 1024 + kRingBytes + (int)sizeof(GemmShared);
+static_assert(kGemmSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 // ---------------------------------------------------------------------------------------
 // PTX wrappers.
@@ -126,7 +135,8 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// 2-D tiled TMA load of box {kBK, kBM} at (k, m) into shared memory, completing on `bar`.
+// 2-D tiled TMA load of the tensor map's box at (k, m) into shared memory, completing on
+// `bar`.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t k, int32_t m,
                                             uint32_t bar) {
     asm volatile(
@@ -134,6 +144,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
             dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(k), "r"(m), "r"(bar)
         : "memory");
+}
+
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from global to
+// shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
 }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
@@ -198,21 +216,62 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 // (bits 7-9 = 1, bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22,
 // M >> 4 in bits 24-28.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
-                            ((uint32_t)(kBM >> 4) << 24);
+                            ((uint32_t)(kMmaM >> 4) << 24);
+
 
 // ---------------------------------------------------------------------------------------
-// The kernel.  One CTA per 128 x 128 output tile; the tile index runs over output features
-// fastest, so CTAs resident together share their activation tile in L2.
+// Tile-major weight records (the operand form of a packed weight).
+//
+// Record (tn, tk) of a weight [N, K] sits at byte (tn * KT + tk) * 4608, KT = ceil(K / 64):
+//   bytes [0, 4096)     row r (0..127) of the tile at 32 r: the 32 code bytes of columns
+//                       64 tk .. 64 tk + 63 of weight row 128 tn + r (element 2j in the low
+//                       nibble of byte j, as in the plain layout)
+//   bytes [4096, 4608)  row r at 4096 + 4 r: the scale bytes of those columns' four blocks
+// Rows past N and columns past K hold code 0 and scale byte 0 (they decode to +0).
+
+__global__ void __launch_bounds__(256)
+    w4a16_pack_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales, int64_t N,
+                      int64_t K, int64_t KT, int64_t total_rows, uint8_t* __restrict__ tiled) {
+    const int64_t kblocks = K / kBlockElems;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total_rows;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i & (kBN - 1), rec = i >> 7;  // row in the tile, record index
+        const int64_t tn = rec / KT, tk = rec - tn * KT;
+        const int64_t n = tn * kBN + r;
+        uint32_t c[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        uint32_t sc = 0u;
+        if (n < N) {
+            const uint8_t* prow = packed + n * (K / 2);
+            const uint8_t* srow = scales + n * kblocks;
+#pragma unroll
+            for (int b = 0; b < kBK / kBlockElems; ++b) {
+                const int64_t blk = tk * (kBK / kBlockElems) + b;
+                if (blk < kblocks) {
+                    ld_b64_ro(prow + blk * kBlockBytesPacked, c[2 * b], c[2 * b + 1]);
+                    sc |= ld_u8_ro(srow + blk) << (8 * b);
+                }
+            }
+        }
+        uint8_t* dst = tiled + rec * kRecBytes;
+        st_b128(dst + r * 32, c[0], c[1], c[2], c[3]);
+        st_b128(dst + r * 32 + 16, c[4], c[5], c[6], c[7]);
+        *reinterpret_cast<uint32_t*>(dst + kRecCodes + r * 4) = sc;
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// The linear kernel.  One CTA per 256 x 128 output tile; the tile index runs over output
+// features fastest, so CTAs resident together share their activation tile in L2.
 
 struct LinearArgs {
-    const uint8_t* packed;  // [N, K/2] E2M1 codes (low nibble first)
-    const uint8_t* scales;  // [N, K/16] E4M3 bytes
+    const uint8_t* tiled;   // weight records
     const float* d_gs;      // encode global scale of the weight
     const uint16_t* bias;   // [N] bf16, or null
     uint8_t* y;             // [M, N] bf16
     Workspace* ws;
     int64_t M, N, K;
     int64_t tiles_n;
+    int64_t kt;             // records per weight row of tiles = ceil(K / 64)
     int vec_store;          // rows of y allow 16-byte stores
 };
 
@@ -228,19 +287,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* ring = dsmem + (base - raw);
     GemmShared& sh = *reinterpret_cast<GemmShared*>(ring + kRingBytes);
-    // stage s: activation tile at base + s * 16 KB, weight tile at base + (kRing + s) * 16 KB
-    const uint32_t sA0 = base, sB0 = base + kRing * kTileABytes;
+    // activation tiles, then decoded weight tiles (both 1024-byte aligned), then records
+    const uint32_t sA0 = base, sB0 = base + kRing * kTileABytes, sW0 = sB0 + kRing * kTileBBytes;
     uint8_t* gB0 = ring + kRing * kTileABytes;
+    const uint8_t* gW0 = gB0 + kRing * kTileBBytes;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t tm = (int64_t)blockIdx.x / a.tiles_n, tn = (int64_t)blockIdx.x % a.tiles_n;
     const int64_t m0 = tm * kBM, n0 = tn * kBN;
-    const int nk = (int)((a.K + kBK - 1) / kBK);
+    const int nk = (int)a.kt;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kRing; ++s) {
-            mbar_init(smem_u32(&sh.full_a[s]), 1);
-            mbar_init(smem_u32(&sh.full_b[s]), kDecodeWarps);
+            mbar_init(smem_u32(&sh.full[s]), 1);
+            mbar_init(smem_u32(&sh.decoded[s]), kDecodeWarps);
             mbar_init(smem_u32(&sh.empty[s]), 1);
         }
         mbar_init(smem_u32(&sh.accum), 1);
@@ -265,6 +325,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
+            const uint8_t* rec0 = a.tiled + tn * a.kt * kRecBytes;
             int issued = 0;
             for (int kb = 0; kb < nk; ++kb) {
                 const int s = kb % kRing;
@@ -273,14 +334,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     stop_all(sh, a.ws);
                     break;
                 }
-                mbar_arrive_expect_tx(smem_u32(&sh.full_a[s]), kTileABytes);
-                tma_load_2d(sA0 + s * kTileABytes, &tmap_x, kb * kBK, (int32_t)m0, smem_u32(&sh.full_a[s]));
+                const uint32_t bar = smem_u32(&sh.full[s]);
+                mbar_arrive_expect_tx(bar, kTileABytes + kRecBytes);
+                tma_load_2d(sA0 + s * kTileABytes, &tmap_x, kb * kBK, (int32_t)m0, bar);
+                bulk_load(sW0 + s * kRecBytes, rec0 + (int64_t)kb * kRecBytes, kRecBytes, bar);
                 ++issued;
             }
             // The copies in flight land before the CTA may exit (immediate when every
             // stage was consumed).
             for (int kb = issued > kRing ? issued - kRing : 0; kb < issued; ++kb)
-                if (!mbar_wait(smem_u32(&sh.full_a[kb % kRing]), (uint32_t)(kb / kRing) & 1u, abort, true))
+                if (!mbar_wait(smem_u32(&sh.full[kb % kRing]), (uint32_t)(kb / kRing) & 1u, abort, true))
                     stop_all(sh, a.ws);
         }
     } else if (warp == kMmaWarp) {
@@ -289,16 +352,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int kb = 0; kb < nk; ++kb) {
                 const int s = kb % kRing;
                 const uint32_t ph = (uint32_t)(kb / kRing) & 1u;
-                if (!mbar_wait(smem_u32(&sh.full_a[s]), ph, abort) || !mbar_wait(smem_u32(&sh.full_b[s]), ph, abort)) {
+                if (!mbar_wait(smem_u32(&sh.full[s]), ph, abort) || !mbar_wait(smem_u32(&sh.decoded[s]), ph, abort)) {
                     stop_all(sh, a.ws);
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint64_t ad = sw128_desc(sA0 + s * kTileABytes), bd = sw128_desc(sB0 + s * kTileBBytes);
+                const uint64_t bd = sw128_desc(sB0 + s * kTileBBytes);
+                const uint64_t ad0 = sw128_desc(sA0 + s * kTileABytes);
+                const uint64_t ad1 = sw128_desc(sA0 + s * kTileABytes + kMmaM * 128);
 #pragma unroll
-                for (int j = 0; j < kBK / kUmmaK; ++j)  // +32 bytes along K per step
-                    umma_f16(tmem, ad + 2u * j, bd + 2u * j, kIdesc, (kb | j) != 0 ? 1u : 0u);
+                for (int j = 0; j < kBK / kUmmaK; ++j) {  // +32 bytes along K per step
+                    const uint32_t acc = (kb | j) != 0 ? 1u : 0u;
+                    umma_f16(tmem, ad0 + 2u * j, bd + 2u * j, kIdesc, acc);
+                    umma_f16(tmem + kBN, ad1 + 2u * j, bd + 2u * j, kIdesc, acc);
+                }
                 umma_commit(smem_u32(&sh.empty[s]));
             }
             if (ok) {
@@ -310,87 +378,65 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
     } else {
-        // ---- decode warps: two threads per weight row, 32 elements (two blocks) each ----
+        // ---- decode warps: two threads per weight row, 32 columns (two blocks) each ----
+        // A stage's weight tile may be rewritten once its record has landed: the record's
+        // copy was issued only after the MMAs of the stage's previous use completed.
         const int t = threadIdx.x;
-        const int row = t & (kBN - 1);
-        const int half = t >> 7;
-        const int64_t n = n0 + row;
-        const bool row_ok = n < a.N;
-        const int64_t kblocks = a.K / kBlockElems;
-        const uint8_t* prow = a.packed + (row_ok ? n : 0) * (a.K / 2);
-        const uint8_t* srow = a.scales + (row_ok ? n : 0) * kblocks;
-
-        // codes of this thread's two blocks of stage kb (16 bytes) and their scale bytes;
-        // zeros past the row's end, past N, and past the last stage
-        auto load = [&](int kb, uint32_t (&c)[4], uint32_t& sc) {
-            c[0] = c[1] = c[2] = c[3] = 0u;
-            sc = 0u;
-            const int64_t b0 = (int64_t)kb * (kBK / kBlockElems) + 2 * half;
-            if (row_ok && kb < nk) {
-                if (b0 < kblocks) {
-                    ld_b64_ro(prow + b0 * kBlockBytesPacked, c[0], c[1]);
-                    sc = ld_u8_ro(srow + b0);
-                }
-                if (b0 + 1 < kblocks) {
-                    ld_b64_ro(prow + (b0 + 1) * kBlockBytesPacked, c[2], c[3]);
-                    sc |= ld_u8_ro(srow + b0 + 1) << 8;
-                }
-            }
-        };
-        uint32_t pc[kPrefetch][4], ps[kPrefetch];
-#pragma unroll
-        for (int u = 0; u < kPrefetch; ++u) load(u, pc[u], ps[u]);
-
+        const int row = t >> 1;
+        const int half = t & 1;
         bool ok = true;
-        for (int kb0 = 0; kb0 < nk && ok; kb0 += kPrefetch) {
-#pragma unroll
-            for (int u = 0; u < kPrefetch; ++u) {
-                const int kb = kb0 + u;
-                if (kb >= nk) break;
-                const int s = kb % kRing;
-                const uint32_t ph = (uint32_t)(kb / kRing) & 1u;
-                const bool got = mbar_wait(smem_u32(&sh.empty[s]), ph ^ 1u, abort);
-                if (!__all_sync(0xFFFFFFFFu, got)) {
-                    if (lane == 0) stop_all(sh, a.ws);
-                    ok = false;
-                    break;
-                }
-                uint8_t* tile_row = gB0 + s * kTileBBytes + row * 128;
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const float sd = sh.sd[(ps[u] >> (8 * i)) & 0xFFu];
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const uint32_t w = pc[u][2 * i + q];
-                        const uint32_t o0 = decode_pair(w & 0xFFu, sd), o1 = decode_pair((w >> 8) & 0xFFu, sd);
-                        const uint32_t o2 = decode_pair((w >> 16) & 0xFFu, sd), o3 = decode_pair(w >> 24, sd);
-                        const int chunk = 4 * half + 2 * i + q;  // 8 elements = 16 bytes
-                        const uint32_t dst = smem_u32(tile_row + ((chunk ^ (row & 7)) << 4));
-                        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(o0), "r"(o1), "r"(o2),
-                                     "r"(o3)
-                                     : "memory");
-                    }
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&sh.full_b[s]));
-                load(kb + kPrefetch, pc[u], ps[u]);
+        for (int kb = 0; kb < nk; ++kb) {
+            const int s = kb % kRing;
+            const uint32_t ph = (uint32_t)(kb / kRing) & 1u;
+            const bool got = mbar_wait(smem_u32(&sh.full[s]), ph, abort);
+            if (!__all_sync(0xFFFFFFFFu, got)) {
+                if (lane == 0) stop_all(sh, a.ws);
+                ok = false;
+                break;
             }
+            const uint8_t* rec = gW0 + s * kRecBytes;
+            uint32_t c[4];
+            {
+                const uint4 v = *reinterpret_cast<const uint4*>(rec + row * 32 + half * 16);
+                c[0] = v.x;
+                c[1] = v.y;
+                c[2] = v.z;
+                c[3] = v.w;
+            }
+            const uint32_t sc = *reinterpret_cast<const uint16_t*>(rec + kRecCodes + row * 4 + half * 2);
+            uint8_t* tile_row = gB0 + s * kTileBBytes + row * 128;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float sd = sh.sd[(sc >> (8 * i)) & 0xFFu];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const uint32_t w = c[2 * i + q];
+                    const uint32_t o0 = decode_pair(w & 0xFFu, sd), o1 = decode_pair((w >> 8) & 0xFFu, sd);
+                    const uint32_t o2 = decode_pair((w >> 16) & 0xFFu, sd), o3 = decode_pair(w >> 24, sd);
+                    const int chunk = 4 * half + 2 * i + q;  // 8 elements = 16 bytes
+                    const uint32_t dst = smem_u32(tile_row + ((chunk ^ (row & 7)) << 4));
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(o0), "r"(o1), "r"(o2), "r"(o3)
+                                 : "memory");
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sh.decoded[s]));
         }
 
-        // ---- epilogue: accumulator rows 32 * (warp % 4) + lane, 64 columns per warp ----
+        // ---- epilogue: warp w reads accumulator w / 4, lanes 32 * (w % 4) .. + 31 ----
         if (ok) {
             const bool got = mbar_wait(smem_u32(&sh.accum), 0u, abort);
             if (!__all_sync(0xFFFFFFFFu, got)) {
                 if (lane == 0) stop_all(sh, a.ws);
             } else {
                 tc_fence_after();
-                const int q = warp & 3, ch = warp >> 2;
-                const int64_t m = m0 + 32 * q + lane;
-                const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16);
+                const int q = warp & 3, acc = warp >> 2;
+                const int64_t m = m0 + kMmaM * acc + 32 * q + lane;
+                const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * kBN);
 #pragma unroll 1
-                for (int j = 0; j < 4; ++j) {
-                    const int col0 = ch * 64 + 16 * j;
+                for (int j = 0; j < kBN / 16; ++j) {
+                    const int col0 = 16 * j;
                     uint32_t v[16];
                     tmem_ld16(trow + (uint32_t)col0, v);
                     const int64_t nc = n0 + col0;
@@ -443,6 +489,7 @@ std::mutex g_w4_mu;
 EncodeTiledFn g_encode = nullptr;
 constexpr int kMaxDevs = 64;
 bool g_smem_set[kMaxDevs];
+int g_sms[kMaxDevs];
 
 nvfp4_status encode_fn(EncodeTiledFn* out) {
     std::lock_guard<std::mutex> lock(g_w4_mu);
@@ -471,27 +518,67 @@ nvfp4_status gemm_smem_optin() {
     return NVFP4_OK;
 }
 
+nvfp4_status sm_count_w4(int* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevs) return NVFP4_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_w4_mu);
+    if (g_sms[dev] == 0 && cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    *out = g_sms[dev];
+    return NVFP4_OK;
+}
+
 bool is_aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Shapes the operand records accept: K a positive multiple of 16, sizes whose byte offsets
+// and TMA coordinates stay in range.
+bool weight_shape_ok(int64_t N, int64_t K) {
+    return N >= 0 && K > 0 && K % kBlockElems == 0 && K <= 0x7FFFFF00ll && N <= ((int64_t)1 << 40);
+}
+
+int64_t record_bytes(int64_t N, int64_t K) {
+    return ((N + kBN - 1) / kBN) * ((K + kBK - 1) / kBK) * (int64_t)kRecBytes;
+}
 
 }  // namespace
 }  // namespace nvfp4
 
 using namespace nvfp4;
 
-NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* packed,
-                                          const uint8_t* scales, const float* d_global_scale, int64_t N,
-                                          const void* bias, void* y, void* d_workspace, nvfp4_stream_t stream) {
-    if (M < 0 || N < 0 || K <= 0 || K % kBlockElems != 0) return NVFP4_ERR_SHAPE;
-    // TMA coordinates are 32-bit; the grid is one CTA per output tile.
-    if (M > 0x7FFFFF00ll || K > 0x7FFFFF00ll || N > ((int64_t)1 << 40)) return NVFP4_ERR_SHAPE;
+NVFP4_API int64_t nvfp4_w4a16_tiled_bytes(int64_t N, int64_t K) {
+    return weight_shape_ok(N, K) ? record_bytes(N, K) : -1;
+}
+
+NVFP4_API nvfp4_status nvfp4_w4a16_pack(const uint8_t* packed, const uint8_t* scales, int64_t N, int64_t K,
+                                        uint8_t* tiled, nvfp4_stream_t stream) {
+    if (!weight_shape_ok(N, K)) return NVFP4_ERR_SHAPE;
+    if (N == 0) return NVFP4_OK;
+    if (packed == nullptr || scales == nullptr || tiled == nullptr) return NVFP4_ERR_NULL;
+    if (!is_aligned(packed, 8) || !is_aligned(tiled, 16)) return NVFP4_ERR_ALIGN;
+    const int64_t KT = (K + kBK - 1) / kBK;
+    const int64_t rows = ((N + kBN - 1) / kBN) * KT * kBN;  // one thread per record row
+    int sms = 0;
+    nvfp4_status st = sm_count_w4(&sms);
+    if (st != NVFP4_OK) return st;
+    int64_t grid = (rows + 255) / 256;
+    if (grid > (int64_t)sms * 32) grid = (int64_t)sms * 32;
+    w4a16_pack_kernel<<<(unsigned)grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(packed, scales, N, K, KT,
+                                                                                          rows, tiled);
+    note_launch();
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* tiled,
+                                          const float* d_global_scale, int64_t N, const void* bias, void* y,
+                                          void* d_workspace, nvfp4_stream_t stream) {
+    if (M < 0 || !weight_shape_ok(N, K) || M > 0x7FFFFF00ll) return NVFP4_ERR_SHAPE;
     const int64_t tiles_m = (M + kBM - 1) / kBM, tiles_n = (N + kBN - 1) / kBN;
     if (tiles_m * tiles_n > 0x7FFFFFFFll) return NVFP4_ERR_SHAPE;
     if (d_global_scale == nullptr || d_workspace == nullptr) return NVFP4_ERR_NULL;
-    if (M > 0 && N > 0 && (x == nullptr || packed == nullptr || scales == nullptr || y == nullptr))
-        return NVFP4_ERR_NULL;
+    if (M > 0 && N > 0 && (x == nullptr || tiled == nullptr || y == nullptr)) return NVFP4_ERR_NULL;
     if (!is_aligned(d_global_scale, 4) || !is_aligned(d_workspace, 16)) return NVFP4_ERR_ALIGN;
     if (M > 0 && N > 0 &&
-        (!is_aligned(x, 16) || !is_aligned(packed, 8) || !is_aligned(y, 2) || (bias && !is_aligned(bias, 2))))
+        (!is_aligned(x, 16) || !is_aligned(tiled, 16) || !is_aligned(y, 2) || (bias && !is_aligned(bias, 2))))
         return NVFP4_ERR_ALIGN;
     if (M == 0 || N == 0) return NVFP4_OK;
 
@@ -501,7 +588,7 @@ NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, c
     st = gemm_smem_optin();
     if (st != NVFP4_OK) return st;
 
-    // x as a [M, K] bf16 tensor, boxes of 128 rows x 64 columns, 128-byte swizzle, zero
+    // x as a [M, K] bf16 tensor, boxes of 256 rows x 64 columns, 128-byte swizzle, zero
     // fill past either edge.
     CUtensorMap map;
     std::memset(&map, 0, sizeof(map));
@@ -515,8 +602,7 @@ NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, c
         return NVFP4_ERR_ARG;
 
     LinearArgs a;
-    a.packed = packed;
-    a.scales = scales;
+    a.tiled = tiled;
     a.d_gs = d_global_scale;
     a.bias = static_cast<const uint16_t*>(bias);
     a.y = static_cast<uint8_t*>(y);
@@ -525,6 +611,7 @@ NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, c
     a.N = N;
     a.K = K;
     a.tiles_n = tiles_n;
+    a.kt = (K + kBK - 1) / kBK;
     a.vec_store = (is_aligned(y, 16) && N % 8 == 0) ? 1 : 0;
     w4a16_linear_kernel<<<(unsigned)(tiles_m * tiles_n), kGemmThreads, kGemmSmemBytes,
                           reinterpret_cast<cudaStream_t>(stream)>>>(map, a);

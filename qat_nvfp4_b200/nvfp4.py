@@ -68,7 +68,9 @@ _c_fake_quant_bs = _sig("nvfp4_fake_quant_bs", [_vp, _vp, _i64, _i64, ctypes.c_i
 _c_fake_quant_siblings = _sig("nvfp4_fake_quant_siblings",
                               [ctypes.c_int, ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_i64),
                                ctypes.POINTER(_i64), _vp, _vp])
-_c_w4a16_linear = _sig("nvfp4_w4a16_linear", [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp])
+_c_w4a16_tiled_bytes = _sig("nvfp4_w4a16_tiled_bytes", [_i64, _i64], _i64)
+_c_w4a16_pack = _sig("nvfp4_w4a16_pack", [_vp, _vp, _i64, _i64, _vp, _vp])
+_c_w4a16_linear = _sig("nvfp4_w4a16_linear", [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _vp])
 _c_status_string = _sig("nvfp4_status_string", [ctypes.c_int], ctypes.c_char_p)
 _c_launch_count = _sig("nvfp4_kernel_launch_count", [], ctypes.c_uint64)
 
@@ -434,26 +436,52 @@ def nvfp4_selftest_barrier_timeout(x: torch.Tensor, workspace: torch.Tensor, tim
                                                workspace.data_ptr(), int(timeout_us), _stream(x.device)))
 
 
-def nvfp4_w4a16_linear(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, global_scale: torch.Tensor,
-                       bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
-                       workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """Forward of a Linear layer on an NVFP4-packed weight: x [..., K] bf16 times the
-    weight that (packed [N, K/2], scales [N, K/16], global_scale) encode, transposed, plus
-    bias [N] -> bf16 [..., N].  The weight is decoded inside the tensor-core kernel and is
-    never materialised in device memory."""
-    M, K = _matrix(x)
+def nvfp4_w4a16_tiled_bytes(N: int, K: int) -> int:
+    """Bytes of the operand form of an [N, K] packed weight (-1 if the shape is refused)."""
+    return int(_c_w4a16_tiled_bytes(N, K))
+
+
+def nvfp4_w4a16_pack(packed: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Packed weight (packed [N, K/2], scales [N, K/16]) -> its operand form for
+    nvfp4_w4a16_linear: one 4608-byte record per 128 x 64 tile (uint8, 1-D)."""
     _cuda(packed, "packed", torch.uint8)
     _cuda(scales, "scales", torch.uint8)
-    _scalar(global_scale, "global_scale")
-    if packed.dim() != 2 or packed.shape[1] * 2 != K:
-        raise RuntimeError(f"packed must be [N, K/2] with K = {K}")
-    N = packed.shape[0]
+    if packed.dim() != 2:
+        raise RuntimeError("packed must be [N, K/2]")
+    N, K = packed.shape[0], packed.shape[1] * 2
     if scales.numel() != N * (K // 16):
         raise RuntimeError("scales has the wrong number of elements")
+    nbytes = nvfp4_w4a16_tiled_bytes(N, K)
+    if nbytes < 0:
+        raise RuntimeError(f"weight shape ({N}, {K}) not accepted (K must be a positive multiple of 16)")
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=packed.device)
+    _cuda(out, "out", torch.uint8)
+    if out.numel() != nbytes:
+        raise RuntimeError(f"out must hold {nbytes} bytes")
+    with torch.cuda.device(packed.device):
+        _check(_c_w4a16_pack(packed.data_ptr(), scales.data_ptr(), N, K, out.data_ptr(), _stream(packed.device)),
+               "nvfp4_w4a16_pack")
+    return out
+
+
+def nvfp4_w4a16_linear(x: torch.Tensor, tiled: torch.Tensor, global_scale: torch.Tensor, n_out: int,
+                       bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                       workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Forward of a Linear layer on an NVFP4 weight [n_out, K] in operand form (tiled, from
+    nvfp4_w4a16_pack) with its encode global scale: x [..., K] bf16 -> bf16 [..., n_out] =
+    x W^T + bias.  The weight is decoded inside the tensor-core kernel and is never
+    materialised in device memory."""
+    M, K = _matrix(x)
+    _cuda(tiled, "tiled", torch.uint8)
+    _scalar(global_scale, "global_scale")
+    N = int(n_out)
+    if tiled.numel() != nvfp4_w4a16_tiled_bytes(N, K):
+        raise RuntimeError(f"tiled does not hold a [{N}, {K}] weight")
     if bias is not None:
         _cuda(bias, "bias", torch.bfloat16)
         if bias.numel() != N:
-            raise RuntimeError("bias must have N elements")
+            raise RuntimeError("bias must have n_out elements")
     if out is None:
         out = torch.empty(tuple(x.shape[:-1]) + (N,), dtype=torch.bfloat16, device=x.device)
     _cuda(out, "out", torch.bfloat16)
@@ -461,7 +489,7 @@ def nvfp4_w4a16_linear(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tens
         raise RuntimeError("out has the wrong number of elements")
     ws = new_workspace(x.device) if workspace is None else _workspace(workspace, x.device)
     with torch.cuda.device(x.device):
-        _check(_c_w4a16_linear(x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(), global_scale.data_ptr(), N,
+        _check(_c_w4a16_linear(x.data_ptr(), M, K, tiled.data_ptr(), global_scale.data_ptr(), N,
                                bias.data_ptr() if bias is not None else None, out.data_ptr(), ws.data_ptr(),
                                _stream(x.device)), "nvfp4_w4a16_linear")
     return out

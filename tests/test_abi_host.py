@@ -32,6 +32,7 @@ def test_header_declares_the_entry_points():
     for required in ["nvfp4_amax", "nvfp4_amax_multi", "nvfp4_observer_update", "nvfp4_observe_amax",
                      "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fake_quant", "nvfp4_fake_quant_siblings",
                      "nvfp4_quantize_bs", "nvfp4_dequantize_bs", "nvfp4_fake_quant_bs", "nvfp4_w4a16_linear",
+                     "nvfp4_w4a16_pack", "nvfp4_w4a16_tiled_bytes",
                      "nvfp4_status_string", "nvfp4_kernel_launch_count"]:
         assert required in names
 
@@ -126,22 +127,19 @@ def test_validation_errors_launch_nothing(lib):
         (ERR_SHAPE, "nvfp4_quantize_bs", _p(A32), _i(1 << 56), _i(33), _c(32), amax, _p(A32), _p(A32), gs, S),
         (ERR_SHAPE, "nvfp4_fake_quant_bs", _p(A32), _p(A32 + 4096), _i(2), _i(-32), _c(32), amax, S),
         (ERR_NULL, "nvfp4_fake_quant_bs", _p(A32), _p(A32 + 4096), _i(2), _i(64), _c(32), _p(0), S),
-        # W4A16 linear: x, M, K, packed, scales, gs, N, bias, y, workspace
-        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(24), _p(A32), _p(A32), gs, _i(8), _p(0), _p(A32),
-         _p(A32), S),
-        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(0), _p(A32), _p(A32), gs, _i(8), _p(0), _p(A32),
-         _p(A32), S),
-        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(-1), _i(64), _p(A32), _p(A32), gs, _i(8), _p(0), _p(A32),
-         _p(A32), S),
-        (ERR_NULL, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(A32), _p(A32), gs, _i(8), _p(0), _p(A32),
-         _p(0), S),
-        (ERR_NULL, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(0), _p(A32), gs, _i(8), _p(0), _p(A32),
-         _p(A32), S),
-        (ERR_ALIGN, "nvfp4_w4a16_linear", _p(A8), _i(4), _i(64), _p(A32), _p(A32), gs, _i(8), _p(0), _p(A32),
-         _p(A32), S),
-        (ERR_ALIGN, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(A32 + 4), _p(A32), gs, _i(8), _p(0), _p(A32),
-         _p(A32), S),
-        (NVFP4_OK, "nvfp4_w4a16_linear", _p(0), _i(0), _i(64), _p(0), _p(0), gs, _i(8), _p(0), _p(0), _p(A32), S),
+        # W4A16: linear(x, M, K, tiled, gs, N, bias, y, workspace), pack(packed, scales, N, K, tiled)
+        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(24), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), S),
+        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(0), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), S),
+        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(-1), _i(64), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), S),
+        (ERR_NULL, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(A32), gs, _i(8), _p(0), _p(A32), _p(0), S),
+        (ERR_NULL, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(0), gs, _i(8), _p(0), _p(A32), _p(A32), S),
+        (ERR_ALIGN, "nvfp4_w4a16_linear", _p(A8), _i(4), _i(64), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), S),
+        (ERR_ALIGN, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(A8), gs, _i(8), _p(0), _p(A32), _p(A32), S),
+        (NVFP4_OK, "nvfp4_w4a16_linear", _p(0), _i(0), _i(64), _p(0), gs, _i(8), _p(0), _p(0), _p(A32), S),
+        (ERR_SHAPE, "nvfp4_w4a16_pack", _p(A32), _p(A32), _i(8), _i(40), _p(A32), S),
+        (ERR_NULL, "nvfp4_w4a16_pack", _p(A32), _p(0), _i(8), _i(64), _p(A32), S),
+        (ERR_ALIGN, "nvfp4_w4a16_pack", _p(A32), _p(A32), _i(8), _i(64), _p(A8), S),
+        (NVFP4_OK, "nvfp4_w4a16_pack", _p(0), _p(0), _i(0), _i(64), _p(0), S),
         # amax
         (ERR_NULL, "nvfp4_amax", _p(A32), _i(16), _p(0), S),
         (ERR_NULL, "nvfp4_amax", _p(0), _i(16), amax, S),
@@ -219,3 +217,14 @@ def test_binding_refuses_cpu_tensors():
         with pytest.raises(RuntimeError, match="CUDA tensor"):
             call()
 
+
+
+def test_w4a16_record_sizes(lib):
+    """Host-only: ceil(N / 128) * ceil(K / 64) records of 4608 bytes; refused shapes -> -1."""
+    f = lib.nvfp4_w4a16_tiled_bytes
+    f.restype = ctypes.c_int64
+    f.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    for N, K in [(1, 16), (128, 64), (129, 64), (128, 65 - 1 + 16), (14336, 4096), (0, 16)]:
+        assert f(N, K) == -(-N // 128) * -(-K // 64) * 4608
+    for N, K in [(8, 0), (8, 24), (-1, 64), (8, -16)]:
+        assert f(N, K) == -1

@@ -35,6 +35,38 @@ def _weight(n_out, K, seed, std=0.02):
     return packed, scales, gs
 
 
+def _records_from_definition(pk, sc, N, K):
+    """The operand form written out from its definition: record (tn, tk) holds rows
+    128 tn .. + 127, columns 64 tk .. + 63; codes row-major 32 bytes a row, then the 4
+    scale bytes of each row; zeros past N and K."""
+    NT, KT = -(-N // 128), -(-K // 64)
+    codes = np.zeros((NT * 128, KT * 32), dtype=np.uint8)
+    codes[:N, :K // 2] = pk
+    scl = np.zeros((NT * 128, KT * 4), dtype=np.uint8)
+    scl[:N, :K // 16] = sc
+    out = np.empty((NT, KT, 4608), dtype=np.uint8)
+    for tn in range(NT):
+        for tk in range(KT):
+            rows = slice(128 * tn, 128 * tn + 128)
+            out[tn, tk, :4096] = codes[rows, 32 * tk:32 * tk + 32].reshape(-1)
+            out[tn, tk, 4096:] = scl[rows, 4 * tk:4 * tk + 4].reshape(-1)
+    return out.reshape(-1)
+
+
+def _linear(x, packed, scales, gs, **kw):
+    tiled = nv.nvfp4_w4a16_pack(packed, scales)
+    return nv.nvfp4_w4a16_linear(x, tiled, gs, packed.shape[0], **kw)
+
+
+@pytest.mark.parametrize("N,K", [(128, 64), (300, 1040), (13, 16), (1000, 4096)])
+def test_pack_matches_the_record_layout(N, K):
+    packed, scales, gs = _weight(N, K, N + K)
+    tiled = nv.nvfp4_w4a16_pack(packed, scales)
+    assert tiled.numel() == nv.nvfp4_w4a16_tiled_bytes(N, K) == -(-N // 128) * -(-K // 64) * 4608
+    want = _records_from_definition(u8(packed), u8(scales), N, K)
+    assert np.array_equal(u8(tiled), want)
+
+
 def _assert_within_bound(y_bits, x_bits, packed, scales, gs, bias_bits, what):
     """y_bits: uint16 [R, N] for the activation rows x_bits [R, K]."""
     pk, sc = u8(packed), u8(scales)
@@ -55,7 +87,9 @@ def _assert_within_bound(y_bits, x_bits, packed, scales, gs, bias_bits, what):
 
 
 @pytest.mark.parametrize("M,K,N,with_bias", [
-    (128, 64, 128, False),     # one tile, one stage
+    (128, 64, 128, False),     # one stage; rows 128-255 of the tile are past M
+    (256, 128, 256, False),    # both accumulators of one tile full
+    (700, 512, 384, True),     # three row tiles, the last ragged
     (128, 1024, 256, True),    # 16 stages, two output tiles
     (300, 1040, 200, True),    # ragged M, N and K (K % 64 == 16)
     (37, 48, 24, False),       # K below one stage
@@ -69,8 +103,7 @@ def test_linear_matches_oracle(M, K, N, with_bias):
     packed, scales, gs = _weight(N, K, M + K + N)
     bias = synthetic.to_bf16_bits(rng.standard_normal(N).astype(np.float32)) if with_bias else None
     ws = nv.new_workspace("cuda")
-    y = nv.nvfp4_w4a16_linear(to_dev(x), packed, scales, gs, bias=to_dev(bias) if with_bias else None,
-                              workspace=ws)
+    y = _linear(to_dev(x), packed, scales, gs, bias=to_dev(bias) if with_bias else None, workspace=ws)
     torch.cuda.synchronize()
     assert nv.nvfp4_workspace_check(ws) == 0
     assert tuple(y.shape) == (M, N)
@@ -86,7 +119,7 @@ def test_linear_agrees_with_a_library_gemm_on_the_dequantized_weight():
     x = to_dev(synthetic.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32)))
     packed, scales, gs = _weight(N, K, 6)
     bias = to_dev(synthetic.to_bf16_bits(rng.standard_normal(N).astype(np.float32)))
-    ours = nv.nvfp4_w4a16_linear(x, packed, scales, gs, bias=bias)
+    ours = _linear(x, packed, scales, gs, bias=bias)
     w = nv.nvfp4_dequantize(packed, scales, gs)
     ref = torch.nn.functional.linear(x, w, bias)
     rows = sample_rows(M, 32, seed=1)
@@ -103,7 +136,7 @@ def test_mlp_weight_4096_tokens_sampled_rows():
     x = synthetic.activation_normal_device((M, K), 31, "cuda")
     w = synthetic.activation_normal_device((N, K), 32, "cuda") * 0.02
     packed, scales, gs = nv.nvfp4_quantize(w, nv.nvfp4_amax(w))
-    y = nv.nvfp4_w4a16_linear(x, packed, scales, gs)
+    y = _linear(x, packed, scales, gs)
     rows = sample_rows(M, 24, seed=3)
     _assert_within_bound(bits(y)[rows], bits(x)[rows], packed, scales, gs, None, "MLP 4096 tokens")
 
@@ -113,7 +146,7 @@ def test_out_parameter_and_leading_dimensions():
     x = to_dev(synthetic.to_bf16_bits(rng.standard_normal((2, 3, 256)).astype(np.float32)))
     packed, scales, gs = _weight(64, 256, 10)
     out = torch.full((2, 3, 64), 7.0, dtype=torch.bfloat16, device="cuda")
-    y = nv.nvfp4_w4a16_linear(x, packed, scales, gs, out=out)
+    y = _linear(x, packed, scales, gs, out=out)
     assert y.data_ptr() == out.data_ptr()
     _assert_within_bound(bits(y).reshape(6, 64), bits(x).reshape(6, 256), packed, scales, gs, None, "3-D x")
 
@@ -121,7 +154,8 @@ def test_out_parameter_and_leading_dimensions():
 def test_empty_rows_launch_nothing():
     packed, scales, gs = _weight(32, 64, 11)
     x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    tiled = nv.nvfp4_w4a16_pack(packed, scales)
     before = nv.nvfp4_kernel_launch_count()
-    y = nv.nvfp4_w4a16_linear(x, packed, scales, gs, workspace=nv.new_workspace("cuda"))
+    y = nv.nvfp4_w4a16_linear(x, tiled, gs, 32, workspace=nv.new_workspace("cuda"))
     assert tuple(y.shape) == (0, 32)
     assert nv.nvfp4_kernel_launch_count() == before
