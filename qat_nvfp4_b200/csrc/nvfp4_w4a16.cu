@@ -13,9 +13,13 @@
 // nvfp4_dequantize, bf16_rn(fl(LUT[code] * fl(E4M3(byte) / gs))).  A CTA computes a
 // 256 x 128 output tile as two 128 x 128 accumulators that share each decoded weight tile.
 //
-//   warps 0-7  decode weight tiles into the ring, then the epilogue (TMEM -> bf16 -> y)
-//   warp 8     TMA load of the activation tile + bulk copy of the weight record per stage
-//   warp 9     TMEM allocation, MMA issue (one elected thread), TMEM release
+//   warps 0-15 decode weight records into weight tiles (one 16-element block per thread and
+//              stage), then the epilogue (TMEM -> bf16 -> y)
+//   warp 16    TMA loads of activation tiles (ring of 4)
+//   warp 17    TMEM allocation, MMA issue (one elected thread), TMEM release
+//   warp 18    bulk copies of weight records (ring of 8, running ahead of the activations)
+// Decoded weight tiles pass from the decode warps to the MMAs through a ring of 3, so the
+// decode of a stage overlaps the MMAs of the stages before it.
 //
 // Every wait on an mbarrier is bounded (kWaitLimitNs of %globaltimer); a wait that runs
 // out records NVFP4_ERR_TIMEOUT in the caller's workspace, tells the other roles to stop,
@@ -40,41 +44,49 @@ namespace {
 
 constexpr int kBM = 256;                  // rows of x per tile: two MMAs of M = 128
 constexpr int kMmaM = 128;
-constexpr int kBN = 128;                  // weight rows (output features) per tile (MMA N)
+constexpr int kBN = 256;                  // weight rows (output features) per tile (MMA N)
+constexpr int kRecRows = 128;             // weight rows per record
 constexpr int kBK = 64;                   // K per stage: 64 bf16 = one 128-byte swizzle row
 constexpr int kUmmaK = 16;                // K of one kind::f16 MMA
-constexpr int kRing = 4;                  // stages in the shared-memory ring
-constexpr int kDecodeWarps = 8;
-constexpr int kTmaWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kGemmThreads = 320;
+constexpr int kRingA = 3;                 // activation tiles in flight
+constexpr int kRingW = 4;                 // weight-record pairs in flight
+constexpr int kRingB = 2;                 // decoded weight tiles between the decode warps and the MMAs
+constexpr int kDecodeWarps = 16;
+constexpr int kTmaWarp = 16;              // activation loads
+constexpr int kMmaWarp = 17;
+constexpr int kRecWarp = 18;              // weight-record loads
+constexpr int kGemmThreads = 608;
 constexpr int kTileABytes = kBM * kBK * 2;   // 32 KB
-constexpr int kTileBBytes = kBN * kBK * 2;   // 16 KB
-constexpr int kRecCodes = kBN * kBK / 2;     // 4096 bytes of E2M1 codes per weight tile
-constexpr int kRecBytes = kRecCodes + kBN * (kBK / kBlockElems);  // + 512 scale bytes = 4608
-constexpr int kStageBytes = kTileABytes + kTileBBytes + kRecBytes;
-constexpr int kTmemCols = 2 * kBN;           // two fp32 accumulators of 128 lanes x kBN columns
+constexpr int kTileBBytes = kBN * kBK * 2;   // 32 KB
+constexpr int kRecCodes = kRecRows * kBK / 2;  // 4096 bytes of E2M1 codes per record
+constexpr int kRecBytes = kRecCodes + kRecRows * (kBK / kBlockElems);  // + 512 scale bytes = 4608
+constexpr int kRecPerTile = kBN / kRecRows;    // records per stage
+constexpr int kTmemCols = 2 * kBN;           // two fp32 accumulators of 128 lanes x kBN columns: all 512
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 static_assert(kBK * 2 == 128, "one swizzle row per tile row");
 static_assert(kDecodeWarps * 32 == 2 * kBN, "two decode threads per weight row");
-static_assert(kGemmThreads == 32 * (kDecodeWarps + 2), "warp roles");
+static_assert(kTmemCols <= 512, "tensor memory columns");
+static_assert(kGemmThreads == 32 * (kDecodeWarps + 3), "warp roles");
 static_assert(kRecBytes % 16 == 0, "bulk copy size");
-static_assert((kTileABytes + kTileBBytes) % 1024 == 0, "operand tiles stay 1024-byte aligned");
+static_assert(kTileABytes % 1024 == 0 && kTileBBytes % 1024 == 0, "operand tiles stay 1024-byte aligned");
 
-// Shared memory: the ring (activation and decoded weight tiles 1024-byte aligned, then the
-// weight records), then the barriers and the table.
+// Shared memory: activation tiles, decoded weight tiles (both 1024-byte aligned), weight
+// records, then the barriers and the table.
 struct GemmShared {
-    uint64_t full[kRing];     // activation tile and weight record landed (TMA bytes)
-    uint64_t decoded[kRing];  // the decode warps wrote the weight tile
-    uint64_t empty[kRing];    // the MMAs that read the stage completed
-    uint64_t accum;           // every MMA of the tile completed
-    uint64_t drain;           // used only when stopping early
+    uint64_t a_full[kRingA];   // activation tile landed (TMA bytes)
+    uint64_t a_empty[kRingA];  // the MMAs that read it completed
+    uint64_t w_full[kRingW];   // weight records landed (bulk-copy bytes)
+    uint64_t w_empty[kRingW];  // the decode warps have read it
+    uint64_t b_full[kRingB];   // the decode warps wrote the weight tile
+    uint64_t b_empty[kRingB];  // the MMAs that read it completed
+    uint64_t accum;            // every MMA of the tile completed
+    uint64_t drain;            // used only when stopping early
     uint32_t tmem_base;
     uint32_t abort;
-    float sd[256];            // decode scale for every E4M3 byte: fl(E4M3(b) / gs)
+    float sd[256];             // decode scale for every E4M3 byte: fl(E4M3(b) / gs)
 };
-constexpr int kRingBytes = kRing * kStageBytes;
+constexpr int kRingBytes = kRingA * kTileABytes + kRingB * kTileBBytes + kRingW * kRecPerTile * kRecBytes;
 constexpr int kGemmSmemBytes = 1024 + kRingBytes + (int)sizeof(GemmShared);
 static_assert(kGemmSmemBytes <= 227 * 1024, "shared memory per CTA");
 
@@ -235,9 +247,9 @@ __global__ void __launch_bounds__(256)
     const int64_t kblocks = K / kBlockElems;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total_rows;
          i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i & (kBN - 1), rec = i >> 7;  // row in the tile, record index
+        const int64_t r = i % kRecRows, rec = i / kRecRows;  // row in the record, record index
         const int64_t tn = rec / KT, tk = rec - tn * KT;
-        const int64_t n = tn * kBN + r;
+        const int64_t n = tn * kRecRows + r;
         uint32_t c[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
         uint32_t sc = 0u;
         if (n < N) {
@@ -280,6 +292,12 @@ __device__ __forceinline__ void stop_all(GemmShared& sh, Workspace* ws) {
     atomicExch(&ws->error, (unsigned)NVFP4_ERR_TIMEOUT);
 }
 
+// Wait on `bar` from every lane of a warp; true in all lanes only if every lane saw it.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const volatile uint32_t* abort) {
+    const bool got = mbar_wait(bar, parity, abort);
+    return __all_sync(0xFFFFFFFFu, got);
+}
+
 __global__ void __launch_bounds__(kGemmThreads, 1)
     w4a16_linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const LinearArgs a) {
     extern __shared__ uint8_t dsmem[];
@@ -287,10 +305,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* ring = dsmem + (base - raw);
     GemmShared& sh = *reinterpret_cast<GemmShared*>(ring + kRingBytes);
-    // activation tiles, then decoded weight tiles (both 1024-byte aligned), then records
-    const uint32_t sA0 = base, sB0 = base + kRing * kTileABytes, sW0 = sB0 + kRing * kTileBBytes;
-    uint8_t* gB0 = ring + kRing * kTileABytes;
-    const uint8_t* gW0 = gB0 + kRing * kTileBBytes;
+    const uint32_t sA0 = base;
+    const uint32_t sB0 = sA0 + kRingA * kTileABytes;
+    const uint32_t sW0 = sB0 + kRingB * kTileBBytes;
+    uint8_t* gB0 = ring + kRingA * kTileABytes;
+    const uint8_t* gW0 = gB0 + kRingB * kTileBBytes;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t tm = (int64_t)blockIdx.x / a.tiles_n, tn = (int64_t)blockIdx.x % a.tiles_n;
@@ -298,10 +317,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int nk = (int)a.kt;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kRing; ++s) {
-            mbar_init(smem_u32(&sh.full[s]), 1);
-            mbar_init(smem_u32(&sh.decoded[s]), kDecodeWarps);
-            mbar_init(smem_u32(&sh.empty[s]), 1);
+        for (int s = 0; s < kRingA; ++s) {
+            mbar_init(smem_u32(&sh.a_full[s]), 1);
+            mbar_init(smem_u32(&sh.a_empty[s]), 1);
+        }
+        for (int s = 0; s < kRingW; ++s) {
+            mbar_init(smem_u32(&sh.w_full[s]), 1);
+            mbar_init(smem_u32(&sh.w_empty[s]), kDecodeWarps);
+        }
+        for (int s = 0; s < kRingB; ++s) {
+            mbar_init(smem_u32(&sh.b_full[s]), kDecodeWarps);
+            mbar_init(smem_u32(&sh.b_empty[s]), 1);
         }
         mbar_init(smem_u32(&sh.accum), 1);
         mbar_init(smem_u32(&sh.drain), 1);
@@ -323,51 +349,69 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tmem = sh.tmem_base;
     const volatile uint32_t* abort = &sh.abort;
 
-    if (warp == kTmaWarp) {
+    if (warp == kTmaWarp || warp == kRecWarp) {
+        // ---- producers: activation tiles (TMA) or weight records (bulk copy) ----
         if (lane == 0) {
-            const uint8_t* rec0 = a.tiled + tn * a.kt * kRecBytes;
+            const bool act = warp == kTmaWarp;
+            const int R = act ? kRingA : kRingW;
+            const uint64_t* full = act ? sh.a_full : sh.w_full;
+            const uint64_t* empty = act ? sh.a_empty : sh.w_empty;
+            // the tile's weight rows are records (kRecPerTile * tn + i, kb); rows past the
+            // last record of the weight (N not a multiple of 256) read the last record again
+            // and are dropped by the epilogue
+            const int64_t nrec = (a.N + kRecRows - 1) / kRecRows;
             int issued = 0;
             for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % kRing;
-                const uint32_t ph = (uint32_t)(kb / kRing) & 1u;
-                if (!mbar_wait(smem_u32(&sh.empty[s]), ph ^ 1u, abort)) {
+                const int s = kb % R;
+                const uint32_t ph = (uint32_t)(kb / R) & 1u;
+                if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, abort)) {
                     stop_all(sh, a.ws);
                     break;
                 }
-                const uint32_t bar = smem_u32(&sh.full[s]);
-                mbar_arrive_expect_tx(bar, kTileABytes + kRecBytes);
-                tma_load_2d(sA0 + s * kTileABytes, &tmap_x, kb * kBK, (int32_t)m0, bar);
-                bulk_load(sW0 + s * kRecBytes, rec0 + (int64_t)kb * kRecBytes, kRecBytes, bar);
+                const uint32_t bar = smem_u32(&full[s]);
+                if (act) {
+                    mbar_arrive_expect_tx(bar, kTileABytes);
+                    tma_load_2d(sA0 + s * kTileABytes, &tmap_x, kb * kBK, (int32_t)m0, bar);
+                } else {
+                    mbar_arrive_expect_tx(bar, kRecPerTile * kRecBytes);
+#pragma unroll
+                    for (int i = 0; i < kRecPerTile; ++i) {
+                        int64_t rn = kRecPerTile * tn + i;
+                        if (rn >= nrec) rn = nrec - 1;
+                        bulk_load(sW0 + (s * kRecPerTile + i) * kRecBytes, a.tiled + (rn * a.kt + kb) * kRecBytes,
+                                  kRecBytes, bar);
+                    }
+                }
                 ++issued;
             }
             // The copies in flight land before the CTA may exit (immediate when every
             // stage was consumed).
-            for (int kb = issued > kRing ? issued - kRing : 0; kb < issued; ++kb)
-                if (!mbar_wait(smem_u32(&sh.full[kb % kRing]), (uint32_t)(kb / kRing) & 1u, abort, true))
-                    stop_all(sh, a.ws);
+            for (int kb = issued > R ? issued - R : 0; kb < issued; ++kb)
+                if (!mbar_wait(smem_u32(&full[kb % R]), (uint32_t)(kb / R) & 1u, abort, true)) stop_all(sh, a.ws);
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
             bool ok = true;
             for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % kRing;
-                const uint32_t ph = (uint32_t)(kb / kRing) & 1u;
-                if (!mbar_wait(smem_u32(&sh.full[s]), ph, abort) || !mbar_wait(smem_u32(&sh.decoded[s]), ph, abort)) {
+                const int sa = kb % kRingA, sb = kb % kRingB;
+                if (!mbar_wait(smem_u32(&sh.a_full[sa]), (uint32_t)(kb / kRingA) & 1u, abort) ||
+                    !mbar_wait(smem_u32(&sh.b_full[sb]), (uint32_t)(kb / kRingB) & 1u, abort)) {
                     stop_all(sh, a.ws);
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint64_t bd = sw128_desc(sB0 + s * kTileBBytes);
-                const uint64_t ad0 = sw128_desc(sA0 + s * kTileABytes);
-                const uint64_t ad1 = sw128_desc(sA0 + s * kTileABytes + kMmaM * 128);
+                const uint64_t bd = sw128_desc(sB0 + sb * kTileBBytes);
+                const uint64_t ad0 = sw128_desc(sA0 + sa * kTileABytes);
+                const uint64_t ad1 = sw128_desc(sA0 + sa * kTileABytes + kMmaM * 128);
 #pragma unroll
                 for (int j = 0; j < kBK / kUmmaK; ++j) {  // +32 bytes along K per step
                     const uint32_t acc = (kb | j) != 0 ? 1u : 0u;
                     umma_f16(tmem, ad0 + 2u * j, bd + 2u * j, kIdesc, acc);
                     umma_f16(tmem + kBN, ad1 + 2u * j, bd + 2u * j, kIdesc, acc);
                 }
-                umma_commit(smem_u32(&sh.empty[s]));
+                umma_commit(smem_u32(&sh.a_empty[sa]));
+                umma_commit(smem_u32(&sh.b_empty[sb]));
             }
             if (ok) {
                 umma_commit(smem_u32(&sh.accum));
@@ -379,32 +423,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
     } else {
         // ---- decode warps: two threads per weight row, 32 columns (two blocks) each ----
-        // A stage's weight tile may be rewritten once its record has landed: the record's
-        // copy was issued only after the MMAs of the stage's previous use completed.
         const int t = threadIdx.x;
         const int row = t >> 1;
         const int half = t & 1;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
-            const int s = kb % kRing;
-            const uint32_t ph = (uint32_t)(kb / kRing) & 1u;
-            const bool got = mbar_wait(smem_u32(&sh.full[s]), ph, abort);
-            if (!__all_sync(0xFFFFFFFFu, got)) {
+            const int sw = kb % kRingW, sb = kb % kRingB;
+            if (!warp_wait(smem_u32(&sh.w_full[sw]), (uint32_t)(kb / kRingW) & 1u, abort) ||
+                !warp_wait(smem_u32(&sh.b_empty[sb]), ((uint32_t)(kb / kRingB) & 1u) ^ 1u, abort)) {
                 if (lane == 0) stop_all(sh, a.ws);
                 ok = false;
                 break;
             }
-            const uint8_t* rec = gW0 + s * kRecBytes;
+            const uint8_t* rec = gW0 + (sw * kRecPerTile + row / kRecRows) * kRecBytes;
+            const int rr = row % kRecRows;
             uint32_t c[4];
             {
-                const uint4 v = *reinterpret_cast<const uint4*>(rec + row * 32 + half * 16);
+                const uint4 v = *reinterpret_cast<const uint4*>(rec + rr * 32 + half * 16);
                 c[0] = v.x;
                 c[1] = v.y;
                 c[2] = v.z;
                 c[3] = v.w;
             }
-            const uint32_t sc = *reinterpret_cast<const uint16_t*>(rec + kRecCodes + row * 4 + half * 2);
-            uint8_t* tile_row = gB0 + s * kTileBBytes + row * 128;
+            const uint32_t sc = *reinterpret_cast<const uint16_t*>(rec + kRecCodes + rr * 4 + half * 2);
+            uint8_t* tile_row = gB0 + sb * kTileBBytes + row * 128;
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 const float sd = sh.sd[(sc >> (8 * i)) & 0xFFu];
@@ -419,24 +461,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                  : "memory");
                 }
             }
+            // orders this thread's reads of the record and writes of the tile before the
+            // async-proxy operations that follow the arrivals (the next copy into the
+            // record slot, the MMAs reading the tile)
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sh.decoded[s]));
+            if (lane == 0) {
+                mbar_arrive(smem_u32(&sh.w_empty[sw]));
+                mbar_arrive(smem_u32(&sh.b_full[sb]));
+            }
         }
 
-        // ---- epilogue: warp w reads accumulator w / 4, lanes 32 * (w % 4) .. + 31 ----
+        // ---- epilogue: warp w reads lanes 32 * (w % 4) .. + 31 of accumulator (w / 4) % 2,
+        //      columns 128 * (w / 8) .. + 127 ----
         if (ok) {
-            const bool got = mbar_wait(smem_u32(&sh.accum), 0u, abort);
-            if (!__all_sync(0xFFFFFFFFu, got)) {
+            if (!warp_wait(smem_u32(&sh.accum), 0u, abort)) {
                 if (lane == 0) stop_all(sh, a.ws);
             } else {
                 tc_fence_after();
-                const int q = warp & 3, acc = warp >> 2;
+                const int q = warp & 3, acc = (warp >> 2) & 1, ch = warp >> 3;
                 const int64_t m = m0 + kMmaM * acc + 32 * q + lane;
                 const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * kBN);
 #pragma unroll 1
-                for (int j = 0; j < kBN / 16; ++j) {
-                    const int col0 = 16 * j;
+                for (int j = 0; j < kBN / 32; ++j) {
+                    const int col0 = ch * (kBN / 2) + 16 * j;
                     uint32_t v[16];
                     tmem_ld16(trow + (uint32_t)col0, v);
                     const int64_t nc = n0 + col0;
@@ -537,7 +585,7 @@ bool weight_shape_ok(int64_t N, int64_t K) {
 }
 
 int64_t record_bytes(int64_t N, int64_t K) {
-    return ((N + kBN - 1) / kBN) * ((K + kBK - 1) / kBK) * (int64_t)kRecBytes;
+    return ((N + kRecRows - 1) / kRecRows) * ((K + kBK - 1) / kBK) * (int64_t)kRecBytes;
 }
 
 }  // namespace
@@ -556,7 +604,7 @@ NVFP4_API nvfp4_status nvfp4_w4a16_pack(const uint8_t* packed, const uint8_t* sc
     if (packed == nullptr || scales == nullptr || tiled == nullptr) return NVFP4_ERR_NULL;
     if (!is_aligned(packed, 8) || !is_aligned(tiled, 16)) return NVFP4_ERR_ALIGN;
     const int64_t KT = (K + kBK - 1) / kBK;
-    const int64_t rows = ((N + kBN - 1) / kBN) * KT * kBN;  // one thread per record row
+    const int64_t rows = ((N + kRecRows - 1) / kRecRows) * KT * kRecRows;  // one thread per record row
     int sms = 0;
     nvfp4_status st = sm_count_w4(&sms);
     if (st != NVFP4_OK) return st;
