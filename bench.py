@@ -37,6 +37,7 @@ UNIT = "GB/s"
 KERNEL_BYTES = {"amax": 2.0, "fake_quant": 4.0, "quantize": 2.0 + 0.5 + 1.0 / 16, "dequantize": 0.5 + 1.0 / 16 + 2.0}
 STEP_BYTES = sum(KERNEL_BYTES.values())  # 11.125 bytes per element
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 CSRC = os.path.join(ROOT, "qat_nvfp4_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
@@ -56,6 +57,10 @@ def parse_args():
     p.add_argument("--sweep", metavar="OUT_JSON", default=None,
                    help="instead of the one-line step benchmark, time each kernel on every workload size "
                         "(L2 flushed before each rep), print a table and write it as JSON to OUT_JSON")
+    p.add_argument("--linear", metavar="OUT_JSON", default=None,
+                   help="instead of the step benchmark, time the W4A16 linear (x . W^T with W stored as NVFP4 "
+                        "records) for several token counts on the pages' weight shapes, beside dequantize + "
+                        "torch bf16 linear and a bf16 linear on an unquantized weight; print a table, write JSON")
     return p.parse_args()
 
 
@@ -71,12 +76,27 @@ def workload_config(args, world):
     }
 
 
+# The sources of the kernels the step runs (the W4A16 linear has its own file).
+STEP_SOURCES = ("nvfp4_device.cuh", "nvfp4_kernels.cu", "nvfp4_runtime.h")
+
+
 def source_digest():
     h = hashlib.sha256()
-    for fn in sorted(os.listdir(CSRC)):
+    for fn in STEP_SOURCES:
         with open(os.path.join(CSRC, fn), "rb") as f:
             h.update(fn.encode() + b"\0" + f.read())
     return h.hexdigest()
+
+
+def bf16_peak():
+    """Measured dense bf16 tensor throughput (TFLOP/s), burst figure: the linear kernels are
+    timed one launch at a time."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst cuBLAS GEMM)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, "fallback (earlier measurement on this pool)"
 
 
 def hbm_peak():
@@ -492,10 +512,79 @@ def run_sweep(args):
     return 0
 
 
+def run_linear(args):
+    """W4A16 linear on the pages' weights (4096 x 4096, 14336 x 4096) under 1 .. 8192 tokens of
+    N(0, 1) activations.  Roofline per shape: the larger of 2MNK / measured bf16 peak and
+    (x + packed weight + y bytes) / measured HBM peak; frac = that time / measured time.
+    Beside it: the pages' own order of work (nvfp4_dequantize into a bf16 buffer, then torch's
+    bf16 linear) and a bf16 linear on an unquantized bf16 weight.  L2 flushed before each rep
+    (a write of 256 MB); CUDA events; median of 15 reps."""
+    import torch
+    from qat_nvfp4_b200 import nvfp4 as nv
+    from qat_nvfp4_b200 import synthetic
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hbm, hbm_src = hbm_peak()
+    tc, tc_src = bf16_peak()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ws = nv.new_workspace(dev)
+
+    def timed(fn, reps=15):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1))
+        return sorted(ts)[len(ts) // 2] / 1e3
+
+    rows = []
+    for (N, K) in [(4096, 4096), (14336, 4096)]:
+        w = synthetic.activation_normal_device((N, K), 7, dev) * 0.02
+        packed, scales, gs = nv.nvfp4_quantize(w, nv.nvfp4_amax(w))
+        tiled = nv.nvfp4_w4a16_pack(packed, scales)
+        wbuf = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+        for M in (1, 16, 128, 1024, 4096, 8192):
+            x = synthetic.activation_normal_device((M, K), 8 + M, dev)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            t_fused = timed(lambda: nv.nvfp4_w4a16_linear(x, tiled, gs, N, out=y, workspace=ws))
+            t_pages = timed(lambda: (nv.nvfp4_dequantize(packed, scales, gs, out=wbuf), torch.matmul(x, wbuf.t(), out=y)))
+            t_bf16 = timed(lambda: torch.matmul(x, w.t(), out=y))
+            flops = 2.0 * M * N * K
+            nbytes = 2.0 * M * K + 0.5625 * N * K + 2.0 * M * N
+            ideal = max(flops / (tc * 1e12), nbytes / (hbm * 1e9))
+            rows.append({"weight": [N, K], "tokens": M, "fused_us": t_fused * 1e6,
+                         "TFLOP/s": flops / t_fused / 1e12, "GB/s": nbytes / t_fused / 1e9,
+                         "bound": "tensor" if flops / (tc * 1e12) >= nbytes / (hbm * 1e9) else "hbm",
+                         "frac": ideal / t_fused, "dequant_then_linear_us": t_pages * 1e6,
+                         "bf16_linear_us": t_bf16 * 1e6})
+            del x, y
+        del w, packed, scales, tiled, wbuf
+    print(f"bf16 peak {tc:.1f} TFLOP/s ({tc_src}); HBM peak {hbm:.1f} GB/s ({hbm_src})")
+    print("| weight | tokens | W4A16 us | TFLOP/s | GB/s | bound | frac of roofline | dequantize + linear us "
+          "| bf16 linear (unquantized weight) us |")
+    print("|---|---|---|---|---|---|---|---|---|")
+    for r in rows:
+        print(f"| {r['weight'][0]}x{r['weight'][1]} | {r['tokens']} | {r['fused_us']:.1f} | {r['TFLOP/s']:.0f} | "
+              f"{r['GB/s']:.0f} | {r['bound']} | {r['frac']:.2f} | {r['dequant_then_linear_us']:.1f} | "
+              f"{r['bf16_linear_us']:.1f} |")
+    with open(args.linear, "w") as f:
+        json.dump({"bf16_tflops": tc, "hbm_gbs": hbm, "rows": rows}, f, indent=1)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.sweep:
         return run_sweep(args)
+    if args.linear:
+        return run_linear(args)
     if args.cols < 1 or args.rows < 1:
         raise SystemExit("--rows and --cols must be positive")
     if args.impl == "reference":

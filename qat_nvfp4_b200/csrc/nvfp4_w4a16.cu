@@ -42,53 +42,74 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int kBM = 256;                  // rows of x per tile: two MMAs of M = 128
-constexpr int kMmaM = 128;
-constexpr int kBN = 256;                  // weight rows (output features) per tile (MMA N)
+constexpr int kMmaM = 128;                // rows of x per accumulator (MMA M)
 constexpr int kRecRows = 128;             // weight rows per record
 constexpr int kBK = 64;                   // K per stage: 64 bf16 = one 128-byte swizzle row
 constexpr int kUmmaK = 16;                // K of one kind::f16 MMA
-constexpr int kRingA = 3;                 // activation tiles in flight
-constexpr int kRingW = 4;                 // weight-record pairs in flight
-constexpr int kRingB = 2;                 // decoded weight tiles between the decode warps and the MMAs
 constexpr int kDecodeWarps = 16;
+constexpr int kDecodeThreads = 32 * kDecodeWarps;
 constexpr int kTmaWarp = 16;              // activation loads
 constexpr int kMmaWarp = 17;
 constexpr int kRecWarp = 18;              // weight-record loads
 constexpr int kGemmThreads = 608;
-constexpr int kTileABytes = kBM * kBK * 2;   // 32 KB
-constexpr int kTileBBytes = kBN * kBK * 2;   // 32 KB
 constexpr int kRecCodes = kRecRows * kBK / 2;  // 4096 bytes of E2M1 codes per record
 constexpr int kRecBytes = kRecCodes + kRecRows * (kBK / kBlockElems);  // + 512 scale bytes = 4608
-constexpr int kRecPerTile = kBN / kRecRows;    // records per stage
-constexpr int kTmemCols = 2 * kBN;           // two fp32 accumulators of 128 lanes x kBN columns: all 512
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 static_assert(kBK * 2 == 128, "one swizzle row per tile row");
-static_assert(kDecodeWarps * 32 == 2 * kBN, "two decode threads per weight row");
-static_assert(kTmemCols <= 512, "tensor memory columns");
 static_assert(kGemmThreads == 32 * (kDecodeWarps + 3), "warp roles");
 static_assert(kRecBytes % 16 == 0, "bulk copy size");
-static_assert(kTileABytes % 1024 == 0 && kTileBBytes % 1024 == 0, "operand tiles stay 1024-byte aligned");
 
-// Shared memory: activation tiles, decoded weight tiles (both 1024-byte aligned), weight
-// records, then the barriers and the table.
-struct GemmShared {
-    uint64_t a_full[kRingA];   // activation tile landed (TMA bytes)
-    uint64_t a_empty[kRingA];  // the MMAs that read it completed
-    uint64_t w_full[kRingW];   // weight records landed (bulk-copy bytes)
-    uint64_t w_empty[kRingW];  // the decode warps have read it
-    uint64_t b_full[kRingB];   // the decode warps wrote the weight tile
-    uint64_t b_empty[kRingB];  // the MMAs that read it completed
-    uint64_t accum;            // every MMA of the tile completed
-    uint64_t drain;            // used only when stopping early
-    uint32_t tmem_base;
-    uint32_t abort;
-    float sd[256];             // decode scale for every E4M3 byte: fl(E4M3(b) / gs)
+// One configuration per output tile: kAcc accumulators of 128 rows of x (kBM = 128 kAcc rows)
+// by BN weight rows (output features, the MMA's N).  256 x 256 for many rows of x (half
+// the activation traffic per FLOP of BN = 128); 256 x 128 (twice the CTAs) when x has 129
+// to 256 rows; 128 x 128 when it has at most 128 (half the MMA work and activation bytes
+// per stage, and deeper rings for the weight stream).
+template <int BN, int ACC>
+struct Cfg {
+    static constexpr int kBN = BN;
+    static constexpr int kBM = kMmaM * ACC;
+    static constexpr int kTileABytes = kBM * kBK * 2;
+    static constexpr int kRecPerTile = BN / kRecRows;           // records per stage
+    static constexpr int kTileBBytes = BN * kBK * 2;             // decoded weight tile
+    static constexpr int kTmemCols = ACC * BN;                   // fp32 accumulators, 128 lanes x BN each
+    static constexpr int kRingA = BN == 256 ? 3 : (ACC == 2 ? 4 : 6);  // activation tiles in flight
+    static constexpr int kRingW = BN == 256 ? 4 : (ACC == 2 ? 8 : 12); // record groups in flight
+    static constexpr int kRingB = BN == 256 ? 2 : 3;             // decoded tiles, decode -> MMA
+    static constexpr int kColParts = 4 / ACC;                    // epilogue warps per accumulator lane group
+    static constexpr int kTpr = kDecodeThreads / BN;             // decode threads per weight row
+    static constexpr int kBpt = (kBK / kBlockElems) / kTpr;      // 16-element blocks per thread
+    // Instruction descriptor of kind::f16: fp32 accumulator (bits 4-5 = 1), A and B bf16
+    // (bits 7-9 = 1, bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 in bits
+    // 17-22, M >> 4 in bits 24-28.
+    static constexpr uint32_t kIdesc =
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kMmaM >> 4) << 24);
+
+    // Shared memory: activation tiles, decoded weight tiles (both 1024-byte aligned),
+    // weight records, then the barriers and the table.
+    struct Shared {
+        uint64_t a_full[kRingA];   // activation tile landed (TMA bytes)
+        uint64_t a_empty[kRingA];  // the MMAs that read it completed
+        uint64_t w_full[kRingW];   // weight records landed (bulk-copy bytes)
+        uint64_t w_empty[kRingW];  // the decode warps have read them
+        uint64_t b_full[kRingB];   // the decode warps wrote the weight tile
+        uint64_t b_empty[kRingB];  // the MMAs that read it completed
+        uint64_t accum;            // every MMA of the tile completed
+        uint64_t drain;            // used only when stopping early
+        uint32_t tmem_base;
+        uint32_t abort;
+        float sd[256];             // decode scale for every E4M3 byte: fl(E4M3(b) / gs)
+    };
+    static constexpr int kRingBytes = kRingA * kTileABytes + kRingB * kTileBBytes + kRingW * kRecPerTile * kRecBytes;
+    static constexpr int kSmemBytes = 1024 + kRingBytes + (int)sizeof(Shared);
+
+    static_assert(BN % kRecRows == 0 && BN >= 16 && BN <= 256, "MMA N");
+    static_assert(kTpr * kBpt == kBK / kBlockElems && kBpt >= 1, "decode split");
+    static_assert(kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0, "tensor memory columns");
+    static_assert(kTileABytes % 1024 == 0 && kTileBBytes % 1024 == 0, "operand tiles stay 1024-byte aligned");
+    static_assert(kDecodeWarps == 4 * ACC * kColParts, "epilogue warps");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
-constexpr int kRingBytes = kRingA * kTileABytes + kRingB * kTileBBytes + kRingW * kRecPerTile * kRecBytes;
-constexpr int kGemmSmemBytes = 1024 + kRingBytes + (int)sizeof(GemmShared);
-static_assert(kGemmSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 // ---------------------------------------------------------------------------------------
 // PTX wrappers.
@@ -224,11 +245,7 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     return d;
 }
 
-// Instruction descriptor of kind::f16: fp32 accumulator (bits 4-5 = 1), A and B bf16
-// (bits 7-9 = 1, bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22,
-// M >> 4 in bits 24-28.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
-                            ((uint32_t)(kMmaM >> 4) << 24);
+
 
 
 // ---------------------------------------------------------------------------------------
@@ -284,10 +301,12 @@ struct LinearArgs {
     int64_t M, N, K;
     int64_t tiles_n;
     int64_t kt;             // records per weight row of tiles = ceil(K / 64)
+    uint32_t a_bytes;       // bytes of one activation box (rows loaded per stage x 128)
     int vec_store;          // rows of y allow 16-byte stores
 };
 
-__device__ __forceinline__ void stop_all(GemmShared& sh, Workspace* ws) {
+template <class Sh>
+__device__ __forceinline__ void stop_all(Sh& sh, Workspace* ws) {
     *reinterpret_cast<volatile uint32_t*>(&sh.abort) = 1u;
     atomicExch(&ws->error, (unsigned)NVFP4_ERR_TIMEOUT);
 }
@@ -298,13 +317,19 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const v
     return __all_sync(0xFFFFFFFFu, got);
 }
 
+template <int BN, int ACC>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     w4a16_linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const LinearArgs a) {
+    using C = Cfg<BN, ACC>;
+    constexpr int kBN = C::kBN, kRingA = C::kRingA, kRingB = C::kRingB, kRingW = C::kRingW;
+    constexpr int kBM = C::kBM, kTileABytes = C::kTileABytes;
+    constexpr int kTileBBytes = C::kTileBBytes, kRecPerTile = C::kRecPerTile, kTpr = C::kTpr, kBpt = C::kBpt;
+    constexpr uint32_t kIdesc = C::kIdesc;
     extern __shared__ uint8_t dsmem[];
     const uint32_t raw = smem_u32(dsmem);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* ring = dsmem + (base - raw);
-    GemmShared& sh = *reinterpret_cast<GemmShared*>(ring + kRingBytes);
+    typename C::Shared& sh = *reinterpret_cast<typename C::Shared*>(ring + C::kRingBytes);
     const uint32_t sA0 = base;
     const uint32_t sB0 = sA0 + kRingA * kTileABytes;
     const uint32_t sW0 = sB0 + kRingB * kTileBBytes;
@@ -340,7 +365,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int i = threadIdx.x; i < 256; i += blockDim.x) sh.sd[i] = __fdiv_rn(e4m3_to_f32((uint32_t)i), gs);
     }
     if (warp == kMmaWarp) {
-        tmem_alloc(smem_u32(&sh.tmem_base), kTmemCols);
+        tmem_alloc(smem_u32(&sh.tmem_base), C::kTmemCols);
         tmem_relinquish();
         tc_fence_before();
     }
@@ -370,7 +395,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 const uint32_t bar = smem_u32(&full[s]);
                 if (act) {
-                    mbar_arrive_expect_tx(bar, kTileABytes);
+                    mbar_arrive_expect_tx(bar, a.a_bytes);
                     tma_load_2d(sA0 + s * kTileABytes, &tmap_x, kb * kBK, (int32_t)m0, bar);
                 } else {
                     mbar_arrive_expect_tx(bar, kRecPerTile * kRecBytes);
@@ -402,13 +427,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 tc_fence_after();
                 const uint64_t bd = sw128_desc(sB0 + sb * kTileBBytes);
-                const uint64_t ad0 = sw128_desc(sA0 + sa * kTileABytes);
-                const uint64_t ad1 = sw128_desc(sA0 + sa * kTileABytes + kMmaM * 128);
 #pragma unroll
                 for (int j = 0; j < kBK / kUmmaK; ++j) {  // +32 bytes along K per step
                     const uint32_t acc = (kb | j) != 0 ? 1u : 0u;
-                    umma_f16(tmem, ad0 + 2u * j, bd + 2u * j, kIdesc, acc);
-                    umma_f16(tmem + kBN, ad1 + 2u * j, bd + 2u * j, kIdesc, acc);
+#pragma unroll
+                    for (int h = 0; h < ACC; ++h)  // accumulator h: rows 128 h .. of the tile
+                        umma_f16(tmem + h * kBN, sw128_desc(sA0 + sa * kTileABytes + h * kMmaM * 128) + 2u * j,
+                                 bd + 2u * j, kIdesc, acc);
                 }
                 umma_commit(smem_u32(&sh.a_empty[sa]));
                 umma_commit(smem_u32(&sh.b_empty[sb]));
@@ -422,10 +447,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
     } else {
-        // ---- decode warps: two threads per weight row, 32 columns (two blocks) each ----
+        // ---- decode warps: kTpr threads per weight row, kBpt 16-element blocks each ----
         const int t = threadIdx.x;
-        const int row = t >> 1;
-        const int half = t & 1;
+        const int row = t / kTpr;
+        const int part = t % kTpr;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
             const int sw = kb % kRingW, sb = kb % kRingB;
@@ -437,27 +462,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             const uint8_t* rec = gW0 + (sw * kRecPerTile + row / kRecRows) * kRecBytes;
             const int rr = row % kRecRows;
-            uint32_t c[4];
-            {
-                const uint4 v = *reinterpret_cast<const uint4*>(rec + rr * 32 + half * 16);
+            uint32_t c[2 * kBpt];
+            uint32_t sc;
+            if constexpr (kBpt == 2) {
+                const uint4 v = *reinterpret_cast<const uint4*>(rec + rr * 32 + part * 16);
                 c[0] = v.x;
                 c[1] = v.y;
                 c[2] = v.z;
                 c[3] = v.w;
+                sc = *reinterpret_cast<const uint16_t*>(rec + kRecCodes + rr * 4 + part * 2);
+            } else {
+                const uint2 v = *reinterpret_cast<const uint2*>(rec + rr * 32 + part * 8);
+                c[0] = v.x;
+                c[1] = v.y;
+                sc = rec[kRecCodes + rr * 4 + part];
             }
-            const uint32_t sc = *reinterpret_cast<const uint16_t*>(rec + kRecCodes + rr * 4 + half * 2);
             uint8_t* tile_row = gB0 + sb * kTileBBytes + row * 128;
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
+            for (int i = 0; i < kBpt; ++i) {
                 const float sd = sh.sd[(sc >> (8 * i)) & 0xFFu];
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     const uint32_t w = c[2 * i + q];
-                    const uint32_t o0 = decode_pair(w & 0xFFu, sd), o1 = decode_pair((w >> 8) & 0xFFu, sd);
-                    const uint32_t o2 = decode_pair((w >> 16) & 0xFFu, sd), o3 = decode_pair(w >> 24, sd);
-                    const int chunk = 4 * half + 2 * i + q;  // 8 elements = 16 bytes
+                    uint32_t o[4];
+                    o[0] = decode_pair(w & 0xFFu, sd);
+                    o[1] = decode_pair((w >> 8) & 0xFFu, sd);
+                    o[2] = decode_pair((w >> 16) & 0xFFu, sd);
+                    o[3] = decode_pair(w >> 24, sd);
+                    const int chunk = 2 * (kBpt * part + i) + q;  // 8 elements = 16 bytes
                     const uint32_t dst = smem_u32(tile_row + ((chunk ^ (row & 7)) << 4));
-                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(o0), "r"(o1), "r"(o2), "r"(o3)
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(o[0]), "r"(o[1]), "r"(o[2]),
+                                 "r"(o[3])
                                  : "memory");
                 }
             }
@@ -472,19 +507,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
 
-        // ---- epilogue: warp w reads lanes 32 * (w % 4) .. + 31 of accumulator (w / 4) % 2,
-        //      columns 128 * (w / 8) .. + 127 ----
+        // ---- epilogue: warp w reads lanes 32 * (w % 4) .. + 31 of accumulator (w / 4) % ACC,
+        //      column part w / (4 ACC) of kColParts ----
         if (ok) {
             if (!warp_wait(smem_u32(&sh.accum), 0u, abort)) {
                 if (lane == 0) stop_all(sh, a.ws);
             } else {
                 tc_fence_after();
-                const int q = warp & 3, acc = (warp >> 2) & 1, ch = warp >> 3;
+                constexpr int kCols = kBN / C::kColParts;  // columns per warp
+                const int q = warp & 3, acc = (warp >> 2) % ACC, ch = warp / (4 * ACC);
                 const int64_t m = m0 + kMmaM * acc + 32 * q + lane;
                 const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * kBN);
 #pragma unroll 1
-                for (int j = 0; j < kBN / 32; ++j) {
-                    const int col0 = ch * (kBN / 2) + 16 * j;
+                for (int j = 0; j < kCols / 16; ++j) {
+                    const int col0 = ch * kCols + 16 * j;
                     uint32_t v[16];
                     tmem_ld16(trow + (uint32_t)col0, v);
                     const int64_t nc = n0 + col0;
@@ -522,7 +558,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     if (warp == kMmaWarp) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, C::kTmemCols);
     }
 }
 
@@ -558,8 +594,12 @@ nvfp4_status gemm_smem_optin() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevs) return NVFP4_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_w4_mu);
     if (!g_smem_set[dev]) {
-        if (cudaFuncSetAttribute(w4a16_linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(w4a16_linear_kernel<256, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<256, 2>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(w4a16_linear_kernel<128, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<128, 2>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(w4a16_linear_kernel<128, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<128, 1>::kSmemBytes) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         g_smem_set[dev] = true;
     }
@@ -620,7 +660,13 @@ NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, c
                                           const float* d_global_scale, int64_t N, const void* bias, void* y,
                                           void* d_workspace, nvfp4_stream_t stream) {
     if (M < 0 || !weight_shape_ok(N, K) || M > 0x7FFFFF00ll) return NVFP4_ERR_SHAPE;
-    const int64_t tiles_m = (M + kBM - 1) / kBM, tiles_n = (N + kBN - 1) / kBN;
+    // Output tiles 256 x 256 when x has more than 256 rows, 256 x 128 for 129 to 256 rows,
+    // 128 x 128 for at most 128.
+    const int acc = M > kMmaM ? 2 : 1;
+    const int bm = kMmaM * acc;
+    const int bn = M > 2 * kMmaM ? 256 : 128;
+    const int64_t tiles_m = (M + bm - 1) / bm;
+    const int64_t tiles_n = (N + bn - 1) / bn;
     if (tiles_m * tiles_n > 0x7FFFFFFFll) return NVFP4_ERR_SHAPE;
     if (d_global_scale == nullptr || d_workspace == nullptr) return NVFP4_ERR_NULL;
     if (M > 0 && N > 0 && (x == nullptr || tiled == nullptr || y == nullptr)) return NVFP4_ERR_NULL;
@@ -636,13 +682,17 @@ NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, c
     st = gemm_smem_optin();
     if (st != NVFP4_OK) return st;
 
-    // x as a [M, K] bf16 tensor, boxes of 256 rows x 64 columns, 128-byte swizzle, zero
-    // fill past either edge.
+    // x as a [M, K] bf16 tensor, boxes of bm rows x 64 columns, 128-byte swizzle, zero fill
+    // past either edge.  When x fits in one row tile the box is cut to M rounded up to 8
+    // rows: the rows of the tile past it are never written, and the MMA rows they feed are
+    // output rows past M, which are not stored (each output row depends only on its own
+    // row of x).
     CUtensorMap map;
     std::memset(&map, 0, sizeof(map));
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBM};
+    const int box_rows = tiles_m == 1 ? (int)((M + 7) / 8 * 8) : bm;
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -661,8 +711,15 @@ NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, c
     a.tiles_n = tiles_n;
     a.kt = (K + kBK - 1) / kBK;
     a.vec_store = (is_aligned(y, 16) && N % 8 == 0) ? 1 : 0;
-    w4a16_linear_kernel<<<(unsigned)(tiles_m * tiles_n), kGemmThreads, kGemmSmemBytes,
-                          reinterpret_cast<cudaStream_t>(stream)>>>(map, a);
+    a.a_bytes = (uint32_t)box_rows * kBK * 2;
+    const unsigned grid = (unsigned)(tiles_m * tiles_n);
+    cudaStream_t cst = reinterpret_cast<cudaStream_t>(stream);
+    if (bn == 256)
+        w4a16_linear_kernel<256, 2><<<grid, kGemmThreads, Cfg<256, 2>::kSmemBytes, cst>>>(map, a);
+    else if (acc == 2)
+        w4a16_linear_kernel<128, 2><<<grid, kGemmThreads, Cfg<128, 2>::kSmemBytes, cst>>>(map, a);
+    else
+        w4a16_linear_kernel<128, 1><<<grid, kGemmThreads, Cfg<128, 1>::kSmemBytes, cst>>>(map, a);
     note_launch();
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

@@ -21,6 +21,7 @@ import torch
 import oracle
 from qat_nvfp4_b200 import synthetic
 from nvfp4_testutil import bits, sample_rows, to_dev, u8
+from nvfp4_testutil import u8_to_dev as to_dev_u8
 
 pytestmark = pytest.mark.gpu
 
@@ -84,6 +85,28 @@ def _assert_within_bound(y_bits, x_bits, packed, scales, gs, bias_bits, what):
     assert bad.size == 0, (f"{what}: {len(bad)} elements outside the bound, first {bad[:3].tolist()}: "
                            f"got {got[tuple(bad[0])]}, exact {exact[tuple(bad[0])]}, tol {tol[tuple(bad[0])]}")
     return exact
+
+
+@pytest.mark.parametrize("K", [128, 256, 512])
+def test_decoded_weight_is_exact_through_one_hot_rows(K):
+    """x = the K x K identity: output row k is 1 * W[:, k] plus exact zeros, so y^T must be
+    the oracle's dequantized weight bit for bit (up to the sign of a zero sum).  Random
+    bytes cover every code and every finite scale byte, negative E4M3 scales included;
+    K = 128, 256 and 512 run the 128 x 128, 256 x 128 and 256 x 256 tile configurations."""
+    rng = np.random.default_rng(K)
+    N = 300
+    packed = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    scales = rng.integers(0, 256, size=(N, K // 16), dtype=np.uint8)
+    scales[(scales & 0x7F) == 0x7F] = 0x3C  # NaN bytes are outside the method
+    gs = 7168.0
+    tiled = nv.nvfp4_w4a16_pack(to_dev_u8(packed), to_dev_u8(scales))
+    eye = to_dev(synthetic.to_bf16_bits(np.eye(K, dtype=np.float32)))
+    y = bits(nv.nvfp4_w4a16_linear(eye, tiled, torch.tensor([gs], device="cuda"), N))
+    want = oracle.dequantize(packed, scales, gs, N, K).T
+    y = np.where((y & 0x7FFF) == 0, 0, y)
+    want = np.where((want & 0x7FFF) == 0, 0, want)
+    bad = np.argwhere(y != want)
+    assert bad.size == 0, f"{len(bad)} decoded weights differ, first {bad[:3].tolist()}"
 
 
 @pytest.mark.parametrize("M,K,N,with_bias", [
