@@ -61,6 +61,9 @@ def parse_args():
                    help="instead of the step benchmark, time the W4A16 linear (x . W^T with W stored as NVFP4 "
                         "records) for several token counts on the pages' weight shapes, beside dequantize + "
                         "torch bf16 linear and a bf16 linear on an unquantized weight; print a table, write JSON")
+    p.add_argument("--linear-shape", metavar="M,K,N", default=None,
+                   help="run the W4A16 linear three times on one shape (tokens M, in-features K, out-features "
+                        "N; N(0, 1) activations, N(0, 0.02) weight) and exit: the command profiled by ncu")
     return p.parse_args()
 
 
@@ -579,12 +582,36 @@ def run_linear(args):
     return 0
 
 
+def run_linear_shape(args):
+    import torch
+    from qat_nvfp4_b200 import nvfp4 as nv
+    from qat_nvfp4_b200 import synthetic
+
+    M, K, N = (int(v) for v in args.linear_shape.split(","))
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    x = synthetic.activation_normal_device((M, K), 1, dev)
+    w = synthetic.activation_normal_device((N, K), 2, dev) * 0.02
+    packed, scales, gs = nv.nvfp4_quantize(w, nv.nvfp4_amax(w))
+    tiled = nv.nvfp4_w4a16_pack(packed, scales)
+    ws = nv.new_workspace(dev)
+    for _ in range(3):
+        y = nv.nvfp4_w4a16_linear(x, tiled, gs, N, workspace=ws)
+    torch.cuda.synchronize(dev)
+    if nv.nvfp4_workspace_check(ws) != 0:
+        raise SystemExit("W4A16 linear reported a timeout")
+    print(json.dumps({"linear_shape": [M, K, N], "y_abs_mean": float(y.float().abs().mean())}))
+    return 0
+
+
 def main():
     args = parse_args()
     if args.sweep:
         return run_sweep(args)
     if args.linear:
         return run_linear(args)
+    if args.linear_shape:
+        return run_linear_shape(args)
     if args.cols < 1 or args.rows < 1:
         raise SystemExit("--rows and --cols must be positive")
     if args.impl == "reference":
