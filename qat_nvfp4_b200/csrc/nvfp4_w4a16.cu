@@ -30,7 +30,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -564,377 +563,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------
-// Pair kernel: two CTAs of a cluster (two SMs) share each MMA (tcgen05 cta_group::2,
-// M = 256 across the pair, N = 256).  Per pair the output tile is 512 x 256: accumulator h
-// (h = 0, 1) covers rows 256 h .. 256 h + 255 of the tile, of which CTA r holds rows
-// 256 h + 128 r .. + 127 in its own tensor memory; the weight tile's 256 rows are split the
-// same way, CTA r decoding rows 128 r .. + 127 into its own shared memory.  So each SM
-// decodes half of what a one-SM 256 x 256 tile needs and its shared memory serves half of
-// the weight operand reads, for the same MMA work per SM.
-//
-// CTA 0 (the leader) issues every MMA and commit.  It learns that a stage is ready from
-//   p_full[s]:  1 arrival from the peer's MMA warp once the peer's activation tile landed
-//               (the leader's own tile is its local a_full[s]);
-//   b_full[s]:  one arrival per decode warp of both CTAs (the peer's arrive remotely).
-// Its commits arrive on both CTAs' a_empty / b_empty / accum barriers.  No copy is
-// multicast: each CTA loads only into its own shared memory.
-// A bounded wait that runs out stops both CTAs (stop flags in both), and the pair ends with
-// a bounded handshake so that neither CTA exits while the other may still touch its shared
-// memory.
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// shared::cluster address of the variable at local shared address `a` in CTA `rank`
-__device__ __forceinline__ uint32_t map_to(uint32_t a, uint32_t rank) {
-    uint32_t d;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(rank));
-    return d;
-}
-
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
-}
-
-__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc2(uint32_t dst_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish2() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-__device__ __forceinline__ void umma_f16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                              uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Arrive once on this CTA's barrier at shared address `bar` when every pair MMA this
-// thread issued so far completed.
-__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-// The same arrival on the barrier at shared address `bar` in both CTAs of the pair (the
-// commit's CTA mask; this is a completion signal, not a copy).
-__device__ __forceinline__ void umma_commit_both(uint32_t bar) {
-    const uint16_t mask = 0x3;
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
-                 "h"(mask)
-                 : "memory");
-}
-
-struct PairCfg {
-    static constexpr int kBN = 256;                      // weight rows per pair tile (MMA N)
-    static constexpr int kHalfN = kBN / 2;               // weight rows decoded by one CTA
-    static constexpr int kAcc = 2;
-    static constexpr int kPairM = 2 * kMmaM * kAcc;      // 512 rows of x per pair tile
-    static constexpr int kTileABytes = kAcc * kMmaM * kBK * 2;  // this CTA's 256 rows: 32 KB
-    static constexpr int kTileBBytes = kHalfN * kBK * 2;        // this CTA's half weight tile: 16 KB
-    static constexpr int kRingA = 4, kRingB = 3, kRingW = 6;
-    static constexpr int kTmemCols = kAcc * kBN;         // 512
-    static constexpr int kTpr = kDecodeThreads / kHalfN; // 4 decode threads per weight row
-    static constexpr int kBpt = (kBK / kBlockElems) / kTpr;
-    // kind::f16, fp32 accumulator, bf16 A and B, K-major, N = 256, M = 256 (pair)
-    static constexpr uint32_t kIdesc =
-        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)((2 * kMmaM) >> 4) << 24);
-    struct Shared {
-        uint64_t a_full[kRingA];    // local activation tile landed
-        uint64_t a_empty[kRingA];   // the pair MMAs that read it completed (leader's commit)
-        uint64_t p_full[kRingA];    // leader only: the peer's activation tile landed
-        uint64_t w_full[kRingW];
-        uint64_t w_empty[kRingW];
-        uint64_t b_full[kRingB];    // leader only: decode warps of both CTAs wrote their halves
-        uint64_t b_empty[kRingB];   // the pair MMAs that read it completed (leader's commit)
-        uint64_t accum;
-        uint64_t drain;
-        uint64_t done;              // the other CTA has finished with this one
-        uint32_t tmem_base;
-        uint32_t abort;
-        float sd[256];
-    };
-    static constexpr int kRingBytes = kRingA * kTileABytes + kRingB * kTileBBytes + kRingW * kRecBytes;
-    static constexpr int kSmemBytes = 1024 + kRingBytes + (int)sizeof(Shared);
-    static_assert(kTpr * kBpt == kBK / kBlockElems && kBpt >= 1, "decode split");
-    static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
-    static_assert(kDecodeWarps == 4 * kAcc * 2, "epilogue warps: 4 lane groups x 2 accumulators x 2 column halves");
-};
-
-__device__ __forceinline__ void stop_pair(PairCfg::Shared& sh, Workspace* ws, uint32_t peer) {
-    *reinterpret_cast<volatile uint32_t*>(&sh.abort) = 1u;
-    st_cluster_u32(map_to(smem_u32(&sh.abort), peer), 1u);
-    atomicExch(&ws->error, (unsigned)NVFP4_ERR_TIMEOUT);
-}
-
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    w4a16_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const LinearArgs a) {
-    using C = PairCfg;
-    extern __shared__ uint8_t dsmem[];
-    const uint32_t raw = smem_u32(dsmem);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t* ring = dsmem + (base - raw);
-    C::Shared& sh = *reinterpret_cast<C::Shared*>(ring + C::kRingBytes);
-    const uint32_t sA0 = base;
-    const uint32_t sB0 = sA0 + C::kRingA * C::kTileABytes;
-    const uint32_t sW0 = sB0 + C::kRingB * C::kTileBBytes;
-    uint8_t* gB0 = ring + C::kRingA * C::kTileABytes;
-    const uint8_t* gW0 = gB0 + C::kRingB * C::kTileBBytes;
-
-    const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
-    const bool leader = rank == 0;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t pt = (int64_t)(blockIdx.x >> 1);
-    const int64_t tm = pt / a.tiles_n, tn = pt % a.tiles_n;
-    const int64_t m0 = tm * C::kPairM, n0 = tn * C::kBN;
-    const int nk = (int)a.kt;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kRingA; ++s) {
-            mbar_init(smem_u32(&sh.a_full[s]), 1);
-            mbar_init(smem_u32(&sh.a_empty[s]), 1);
-            mbar_init(smem_u32(&sh.p_full[s]), 1);
-        }
-        for (int s = 0; s < C::kRingW; ++s) {
-            mbar_init(smem_u32(&sh.w_full[s]), 1);
-            mbar_init(smem_u32(&sh.w_empty[s]), kDecodeWarps);
-        }
-        for (int s = 0; s < C::kRingB; ++s) {
-            mbar_init(smem_u32(&sh.b_full[s]), 2 * kDecodeWarps);
-            mbar_init(smem_u32(&sh.b_empty[s]), 1);
-        }
-        mbar_init(smem_u32(&sh.accum), 1);
-        mbar_init(smem_u32(&sh.drain), 1);
-        mbar_init(smem_u32(&sh.done), 1);
-        sh.abort = 0u;
-        fence_barrier_init();
-        fence_proxy_async_smem();
-    }
-    {
-        const float gs = __ldg(a.d_gs);
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) sh.sd[i] = __fdiv_rn(e4m3_to_f32((uint32_t)i), gs);
-    }
-    if (warp == kMmaWarp) {
-        tmem_alloc2(smem_u32(&sh.tmem_base), C::kTmemCols);
-        tmem_relinquish2();
-        tc_fence_before();
-    }
-    __syncthreads();
-    cluster_sync_all();  // both CTAs' barriers are initialised before any remote arrival
-    tc_fence_after();
-    const uint32_t tmem = sh.tmem_base;
-    const volatile uint32_t* abort = &sh.abort;
-
-    if (warp == kTmaWarp) {
-        // ---- this CTA's 2 x 128 activation rows per stage ----
-        if (lane == 0) {
-            int issued = 0;
-            for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % C::kRingA;
-                const uint32_t ph = (uint32_t)(kb / C::kRingA) & 1u;
-                if (!mbar_wait(smem_u32(&sh.a_empty[s]), ph ^ 1u, abort)) {
-                    stop_pair(sh, a.ws, peer);
-                    break;
-                }
-                const uint32_t bar = smem_u32(&sh.a_full[s]);
-                mbar_arrive_expect_tx(bar, C::kTileABytes);
-#pragma unroll
-                for (int h = 0; h < C::kAcc; ++h)
-                    tma_load_2d(sA0 + s * C::kTileABytes + h * kMmaM * 128, &tmap_x, kb * kBK,
-                                (int32_t)(m0 + 2 * kMmaM * h + kMmaM * rank), bar);
-                ++issued;
-            }
-            for (int kb = issued > C::kRingA ? issued - C::kRingA : 0; kb < issued; ++kb)
-                if (!mbar_wait(smem_u32(&sh.a_full[kb % C::kRingA]), (uint32_t)(kb / C::kRingA) & 1u, abort, true))
-                    stop_pair(sh, a.ws, peer);
-        }
-    } else if (warp == kRecWarp) {
-        // ---- this CTA's weight record per stage: rows 128 rank .. + 127 of the pair tile ----
-        if (lane == 0) {
-            const int64_t nrec = (a.N + kRecRows - 1) / kRecRows;
-            int64_t rn = 2 * tn + rank;
-            if (rn >= nrec) rn = nrec - 1;  // rows past N: decoded, never stored
-            const uint8_t* rec0 = a.tiled + rn * a.kt * kRecBytes;
-            int issued = 0;
-            for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % C::kRingW;
-                const uint32_t ph = (uint32_t)(kb / C::kRingW) & 1u;
-                if (!mbar_wait(smem_u32(&sh.w_empty[s]), ph ^ 1u, abort)) {
-                    stop_pair(sh, a.ws, peer);
-                    break;
-                }
-                const uint32_t bar = smem_u32(&sh.w_full[s]);
-                mbar_arrive_expect_tx(bar, kRecBytes);
-                bulk_load(sW0 + s * kRecBytes, rec0 + (int64_t)kb * kRecBytes, kRecBytes, bar);
-                ++issued;
-            }
-            for (int kb = issued > C::kRingW ? issued - C::kRingW : 0; kb < issued; ++kb)
-                if (!mbar_wait(smem_u32(&sh.w_full[kb % C::kRingW]), (uint32_t)(kb / C::kRingW) & 1u, abort, true))
-                    stop_pair(sh, a.ws, peer);
-        }
-    } else if (warp == kMmaWarp) {
-        if (lane == 0) {
-            if (leader) {
-                bool ok = true;
-                for (int kb = 0; kb < nk; ++kb) {
-                    const int sa = kb % C::kRingA, sb = kb % C::kRingB;
-                    const uint32_t pa = (uint32_t)(kb / C::kRingA) & 1u, pb = (uint32_t)(kb / C::kRingB) & 1u;
-                    if (!mbar_wait(smem_u32(&sh.a_full[sa]), pa, abort) || !mbar_wait(smem_u32(&sh.p_full[sa]), pa, abort) ||
-                        !mbar_wait(smem_u32(&sh.b_full[sb]), pb, abort)) {
-                        stop_pair(sh, a.ws, peer);
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t bd = sw128_desc(sB0 + sb * C::kTileBBytes);
-#pragma unroll
-                    for (int j = 0; j < kBK / kUmmaK; ++j) {
-                        const uint32_t acc = (kb | j) != 0 ? 1u : 0u;
-#pragma unroll
-                        for (int h = 0; h < C::kAcc; ++h)
-                            umma_f16_pair(tmem + h * C::kBN, sw128_desc(sA0 + sa * C::kTileABytes + h * kMmaM * 128) + 2u * j,
-                                          bd + 2u * j, C::kIdesc, acc);
-                    }
-                    umma_commit_both(smem_u32(&sh.a_empty[sa]));
-                    umma_commit_both(smem_u32(&sh.b_empty[sb]));
-                }
-                if (ok) {
-                    umma_commit_both(smem_u32(&sh.accum));
-                } else {  // the MMAs already issued finish before either CTA releases memory
-                    umma_commit_pair(smem_u32(&sh.drain));
-                    mbar_wait(smem_u32(&sh.drain), 0u, abort, true);
-                }
-            } else {
-                // ---- peer: forward "activation tile landed" to the leader ----
-                for (int kb = 0; kb < nk; ++kb) {
-                    const int sa = kb % C::kRingA;
-                    if (!mbar_wait(smem_u32(&sh.a_full[sa]), (uint32_t)(kb / C::kRingA) & 1u, abort)) {
-                        stop_pair(sh, a.ws, peer);
-                        break;
-                    }
-                    mbar_arrive_cluster(map_to(smem_u32(&sh.p_full[sa]), 0));
-                }
-            }
-        }
-        __syncwarp();
-    } else {
-        // ---- decode warps: this CTA's 128 weight rows, kTpr threads per row ----
-        const int t = threadIdx.x;
-        const int row = t / C::kTpr;
-        const int part = t % C::kTpr;
-        bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
-            const int sw = kb % C::kRingW, sb = kb % C::kRingB;
-            if (!warp_wait(smem_u32(&sh.w_full[sw]), (uint32_t)(kb / C::kRingW) & 1u, abort) ||
-                !warp_wait(smem_u32(&sh.b_empty[sb]), ((uint32_t)(kb / C::kRingB) & 1u) ^ 1u, abort)) {
-                if (lane == 0) stop_pair(sh, a.ws, peer);
-                ok = false;
-                break;
-            }
-            const uint8_t* rec = gW0 + sw * kRecBytes;
-            const uint2 v = *reinterpret_cast<const uint2*>(rec + row * 32 + part * 8);
-            const float sd = sh.sd[rec[kRecCodes + row * 4 + part]];
-            uint8_t* tile_row = gB0 + sb * C::kTileBBytes + row * 128;
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const uint32_t w = q ? v.y : v.x;
-                const uint32_t o0 = decode_pair(w & 0xFFu, sd), o1 = decode_pair((w >> 8) & 0xFFu, sd);
-                const uint32_t o2 = decode_pair((w >> 16) & 0xFFu, sd), o3 = decode_pair(w >> 24, sd);
-                const int chunk = 2 * part + q;
-                const uint32_t dst = smem_u32(tile_row + ((chunk ^ (row & 7)) << 4));
-                asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(o0), "r"(o1), "r"(o2), "r"(o3)
-                             : "memory");
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(smem_u32(&sh.w_empty[sw]));
-                mbar_arrive_cluster(map_to(smem_u32(&sh.b_full[sb]), 0));
-            }
-        }
-
-        // ---- epilogue: rows 256 h + 128 rank + 32 (w % 4) + lane, h = (w / 4) % 2; columns
-        //      128 (w / 8) .. + 127 ----
-        if (ok) {
-            if (!warp_wait(smem_u32(&sh.accum), 0u, abort)) {
-                if (lane == 0) stop_pair(sh, a.ws, peer);
-            } else {
-                tc_fence_after();
-                const int q = warp & 3, h = (warp >> 2) & 1, ch = warp >> 3;
-                const int64_t m = m0 + 2 * kMmaM * h + kMmaM * rank + 32 * q + lane;
-                const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(h * C::kBN);
-#pragma unroll 1
-                for (int j = 0; j < 8; ++j) {
-                    const int col0 = ch * 128 + 16 * j;
-                    uint32_t v[16];
-                    tmem_ld16(trow + (uint32_t)col0, v);
-                    const int64_t nc = n0 + col0;
-                    float f[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(v[e]);
-                    if (a.bias != nullptr) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            if (nc + e < a.N) f[e] = __fadd_rn(f[e], __uint_as_float((uint32_t)__ldg(a.bias + nc + e) << 16));
-                    }
-                    uint32_t o[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        __nv_bfloat162 hb = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
-                        o[e] = *reinterpret_cast<uint32_t*>(&hb);
-                    }
-                    if (m < a.M) {
-                        uint8_t* dst = a.y + (m * a.N + nc) * 2;
-                        if (a.vec_store && nc + 16 <= a.N) {
-                            st_b128(dst, o[0], o[1], o[2], o[3]);
-                            st_b128(dst + 16, o[4], o[5], o[6], o[7]);
-                        } else {
-                            for (int e = 0; e < 16; ++e)
-                                if (nc + e < a.N)
-                                    reinterpret_cast<uint16_t*>(dst)[e] = (uint16_t)(o[e >> 1] >> (16 * (e & 1)));
-                        }
-                    }
-                }
-            }
-        }
-    }
-
-    // ---- teardown: neither CTA leaves while the other may still read or signal its shared
-    //      memory (the leader's MMAs read the peer's tiles; both signal each other) ----
-    tc_fence_before();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        mbar_arrive_cluster(map_to(smem_u32(&sh.done), peer));
-        if (!mbar_wait(smem_u32(&sh.done), 0u, abort, true)) atomicExch(&a.ws->error, (unsigned)NVFP4_ERR_TIMEOUT);
-    }
-    __syncthreads();
-    if (warp == kMmaWarp) {
-        tc_fence_after();
-        tmem_dealloc2(tmem, C::kTmemCols);
-    }
-}
-
-// ---------------------------------------------------------------------------------------
 // Host side.
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -971,9 +599,7 @@ nvfp4_status gemm_smem_optin() {
             cudaFuncSetAttribute(w4a16_linear_kernel<128, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg<128, 2>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(w4a16_linear_kernel<128, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg<128, 1>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(w4a16_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 PairCfg::kSmemBytes) != cudaSuccess)
+                                 Cfg<128, 1>::kSmemBytes) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         g_smem_set[dev] = true;
     }
@@ -991,15 +617,6 @@ nvfp4_status sm_count_w4(int* out) {
 }
 
 bool is_aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
-
-// Pair kernel for large M unless NVFP4_W4A16_PAIR=0 (read once per process).
-bool pair_enabled() {
-    static const bool on = [] {
-        const char* v = std::getenv("NVFP4_W4A16_PAIR");
-        return !(v != nullptr && v[0] == '0');
-    }();
-    return on;
-}
 
 // Shapes the operand records accept: K a positive multiple of 16, sizes whose byte offsets
 // and TMA coordinates stay in range.
@@ -1045,15 +662,12 @@ NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, c
     if (M < 0 || !weight_shape_ok(N, K) || M > 0x7FFFFF00ll) return NVFP4_ERR_SHAPE;
     // Output tiles 256 x 256 when x has more than 256 rows, 256 x 128 for 129 to 256 rows,
     // 128 x 128 for at most 128.
-    // More than 256 rows of x: 512 x 256 tiles on pairs of SMs (the pair kernel), unless
-    // NVFP4_W4A16_PAIR=0 in the environment asks for the one-SM 256 x 256 tiles.
     const int acc = M > kMmaM ? 2 : 1;
     const int bm = kMmaM * acc;
     const int bn = M > 2 * kMmaM ? 256 : 128;
-    const bool pair = bn == 256 && pair_enabled();
-    const int64_t tiles_m = pair ? (M + PairCfg::kPairM - 1) / PairCfg::kPairM : (M + bm - 1) / bm;
+    const int64_t tiles_m = (M + bm - 1) / bm;
     const int64_t tiles_n = (N + bn - 1) / bn;
-    if (tiles_m * tiles_n * (pair ? 2 : 1) > 0x7FFFFFFFll) return NVFP4_ERR_SHAPE;
+    if (tiles_m * tiles_n > 0x7FFFFFFFll) return NVFP4_ERR_SHAPE;
     if (d_global_scale == nullptr || d_workspace == nullptr) return NVFP4_ERR_NULL;
     if (M > 0 && N > 0 && (x == nullptr || tiled == nullptr || y == nullptr)) return NVFP4_ERR_NULL;
     if (!is_aligned(d_global_scale, 4) || !is_aligned(d_workspace, 16)) return NVFP4_ERR_ALIGN;
@@ -1077,7 +691,7 @@ NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, c
     std::memset(&map, 0, sizeof(map));
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const int box_rows = pair ? kMmaM : (tiles_m == 1 ? (int)((M + 7) / 8 * 8) : bm);
+    const int box_rows = tiles_m == 1 ? (int)((M + 7) / 8 * 8) : bm;
     const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
@@ -1100,24 +714,6 @@ NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, c
     a.a_bytes = (uint32_t)box_rows * kBK * 2;
     const unsigned grid = (unsigned)(tiles_m * tiles_n);
     cudaStream_t cst = reinterpret_cast<cudaStream_t>(stream);
-    if (pair) {
-        cudaLaunchConfig_t cfg;
-        std::memset(&cfg, 0, sizeof(cfg));
-        cfg.gridDim = dim3(2 * grid, 1, 1);
-        cfg.blockDim = dim3(kGemmThreads, 1, 1);
-        cfg.dynamicSmemBytes = PairCfg::kSmemBytes;
-        cfg.stream = cst;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        const cudaError_t e = cudaLaunchKernelEx(&cfg, w4a16_pair_kernel, map, a);
-        note_launch();
-        return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
-    }
     if (bn == 256)
         w4a16_linear_kernel<256, 2><<<grid, kGemmThreads, Cfg<256, 2>::kSmemBytes, cst>>>(map, a);
     else if (acc == 2)
