@@ -474,6 +474,8 @@ def run_sweep(args):
             "fake_quant_with_own_amax": (4.0, timed(lambda: nv.nvfp4_fake_quant_fused(x, out=y, amax_out=amax,
                                                                                       workspace=ws))),
             "quantize": (2.5625, timed(lambda: nv.nvfp4_quantize(x, amax, packed, scales, gs))),
+            "quantize_with_own_amax": (2.5625, timed(lambda: nv.nvfp4_quantize_fused(x, packed, scales, gs, amax,
+                                                                                      workspace=ws))),
             "quantize_mma": (2.5625, timed(lambda: nv.nvfp4_quantize_mma(x, amax, packed, scales_mma, gs))),
             "dequantize": (2.5625, timed(lambda: nv.nvfp4_dequantize(packed, scales, gs, out=y))),
             # blocks of 32: 1/32 of a scale byte per element
@@ -497,8 +499,8 @@ def run_sweep(args):
                  "bytes": 2 * n, "siblings": {"us": sec * 1e6, "GB/s": n * 6.0 / sec / 1e9,
                                                "frac": n * 6.0 / sec / 1e9 / peak}})
 
-    cols = ["amax", "fake_quant", "fake_quant_with_own_amax", "quantize", "quantize_mma", "dequantize",
-            "fake_quant_b32", "quantize_b32", "dequantize_b32"]
+    cols = ["amax", "fake_quant", "fake_quant_with_own_amax", "quantize", "quantize_with_own_amax", "quantize_mma",
+            "dequantize", "fake_quant_b32", "quantize_b32", "dequantize_b32"]
     print(f"peak {peak:.1f} GB/s ({peak_src}); GB/s of algorithmic bytes (frac of peak); L2 flushed by a read")
     print("| workload | shape | " + " | ".join(cols) + " |")
     print("|---|---|" + "---|" * len(cols))

@@ -233,6 +233,19 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t N, const float* d_
 nvfp4_status nvfp4_quantize_mma(const void* x, int64_t M, int64_t N, const float* d_amax, uint8_t* packed,
                                 uint8_t* scales_mma, float* d_global_scale, nvfp4_stream_t stream);
 
+/* The whole of [FP4OPT] quantize_weight_to_float4 on a tensor: its own global amax, then
+ * nvfp4_quantize with it.  Up to twice the L2 size (and N % 16 == 0) this is one cooperative
+ * kernel that reads x from HBM once (the amax pass keeps x in L2 for the encode pass, behind a
+ * bounded grid barrier); otherwise one amax launch (through the workspace) and the quantize
+ * kernel.  Outputs as for nvfp4_quantize; codes, scale bytes and global scale identical.
+ *   d_amax       fp32 out: max |x| (0 for an empty tensor)
+ *   d_workspace  NVFP4_WORKSPACE_BYTES, zeroed before the first use, 16-byte aligned; one
+ *                call at a time per workspace.  A timeout of the grid barrier is reported by
+ *                nvfp4_workspace_check (the outputs are then unspecified).
+ * Other arguments, alignment and errors as for nvfp4_quantize. */
+nvfp4_status nvfp4_quantize_fused(const void* x, int64_t M, int64_t N, float* d_amax, uint8_t* packed,
+                                  uint8_t* scales, float* d_global_scale, void* d_workspace, nvfp4_stream_t stream);
+
 /* Dequantize: y = bf16_rne(LUT[code] * (E4M3(byte) / gs)), no clamp on this side.
  * [FP4OPT] dequantize_weight_from_float4.
  *   packed  uint8 [M, P/2], 8-byte aligned     scales  uint8 [M, P/16]

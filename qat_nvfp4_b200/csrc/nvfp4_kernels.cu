@@ -447,17 +447,20 @@ __global__ void __launch_bounds__(kThreads) fake_quant_kernel(FqList L, int64_t 
 }
 
 // ---------------------------------------------------------------------------------------
-// Fused amax -> fake-quant in one cooperative launch (all CTAs resident at once).
+// Fused amax -> fake-quant (kMode 0) or amax -> quantize (kMode 1) in one cooperative
+// launch (all CTAs resident at once).
 //   phase 1: each CTA reduces max |x| over its contiguous chunk, loading with an L2
 //            evict_last policy so that x stays in L2, and folds it into ws->acc;
 //   barrier: every CTA counts itself in ws->arrived and waits until all have (the wait is
 //            bounded by kBarrierTimeoutNs of %globaltimer; on timeout the CTA sets
 //            ws->error = NVFP4_ERR_TIMEOUT and returns without writing y);
 //   phase 2: every CTA forms the same global scale from the amax (after the observer
-//            step when asked) and fake-quantizes its chunk again, now mostly from L2; the
-//            last CTA to leave the barrier zeroes the workspace for the next call.
-// When x fits in L2 the HBM traffic is one read of x and one write of y (4 bytes per
-// element) instead of 6 for the amax kernel followed by the fake-quant kernel.
+//            step when asked) and fake-quantizes (or quantizes) its chunk again, now
+//            mostly from L2; the last CTA to leave the barrier zeroes the workspace for
+//            the next call.
+// When x fits in L2 the HBM traffic is one read of x and one write of the outputs (4
+// bytes per element for fake-quant, 2.5625 for quantize) instead of 2 bytes more for the
+// amax kernel followed by the second kernel.
 
 constexpr uint64_t kBarrierTimeoutNs = 2000000000ull;  // 2 s: far above any real wait
 
@@ -488,10 +491,20 @@ __device__ __forceinline__ void fill_scale_table(float4* tab, float gs) {
     __syncthreads();
 }
 
-template <bool kObserve>
+// Outputs of the fused kernel: y for fake-quant; packed, scales and (optionally) the
+// global scale for quantize.
+struct FusedOut {
+    uint8_t* y;
+    uint8_t* packed;
+    uint8_t* scales;
+    float* d_gs;
+};
+
+template <bool kObserve, int kMode>
 __global__ void __launch_bounds__(kThreads, 1024 / kThreads)
-    fused_fake_quant_kernel(const uint8_t* x, uint8_t* y, int64_t nblk, Workspace* ws, float* d_amax_out, float* state,
-                            int kind, float keep, float take, unsigned barrier_extra, uint64_t timeout_ns) {
+    fused_fake_quant_kernel(const uint8_t* x, FusedOut out, int64_t nblk, Workspace* ws, float* d_amax_out,
+                            float* state, int kind, float keep, float take, unsigned barrier_extra,
+                            uint64_t timeout_ns) {
     __shared__ float4 tab[128];
     __shared__ float s_amax;
     float state_old = 0.0f;
@@ -529,17 +542,30 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads)
     fill_scale_table(tab, gs);
 
     const uint64_t stream_out = l2_policy_evict_first();
-    stream_sched<1, kUnrollFq, false, Block32>(
-        nblk, [&](int64_t bi, Block32& b) { ld_b256_hint(x + bi * kBlockBytesIn, b.w, stream_out); },
-        [&](int64_t bi, Block32& b) {
-            uint32_t c[8];
-            float sd;
-            encode_block(b.w, gs, tab, c, sd);
-            uint32_t o[8];
+    if constexpr (kMode == 0) {
+        stream_sched<1, kUnrollFq, false, Block32>(
+            nblk, [&](int64_t bi, Block32& b) { ld_b256_hint(x + bi * kBlockBytesIn, b.w, stream_out); },
+            [&](int64_t bi, Block32& b) {
+                uint32_t c[8];
+                float sd;
+                encode_block(b.w, gs, tab, c, sd);
+                uint32_t o[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
-            st_b256_hint(y + bi * kBlockBytesIn, o, stream_out);
-        });
+                for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
+                st_b256_hint(out.y + bi * kBlockBytesIn, o, stream_out);
+            });
+    } else {
+        if (out.d_gs != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *out.d_gs = gs;
+        stream_sched<1, kUnrollFq, false, Block32>(
+            nblk, [&](int64_t bi, Block32& b) { ld_b256_hint(x + bi * kBlockBytesIn, b.w, stream_out); },
+            [&](int64_t bi, Block32& b) {
+                uint32_t c[8];
+                float sd;
+                const uint32_t s8 = encode_block(b.w, gs, tab, c, sd);
+                st_b64(out.packed + bi * kBlockBytesPacked, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
+                st_u8(out.scales + bi, s8);
+            });
+    }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -1034,11 +1060,13 @@ nvfp4_status l2_bytes(int64_t* out) {
 }
 
 // One cooperative launch of the fused kernel.  state == nullptr: plain amax.
-nvfp4_status launch_fused(const uint8_t* x, uint8_t* y, int64_t nblk, void* d_ws, float* d_amax_out, float* state,
-                          int kind, float keep, float take, unsigned barrier_extra, uint64_t timeout_ns,
+nvfp4_status launch_fused(const uint8_t* x, FusedOut out, int mode, int64_t nblk, void* d_ws, float* d_amax_out,
+                          float* state, int kind, float keep, float take, unsigned barrier_extra, uint64_t timeout_ns,
                           nvfp4_stream_t stream) {
-    const void* fn = state ? reinterpret_cast<const void*>(&fused_fake_quant_kernel<true>)
-                           : reinterpret_cast<const void*>(&fused_fake_quant_kernel<false>);
+    const void* fn = mode == 0 ? (state ? reinterpret_cast<const void*>(&fused_fake_quant_kernel<true, 0>)
+                                        : reinterpret_cast<const void*>(&fused_fake_quant_kernel<false, 0>))
+                               : (state ? reinterpret_cast<const void*>(&fused_fake_quant_kernel<true, 1>)
+                                        : reinterpret_cast<const void*>(&fused_fake_quant_kernel<false, 1>));
     int sms = 0, occ = 0;
     nvfp4_status st = sm_count(&sms);
     if (st != NVFP4_OK) return st;
@@ -1049,7 +1077,7 @@ nvfp4_status launch_fused(const uint8_t* x, uint8_t* y, int64_t nblk, void* d_ws
     const int64_t resident = (int64_t)sms * occ;
     int grid = (int)(need < 1 ? 1 : (need < resident ? need : resident));
     Workspace* ws = static_cast<Workspace*>(d_ws);
-    void* args[] = {(void*)&x, (void*)&y, (void*)&nblk, (void*)&ws, (void*)&d_amax_out, (void*)&state,
+    void* args[] = {(void*)&x, (void*)&out, (void*)&nblk, (void*)&ws, (void*)&d_amax_out, (void*)&state,
                     (void*)&kind, (void*)&keep, (void*)&take, (void*)&barrier_extra, (void*)&timeout_ns};
     if (cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kThreads), args, 0, cs(stream)) != cudaSuccess) {
         cudaGetLastError();
@@ -1270,8 +1298,8 @@ static nvfp4_status fake_quant_auto(const void* x, void* y, int64_t M, int64_t N
     if (st != NVFP4_OK) return st;
     const int64_t bytes = nblk * kBlockBytesIn;
     if ((double)bytes <= NVFP4_FUSED_MAX_FRACTION_OF_L2 * (double)l2)
-        return launch_fused(static_cast<const uint8_t*>(x), static_cast<uint8_t*>(y), nblk, d_ws, d_amax_out, state,
-                            kind, keep, take, 0u, kBarrierTimeoutNs, stream);
+        return launch_fused(static_cast<const uint8_t*>(x), FusedOut{static_cast<uint8_t*>(y), nullptr, nullptr, nullptr},
+                            0, nblk, d_ws, d_amax_out, state, kind, keep, take, 0u, kBarrierTimeoutNs, stream);
     AmaxList L;
     const void* xs[1] = {x};
     const int64_t ns[1] = {nblk * kBlockElems};
@@ -1338,8 +1366,8 @@ NVFP4_API nvfp4_status nvfp4_selftest_barrier_timeout(const void* x, void* y, in
     if (N % kBlockElems != 0) return NVFP4_ERR_SHAPE;
     if (nblk == 0 || timeout_us == 0 || timeout_us > 100000) return NVFP4_ERR_ARG;
     // One arrival more than the grid has: nothing ever completes the barrier.
-    return launch_fused(static_cast<const uint8_t*>(x), static_cast<uint8_t*>(y), nblk, d_workspace, d_amax, nullptr,
-                        0, 0.f, 0.f, 1u, (uint64_t)timeout_us * 1000ull, stream);
+    return launch_fused(static_cast<const uint8_t*>(x), FusedOut{static_cast<uint8_t*>(y), nullptr, nullptr, nullptr}, 0,
+                        nblk, d_workspace, d_amax, nullptr, 0, 0.f, 0.f, 1u, (uint64_t)timeout_us * 1000ull, stream);
 }
 
 template <bool kMma, int kW>
@@ -1456,6 +1484,37 @@ NVFP4_API nvfp4_status nvfp4_quantize_mma(const void* x, int64_t M, int64_t N, c
                                           uint8_t* scales_mma, float* d_global_scale, nvfp4_stream_t stream) {
     if (M > 0 && N > 0 && scales_mma != nullptr && !aligned(scales_mma, 16)) return NVFP4_ERR_ALIGN;
     return quantize_impl<true, 8>(x, M, N, d_amax, packed, scales_mma, d_global_scale, stream);
+}
+
+NVFP4_API nvfp4_status nvfp4_quantize_fused(const void* x, int64_t M, int64_t N, float* d_amax, uint8_t* packed,
+                                            uint8_t* scales, float* d_global_scale, void* d_workspace,
+                                            nvfp4_stream_t stream) {
+    int64_t numel = 0;
+    nvfp4_status st = check_matrix(M, N, &numel);
+    if (st != NVFP4_OK) return st;
+    if (d_amax == nullptr || d_workspace == nullptr) return NVFP4_ERR_NULL;
+    if (numel > 0 && (x == nullptr || packed == nullptr || scales == nullptr)) return NVFP4_ERR_NULL;
+    if (!aligned(d_amax, 4) || !aligned(d_workspace, 16) || (d_global_scale && !aligned(d_global_scale, 4)))
+        return NVFP4_ERR_ALIGN;
+    if (numel > 0 && (!aligned(x, 32) || !aligned(packed, 8))) return NVFP4_ERR_ALIGN;
+    const int64_t nblk = numel / kBlockElems;
+    if (N % kBlockElems == 0 && nblk > 0) {
+        int64_t l2 = 0;
+        st = l2_bytes(&l2);
+        if (st != NVFP4_OK) return st;
+        if ((double)(nblk * kBlockBytesIn) <= NVFP4_FUSED_MAX_FRACTION_OF_L2 * (double)l2)
+            return launch_fused(static_cast<const uint8_t*>(x), FusedOut{nullptr, packed, scales, d_global_scale}, 1,
+                                nblk, d_workspace, d_amax, nullptr, 0, 0.f, 0.f, 0u, kBarrierTimeoutNs, stream);
+    }
+    // Larger than the L2 rule, or rows of any length: the single-launch amax, then quantize.
+    AmaxList L;
+    const void* xs[1] = {x};
+    const int64_t ns[1] = {numel};
+    st = build_amax_list(xs, ns, 1, &L);
+    if (st != NVFP4_OK) return st;
+    st = launch_amax_ws(L, d_amax, d_workspace, nullptr, 0, 0.f, 0.f, stream);
+    if (st != NVFP4_OK) return st;
+    return quantize_impl<false, 8>(x, M, N, d_amax, packed, scales, d_global_scale, stream);
 }
 
 NVFP4_API nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* scales, const float* d_global_scale,

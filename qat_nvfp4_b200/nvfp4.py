@@ -60,6 +60,7 @@ _c_selftest_barrier_timeout = _sig("nvfp4_selftest_barrier_timeout",
                                    [_vp, _vp, _i64, _i64, _vp, _vp, ctypes.c_uint32, _vp])
 _c_quantize = _sig("nvfp4_quantize", [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp])
 _c_quantize_mma = _sig("nvfp4_quantize_mma", [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp])
+_c_quantize_fused = _sig("nvfp4_quantize_fused", [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp])
 _c_dequantize = _sig("nvfp4_dequantize", [_vp, _vp, _vp, _i64, _i64, _vp, _vp])
 _c_fake_quant = _sig("nvfp4_fake_quant", [_vp, _vp, _i64, _i64, _vp, _vp])
 _c_quantize_bs = _sig("nvfp4_quantize_bs", [_vp, _i64, _i64, ctypes.c_int, _vp, _vp, _vp, _vp, _vp])
@@ -260,6 +261,36 @@ def nvfp4_quantize(x: torch.Tensor, amax: torch.Tensor, packed: torch.Tensor | N
                                 global_scale.data_ptr(), _stream(x.device))
         _check(st, "nvfp4_quantize")
     return packed, scales, global_scale
+
+
+def nvfp4_quantize_fused(x: torch.Tensor, packed: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                         global_scale: torch.Tensor | None = None, amax_out: torch.Tensor | None = None,
+                         workspace: torch.Tensor | None = None):
+    """quantize_weight_to_float4 in one call: the tensor's own amax, then quantize with it
+    (one kernel launch up to twice the L2 size).  Returns (packed, scales, global scale,
+    amax)."""
+    M, N = _matrix(x)
+    B = padded_blocks(N)
+    lead = tuple(x.shape[:-1])
+    if packed is None:
+        packed = torch.empty(lead + (8 * B,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(lead + (B,), dtype=torch.uint8, device=x.device)
+    if global_scale is None:
+        global_scale = torch.empty(1, dtype=torch.float32, device=x.device)
+    if amax_out is None:
+        amax_out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _cuda(packed, "packed", torch.uint8)
+    _cuda(scales, "scales", torch.uint8)
+    _scalar(global_scale, "global_scale")
+    _scalar(amax_out, "amax_out")
+    if packed.numel() != M * 8 * B or scales.numel() != M * B:
+        raise RuntimeError("packed / scales have the wrong number of elements")
+    ws = new_workspace(x.device) if workspace is None else _workspace(workspace, x.device)
+    with torch.cuda.device(x.device):
+        _check(_c_quantize_fused(x.data_ptr(), M, N, amax_out.data_ptr(), packed.data_ptr(), scales.data_ptr(),
+                                 global_scale.data_ptr(), ws.data_ptr(), _stream(x.device)), "nvfp4_quantize_fused")
+    return packed, scales, global_scale, amax_out
 
 
 def mma_scale_bytes(M: int, N: int) -> int:

@@ -32,7 +32,7 @@ def test_header_declares_the_entry_points():
     for required in ["nvfp4_amax", "nvfp4_amax_multi", "nvfp4_observer_update", "nvfp4_observe_amax",
                      "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fake_quant", "nvfp4_fake_quant_siblings",
                      "nvfp4_quantize_bs", "nvfp4_dequantize_bs", "nvfp4_fake_quant_bs", "nvfp4_w4a16_linear",
-                     "nvfp4_w4a16_pack", "nvfp4_w4a16_tiled_bytes",
+                     "nvfp4_w4a16_pack", "nvfp4_w4a16_tiled_bytes", "nvfp4_quantize_fused",
                      "nvfp4_status_string", "nvfp4_kernel_launch_count"]:
         assert required in names
 
@@ -140,6 +140,10 @@ def test_validation_errors_launch_nothing(lib):
         (ERR_NULL, "nvfp4_w4a16_pack", _p(A32), _p(0), _i(8), _i(64), _p(A32), S),
         (ERR_ALIGN, "nvfp4_w4a16_pack", _p(A32), _p(A32), _i(8), _i(64), _p(A8), S),
         (NVFP4_OK, "nvfp4_w4a16_pack", _p(0), _p(0), _i(0), _i(64), _p(0), S),
+        # fused quantize: x, M, N, amax, packed, scales, gs, workspace
+        (ERR_NULL, "nvfp4_quantize_fused", _p(A32), _i(2), _i(16), amax, _p(A32), _p(A32), gs, _p(0), S),
+        (ERR_ALIGN, "nvfp4_quantize_fused", _p(A32), _i(2), _i(16), amax, _p(A32), _p(A32), gs, _p(A32 + 8), S),
+        (ERR_SHAPE, "nvfp4_quantize_fused", _p(A32), _i(-2), _i(16), amax, _p(A32), _p(A32), gs, _p(A32), S),
         # amax
         (ERR_NULL, "nvfp4_amax", _p(A32), _i(16), _p(0), S),
         (ERR_NULL, "nvfp4_amax", _p(0), _i(16), amax, S),

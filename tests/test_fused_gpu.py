@@ -7,7 +7,8 @@ import torch
 
 import oracle
 from qat_nvfp4_b200 import synthetic
-from nvfp4_testutil import assert_equal_bits, bits, f32_bits, oracle_fake_quant_rows, sample_rows, scalar, to_dev
+from nvfp4_testutil import (assert_equal_bits, bits, f32_bits, oracle_fake_quant_rows, oracle_quantize_rows,
+                            sample_rows, scalar, to_dev, u8)
 
 pytestmark = pytest.mark.gpu
 
@@ -69,3 +70,30 @@ def test_barrier_wait_gives_up_and_context_stays_usable():
     assert nv.nvfp4_workspace_check(ws) == 0
     y, a = nv.nvfp4_fake_quant_fused(xd, workspace=ws)
     assert_equal_bits(bits(y), oracle_fake_quant_rows(x, oracle.amax(x)), "after a timeout")
+
+
+# ---- fused amax -> quantize (quantize_weight_to_float4 in one call) -----------------------
+
+@pytest.mark.parametrize("shape,seed", [((256, 1024), 1), ((4096, 4096), 2), ((1024, 4096), 3), ((7, 48), 4),
+                                        ((3, 20), 5), ((16384, 8192), 6), ((0, 64), 7)])
+def test_quantize_fused_matches_oracle(shape, seed):
+    """Small, page-sized (4096 x 4096 weight), ragged (N % 16 != 0: amax + quantize
+    launches), larger than twice L2 (16384 x 8192 bf16 = 256 MiB: the same two launches)
+    and empty tensors; codes, scale bytes, global scale and amax bit for bit.  The
+    workspace is reused across calls."""
+    M, N = shape
+    x = synthetic.activation_normal((M, N), 500 + seed)
+    xd = to_dev(x)
+    ws = nv.new_workspace("cuda")
+    for _ in range(2):
+        packed, scales, gs, a = nv.nvfp4_quantize_fused(xd, workspace=ws)
+    assert nv.nvfp4_workspace_check(ws) == 0
+    want_a = oracle.amax(x) if x.size else 0.0
+    assert f32_bits(a) == f32_bits(want_a)
+    assert f32_bits(gs) == f32_bits(oracle.global_scale(want_a))
+    if M * N == 0:
+        return
+    rows = np.arange(M) if M <= 4096 else sample_rows(M, 48, seed=seed)
+    want_p, want_s = oracle_quantize_rows(x[rows], oracle.global_scale(want_a))
+    assert_equal_bits(u8(packed)[rows], want_p, f"{shape}: packed")
+    assert_equal_bits(u8(scales)[rows], want_s, f"{shape}: scales")
