@@ -558,7 +558,8 @@ def run_linear(args):
         for M in (1, 16, 128, 1024, 4096, 8192):
             x = synthetic.activation_normal_device((M, K), 8 + M, dev)
             y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-            t_fused = timed(lambda: nv.nvfp4_w4a16_linear(x, tiled, gs, N, out=y, workspace=ws))
+            lws = nv.nvfp4_w4a16_workspace(M, N, K, dev)
+            t_fused = timed(lambda: nv.nvfp4_w4a16_linear(x, tiled, gs, N, out=y, workspace=lws))
             t_pages = timed(lambda: (nv.nvfp4_dequantize(packed, scales, gs, out=wbuf), torch.matmul(x, wbuf.t(), out=y)))
             t_bf16 = timed(lambda: torch.matmul(x, w.t(), out=y))
             flops = 2.0 * M * N * K
@@ -596,11 +597,11 @@ def run_linear_shape(args):
     w = synthetic.activation_normal_device((N, K), 2, dev) * 0.02
     packed, scales, gs = nv.nvfp4_quantize(w, nv.nvfp4_amax(w))
     tiled = nv.nvfp4_w4a16_pack(packed, scales)
-    ws = nv.new_workspace(dev)
+    ws = nv.nvfp4_w4a16_workspace(M, N, K, dev)
     for _ in range(3):
         y = nv.nvfp4_w4a16_linear(x, tiled, gs, N, workspace=ws)
     torch.cuda.synchronize(dev)
-    if nv.nvfp4_workspace_check(ws) != 0:
+    if nv.nvfp4_workspace_check(ws[:nv.WORKSPACE_BYTES]) != 0:
         raise SystemExit("W4A16 linear reported a timeout")
     print(json.dumps({"linear_shape": [M, K, N], "y_abs_mean": float(y.float().abs().mean())}))
     return 0

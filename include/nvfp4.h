@@ -80,6 +80,13 @@ typedef enum {
  * Enqueues a 4-byte memset and one kernel. */
 nvfp4_status nvfp4_amax(const void* x, int64_t numel, float* d_amax, nvfp4_stream_t stream);
 
+/* Running amax: *d_amax = max(*d_amax, max |x_i|), for folding several tensors (or the
+ * shards of one) into one amax call by call.  *d_amax must hold a non-negative fp32 value
+ * on entry (0 to start); the maximum is taken on the fp32 bit patterns, which order like
+ * the values for non-negative floats.  numel == 0 leaves *d_amax unchanged and launches
+ * nothing.  Arguments and errors as for nvfp4_amax.  Enqueues one kernel, no memset. */
+nvfp4_status nvfp4_amax_accumulate(const void* x, int64_t numel, float* d_amax, nvfp4_stream_t stream);
+
 /* Fused-siblings amax: *d_amax = max over the k tensors of max |x|, so that layers fused
  * into one GEMM (q/k/v) share one global scale.  [QATLIN] section 4
  * (max(stack([m.weight.abs().max() for m in [self] + siblings]))).
@@ -334,15 +341,27 @@ nvfp4_status nvfp4_w4a16_pack(const uint8_t* packed, const uint8_t* scales, int6
  *   bias    bf16 [N] or NULL
  *   y       bf16 out [M, N] row-major, 2-byte aligned (16-byte aligned with N % 8 == 0 is
  *           faster); must not overlap the inputs
- *   d_workspace  a workspace as above: a bounded wait inside the kernel that runs out
- *           records NVFP4_ERR_TIMEOUT there (nvfp4_workspace_check), the kernel stops and y is
- *           unspecified.  The call does not otherwise use it.
+ *   d_workspace, workspace_bytes  device memory, 256-byte aligned, zeroed before its first
+ *           use, of workspace_bytes >= NVFP4_WORKSPACE_BYTES bytes; one call at a time per
+ *           workspace.  Its first NVFP4_WORKSPACE_BYTES are a workspace as above: a bounded
+ *           wait inside the kernel that runs out records NVFP4_ERR_TIMEOUT there
+ *           (nvfp4_workspace_check; zero the whole workspace before reusing it then), the
+ *           kernel stops and y is unspecified.  With at least nvfp4_w4a16_workspace_bytes(M,
+ *           N, K) bytes, a call with at most 128 rows of x may split K over several CTAs per
+ *           output tile: each writes fp32 partial sums there and the last to finish adds them
+ *           in a fixed order (so results do not depend on timing) and leaves its counter at
+ *           zero again.  With less, K is not split.
  * Errors: NVFP4_ERR_SHAPE (K, sizes past the 32-bit tensor-map limits), NVFP4_ERR_NULL,
- * NVFP4_ERR_ALIGN, NVFP4_ERR_ARG (tensor map rejected).  M == 0 or N == 0 launches nothing.
- * Enqueues one kernel. */
+ * NVFP4_ERR_ALIGN, NVFP4_ERR_ARG (tensor map rejected, workspace_bytes too small).  M == 0 or
+ * N == 0 launches nothing.  Enqueues one kernel. */
 nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* tiled,
                                 const float* d_global_scale, int64_t N, const void* bias, void* y,
-                                void* d_workspace, nvfp4_stream_t stream);
+                                void* d_workspace, int64_t workspace_bytes, nvfp4_stream_t stream);
+
+/* Workspace bytes with which nvfp4_w4a16_linear may split K for this shape (at least
+ * NVFP4_WORKSPACE_BYTES; -1 for a shape it refuses).  Depends on the current device's SM
+ * count. */
+int64_t nvfp4_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* Human-readable name of a status code (a static string). */
 const char* nvfp4_status_string(nvfp4_status status);

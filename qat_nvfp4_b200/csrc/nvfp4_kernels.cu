@@ -1015,8 +1015,8 @@ bool overlap(const void* a, const void* b, int64_t bytes) {
 
 
 // Enqueue memset + amax kernel over an already validated list.
-nvfp4_status launch_amax(const AmaxList& L, float* d_amax, nvfp4_stream_t stream) {
-    if (cudaMemsetAsync(d_amax, 0, sizeof(float), cs(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
+nvfp4_status launch_amax(const AmaxList& L, float* d_amax, nvfp4_stream_t stream, bool accumulate = false) {
+    if (!accumulate && cudaMemsetAsync(d_amax, 0, sizeof(float), cs(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
     const int64_t units = L.full_end[L.k - 1];
     int grid = 1;
     nvfp4_status st = grid_for(reinterpret_cast<const void*>(&amax_kernel), units, kUnrollAmax, NVFP4_GRID_AMAX, &grid);
@@ -1138,6 +1138,18 @@ NVFP4_API nvfp4_status nvfp4_amax(const void* x, int64_t numel, float* d_amax, n
     nvfp4_status st = build_amax_list(xs, ns, 1, &L);
     if (st != NVFP4_OK) return st;
     return launch_amax(L, d_amax, stream);
+}
+
+NVFP4_API nvfp4_status nvfp4_amax_accumulate(const void* x, int64_t numel, float* d_amax, nvfp4_stream_t stream) {
+    if (d_amax == nullptr) return NVFP4_ERR_NULL;
+    if (!aligned(d_amax, 4)) return NVFP4_ERR_ALIGN;
+    AmaxList L;
+    const void* xs[1] = {x};
+    const int64_t ns[1] = {numel};
+    nvfp4_status st = build_amax_list(xs, ns, 1, &L);
+    if (st != NVFP4_OK) return st;
+    if (numel == 0) return NVFP4_OK;  // max(*d_amax, nothing) leaves it as it is
+    return launch_amax(L, d_amax, stream, true);
 }
 
 NVFP4_API nvfp4_status nvfp4_amax_multi(const void* const* xs, const int64_t* numels, int k, float* d_amax,

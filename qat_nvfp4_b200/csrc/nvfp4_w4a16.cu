@@ -98,6 +98,7 @@ struct Cfg {
         uint64_t drain;            // used only when stopping early
         uint32_t tmem_base;
         uint32_t abort;
+        uint32_t last;             // split K: this CTA finishes the tile
         float sd[256];             // decode scale for every E4M3 byte: fl(E4M3(b) / gs)
     };
     static constexpr int kRingBytes = kRingA * kTileABytes + kRingB * kTileBBytes + kRingW * kRecPerTile * kRecBytes;
@@ -303,7 +304,36 @@ struct LinearArgs {
     int64_t kt;             // records per weight row of tiles = ceil(K / 64)
     uint32_t a_bytes;       // bytes of one activation box (rows loaded per stage x 128)
     int vec_store;          // rows of y allow 16-byte stores
+    int splits;             // CTAs per output tile, each over a contiguous share of the K stages
+    unsigned* counters;     // splits > 1: per output tile, CTAs done (the last one resets it)
+    float* partial;         // splits > 1: fp32 partial sums [splits][output tiles][128 columns][128
+                            // rows] (rows fastest: a warp's 32 rows are 128 contiguous bytes)
 };
+
+// Output row m, columns nc .. nc + 15: add the bias, round to bf16 once, store the columns
+// that exist.
+__device__ __forceinline__ void store_out16(const LinearArgs& a, int64_t m, int64_t nc, float (&f)[16]) {
+    if (a.bias != nullptr) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            if (nc + e < a.N) f[e] = __fadd_rn(f[e], __uint_as_float((uint32_t)__ldg(a.bias + nc + e) << 16));
+    }
+    uint32_t o[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+        o[e] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    if (m >= a.M) return;
+    uint8_t* dst = a.y + (m * a.N + nc) * 2;
+    if (a.vec_store && nc + 16 <= a.N) {
+        st_b128(dst, o[0], o[1], o[2], o[3]);
+        st_b128(dst + 16, o[4], o[5], o[6], o[7]);
+    } else {
+        for (int e = 0; e < 16; ++e)
+            if (nc + e < a.N) reinterpret_cast<uint16_t*>(dst)[e] = (uint16_t)(o[e >> 1] >> (16 * (e & 1)));
+    }
+}
 
 template <class Sh>
 __device__ __forceinline__ void stop_all(Sh& sh, Workspace* ws) {
@@ -337,9 +367,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint8_t* gW0 = gB0 + kRingB * kTileBBytes;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t tm = (int64_t)blockIdx.x / a.tiles_n, tn = (int64_t)blockIdx.x % a.tiles_n;
+    const int64_t tile = (int64_t)blockIdx.x / a.splits;
+    const int sp = (int)((int64_t)blockIdx.x % a.splits);
+    const int64_t tm = tile / a.tiles_n, tn = tile % a.tiles_n;
     const int64_t m0 = tm * kBM, n0 = tn * kBN;
-    const int nk = (int)a.kt;
+    // this CTA's K stages: [kb0, kb0 + nk); stage i of the loops below is kb0 + i
+    const int kb0 = (int)((int64_t)sp * a.kt / a.splits);
+    const int nk = (int)((int64_t)(sp + 1) * a.kt / a.splits) - kb0;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kRingA; ++s) {
@@ -396,15 +430,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const uint32_t bar = smem_u32(&full[s]);
                 if (act) {
                     mbar_arrive_expect_tx(bar, a.a_bytes);
-                    tma_load_2d(sA0 + s * kTileABytes, &tmap_x, kb * kBK, (int32_t)m0, bar);
+                    tma_load_2d(sA0 + s * kTileABytes, &tmap_x, (kb0 + kb) * kBK, (int32_t)m0, bar);
                 } else {
                     mbar_arrive_expect_tx(bar, kRecPerTile * kRecBytes);
 #pragma unroll
                     for (int i = 0; i < kRecPerTile; ++i) {
                         int64_t rn = kRecPerTile * tn + i;
                         if (rn >= nrec) rn = nrec - 1;
-                        bulk_load(sW0 + (s * kRecPerTile + i) * kRecBytes, a.tiled + (rn * a.kt + kb) * kRecBytes,
-                                  kRecBytes, bar);
+                        bulk_load(sW0 + (s * kRecPerTile + i) * kRecBytes,
+                                  a.tiled + (rn * a.kt + kb0 + kb) * kRecBytes, kRecBytes, bar);
                     }
                 }
                 ++issued;
@@ -527,28 +561,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     float f[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(v[e]);
-                    if (a.bias != nullptr) {
+                    if (a.splits == 1) {
+                        store_out16(a, m, nc, f);
+                    } else if (m < a.M) {  // this split's fp32 partial sums
+                        float* dst = a.partial + (((int64_t)sp * a.tiles_n + tile) * kBN + col0) * kMmaM + (m - m0);
 #pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            if (nc + e < a.N) f[e] = __fadd_rn(f[e], __uint_as_float((uint32_t)__ldg(a.bias + nc + e) << 16));
+                        for (int e = 0; e < 16; ++e) __stcg(dst + e * kMmaM, f[e]);
                     }
-                    uint32_t o[8];
+                }
+            }
+        }
+    }
+
+    // ---- split K: the last CTA of the tile to finish adds the partial sums of all splits
+    //      in split order (the same order whichever CTA that is), then resets the tile's
+    //      counter for the next call ----
+    if (a.splits > 1) {
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const unsigned prev = atomicAdd(a.counters + tile, 1u);
+            sh.last = prev == (unsigned)(a.splits - 1) ? 1u : 0u;
+            if (sh.last) atomicExch(a.counters + tile, 0u);
+        }
+        __syncthreads();
+        if (sh.last && !*abort && warp < kDecodeWarps) {
+            __threadfence();
+            constexpr int kCols = kBN / C::kColParts;
+            const int q = warp & 3, acc = (warp >> 2) % ACC, ch = warp / (4 * ACC);
+            const int64_t m = m0 + kMmaM * acc + 32 * q + lane;
+            if (m < a.M) {
+                for (int j = 0; j < kCols / 16; ++j) {
+                    const int col0 = ch * kCols + 16 * j;
+                    float f[16];
+                    for (int k = 0; k < a.splits; ++k) {
+                        const float* src =
+                            a.partial + (((int64_t)k * a.tiles_n + tile) * kBN + col0) * kMmaM + (m - m0);
+                        float v[16];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
-                        o[e] = *reinterpret_cast<uint32_t*>(&h);
+                        for (int e = 0; e < 16; ++e) v[e] = __ldcg(src + e * kMmaM);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) f[e] = k == 0 ? v[e] : __fadd_rn(f[e], v[e]);
                     }
-                    if (m < a.M) {
-                        uint8_t* dst = a.y + (m * a.N + nc) * 2;
-                        if (a.vec_store && nc + 16 <= a.N) {
-                            st_b128(dst, o[0], o[1], o[2], o[3]);
-                            st_b128(dst + 16, o[4], o[5], o[6], o[7]);
-                        } else {
-                            for (int e = 0; e < 16; ++e)
-                                if (nc + e < a.N)
-                                    reinterpret_cast<uint16_t*>(dst)[e] = (uint16_t)(o[e >> 1] >> (16 * (e & 1)));
-                        }
-                    }
+                    store_out16(a, m, n0 + col0, f);
                 }
             }
         }
@@ -628,6 +683,28 @@ int64_t record_bytes(int64_t N, int64_t K) {
     return ((N + kRecRows - 1) / kRecRows) * ((K + kBK - 1) / kBK) * (int64_t)kRecBytes;
 }
 
+// Split K for at most 128 rows of x: enough CTAs per 128-column tile to fill the SMs (one
+// CTA per SM), each with at least 8 K stages.
+int split_count(int64_t M, int64_t N, int64_t K, int sms) {
+    if (M > kMmaM) return 1;
+    const int64_t tiles = (N + 127) / 128;
+    const int64_t kt = (K + kBK - 1) / kBK;
+    int64_t s = sms / (tiles > 0 ? tiles : 1);
+    if (s > kt / 8) s = kt / 8;
+    if (s > 16) s = 16;
+    return s < 2 ? 1 : (int)s;
+}
+
+// Workspace layout for `splits` > 1: the status block, one counter per output tile, the
+// fp32 partial sums [splits][tiles][128][128] (256-byte aligned).
+int64_t counters_offset() { return (int64_t)sizeof(Workspace); }
+int64_t partial_offset(int64_t tiles) { return ((int64_t)sizeof(Workspace) + 4 * tiles + 255) / 256 * 256; }
+int64_t split_workspace_bytes(int64_t M, int64_t N, int splits) {
+    (void)M;
+    const int64_t tiles = (N + 127) / 128;
+    return partial_offset(tiles) + (int64_t)splits * tiles * 128 * 128 * 4;
+}
+
 }  // namespace
 }  // namespace nvfp4
 
@@ -656,9 +733,17 @@ NVFP4_API nvfp4_status nvfp4_w4a16_pack(const uint8_t* packed, const uint8_t* sc
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+NVFP4_API int64_t nvfp4_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    if (M < 0 || !weight_shape_ok(N, K)) return -1;
+    int sms = 0;
+    if (sm_count_w4(&sms) != NVFP4_OK) sms = 148;
+    const int splits = split_count(M, N, K, sms);
+    return splits > 1 ? split_workspace_bytes(M, N, splits) : (int64_t)sizeof(Workspace);
+}
+
 NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* tiled,
                                           const float* d_global_scale, int64_t N, const void* bias, void* y,
-                                          void* d_workspace, nvfp4_stream_t stream) {
+                                          void* d_workspace, int64_t workspace_bytes, nvfp4_stream_t stream) {
     if (M < 0 || !weight_shape_ok(N, K) || M > 0x7FFFFF00ll) return NVFP4_ERR_SHAPE;
     // Output tiles 256 x 256 when x has more than 256 rows, 256 x 128 for 129 to 256 rows,
     // 128 x 128 for at most 128.
@@ -670,7 +755,8 @@ NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, c
     if (tiles_m * tiles_n > 0x7FFFFFFFll) return NVFP4_ERR_SHAPE;
     if (d_global_scale == nullptr || d_workspace == nullptr) return NVFP4_ERR_NULL;
     if (M > 0 && N > 0 && (x == nullptr || tiled == nullptr || y == nullptr)) return NVFP4_ERR_NULL;
-    if (!is_aligned(d_global_scale, 4) || !is_aligned(d_workspace, 16)) return NVFP4_ERR_ALIGN;
+    if (!is_aligned(d_global_scale, 4) || !is_aligned(d_workspace, 256)) return NVFP4_ERR_ALIGN;
+    if (workspace_bytes < (int64_t)sizeof(Workspace)) return NVFP4_ERR_ARG;
     if (M > 0 && N > 0 &&
         (!is_aligned(x, 16) || !is_aligned(tiled, 16) || !is_aligned(y, 2) || (bias && !is_aligned(bias, 2))))
         return NVFP4_ERR_ALIGN;
@@ -712,7 +798,15 @@ NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, c
     a.kt = (K + kBK - 1) / kBK;
     a.vec_store = (is_aligned(y, 16) && N % 8 == 0) ? 1 : 0;
     a.a_bytes = (uint32_t)box_rows * kBK * 2;
-    const unsigned grid = (unsigned)(tiles_m * tiles_n);
+    // split K only with a workspace large enough for the partial sums
+    int sms = 0;
+    st = sm_count_w4(&sms);
+    if (st != NVFP4_OK) return st;
+    a.splits = acc == 1 ? split_count(M, N, K, sms) : 1;
+    if (a.splits > 1 && workspace_bytes < split_workspace_bytes(M, N, a.splits)) a.splits = 1;
+    a.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(d_workspace) + counters_offset());
+    a.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(d_workspace) + partial_offset(tiles_n));
+    const unsigned grid = (unsigned)(tiles_m * tiles_n * a.splits);
     cudaStream_t cst = reinterpret_cast<cudaStream_t>(stream);
     if (bn == 256)
         w4a16_linear_kernel<256, 2><<<grid, kGemmThreads, Cfg<256, 2>::kSmemBytes, cst>>>(map, a);

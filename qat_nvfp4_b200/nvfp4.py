@@ -47,6 +47,7 @@ def _sig(name, args, res=_status):
 
 
 _c_amax = _sig("nvfp4_amax", [_vp, _i64, _vp, _vp])
+_c_amax_accumulate = _sig("nvfp4_amax_accumulate", [_vp, _i64, _vp, _vp])
 _c_amax_multi = _sig("nvfp4_amax_multi", [ctypes.POINTER(_vp), ctypes.POINTER(_i64), ctypes.c_int, _vp, _vp])
 _c_observer_update = _sig("nvfp4_observer_update", [_vp, _vp, ctypes.c_int, ctypes.c_double, _vp])
 _c_observe_amax = _sig("nvfp4_observe_amax", [_vp, _i64, _vp, ctypes.c_int, ctypes.c_double, _vp, _vp])
@@ -71,7 +72,8 @@ _c_fake_quant_siblings = _sig("nvfp4_fake_quant_siblings",
                                ctypes.POINTER(_i64), _vp, _vp])
 _c_w4a16_tiled_bytes = _sig("nvfp4_w4a16_tiled_bytes", [_i64, _i64], _i64)
 _c_w4a16_pack = _sig("nvfp4_w4a16_pack", [_vp, _vp, _i64, _i64, _vp, _vp])
-_c_w4a16_linear = _sig("nvfp4_w4a16_linear", [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _vp])
+_c_w4a16_linear = _sig("nvfp4_w4a16_linear", [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _vp])
+_c_w4a16_workspace_bytes = _sig("nvfp4_w4a16_workspace_bytes", [_i64, _i64, _i64], _i64)
 _c_status_string = _sig("nvfp4_status_string", [ctypes.c_int], ctypes.c_char_p)
 _c_launch_count = _sig("nvfp4_kernel_launch_count", [], ctypes.c_uint64)
 
@@ -168,6 +170,19 @@ def nvfp4_amax(x: torch.Tensor, out: torch.Tensor | None = None,
             _check(_c_amax_ws(x.data_ptr(), x.numel(), out.data_ptr(), workspace.data_ptr(), _stream(x.device)),
                    "nvfp4_amax_ws")
     return out
+
+
+def nvfp4_amax_accumulate(x: torch.Tensor, running: torch.Tensor) -> torch.Tensor:
+    """running <- max(running, max |x|) on the device; running is a 1-element fp32 CUDA
+    tensor holding a non-negative value (0 to start)."""
+    _cuda(x, "x", torch.bfloat16)
+    if not x.is_contiguous():
+        raise RuntimeError("x must be contiguous")
+    _scalar(running, "running")
+    with torch.cuda.device(x.device):
+        _check(_c_amax_accumulate(x.data_ptr(), x.numel(), running.data_ptr(), _stream(x.device)),
+               "nvfp4_amax_accumulate")
+    return running
 
 
 def nvfp4_amax_multi(xs: Sequence[torch.Tensor], out: torch.Tensor | None = None) -> torch.Tensor:
@@ -518,12 +533,30 @@ def nvfp4_w4a16_linear(x: torch.Tensor, tiled: torch.Tensor, global_scale: torch
     _cuda(out, "out", torch.bfloat16)
     if out.numel() != M * N:
         raise RuntimeError("out has the wrong number of elements")
-    ws = new_workspace(x.device) if workspace is None else _workspace(workspace, x.device)
     with torch.cuda.device(x.device):
+        if workspace is None:
+            workspace = nvfp4_w4a16_workspace(M, N, K, x.device)
+        ws = _workspace(workspace, x.device)
         _check(_c_w4a16_linear(x.data_ptr(), M, K, tiled.data_ptr(), global_scale.data_ptr(), N,
                                bias.data_ptr() if bias is not None else None, out.data_ptr(), ws.data_ptr(),
-                               _stream(x.device)), "nvfp4_w4a16_linear")
+                               ws.numel(), _stream(x.device)), "nvfp4_w4a16_linear")
     return out
+
+
+def nvfp4_w4a16_workspace_bytes(M: int, N: int, K: int) -> int:
+    """Workspace bytes with which nvfp4_w4a16_linear may split K on this shape (current
+    device), at least WORKSPACE_BYTES; -1 if the shape is refused."""
+    return int(_c_w4a16_workspace_bytes(M, N, K))
+
+
+def nvfp4_w4a16_workspace(M: int, N: int, K: int, device) -> torch.Tensor:
+    """A zeroed workspace large enough for nvfp4_w4a16_linear to split K on this shape
+    (reusable across calls of the same or smaller shape, one call at a time)."""
+    with torch.cuda.device(device):
+        nbytes = int(_c_w4a16_workspace_bytes(M, N, K))
+    if nbytes < 0:
+        raise RuntimeError(f"linear shape M={M}, N={N}, K={K} not accepted")
+    return torch.zeros(max(nbytes, WORKSPACE_BYTES), dtype=torch.uint8, device=device)
 
 
 class FakeQuantSTE(torch.autograd.Function):

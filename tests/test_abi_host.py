@@ -33,6 +33,7 @@ def test_header_declares_the_entry_points():
                      "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fake_quant", "nvfp4_fake_quant_siblings",
                      "nvfp4_quantize_bs", "nvfp4_dequantize_bs", "nvfp4_fake_quant_bs", "nvfp4_w4a16_linear",
                      "nvfp4_w4a16_pack", "nvfp4_w4a16_tiled_bytes", "nvfp4_quantize_fused",
+                     "nvfp4_amax_accumulate", "nvfp4_w4a16_workspace_bytes",
                      "nvfp4_status_string", "nvfp4_kernel_launch_count"]:
         assert required in names
 
@@ -128,14 +129,17 @@ def test_validation_errors_launch_nothing(lib):
         (ERR_SHAPE, "nvfp4_fake_quant_bs", _p(A32), _p(A32 + 4096), _i(2), _i(-32), _c(32), amax, S),
         (ERR_NULL, "nvfp4_fake_quant_bs", _p(A32), _p(A32 + 4096), _i(2), _i(64), _c(32), _p(0), S),
         # W4A16: linear(x, M, K, tiled, gs, N, bias, y, workspace), pack(packed, scales, N, K, tiled)
-        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(24), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), S),
-        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(0), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), S),
-        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(-1), _i(64), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), S),
-        (ERR_NULL, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(A32), gs, _i(8), _p(0), _p(A32), _p(0), S),
-        (ERR_NULL, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(0), gs, _i(8), _p(0), _p(A32), _p(A32), S),
-        (ERR_ALIGN, "nvfp4_w4a16_linear", _p(A8), _i(4), _i(64), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), S),
-        (ERR_ALIGN, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(A8), gs, _i(8), _p(0), _p(A32), _p(A32), S),
-        (NVFP4_OK, "nvfp4_w4a16_linear", _p(0), _i(0), _i(64), _p(0), gs, _i(8), _p(0), _p(0), _p(A32), S),
+        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(24), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), _i(256), S),
+        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(0), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), _i(256), S),
+        (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(-1), _i(64), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), _i(256), S),
+        (ERR_NULL, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(A32), gs, _i(8), _p(0), _p(A32), _p(0), _i(256), S),
+        (ERR_NULL, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(0), gs, _i(8), _p(0), _p(A32), _p(A32), _i(256), S),
+        (ERR_ALIGN, "nvfp4_w4a16_linear", _p(A8), _i(4), _i(64), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), _i(256), S),
+        (ERR_ALIGN, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(A8), gs, _i(8), _p(0), _p(A32), _p(A32), _i(256), S),
+        (NVFP4_OK, "nvfp4_w4a16_linear", _p(0), _i(0), _i(64), _p(0), gs, _i(8), _p(0), _p(0), _p(A32), _i(256), S),
+        (ERR_ARG, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), _i(64), S),
+        (ERR_ALIGN, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(64), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32 + 128),
+         _i(256), S),
         (ERR_SHAPE, "nvfp4_w4a16_pack", _p(A32), _p(A32), _i(8), _i(40), _p(A32), S),
         (ERR_NULL, "nvfp4_w4a16_pack", _p(A32), _p(0), _i(8), _i(64), _p(A32), S),
         (ERR_ALIGN, "nvfp4_w4a16_pack", _p(A32), _p(A32), _i(8), _i(64), _p(A8), S),
@@ -144,6 +148,11 @@ def test_validation_errors_launch_nothing(lib):
         (ERR_NULL, "nvfp4_quantize_fused", _p(A32), _i(2), _i(16), amax, _p(A32), _p(A32), gs, _p(0), S),
         (ERR_ALIGN, "nvfp4_quantize_fused", _p(A32), _i(2), _i(16), amax, _p(A32), _p(A32), gs, _p(A32 + 8), S),
         (ERR_SHAPE, "nvfp4_quantize_fused", _p(A32), _i(-2), _i(16), amax, _p(A32), _p(A32), gs, _p(A32), S),
+        # running amax
+        (ERR_NULL, "nvfp4_amax_accumulate", _p(A32), _i(16), _p(0), S),
+        (ERR_ALIGN, "nvfp4_amax_accumulate", _p(A32), _i(16), _p(A32 + 2), S),
+        (ERR_SHAPE, "nvfp4_amax_accumulate", _p(A32), _i(-3), amax, S),
+        (NVFP4_OK, "nvfp4_amax_accumulate", _p(0), _i(0), amax, S),
         # amax
         (ERR_NULL, "nvfp4_amax", _p(A32), _i(16), _p(0), S),
         (ERR_NULL, "nvfp4_amax", _p(0), _i(16), amax, S),

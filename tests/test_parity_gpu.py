@@ -434,3 +434,18 @@ def test_ragged_outputs_stay_inside_their_tensor(M, N):
         assert_equal_bits(bits(y), want, what)
         buf.view(torch.uint8).fill_(0xA5)
         nv.nvfp4_dequantize(p, s, gs, out=y, n_cols=N)
+
+
+def test_running_amax_over_several_tensors():
+    """nvfp4_amax_accumulate folds tensors of any length (tails, an empty one) into one
+    running max that equals the amax of them all; a larger starting value is kept."""
+    rng = np.random.default_rng(77)
+    parts = [synthetic.to_bf16_bits(rng.standard_normal(n).astype(np.float32) * np.float32(s))
+             for n, s in ((4099, 1.0), (16, 3.0), (0, 1.0), (1000003, 0.5))]
+    run = torch.zeros(1, dtype=torch.float32, device="cuda")
+    for p in parts:
+        nv.nvfp4_amax_accumulate(to_dev(p), run)
+    assert f32_bits(run) == f32_bits(oracle.amax_multi([p for p in parts if p.size]))
+    big = torch.full((1,), 1e6, dtype=torch.float32, device="cuda")
+    nv.nvfp4_amax_accumulate(to_dev(parts[0]), big)
+    assert big.item() == 1e6

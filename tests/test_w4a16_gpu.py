@@ -182,3 +182,29 @@ def test_empty_rows_launch_nothing():
     y = nv.nvfp4_w4a16_linear(x, tiled, gs, 32, workspace=nv.new_workspace("cuda"))
     assert tuple(y.shape) == (0, 32)
     assert nv.nvfp4_kernel_launch_count() == before
+
+
+@pytest.mark.parametrize("M", [1, 16, 100])
+def test_split_k_for_few_rows(M):
+    """Up to 128 rows of x on a weight with few output tiles (4096 x 4096: 32 tiles) the call
+    splits K over several CTAs when the workspace is large enough; the result is within the
+    bound, bit-identical from call to call (the partial sums are added in a fixed order),
+    and the workspace can be reused.  Without the room to split, the same call runs
+    unsplit and is within the bound too."""
+    K, N = 4096, 4096
+    assert nv.nvfp4_w4a16_workspace_bytes(M, N, K) > nv.WORKSPACE_BYTES
+    rng = np.random.default_rng(M + 900)
+    x = synthetic.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    bias = synthetic.to_bf16_bits(rng.standard_normal(N).astype(np.float32))
+    packed, scales, gs = _weight(N, K, 901)
+    tiled = nv.nvfp4_w4a16_pack(packed, scales)
+    ws = nv.nvfp4_w4a16_workspace(M, N, K, "cuda")
+    xd, bd = to_dev(x), to_dev(bias)
+    y1 = nv.nvfp4_w4a16_linear(xd, tiled, gs, N, bias=bd, workspace=ws)
+    y2 = nv.nvfp4_w4a16_linear(xd, tiled, gs, N, bias=bd, workspace=ws)
+    torch.cuda.synchronize()
+    assert nv.nvfp4_workspace_check(ws[:nv.WORKSPACE_BYTES]) == 0
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    _assert_within_bound(bits(y1), x, packed, scales, gs, bias, f"split K, {M} rows")
+    y3 = nv.nvfp4_w4a16_linear(xd, tiled, gs, N, bias=bd, workspace=nv.new_workspace("cuda"))
+    _assert_within_bound(bits(y3), x, packed, scales, gs, bias, f"unsplit, {M} rows")
