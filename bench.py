@@ -524,6 +524,7 @@ def run_linear(args):
     Beside it: the pages' own order of work (nvfp4_dequantize into a bf16 buffer, then torch's
     bf16 linear) and a bf16 linear on an unquantized bf16 weight.  L2 flushed before each rep
     (a write of 256 MB); CUDA events; median of 15 reps."""
+    import numpy as np
     import torch
     from qat_nvfp4_b200 import nvfp4 as nv
     from qat_nvfp4_b200 import synthetic
@@ -565,7 +566,15 @@ def run_linear(args):
             flops = 2.0 * M * N * K
             nbytes = 2.0 * M * K + 0.5625 * N * K + 2.0 * M * N
             ideal = max(flops / (tc * 1e12), nbytes / (hbm * 1e9))
-            rows.append({"weight": [N, K], "tokens": M, "fused_us": t_fused * 1e6,
+            cpu_us = None
+            if M == 16:  # the oracle's forward (C dequantize + float64 matmul), one call on the host
+                import oracle
+                xb = x.view(torch.int16).cpu().numpy().view(np.uint16)
+                pk, sc, g = packed.cpu().numpy(), scales.cpu().numpy(), float(gs.item())
+                t0 = time.perf_counter()
+                oracle.w4a16_linear(xb, pk, sc, g, N)
+                cpu_us = (time.perf_counter() - t0) * 1e6
+            rows.append({"weight": [N, K], "tokens": M, "fused_us": t_fused * 1e6, "oracle_cpu_us": cpu_us,
                          "TFLOP/s": flops / t_fused / 1e12, "GB/s": nbytes / t_fused / 1e9,
                          "bound": "tensor" if flops / (tc * 1e12) >= nbytes / (hbm * 1e9) else "hbm",
                          "frac": ideal / t_fused, "dequant_then_linear_us": t_pages * 1e6,
@@ -574,12 +583,13 @@ def run_linear(args):
         del w, packed, scales, tiled, wbuf
     print(f"bf16 peak {tc:.1f} TFLOP/s ({tc_src}); HBM peak {hbm:.1f} GB/s ({hbm_src})")
     print("| weight | tokens | W4A16 us | TFLOP/s | GB/s | bound | frac of roofline | dequantize + linear us "
-          "| bf16 linear (unquantized weight) us |")
-    print("|---|---|---|---|---|---|---|---|---|")
+          "| bf16 linear (unquantized weight) us | CPU oracle us (1 thread) |")
+    print("|---|---|---|---|---|---|---|---|---|---|")
     for r in rows:
+        cpu = f"{r['oracle_cpu_us']:.0f}" if r["oracle_cpu_us"] is not None else ""
         print(f"| {r['weight'][0]}x{r['weight'][1]} | {r['tokens']} | {r['fused_us']:.1f} | {r['TFLOP/s']:.0f} | "
               f"{r['GB/s']:.0f} | {r['bound']} | {r['frac']:.2f} | {r['dequant_then_linear_us']:.1f} | "
-              f"{r['bf16_linear_us']:.1f} |")
+              f"{r['bf16_linear_us']:.1f} | {cpu} |")
     with open(args.linear, "w") as f:
         json.dump({"bf16_tflops": tc, "hbm_gbs": hbm, "rows": rows}, f, indent=1)
     return 0
