@@ -358,6 +358,17 @@ nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, const uint8
                                 const float* d_global_scale, int64_t N, const void* bias, void* y,
                                 void* d_workspace, int64_t workspace_bytes, nvfp4_stream_t stream);
 
+/* Self-test of the bounded waits of the W4A16 kernel: the call of nvfp4_w4a16_linear (no
+ * bias) with one extra wait, at the start of the MMA issue, on a barrier that nothing
+ * completes, limited to timeout_us (1 .. 100000).  That wait runs out, every role of every
+ * CTA stops through the kernel's stop flag, the copies already issued land, tensor memory is
+ * released, and NVFP4_ERR_TIMEOUT is left in the workspace for nvfp4_workspace_check; y is
+ * unspecified.  The context stays usable.  M > 0 and N > 0 (else NVFP4_ERR_ARG); other
+ * arguments and errors as for nvfp4_w4a16_linear. */
+nvfp4_status nvfp4_w4a16_selftest_timeout(const void* x, int64_t M, int64_t K, const uint8_t* tiled,
+                                          const float* d_global_scale, int64_t N, void* y, void* d_workspace,
+                                          int64_t workspace_bytes, uint32_t timeout_us, nvfp4_stream_t stream);
+
 /* Workspace bytes with which nvfp4_w4a16_linear may split K for this shape (at least
  * NVFP4_WORKSPACE_BYTES; -1 for a shape it refuses).  Depends on the current device's SM
  * count. */

@@ -96,6 +96,7 @@ struct Cfg {
         uint64_t b_empty[kRingB];  // the MMAs that read it completed
         uint64_t accum;            // every MMA of the tile completed
         uint64_t drain;            // used only when stopping early
+        uint64_t never;            // self-test: a barrier nothing arrives on
         uint32_t tmem_base;
         uint32_t abort;
         uint32_t last;             // split K: this CTA finishes the tile
@@ -146,7 +147,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait until the phase of parity `parity` of the barrier has completed.  Gives up (false)
 // after kWaitLimitNs, or early when another role has set *abort (unless ignore_abort).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile uint32_t* abort,
-                                          bool ignore_abort = false) {
+                                          bool ignore_abort = false, uint64_t limit_ns = kWaitLimitNs) {
     uint64_t t0 = 0;
     for (uint32_t i = 0;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -154,7 +155,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const v
             if (!ignore_abort && *abort) return false;
             const uint64_t now = global_ns();
             if (t0 == 0) t0 = now;
-            else if (now - t0 > kWaitLimitNs) return false;
+            else if (now - t0 > limit_ns) return false;
         }
     }
 }
@@ -306,6 +307,7 @@ struct LinearArgs {
     int vec_store;          // rows of y allow 16-byte stores
     int splits;             // CTAs per output tile, each over a contiguous share of the K stages
     unsigned* counters;     // splits > 1: per output tile, CTAs done (the last one resets it)
+    uint64_t selftest_ns;   // nonzero: first wait on a barrier nothing completes, for this long
     float* partial;         // splits > 1: fp32 partial sums [splits][output tiles][128 columns][128
                             // rows] (rows fastest: a warp's 32 rows are 128 contiguous bytes)
 };
@@ -390,6 +392,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         mbar_init(smem_u32(&sh.accum), 1);
         mbar_init(smem_u32(&sh.drain), 1);
+        mbar_init(smem_u32(&sh.never), 1);
         sh.abort = 0u;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -451,7 +454,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
             bool ok = true;
-            for (int kb = 0; kb < nk; ++kb) {
+            // self-test of the bounded waits: the limit runs out, every role stops
+            if (a.selftest_ns != 0 && !mbar_wait(smem_u32(&sh.never), 0u, abort, false, a.selftest_ns)) {
+                stop_all(sh, a.ws);
+                ok = false;
+            }
+            for (int kb = 0; ok && kb < nk; ++kb) {
                 const int sa = kb % kRingA, sb = kb % kRingB;
                 if (!mbar_wait(smem_u32(&sh.a_full[sa]), (uint32_t)(kb / kRingA) & 1u, abort) ||
                     !mbar_wait(smem_u32(&sh.b_full[sb]), (uint32_t)(kb / kRingB) & 1u, abort)) {
@@ -741,9 +749,10 @@ NVFP4_API int64_t nvfp4_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     return splits > 1 ? split_workspace_bytes(M, N, splits) : (int64_t)sizeof(Workspace);
 }
 
-NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* tiled,
-                                          const float* d_global_scale, int64_t N, const void* bias, void* y,
-                                          void* d_workspace, int64_t workspace_bytes, nvfp4_stream_t stream) {
+static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const uint8_t* tiled,
+                                      const float* d_global_scale, int64_t N, const void* bias, void* y,
+                                      void* d_workspace, int64_t workspace_bytes, uint64_t selftest_ns,
+                                      nvfp4_stream_t stream) {
     if (M < 0 || !weight_shape_ok(N, K) || M > 0x7FFFFF00ll) return NVFP4_ERR_SHAPE;
     // Output tiles 256 x 256 when x has more than 256 rows, 256 x 128 for 129 to 256 rows,
     // 128 x 128 for at most 128.
@@ -798,6 +807,7 @@ NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, c
     a.kt = (K + kBK - 1) / kBK;
     a.vec_store = (is_aligned(y, 16) && N % 8 == 0) ? 1 : 0;
     a.a_bytes = (uint32_t)box_rows * kBK * 2;
+    a.selftest_ns = selftest_ns;
     // split K only with a workspace large enough for the partial sums
     int sms = 0;
     st = sm_count_w4(&sms);
@@ -816,4 +826,19 @@ NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, c
         w4a16_linear_kernel<128, 1><<<grid, kGemmThreads, Cfg<128, 1>::kSmemBytes, cst>>>(map, a);
     note_launch();
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+NVFP4_API nvfp4_status nvfp4_w4a16_linear(const void* x, int64_t M, int64_t K, const uint8_t* tiled,
+                                          const float* d_global_scale, int64_t N, const void* bias, void* y,
+                                          void* d_workspace, int64_t workspace_bytes, nvfp4_stream_t stream) {
+    return w4a16_linear_impl(x, M, K, tiled, d_global_scale, N, bias, y, d_workspace, workspace_bytes, 0, stream);
+}
+
+NVFP4_API nvfp4_status nvfp4_w4a16_selftest_timeout(const void* x, int64_t M, int64_t K, const uint8_t* tiled,
+                                                    const float* d_global_scale, int64_t N, void* y, void* d_workspace,
+                                                    int64_t workspace_bytes, uint32_t timeout_us,
+                                                    nvfp4_stream_t stream) {
+    if (M <= 0 || N <= 0 || timeout_us == 0 || timeout_us > 100000) return NVFP4_ERR_ARG;
+    return w4a16_linear_impl(x, M, K, tiled, d_global_scale, N, nullptr, y, d_workspace, workspace_bytes,
+                             (uint64_t)timeout_us * 1000ull, stream);
 }

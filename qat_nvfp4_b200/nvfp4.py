@@ -74,6 +74,8 @@ _c_w4a16_tiled_bytes = _sig("nvfp4_w4a16_tiled_bytes", [_i64, _i64], _i64)
 _c_w4a16_pack = _sig("nvfp4_w4a16_pack", [_vp, _vp, _i64, _i64, _vp, _vp])
 _c_w4a16_linear = _sig("nvfp4_w4a16_linear", [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _vp])
 _c_w4a16_workspace_bytes = _sig("nvfp4_w4a16_workspace_bytes", [_i64, _i64, _i64], _i64)
+_c_w4a16_selftest_timeout = _sig("nvfp4_w4a16_selftest_timeout",
+                                 [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _i64, ctypes.c_uint32, _vp])
 _c_status_string = _sig("nvfp4_status_string", [ctypes.c_int], ctypes.c_char_p)
 _c_launch_count = _sig("nvfp4_kernel_launch_count", [], ctypes.c_uint64)
 
@@ -541,6 +543,22 @@ def nvfp4_w4a16_linear(x: torch.Tensor, tiled: torch.Tensor, global_scale: torch
                                bias.data_ptr() if bias is not None else None, out.data_ptr(), ws.data_ptr(),
                                ws.numel(), _stream(x.device)), "nvfp4_w4a16_linear")
     return out
+
+
+def nvfp4_w4a16_selftest_timeout(x: torch.Tensor, tiled: torch.Tensor, global_scale: torch.Tensor, n_out: int,
+                                 workspace: torch.Tensor, timeout_us: int = 2000) -> int:
+    """Run the W4A16 kernel with a wait that nothing completes (limited to timeout_us) and
+    return the status nvfp4_workspace_check then reports (NVFP4_ERR_TIMEOUT = 6 expected)."""
+    M, K = _matrix(x)
+    _cuda(tiled, "tiled", torch.uint8)
+    _scalar(global_scale, "global_scale")
+    ws = _workspace(workspace, x.device)
+    y = torch.empty(tuple(x.shape[:-1]) + (int(n_out),), dtype=torch.bfloat16, device=x.device)
+    with torch.cuda.device(x.device):
+        _check(_c_w4a16_selftest_timeout(x.data_ptr(), M, K, tiled.data_ptr(), global_scale.data_ptr(), int(n_out),
+                                         y.data_ptr(), ws.data_ptr(), ws.numel(), int(timeout_us),
+                                         _stream(x.device)), "nvfp4_w4a16_selftest_timeout")
+        return int(_c_workspace_check(ws.data_ptr(), _stream(x.device)))
 
 
 def nvfp4_w4a16_workspace_bytes(M: int, N: int, K: int) -> int:

@@ -144,6 +144,11 @@ def test_validation_errors_launch_nothing(lib):
         (ERR_NULL, "nvfp4_w4a16_pack", _p(A32), _p(0), _i(8), _i(64), _p(A32), S),
         (ERR_ALIGN, "nvfp4_w4a16_pack", _p(A32), _p(A32), _i(8), _i(64), _p(A8), S),
         (NVFP4_OK, "nvfp4_w4a16_pack", _p(0), _p(0), _i(0), _i(64), _p(0), S),
+        # W4A16 self-test: x, M, K, tiled, gs, N, y, workspace, bytes, timeout_us
+        (ERR_ARG, "nvfp4_w4a16_selftest_timeout", _p(A32), _i(4), _i(64), _p(A32), gs, _i(8), _p(A32), _p(A32),
+         _i(256), ctypes.c_uint32(0), S),
+        (ERR_ARG, "nvfp4_w4a16_selftest_timeout", _p(A32), _i(0), _i(64), _p(A32), gs, _i(8), _p(A32), _p(A32),
+         _i(256), ctypes.c_uint32(1000), S),
         # fused quantize: x, M, N, amax, packed, scales, gs, workspace
         (ERR_NULL, "nvfp4_quantize_fused", _p(A32), _i(2), _i(16), amax, _p(A32), _p(A32), gs, _p(0), S),
         (ERR_ALIGN, "nvfp4_quantize_fused", _p(A32), _i(2), _i(16), amax, _p(A32), _p(A32), gs, _p(A32 + 8), S),

@@ -208,3 +208,24 @@ def test_split_k_for_few_rows(M):
     _assert_within_bound(bits(y1), x, packed, scales, gs, bias, f"split K, {M} rows")
     y3 = nv.nvfp4_w4a16_linear(xd, tiled, gs, N, bias=bd, workspace=nv.new_workspace("cuda"))
     _assert_within_bound(bits(y3), x, packed, scales, gs, bias, f"unsplit, {M} rows")
+
+
+@pytest.mark.parametrize("M,N", [(16, 4096), (700, 512)])
+def test_bounded_wait_reports_a_timeout_and_the_context_recovers(M, N):
+    """A wait on a barrier that nothing completes (2 ms limit) runs out: the call reports
+    NVFP4_ERR_TIMEOUT through the workspace instead of hanging, every role stops, and the
+    next call on the same context and workspace is correct.  16 rows take the split-K
+    path, 700 rows the 256 x 256 tiles."""
+    K = 1024
+    rng = np.random.default_rng(M + N)
+    x = synthetic.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    packed, scales, gs = _weight(N, K, 77)
+    tiled = nv.nvfp4_w4a16_pack(packed, scales)
+    ws = nv.nvfp4_w4a16_workspace(M, N, K, "cuda")
+    xd = to_dev(x)
+    assert nv.nvfp4_w4a16_selftest_timeout(xd, tiled, gs, N, ws, timeout_us=2000) == 6
+    ws.zero_()
+    y = nv.nvfp4_w4a16_linear(xd, tiled, gs, N, workspace=ws)
+    torch.cuda.synchronize()
+    assert nv.nvfp4_workspace_check(ws) == 0
+    _assert_within_bound(bits(y), x, packed, scales, gs, None, "after a timeout")
