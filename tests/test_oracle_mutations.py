@@ -68,3 +68,79 @@ def test_pins_reject_mutant(tmp_path, name, old, new):
                         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"mutant {name!r} passed every pin:\n{r.stdout[-2000:]}"
+
+
+# ---- the W4A16 forward (oracle.w4a16_linear, Python) ------------------------------------
+#
+# Each mutant replaces oracle.w4a16_linear for the duration of the test; at least one of the
+# W4A16 pins in test_oracle_pins.py must then fail (an assertion or any other error).
+
+def _linear_mutants():
+    import numpy as np
+    import oracle
+
+    real = oracle.w4a16_linear
+
+    def transposed(x_bits, packed, scales, gs, n_out, block=16, bias_bits=None):
+        x = oracle.bf16_to_f64(x_bits)
+        w = oracle.bf16_to_f64(oracle.dequantize(packed, scales, gs, n_out, x.shape[1], block))
+        y = x @ w.T
+        return y.T.reshape(y.shape) if y.shape[0] == y.shape[1] else x[:, :n_out] @ w[:, :n_out]
+
+    def no_bias(x_bits, packed, scales, gs, n_out, block=16, bias_bits=None):
+        return real(x_bits, packed, scales, gs, n_out, block)
+
+    def bias_twice(x_bits, packed, scales, gs, n_out, block=16, bias_bits=None):
+        y = real(x_bits, packed, scales, gs, n_out, block, bias_bits)
+        if bias_bits is not None:
+            y = y + oracle.bf16_to_f64(np.asarray(bias_bits).reshape(1, n_out))
+        return y
+
+    def block32(x_bits, packed, scales, gs, n_out, block=16, bias_bits=None):
+        K = np.asarray(x_bits).shape[1]
+        x = oracle.bf16_to_f64(x_bits)
+        w = oracle.bf16_to_f64(oracle.dequantize(packed, scales[:, ::2].copy(), gs, n_out, K, 32))
+        y = x @ w.T
+        if bias_bits is not None:
+            y = y + oracle.bf16_to_f64(np.asarray(bias_bits).reshape(1, n_out))
+        return y
+
+    def negated(x_bits, packed, scales, gs, n_out, block=16, bias_bits=None):
+        return -real(x_bits, packed, scales, gs, n_out, block, bias_bits)
+
+    def fp32_sums(x_bits, packed, scales, gs, n_out, block=16, bias_bits=None):
+        x = oracle.bf16_to_f64(x_bits).astype(np.float32)
+        K = x.shape[1]
+        w = oracle.bf16_to_f64(oracle.dequantize(packed, scales, gs, n_out, K, block)).astype(np.float32)
+        y = np.zeros((x.shape[0], n_out), dtype=np.float32)
+        for k in range(K):  # sequential fp32 accumulation
+            y += np.outer(x[:, k], w[:, k]).astype(np.float32)
+        if bias_bits is not None:
+            y = y + oracle.bf16_to_f64(np.asarray(bias_bits).reshape(1, n_out)).astype(np.float32)
+        return y.astype(np.float64)
+
+    def drops_last_block(x_bits, packed, scales, gs, n_out, block=16, bias_bits=None):
+        x = np.array(x_bits, dtype=np.uint16, copy=True)
+        x[:, -16:] = 0
+        return real(x, packed, scales, gs, n_out, block, bias_bits)
+
+    return {"transposed weight": transposed, "bias dropped": no_bias, "bias added twice": bias_twice,
+            "blocks of 32": block32, "sign flipped": negated, "fp32 sequential sums": fp32_sums,
+            "last K block dropped": drops_last_block}
+
+
+@pytest.mark.parametrize("name", list(_linear_mutants()))
+def test_linear_pins_reject_mutant(monkeypatch, name):
+    import oracle
+    import test_oracle_pins as pins
+
+    monkeypatch.setattr(oracle, "w4a16_linear", _linear_mutants()[name])
+    checks = [pins.test_linear_one_hot_rows_select_weight_columns, pins.test_linear_brute_force_exact_rationals,
+              pins.test_linear_zero_activations_give_the_bias, pins.test_linear_uses_the_dequantized_weight]
+    caught = 0
+    for check in checks:
+        try:
+            check()
+        except Exception:  # an assertion, a shape error: the pin caught the mutant
+            caught += 1
+    assert caught >= 1, f"mutant '{name}' passed every W4A16 pin"
