@@ -80,7 +80,8 @@ def workload_config(args, world):
 
 
 # The sources of the kernels the step runs (the W4A16 linear has its own file).
-STEP_SOURCES = ("nvfp4_device.cuh", "nvfp4_kernels.cu", "nvfp4_runtime.h")
+STEP_SOURCES = ("nvfp4_device.cuh", "nvfp4_runtime.h", "nvfp4_stream.cuh", "nvfp4_reduce.cuh", "nvfp4_encode.cuh",
+                "nvfp4_ragged.cuh", "nvfp4_kernels.cu")
 
 
 def source_digest():
