@@ -65,20 +65,30 @@ static_assert(kRecBytes % 16 == 0, "bulk copy size");
 // the activation traffic per FLOP of BN = 128); 256 x 128 (twice the CTAs) when x has 129
 // to 256 rows; 128 x 128 when it has at most 128 (half the MMA work and activation bytes
 // per stage, and deeper rings for the weight stream).
+//
+// A stage covers kAtoms atoms of K (64 columns each, one 128-byte swizzle row per tile row):
+// 2 for the 128 x 128 tiles, where the time of a stage is mostly the fixed cost of handing it
+// from role to role, so that cost is paid once per 128 columns; 1 for the others.  Within a
+// stage, atom t of the activation tile sits at t * kBM * 128 bytes (accumulator h's 128 rows
+// at + h * 16 KB) and atom t of the decoded weight tile at t * BN * 128 bytes.
 template <int BN, int ACC>
 struct Cfg {
     static constexpr int kBN = BN;
     static constexpr int kBM = kMmaM * ACC;
-    static constexpr int kTileABytes = kBM * kBK * 2;
-    static constexpr int kRecPerTile = BN / kRecRows;           // records per stage
-    static constexpr int kTileBBytes = BN * kBK * 2;             // decoded weight tile
+    static constexpr int kAtoms = ACC == 1 ? 2 : 1;
+    static constexpr int kAtomABytes = kBM * kBK * 2;            // one 64-column atom of the activation tile
+    static constexpr int kAtomBBytes = BN * kBK * 2;             // one 64-column atom of the weight tile
+    static constexpr int kTileABytes = kAtoms * kAtomABytes;
+    static constexpr int kRecPerTile = BN / kRecRows;            // records per atom
+    static constexpr int kRecPerStage = kRecPerTile * kAtoms;
+    static constexpr int kTileBBytes = kAtoms * kAtomBBytes;     // decoded weight tile
     static constexpr int kTmemCols = ACC * BN;                   // fp32 accumulators, 128 lanes x BN each
-    static constexpr int kRingA = BN == 256 ? 3 : (ACC == 2 ? 4 : 6);  // activation tiles in flight
-    static constexpr int kRingW = BN == 256 ? 4 : (ACC == 2 ? 8 : 12); // record groups in flight
-    static constexpr int kRingB = BN == 256 ? 2 : 3;             // decoded tiles, decode -> MMA
+    static constexpr int kRingA = BN == 256 ? 3 : (ACC == 2 ? 4 : 3);  // activation tiles in flight
+    static constexpr int kRingW = BN == 256 ? 4 : (ACC == 2 ? 8 : 4);  // record groups in flight
+    static constexpr int kRingB = BN == 256 ? 2 : (ACC == 2 ? 3 : 2);  // decoded tiles, decode -> MMA
     static constexpr int kColParts = 4 / ACC;                    // epilogue warps per accumulator lane group
     static constexpr int kTpr = kDecodeThreads / BN;             // decode threads per weight row
-    static constexpr int kBpt = (kBK / kBlockElems) / kTpr;      // 16-element blocks per thread
+    static constexpr int kBpt = kAtoms * (kBK / kBlockElems) / kTpr;  // 16-element blocks per thread
     // Instruction descriptor of kind::f16: fp32 accumulator (bits 4-5 = 1), A and B bf16
     // (bits 7-9 = 1, bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 in bits
     // 17-22, M >> 4 in bits 24-28.
@@ -102,13 +112,14 @@ struct Cfg {
         uint32_t last;             // split K: this CTA finishes the tile
         float sd[256];             // decode scale for every E4M3 byte: fl(E4M3(b) / gs)
     };
-    static constexpr int kRingBytes = kRingA * kTileABytes + kRingB * kTileBBytes + kRingW * kRecPerTile * kRecBytes;
+    static constexpr int kRingBytes = kRingA * kTileABytes + kRingB * kTileBBytes + kRingW * kRecPerStage * kRecBytes;
     static constexpr int kSmemBytes = 1024 + kRingBytes + (int)sizeof(Shared);
 
     static_assert(BN % kRecRows == 0 && BN >= 16 && BN <= 256, "MMA N");
-    static_assert(kTpr * kBpt == kBK / kBlockElems && kBpt >= 1, "decode split");
+    static_assert(kTpr * kBpt == kAtoms * (kBK / kBlockElems) && kBpt >= 1 && kBpt <= 2, "decode split");
+    static_assert(kBpt == 1 || (kBK / kBlockElems) % kBpt == 0, "a thread's blocks lie in one atom");
     static_assert(kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0, "tensor memory columns");
-    static_assert(kTileABytes % 1024 == 0 && kTileBBytes % 1024 == 0, "operand tiles stay 1024-byte aligned");
+    static_assert(kAtomABytes % 1024 == 0 && kAtomBBytes % 1024 == 0, "operand tiles stay 1024-byte aligned");
     static_assert(kDecodeWarps == 4 * ACC * kColParts, "epilogue warps");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
@@ -354,7 +365,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     w4a16_linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const LinearArgs a) {
     using C = Cfg<BN, ACC>;
     constexpr int kBN = C::kBN, kRingA = C::kRingA, kRingB = C::kRingB, kRingW = C::kRingW;
-    constexpr int kBM = C::kBM, kTileABytes = C::kTileABytes;
+    constexpr int kBM = C::kBM, kTileABytes = C::kTileABytes, kAtoms = C::kAtoms;
+    constexpr int kAtomABytes = C::kAtomABytes, kAtomBBytes = C::kAtomBBytes, kRecPerStage = C::kRecPerStage;
     constexpr int kTileBBytes = C::kTileBBytes, kRecPerTile = C::kRecPerTile, kTpr = C::kTpr, kBpt = C::kBpt;
     constexpr uint32_t kIdesc = C::kIdesc;
     extern __shared__ uint8_t dsmem[];
@@ -373,9 +385,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int sp = (int)((int64_t)blockIdx.x % a.splits);
     const int64_t tm = tile / a.tiles_n, tn = tile % a.tiles_n;
     const int64_t m0 = tm * kBM, n0 = tn * kBN;
-    // this CTA's K stages: [kb0, kb0 + nk); stage i of the loops below is kb0 + i
-    const int kb0 = (int)((int64_t)sp * a.kt / a.splits);
-    const int nk = (int)((int64_t)(sp + 1) * a.kt / a.splits) - kb0;
+    // this CTA's K stages: [kb0, kb0 + nk); stage i of the loops below is kb0 + i and holds
+    // the atoms (64 columns of K each) (kb0 + i) kAtoms .. + kAtoms - 1 that are below kt
+    const int nstages = (int)((a.kt + kAtoms - 1) / kAtoms);
+    const int kb0 = (int)((int64_t)sp * nstages / a.splits);
+    const int nk = (int)((int64_t)(sp + 1) * nstages / a.splits) - kb0;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kRingA; ++s) {
@@ -431,17 +445,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     break;
                 }
                 const uint32_t bar = smem_u32(&full[s]);
+                const int at0 = (kb0 + kb) * kAtoms;
+                const int na = min(kAtoms, (int)(a.kt - at0));  // atoms of this stage inside K
                 if (act) {
-                    mbar_arrive_expect_tx(bar, a.a_bytes);
-                    tma_load_2d(sA0 + s * kTileABytes, &tmap_x, (kb0 + kb) * kBK, (int32_t)m0, bar);
+                    mbar_arrive_expect_tx(bar, a.a_bytes * (uint32_t)na);
+                    for (int t = 0; t < na; ++t)
+                        tma_load_2d(sA0 + s * kTileABytes + t * kAtomABytes, &tmap_x, (at0 + t) * kBK, (int32_t)m0, bar);
                 } else {
-                    mbar_arrive_expect_tx(bar, kRecPerTile * kRecBytes);
+                    mbar_arrive_expect_tx(bar, (uint32_t)(na * kRecPerTile * kRecBytes));
+                    for (int t = 0; t < na; ++t) {
 #pragma unroll
-                    for (int i = 0; i < kRecPerTile; ++i) {
-                        int64_t rn = kRecPerTile * tn + i;
-                        if (rn >= nrec) rn = nrec - 1;
-                        bulk_load(sW0 + (s * kRecPerTile + i) * kRecBytes,
-                                  a.tiled + (rn * a.kt + kb0 + kb) * kRecBytes, kRecBytes, bar);
+                        for (int i = 0; i < kRecPerTile; ++i) {
+                            int64_t rn = kRecPerTile * tn + i;
+                            if (rn >= nrec) rn = nrec - 1;
+                            bulk_load(sW0 + (s * kRecPerStage + t * kRecPerTile + i) * kRecBytes,
+                                      a.tiled + (rn * a.kt + at0 + t) * kRecBytes, kRecBytes, bar);
+                        }
                     }
                 }
                 ++issued;
@@ -468,14 +487,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint64_t bd = sw128_desc(sB0 + sb * kTileBBytes);
+                const int na = min(kAtoms, (int)(a.kt - (int64_t)(kb0 + kb) * kAtoms));
 #pragma unroll
-                for (int j = 0; j < kBK / kUmmaK; ++j) {  // +32 bytes along K per step
-                    const uint32_t acc = (kb | j) != 0 ? 1u : 0u;
+                for (int t = 0; t < kAtoms; ++t) {
+                    if (t >= na) break;
+                    const uint64_t bd = sw128_desc(sB0 + sb * kTileBBytes + t * kAtomBBytes);
+                    const uint32_t at = sA0 + sa * kTileABytes + t * kAtomABytes;
 #pragma unroll
-                    for (int h = 0; h < ACC; ++h)  // accumulator h: rows 128 h .. of the tile
-                        umma_f16(tmem + h * kBN, sw128_desc(sA0 + sa * kTileABytes + h * kMmaM * 128) + 2u * j,
-                                 bd + 2u * j, kIdesc, acc);
+                    for (int j = 0; j < kBK / kUmmaK; ++j) {  // +32 bytes along K per step
+                        const uint32_t acc = (kb | t | j) != 0 ? 1u : 0u;
+#pragma unroll
+                        for (int h = 0; h < ACC; ++h)  // accumulator h: rows 128 h .. of the tile
+                            umma_f16(tmem + h * kBN, sw128_desc(at + h * kMmaM * 128) + 2u * j, bd + 2u * j, kIdesc, acc);
+                    }
                 }
                 umma_commit(smem_u32(&sh.a_empty[sa]));
                 umma_commit(smem_u32(&sh.b_empty[sb]));
@@ -489,10 +513,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
     } else {
-        // ---- decode warps: kTpr threads per weight row, kBpt 16-element blocks each ----
-        const int t = threadIdx.x;
-        const int row = t / kTpr;
-        const int part = t % kTpr;
+        // ---- decode warps: kTpr threads per weight row, kBpt 16-element blocks each, all
+        //      in atom `atom` of the stage, from its block `bl0` on ----
+        const int row = threadIdx.x / kTpr;
+        const int part = threadIdx.x % kTpr;
+        const int atom = kBpt * part / (kBK / kBlockElems);
+        const int bl0 = kBpt * part % (kBK / kBlockElems);
+        const int rr = row % kRecRows;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
             const int sw = kb % kRingW, sb = kb % kRingB;
@@ -502,24 +529,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 ok = false;
                 break;
             }
-            const uint8_t* rec = gW0 + (sw * kRecPerTile + row / kRecRows) * kRecBytes;
-            const int rr = row % kRecRows;
+            // an atom past the end of K is neither loaded nor multiplied
+            const bool live = (kb0 + kb) * kAtoms + atom < a.kt;
+            const uint8_t* rec = gW0 + (sw * kRecPerStage + atom * kRecPerTile + row / kRecRows) * kRecBytes;
             uint32_t c[2 * kBpt];
-            uint32_t sc;
-            if constexpr (kBpt == 2) {
-                const uint4 v = *reinterpret_cast<const uint4*>(rec + rr * 32 + part * 16);
+            uint32_t sc = 0;
+            if (!live) {
+#pragma unroll
+                for (int i = 0; i < 2 * kBpt; ++i) c[i] = 0;
+            } else if constexpr (kBpt == 2) {
+                const uint4 v = *reinterpret_cast<const uint4*>(rec + rr * 32 + bl0 * 8);
                 c[0] = v.x;
                 c[1] = v.y;
                 c[2] = v.z;
                 c[3] = v.w;
-                sc = *reinterpret_cast<const uint16_t*>(rec + kRecCodes + rr * 4 + part * 2);
+                sc = *reinterpret_cast<const uint16_t*>(rec + kRecCodes + rr * 4 + bl0);
             } else {
-                const uint2 v = *reinterpret_cast<const uint2*>(rec + rr * 32 + part * 8);
+                const uint2 v = *reinterpret_cast<const uint2*>(rec + rr * 32 + bl0 * 8);
                 c[0] = v.x;
                 c[1] = v.y;
-                sc = rec[kRecCodes + rr * 4 + part];
+                sc = rec[kRecCodes + rr * 4 + bl0];
             }
-            uint8_t* tile_row = gB0 + sb * kTileBBytes + row * 128;
+            uint8_t* tile_row = gB0 + sb * kTileBBytes + atom * kAtomBBytes + row * 128;
 #pragma unroll
             for (int i = 0; i < kBpt; ++i) {
                 const float sd = sh.sd[(sc >> (8 * i)) & 0xFFu];
@@ -531,7 +562,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     o[1] = decode_pair((w >> 8) & 0xFFu, sd);
                     o[2] = decode_pair((w >> 16) & 0xFFu, sd);
                     o[3] = decode_pair(w >> 24, sd);
-                    const int chunk = 2 * (kBpt * part + i) + q;  // 8 elements = 16 bytes
+                    const int chunk = 2 * (bl0 + i) + q;  // 8 elements = 16 bytes
                     const uint32_t dst = smem_u32(tile_row + ((chunk ^ (row & 7)) << 4));
                     asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(o[0]), "r"(o[1]), "r"(o[2]),
                                  "r"(o[3])
@@ -692,7 +723,7 @@ int64_t record_bytes(int64_t N, int64_t K) {
 }
 
 // Split K for at most 128 rows of x: enough CTAs per 128-column tile to fill the SMs (one
-// CTA per SM), each with at least 8 K stages.
+// CTA per SM), each with at least 8 atoms (512 columns) of K.
 int split_count(int64_t M, int64_t N, int64_t K, int sms) {
     if (M > kMmaM) return 1;
     const int64_t tiles = (N + 127) / 128;

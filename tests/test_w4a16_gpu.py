@@ -119,6 +119,8 @@ def test_decoded_weight_is_exact_through_one_hot_rows(K):
     (5, 16, 13, True),         # N odd: element stores
     (1, 4096, 4096, False),    # one token
     (513, 2048, 1000, True),
+    (100, 1040, 200, True),    # 128-row tiles: 17 atoms of K, the last stage half full and ragged
+    (64, 192, 256, False),     # 128-row tiles: 3 atoms, the second stage half full
 ])
 def test_linear_matches_oracle(M, K, N, with_bias):
     rng = np.random.default_rng(M * 7 + K * 3 + N)
@@ -184,14 +186,15 @@ def test_empty_rows_launch_nothing():
     assert nv.nvfp4_kernel_launch_count() == before
 
 
-@pytest.mark.parametrize("M", [1, 16, 100])
-def test_split_k_for_few_rows(M):
+@pytest.mark.parametrize("M,K", [(1, 4096), (16, 4096), (100, 4096), (16, 1088), (7, 4160)])
+def test_split_k_for_few_rows(M, K):
     """Up to 128 rows of x on a weight with few output tiles (4096 x 4096: 32 tiles) the call
     splits K over several CTAs when the workspace is large enough; the result is within the
     bound, bit-identical from call to call (the partial sums are added in a fixed order),
     and the workspace can be reused.  Without the room to split, the same call runs
-    unsplit and is within the bound too."""
-    K, N = 4096, 4096
+    unsplit and is within the bound too.  K = 1088 and 4160 (17 and 65 atoms of 64) give
+    the splits unequal stage counts and a last stage with one atom."""
+    N = 4096
     assert nv.nvfp4_w4a16_workspace_bytes(M, N, K) > nv.WORKSPACE_BYTES
     rng = np.random.default_rng(M + 900)
     x = synthetic.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
