@@ -309,8 +309,9 @@ nvfp4_status nvfp4_fake_quant_bs(const void* x, void* y, int64_t M, int64_t N, i
 /* ---- forward of a Linear layer on a packed weight (W4A16) ---------------------------- */
 
 /* The weight's operand form: the packed weight cut into 128-row x 64-column tiles, one
- * contiguous 4608-byte record per tile, so that the linear kernel fetches a tile with one
- * bulk copy.  Not on the pages, which keep the plain layout; the same bytes, reordered
+ * contiguous 4608-byte record per tile, so that the bytes of the tile a pipeline stage of
+ * the linear kernel decodes are contiguous and each thread's share is one aligned copy.
+ * Not on the pages, which keep the plain layout; the same bytes, reordered
  * once when the weight is converted (as [FP4OPT] convert_model_weight_to_float4 packs each
  * weight once).  Record (tn, tk), KT = ceil(K / 64), starts at byte (tn * KT + tk) * 4608:
  *   bytes [0, 4096)     row r (0..127) at 32 r: the code bytes of columns 64 tk .. 64 tk + 63

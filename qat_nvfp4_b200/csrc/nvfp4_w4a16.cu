@@ -7,19 +7,18 @@
 // One kernel on the sm_100a tensor cores (tcgen05, kind::f16, bf16 operands, fp32
 // accumulators in tensor memory).  The bf16 weight is never written to HBM.  The weight is
 // read in a tile-major copy of its packed form (nvfp4_w4a16_pack: one contiguous 4608-byte
-// record per 128-row x 64-column tile, codes then scale bytes), so each pipeline stage
-// fetches its weight tile with one bulk copy; producer warps decode it in shared memory into
-// the MMA operand layout (128-byte swizzle, K-major) with the same arithmetic as
-// nvfp4_dequantize, bf16_rn(fl(LUT[code] * fl(E4M3(byte) / gs))).  A CTA computes a
-// 256 x 128 output tile as two 128 x 128 accumulators that share each decoded weight tile.
+// record per 128-row x 64-column tile, codes then scale bytes); the decode warps copy the
+// bytes they need into shared memory themselves and decode them into the MMA operand
+// layout (128-byte swizzle, K-major) with the same arithmetic as nvfp4_dequantize,
+// bf16_rn(fl(LUT[code] * fl(E4M3(byte) / gs))).
 //
-//   warps 0-15 decode weight records into weight tiles (one 16-element block per thread and
-//              stage), then the epilogue (TMEM -> bf16 -> y)
-//   warp 16    TMA loads of activation tiles (ring of 4)
+//   warps 0-15 copy (cp.async, several stages ahead, into private slots) and decode weight
+//              rows into weight tiles, 32 rows per warp, then the epilogue
+//              (TMEM -> fp32 + bias -> bf16)
+//   warp 16    TMA loads of activation tiles
 //   warp 17    TMEM allocation, MMA issue (one elected thread), TMEM release
-//   warp 18    bulk copies of weight records (ring of 8, running ahead of the activations)
-// Decoded weight tiles pass from the decode warps to the MMAs through a ring of 3, so the
-// decode of a stage overlaps the MMAs of the stages before it.
+// Decoded weight tiles pass from the decode warps to the MMAs through a ring of 2 or 3, so
+// the decode of a stage overlaps the MMAs of the stages before it.
 //
 // Every wait on an mbarrier is bounded (kWaitLimitNs of %globaltimer); a wait that runs
 // out records NVFP4_ERR_TIMEOUT in the caller's workspace, tells the other roles to stop,
@@ -50,14 +49,13 @@ constexpr int kDecodeWarps = 16;
 constexpr int kDecodeThreads = 32 * kDecodeWarps;
 constexpr int kTmaWarp = 16;              // activation loads
 constexpr int kMmaWarp = 17;
-constexpr int kRecWarp = 18;              // weight-record loads
-constexpr int kGemmThreads = 608;
+constexpr int kGemmThreads = 576;
 constexpr int kRecCodes = kRecRows * kBK / 2;  // 4096 bytes of E2M1 codes per record
 constexpr int kRecBytes = kRecCodes + kRecRows * (kBK / kBlockElems);  // + 512 scale bytes = 4608
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 static_assert(kBK * 2 == 128, "one swizzle row per tile row");
-static_assert(kGemmThreads == 32 * (kDecodeWarps + 3), "warp roles");
+static_assert(kGemmThreads == 32 * (kDecodeWarps + 2), "warp roles");
 static_assert(kRecBytes % 16 == 0, "bulk copy size");
 
 // One configuration per output tile: kAcc accumulators of 128 rows of x (kBM = 128 kAcc rows)
@@ -66,26 +64,33 @@ static_assert(kRecBytes % 16 == 0, "bulk copy size");
 // to 256 rows; 128 x 128 when it has at most 128 (half the MMA work and activation bytes
 // per stage, and deeper rings for the weight stream).
 //
+// ROWS is the number of rows of x a tile keeps in shared memory: kBM, or 64 for the 128 x 128
+// tiles when x has at most 64 rows.  The MMA always reads 128 rows per accumulator; with
+// ROWS = 64 rows 64-127 of an atom are whatever bytes follow it in shared memory (the next
+// atom, or the decoded weight ring after the last one), and they only feed accumulator lanes
+// that the epilogue never stores.  The 64 KB this frees go to the weight ring: its depth sets
+// the bytes in flight from HBM, which is what bounds a tile at a few rows of x (a record is
+// ~2.5 us from issue to arrival under load).
+//
 // A stage covers kAtoms atoms of K (64 columns each, one 128-byte swizzle row per tile row):
 // 2 for the 128 x 128 tiles, where the time of a stage is mostly the fixed cost of handing it
 // from role to role, so that cost is paid once per 128 columns; 1 for the others.  Within a
-// stage, atom t of the activation tile sits at t * kBM * 128 bytes (accumulator h's 128 rows
+// stage, atom t of the activation tile sits at t * ROWS * 128 bytes (accumulator h's 128 rows
 // at + h * 16 KB) and atom t of the decoded weight tile at t * BN * 128 bytes.
-template <int BN, int ACC>
+template <int BN, int ACC, int ROWS = kMmaM * ACC>
 struct Cfg {
     static constexpr int kBN = BN;
     static constexpr int kBM = kMmaM * ACC;
     static constexpr int kAtoms = ACC == 1 ? 2 : 1;
-    static constexpr int kAtomABytes = kBM * kBK * 2;            // one 64-column atom of the activation tile
+    static constexpr int kAtomABytes = ROWS * kBK * 2;           // one 64-column atom of the activation tile
     static constexpr int kAtomBBytes = BN * kBK * 2;             // one 64-column atom of the weight tile
     static constexpr int kTileABytes = kAtoms * kAtomABytes;
     static constexpr int kRecPerTile = BN / kRecRows;            // records per atom
-    static constexpr int kRecPerStage = kRecPerTile * kAtoms;
     static constexpr int kTileBBytes = kAtoms * kAtomBBytes;     // decoded weight tile
     static constexpr int kTmemCols = ACC * BN;                   // fp32 accumulators, 128 lanes x BN each
     static constexpr int kRingA = BN == 256 ? 3 : (ACC == 2 ? 4 : 3);  // activation tiles in flight
-    static constexpr int kRingW = BN == 256 ? 4 : (ACC == 2 ? 8 : 4);  // record groups in flight
-    static constexpr int kRingB = BN == 256 ? 2 : (ACC == 2 ? 3 : 2);  // decoded tiles, decode -> MMA
+    static constexpr int kRingW = BN == 256 ? 4 : (ACC == 2 ? 8 : (ROWS == 64 ? 8 : 6));  // weight stages in flight
+    static constexpr int kRingB = BN == 256 ? 2 : (ACC == 2 ? 3 : (ROWS == 64 ? 3 : 2));  // decoded tiles, decode -> MMA
     static constexpr int kColParts = 4 / ACC;                    // epilogue warps per accumulator lane group
     static constexpr int kTpr = kDecodeThreads / BN;             // decode threads per weight row
     static constexpr int kBpt = kAtoms * (kBK / kBlockElems) / kTpr;  // 16-element blocks per thread
@@ -100,8 +105,6 @@ struct Cfg {
     struct Shared {
         uint64_t a_full[kRingA];   // activation tile landed (TMA bytes)
         uint64_t a_empty[kRingA];  // the MMAs that read it completed
-        uint64_t w_full[kRingW];   // weight records landed (bulk-copy bytes)
-        uint64_t w_empty[kRingW];  // the decode warps have read them
         uint64_t b_full[kRingB];   // the decode warps wrote the weight tile
         uint64_t b_empty[kRingB];  // the MMAs that read it completed
         uint64_t accum;            // every MMA of the tile completed
@@ -112,7 +115,11 @@ struct Cfg {
         uint32_t last;             // split K: this CTA finishes the tile
         float sd[256];             // decode scale for every E4M3 byte: fl(E4M3(b) / gs)
     };
-    static constexpr int kRingBytes = kRingA * kTileABytes + kRingB * kTileBBytes + kRingW * kRecPerStage * kRecBytes;
+    // weight ring slot: per decode thread its 8 kBpt code bytes, then per thread a 4-byte
+    // scale word
+    static constexpr int kCodeBytes = 8 * kBpt;
+    static constexpr int kWSlotBytes = kDecodeThreads * (kCodeBytes + 4);
+    static constexpr int kRingBytes = kRingA * kTileABytes + kRingB * kTileBBytes + kRingW * kWSlotBytes;
     static constexpr int kSmemBytes = 1024 + kRingBytes + (int)sizeof(Shared);
 
     static_assert(BN % kRecRows == 0 && BN >= 16 && BN <= 256, "MMA N");
@@ -122,6 +129,9 @@ struct Cfg {
     static_assert(kAtomABytes % 1024 == 0 && kAtomBBytes % 1024 == 0, "operand tiles stay 1024-byte aligned");
     static_assert(kDecodeWarps == 4 * ACC * kColParts, "epilogue warps");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+    static_assert(ROWS == kBM || (ACC == 1 && ROWS % 8 == 0 && ROWS < kBM), "rows kept in shared memory");
+    // the 128 rows the MMA reads from the last activation atom stay inside the rings
+    static_assert(kRingA * kTileABytes - kAtomABytes + kMmaM * kBK * 2 <= kRingBytes, "MMA reads stay in bounds");
 };
 
 // ---------------------------------------------------------------------------------------
@@ -192,12 +202,23 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
-// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from global to
-// shared memory, completing on `bar`.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(src), "r"(bytes), "r"(bar)
-                 : "memory");
+// Asynchronous copy of B bytes (4, 8 or 16; both addresses B-aligned) from global to shared
+// memory through the load path; complete for this thread after cp_async_wait.
+template <int B>
+__device__ __forceinline__ void cp_async(uint32_t dst, const void* src) {
+    static_assert(B == 4 || B == 8 || B == 16, "cp.async size");
+    if constexpr (B == 16)
+        asm volatile("cp.async.cg.shared.global.L2::128B [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(dst), "l"(src), "n"(B) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// Waits until at most N of this thread's commit groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
@@ -360,14 +381,29 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const v
     return __all_sync(0xFFFFFFFFu, got);
 }
 
-template <int BN, int ACC>
+// bf16x2 of bf16_rn(fl(LUT[code] * sd)) for the two codes of a byte (low nibble -> low
+// half), the two products as one packed f32x2 multiply.  sd2 holds sd in both halves.
+__device__ __forceinline__ uint32_t decode_pair_x2(uint32_t code_byte, uint64_t sd2) {
+    const uint32_t h2 = e2m1x2_to_f16x2(code_byte);
+    const float lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+    const float hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
+    uint64_t v, prod;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(prod) : "l"(v), "l"(sd2));
+    float plo, phi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(plo), "=f"(phi) : "l"(prod));
+    __nv_bfloat162 r = __floats2bfloat162_rn(plo, phi);
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+template <int BN, int ACC, int ROWS>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     w4a16_linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const LinearArgs a) {
-    using C = Cfg<BN, ACC>;
+    using C = Cfg<BN, ACC, ROWS>;
     constexpr int kBN = C::kBN, kRingA = C::kRingA, kRingB = C::kRingB, kRingW = C::kRingW;
     constexpr int kBM = C::kBM, kTileABytes = C::kTileABytes, kAtoms = C::kAtoms;
-    constexpr int kAtomABytes = C::kAtomABytes, kAtomBBytes = C::kAtomBBytes, kRecPerStage = C::kRecPerStage;
-    constexpr int kTileBBytes = C::kTileBBytes, kRecPerTile = C::kRecPerTile, kTpr = C::kTpr, kBpt = C::kBpt;
+    constexpr int kAtomABytes = C::kAtomABytes, kAtomBBytes = C::kAtomBBytes;
+    constexpr int kTileBBytes = C::kTileBBytes, kRecPerTile = C::kRecPerTile, kBpt = C::kBpt;
     constexpr uint32_t kIdesc = C::kIdesc;
     extern __shared__ uint8_t dsmem[];
     const uint32_t raw = smem_u32(dsmem);
@@ -396,10 +432,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(smem_u32(&sh.a_full[s]), 1);
             mbar_init(smem_u32(&sh.a_empty[s]), 1);
         }
-        for (int s = 0; s < kRingW; ++s) {
-            mbar_init(smem_u32(&sh.w_full[s]), 1);
-            mbar_init(smem_u32(&sh.w_empty[s]), kDecodeWarps);
-        }
         for (int s = 0; s < kRingB; ++s) {
             mbar_init(smem_u32(&sh.b_full[s]), kDecodeWarps);
             mbar_init(smem_u32(&sh.b_empty[s]), 1);
@@ -425,50 +457,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tmem = sh.tmem_base;
     const volatile uint32_t* abort = &sh.abort;
 
-    if (warp == kTmaWarp || warp == kRecWarp) {
-        // ---- producers: activation tiles (TMA) or weight records (bulk copy) ----
+    if (warp == kTmaWarp) {
+        // ---- producer: activation tiles (TMA) ----
         if (lane == 0) {
-            const bool act = warp == kTmaWarp;
-            const int R = act ? kRingA : kRingW;
-            const uint64_t* full = act ? sh.a_full : sh.w_full;
-            const uint64_t* empty = act ? sh.a_empty : sh.w_empty;
-            // the tile's weight rows are records (kRecPerTile * tn + i, kb); rows past the
-            // last record of the weight (N not a multiple of 256) read the last record again
-            // and are dropped by the epilogue
-            const int64_t nrec = (a.N + kRecRows - 1) / kRecRows;
             int issued = 0;
             for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % R;
-                const uint32_t ph = (uint32_t)(kb / R) & 1u;
-                if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, abort)) {
+                const int s = kb % kRingA;
+                if (!mbar_wait(smem_u32(&sh.a_empty[s]), ((uint32_t)(kb / kRingA) & 1u) ^ 1u, abort)) {
                     stop_all(sh, a.ws);
                     break;
                 }
-                const uint32_t bar = smem_u32(&full[s]);
+                const uint32_t bar = smem_u32(&sh.a_full[s]);
                 const int at0 = (kb0 + kb) * kAtoms;
                 const int na = min(kAtoms, (int)(a.kt - at0));  // atoms of this stage inside K
-                if (act) {
-                    mbar_arrive_expect_tx(bar, a.a_bytes * (uint32_t)na);
-                    for (int t = 0; t < na; ++t)
-                        tma_load_2d(sA0 + s * kTileABytes + t * kAtomABytes, &tmap_x, (at0 + t) * kBK, (int32_t)m0, bar);
-                } else {
-                    mbar_arrive_expect_tx(bar, (uint32_t)(na * kRecPerTile * kRecBytes));
-                    for (int t = 0; t < na; ++t) {
-#pragma unroll
-                        for (int i = 0; i < kRecPerTile; ++i) {
-                            int64_t rn = kRecPerTile * tn + i;
-                            if (rn >= nrec) rn = nrec - 1;
-                            bulk_load(sW0 + (s * kRecPerStage + t * kRecPerTile + i) * kRecBytes,
-                                      a.tiled + (rn * a.kt + at0 + t) * kRecBytes, kRecBytes, bar);
-                        }
-                    }
-                }
+                mbar_arrive_expect_tx(bar, a.a_bytes * (uint32_t)na);
+                for (int t = 0; t < na; ++t)
+                    tma_load_2d(sA0 + s * kTileABytes + t * kAtomABytes, &tmap_x, (at0 + t) * kBK, (int32_t)m0, bar);
                 ++issued;
             }
             // The copies in flight land before the CTA may exit (immediate when every
             // stage was consumed).
-            for (int kb = issued > R ? issued - R : 0; kb < issued; ++kb)
-                if (!mbar_wait(smem_u32(&full[kb % R]), (uint32_t)(kb / R) & 1u, abort, true)) stop_all(sh, a.ws);
+            for (int kb = issued > kRingA ? issued - kRingA : 0; kb < issued; ++kb)
+                if (!mbar_wait(smem_u32(&sh.a_full[kb % kRingA]), (uint32_t)(kb / kRingA) & 1u, abort, true))
+                    stop_all(sh, a.ws);
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
@@ -513,55 +524,88 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
     } else {
-        // ---- decode warps: kTpr threads per weight row, kBpt 16-element blocks each, all
-        //      in atom `atom` of the stage, from its block `bl0` on ----
-        const int row = threadIdx.x / kTpr;
-        const int part = threadIdx.x % kTpr;
+        // ---- decode warps: warp w decodes weight rows 32 (w % kRowWarps) .. + 31 of the tile,
+        //      one per lane, for part w / kRowWarps of each stage: kBpt 16-element blocks of
+        //      atom `atom`, from block `bl0` on.  Each thread copies what it decodes into a
+        //      private slot of the weight ring itself (cp.async, kRingW - 1 stages ahead): its
+        //      8 kBpt code bytes and its row's 4 scale bytes.  A warp's 16-byte stores into
+        //      the swizzled tile then cover 8 distinct bank groups per 8 lanes, and its reads
+        //      of the ring are consecutive words ----
+        constexpr int kRowWarps = kBN / 32;
+        const int row = 32 * (warp % kRowWarps) + lane;
+        const int part = warp / kRowWarps;
         const int atom = kBpt * part / (kBK / kBlockElems);
         const int bl0 = kBpt * part % (kBK / kBlockElems);
         const int rr = row % kRecRows;
+        // the tile's weight rows are records (kRecPerTile * tn + i, atom); rows past the last
+        // record of the weight (N not a multiple of 256) read the last record again and are
+        // dropped by the epilogue
+        const int64_t nrec = (a.N + kRecRows - 1) / kRecRows;
+        const int64_t rn = min(kRecPerTile * tn + row / kRecRows, nrec - 1);
+        const uint8_t* gcode = a.tiled + rn * a.kt * kRecBytes + rr * 32 + bl0 * 8;  // in record (rn, 0)
+        const uint8_t* gscale = a.tiled + rn * a.kt * kRecBytes + kRecCodes + rr * 4;
+        const uint32_t my_code = sW0 + threadIdx.x * C::kCodeBytes;
+        const uint32_t my_scale = sW0 + kDecodeThreads * C::kCodeBytes + threadIdx.x * 4;
+        const uint8_t* gmy_code = gW0 + threadIdx.x * C::kCodeBytes;
+        const uint8_t* gmy_scale = gW0 + kDecodeThreads * C::kCodeBytes + threadIdx.x * 4;
+        // stage s of this CTA into its ring slot; one commit group per stage, empty past the
+        // last stage or for an atom past the end of K
+        auto fetch = [&](int s) {
+            const int64_t at = (int64_t)(kb0 + s) * kAtoms + atom;
+            if (s < nk && at < a.kt) {
+                const uint32_t slot = (uint32_t)((s % kRingW) * C::kWSlotBytes);
+                cp_async<C::kCodeBytes>(my_code + slot, gcode + at * kRecBytes);
+                cp_async<4>(my_scale + slot, gscale + at * kRecBytes);
+            }
+            cp_async_commit();
+        };
+#pragma unroll 1
+        for (int s = 0; s < kRingW - 1; ++s) fetch(s);
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
             const int sw = kb % kRingW, sb = kb % kRingB;
-            if (!warp_wait(smem_u32(&sh.w_full[sw]), (uint32_t)(kb / kRingW) & 1u, abort) ||
-                !warp_wait(smem_u32(&sh.b_empty[sb]), ((uint32_t)(kb / kRingB) & 1u) ^ 1u, abort)) {
+            fetch(kb + kRingW - 1);       // into the slot of stage kb - 1, read by now
+            cp_async_wait<kRingW - 1>();  // the bytes of stage kb have landed
+            if (!warp_wait(smem_u32(&sh.b_empty[sb]), ((uint32_t)(kb / kRingB) & 1u) ^ 1u, abort)) {
                 if (lane == 0) stop_all(sh, a.ws);
                 ok = false;
                 break;
             }
             // an atom past the end of K is neither loaded nor multiplied
             const bool live = (kb0 + kb) * kAtoms + atom < a.kt;
-            const uint8_t* rec = gW0 + (sw * kRecPerStage + atom * kRecPerTile + row / kRecRows) * kRecBytes;
             uint32_t c[2 * kBpt];
             uint32_t sc = 0;
             if (!live) {
 #pragma unroll
                 for (int i = 0; i < 2 * kBpt; ++i) c[i] = 0;
-            } else if constexpr (kBpt == 2) {
-                const uint4 v = *reinterpret_cast<const uint4*>(rec + rr * 32 + bl0 * 8);
-                c[0] = v.x;
-                c[1] = v.y;
-                c[2] = v.z;
-                c[3] = v.w;
-                sc = *reinterpret_cast<const uint16_t*>(rec + kRecCodes + rr * 4 + bl0);
             } else {
-                const uint2 v = *reinterpret_cast<const uint2*>(rec + rr * 32 + bl0 * 8);
-                c[0] = v.x;
-                c[1] = v.y;
-                sc = rec[kRecCodes + rr * 4 + bl0];
+                if constexpr (kBpt == 2) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(gmy_code + sw * C::kWSlotBytes);
+                    c[0] = v.x;
+                    c[1] = v.y;
+                    c[2] = v.z;
+                    c[3] = v.w;
+                } else {
+                    const uint2 v = *reinterpret_cast<const uint2*>(gmy_code + sw * C::kWSlotBytes);
+                    c[0] = v.x;
+                    c[1] = v.y;
+                }
+                sc = *reinterpret_cast<const uint32_t*>(gmy_scale + sw * C::kWSlotBytes) >> (8 * bl0);
             }
             uint8_t* tile_row = gB0 + sb * kTileBBytes + atom * kAtomBBytes + row * 128;
 #pragma unroll
             for (int i = 0; i < kBpt; ++i) {
                 const float sd = sh.sd[(sc >> (8 * i)) & 0xFFu];
+                uint64_t sd2;
+                asm("mov.b64 %0, {%1, %1};" : "=l"(sd2) : "f"(sd));
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     const uint32_t w = c[2 * i + q];
                     uint32_t o[4];
-                    o[0] = decode_pair(w & 0xFFu, sd);
-                    o[1] = decode_pair((w >> 8) & 0xFFu, sd);
-                    o[2] = decode_pair((w >> 16) & 0xFFu, sd);
-                    o[3] = decode_pair(w >> 24, sd);
+                    o[0] = decode_pair_x2(w & 0xFFu, sd2);
+                    o[1] = decode_pair_x2((w >> 8) & 0xFFu, sd2);
+                    o[2] = decode_pair_x2((w >> 16) & 0xFFu, sd2);
+                    o[3] = decode_pair_x2(w >> 24, sd2);
                     const int chunk = 2 * (bl0 + i) + q;  // 8 elements = 16 bytes
                     const uint32_t dst = smem_u32(tile_row + ((chunk ^ (row & 7)) << 4));
                     asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(o[0]), "r"(o[1]), "r"(o[2]),
@@ -569,16 +613,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                  : "memory");
                 }
             }
-            // orders this thread's reads of the record and writes of the tile before the
-            // async-proxy operations that follow the arrivals (the next copy into the
-            // record slot, the MMAs reading the tile)
+            // orders this thread's writes of the tile before the MMAs that read it (async
+            // proxy), which follow the arrival
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(smem_u32(&sh.w_empty[sw]));
-                mbar_arrive(smem_u32(&sh.b_full[sb]));
-            }
+            if (lane == 0) mbar_arrive(smem_u32(&sh.b_full[sb]));
         }
+        cp_async_wait<0>();  // no copy of this thread lands after it leaves the loop
 
         // ---- epilogue: warp w reads lanes 32 * (w % 4) .. + 31 of accumulator (w / 4) % ACC,
         //      column part w / (4 ACC) of kColParts ----
@@ -688,12 +729,14 @@ nvfp4_status gemm_smem_optin() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevs) return NVFP4_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_w4_mu);
     if (!g_smem_set[dev]) {
-        if (cudaFuncSetAttribute(w4a16_linear_kernel<256, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(w4a16_linear_kernel<256, 2, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg<256, 2>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(w4a16_linear_kernel<128, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(w4a16_linear_kernel<128, 2, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg<128, 2>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(w4a16_linear_kernel<128, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg<128, 1>::kSmemBytes) != cudaSuccess)
+            cudaFuncSetAttribute(w4a16_linear_kernel<128, 1, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<128, 1>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(w4a16_linear_kernel<128, 1, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<128, 1, 64>::kSmemBytes) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         g_smem_set[dev] = true;
     }
@@ -850,11 +893,13 @@ static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const
     const unsigned grid = (unsigned)(tiles_m * tiles_n * a.splits);
     cudaStream_t cst = reinterpret_cast<cudaStream_t>(stream);
     if (bn == 256)
-        w4a16_linear_kernel<256, 2><<<grid, kGemmThreads, Cfg<256, 2>::kSmemBytes, cst>>>(map, a);
+        w4a16_linear_kernel<256, 2, 256><<<grid, kGemmThreads, Cfg<256, 2>::kSmemBytes, cst>>>(map, a);
     else if (acc == 2)
-        w4a16_linear_kernel<128, 2><<<grid, kGemmThreads, Cfg<128, 2>::kSmemBytes, cst>>>(map, a);
-    else
-        w4a16_linear_kernel<128, 1><<<grid, kGemmThreads, Cfg<128, 1>::kSmemBytes, cst>>>(map, a);
+        w4a16_linear_kernel<128, 2, 256><<<grid, kGemmThreads, Cfg<128, 2>::kSmemBytes, cst>>>(map, a);
+    else if (M > 64)
+        w4a16_linear_kernel<128, 1, 128><<<grid, kGemmThreads, Cfg<128, 1>::kSmemBytes, cst>>>(map, a);
+    else  // at most 64 rows: 64 rows of x per stage in shared memory, a deeper weight ring
+        w4a16_linear_kernel<128, 1, 64><<<grid, kGemmThreads, Cfg<128, 1, 64>::kSmemBytes, cst>>>(map, a);
     note_launch();
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

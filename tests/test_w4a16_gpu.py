@@ -120,7 +120,8 @@ def test_decoded_weight_is_exact_through_one_hot_rows(K):
     (1, 4096, 4096, False),    # one token
     (513, 2048, 1000, True),
     (100, 1040, 200, True),    # 128-row tiles: 17 atoms of K, the last stage half full and ragged
-    (64, 192, 256, False),     # 128-row tiles: 3 atoms, the second stage half full
+    (64, 192, 256, False),     # 128-row tiles: 3 atoms, the second stage half full; 64 rows kept
+    (65, 320, 130, True),      # 128-row tiles with all 128 rows kept, 5 atoms
 ])
 def test_linear_matches_oracle(M, K, N, with_bias):
     rng = np.random.default_rng(M * 7 + K * 3 + N)
