@@ -64,32 +64,33 @@ static_assert(kRecBytes % 16 == 0, "bulk copy size");
 // to 256 rows; 128 x 128 when it has at most 128 (half the MMA work and activation bytes
 // per stage, and deeper rings for the weight stream).
 //
-// ROWS is the number of rows of x a tile keeps in shared memory: kBM, or 64 for the 128 x 128
-// tiles when x has at most 64 rows.  The MMA always reads 128 rows per accumulator; with
-// ROWS = 64 rows 64-127 of an atom are whatever bytes follow it in shared memory (the next
+// ROWS is the number of rows of x a tile keeps in shared memory: kBM, or 64 / 32 for the
+// 128 x 128 tiles when x has at most 64 / 32 rows.  The MMA always reads 128 rows per
+// accumulator; past ROWS they are whatever bytes follow the atom in shared memory (the next
 // atom, or the decoded weight ring after the last one), and they only feed accumulator lanes
-// that the epilogue never stores.  The 64 KB this frees go to the weight ring: its depth sets
-// the bytes in flight from HBM, which is what bounds a tile at a few rows of x (a record is
-// ~2.5 us from issue to arrival under load).
+// that the epilogue never stores.  The room this frees goes to deeper rings (64 rows) or to
+// longer stages (32 rows).
 //
 // A stage covers kAtoms atoms of K (64 columns each, one 128-byte swizzle row per tile row):
-// 2 for the 128 x 128 tiles, where the time of a stage is mostly the fixed cost of handing it
-// from role to role, so that cost is paid once per 128 columns; 1 for the others.  Within a
+// 4 for the 128 x 128 tiles that keep 32 rows of x, 2 for the other 128 x 128 tiles, where a
+// good part of a stage's time is the fixed cost of handing it from role to role, so that
+// cost is paid once per 256 or 128 columns; 1 for the others.  Within a
 // stage, atom t of the activation tile sits at t * ROWS * 128 bytes (accumulator h's 128 rows
 // at + h * 16 KB) and atom t of the decoded weight tile at t * BN * 128 bytes.
 template <int BN, int ACC, int ROWS = kMmaM * ACC>
 struct Cfg {
     static constexpr int kBN = BN;
     static constexpr int kBM = kMmaM * ACC;
-    static constexpr int kAtoms = ACC == 1 ? 2 : 1;
+    static constexpr int kAtoms = ACC == 1 ? (ROWS == 32 ? 4 : 2) : 1;
     static constexpr int kAtomABytes = ROWS * kBK * 2;           // one 64-column atom of the activation tile
     static constexpr int kAtomBBytes = BN * kBK * 2;             // one 64-column atom of the weight tile
     static constexpr int kTileABytes = kAtoms * kAtomABytes;
     static constexpr int kRecPerTile = BN / kRecRows;            // records per atom
     static constexpr int kTileBBytes = kAtoms * kAtomBBytes;     // decoded weight tile
     static constexpr int kTmemCols = ACC * BN;                   // fp32 accumulators, 128 lanes x BN each
-    static constexpr int kRingA = BN == 256 ? 3 : (ACC == 2 ? 4 : 3);  // activation tiles in flight
-    static constexpr int kRingW = BN == 256 ? 4 : (ACC == 2 ? 8 : (ROWS == 64 ? 8 : 6));  // weight stages in flight
+    static constexpr int kRingA = BN == 256 ? 3 : (ACC == 2 ? 4 : (ROWS == 32 ? 2 : 3));  // activation tiles in flight
+    static constexpr int kRingW =  // weight stages in flight
+        BN == 256 ? 4 : (ACC == 2 ? 8 : (ROWS == 32 ? 3 : (ROWS == 64 ? 8 : 6)));
     static constexpr int kRingB = BN == 256 ? 2 : (ACC == 2 ? 3 : (ROWS == 64 ? 3 : 2));  // decoded tiles, decode -> MMA
     static constexpr int kColParts = 4 / ACC;                    // epilogue warps per accumulator lane group
     static constexpr int kTpr = kDecodeThreads / BN;             // decode threads per weight row
@@ -123,7 +124,8 @@ struct Cfg {
     static constexpr int kSmemBytes = 1024 + kRingBytes + (int)sizeof(Shared);
 
     static_assert(BN % kRecRows == 0 && BN >= 16 && BN <= 256, "MMA N");
-    static_assert(kTpr * kBpt == kAtoms * (kBK / kBlockElems) && kBpt >= 1 && kBpt <= 2, "decode split");
+    static_assert(kTpr * kBpt == kAtoms * (kBK / kBlockElems) && (kBpt == 1 || kBpt == 2 || kBpt == 4),
+                  "decode split");
     static_assert(kBpt == 1 || (kBK / kBlockElems) % kBpt == 0, "a thread's blocks lie in one atom");
     static_assert(kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0, "tensor memory columns");
     static_assert(kAtomABytes % 1024 == 0 && kAtomBBytes % 1024 == 0, "operand tiles stay 1024-byte aligned");
@@ -554,7 +556,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int64_t at = (int64_t)(kb0 + s) * kAtoms + atom;
             if (s < nk && at < a.kt) {
                 const uint32_t slot = (uint32_t)((s % kRingW) * C::kWSlotBytes);
-                cp_async<C::kCodeBytes>(my_code + slot, gcode + at * kRecBytes);
+                if constexpr (C::kCodeBytes == 32) {  // a whole row of the atom: two copies
+                    cp_async<16>(my_code + slot, gcode + at * kRecBytes);
+                    cp_async<16>(my_code + slot + 16, gcode + at * kRecBytes + 16);
+                } else {
+                    cp_async<C::kCodeBytes>(my_code + slot, gcode + at * kRecBytes);
+                }
                 cp_async<4>(my_scale + slot, gscale + at * kRecBytes);
             }
             cp_async_commit();
@@ -579,7 +586,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 2 * kBpt; ++i) c[i] = 0;
             } else {
-                if constexpr (kBpt == 2) {
+                if constexpr (kBpt == 4) {
+                    const uint4 v0 = *reinterpret_cast<const uint4*>(gmy_code + sw * C::kWSlotBytes);
+                    const uint4 v1 = *reinterpret_cast<const uint4*>(gmy_code + sw * C::kWSlotBytes + 16);
+                    c[0] = v0.x;
+                    c[1] = v0.y;
+                    c[2] = v0.z;
+                    c[3] = v0.w;
+                    c[4] = v1.x;
+                    c[5] = v1.y;
+                    c[6] = v1.z;
+                    c[7] = v1.w;
+                } else if constexpr (kBpt == 2) {
                     const uint4 v = *reinterpret_cast<const uint4*>(gmy_code + sw * C::kWSlotBytes);
                     c[0] = v.x;
                     c[1] = v.y;
@@ -736,7 +754,9 @@ nvfp4_status gemm_smem_optin() {
             cudaFuncSetAttribute(w4a16_linear_kernel<128, 1, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg<128, 1>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(w4a16_linear_kernel<128, 1, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg<128, 1, 64>::kSmemBytes) != cudaSuccess)
+                                 Cfg<128, 1, 64>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(w4a16_linear_kernel<128, 1, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<128, 1, 32>::kSmemBytes) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         g_smem_set[dev] = true;
     }
@@ -898,8 +918,10 @@ static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const
         w4a16_linear_kernel<128, 2, 256><<<grid, kGemmThreads, Cfg<128, 2>::kSmemBytes, cst>>>(map, a);
     else if (M > 64)
         w4a16_linear_kernel<128, 1, 128><<<grid, kGemmThreads, Cfg<128, 1>::kSmemBytes, cst>>>(map, a);
-    else  // at most 64 rows: 64 rows of x per stage in shared memory, a deeper weight ring
+    else if (M > 32)  // at most 64 rows: 64 rows of x per atom in shared memory, deeper rings
         w4a16_linear_kernel<128, 1, 64><<<grid, kGemmThreads, Cfg<128, 1, 64>::kSmemBytes, cst>>>(map, a);
+    else  // at most 32 rows: 32 rows of x per atom, stages of 256 columns of K
+        w4a16_linear_kernel<128, 1, 32><<<grid, kGemmThreads, Cfg<128, 1, 32>::kSmemBytes, cst>>>(map, a);
     note_launch();
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

@@ -122,6 +122,8 @@ def test_decoded_weight_is_exact_through_one_hot_rows(K):
     (100, 1040, 200, True),    # 128-row tiles: 17 atoms of K, the last stage half full and ragged
     (64, 192, 256, False),     # 128-row tiles: 3 atoms, the second stage half full; 64 rows kept
     (65, 320, 130, True),      # 128-row tiles with all 128 rows kept, 5 atoms
+    (20, 704, 300, True),      # 32 rows kept, stages of 4 atoms: 11 atoms, the last stage 3
+    (32, 1040, 200, True),     # 32 rows kept: 17 atoms, K % 64 == 16, the last stage 1 atom
 ])
 def test_linear_matches_oracle(M, K, N, with_bias):
     rng = np.random.default_rng(M * 7 + K * 3 + N)
