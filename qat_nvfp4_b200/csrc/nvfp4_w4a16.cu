@@ -72,11 +72,11 @@ static_assert(kRecBytes % 16 == 0, "bulk copy size");
 // longer stages (32 rows).
 //
 // A stage covers kAtoms atoms of K (64 columns each, one 128-byte swizzle row per tile row):
-// 4 for the 128 x 128 tiles that keep 32 rows of x, 2 for the other 128 x 128 tiles, where a
-// good part of a stage's time is the fixed cost of handing it from role to role, so that
-// cost is paid once per 256 or 128 columns; 1 for the others.  Within a
-// stage, atom t of the activation tile sits at t * ROWS * 128 bytes (accumulator h's 128 rows
-// at + h * 16 KB) and atom t of the decoded weight tile at t * BN * 128 bytes.
+// 4 for the 128 x 128 tiles that keep 32 rows of x, 2 for the other 128 x 128 tiles (a good
+// part of a stage's time there is the fixed cost of handing it from role to role, so that
+// cost is paid once per 256 or 128 columns), 1 for the others.  Within a stage, atom t of
+// the activation tile sits at t * ROWS * 128 bytes (accumulator h's 128 rows at + h * 16 KB)
+// and atom t of the decoded weight tile at t * BN * 128 bytes.
 template <int BN, int ACC, int ROWS = kMmaM * ACC>
 struct Cfg {
     static constexpr int kBN = BN;
@@ -101,8 +101,8 @@ struct Cfg {
     static constexpr uint32_t kIdesc =
         (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kMmaM >> 4) << 24);
 
-    // Shared memory: activation tiles, decoded weight tiles (both 1024-byte aligned),
-    // weight records, then the barriers and the table.
+    // Shared memory: activation tiles, decoded weight tiles (both 1024-byte aligned), the
+    // weight ring, then the barriers and the table.
     struct Shared {
         uint64_t a_full[kRingA];   // activation tile landed (TMA bytes)
         uint64_t a_empty[kRingA];  // the MMAs that read it completed
