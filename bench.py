@@ -61,6 +61,10 @@ def parse_args():
                    help="instead of the step benchmark, time the W4A16 linear (x . W^T with W stored as NVFP4 "
                         "records) for several token counts on the pages' weight shapes, beside dequantize + "
                         "torch bf16 linear and a bf16 linear on an unquantized weight; print a table, write JSON")
+    p.add_argument("--strided", metavar="OUT_JSON", default=None,
+                   help="time amax / quantize / in-place fake-quant on the q, k and v column views of a fused "
+                        "[16384, 6144] projection output against the same calls on contiguous copies "
+                        "(L2 flushed before each rep), print a table and write it as JSON to OUT_JSON")
     p.add_argument("--linear-shape", metavar="M,K,N", default=None,
                    help="run the W4A16 linear three times on one shape (tokens M, in-features K, out-features "
                         "N; N(0, 1) activations, N(0, 0.02) weight) and exit: the command profiled by ncu")
@@ -81,7 +85,7 @@ def workload_config(args, world):
 
 # The sources of the kernels the step runs (the W4A16 linear has its own file).
 STEP_SOURCES = ("nvfp4_device.cuh", "nvfp4_runtime.h", "nvfp4_stream.cuh", "nvfp4_reduce.cuh", "nvfp4_encode.cuh",
-                "nvfp4_ragged.cuh", "nvfp4_kernels.cu")
+                "nvfp4_ragged.cuh", "nvfp4_strided.cuh", "nvfp4_kernels.cu")
 
 
 def source_digest():
@@ -596,6 +600,73 @@ def run_linear(args):
     return 0
 
 
+def run_strided(args):
+    """amax, quantize and in-place fake-quant of row-strided views: the q, k and v columns
+    (4096, 1024, 1024 wide) of a fused projection output of 16384 tokens (row stride 6144),
+    each > L2, against the same calls on contiguous copies of the views.  GB/s counts the
+    algorithmic bytes of the view (2, 2.5625 and 4 per element); CUDA events, median of 15,
+    L2 flushed by a 512 MB read before each rep."""
+    import torch
+    from qat_nvfp4_b200 import nvfp4 as nv
+    from qat_nvfp4_b200 import synthetic
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, peak_src = hbm_peak()
+    flush = torch.ones(512 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn, reps=15):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.sum(dtype=torch.int32)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1))
+        return sorted(ts)[len(ts) // 2] / 1e3
+
+    T, widths = 16384, (4096, 1024, 1024)
+    fused = synthetic.activation_normal_device((T, sum(widths)), 21, dev)
+    rows, c0 = [], 0
+    for name, w in zip(("q", "k", "v"), widths):
+        view = fused[:, c0:c0 + w]
+        c0 += w
+        copy = view.contiguous()
+        n = view.numel()
+        amax = nv.nvfp4_amax(view)
+        packed = torch.empty((T, w // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty((T, w // 16), dtype=torch.uint8, device=dev)
+        gs = torch.empty(1, dtype=torch.float32, device=dev)
+        r = {"view": name, "shape": [T, w], "row_stride": sum(widths)}
+        for label, x in (("strided", view), ("contiguous", copy)):
+            a = torch.empty(1, dtype=torch.float32, device=dev)
+            keep = x.clone()
+            t_amax = timed(lambda: nv.nvfp4_amax(x, out=a))
+            t_q = timed(lambda: nv.nvfp4_quantize(x, amax, packed, scales, gs))
+            t_fq = timed(lambda: nv.nvfp4_fake_quant(x, amax, out=x))  # in place, as a QAT forward on a view
+            x.copy_(keep)
+            for op, t, bpe in (("amax", t_amax, 2.0), ("quantize", t_q, 2.5625), ("fake_quant", t_fq, 4.0)):
+                r[f"{op}_{label}_us"] = t * 1e6
+                r[f"{op}_{label}_gbs"] = n * bpe / t / 1e9
+        rows.append(r)
+    print(f"HBM peak {peak:.1f} GB/s ({peak_src})")
+    print("| view | shape (row stride) | op | strided us | GB/s (frac) | contiguous copy us | GB/s (frac) |")
+    print("|---|---|---|---|---|---|---|")
+    for r in rows:
+        for op in ("amax", "quantize", "fake_quant"):
+            gs_s, gs_c = r[f"{op}_strided_gbs"], r[f"{op}_contiguous_gbs"]
+            print(f"| {r['view']} | {r['shape'][0]}x{r['shape'][1]} ({r['row_stride']}) | {op} | "
+                  f"{r[f'{op}_strided_us']:.1f} | {gs_s:.0f} ({gs_s / peak:.2f}) | "
+                  f"{r[f'{op}_contiguous_us']:.1f} | {gs_c:.0f} ({gs_c / peak:.2f}) |")
+    with open(args.strided, "w") as f:
+        json.dump({"hbm_gbs": peak, "rows": rows}, f, indent=1)
+    return 0
+
+
 def run_linear_shape(args):
     import torch
     from qat_nvfp4_b200 import nvfp4 as nv
@@ -626,6 +697,8 @@ def main():
         return run_linear(args)
     if args.linear_shape:
         return run_linear_shape(args)
+    if args.strided:
+        return run_strided(args)
     if args.cols < 1 or args.rows < 1:
         raise SystemExit("--rows and --cols must be positive")
     if args.impl == "reference":

@@ -284,6 +284,25 @@ nvfp4_status nvfp4_fake_quant(const void* x, void* y, int64_t M, int64_t N, cons
 nvfp4_status nvfp4_fake_quant_siblings(int k, const void* const* xs, void* const* ys, const int64_t* Ms,
                                        const int64_t* Ns, float* d_shared_amax, nvfp4_stream_t stream);
 
+/* ---- row-strided views -------------------------------------------------------------- */
+
+/* The same amax, quantize and fake-quant on a row-strided view: x is [M, N] bf16 whose row
+ * r starts ldx elements after row r - 1 (ldx >= N), e.g. the q, k or v columns of a fused
+ * projection's output ([QATLIN] section 4 treats such siblings as separate tensors), read in
+ * place instead of copied out first.  Requirements: N % 16 == 0 (else NVFP4_ERR_SHAPE),
+ * ldx (and ldy) >= N and a multiple of 16 (else NVFP4_ERR_ARG), x and y 32-byte aligned.
+ * Results are bit for bit those of the contiguous calls on the same values; packed and
+ * scales are written contiguous ([M, N/2] and [M, N/16]).  For fake-quant, y is a view of
+ * the same shape with row stride ldy; y == x with ldy == ldx is in place, and any other
+ * overlap of the two spans ((M - 1) ld + N elements each) is NVFP4_ERR_ARG.  amax enqueues
+ * a memset and one kernel, the others one kernel each. */
+nvfp4_status nvfp4_amax_strided(const void* x, int64_t M, int64_t N, int64_t ldx, float* d_amax,
+                                nvfp4_stream_t stream);
+nvfp4_status nvfp4_quantize_strided(const void* x, int64_t M, int64_t N, int64_t ldx, const float* d_amax,
+                                    uint8_t* packed, uint8_t* scales, float* d_global_scale, nvfp4_stream_t stream);
+nvfp4_status nvfp4_fake_quant_strided(const void* x, int64_t ldx, void* y, int64_t ldy, int64_t M, int64_t N,
+                                      const float* d_amax, nvfp4_stream_t stream);
+
 /* ---- blocks of 16 or 32 elements ---------------------------------------------------- */
 
 /* The three block calls with the block length as an argument, as [FP4OPT]

@@ -38,6 +38,7 @@
 #include "nvfp4_reduce.cuh"
 #include "nvfp4_encode.cuh"
 #include "nvfp4_ragged.cuh"
+#include "nvfp4_strided.cuh"
 
 namespace nvfp4 {
 namespace {
@@ -644,6 +645,85 @@ static nvfp4_status fake_quant_impl(const void* x, void* y, int64_t M, int64_t N
                   NVFP4_GRID_FQ, &grid);
     if (st != NVFP4_OK) return st;
     fake_quant_kernel<false, kW><<<grid, kThreads, 0, cs(stream)>>>(L, nblk, d_amax);
+    return after_launch();
+}
+
+// A row-strided [M, N] view: N % 16 == 0, row stride ld >= N elements with ld % 16 == 0,
+// and a span of (M - 1) ld + N elements that stays below kMaxElems.
+static nvfp4_status check_strided(int64_t M, int64_t N, int64_t ld, Strided* S, int64_t* span) {
+    int64_t numel = 0;
+    nvfp4_status st = check_matrix(M, N, &numel);
+    if (st != NVFP4_OK) return st;
+    if (N % kBlockElems != 0) return NVFP4_ERR_SHAPE;
+    if (ld < N || ld % kBlockElems != 0 || ld > kMaxElems) return NVFP4_ERR_ARG;
+    if (M > 1 && ld > 0 && M - 1 > (kMaxElems - N) / ld) return NVFP4_ERR_SHAPE;
+    S->nb = N / kBlockElems;
+    S->ld_bytes = ld * 2;
+    S->total = M * S->nb;
+    *span = M > 0 ? (M - 1) * ld + N : 0;
+    return NVFP4_OK;
+}
+
+NVFP4_API nvfp4_status nvfp4_amax_strided(const void* x, int64_t M, int64_t N, int64_t ldx, float* d_amax,
+                                          nvfp4_stream_t stream) {
+    Strided S;
+    int64_t span = 0;
+    nvfp4_status st = check_strided(M, N, ldx, &S, &span);
+    if (st != NVFP4_OK) return st;
+    if (d_amax == nullptr || (S.total > 0 && x == nullptr)) return NVFP4_ERR_NULL;
+    if (!aligned(d_amax, 4) || (S.total > 0 && !aligned(x, 32))) return NVFP4_ERR_ALIGN;
+    if (cudaMemsetAsync(d_amax, 0, sizeof(float), cs(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (S.total == 0) return NVFP4_OK;
+    int grid = 1;
+    st = grid_for(reinterpret_cast<const void*>(&amax_strided_kernel), S.total, kUnrollAmax, NVFP4_GRID_AMAX, &grid);
+    if (st != NVFP4_OK) return st;
+    amax_strided_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), S,
+                                                           reinterpret_cast<unsigned*>(d_amax));
+    return after_launch();
+}
+
+NVFP4_API nvfp4_status nvfp4_quantize_strided(const void* x, int64_t M, int64_t N, int64_t ldx, const float* d_amax,
+                                              uint8_t* packed, uint8_t* scales, float* d_global_scale,
+                                              nvfp4_stream_t stream) {
+    Strided S;
+    int64_t span = 0;
+    nvfp4_status st = check_strided(M, N, ldx, &S, &span);
+    if (st != NVFP4_OK) return st;
+    if (d_amax == nullptr) return NVFP4_ERR_NULL;
+    if (S.total > 0 && (x == nullptr || packed == nullptr || scales == nullptr)) return NVFP4_ERR_NULL;
+    if (!aligned(d_amax, 4) || (d_global_scale && !aligned(d_global_scale, 4))) return NVFP4_ERR_ALIGN;
+    if (S.total > 0 && (!aligned(x, 32) || !aligned(packed, 8))) return NVFP4_ERR_ALIGN;
+    if (S.total == 0 && d_global_scale == nullptr) return NVFP4_OK;
+    int grid = 1;
+    st = grid_for(reinterpret_cast<const void*>(&quantize_strided_kernel), S.total, kUnrollQ, NVFP4_GRID_Q, &grid);
+    if (st != NVFP4_OK) return st;
+    quantize_strided_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), S, d_amax, packed,
+                                                               scales, d_global_scale);
+    return after_launch();
+}
+
+NVFP4_API nvfp4_status nvfp4_fake_quant_strided(const void* x, int64_t ldx, void* y, int64_t ldy, int64_t M, int64_t N,
+                                                const float* d_amax, nvfp4_stream_t stream) {
+    Strided S, Sy;
+    int64_t span = 0, span_y = 0;
+    nvfp4_status st = check_strided(M, N, ldx, &S, &span);
+    if (st != NVFP4_OK) return st;
+    st = check_strided(M, N, ldy, &Sy, &span_y);
+    if (st != NVFP4_OK) return st;
+    if (d_amax == nullptr || (S.total > 0 && (x == nullptr || y == nullptr))) return NVFP4_ERR_NULL;
+    if (!aligned(d_amax, 4) || (S.total > 0 && (!aligned(x, 32) || !aligned(y, 32)))) return NVFP4_ERR_ALIGN;
+    if (S.total == 0) return NVFP4_OK;
+    // in place only as the same view; otherwise the two spans may not meet
+    const bool same = x == y && ldx == ldy;
+    if (!same) {
+        const uintptr_t px = reinterpret_cast<uintptr_t>(x), py = reinterpret_cast<uintptr_t>(y);
+        if (px < py + (uintptr_t)(span_y * 2) && py < px + (uintptr_t)(span * 2)) return NVFP4_ERR_ARG;
+    }
+    int grid = 1;
+    st = grid_for(reinterpret_cast<const void*>(&fake_quant_strided_kernel), S.total, kUnrollFq, NVFP4_GRID_FQ, &grid);
+    if (st != NVFP4_OK) return st;
+    fake_quant_strided_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), S,
+                                                                 static_cast<uint8_t*>(y), ldy * 2, d_amax);
     return after_launch();
 }
 

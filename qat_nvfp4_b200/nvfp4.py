@@ -64,6 +64,9 @@ _c_quantize_mma = _sig("nvfp4_quantize_mma", [_vp, _i64, _i64, _vp, _vp, _vp, _v
 _c_quantize_fused = _sig("nvfp4_quantize_fused", [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp])
 _c_dequantize = _sig("nvfp4_dequantize", [_vp, _vp, _vp, _i64, _i64, _vp, _vp])
 _c_fake_quant = _sig("nvfp4_fake_quant", [_vp, _vp, _i64, _i64, _vp, _vp])
+_c_amax_strided = _sig("nvfp4_amax_strided", [_vp, _i64, _i64, _i64, _vp, _vp])
+_c_quantize_strided = _sig("nvfp4_quantize_strided", [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp])
+_c_fake_quant_strided = _sig("nvfp4_fake_quant_strided", [_vp, _i64, _vp, _i64, _i64, _i64, _vp, _vp])
 _c_quantize_bs = _sig("nvfp4_quantize_bs", [_vp, _i64, _i64, ctypes.c_int, _vp, _vp, _vp, _vp, _vp])
 _c_dequantize_bs = _sig("nvfp4_dequantize_bs", [_vp, _vp, _vp, _i64, _i64, ctypes.c_int, _vp, _vp])
 _c_fake_quant_bs = _sig("nvfp4_fake_quant_bs", [_vp, _vp, _i64, _i64, ctypes.c_int, _vp, _vp])
@@ -102,16 +105,29 @@ def _stream(device: torch.device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
-def _cuda(t: torch.Tensor, name: str, dtype=None):
+def _cuda(t: torch.Tensor, name: str, dtype=None, contiguous: bool = True):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if not t.is_cuda:
         raise RuntimeError(f"{name} must be a CUDA tensor (libnvfp4 has no CPU path)")
     if dtype is not None and t.dtype != dtype:
         raise RuntimeError(f"{name} must be {dtype}, got {t.dtype}")
-    if not t.is_contiguous():
+    if contiguous and not t.is_contiguous():
         raise RuntimeError(f"{name} must be contiguous")
     return t
+
+
+def _row_stride(t: torch.Tensor, name: str):
+    """None for a contiguous tensor; the row stride (elements) of a 2-D bf16 view that the
+    strided calls take: unit column stride, N % 16 == 0, row stride a multiple of 16 and at
+    least N -- one of q/k/v inside a fused projection output, for instance."""
+    _cuda(t, name, torch.bfloat16, contiguous=False)
+    if t.is_contiguous():
+        return None
+    if t.dim() != 2 or t.stride(1) != 1 or t.shape[1] % 16 or t.stride(0) % 16 or t.stride(0) < t.shape[1]:
+        raise RuntimeError(f"{name} must be contiguous, or a 2-D view with contiguous rows, a row stride that "
+                           f"is a multiple of 16 elements and a multiple-of-16 row length")
+    return t.stride(0)
 
 
 def _scalar(t: torch.Tensor, name: str):
@@ -159,13 +175,18 @@ def _workspace(ws: torch.Tensor, device):
 def nvfp4_amax(x: torch.Tensor, out: torch.Tensor | None = None,
                workspace: torch.Tensor | None = None) -> torch.Tensor:
     """Exact max |x| of a bf16 tensor, as a 1-element fp32 CUDA tensor.  With a workspace
-    (see new_workspace) it is one kernel launch instead of a memset and a kernel."""
-    _cuda(x, "x", torch.bfloat16)
+    (see new_workspace) it is one kernel launch instead of a memset and a kernel.  x may also
+    be a row-strided 2-D view (one of q/k/v inside a fused projection output), read in place
+    by nvfp4_amax_strided."""
+    ld = _row_stride(x, "x")
     if out is None:
         out = torch.empty(1, dtype=torch.float32, device=x.device)
     _scalar(out, "out")
     with torch.cuda.device(x.device):
-        if workspace is None:
+        if ld is not None:
+            _check(_c_amax_strided(x.data_ptr(), x.shape[0], x.shape[1], ld, out.data_ptr(), _stream(x.device)),
+                   "nvfp4_amax_strided")
+        elif workspace is None:
             _check(_c_amax(x.data_ptr(), x.numel(), out.data_ptr(), _stream(x.device)), "nvfp4_amax")
         else:
             _workspace(workspace, x.device)
@@ -254,7 +275,10 @@ def nvfp4_quantize(x: torch.Tensor, amax: torch.Tensor, packed: torch.Tensor | N
     global scale fp32 [1]), P = block * ceil(N / block).  ``amax`` is the tensor's (or
     siblings', or observer's) amax; ``block`` is 16 (NVFP4) or 32."""
     block = _block(block)
-    M, N = _matrix(x)
+    ld = _row_stride(x, "x")
+    if ld is not None and block != 16:
+        raise RuntimeError("row-strided views are quantized in blocks of 16")
+    M, N = (x.shape[0], x.shape[1]) if ld is not None else _matrix(x)
     _scalar(amax, "amax")
     B = padded_blocks(N, block)
     lead = tuple(x.shape[:-1])
@@ -270,7 +294,10 @@ def nvfp4_quantize(x: torch.Tensor, amax: torch.Tensor, packed: torch.Tensor | N
     if packed.numel() != M * block // 2 * B or scales.numel() != M * B:
         raise RuntimeError("packed / scales have the wrong number of elements")
     with torch.cuda.device(x.device):
-        if block == 16:
+        if ld is not None:
+            st = _c_quantize_strided(x.data_ptr(), M, N, ld, amax.data_ptr(), packed.data_ptr(), scales.data_ptr(),
+                                     global_scale.data_ptr(), _stream(x.device))
+        elif block == 16:
             st = _c_quantize(x.data_ptr(), M, N, amax.data_ptr(), packed.data_ptr(), scales.data_ptr(),
                              global_scale.data_ptr(), _stream(x.device))
         else:
@@ -376,15 +403,26 @@ def nvfp4_dequantize(packed: torch.Tensor, scales: torch.Tensor, global_scale: t
 def nvfp4_fake_quant(x: torch.Tensor, amax: torch.Tensor, out: torch.Tensor | None = None,
                      block: int = 16) -> torch.Tensor:
     """bf16 -> bf16 fake-quantization (dequantize(quantize(x)) in one pass).  ``out`` may be x;
-    ``block`` is 16 (NVFP4) or 32."""
+    ``block`` is 16 (NVFP4) or 32.  With blocks of 16, x and out may also be row-strided 2-D
+    views (q/k/v inside a fused projection output), read and written in place."""
     block = _block(block)
-    M, N = _matrix(x)
-    _scalar(amax, "amax")
+    ld = _row_stride(x, "x")
     if out is None:
-        out = torch.empty_like(x)
-    _cuda(out, "out", torch.bfloat16)
+        out = torch.empty(x.shape, dtype=x.dtype, device=x.device)
+    ld_out = _row_stride(out, "out")
+    _scalar(amax, "amax")
     if out.numel() != x.numel():
         raise RuntimeError("out has the wrong number of elements")
+    if ld is not None or ld_out is not None:
+        if block != 16 or x.dim() != 2 or tuple(out.shape) != tuple(x.shape):
+            raise RuntimeError("row-strided fake-quant takes 2-D views of one shape and blocks of 16")
+        M, N = x.shape
+        with torch.cuda.device(x.device):
+            _check(_c_fake_quant_strided(x.data_ptr(), N if ld is None else ld, out.data_ptr(),
+                                         N if ld_out is None else ld_out, M, N, amax.data_ptr(), _stream(x.device)),
+                   "nvfp4_fake_quant_strided")
+        return out
+    M, N = _matrix(x)
     with torch.cuda.device(x.device):
         if block == 16:
             st = _c_fake_quant(x.data_ptr(), out.data_ptr(), M, N, amax.data_ptr(), _stream(x.device))
@@ -583,7 +621,11 @@ class FakeQuantSTE(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, x, amax, block=16):
-        return nvfp4_fake_quant(x.contiguous(), amax, block=block)
+        # row-strided 2-D views go to the strided kernel as they are; other layouts are
+        # made contiguous first
+        strided_ok = (x.dim() == 2 and x.stride(1) == 1 and x.shape[1] % 16 == 0 and x.stride(0) % 16 == 0
+                      and x.stride(0) >= x.shape[1] and block == 16)
+        return nvfp4_fake_quant(x if x.is_contiguous() or strided_ok else x.contiguous(), amax, block=block)
 
     @staticmethod
     def backward(ctx, grad_output):

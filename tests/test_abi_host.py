@@ -33,7 +33,8 @@ def test_header_declares_the_entry_points():
                      "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fake_quant", "nvfp4_fake_quant_siblings",
                      "nvfp4_quantize_bs", "nvfp4_dequantize_bs", "nvfp4_fake_quant_bs", "nvfp4_w4a16_linear",
                      "nvfp4_w4a16_pack", "nvfp4_w4a16_tiled_bytes", "nvfp4_quantize_fused",
-                     "nvfp4_amax_accumulate", "nvfp4_w4a16_workspace_bytes",
+                     "nvfp4_amax_accumulate", "nvfp4_w4a16_workspace_bytes", "nvfp4_amax_strided",
+                     "nvfp4_quantize_strided", "nvfp4_fake_quant_strided",
                      "nvfp4_status_string", "nvfp4_kernel_launch_count"]:
         assert required in names
 
@@ -114,6 +115,22 @@ def test_validation_errors_launch_nothing(lib):
         (ERR_NULL, "nvfp4_quantize", _p(A32), _i(2), _i(16), amax, _p(A32), _p(0), gs, S),
         (ERR_ALIGN, "nvfp4_quantize", _p(A32), _i(2), _i(16), amax, _p(A32 + 4), _p(A32), gs, S),
         (ERR_ALIGN, "nvfp4_quantize", _p(A8), _i(2), _i(16), amax, _p(A32), _p(A32), gs, S),
+        # row-strided views: amax(x, M, N, ldx, amax), quantize(x, M, N, ldx, amax, packed, scales, gs),
+        # fake_quant(x, ldx, y, ldy, M, N, amax)
+        (ERR_ARG, "nvfp4_amax_strided", _p(A32), _i(4), _i(32), _i(16), amax, S),          # ldx < N
+        (ERR_ARG, "nvfp4_amax_strided", _p(A32), _i(4), _i(32), _i(40), amax, S),          # ldx % 16
+        (ERR_SHAPE, "nvfp4_amax_strided", _p(A32), _i(4), _i(24), _i(48), amax, S),        # N % 16
+        (ERR_SHAPE, "nvfp4_amax_strided", _p(A32), _i(1 << 50), _i(16), _i(1 << 20), amax, S),  # span too large
+        (ERR_NULL, "nvfp4_amax_strided", _p(0), _i(4), _i(32), _i(64), amax, S),
+        (ERR_ALIGN, "nvfp4_amax_strided", _p(A8), _i(4), _i(32), _i(64), amax, S),
+        (ERR_ARG, "nvfp4_quantize_strided", _p(A32), _i(2), _i(32), _i(16), amax, _p(A32), _p(A32), gs, S),
+        (ERR_NULL, "nvfp4_quantize_strided", _p(A32), _i(2), _i(32), _i(64), _p(0), _p(A32), _p(A32), gs, S),
+        (ERR_ALIGN, "nvfp4_quantize_strided", _p(A32), _i(2), _i(32), _i(64), amax, _p(A32 + 4), _p(A32), gs, S),
+        (ERR_ARG, "nvfp4_fake_quant_strided", _p(A32), _i(64), _p(A32 + 64), _i(64), _i(2), _i(32), amax, S),  # k inside q's span
+        (ERR_ARG, "nvfp4_fake_quant_strided", _p(A32), _i(64), _p(A32), _i(96), _i(2), _i(32), amax, S),  # same start, other stride
+        (ERR_ARG, "nvfp4_fake_quant_strided", _p(A32), _i(64), _p(A32 + 8192), _i(24), _i(2), _i(32), amax, S),  # ldy < N
+        (ERR_ALIGN, "nvfp4_fake_quant_strided", _p(A32), _i(64), _p(A32 + 8200), _i(64), _i(2), _i(32), amax, S),
+        (ERR_NULL, "nvfp4_fake_quant_strided", _p(A32), _i(64), _p(A32 + 8192), _i(64), _i(2), _i(32), _p(0), S),
         # dequantize
         (ERR_NULL, "nvfp4_dequantize", _p(A32), _p(A32), _p(0), _i(2), _i(16), _p(A32), S),
         (ERR_ALIGN, "nvfp4_dequantize", _p(A32), _p(A32), gs, _i(2), _i(16), _p(A8), S),

@@ -124,6 +124,7 @@ def test_decoded_weight_is_exact_through_one_hot_rows(K):
     (65, 320, 130, True),      # 128-row tiles with all 128 rows kept, 5 atoms
     (20, 704, 300, True),      # 32 rows kept, stages of 4 atoms: 11 atoms, the last stage 3
     (32, 1040, 200, True),     # 32 rows kept: 17 atoms, K % 64 == 16, the last stage 1 atom
+    (33, 1040, 200, True),     # one row past the 32-row configuration
 ])
 def test_linear_matches_oracle(M, K, N, with_bias):
     rng = np.random.default_rng(M * 7 + K * 3 + N)
@@ -189,7 +190,7 @@ def test_empty_rows_launch_nothing():
     assert nv.nvfp4_kernel_launch_count() == before
 
 
-@pytest.mark.parametrize("M,K", [(1, 4096), (16, 4096), (100, 4096), (16, 1088), (7, 4160)])
+@pytest.mark.parametrize("M,K", [(1, 4096), (16, 4096), (32, 4096), (33, 4096), (100, 4096), (16, 1088), (7, 4160)])
 def test_split_k_for_few_rows(M, K):
     """Up to 128 rows of x on a weight with few output tiles (4096 x 4096: 32 tiles) the call
     splits K over several CTAs when the workspace is large enough; the result is within the
