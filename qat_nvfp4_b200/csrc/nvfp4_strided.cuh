@@ -22,11 +22,38 @@ struct Strided {
     int64_t total;     // M * nb
 };
 
-// Byte offset of block g (32-bit division whenever the sizes allow).
-__device__ __forceinline__ int64_t strided_offset(const Strided& S, int64_t g) {
-    int64_t r;
-    if (S.total <= 0xFFFFFFFFll) r = (int64_t)((uint32_t)g / (uint32_t)S.nb);
-    else r = g / S.nb;
+// Unsigned 32-bit division by an invariant d >= 1 as a multiply-high, two shifts and two
+// adds (Granlund and Montgomery, "Division by invariant integers using multiplication",
+// 1994, the unsigned N-bit method): with l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d)
+// + 1, n / d = (t + ((n - t) >> min(l, 1))) >> max(l - 1, 0) for t = mulhi(m, n), for every
+// n < 2^32.  Each thread sets it up once, so a block's row costs no division.
+struct Div32 {
+    uint32_t m, s1, s2;
+};
+
+__device__ __forceinline__ Div32 div32_of(uint32_t d) {
+    const uint32_t l = 32u - (uint32_t)__clz((int)(d - 1u));  // ceil(log2 d); 0 for d = 1
+    Div32 v;
+    v.m = (uint32_t)((((uint64_t)1 << 32) * (((uint64_t)1 << l) - d)) / d + 1u);
+    v.s1 = l < 1u ? l : 1u;
+    v.s2 = l > 1u ? l - 1u : 0u;
+    return v;
+}
+
+__device__ __forceinline__ uint32_t div32(uint32_t n, const Div32& v) {
+    const uint32_t t = __umulhi(v.m, n);
+    return (t + ((n - t) >> v.s1)) >> v.s2;
+}
+
+// Row of block g: the multiply-high form while block indices fit 32 bits, else a 64-bit
+// division.
+__device__ __forceinline__ int64_t strided_row(const Strided& S, const Div32& v, int64_t g) {
+    return S.total <= 0xFFFFFFFFll ? (int64_t)div32((uint32_t)g, v) : g / S.nb;
+}
+
+// Byte offset of block g.
+__device__ __forceinline__ int64_t strided_offset(const Strided& S, const Div32& v, int64_t g) {
+    const int64_t r = strided_row(S, v, g);
     return r * S.ld_bytes + (g - r * S.nb) * kBlockBytesIn;
 }
 
@@ -34,8 +61,9 @@ __device__ __forceinline__ int64_t strided_offset(const Strided& S, int64_t g) {
 // host beforehand), as amax_kernel does for contiguous tensors.
 __global__ void __launch_bounds__(kThreads) amax_strided_kernel(const uint8_t* __restrict__ x, Strided S, unsigned* out) {
     uint32_t m = 0;
+    const Div32 v = div32_of((uint32_t)S.nb);
     stream_blocks<kUnrollAmax, false, Block32>(
-        S.total, [&](int64_t g, Block32& b) { ld_b256_ro(x + strided_offset(S, g), b.w); },
+        S.total, [&](int64_t g, Block32& b) { ld_b256_ro(x + strided_offset(S, v, g), b.w); },
         [&](int64_t, Block32& b) {
             m = absmax_bf16x2(m, absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(b.w[0], b.w[1]), absmax_bf16x2(b.w[2], b.w[3])),
                                                absmax_bf16x2(absmax_bf16x2(b.w[4], b.w[5]), absmax_bf16x2(b.w[6], b.w[7]))));
@@ -50,8 +78,9 @@ __global__ void __launch_bounds__(kThreads)
                             uint8_t* __restrict__ packed, uint8_t* __restrict__ scales, float* __restrict__ d_gs) {
     __shared__ float4 tab[128];
     float gs = 0.0f;
+    const Div32 v = div32_of((uint32_t)S.nb);
     stream_blocks<kUnrollQ, NVFP4_PIPE_Q != 0, Block32>(
-        S.total, [&](int64_t g, Block32& b) { ld_block_ro(x + strided_offset(S, g), b.w); },
+        S.total, [&](int64_t g, Block32& b) { ld_block_ro(x + strided_offset(S, v, g), b.w); },
         [&](int64_t g, Block32& b) {
             uint32_t c[8];
             float sd;
@@ -71,12 +100,11 @@ __global__ void __launch_bounds__(kThreads)
     fake_quant_strided_kernel(const uint8_t* x, Strided S, uint8_t* y, int64_t ld_y, const float* d_amax) {
     __shared__ float4 tab[128];
     float gs = 0.0f;
+    const Div32 v = div32_of((uint32_t)S.nb);
     stream_blocks<kUnrollFq, NVFP4_PIPE_FQ != 0, FqSlot<8>>(
         S.total,
         [&](int64_t g, FqSlot<8>& sl) {
-            int64_t r;
-            if (S.total <= 0xFFFFFFFFll) r = (int64_t)((uint32_t)g / (uint32_t)S.nb);
-            else r = g / S.nb;
+            const int64_t r = strided_row(S, v, g);
             const int64_t c = (g - r * S.nb) * kBlockBytesIn;
             sl.y = y + r * ld_y + c;
             ld_block(x + r * S.ld_bytes + c, sl.w);

@@ -101,3 +101,18 @@ def test_strided_calls_refuse_what_they_cannot_take():
     # overlapping but different views: refused rather than raced
     with pytest.raises(RuntimeError):
         nv.nvfp4_fake_quant(big[:, 0:32], a, out=big[:, 32:64])
+
+
+def test_shared_amax_views_equal_the_parent_call():
+    """Siblings that are column views of one fused output, fake-quantized with their shared
+    amax (the amax of the whole output), give exactly the parent's fake-quant: no block
+    straddles two views when the view widths are multiples of 16."""
+    host, dev, views = _qkv(1024, 256, 64, 5)
+    shared = nv.nvfp4_amax(dev)
+    whole = nv.nvfp4_fake_quant(dev, shared)
+    per_view = dev.clone()
+    for c0, c1 in views:
+        v = per_view[:, c0:c1]
+        nv.nvfp4_fake_quant(v, shared, out=v)
+    assert torch.equal(whole.view(torch.int16), per_view.view(torch.int16))
+    assert_equal_bits(bits(whole), oracle_fake_quant_rows(host, oracle.amax(host)), "parent fake-quant")
