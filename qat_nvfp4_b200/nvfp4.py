@@ -117,17 +117,26 @@ def _cuda(t: torch.Tensor, name: str, dtype=None, contiguous: bool = True):
     return t
 
 
-def _row_stride(t: torch.Tensor, name: str):
-    """None for a contiguous tensor; the row stride (elements) of a 2-D bf16 view that the
-    strided calls take: unit column stride, N % 16 == 0, row stride a multiple of 16 and at
-    least N -- one of q/k/v inside a fused projection output, for instance."""
+def _as_rows(t: torch.Tensor, name: str):
+    """(t, None) for a contiguous bf16 tensor; (rows, ld) for a view the strided calls take:
+    its leading dimensions flatten into rows without a copy (a 2-D view, or e.g. [B, T, N]
+    cut from a [B, T, 3N] fused output), its columns are contiguous, N % 16 == 0 and the row
+    stride ld is a multiple of 16 and at least N."""
     _cuda(t, name, torch.bfloat16, contiguous=False)
     if t.is_contiguous():
-        return None
-    if t.dim() != 2 or t.stride(1) != 1 or t.shape[1] % 16 or t.stride(0) % 16 or t.stride(0) < t.shape[1]:
-        raise RuntimeError(f"{name} must be contiguous, or a 2-D view with contiguous rows, a row stride that "
-                           f"is a multiple of 16 elements and a multiple-of-16 row length")
-    return t.stride(0)
+        return t, None
+    rows = None
+    if t.dim() >= 2:
+        try:
+            rows = t.view(-1, t.shape[-1])
+        except RuntimeError:
+            rows = None
+    if (rows is None or rows.stride(1) != 1 or rows.shape[1] % 16 or rows.stride(0) % 16
+            or rows.stride(0) < rows.shape[1]):
+        raise RuntimeError(f"{name} must be contiguous, or a view with contiguous rows (leading dimensions that "
+                           f"flatten without a copy), a row stride that is a multiple of 16 elements and a "
+                           f"multiple-of-16 row length")
+    return rows, rows.stride(0)
 
 
 def _scalar(t: torch.Tensor, name: str):
@@ -178,14 +187,14 @@ def nvfp4_amax(x: torch.Tensor, out: torch.Tensor | None = None,
     (see new_workspace) it is one kernel launch instead of a memset and a kernel.  x may also
     be a row-strided 2-D view (one of q/k/v inside a fused projection output), read in place
     by nvfp4_amax_strided."""
-    ld = _row_stride(x, "x")
+    rows, ld = _as_rows(x, "x")
     if out is None:
         out = torch.empty(1, dtype=torch.float32, device=x.device)
     _scalar(out, "out")
     with torch.cuda.device(x.device):
         if ld is not None:
-            _check(_c_amax_strided(x.data_ptr(), x.shape[0], x.shape[1], ld, out.data_ptr(), _stream(x.device)),
-                   "nvfp4_amax_strided")
+            _check(_c_amax_strided(rows.data_ptr(), rows.shape[0], rows.shape[1], ld, out.data_ptr(),
+                                   _stream(x.device)), "nvfp4_amax_strided")
         elif workspace is None:
             _check(_c_amax(x.data_ptr(), x.numel(), out.data_ptr(), _stream(x.device)), "nvfp4_amax")
         else:
@@ -250,12 +259,17 @@ def nvfp4_observer_update(state: torch.Tensor, cur_amax: torch.Tensor, kind="sta
 def nvfp4_observe_amax(x: torch.Tensor, state: torch.Tensor, kind="static_minmax", decay: float = 0.01,
                        cur_out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
     """amax of x, then the observer step on ``state`` (in place); returns this step's amax.
-    With a workspace it is one kernel launch."""
-    _cuda(x, "x", torch.bfloat16)
+    With a workspace it is one kernel launch.  A row-strided view x takes the strided amax
+    and a separate observer step."""
+    rows, ld = _as_rows(x, "x")
     _scalar(state, "state")
     if cur_out is None:
         cur_out = torch.empty(1, dtype=torch.float32, device=x.device)
     _scalar(cur_out, "cur_out")
+    if ld is not None:
+        nvfp4_amax(x, out=cur_out)
+        nvfp4_observer_update(state, cur_out, kind, decay)
+        return cur_out
     with torch.cuda.device(x.device):
         if workspace is None:
             _check(_c_observe_amax(x.data_ptr(), x.numel(), state.data_ptr(), _kind(kind), float(decay),
@@ -275,10 +289,10 @@ def nvfp4_quantize(x: torch.Tensor, amax: torch.Tensor, packed: torch.Tensor | N
     global scale fp32 [1]), P = block * ceil(N / block).  ``amax`` is the tensor's (or
     siblings', or observer's) amax; ``block`` is 16 (NVFP4) or 32."""
     block = _block(block)
-    ld = _row_stride(x, "x")
+    rows, ld = _as_rows(x, "x")
     if ld is not None and block != 16:
         raise RuntimeError("row-strided views are quantized in blocks of 16")
-    M, N = (x.shape[0], x.shape[1]) if ld is not None else _matrix(x)
+    M, N = (rows.shape[0], rows.shape[1]) if ld is not None else _matrix(x)
     _scalar(amax, "amax")
     B = padded_blocks(N, block)
     lead = tuple(x.shape[:-1])
@@ -295,8 +309,8 @@ def nvfp4_quantize(x: torch.Tensor, amax: torch.Tensor, packed: torch.Tensor | N
         raise RuntimeError("packed / scales have the wrong number of elements")
     with torch.cuda.device(x.device):
         if ld is not None:
-            st = _c_quantize_strided(x.data_ptr(), M, N, ld, amax.data_ptr(), packed.data_ptr(), scales.data_ptr(),
-                                     global_scale.data_ptr(), _stream(x.device))
+            st = _c_quantize_strided(rows.data_ptr(), M, N, ld, amax.data_ptr(), packed.data_ptr(),
+                                     scales.data_ptr(), global_scale.data_ptr(), _stream(x.device))
         elif block == 16:
             st = _c_quantize(x.data_ptr(), M, N, amax.data_ptr(), packed.data_ptr(), scales.data_ptr(),
                              global_scale.data_ptr(), _stream(x.device))
@@ -403,24 +417,19 @@ def nvfp4_dequantize(packed: torch.Tensor, scales: torch.Tensor, global_scale: t
 def nvfp4_fake_quant(x: torch.Tensor, amax: torch.Tensor, out: torch.Tensor | None = None,
                      block: int = 16) -> torch.Tensor:
     """bf16 -> bf16 fake-quantization (dequantize(quantize(x)) in one pass).  ``out`` may be x;
-    ``block`` is 16 (NVFP4) or 32.  With blocks of 16, x and out may also be row-strided 2-D
-    views (q/k/v inside a fused projection output), read and written in place."""
+    ``block`` is 16 (NVFP4) or 32.  With blocks of 16, x and out may also be row-strided
+    views (q/k/v inside a fused projection output, 2-D or with leading dimensions that
+    flatten into rows), read and written in place."""
     block = _block(block)
-    ld = _row_stride(x, "x")
+    xr, ld = _as_rows(x, "x")
     if out is None:
         out = torch.empty(x.shape, dtype=x.dtype, device=x.device)
-    ld_out = _row_stride(out, "out")
+    outr, ld_out = _as_rows(out, "out")
     _scalar(amax, "amax")
     if out.numel() != x.numel():
         raise RuntimeError("out has the wrong number of elements")
     if ld is not None or ld_out is not None:
-        if block != 16 or x.dim() != 2 or tuple(out.shape) != tuple(x.shape):
-            raise RuntimeError("row-strided fake-quant takes 2-D views of one shape and blocks of 16")
-        M, N = x.shape
-        with torch.cuda.device(x.device):
-            _check(_c_fake_quant_strided(x.data_ptr(), N if ld is None else ld, out.data_ptr(),
-                                         N if ld_out is None else ld_out, M, N, amax.data_ptr(), _stream(x.device)),
-                   "nvfp4_fake_quant_strided")
+        _fake_quant_rows(xr, ld, outr, ld_out, amax, block)
         return out
     M, N = _matrix(x)
     with torch.cuda.device(x.device):
@@ -430,6 +439,21 @@ def nvfp4_fake_quant(x: torch.Tensor, amax: torch.Tensor, out: torch.Tensor | No
             st = _c_fake_quant_bs(x.data_ptr(), out.data_ptr(), M, N, block, amax.data_ptr(), _stream(x.device))
         _check(st, "nvfp4_fake_quant")
     return out
+
+
+def _fake_quant_rows(xr, ld, outr, ld_out, amax, block):
+    """Fake-quant between row views (either may be strided) through nvfp4_fake_quant_strided."""
+    if ld is None:
+        xr = xr.reshape(-1, xr.shape[-1])  # contiguous: a view
+    if ld_out is None:
+        outr = outr.reshape(-1, outr.shape[-1])
+    if block != 16 or tuple(outr.shape) != tuple(xr.shape):
+        raise RuntimeError("row-strided fake-quant takes views of one shape and blocks of 16")
+    M, N = xr.shape
+    with torch.cuda.device(xr.device):
+        _check(_c_fake_quant_strided(xr.data_ptr(), N if ld is None else ld, outr.data_ptr(),
+                                     N if ld_out is None else ld_out, M, N, amax.data_ptr(), _stream(xr.device)),
+               "nvfp4_fake_quant_strided")
 
 
 def nvfp4_fake_quant_siblings(xs: Sequence[torch.Tensor], outs: Sequence[torch.Tensor] | None = None,
@@ -485,15 +509,23 @@ def nvfp4_observe_fake_quant(x: torch.Tensor, state: torch.Tensor, kind="static_
                              out: torch.Tensor | None = None, cur_out: torch.Tensor | None = None,
                              workspace: torch.Tensor | None = None):
     """One W4A4 activation step in one pass: amax of x, observer step on ``state`` (in
-    place), fake-quant with the updated state.  Returns (y, this step's amax)."""
-    M, N = _matrix(x)
+    place), fake-quant with the updated state.  Returns (y, this step's amax).  Row-strided
+    views (x or out) take three launches instead: strided amax, observer step, strided
+    fake-quant."""
+    xr, ld = _as_rows(x, "x")
     _scalar(state, "state")
-    out = torch.empty_like(x) if out is None else out
-    _cuda(out, "out", torch.bfloat16)
+    out = torch.empty(x.shape, dtype=x.dtype, device=x.device) if out is None else out
+    outr, ld_out = _as_rows(out, "out")
     if out.numel() != x.numel():
         raise RuntimeError("out has the wrong number of elements")
     cur_out = torch.empty(1, dtype=torch.float32, device=x.device) if cur_out is None else cur_out
     _scalar(cur_out, "cur_out")
+    if ld is not None or ld_out is not None:
+        nvfp4_amax(x, out=cur_out)
+        nvfp4_observer_update(state, cur_out, kind, decay)
+        _fake_quant_rows(xr, ld, outr, ld_out, state, 16)
+        return out, cur_out
+    M, N = _matrix(x)
     workspace = new_workspace(x.device) if workspace is None else _workspace(workspace, x.device)
     with torch.cuda.device(x.device):
         _check(_c_observe_fake_quant(x.data_ptr(), out.data_ptr(), M, N, state.data_ptr(), _kind(kind), float(decay),
@@ -621,11 +653,16 @@ class FakeQuantSTE(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, x, amax, block=16):
-        # row-strided 2-D views go to the strided kernel as they are; other layouts are
-        # made contiguous first
-        strided_ok = (x.dim() == 2 and x.stride(1) == 1 and x.shape[1] % 16 == 0 and x.stride(0) % 16 == 0
-                      and x.stride(0) >= x.shape[1] and block == 16)
-        return nvfp4_fake_quant(x if x.is_contiguous() or strided_ok else x.contiguous(), amax, block=block)
+        # row-strided views go to the strided kernel as they are; other layouts are made
+        # contiguous first
+        if not x.is_contiguous():
+            try:
+                _as_rows(x, "x")
+                if block != 16:
+                    x = x.contiguous()
+            except RuntimeError:
+                x = x.contiguous()
+        return nvfp4_fake_quant(x, amax, block=block)
 
     @staticmethod
     def backward(ctx, grad_output):

@@ -116,3 +116,31 @@ def test_shared_amax_views_equal_the_parent_call():
         nv.nvfp4_fake_quant(v, shared, out=v)
     assert torch.equal(whole.view(torch.int16), per_view.view(torch.int16))
     assert_equal_bits(bits(whole), oracle_fake_quant_rows(host, oracle.amax(host)), "parent fake-quant")
+
+
+def test_three_dimensional_views_and_the_observer_path():
+    """[B, T, N] column views of a [B, T, 3N] fused output flatten into rows without a copy;
+    amax, fake-quant (into a contiguous output and in place) and the observer calls take them
+    and give the oracle's bytes; the observer state follows the oracle's update."""
+    B, T, n = 3, 100, 128
+    host, dev, views = _qkv(B * T, n, n, 9)
+    dev3 = dev.view(B, T, 3 * n)
+    for c0, c1 in views:
+        v = dev3[:, :, c0:c1]
+        assert not v.is_contiguous()
+        ref = np.ascontiguousarray(host[:, c0:c1])
+        a = nv.nvfp4_amax(v)
+        assert f32_bits(a) == f32_bits(oracle.amax(ref))
+        y = nv.nvfp4_fake_quant(v, a)
+        assert tuple(y.shape) == (B, T, c1 - c0)
+        assert_equal_bits(bits(y).reshape(B * T, -1), oracle_fake_quant_rows(ref, oracle.amax(ref)), "3-D view")
+    # observer: static minmax over two steps on the k view, then fake-quant in place with it
+    k = dev3[:, :, n:2 * n]
+    ref_k = np.ascontiguousarray(host[:, n:2 * n])
+    state = torch.full((1,), -1.0, dtype=torch.float32, device="cuda")
+    cur = nv.nvfp4_observe_amax(k, state, kind="static_minmax")
+    assert f32_bits(cur) == f32_bits(state) == f32_bits(oracle.amax(ref_k))
+    y, cur2 = nv.nvfp4_observe_fake_quant(k, state, kind="static_minmax", out=k)
+    assert y.data_ptr() == k.data_ptr()
+    assert_equal_bits(bits(k).reshape(B * T, -1), oracle_fake_quant_rows(ref_k, oracle.amax(ref_k)),
+                      "observer fake-quant in place on a 3-D view")
