@@ -150,9 +150,32 @@ nvfp4_status ragged_smem_optin(K* kernel, int bytes) {
                : NVFP4_ERR_CUDA;
 }
 
+// Contiguous rows of N = 16 k + 8 elements (16-byte aligned rows, a half block at the end):
+// the two-access kernels of nvfp4_strided.cuh instead of the staged ragged ones.
+bool half_rows(int64_t N, int kW) { return kW == 8 && N % 16 == 8; }
+
+HalfRows half_rows_of(int64_t M, int64_t N) {
+    HalfRows H;
+    H.nb = (N + 15) / 16;
+    H.ld_x = H.ld_y = N * 2;
+    H.total = M * H.nb;
+    return H;
+}
+
 // Ragged launches shared by the entry points (arguments already validated).
 template <int kW>
 nvfp4_status launch_fq_ragged(const void* x, void* y, int64_t M, int64_t N, const float* d_amax, nvfp4_stream_t stream) {
+    if (half_rows(N, kW)) {
+        const HalfRows H = half_rows_of(M, N);
+        if (H.total == 0) return NVFP4_OK;
+        int grid = 1;
+        nvfp4_status st = grid_for(reinterpret_cast<const void*>(&fake_quant_half_kernel), H.total, kUnrollFq,
+                                   NVFP4_GRID_FQ, &grid);
+        if (st != NVFP4_OK) return st;
+        fake_quant_half_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), H,
+                                                                  static_cast<uint8_t*>(y), d_amax);
+        return after_launch();
+    }
     const Ragged R = ragged_of(M, N, 2 * kW);
     if (R.total == 0) return NVFP4_OK;
     int grid = 1;
@@ -562,6 +585,16 @@ static nvfp4_status quantize_impl(const void* x, int64_t M, int64_t N, const flo
         if (rows_p != M || ncb * 4 != R.nb)
             if (cudaMemsetAsync(scales, 0, (size_t)(rows_p * ncb * 4), cs(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
     }
+    if (!kMma && half_rows(N, kW)) {
+        const HalfRows H = half_rows_of(M, N);
+        if (H.total == 0 && d_global_scale == nullptr) return NVFP4_OK;
+        int grid = 1;
+        st = grid_for(reinterpret_cast<const void*>(&quantize_half_kernel), H.total, kUnrollQ, NVFP4_GRID_Q, &grid);
+        if (st != NVFP4_OK) return st;
+        quantize_half_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), H, d_amax, packed, scales,
+                                                                d_global_scale);
+        return after_launch();
+    }
     if (N % kE != 0) {
         int grid = 1;
         st = ragged_smem_optin(quantize_ragged_kernel<kMma, kW>, kStageBytes);
@@ -595,6 +628,17 @@ static nvfp4_status dequantize_impl(const uint8_t* packed, const uint8_t* scales
     if (numel > 0 && (packed == nullptr || scales == nullptr || y == nullptr)) return NVFP4_ERR_NULL;
     if (!aligned(d_global_scale, 4)) return NVFP4_ERR_ALIGN;
     if (numel > 0 && (!aligned(packed, kW) || !aligned(y, 32))) return NVFP4_ERR_ALIGN;
+    if (half_rows(N, kW)) {
+        const HalfRows H = half_rows_of(M, N);
+        if (H.total == 0) return NVFP4_OK;
+        int grid = 1;
+        st = grid_for(reinterpret_cast<const void*>(&dequantize_half_kernel), H.total, kUnrollDecode, NVFP4_GRID_DEC,
+                      &grid);
+        if (st != NVFP4_OK) return st;
+        dequantize_half_kernel<<<grid, kThreads, 0, cs(stream)>>>(packed, scales, d_global_scale, H,
+                                                                  static_cast<uint8_t*>(y));
+        return after_launch();
+    }
     if (N % kE != 0) {
         const Ragged R = ragged_of(M, N, kE);
         if (R.total == 0) return NVFP4_OK;

@@ -121,5 +121,132 @@ __global__ void __launch_bounds__(kThreads)
         [&] { gs = build_scale_table(tab, d_amax); });
 }
 
+// ---------------------------------------------------------------------------------------
+// Rows of N = 16 k + 8 elements (a multiple of 8, not of 16), zero-padded to 16 (k + 1)
+// columns as fp4_optimization.py pads them: every row then starts on a 16-byte boundary,
+// so block b of row r is two aligned 128-bit accesses at r * ld + 32 b (one, and eight
+// zeros, for the last block of the row, whose second half is padding).  These kernels
+// replace the shared-memory staging of nvfp4_ragged.cuh for this case; packed and scales
+// keep the padded layout ([M, 8 (k + 1)] and [M, k + 1], block g = r (k + 1) + b).
+
+struct HalfRows {
+    int64_t nb;        // blocks per row, k + 1
+    int64_t ld_x;      // row stride of the bf16 input in bytes (a multiple of 16)
+    int64_t ld_y;      // row stride of the bf16 output in bytes (a multiple of 16)
+    int64_t total;     // M * nb
+};
+
+__device__ __forceinline__ void ld_b128(const void* p, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
+    asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "l"(p));
+}
+
+// Block g's row and whether it is the row's half block.
+__device__ __forceinline__ int64_t half_row(const HalfRows& H, const Div32& v, int64_t g, bool& half) {
+    const int64_t r = H.total <= 0xFFFFFFFFll ? (int64_t)div32((uint32_t)g, v) : g / H.nb;
+    half = g - r * H.nb == H.nb - 1;
+    return r;
+}
+
+template <bool kCoherent>
+__device__ __forceinline__ void ld_half_block(const uint8_t* p, bool half, uint32_t (&w)[8]) {
+    if (kCoherent) ld_b128(p, w[0], w[1], w[2], w[3]);
+    else ld_b128_ro(p, w[0], w[1], w[2], w[3]);
+    if (half) {
+        w[4] = w[5] = w[6] = w[7] = 0u;  // the padding columns read as +0.0
+    } else if (kCoherent) {
+        ld_b128(p + 16, w[4], w[5], w[6], w[7]);
+    } else {
+        ld_b128_ro(p + 16, w[4], w[5], w[6], w[7]);
+    }
+}
+
+__device__ __forceinline__ void st_half_block(uint8_t* p, bool half, const uint32_t (&o)[8]) {
+    st_b128(p, o[0], o[1], o[2], o[3]);
+    if (!half) st_b128(p + 16, o[4], o[5], o[6], o[7]);
+}
+
+struct HalfSlot {
+    uint32_t w[8];
+    uint8_t* y;
+    bool half;
+};
+
+__global__ void __launch_bounds__(kThreads)
+    quantize_half_kernel(const uint8_t* __restrict__ x, HalfRows H, const float* __restrict__ d_amax,
+                         uint8_t* __restrict__ packed, uint8_t* __restrict__ scales, float* __restrict__ d_gs) {
+    __shared__ float4 tab[128];
+    float gs = 0.0f;
+    const Div32 v = div32_of((uint32_t)H.nb);
+    stream_blocks<kUnrollQ, NVFP4_PIPE_Q != 0, Block32>(
+        H.total,
+        [&](int64_t g, Block32& b) {
+            bool half;
+            const int64_t r = half_row(H, v, g, half);
+            ld_half_block<false>(x + r * H.ld_x + (g - r * H.nb) * kBlockBytesIn, half, b.w);
+        },
+        [&](int64_t g, Block32& b) {
+            uint32_t c[8];
+            float sd;
+            const uint32_t s8 = encode_block(b.w, gs, tab, c, sd);
+            st_codes<8>(packed + g * 8, c);
+            st_u8(scales + g, s8);
+        },
+        [&] {
+            gs = build_scale_table(tab, d_amax);
+            if (d_gs != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *d_gs = gs;
+        });
+}
+
+// x and y may be the same rows (in place), so the loads use the coherent path.
+__global__ void __launch_bounds__(kThreads)
+    fake_quant_half_kernel(const uint8_t* x, HalfRows H, uint8_t* y, const float* d_amax) {
+    __shared__ float4 tab[128];
+    float gs = 0.0f;
+    const Div32 v = div32_of((uint32_t)H.nb);
+    stream_blocks<kUnrollFq, NVFP4_PIPE_FQ != 0, HalfSlot>(
+        H.total,
+        [&](int64_t g, HalfSlot& sl) {
+            const int64_t r = half_row(H, v, g, sl.half);
+            const int64_t c = (g - r * H.nb) * kBlockBytesIn;
+            sl.y = y + r * H.ld_y + c;
+            ld_half_block<true>(x + r * H.ld_x + c, sl.half, sl.w);
+        },
+        [&](int64_t, HalfSlot& sl) {
+            uint32_t c[8];
+            float sd;
+            encode_block(sl.w, gs, tab, c, sd);
+            uint32_t o[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
+            st_half_block(sl.y, sl.half, o);
+        },
+        [&] { gs = build_scale_table(tab, d_amax); });
+}
+
+__global__ void __launch_bounds__(kThreads)
+    dequantize_half_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
+                           const float* __restrict__ d_gs, HalfRows H, uint8_t* __restrict__ y) {
+    __shared__ float tab_sd[256];  // sd for every possible scale byte
+    const Div32 v = div32_of((uint32_t)H.nb);
+    stream_blocks<kUnrollDecode, NVFP4_PIPE_DEC != 0, PackedSlot<8>>(
+        H.total,
+        [&](int64_t g, PackedSlot<8>& sl) {
+            ld_codes_ro<8>(packed + g * 8, sl.p);
+            sl.s = ld_u8_ro(scales + g);
+        },
+        [&](int64_t g, PackedSlot<8>& sl) {
+            uint32_t o[8];
+            decode_codes<8>(sl.p, tab_sd[sl.s & 0xFFu], o);
+            bool half;
+            const int64_t r = half_row(H, v, g, half);
+            st_half_block(y + r * H.ld_y + (g - r * H.nb) * kBlockBytesIn, half, o);
+        },
+        [&] {
+            const float gs = __ldg(d_gs);
+            for (int i = threadIdx.x; i < 256; i += blockDim.x) tab_sd[i] = __fdiv_rn(e4m3_to_f32(i), gs);
+            __syncthreads();
+        });
+}
+
 }  // namespace
 }  // namespace nvfp4
