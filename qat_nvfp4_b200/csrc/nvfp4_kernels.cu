@@ -150,31 +150,71 @@ nvfp4_status ragged_smem_optin(K* kernel, int bytes) {
                : NVFP4_ERR_CUDA;
 }
 
-// Contiguous rows of N = 16 k + 8 elements (16-byte aligned rows, a half block at the end):
-// the two-access kernels of nvfp4_strided.cuh instead of the staged ragged ones.
-bool half_rows(int64_t N, int kW) { return kW == 8 && N % 16 == 8; }
+// Contiguous rows of an even length N that is not a multiple of 16: every row start is
+// kA-byte aligned (16 for N % 16 == 8, 8 for N % 8 == 4, 4 for N % 4 == 2), so the aligned
+// access kernels of nvfp4_strided.cuh can take them instead of the staged ragged ones.  Their
+// narrow loads are cheap (a warp's later accesses hit the sectors its first one brought to
+// L1), but narrow bf16 stores 32 bytes apart are not: measured on 65536-row tensors, they
+// win for quantize at every kA, for fake-quant down to kA = 8 and for dequantize only at
+// kA = 16, which is what min_store_access selects.  0 when they do not apply (odd N, blocks
+// of 32, stores narrower than min_store_access).
+int ragged_access(int64_t N, int kW, int min_store_access) {
+    if (kW != 8 || N % 16 == 0 || N % 2 != 0) return 0;
+    const int kA = N % 8 == 0 ? 16 : (N % 4 == 0 ? 8 : 4);
+    return kA >= min_store_access ? kA : 0;
+}
 
-HalfRows half_rows_of(int64_t M, int64_t N) {
-    HalfRows H;
+RaggedRows ragged_rows_of(int64_t M, int64_t N, int kA) {
+    RaggedRows H;
     H.nb = (N + 15) / 16;
     H.ld_x = H.ld_y = N * 2;
     H.total = M * H.nb;
+    H.tail = (int)(N % 16) * 2 / kA;
     return H;
+}
+
+template <int kA>
+nvfp4_status launch_fq_rows(const void* x, void* y, const RaggedRows& H, const float* d_amax, nvfp4_stream_t stream) {
+    int grid = 1;
+    nvfp4_status st = grid_for(reinterpret_cast<const void*>(&fake_quant_rows_kernel<kA>), H.total, kUnrollFq,
+                               NVFP4_GRID_FQ, &grid);
+    if (st != NVFP4_OK) return st;
+    fake_quant_rows_kernel<kA><<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), H,
+                                                                  static_cast<uint8_t*>(y), d_amax);
+    return after_launch();
+}
+
+template <int kA>
+nvfp4_status launch_quantize_rows(const void* x, const RaggedRows& H, const float* d_amax, uint8_t* packed,
+                                  uint8_t* scales, float* d_gs, nvfp4_stream_t stream) {
+    int grid = 1;
+    nvfp4_status st = grid_for(reinterpret_cast<const void*>(&quantize_rows_kernel<kA>), H.total, kUnrollQ,
+                               NVFP4_GRID_Q, &grid);
+    if (st != NVFP4_OK) return st;
+    quantize_rows_kernel<kA><<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), H, d_amax, packed,
+                                                                scales, d_gs);
+    return after_launch();
+}
+
+template <int kA>
+nvfp4_status launch_dequantize_rows(const uint8_t* packed, const uint8_t* scales, const float* d_gs,
+                                    const RaggedRows& H, void* y, nvfp4_stream_t stream) {
+    int grid = 1;
+    nvfp4_status st = grid_for(reinterpret_cast<const void*>(&dequantize_rows_kernel<kA>), H.total, kUnrollDecode,
+                               NVFP4_GRID_DEC, &grid);
+    if (st != NVFP4_OK) return st;
+    dequantize_rows_kernel<kA><<<grid, kThreads, 0, cs(stream)>>>(packed, scales, d_gs, H, static_cast<uint8_t*>(y));
+    return after_launch();
 }
 
 // Ragged launches shared by the entry points (arguments already validated).
 template <int kW>
 nvfp4_status launch_fq_ragged(const void* x, void* y, int64_t M, int64_t N, const float* d_amax, nvfp4_stream_t stream) {
-    if (half_rows(N, kW)) {
-        const HalfRows H = half_rows_of(M, N);
+    if (const int kA = ragged_access(N, kW, 8)) {
+        const RaggedRows H = ragged_rows_of(M, N, kA);
         if (H.total == 0) return NVFP4_OK;
-        int grid = 1;
-        nvfp4_status st = grid_for(reinterpret_cast<const void*>(&fake_quant_half_kernel), H.total, kUnrollFq,
-                                   NVFP4_GRID_FQ, &grid);
-        if (st != NVFP4_OK) return st;
-        fake_quant_half_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), H,
-                                                                  static_cast<uint8_t*>(y), d_amax);
-        return after_launch();
+        return kA == 16 ? launch_fq_rows<16>(x, y, H, d_amax, stream)
+                        : kA == 8 ? launch_fq_rows<8>(x, y, H, d_amax, stream) : launch_fq_rows<4>(x, y, H, d_amax, stream);
     }
     const Ragged R = ragged_of(M, N, 2 * kW);
     if (R.total == 0) return NVFP4_OK;
@@ -585,15 +625,12 @@ static nvfp4_status quantize_impl(const void* x, int64_t M, int64_t N, const flo
         if (rows_p != M || ncb * 4 != R.nb)
             if (cudaMemsetAsync(scales, 0, (size_t)(rows_p * ncb * 4), cs(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
     }
-    if (!kMma && half_rows(N, kW)) {
-        const HalfRows H = half_rows_of(M, N);
+    if (const int kA = kMma ? 0 : ragged_access(N, kW, 4)) {
+        const RaggedRows H = ragged_rows_of(M, N, kA);
         if (H.total == 0 && d_global_scale == nullptr) return NVFP4_OK;
-        int grid = 1;
-        st = grid_for(reinterpret_cast<const void*>(&quantize_half_kernel), H.total, kUnrollQ, NVFP4_GRID_Q, &grid);
-        if (st != NVFP4_OK) return st;
-        quantize_half_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), H, d_amax, packed, scales,
-                                                                d_global_scale);
-        return after_launch();
+        return kA == 16 ? launch_quantize_rows<16>(x, H, d_amax, packed, scales, d_global_scale, stream)
+               : kA == 8 ? launch_quantize_rows<8>(x, H, d_amax, packed, scales, d_global_scale, stream)
+                         : launch_quantize_rows<4>(x, H, d_amax, packed, scales, d_global_scale, stream);
     }
     if (N % kE != 0) {
         int grid = 1;
@@ -628,16 +665,12 @@ static nvfp4_status dequantize_impl(const uint8_t* packed, const uint8_t* scales
     if (numel > 0 && (packed == nullptr || scales == nullptr || y == nullptr)) return NVFP4_ERR_NULL;
     if (!aligned(d_global_scale, 4)) return NVFP4_ERR_ALIGN;
     if (numel > 0 && (!aligned(packed, kW) || !aligned(y, 32))) return NVFP4_ERR_ALIGN;
-    if (half_rows(N, kW)) {
-        const HalfRows H = half_rows_of(M, N);
+    if (const int kA = ragged_access(N, kW, 16)) {
+        const RaggedRows H = ragged_rows_of(M, N, kA);
         if (H.total == 0) return NVFP4_OK;
-        int grid = 1;
-        st = grid_for(reinterpret_cast<const void*>(&dequantize_half_kernel), H.total, kUnrollDecode, NVFP4_GRID_DEC,
-                      &grid);
-        if (st != NVFP4_OK) return st;
-        dequantize_half_kernel<<<grid, kThreads, 0, cs(stream)>>>(packed, scales, d_global_scale, H,
-                                                                  static_cast<uint8_t*>(y));
-        return after_launch();
+        return kA == 16 ? launch_dequantize_rows<16>(packed, scales, d_global_scale, H, y, stream)
+               : kA == 8 ? launch_dequantize_rows<8>(packed, scales, d_global_scale, H, y, stream)
+                         : launch_dequantize_rows<4>(packed, scales, d_global_scale, H, y, stream);
     }
     if (N % kE != 0) {
         const Ragged R = ragged_of(M, N, kE);

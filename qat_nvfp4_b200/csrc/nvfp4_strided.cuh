@@ -122,57 +122,83 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ---------------------------------------------------------------------------------------
-// Rows of N = 16 k + 8 elements (a multiple of 8, not of 16), zero-padded to 16 (k + 1)
-// columns as fp4_optimization.py pads them: every row then starts on a 16-byte boundary,
-// so block b of row r is two aligned 128-bit accesses at r * ld + 32 b (one, and eight
-// zeros, for the last block of the row, whose second half is padding).  These kernels
-// replace the shared-memory staging of nvfp4_ragged.cuh for this case; packed and scales
-// keep the padded layout ([M, 8 (k + 1)] and [M, k + 1], block g = r (k + 1) + b).
+// Rows of an even length N that is not a multiple of 16, zero-padded to 16 ceil(N / 16)
+// columns as fp4_optimization.py pads them.  A contiguous tensor's row r starts at 2 N r
+// bytes, so every row start is kA-byte aligned with kA = 16 (N = 16 k + 8), 8 (N % 8 == 4) or
+// 4 (N % 4 == 2): block b of row r is 32 / kA aligned kA-byte accesses at r ld + 32 b, and the
+// row's last block only its first `tail` accesses (the rest of it is padding and reads as
+// +0.0, and is not written).  These kernels replace the shared-memory staging of
+// nvfp4_ragged.cuh for even N (odd N keeps it); packed and scales keep the padded layout
+// ([M, 8 nb] and [M, nb], block g = r nb + b).
 
-struct HalfRows {
-    int64_t nb;        // blocks per row, k + 1
-    int64_t ld_x;      // row stride of the bf16 input in bytes (a multiple of 16)
-    int64_t ld_y;      // row stride of the bf16 output in bytes (a multiple of 16)
+struct RaggedRows {
+    int64_t nb;        // blocks per row, ceil(N / 16)
+    int64_t ld_x;      // row stride of the bf16 input in bytes
+    int64_t ld_y;      // row stride of the bf16 output in bytes
     int64_t total;     // M * nb
+    int tail;          // kA-byte accesses that hold real elements in a row's last block
 };
 
 __device__ __forceinline__ void ld_b128(const void* p, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
     asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "l"(p));
 }
 
-// Block g's row and whether it is the row's half block.
-__device__ __forceinline__ int64_t half_row(const HalfRows& H, const Div32& v, int64_t g, bool& half) {
+// Block g's row, and how many kA-byte accesses of it hold real elements.
+template <int kA>
+__device__ __forceinline__ int64_t ragged_row(const RaggedRows& H, const Div32& v, int64_t g, int& na) {
     const int64_t r = H.total <= 0xFFFFFFFFll ? (int64_t)div32((uint32_t)g, v) : g / H.nb;
-    half = g - r * H.nb == H.nb - 1;
+    na = g - r * H.nb == H.nb - 1 ? H.tail : 32 / kA;
     return r;
 }
 
-template <bool kCoherent>
-__device__ __forceinline__ void ld_half_block(const uint8_t* p, bool half, uint32_t (&w)[8]) {
-    if (kCoherent) ld_b128(p, w[0], w[1], w[2], w[3]);
-    else ld_b128_ro(p, w[0], w[1], w[2], w[3]);
-    if (half) {
-        w[4] = w[5] = w[6] = w[7] = 0u;  // the padding columns read as +0.0
-    } else if (kCoherent) {
-        ld_b128(p + 16, w[4], w[5], w[6], w[7]);
-    } else {
-        ld_b128_ro(p + 16, w[4], w[5], w[6], w[7]);
+// The na real accesses of one block (the others read as zeros); kCoherent for inputs that
+// may be written by the same kernel (in place).
+template <int kA, bool kCoherent>
+__device__ __forceinline__ void ld_ragged_block(const uint8_t* p, int na, uint32_t (&w)[8]) {
+    constexpr int kWords = kA / 4;
+#pragma unroll
+    for (int j = 0; j < 32 / kA; ++j) {
+        uint32_t* q = w + j * kWords;
+        if (j >= na) {
+#pragma unroll
+            for (int i = 0; i < kWords; ++i) q[i] = 0u;
+        } else if constexpr (kA == 16) {
+            if (kCoherent) ld_b128(p + 16 * j, q[0], q[1], q[2], q[3]);
+            else ld_b128_ro(p + 16 * j, q[0], q[1], q[2], q[3]);
+        } else if constexpr (kA == 8) {
+            const uint2 t = kCoherent ? *reinterpret_cast<const uint2*>(p + 8 * j)
+                                      : __ldg(reinterpret_cast<const uint2*>(p + 8 * j));
+            q[0] = t.x;
+            q[1] = t.y;
+        } else {
+            q[0] = kCoherent ? *reinterpret_cast<const uint32_t*>(p + 4 * j)
+                             : __ldg(reinterpret_cast<const uint32_t*>(p + 4 * j));
+        }
     }
 }
 
-__device__ __forceinline__ void st_half_block(uint8_t* p, bool half, const uint32_t (&o)[8]) {
-    st_b128(p, o[0], o[1], o[2], o[3]);
-    if (!half) st_b128(p + 16, o[4], o[5], o[6], o[7]);
+template <int kA>
+__device__ __forceinline__ void st_ragged_block(uint8_t* p, int na, const uint32_t (&o)[8]) {
+    constexpr int kWords = kA / 4;
+#pragma unroll
+    for (int j = 0; j < 32 / kA; ++j) {
+        if (j >= na) break;
+        const uint32_t* q = o + j * kWords;
+        if constexpr (kA == 16) st_b128(p + 16 * j, q[0], q[1], q[2], q[3]);
+        else if constexpr (kA == 8) *reinterpret_cast<uint2*>(p + 8 * j) = make_uint2(q[0], q[1]);
+        else *reinterpret_cast<uint32_t*>(p + 4 * j) = q[0];
+    }
 }
 
-struct HalfSlot {
+struct RaggedSlot {
     uint32_t w[8];
     uint8_t* y;
-    bool half;
+    int na;
 };
 
+template <int kA>
 __global__ void __launch_bounds__(kThreads)
-    quantize_half_kernel(const uint8_t* __restrict__ x, HalfRows H, const float* __restrict__ d_amax,
+    quantize_rows_kernel(const uint8_t* __restrict__ x, RaggedRows H, const float* __restrict__ d_amax,
                          uint8_t* __restrict__ packed, uint8_t* __restrict__ scales, float* __restrict__ d_gs) {
     __shared__ float4 tab[128];
     float gs = 0.0f;
@@ -180,9 +206,9 @@ __global__ void __launch_bounds__(kThreads)
     stream_blocks<kUnrollQ, NVFP4_PIPE_Q != 0, Block32>(
         H.total,
         [&](int64_t g, Block32& b) {
-            bool half;
-            const int64_t r = half_row(H, v, g, half);
-            ld_half_block<false>(x + r * H.ld_x + (g - r * H.nb) * kBlockBytesIn, half, b.w);
+            int na;
+            const int64_t r = ragged_row<kA>(H, v, g, na);
+            ld_ragged_block<kA, false>(x + r * H.ld_x + (g - r * H.nb) * kBlockBytesIn, na, b.w);
         },
         [&](int64_t g, Block32& b) {
             uint32_t c[8];
@@ -198,34 +224,36 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // x and y may be the same rows (in place), so the loads use the coherent path.
+template <int kA>
 __global__ void __launch_bounds__(kThreads)
-    fake_quant_half_kernel(const uint8_t* x, HalfRows H, uint8_t* y, const float* d_amax) {
+    fake_quant_rows_kernel(const uint8_t* x, RaggedRows H, uint8_t* y, const float* d_amax) {
     __shared__ float4 tab[128];
     float gs = 0.0f;
     const Div32 v = div32_of((uint32_t)H.nb);
-    stream_blocks<kUnrollFq, NVFP4_PIPE_FQ != 0, HalfSlot>(
+    stream_blocks<kUnrollFq, NVFP4_PIPE_FQ != 0, RaggedSlot>(
         H.total,
-        [&](int64_t g, HalfSlot& sl) {
-            const int64_t r = half_row(H, v, g, sl.half);
+        [&](int64_t g, RaggedSlot& sl) {
+            const int64_t r = ragged_row<kA>(H, v, g, sl.na);
             const int64_t c = (g - r * H.nb) * kBlockBytesIn;
             sl.y = y + r * H.ld_y + c;
-            ld_half_block<true>(x + r * H.ld_x + c, sl.half, sl.w);
+            ld_ragged_block<kA, true>(x + r * H.ld_x + c, sl.na, sl.w);
         },
-        [&](int64_t, HalfSlot& sl) {
+        [&](int64_t, RaggedSlot& sl) {
             uint32_t c[8];
             float sd;
             encode_block(sl.w, gs, tab, c, sd);
             uint32_t o[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
-            st_half_block(sl.y, sl.half, o);
+            st_ragged_block<kA>(sl.y, sl.na, o);
         },
         [&] { gs = build_scale_table(tab, d_amax); });
 }
 
+template <int kA>
 __global__ void __launch_bounds__(kThreads)
-    dequantize_half_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
-                           const float* __restrict__ d_gs, HalfRows H, uint8_t* __restrict__ y) {
+    dequantize_rows_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
+                           const float* __restrict__ d_gs, RaggedRows H, uint8_t* __restrict__ y) {
     __shared__ float tab_sd[256];  // sd for every possible scale byte
     const Div32 v = div32_of((uint32_t)H.nb);
     stream_blocks<kUnrollDecode, NVFP4_PIPE_DEC != 0, PackedSlot<8>>(
@@ -237,9 +265,9 @@ __global__ void __launch_bounds__(kThreads)
         [&](int64_t g, PackedSlot<8>& sl) {
             uint32_t o[8];
             decode_codes<8>(sl.p, tab_sd[sl.s & 0xFFu], o);
-            bool half;
-            const int64_t r = half_row(H, v, g, half);
-            st_half_block(y + r * H.ld_y + (g - r * H.nb) * kBlockBytesIn, half, o);
+            int na;
+            const int64_t r = ragged_row<kA>(H, v, g, na);
+            st_ragged_block<kA>(y + r * H.ld_y + (g - r * H.nb) * kBlockBytesIn, na, o);
         },
         [&] {
             const float gs = __ldg(d_gs);

@@ -381,7 +381,8 @@ def test_observe_with_workspace_16_steps():
 # ---- rows whose length is not a multiple of 16 (zero padding, crop) -----------------------
 
 @pytest.mark.parametrize("M,N", [(1, 1), (5, 15), (3, 20), (17, 1000), (255, 4097), (64, 8191), (2, 33), (4096, 1000),
-                                 (9, 8), (1, 24), (300, 8184), (2049, 40)])
+                                 (9, 8), (1, 24), (300, 8184), (2049, 40),
+                                 (5, 4), (7, 12), (33, 1028), (3, 1036), (11, 2), (4, 6), (9, 1022), (130, 8190)])
 def test_ragged_rows(M, N):
     rng = np.random.default_rng(M * 131 + N)
     x = synthetic.to_bf16_bits(rng.standard_t(3, (M, N)).astype(np.float32))
@@ -413,11 +414,12 @@ def test_siblings_with_ragged_members():
         assert_equal_bits(bits(o), oracle_fake_quant_rows(t, a), f"{t.shape} sibling")
 
 
-@pytest.mark.parametrize("M,N", [(3, 20), (255, 4097), (1000, 33), (3, 24), (257, 1032), (1, 8)])
+@pytest.mark.parametrize("M,N", [(3, 20), (255, 4097), (1000, 33), (3, 24), (257, 1032), (1, 8), (5, 6), (7, 1036),
+                                 (2, 1022), (1, 2)])
 def test_ragged_outputs_stay_inside_their_tensor(M, N):
-    """Guard bands of 0xA5 bytes around y: the staged edge writes of the ragged kernels, and
-    the half-block stores of the rows of 16 k + 8 elements, touch no byte outside the M*N
-    outputs."""
+    """Guard bands of 0xA5 bytes around y: the staged edge writes of the ragged kernels (odd
+    N), and the partial last-block stores of even N (16-, 8- and 4-byte accesses), touch no
+    byte outside the M*N outputs."""
     rng = np.random.default_rng(M + 7 * N)
     x = synthetic.to_bf16_bits(rng.standard_normal((M, N)).astype(np.float32))
     xd = to_dev(x)
