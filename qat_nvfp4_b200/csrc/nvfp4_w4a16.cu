@@ -81,17 +81,17 @@ template <int BN, int ACC, int ROWS = kMmaM * ACC>
 struct Cfg {
     static constexpr int kBN = BN;
     static constexpr int kBM = kMmaM * ACC;
-    static constexpr int kAtoms = ACC == 1 ? (ROWS == 32 ? 4 : 2) : 1;
+    static constexpr int kAtoms = BN == 256 ? 1 : (ROWS == 32 ? 4 : 2);
     static constexpr int kAtomABytes = ROWS * kBK * 2;           // one 64-column atom of the activation tile
     static constexpr int kAtomBBytes = BN * kBK * 2;             // one 64-column atom of the weight tile
     static constexpr int kTileABytes = kAtoms * kAtomABytes;
     static constexpr int kRecPerTile = BN / kRecRows;            // records per atom
     static constexpr int kTileBBytes = kAtoms * kAtomBBytes;     // decoded weight tile
     static constexpr int kTmemCols = ACC * BN;                   // fp32 accumulators, 128 lanes x BN each
-    static constexpr int kRingA = BN == 256 ? 3 : (ACC == 2 ? 4 : (ROWS == 32 ? 2 : 3));  // activation tiles in flight
+    static constexpr int kRingA = BN == 256 ? 3 : (ACC == 2 || ROWS == 32 ? 2 : 3);  // activation tiles in flight
     static constexpr int kRingW =  // weight stages in flight
-        BN == 256 ? 4 : (ACC == 2 ? 8 : (ROWS == 32 ? 3 : (ROWS == 64 ? 8 : 6)));
-    static constexpr int kRingB = BN == 256 ? 2 : (ACC == 2 ? 3 : (ROWS == 64 ? 3 : 2));  // decoded tiles, decode -> MMA
+        BN == 256 ? 4 : (ACC == 2 || ROWS == 32 ? 3 : (ROWS == 64 ? 8 : 6));
+    static constexpr int kRingB = BN == 256 ? 2 : (ROWS == 64 ? 3 : 2);  // decoded tiles, decode -> MMA
     static constexpr int kColParts = 4 / ACC;                    // epilogue warps per accumulator lane group
     static constexpr int kTpr = kDecodeThreads / BN;             // decode threads per weight row
     static constexpr int kBpt = kAtoms * (kBK / kBlockElems) / kTpr;  // 16-element blocks per thread
@@ -848,14 +848,15 @@ static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const
                                       void* d_workspace, int64_t workspace_bytes, uint64_t selftest_ns,
                                       nvfp4_stream_t stream) {
     if (M < 0 || !weight_shape_ok(N, K) || M > 0x7FFFFF00ll) return NVFP4_ERR_SHAPE;
-    // Output tiles 256 x 256 when x has more than 256 rows, 256 x 128 for 129 to 256 rows,
-    // 128 x 128 for at most 128.
+    // Output tiles: 128 x 128 for at most 128 rows of x; 256 x 128 for 129 to 256 rows;
+    // above that 256 x 256 (half the activation traffic per FLOP) or 256 x 128, whichever
+    // needs less time by waves of one CTA per SM, a 256 x 128 tile taking 2/3 of the time of
+    // a 256 x 256 one (measured: it has half the MMA work but the same fixed costs).  Chosen
+    // below, once the SM count is known; the limits here use the larger tile count.
     const int acc = M > kMmaM ? 2 : 1;
     const int bm = kMmaM * acc;
-    const int bn = M > 2 * kMmaM ? 256 : 128;
     const int64_t tiles_m = (M + bm - 1) / bm;
-    const int64_t tiles_n = (N + bn - 1) / bn;
-    if (tiles_m * tiles_n > 0x7FFFFFFFll) return NVFP4_ERR_SHAPE;
+    if (tiles_m * ((N + 127) / 128) > 0x7FFFFFFFll) return NVFP4_ERR_SHAPE;
     if (d_global_scale == nullptr || d_workspace == nullptr) return NVFP4_ERR_NULL;
     if (M > 0 && N > 0 && (x == nullptr || tiled == nullptr || y == nullptr)) return NVFP4_ERR_NULL;
     if (!is_aligned(d_global_scale, 4) || !is_aligned(d_workspace, 256)) return NVFP4_ERR_ALIGN;
@@ -870,6 +871,16 @@ static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const
     if (st != NVFP4_OK) return st;
     st = gemm_smem_optin();
     if (st != NVFP4_OK) return st;
+    int sms = 0;
+    st = sm_count_w4(&sms);
+    if (st != NVFP4_OK) return st;
+    int bn = 128;
+    if (M > 2 * kMmaM) {
+        const int64_t w256 = (tiles_m * ((N + 255) / 256) + sms - 1) / sms;
+        const int64_t w128 = (tiles_m * ((N + 127) / 128) + sms - 1) / sms;
+        bn = 2 * w128 < 3 * w256 ? 128 : 256;
+    }
+    const int64_t tiles_n = (N + bn - 1) / bn;
 
     // x as a [M, K] bf16 tensor, boxes of bm rows x 64 columns, 128-byte swizzle, zero fill
     // past either edge.  When x fits in one row tile the box is cut to M rounded up to 8
@@ -903,9 +914,6 @@ static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const
     a.a_bytes = (uint32_t)box_rows * kBK * 2;
     a.selftest_ns = selftest_ns;
     // split K only with a workspace large enough for the partial sums
-    int sms = 0;
-    st = sm_count_w4(&sms);
-    if (st != NVFP4_OK) return st;
     a.splits = acc == 1 ? split_count(M, N, K, sms) : 1;
     if (a.splits > 1 && workspace_bytes < split_workspace_bytes(M, N, a.splits)) a.splits = 1;
     a.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(d_workspace) + counters_offset());

@@ -87,14 +87,14 @@ def _assert_within_bound(y_bits, x_bits, packed, scales, gs, bias_bits, what):
     return exact
 
 
-@pytest.mark.parametrize("K", [128, 256, 512])
-def test_decoded_weight_is_exact_through_one_hot_rows(K):
+@pytest.mark.parametrize("K,N", [(128, 300), (256, 300), (512, 300), (4096, 2560)])
+def test_decoded_weight_is_exact_through_one_hot_rows(K, N):
     """x = the K x K identity: output row k is 1 * W[:, k] plus exact zeros, so y^T must be
     the oracle's dequantized weight bit for bit (up to the sign of a zero sum).  Random
     bytes cover every code and every finite scale byte, negative E4M3 scales included;
-    K = 128, 256 and 512 run the 128 x 128, 256 x 128 and 256 x 256 tile configurations."""
+    K = 128 runs the 128 x 128 tiles, 256 and 512 the 256 x 128 tiles, and 4096 rows on a
+    2560-row weight (160 tiles of 256 x 256, at least one per SM) the 256 x 256 tiles."""
     rng = np.random.default_rng(K)
-    N = 300
     packed = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
     scales = rng.integers(0, 256, size=(N, K // 16), dtype=np.uint8)
     scales[(scales & 0x7F) == 0x7F] = 0x3C  # NaN bytes are outside the method
@@ -125,6 +125,7 @@ def test_decoded_weight_is_exact_through_one_hot_rows(K):
     (20, 704, 300, True),      # 32 rows kept, stages of 4 atoms: 11 atoms, the last stage 3
     (32, 1040, 200, True),     # 32 rows kept: 17 atoms, K % 64 == 16, the last stage 1 atom
     (33, 1040, 200, True),     # one row past the 32-row configuration
+    (2305, 256, 4000, True),   # 256 x 256 tiles (160 of them), ragged M and N
 ])
 def test_linear_matches_oracle(M, K, N, with_bias):
     rng = np.random.default_rng(M * 7 + K * 3 + N)
@@ -217,12 +218,12 @@ def test_split_k_for_few_rows(M, K):
     _assert_within_bound(bits(y3), x, packed, scales, gs, bias, f"unsplit, {M} rows")
 
 
-@pytest.mark.parametrize("M,N", [(16, 4096), (700, 512)])
+@pytest.mark.parametrize("M,N", [(16, 4096), (700, 512), (4096, 2560)])
 def test_bounded_wait_reports_a_timeout_and_the_context_recovers(M, N):
     """A wait on a barrier that nothing completes (2 ms limit) runs out: the call reports
     NVFP4_ERR_TIMEOUT through the workspace instead of hanging, every role stops, and the
     next call on the same context and workspace is correct.  16 rows take the split-K
-    path, 700 rows the 256 x 256 tiles."""
+    path, 700 rows the 256 x 128 tiles, 4096 rows on 2560 outputs the 256 x 256 tiles."""
     K = 1024
     rng = np.random.default_rng(M + N)
     x = synthetic.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
