@@ -61,8 +61,9 @@ static_assert(kRecBytes % 16 == 0, "bulk copy size");
 // One configuration per output tile: kAcc accumulators of 128 rows of x (kBM = 128 kAcc rows)
 // by BN weight rows (output features, the MMA's N).  256 x 256 for many rows of x (half
 // the activation traffic per FLOP of BN = 128); 256 x 128 (twice the CTAs) when x has 129
-// to 256 rows; 128 x 128 when it has at most 128 (half the MMA work and activation bytes
-// per stage, and deeper rings for the weight stream).
+// to 256 rows, or more rows but too few 256 x 256 tiles to fill the SMs; 128 x 128 when it
+// has at most 128 (half the MMA work and activation bytes per stage, and deeper rings for
+// the weight stream).
 //
 // ROWS is the number of rows of x a tile keeps in shared memory: kBM, or 64 / 32 for the
 // 128 x 128 tiles when x has at most 64 / 32 rows.  The MMA always reads 128 rows per
@@ -72,9 +73,10 @@ static_assert(kRecBytes % 16 == 0, "bulk copy size");
 // longer stages (32 rows).
 //
 // A stage covers kAtoms atoms of K (64 columns each, one 128-byte swizzle row per tile row):
-// 4 for the 128 x 128 tiles that keep 32 rows of x, 2 for the other 128 x 128 tiles (a good
-// part of a stage's time there is the fixed cost of handing it from role to role, so that
-// cost is paid once per 256 or 128 columns), 1 for the others.  Within a stage, atom t of
+// 4 for the 128 x 128 tiles that keep 32 rows of x, 2 for the other 128 x 128 and for the
+// 256 x 128 tiles (a good part of a stage's time is the fixed cost of handing it from role
+// to role, so that cost is paid once per 256 or 128 columns), 1 for the 256 x 256 tiles,
+// whose two-atom stages would not fit in shared memory.  Within a stage, atom t of
 // the activation tile sits at t * ROWS * 128 bytes (accumulator h's 128 rows at + h * 16 KB)
 // and atom t of the decoded weight tile at t * BN * 128 bytes.
 template <int BN, int ACC, int ROWS = kMmaM * ACC>
