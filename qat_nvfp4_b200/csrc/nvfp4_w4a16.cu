@@ -4,21 +4,22 @@
 // _float4_autocast_forward: the packed weight is unpacked for one forward and the layer's
 // own bf16 forward runs on it).
 //
-// One kernel on the sm_100a tensor cores (tcgen05, kind::f16, bf16 operands, fp32
-// accumulators in tensor memory).  The bf16 weight is never written to HBM.  The weight is
-// read in a tile-major copy of its packed form (nvfp4_w4a16_pack: one contiguous 4608-byte
-// record per 128-row x 64-column tile, codes then scale bytes); the decode warps copy the
-// bytes they need into shared memory themselves and decode them into the MMA operand
-// layout (128-byte swizzle, K-major) with the same arithmetic as nvfp4_dequantize,
-// bf16_rn(fl(LUT[code] * fl(E4M3(byte) / gs))).
+// Kernels on the sm_100a tensor cores (tcgen05, kind::f16, bf16 operands, fp32 accumulators
+// in tensor memory).  The bf16 weight is never written to HBM.  The weight is read in a
+// tile-major copy of its packed form (nvfp4_w4a16_pack: one contiguous 4608-byte record per
+// 128-row x 64-column tile, codes then scale bytes), and decoded by the kernel's own warps
+// with the same arithmetic as nvfp4_dequantize, bf16_rn(fl(LUT[code] * fl(E4M3(byte) / gs))).
 //
-//   warps 0-15 copy (cp.async, several stages ahead, into private slots) and decode weight
-//              rows into weight tiles, 32 rows per warp, then the epilogue
+//   warps 0-15 decode weight rows, 32 rows per warp, then the epilogue
 //              (TMEM -> fp32 + bias -> bf16)
 //   warp 16    TMA loads of activation tiles
 //   warp 17    TMEM allocation, MMA issue (one elected thread), TMEM release
-// Decoded weight tiles pass from the decode warps to the MMAs through a ring of 2 or 3, so
-// the decode of a stage overlaps the MMAs of the stages before it.
+//
+// Up to 128 rows of x (w4a16_linear_kernel): x is the MMA's A operand, the decoded weight
+// tile the B operand in shared memory (128-byte swizzle, K-major), passed from the decode
+// warps to the MMAs through a ring of 2 or 3 tiles; K may be split over several CTAs per
+// tile.  More rows (w4a16_linear_ts_kernel): the decoded weight is the A operand, kept in
+// tensor memory, and x the B operand.
 //
 // Every wait on an mbarrier is bounded (kWaitLimitNs of %globaltimer); a wait that runs
 // out records NVFP4_ERR_TIMEOUT in the caller's workspace, tells the other roles to stop,
@@ -58,50 +59,43 @@ static_assert(kBK * 2 == 128, "one swizzle row per tile row");
 static_assert(kGemmThreads == 32 * (kDecodeWarps + 2), "warp roles");
 static_assert(kRecBytes % 16 == 0, "bulk copy size");
 
-// One configuration per output tile: kAcc accumulators of 128 rows of x (kBM = 128 kAcc rows)
-// by BN weight rows (output features, the MMA's N).  256 x 256 for many rows of x (half
-// the activation traffic per FLOP of BN = 128); 256 x 128 (twice the CTAs) when x has 129
-// to 256 rows, or more rows but too few 256 x 256 tiles to fill the SMs; 128 x 128 when it
-// has at most 128 (half the MMA work and activation bytes per stage, and deeper rings for
-// the weight stream).
+// The tiles for at most 128 rows of x: 128 rows of x (one accumulator) by 128 weight rows
+// (output features, the MMA's N).
 //
-// ROWS is the number of rows of x a tile keeps in shared memory: kBM, or 64 / 32 for the
-// 128 x 128 tiles when x has at most 64 / 32 rows.  The MMA always reads 128 rows per
-// accumulator; past ROWS they are whatever bytes follow the atom in shared memory (the next
-// atom, or the decoded weight ring after the last one), and they only feed accumulator lanes
-// that the epilogue never stores.  The room this frees goes to deeper rings (64 rows) or to
-// longer stages (32 rows).
+// ROWS is the number of rows of x a tile keeps in shared memory: 128, or 64 / 32 when x has
+// at most 64 / 32 rows.  The MMA always reads 128 rows; past ROWS they are whatever bytes
+// follow the atom in shared memory (the next atom, or the decoded weight ring after the last
+// one), and they only feed accumulator lanes that the epilogue never stores.  The room this
+// frees goes to deeper rings (64 rows) or to longer stages (32 rows).
 //
 // A stage covers kAtoms atoms of K (64 columns each, one 128-byte swizzle row per tile row):
-// 4 for the 128 x 128 tiles that keep 32 rows of x, 2 for the other 128 x 128 and for the
-// 256 x 128 tiles (a good part of a stage's time is the fixed cost of handing it from role
-// to role, so that cost is paid once per 256 or 128 columns), 1 for the 256 x 256 tiles,
-// whose two-atom stages would not fit in shared memory.  Within a stage, atom t of
-// the activation tile sits at t * ROWS * 128 bytes (accumulator h's 128 rows at + h * 16 KB)
-// and atom t of the decoded weight tile at t * BN * 128 bytes.
-template <int BN, int ACC, int ROWS = kMmaM * ACC>
+// 4 when 32 rows of x are kept, else 2 (a good part of a stage's time is the fixed cost of
+// handing it from role to role, so that cost is paid once per 256 or 128 columns).  Within a
+// stage, atom t of the activation tile sits at t * ROWS * 128 bytes and atom t of the
+// decoded weight tile at t * 128 * 128 bytes.
+template <int ROWS>
 struct Cfg {
-    static constexpr int kBN = BN;
-    static constexpr int kBM = kMmaM * ACC;
-    static constexpr int kAtoms = BN == 256 ? 1 : (ROWS == 32 ? 4 : 2);
+    static constexpr int kBN = 128;
+    static constexpr int kAcc = 1;
+    static constexpr int kBM = kMmaM;
+    static constexpr int kAtoms = ROWS == 32 ? 4 : 2;
     static constexpr int kAtomABytes = ROWS * kBK * 2;           // one 64-column atom of the activation tile
-    static constexpr int kAtomBBytes = BN * kBK * 2;             // one 64-column atom of the weight tile
+    static constexpr int kAtomBBytes = kBN * kBK * 2;            // one 64-column atom of the weight tile
     static constexpr int kTileABytes = kAtoms * kAtomABytes;
-    static constexpr int kRecPerTile = BN / kRecRows;            // records per atom
+    static constexpr int kRecPerTile = kBN / kRecRows;           // records per atom
     static constexpr int kTileBBytes = kAtoms * kAtomBBytes;     // decoded weight tile
-    static constexpr int kTmemCols = ACC * BN;                   // fp32 accumulators, 128 lanes x BN each
-    static constexpr int kRingA = BN == 256 ? 3 : (ACC == 2 || ROWS == 32 ? 2 : 3);  // activation tiles in flight
-    static constexpr int kRingW =  // weight stages in flight
-        BN == 256 ? 4 : (ACC == 2 || ROWS == 32 ? 3 : (ROWS == 64 ? 8 : 6));
-    static constexpr int kRingB = BN == 256 ? 2 : (ROWS == 64 ? 3 : 2);  // decoded tiles, decode -> MMA
-    static constexpr int kColParts = 4 / ACC;                    // epilogue warps per accumulator lane group
-    static constexpr int kTpr = kDecodeThreads / BN;             // decode threads per weight row
+    static constexpr int kTmemCols = kBN;                        // fp32 accumulator, 128 lanes x kBN
+    static constexpr int kRingA = ROWS == 32 ? 2 : 3;            // activation tiles in flight
+    static constexpr int kRingW = ROWS == 32 ? 3 : (ROWS == 64 ? 8 : 6);  // weight stages in flight
+    static constexpr int kRingB = ROWS == 64 ? 3 : 2;            // decoded tiles, decode -> MMA
+    static constexpr int kColParts = 4;                          // epilogue warps per accumulator lane group
+    static constexpr int kTpr = kDecodeThreads / kBN;             // decode threads per weight row
     static constexpr int kBpt = kAtoms * (kBK / kBlockElems) / kTpr;  // 16-element blocks per thread
     // Instruction descriptor of kind::f16: fp32 accumulator (bits 4-5 = 1), A and B bf16
     // (bits 7-9 = 1, bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 in bits
     // 17-22, M >> 4 in bits 24-28.
     static constexpr uint32_t kIdesc =
-        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kMmaM >> 4) << 24);
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kMmaM >> 4) << 24);
 
     // Shared memory: activation tiles, decoded weight tiles (both 1024-byte aligned), the
     // weight ring, then the barriers and the table.
@@ -125,15 +119,15 @@ struct Cfg {
     static constexpr int kRingBytes = kRingA * kTileABytes + kRingB * kTileBBytes + kRingW * kWSlotBytes;
     static constexpr int kSmemBytes = 1024 + kRingBytes + (int)sizeof(Shared);
 
-    static_assert(BN % kRecRows == 0 && BN >= 16 && BN <= 256, "MMA N");
+    static_assert(kBN % kRecRows == 0, "MMA N");
     static_assert(kTpr * kBpt == kAtoms * (kBK / kBlockElems) && (kBpt == 1 || kBpt == 2 || kBpt == 4),
                   "decode split");
     static_assert(kBpt == 1 || (kBK / kBlockElems) % kBpt == 0, "a thread's blocks lie in one atom");
     static_assert(kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0, "tensor memory columns");
     static_assert(kAtomABytes % 1024 == 0 && kAtomBBytes % 1024 == 0, "operand tiles stay 1024-byte aligned");
-    static_assert(kDecodeWarps == 4 * ACC * kColParts, "epilogue warps");
+    static_assert(kDecodeWarps == 4 * kAcc * kColParts, "epilogue warps");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
-    static_assert(ROWS == kBM || (ACC == 1 && ROWS % 8 == 0 && ROWS < kBM), "rows kept in shared memory");
+    static_assert(ROWS == kBM || (ROWS % 8 == 0 && ROWS < kBM), "rows kept in shared memory");
     // the 128 rows the MMA reads from the last activation atom stay inside the rings
     static_assert(kRingA * kTileABytes - kAtomABytes + kMmaM * kBK * 2 <= kRingBytes, "MMA reads stay in bounds");
 };
@@ -327,8 +321,8 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------------------------------
-// The linear kernel.  One CTA per 256 x 128 output tile; the tile index runs over output
-// features fastest, so CTAs resident together share their activation tile in L2.
+// The linear kernels.  One CTA per output tile (times the K splits); the tile index runs
+// over output features fastest, so CTAs resident together share their activation tile in L2.
 
 struct LinearArgs {
     const uint8_t* tiled;   // weight records
@@ -400,10 +394,11 @@ __device__ __forceinline__ uint32_t decode_pair_x2(uint32_t code_byte, uint64_t 
     return *reinterpret_cast<uint32_t*>(&r);
 }
 
-template <int BN, int ACC, int ROWS>
+template <int ROWS>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     w4a16_linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const LinearArgs a) {
-    using C = Cfg<BN, ACC, ROWS>;
+    using C = Cfg<ROWS>;
+    constexpr int ACC = C::kAcc;
     constexpr int kBN = C::kBN, kRingA = C::kRingA, kRingB = C::kRingB, kRingW = C::kRingW;
     constexpr int kBM = C::kBM, kTileABytes = C::kTileABytes, kAtoms = C::kAtoms;
     constexpr int kAtomABytes = C::kAtomABytes, kAtomBBytes = C::kAtomBBytes;
@@ -718,6 +713,338 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------
+// The linear kernel for more than 128 rows of x: the weight is the MMA's A operand, kept
+// in tensor memory.
+//
+// One CTA per output tile of 128 weight rows (one record row) by BT rows of x.  The MMA
+// computes D[n][m] = sum_k W[n][k] x[m][k]: A = the decoded weight tile, 128 rows x 16 of K
+// per step, read from tensor memory (row n in lane n, two bf16 per 32-bit column, the
+// lower K in the low half); B = the activation tile, BT rows of x in the 128-byte swizzle
+// K-major layout TMA writes.  The decode warps write the bf16 weight straight into tensor
+// memory (tcgen05.st), and read the packed bytes from L2 into registers, so shared memory
+// holds nothing but the activation tiles (TMA writes, MMA reads).
+//
+// A stage is two 64-column atoms of K: two TMA boxes of x, two records of the weight, eight
+// MMAs.  Handing a stage from role to role has a fixed cost (barrier waits, commits and
+// fences on the single MMA-issuing thread) of the order of the MMAs of one atom, so it is
+// paid once per 128 columns.
+//
+// Tensor memory: columns 0 .. BT - 1 hold the accumulator (lane n = weight row n of the
+// tile, column m = row m of x); columns 256 .. 511 a ring of 4 weight slots, 64 columns
+// (128 of K) each.  The 16 decode warps form 2 groups of 8 that take the stages in turn
+// (group g the stages g, g + 2, ...), so each has two stages' time for one; warp (q, t) of
+// a group decodes atom t of the stage for weight rows 32 q .. + 31 (the tensor memory lanes
+// its tcgen05.st may write), one row per thread: 32 code bytes and a scale word, loaded one
+// of its own stages ahead, into 32 columns.
+
+constexpr int kTsAtoms = 2;                        // 64-column atoms of K per stage
+constexpr int kTsGroups = kDecodeWarps / (4 * kTsAtoms);  // decode warp groups, taking stages in turn
+constexpr int kTsSlotCols = kTsAtoms * kBK / 2;    // tensor memory columns of one weight slot
+constexpr int kTsWCol = 256;                       // first column of the weight ring
+constexpr int kTsRingT = (512 - kTsWCol) / kTsSlotCols;  // weight slots in tensor memory
+static_assert(kTsGroups == 2 && kTsRingT == 4, "decode groups and weight slots");
+static_assert(kTsRingT % kTsGroups == 0, "a group's stages keep to its slots");
+
+template <int BT>
+struct TsCfg {
+    static constexpr int kAtomABytes = BT * kBK * 2;          // one activation box
+    static constexpr int kStageABytes = kTsAtoms * kAtomABytes;
+    static constexpr int kRingA = (192 * 1024) / kStageABytes;  // 3 stages for BT = 256, 6 for 128
+    // kind::f16 instruction descriptor: fp32 D, bf16 A and B, both K-major, N = BT, M = 128
+    static constexpr uint32_t kIdesc =
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BT >> 3) << 17) | ((uint32_t)(kMmaM >> 4) << 24);
+    struct Shared {
+        uint64_t a_full[kRingA];     // activation boxes landed (TMA bytes)
+        uint64_t a_empty[kRingA];    // the MMAs that read them completed
+        uint64_t w_full[kTsRingT];   // the decode warps wrote the weight slot
+        uint64_t w_empty[kTsRingT];  // the MMAs that read it completed
+        uint64_t accum;
+        uint64_t drain;
+        uint64_t never;
+        uint32_t tmem_base;
+        uint32_t abort;
+        float sd[256];
+    };
+    static constexpr int kRingBytes = kRingA * kStageABytes;
+    static constexpr int kSmemBytes = 1024 + kRingBytes + (int)sizeof(Shared);
+    static_assert(BT == 128 || BT == 256, "MMA N");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+};
+
+// D (tmem) (+)= A (tmem) . B (smem desc)^T, one 128 x N x 16 step.
+__device__ __forceinline__ void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 consecutive 32-bit columns of this warp's 32 TMEM lanes, then wait until they landed.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]),
+        "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]),
+        "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// 16 consecutive fp32 columns of this warp's 32 TMEM lanes, without waiting (the caller
+// waits once with tcgen05.wait::ld before reading v).
+__device__ __forceinline__ void tmem_ld16_issue(uint32_t taddr, uint32_t* v) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+
+// One record row of an atom (32 code bytes, the scale word) from L2, read-only path.
+struct RecRow {
+    uint32_t c[8];
+    uint32_t sc;
+};
+__device__ __forceinline__ void ld_rec_row(const uint8_t* code, const uint8_t* scale, RecRow& r) {
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.c[0]), "=r"(r.c[1]), "=r"(r.c[2]), "=r"(r.c[3])
+                 : "l"(code));
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.c[4]), "=r"(r.c[5]), "=r"(r.c[6]), "=r"(r.c[7])
+                 : "l"(code + 16));
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(r.sc) : "l"(scale));
+}
+
+template <int BT>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    w4a16_linear_ts_kernel(const __grid_constant__ CUtensorMap tmap_x, const LinearArgs a) {
+    using C = TsCfg<BT>;
+    constexpr int kRingA = C::kRingA, kAtomABytes = C::kAtomABytes, kStageABytes = C::kStageABytes;
+    constexpr uint32_t kIdesc = C::kIdesc;
+    extern __shared__ uint8_t dsmem[];
+    const uint32_t raw = smem_u32(dsmem);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* ring = dsmem + (base - raw);
+    typename C::Shared& sh = *reinterpret_cast<typename C::Shared*>(ring + C::kRingBytes);
+    const uint32_t sA0 = base;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t tile = (int64_t)blockIdx.x;
+    const int64_t tm = tile / a.tiles_n, tn = tile % a.tiles_n;
+    const int64_t m0 = tm * BT, n0 = tn * kRecRows;
+    const int kt = (int)a.kt;                          // atoms of K
+    const int nk = (kt + kTsAtoms - 1) / kTsAtoms;     // stages; the last may hold one atom
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kRingA; ++s) {
+            mbar_init(smem_u32(&sh.a_full[s]), 1);
+            mbar_init(smem_u32(&sh.a_empty[s]), 1);
+        }
+        for (int s = 0; s < kTsRingT; ++s) {
+            mbar_init(smem_u32(&sh.w_full[s]), kDecodeWarps / kTsGroups);
+            mbar_init(smem_u32(&sh.w_empty[s]), 1);
+        }
+        mbar_init(smem_u32(&sh.accum), 1);
+        mbar_init(smem_u32(&sh.drain), 1);
+        mbar_init(smem_u32(&sh.never), 1);
+        sh.abort = 0u;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    {
+        const float gs = __ldg(a.d_gs);
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) sh.sd[i] = __fdiv_rn(e4m3_to_f32((uint32_t)i), gs);
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_u32(&sh.tmem_base), 512);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+    const volatile uint32_t* abort = &sh.abort;
+
+    if (warp == kTmaWarp) {
+        // ---- producer: activation boxes (TMA), the atoms of each stage that lie inside K ----
+        if (lane == 0) {
+            int issued = 0;
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % kRingA;
+                if (!mbar_wait(smem_u32(&sh.a_empty[s]), ((uint32_t)(kb / kRingA) & 1u) ^ 1u, abort)) {
+                    stop_all(sh, a.ws);
+                    break;
+                }
+                const uint32_t bar = smem_u32(&sh.a_full[s]);
+                const int na = min(kTsAtoms, kt - kb * kTsAtoms);
+                mbar_arrive_expect_tx(bar, a.a_bytes * (uint32_t)na);
+                for (int t = 0; t < na; ++t)
+                    tma_load_2d(sA0 + s * kStageABytes + t * kAtomABytes, &tmap_x, (kb * kTsAtoms + t) * kBK,
+                                (int32_t)m0, bar);
+                ++issued;
+            }
+            for (int kb = issued > kRingA ? issued - kRingA : 0; kb < issued; ++kb)
+                if (!mbar_wait(smem_u32(&sh.a_full[kb % kRingA]), (uint32_t)(kb / kRingA) & 1u, abort, true))
+                    stop_all(sh, a.ws);
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            bool ok = true;
+            if (a.selftest_ns != 0 && !mbar_wait(smem_u32(&sh.never), 0u, abort, false, a.selftest_ns)) {
+                stop_all(sh, a.ws);
+                ok = false;
+            }
+            for (int kb = 0; ok && kb < nk; ++kb) {
+                const int sa = kb % kRingA, st = kb % kTsRingT;
+                if (!mbar_wait(smem_u32(&sh.a_full[sa]), (uint32_t)(kb / kRingA) & 1u, abort) ||
+                    !mbar_wait(smem_u32(&sh.w_full[st]), (uint32_t)(kb / kTsRingT) & 1u, abort)) {
+                    stop_all(sh, a.ws);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int na = min(kTsAtoms, kt - kb * kTsAtoms);
+#pragma unroll
+                for (int t = 0; t < kTsAtoms; ++t) {
+                    if (t >= na) break;
+                    const uint64_t bd = sw128_desc(sA0 + sa * kStageABytes + t * kAtomABytes);
+                    const uint32_t ta = tmem + (uint32_t)(kTsWCol + st * kTsSlotCols + t * (kBK / 2));
+#pragma unroll
+                    for (int j = 0; j < kBK / kUmmaK; ++j)  // 16 of K: 8 columns of A, 32 bytes of B
+                        umma_f16_ts(tmem, ta + 8u * j, bd + 2u * j, kIdesc, (kb | t | j) != 0 ? 1u : 0u);
+                }
+                umma_commit(smem_u32(&sh.a_empty[sa]));
+                umma_commit(smem_u32(&sh.w_empty[st]));
+            }
+            if (ok) {
+                umma_commit(smem_u32(&sh.accum));
+            } else {
+                umma_commit(smem_u32(&sh.drain));
+                mbar_wait(smem_u32(&sh.drain), 0u, abort, true);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---- decode warps: group g takes stages g, g + 2, ...; warp (q, t) of the group
+        //      atom t of each, thread = one weight row (TMEM lane) of the tile ----
+        const int q = warp & 3;                          // TMEM lane quarter: rows 32 q .. + 31
+        const int t = (warp >> 2) % kTsAtoms;            // atom of the stage
+        const int g = (warp >> 2) / kTsAtoms;            // decode group
+        const int row = 32 * q + lane;                   // weight row of the tile (record row)
+        const uint8_t* gcode = a.tiled + tn * a.kt * kRecBytes + row * 32;
+        const uint8_t* gscale = a.tiled + tn * a.kt * kRecBytes + kRecCodes + row * 4;
+        const uint32_t tw = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kTsWCol + t * (kBK / 2));
+        // own stage i is stage g + 2 i; its atom for this warp, or -1 past K
+        auto atom_of = [&](int i) {
+            const int at = (g + kTsGroups * i) * kTsAtoms + t;
+            return at < kt ? at : -1;
+        };
+        RecRow next;
+        {
+            const int at = atom_of(0);
+            if (at >= 0) ld_rec_row(gcode + (int64_t)at * kRecBytes, gscale + (int64_t)at * kRecBytes, next);
+        }
+        bool ok = true;
+        for (int i = 0; g + kTsGroups * i < nk; ++i) {
+            const int kb = g + kTsGroups * i, st = kb % kTsRingT;
+            const int at = atom_of(i);
+            const RecRow cur = next;
+            {
+                const int an = atom_of(i + 1);
+                if (an >= 0 && g + kTsGroups * (i + 1) < nk)
+                    ld_rec_row(gcode + (int64_t)an * kRecBytes, gscale + (int64_t)an * kRecBytes, next);
+            }
+            if (!warp_wait(smem_u32(&sh.w_empty[st]), ((uint32_t)(kb / kTsRingT) & 1u) ^ 1u, abort)) {
+                if (lane == 0) stop_all(sh, a.ws);
+                ok = false;
+                break;
+            }
+            if (at >= 0) {  // an atom past the end of K is neither written nor multiplied
+                tc_fence_after();
+                uint32_t o[32];
+#pragma unroll
+                for (int b = 0; b < kBK / kBlockElems; ++b) {  // block b: columns 8 b .. 8 b + 7
+                    const float sd = sh.sd[(cur.sc >> (8 * b)) & 0xFFu];
+                    uint64_t sd2;
+                    asm("mov.b64 %0, {%1, %1};" : "=l"(sd2) : "f"(sd));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        o[8 * b + j] = decode_pair_x2((cur.c[2 * b] >> (8 * j)) & 0xFFu, sd2);
+                        o[8 * b + 4 + j] = decode_pair_x2((cur.c[2 * b + 1] >> (8 * j)) & 0xFFu, sd2);
+                    }
+                }
+                tmem_st32(tw + (uint32_t)(st * kTsSlotCols), o);
+                tc_fence_before();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sh.w_full[st]));
+        }
+
+        // ---- epilogue: warp w reads lanes 32 q .. + 31 (weight rows n), columns (rows m of x)
+        //      (w / 4) BT / 4 .. + BT / 4, adds the bias and rounds to bf16 once.  With rows of y
+        //      that take 16-byte stores, the warp turns its 32 x BT / 4 patch around in its own
+        //      4 KB of the (now idle) activation ring, so that each store covers 8 output
+        //      columns; otherwise each lane stores its column n element by element ----
+        if (ok) {
+            if (!warp_wait(smem_u32(&sh.accum), 0u, abort)) {
+                if (lane == 0) stop_all(sh, a.ws);
+            } else {
+                tc_fence_after();
+                constexpr int kCols = BT / 4;  // rows of x per warp
+                const int part = warp >> 2;
+                const int64_t n = n0 + row;
+                const bool live = n < a.N;
+                const float b = (a.bias != nullptr && live) ? __uint_as_float((uint32_t)__ldg(a.bias + n) << 16) : 0.f;
+                const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(part * kCols);
+                uint32_t v[kCols];
+#pragma unroll
+                for (int j = 0; j < kCols / 16; ++j) tmem_ld16_issue(trow + 16u * j, v + 16 * j);
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                const int64_t mb = m0 + part * kCols;  // first row of x of this warp's patch
+                uint16_t* y = reinterpret_cast<uint16_t*>(a.y);
+                if (a.vec_store) {
+                    uint16_t* patch = reinterpret_cast<uint16_t*>(ring + warp * 4096);  // [kCols][32]
+#pragma unroll
+                    for (int e = 0; e < kCols; ++e) {
+                        float f = __uint_as_float(v[e]);
+                        if (a.bias != nullptr) f = __fadd_rn(f, b);
+                        patch[e * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int r = 0; r < kCols / 8; ++r) {  // 16-byte chunk c: row c / 4, columns 8 (c % 4)
+                        const int c = lane + 32 * r;
+                        const int64_t m = mb + c / 4;
+                        const int64_t nc = n0 + 32 * q + 8 * (c % 4);
+                        const uint4 w = *reinterpret_cast<const uint4*>(patch + (c / 4) * 32 + 8 * (c % 4));
+                        if (m < a.M && nc < a.N) st_b128(y + m * a.N + nc, w.x, w.y, w.z, w.w);
+                    }
+                } else if (live) {
+#pragma unroll
+                    for (int e = 0; e < kCols; ++e) {
+                        float f = __uint_as_float(v[e]);
+                        if (a.bias != nullptr) f = __fadd_rn(f, b);
+                        if (mb + e < a.M) y[(mb + e) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
 // Host side.
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -749,16 +1076,16 @@ nvfp4_status gemm_smem_optin() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevs) return NVFP4_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_w4_mu);
     if (!g_smem_set[dev]) {
-        if (cudaFuncSetAttribute(w4a16_linear_kernel<256, 2, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg<256, 2>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(w4a16_linear_kernel<128, 2, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg<128, 2>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(w4a16_linear_kernel<128, 1, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg<128, 1>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(w4a16_linear_kernel<128, 1, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg<128, 1, 64>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(w4a16_linear_kernel<128, 1, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg<128, 1, 32>::kSmemBytes) != cudaSuccess)
+        if (cudaFuncSetAttribute(w4a16_linear_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<128>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(w4a16_linear_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<64>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(w4a16_linear_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<32>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(w4a16_linear_ts_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 TsCfg<256>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(w4a16_linear_ts_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 TsCfg<128>::kSmemBytes) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         g_smem_set[dev] = true;
     }
@@ -845,20 +1172,70 @@ NVFP4_API int64_t nvfp4_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     return splits > 1 ? split_workspace_bytes(M, N, splits) : (int64_t)sizeof(Workspace);
 }
 
+// More than 128 rows of x: the weight in tensor memory, tiles of 128 weight rows by BT rows
+// of x.  BT = 256 unless 128-row tiles need no more waves of one CTA per SM: a stage of a
+// 128-row tile takes ~85 % of the time of a 256-row one (the fixed cost of a stage does not
+// shrink with the MMAs), so 128-row tiles pay only where they fill SMs that would idle.
+static nvfp4_status w4a16_linear_ts(EncodeTiledFn encode, const void* x, int64_t M, int64_t K, const uint8_t* tiled,
+                                    const float* d_global_scale, int64_t N, const void* bias, void* y,
+                                    void* d_workspace, uint64_t selftest_ns, int sms, nvfp4_stream_t stream) {
+    const int64_t tiles_n = (N + kRecRows - 1) / kRecRows;
+    const int64_t w256 = (tiles_n * ((M + 255) / 256) + sms - 1) / sms;
+    const int64_t w128 = (tiles_n * ((M + 127) / 128) + sms - 1) / sms;
+    const int bt = w128 <= w256 ? 128 : 256;
+    const int64_t tiles_m = (M + bt - 1) / bt;
+
+    // x as a [M, K] bf16 tensor, boxes of bt rows x 64 columns, 128-byte swizzle, zero fill
+    // past either edge.  When x has fewer than bt rows the box is cut to M rounded up to 8:
+    // the slot rows past it are never written, and the accumulator columns they feed are
+    // rows of y past M, which are not stored.
+    CUtensorMap map;
+    std::memset(&map, 0, sizeof(map));
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const int box_rows = M < bt ? (int)((M + 7) / 8 * 8) : bt;
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return NVFP4_ERR_ARG;
+
+    LinearArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.tiled = tiled;
+    a.d_gs = d_global_scale;
+    a.bias = static_cast<const uint16_t*>(bias);
+    a.y = static_cast<uint8_t*>(y);
+    a.ws = static_cast<Workspace*>(d_workspace);
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.tiles_n = tiles_n;
+    a.kt = (K + kBK - 1) / kBK;
+    a.splits = 1;
+    a.vec_store = (is_aligned(y, 16) && N % 8 == 0) ? 1 : 0;
+    a.a_bytes = (uint32_t)box_rows * kBK * 2;
+    a.selftest_ns = selftest_ns;
+    const unsigned grid = (unsigned)(tiles_m * tiles_n);
+    cudaStream_t cst = reinterpret_cast<cudaStream_t>(stream);
+    if (bt == 256)
+        w4a16_linear_ts_kernel<256><<<grid, kGemmThreads, TsCfg<256>::kSmemBytes, cst>>>(map, a);
+    else
+        w4a16_linear_ts_kernel<128><<<grid, kGemmThreads, TsCfg<128>::kSmemBytes, cst>>>(map, a);
+    note_launch();
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
 static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const uint8_t* tiled,
                                       const float* d_global_scale, int64_t N, const void* bias, void* y,
                                       void* d_workspace, int64_t workspace_bytes, uint64_t selftest_ns,
                                       nvfp4_stream_t stream) {
     if (M < 0 || !weight_shape_ok(N, K) || M > 0x7FFFFF00ll) return NVFP4_ERR_SHAPE;
-    // Output tiles: 128 x 128 for at most 128 rows of x; 256 x 128 for 129 to 256 rows;
-    // above that 256 x 256 (half the activation traffic per FLOP) or 256 x 128, whichever
-    // needs less time by waves of one CTA per SM, a 256 x 128 tile taking 2/3 of the time of
-    // a 256 x 256 one (measured: it has half the MMA work but the same fixed costs).  Chosen
-    // below, once the SM count is known; the limits here use the larger tile count.
-    const int acc = M > kMmaM ? 2 : 1;
-    const int bm = kMmaM * acc;
-    const int64_t tiles_m = (M + bm - 1) / bm;
-    if (tiles_m * ((N + 127) / 128) > 0x7FFFFFFFll) return NVFP4_ERR_SHAPE;
+    // Output tiles: 128 x 128 for at most 128 rows of x (weight in shared memory, split K);
+    // above that 128 weight rows by 256 or 128 rows of x with the weight in tensor memory,
+    // chosen below once the SM count is known; the limit here uses the larger tile count.
+    if (((M + kMmaM - 1) / kMmaM) * ((N + 127) / 128) > 0x7FFFFFFFll) return NVFP4_ERR_SHAPE;
     if (d_global_scale == nullptr || d_workspace == nullptr) return NVFP4_ERR_NULL;
     if (M > 0 && N > 0 && (x == nullptr || tiled == nullptr || y == nullptr)) return NVFP4_ERR_NULL;
     if (!is_aligned(d_global_scale, 4) || !is_aligned(d_workspace, 256)) return NVFP4_ERR_ALIGN;
@@ -876,24 +1253,21 @@ static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const
     int sms = 0;
     st = sm_count_w4(&sms);
     if (st != NVFP4_OK) return st;
-    int bn = 128;
-    if (M > 2 * kMmaM) {
-        const int64_t w256 = (tiles_m * ((N + 255) / 256) + sms - 1) / sms;
-        const int64_t w128 = (tiles_m * ((N + 127) / 128) + sms - 1) / sms;
-        bn = 2 * w128 < 3 * w256 ? 128 : 256;
-    }
-    const int64_t tiles_n = (N + bn - 1) / bn;
+    if (M > kMmaM)
+        return w4a16_linear_ts(encode, x, M, K, tiled, d_global_scale, N, bias, y, d_workspace, selftest_ns, sms,
+                               stream);
+    const int64_t tiles_m = (M + kMmaM - 1) / kMmaM;  // 1: at most 128 rows here
+    const int64_t tiles_n = (N + 127) / 128;
 
-    // x as a [M, K] bf16 tensor, boxes of bm rows x 64 columns, 128-byte swizzle, zero fill
-    // past either edge.  When x fits in one row tile the box is cut to M rounded up to 8
-    // rows: the rows of the tile past it are never written, and the MMA rows they feed are
-    // output rows past M, which are not stored (each output row depends only on its own
-    // row of x).
+    // x as a [M, K] bf16 tensor, boxes of M rounded up to 8 rows x 64 columns, 128-byte
+    // swizzle, zero fill past either edge: the rows of the tile past the box are never
+    // written, and the MMA rows they feed are output rows past M, which are not stored (each
+    // output row depends only on its own row of x).
     CUtensorMap map;
     std::memset(&map, 0, sizeof(map));
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const int box_rows = tiles_m == 1 ? (int)((M + 7) / 8 * 8) : bm;
+    const int box_rows = (int)((M + 7) / 8 * 8);
     const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
@@ -916,22 +1290,18 @@ static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const
     a.a_bytes = (uint32_t)box_rows * kBK * 2;
     a.selftest_ns = selftest_ns;
     // split K only with a workspace large enough for the partial sums
-    a.splits = acc == 1 ? split_count(M, N, K, sms) : 1;
+    a.splits = split_count(M, N, K, sms);
     if (a.splits > 1 && workspace_bytes < split_workspace_bytes(M, N, a.splits)) a.splits = 1;
     a.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(d_workspace) + counters_offset());
     a.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(d_workspace) + partial_offset(tiles_n));
     const unsigned grid = (unsigned)(tiles_m * tiles_n * a.splits);
     cudaStream_t cst = reinterpret_cast<cudaStream_t>(stream);
-    if (bn == 256)
-        w4a16_linear_kernel<256, 2, 256><<<grid, kGemmThreads, Cfg<256, 2>::kSmemBytes, cst>>>(map, a);
-    else if (acc == 2)
-        w4a16_linear_kernel<128, 2, 256><<<grid, kGemmThreads, Cfg<128, 2>::kSmemBytes, cst>>>(map, a);
-    else if (M > 64)
-        w4a16_linear_kernel<128, 1, 128><<<grid, kGemmThreads, Cfg<128, 1>::kSmemBytes, cst>>>(map, a);
+    if (M > 64)
+        w4a16_linear_kernel<128><<<grid, kGemmThreads, Cfg<128>::kSmemBytes, cst>>>(map, a);
     else if (M > 32)  // at most 64 rows: 64 rows of x per atom in shared memory, deeper rings
-        w4a16_linear_kernel<128, 1, 64><<<grid, kGemmThreads, Cfg<128, 1, 64>::kSmemBytes, cst>>>(map, a);
+        w4a16_linear_kernel<64><<<grid, kGemmThreads, Cfg<64>::kSmemBytes, cst>>>(map, a);
     else  // at most 32 rows: 32 rows of x per atom, stages of 256 columns of K
-        w4a16_linear_kernel<128, 1, 32><<<grid, kGemmThreads, Cfg<128, 1, 32>::kSmemBytes, cst>>>(map, a);
+        w4a16_linear_kernel<32><<<grid, kGemmThreads, Cfg<32>::kSmemBytes, cst>>>(map, a);
     note_launch();
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

@@ -92,8 +92,9 @@ def test_decoded_weight_is_exact_through_one_hot_rows(K, N):
     """x = the K x K identity: output row k is 1 * W[:, k] plus exact zeros, so y^T must be
     the oracle's dequantized weight bit for bit (up to the sign of a zero sum).  Random
     bytes cover every code and every finite scale byte, negative E4M3 scales included;
-    K = 128 runs the 128 x 128 tiles, 256 and 512 the 256 x 128 tiles, and 4096 rows on a
-    2560-row weight (160 tiles of 256 x 256, at least one per SM) the 256 x 256 tiles."""
+    K = 128 runs the tiles with the weight in shared memory, 256 and 512 the tensor-memory
+    weight with 128-row tiles of x, and 4096 rows on a 2560-row weight (320 tiles, more than
+    one per SM) the 256-row tiles."""
     rng = np.random.default_rng(K)
     packed = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
     scales = rng.integers(0, 256, size=(N, K // 16), dtype=np.uint8)
@@ -110,11 +111,11 @@ def test_decoded_weight_is_exact_through_one_hot_rows(K, N):
 
 
 @pytest.mark.parametrize("M,K,N,with_bias", [
-    (128, 64, 128, False),     # one stage; rows 128-255 of the tile are past M
-    (256, 128, 256, False),    # both accumulators of one tile full
-    (700, 512, 384, True),     # three row tiles, the last ragged
+    (128, 64, 128, False),     # one stage of one atom
+    (256, 128, 256, False),    # weight in tensor memory: two full 128-row tiles of x, one stage
+    (700, 512, 384, True),     # six 128-row tiles of x, the last ragged
     (128, 1024, 256, True),    # 16 stages, two output tiles
-    (300, 1040, 200, True),    # ragged M, N and K (K % 64 == 16)
+    (300, 1040, 200, True),    # ragged M, N and K (K % 64 == 16; the last stage one atom)
     (37, 48, 24, False),       # K below one stage
     (5, 16, 13, True),         # N odd: element stores
     (1, 4096, 4096, False),    # one token
@@ -125,7 +126,11 @@ def test_decoded_weight_is_exact_through_one_hot_rows(K, N):
     (20, 704, 300, True),      # 32 rows kept, stages of 4 atoms: 11 atoms, the last stage 3
     (32, 1040, 200, True),     # 32 rows kept: 17 atoms, K % 64 == 16, the last stage 1 atom
     (33, 1040, 200, True),     # one row past the 32-row configuration
-    (2305, 256, 4000, True),   # 256 x 256 tiles (160 of them), ragged M and N
+    (2305, 256, 4000, True),   # 256-row tiles of x (320 of them), ragged M and N
+    (130, 64, 128, True),      # weight in tensor memory, 128-row boxes: the second holds 2 rows
+    (200, 64, 18944, False),   # 256-row tiles (148 of them) with the box cut to 200 rows
+    (257, 128, 300, True),     # N % 8 != 0: the epilogue stores element by element
+    (150, 64, 13, False),      # one output tile, 13 live weight rows, element stores
 ])
 def test_linear_matches_oracle(M, K, N, with_bias):
     rng = np.random.default_rng(M * 7 + K * 3 + N)
@@ -223,7 +228,8 @@ def test_bounded_wait_reports_a_timeout_and_the_context_recovers(M, N):
     """A wait on a barrier that nothing completes (2 ms limit) runs out: the call reports
     NVFP4_ERR_TIMEOUT through the workspace instead of hanging, every role stops, and the
     next call on the same context and workspace is correct.  16 rows take the split-K
-    path, 700 rows the 256 x 128 tiles, 4096 rows on 2560 outputs the 256 x 256 tiles."""
+    path, 700 rows the tensor-memory weight with 128-row tiles of x, 4096 rows on 2560
+    outputs its 256-row tiles."""
     K = 1024
     rng = np.random.default_rng(M + N)
     x = synthetic.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
