@@ -749,7 +749,8 @@ template <int BT>
 struct TsCfg {
     static constexpr int kAtomABytes = BT * kBK * 2;          // one activation box
     static constexpr int kStageABytes = kTsAtoms * kAtomABytes;
-    static constexpr int kRingA = (192 * 1024) / kStageABytes;  // 3 stages for BT = 256, 6 for 128
+    // activation stages in flight: 192 KB of them (3 for BT = 256, 6 for 128), at most 8
+    static constexpr int kRingA = (192 * 1024) / kStageABytes < 8 ? (192 * 1024) / kStageABytes : 8;
     // kind::f16 instruction descriptor: fp32 D, bf16 A and B, both K-major, N = BT, M = 128
     static constexpr uint32_t kIdesc =
         (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BT >> 3) << 17) | ((uint32_t)(kMmaM >> 4) << 24);
@@ -767,7 +768,8 @@ struct TsCfg {
     };
     static constexpr int kRingBytes = kRingA * kStageABytes;
     static constexpr int kSmemBytes = 1024 + kRingBytes + (int)sizeof(Shared);
-    static_assert(BT == 128 || BT == 256, "MMA N");
+    static_assert(BT == 64 || BT == 128 || BT == 256, "MMA N");
+    static_assert(kRingA * kStageABytes >= kDecodeWarps * BT * 16, "the epilogue's transpose fits in the ring");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -944,27 +946,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int at = (g + kTsGroups * i) * kTsAtoms + t;
             return at < kt ? at : -1;
         };
-        RecRow next;
-        {
-            const int at = atom_of(0);
-            if (at >= 0) ld_rec_row(gcode + (int64_t)at * kRecBytes, gscale + (int64_t)at * kRecBytes, next);
-        }
-        bool ok = true;
-        for (int i = 0; g + kTsGroups * i < nk; ++i) {
-            const int kb = g + kTsGroups * i, st = kb % kTsRingT;
+        auto load = [&](int i, RecRow& r) {
             const int at = atom_of(i);
-            const RecRow cur = next;
-            {
-                const int an = atom_of(i + 1);
-                if (an >= 0 && g + kTsGroups * (i + 1) < nk)
-                    ld_rec_row(gcode + (int64_t)an * kRecBytes, gscale + (int64_t)an * kRecBytes, next);
-            }
+            if (at >= 0) ld_rec_row(gcode + (int64_t)at * kRecBytes, gscale + (int64_t)at * kRecBytes, r);
+        };
+        // own stage i from the record row in `cur`: wait for the slot, decode, store, arrive
+        auto step = [&](int i, const RecRow& cur) -> bool {
+            const int kb = g + kTsGroups * i, st = kb % kTsRingT;
             if (!warp_wait(smem_u32(&sh.w_empty[st]), ((uint32_t)(kb / kTsRingT) & 1u) ^ 1u, abort)) {
                 if (lane == 0) stop_all(sh, a.ws);
-                ok = false;
-                break;
+                return false;
             }
-            if (at >= 0) {  // an atom past the end of K is neither written nor multiplied
+            if (atom_of(i) >= 0) {  // an atom past the end of K is neither written nor multiplied
                 tc_fence_after();
                 uint32_t o[32];
 #pragma unroll
@@ -983,6 +976,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sh.w_full[st]));
+            return true;
+        };
+        // two record rows in flight, each register set refilled right after its own stage, so
+        // a load has two of this group's stages (four stages of the CTA) to arrive; with few
+        // rows of x the packed weight comes from HBM
+        RecRow r0, r1;
+        load(0, r0);
+        load(1, r1);
+        bool ok = true;
+        for (int i = 0; g + kTsGroups * i < nk; i += 2) {
+            if (!step(i, r0)) {
+                ok = false;
+                break;
+            }
+            load(i + 2, r0);
+            if (g + kTsGroups * (i + 1) >= nk) break;
+            if (!step(i + 1, r1)) {
+                ok = false;
+                break;
+            }
+            load(i + 3, r1);
         }
 
         // ---- epilogue: warp w reads lanes 32 q .. + 31 (weight rows n), columns (rows m of x)
@@ -1008,7 +1022,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int64_t mb = m0 + part * kCols;  // first row of x of this warp's patch
                 uint16_t* y = reinterpret_cast<uint16_t*>(a.y);
                 if (a.vec_store) {
-                    uint16_t* patch = reinterpret_cast<uint16_t*>(ring + warp * 4096);  // [kCols][32]
+                    uint16_t* patch = reinterpret_cast<uint16_t*>(ring + warp * kCols * 64);  // [kCols][32]
 #pragma unroll
                     for (int e = 0; e < kCols; ++e) {
                         float f = __uint_as_float(v[e]);
@@ -1085,7 +1099,9 @@ nvfp4_status gemm_smem_optin() {
             cudaFuncSetAttribute(w4a16_linear_ts_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  TsCfg<256>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(w4a16_linear_ts_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 TsCfg<128>::kSmemBytes) != cudaSuccess)
+                                 TsCfg<128>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(w4a16_linear_ts_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 TsCfg<64>::kSmemBytes) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         g_smem_set[dev] = true;
     }
@@ -1172,17 +1188,21 @@ NVFP4_API int64_t nvfp4_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     return splits > 1 ? split_workspace_bytes(M, N, splits) : (int64_t)sizeof(Workspace);
 }
 
-// More than 128 rows of x: the weight in tensor memory, tiles of 128 weight rows by BT rows
-// of x.  BT = 256 unless 128-row tiles need no more waves of one CTA per SM: a stage of a
-// 128-row tile takes ~85 % of the time of a 256-row one (the fixed cost of a stage does not
-// shrink with the MMAs), so 128-row tiles pay only where they fill SMs that would idle.
+// The weight in tensor memory, tiles of 128 weight rows by BT rows of x.  Up to 128 rows of
+// x, BT is M rounded up to 64 or 128.  Above that, BT = 256 unless 128-row tiles need no
+// more waves of one CTA per SM: a stage of a 128-row tile takes ~85 % of the time of a
+// 256-row one (the fixed cost of a stage does not shrink with the MMAs), so 128-row tiles
+// pay only where they fill SMs that would idle.
 static nvfp4_status w4a16_linear_ts(EncodeTiledFn encode, const void* x, int64_t M, int64_t K, const uint8_t* tiled,
                                     const float* d_global_scale, int64_t N, const void* bias, void* y,
                                     void* d_workspace, uint64_t selftest_ns, int sms, nvfp4_stream_t stream) {
     const int64_t tiles_n = (N + kRecRows - 1) / kRecRows;
-    const int64_t w256 = (tiles_n * ((M + 255) / 256) + sms - 1) / sms;
-    const int64_t w128 = (tiles_n * ((M + 127) / 128) + sms - 1) / sms;
-    const int bt = w128 <= w256 ? 128 : 256;
+    int bt = M <= 64 ? 64 : 128;
+    if (M > kMmaM) {
+        const int64_t w256 = (tiles_n * ((M + 255) / 256) + sms - 1) / sms;
+        const int64_t w128 = (tiles_n * ((M + 127) / 128) + sms - 1) / sms;
+        bt = w128 <= w256 ? 128 : 256;
+    }
     const int64_t tiles_m = (M + bt - 1) / bt;
 
     // x as a [M, K] bf16 tensor, boxes of bt rows x 64 columns, 128-byte swizzle, zero fill
@@ -1221,8 +1241,10 @@ static nvfp4_status w4a16_linear_ts(EncodeTiledFn encode, const void* x, int64_t
     cudaStream_t cst = reinterpret_cast<cudaStream_t>(stream);
     if (bt == 256)
         w4a16_linear_ts_kernel<256><<<grid, kGemmThreads, TsCfg<256>::kSmemBytes, cst>>>(map, a);
-    else
+    else if (bt == 128)
         w4a16_linear_ts_kernel<128><<<grid, kGemmThreads, TsCfg<128>::kSmemBytes, cst>>>(map, a);
+    else
+        w4a16_linear_ts_kernel<64><<<grid, kGemmThreads, TsCfg<64>::kSmemBytes, cst>>>(map, a);
     note_launch();
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
@@ -1253,7 +1275,16 @@ static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const
     int sms = 0;
     st = sm_count_w4(&sms);
     if (st != NVFP4_OK) return st;
-    if (M > kMmaM)
+    // The weight in shared memory for up to 128 rows of x with K split over several CTAs per
+    // tile (a weight with few output tiles, and a workspace with room for the partial sums),
+    // and for up to 32 rows unsplit; everything else with the weight in tensor memory.  With
+    // few rows of x both are bound by the rate at which one thread issues MMAs (~50 ns per
+    // 128 x N x 16 step, whatever N), so they only differ in fixed costs: measured, the
+    // shared-memory kernel is ~0.8 us faster up to 32 rows, the tensor-memory one ~4 us
+    // faster at 128.
+    int splits = M > kMmaM ? 1 : split_count(M, N, K, sms);
+    if (splits > 1 && workspace_bytes < split_workspace_bytes(M, N, splits)) splits = 1;
+    if (M > kMmaM || (splits == 1 && M > 32))
         return w4a16_linear_ts(encode, x, M, K, tiled, d_global_scale, N, bias, y, d_workspace, selftest_ns, sms,
                                stream);
     const int64_t tiles_m = (M + kMmaM - 1) / kMmaM;  // 1: at most 128 rows here
@@ -1290,8 +1321,7 @@ static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const
     a.a_bytes = (uint32_t)box_rows * kBK * 2;
     a.selftest_ns = selftest_ns;
     // split K only with a workspace large enough for the partial sums
-    a.splits = split_count(M, N, K, sms);
-    if (a.splits > 1 && workspace_bytes < split_workspace_bytes(M, N, a.splits)) a.splits = 1;
+    a.splits = splits;
     a.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(d_workspace) + counters_offset());
     a.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(d_workspace) + partial_offset(tiles_n));
     const unsigned grid = (unsigned)(tiles_m * tiles_n * a.splits);
