@@ -351,9 +351,9 @@ nvfp4_status nvfp4_w4a16_pack(const uint8_t* packed, const uint8_t* scales, int6
  * the packed weight: [FP4OPT] _float4_autocast_forward, which unpacks the weight for one
  * forward and runs the layer's bf16 forward on it.  One kernel on the tensor cores (bf16 x
  * bf16, fp32 accumulation, output rounded to bf16 once; the bias is added to the fp32 sum
- * before that rounding); the decoded weight is built tile by tile on chip (in shared memory
- * for at most 128 rows of x, in tensor memory for more) and never written to device
- * memory.  Each weight element is decoded exactly as
+ * before that rounding); the decoded weight is built tile by tile on chip (in tensor
+ * memory, or in shared memory for up to 32 rows of x and whenever K is split) and never
+ * written to device memory.  Each weight element is decoded exactly as
  * nvfp4_dequantize does; the sum is not bit-reproducible against another GEMM (the order
  * in which the tensor cores accumulate is not sequential IEEE), the tests state the bound.
  *   x       bf16 [M, K] row-major, 16-byte aligned; K a positive multiple of 16

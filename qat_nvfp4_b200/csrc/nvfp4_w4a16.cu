@@ -15,11 +15,11 @@
 //   warp 16    TMA loads of activation tiles
 //   warp 17    TMEM allocation, MMA issue (one elected thread), TMEM release
 //
-// Up to 128 rows of x (w4a16_linear_kernel): x is the MMA's A operand, the decoded weight
-// tile the B operand in shared memory (128-byte swizzle, K-major), passed from the decode
-// warps to the MMAs through a ring of 2 or 3 tiles; K may be split over several CTAs per
-// tile.  More rows (w4a16_linear_ts_kernel): the decoded weight is the A operand, kept in
-// tensor memory, and x the B operand.
+// w4a16_linear_kernel (up to 128 rows of x with K split over several CTAs per tile, and up
+// to 32 rows unsplit): x is the MMA's A operand, the decoded weight tile the B operand in
+// shared memory (128-byte swizzle, K-major), passed from the decode warps to the MMAs
+// through a ring of 2 or 3 tiles.  w4a16_linear_ts_kernel (everything else): the decoded
+// weight is the A operand, kept in tensor memory, and x the B operand.
 //
 // Every wait on an mbarrier is bounded (kWaitLimitNs of %globaltimer); a wait that runs
 // out records NVFP4_ERR_TIMEOUT in the caller's workspace, tells the other roles to stop,
