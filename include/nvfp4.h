@@ -395,6 +395,20 @@ nvfp4_status nvfp4_w4a16_selftest_timeout(const void* x, int64_t M, int64_t K, c
  * count. */
 int64_t nvfp4_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
+/* How nvfp4_w4a16_linear runs x [M, K] . W[N, K]^T with a workspace of workspace_bytes on a
+ * device with `sms` SMs (the decision that call takes with the current device's SM count).
+ * Host only: launches nothing and needs no GPU.
+ *   *kernel         0: the weight decoded into shared memory (split K, or at most 32 rows of
+ *                   x); 1: the weight decoded into tensor memory (everything else)
+ *   *rows_per_tile  rows of x per output tile (each tile also covers 128 weight rows): 128
+ *                   for kernel 0; for kernel 1, 64 or 128 up to 128 rows of x, above that
+ *                   256, or 128 where 128-row tiles need no more waves of one CTA per SM
+ *   *splits         CTAs per output tile over K (kernel 0 only; 1 otherwise)
+ * Errors: NVFP4_ERR_SHAPE as nvfp4_w4a16_linear, NVFP4_ERR_NULL (an output pointer),
+ * NVFP4_ERR_ARG (sms < 1). */
+nvfp4_status nvfp4_w4a16_plan(int64_t M, int64_t N, int64_t K, int64_t workspace_bytes, int sms, int* kernel,
+                              int* rows_per_tile, int* splits);
+
 /* Human-readable name of a status code (a static string). */
 const char* nvfp4_status_string(nvfp4_status status);
 

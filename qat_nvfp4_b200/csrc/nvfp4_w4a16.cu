@@ -1152,6 +1152,39 @@ int64_t split_workspace_bytes(int64_t M, int64_t N, int splits) {
     return partial_offset(tiles) + (int64_t)splits * tiles * 128 * 128 * 4;
 }
 
+// How a call runs.  The weight in shared memory (w4a16_linear_kernel) for up to 128 rows of
+// x with K split over several CTAs per tile (a weight with few output tiles, and a workspace
+// with room for the partial sums), and for up to 32 rows unsplit; everything else with the
+// weight in tensor memory (w4a16_linear_ts_kernel).  With few rows of x both kernels are
+// bound by the rate at which one thread issues MMAs (~50 ns per 128 x N x 16 step, whatever
+// N), so they only differ in fixed costs: measured, the shared-memory kernel is ~0.8 us
+// faster up to 32 rows, the tensor-memory one ~4 us faster at 128.
+//
+// Tensor-memory tiles are 128 weight rows by bt rows of x.  Up to 128 rows of x, bt is M
+// rounded up to 64 or 128.  Above that, bt = 256 unless 128-row tiles need no more waves of
+// one CTA per SM: a stage of a 128-row tile takes ~85 % of the time of a 256-row one (the
+// fixed cost of a stage does not shrink with the MMAs), so 128-row tiles pay only where
+// they fill SMs that would idle.
+struct Plan {
+    int ts;      // 1: weight in tensor memory, 0: in shared memory
+    int bt;      // rows of x per output tile
+    int splits;  // CTAs per output tile over K
+};
+
+Plan make_plan(int64_t M, int64_t N, int64_t K, int64_t workspace_bytes, int sms) {
+    int splits = M > kMmaM ? 1 : split_count(M, N, K, sms);
+    if (splits > 1 && workspace_bytes < split_workspace_bytes(M, N, splits)) splits = 1;
+    if (M <= kMmaM && (splits > 1 || M <= 32)) return Plan{0, kMmaM, splits};
+    const int64_t tiles_n = (N + kRecRows - 1) / kRecRows;
+    int bt = M <= 64 ? 64 : 128;
+    if (M > kMmaM) {
+        const int64_t w256 = (tiles_n * ((M + 255) / 256) + sms - 1) / sms;
+        const int64_t w128 = (tiles_n * ((M + 127) / 128) + sms - 1) / sms;
+        bt = w128 <= w256 ? 128 : 256;
+    }
+    return Plan{1, bt, 1};
+}
+
 }  // namespace
 }  // namespace nvfp4
 
@@ -1188,21 +1221,11 @@ NVFP4_API int64_t nvfp4_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     return splits > 1 ? split_workspace_bytes(M, N, splits) : (int64_t)sizeof(Workspace);
 }
 
-// The weight in tensor memory, tiles of 128 weight rows by BT rows of x.  Up to 128 rows of
-// x, BT is M rounded up to 64 or 128.  Above that, BT = 256 unless 128-row tiles need no
-// more waves of one CTA per SM: a stage of a 128-row tile takes ~85 % of the time of a
-// 256-row one (the fixed cost of a stage does not shrink with the MMAs), so 128-row tiles
-// pay only where they fill SMs that would idle.
+// The weight in tensor memory, tiles of 128 weight rows by bt rows of x (make_plan).
 static nvfp4_status w4a16_linear_ts(EncodeTiledFn encode, const void* x, int64_t M, int64_t K, const uint8_t* tiled,
                                     const float* d_global_scale, int64_t N, const void* bias, void* y,
-                                    void* d_workspace, uint64_t selftest_ns, int sms, nvfp4_stream_t stream) {
+                                    void* d_workspace, uint64_t selftest_ns, int bt, nvfp4_stream_t stream) {
     const int64_t tiles_n = (N + kRecRows - 1) / kRecRows;
-    int bt = M <= 64 ? 64 : 128;
-    if (M > kMmaM) {
-        const int64_t w256 = (tiles_n * ((M + 255) / 256) + sms - 1) / sms;
-        const int64_t w128 = (tiles_n * ((M + 127) / 128) + sms - 1) / sms;
-        bt = w128 <= w256 ? 128 : 256;
-    }
     const int64_t tiles_m = (M + bt - 1) / bt;
 
     // x as a [M, K] bf16 tensor, boxes of bt rows x 64 columns, 128-byte swizzle, zero fill
@@ -1249,6 +1272,19 @@ static nvfp4_status w4a16_linear_ts(EncodeTiledFn encode, const void* x, int64_t
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+NVFP4_API nvfp4_status nvfp4_w4a16_plan(int64_t M, int64_t N, int64_t K, int64_t workspace_bytes, int sms,
+                                        int* kernel, int* rows_per_tile, int* splits) {
+    if (M < 0 || !weight_shape_ok(N, K) || M > 0x7FFFFF00ll) return NVFP4_ERR_SHAPE;
+    if (((M + kMmaM - 1) / kMmaM) * ((N + 127) / 128) > 0x7FFFFFFFll) return NVFP4_ERR_SHAPE;
+    if (kernel == nullptr || rows_per_tile == nullptr || splits == nullptr) return NVFP4_ERR_NULL;
+    if (sms < 1) return NVFP4_ERR_ARG;
+    const Plan plan = make_plan(M, N, K, workspace_bytes, sms);
+    *kernel = plan.ts;
+    *rows_per_tile = plan.bt;
+    *splits = plan.splits;
+    return NVFP4_OK;
+}
+
 static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const uint8_t* tiled,
                                       const float* d_global_scale, int64_t N, const void* bias, void* y,
                                       void* d_workspace, int64_t workspace_bytes, uint64_t selftest_ns,
@@ -1275,18 +1311,11 @@ static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const
     int sms = 0;
     st = sm_count_w4(&sms);
     if (st != NVFP4_OK) return st;
-    // The weight in shared memory for up to 128 rows of x with K split over several CTAs per
-    // tile (a weight with few output tiles, and a workspace with room for the partial sums),
-    // and for up to 32 rows unsplit; everything else with the weight in tensor memory.  With
-    // few rows of x both are bound by the rate at which one thread issues MMAs (~50 ns per
-    // 128 x N x 16 step, whatever N), so they only differ in fixed costs: measured, the
-    // shared-memory kernel is ~0.8 us faster up to 32 rows, the tensor-memory one ~4 us
-    // faster at 128.
-    int splits = M > kMmaM ? 1 : split_count(M, N, K, sms);
-    if (splits > 1 && workspace_bytes < split_workspace_bytes(M, N, splits)) splits = 1;
-    if (M > kMmaM || (splits == 1 && M > 32))
-        return w4a16_linear_ts(encode, x, M, K, tiled, d_global_scale, N, bias, y, d_workspace, selftest_ns, sms,
+    const Plan plan = make_plan(M, N, K, workspace_bytes, sms);
+    if (plan.ts)
+        return w4a16_linear_ts(encode, x, M, K, tiled, d_global_scale, N, bias, y, d_workspace, selftest_ns, plan.bt,
                                stream);
+    const int splits = plan.splits;
     const int64_t tiles_m = (M + kMmaM - 1) / kMmaM;  // 1: at most 128 rows here
     const int64_t tiles_n = (N + 127) / 128;
 
@@ -1320,8 +1349,7 @@ static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const
     a.vec_store = (is_aligned(y, 16) && N % 8 == 0) ? 1 : 0;
     a.a_bytes = (uint32_t)box_rows * kBK * 2;
     a.selftest_ns = selftest_ns;
-    // split K only with a workspace large enough for the partial sums
-    a.splits = splits;
+    a.splits = splits;  // > 1 only with a workspace large enough for the partial sums
     a.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(d_workspace) + counters_offset());
     a.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(d_workspace) + partial_offset(tiles_n));
     const unsigned grid = (unsigned)(tiles_m * tiles_n * a.splits);

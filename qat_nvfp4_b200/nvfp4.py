@@ -77,6 +77,8 @@ _c_w4a16_tiled_bytes = _sig("nvfp4_w4a16_tiled_bytes", [_i64, _i64], _i64)
 _c_w4a16_pack = _sig("nvfp4_w4a16_pack", [_vp, _vp, _i64, _i64, _vp, _vp])
 _c_w4a16_linear = _sig("nvfp4_w4a16_linear", [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _vp])
 _c_w4a16_workspace_bytes = _sig("nvfp4_w4a16_workspace_bytes", [_i64, _i64, _i64], _i64)
+_c_w4a16_plan = _sig("nvfp4_w4a16_plan", [_i64, _i64, _i64, _i64, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                                          ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)])
 _c_w4a16_selftest_timeout = _sig("nvfp4_w4a16_selftest_timeout",
                                  [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _i64, ctypes.c_uint32, _vp])
 _c_status_string = _sig("nvfp4_status_string", [ctypes.c_int], ctypes.c_char_p)
@@ -635,6 +637,16 @@ def nvfp4_w4a16_workspace_bytes(M: int, N: int, K: int) -> int:
     """Workspace bytes with which nvfp4_w4a16_linear may split K on this shape (current
     device), at least WORKSPACE_BYTES; -1 if the shape is refused."""
     return int(_c_w4a16_workspace_bytes(M, N, K))
+
+
+def nvfp4_w4a16_plan(M: int, N: int, K: int, workspace_bytes: int, sms: int) -> tuple[str, int, int]:
+    """How nvfp4_w4a16_linear runs this shape with a workspace of workspace_bytes on a device
+    with `sms` SMs: where the decoded weight lives ("shared" or "tensor" memory), the rows of
+    x per output tile, and the CTAs per tile over K.  Host only, no GPU needed."""
+    kernel, rows, splits = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(_c_w4a16_plan(M, N, K, workspace_bytes, sms, ctypes.byref(kernel), ctypes.byref(rows),
+                         ctypes.byref(splits)), "nvfp4_w4a16_plan")
+    return ("tensor" if kernel.value else "shared"), rows.value, splits.value
 
 
 def nvfp4_w4a16_workspace(M: int, N: int, K: int, device) -> torch.Tensor:

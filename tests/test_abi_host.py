@@ -34,7 +34,7 @@ def test_header_declares_the_entry_points():
                      "nvfp4_quantize_bs", "nvfp4_dequantize_bs", "nvfp4_fake_quant_bs", "nvfp4_w4a16_linear",
                      "nvfp4_w4a16_pack", "nvfp4_w4a16_tiled_bytes", "nvfp4_quantize_fused",
                      "nvfp4_amax_accumulate", "nvfp4_w4a16_workspace_bytes", "nvfp4_amax_strided",
-                     "nvfp4_quantize_strided", "nvfp4_fake_quant_strided",
+                     "nvfp4_quantize_strided", "nvfp4_fake_quant_strided", "nvfp4_w4a16_plan",
                      "nvfp4_status_string", "nvfp4_kernel_launch_count"]:
         assert required in names
 
@@ -252,6 +252,58 @@ def test_binding_refuses_cpu_tensors():
         with pytest.raises(RuntimeError, match="CUDA tensor"):
             call()
 
+
+
+BIG_WS = 1 << 40
+
+
+@pytest.mark.parametrize("M,N,K,ws,sms,want", [
+    # up to 128 rows of x on a weight with few tiles: split K in shared memory when the
+    # workspace has room (148 SMs / 32 tiles = 4 CTAs per tile, at least 8 atoms each) ...
+    (16, 4096, 4096, BIG_WS, 148, ("shared", 128, 4)),
+    (100, 4096, 4096, BIG_WS, 148, ("shared", 128, 4)),
+    (16, 4096, 4096, BIG_WS, 132, ("shared", 128, 4)),
+    # ... and without room, or with too little K to split (8 atoms): shared memory up to 32
+    # rows, tensor memory above, tiles of 64 or 128 rows of x
+    (16, 4096, 4096, 256, 148, ("shared", 128, 1)),
+    (100, 4096, 4096, 256, 148, ("tensor", 128, 1)),
+    (16, 4096, 512, BIG_WS, 148, ("shared", 128, 1)),
+    (100, 4096, 512, BIG_WS, 148, ("tensor", 128, 1)),
+    # a weight with 112 tiles is never split (148 / 112 = 1)
+    (16, 14336, 4096, BIG_WS, 148, ("shared", 128, 1)),
+    (32, 14336, 4096, BIG_WS, 148, ("shared", 128, 1)),
+    (33, 14336, 4096, BIG_WS, 148, ("tensor", 64, 1)),
+    (64, 14336, 4096, BIG_WS, 148, ("tensor", 64, 1)),
+    (65, 14336, 4096, BIG_WS, 148, ("tensor", 128, 1)),
+    (128, 14336, 4096, BIG_WS, 148, ("tensor", 128, 1)),
+    # more rows: 256-row tiles unless 128-row tiles need no more waves of one CTA per SM
+    (129, 4096, 4096, BIG_WS, 148, ("tensor", 128, 1)),      # 32 vs 64 tiles: one wave either way
+    (512, 4096, 4096, BIG_WS, 148, ("tensor", 128, 1)),      # 64 vs 128 tiles: one wave either way
+    (1024, 4096, 4096, BIG_WS, 148, ("tensor", 256, 1)),     # 128 tiles: 1 wave vs 2
+    (4096, 4096, 4096, BIG_WS, 148, ("tensor", 256, 1)),     # 512 vs 1024 tiles: 4 waves vs 7
+    (1024, 14336, 4096, BIG_WS, 148, ("tensor", 256, 1)),    # 448 vs 896 tiles: 4 waves vs 7
+    (1024, 4096, 4096, BIG_WS, 64, ("tensor", 256, 1)),      # 2 waves vs 4
+    (1024, 4096, 4096, BIG_WS, 512, ("tensor", 128, 1)),     # 1 wave either way
+    (200, 18944, 64, BIG_WS, 148, ("tensor", 256, 1)),       # 148 tiles: 1 wave vs 2
+])
+def test_w4a16_plan(M, N, K, ws, sms, want):
+    """Host-only: which kernel, tile height and K split nvfp4_w4a16_linear takes, from the
+    rules stated in the header (worked out by hand here)."""
+    from qat_nvfp4_b200 import nvfp4 as nv
+    assert nv.nvfp4_w4a16_plan(M, N, K, ws, sms) == want
+
+
+def test_w4a16_plan_refusals(lib):
+    f = lib.nvfp4_w4a16_plan
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int64] * 4 + [ctypes.c_int] + [ctypes.POINTER(ctypes.c_int)] * 3
+    k, r, s = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    out = (ctypes.byref(k), ctypes.byref(r), ctypes.byref(s))
+    assert f(16, 4096, 4096, 256, 148, *out) == NVFP4_OK
+    assert f(16, 4096, 4096, 256, 0, *out) == ERR_ARG
+    assert f(16, 4096, 24, 256, 148, *out) == ERR_SHAPE
+    assert f(-1, 4096, 4096, 256, 148, *out) == ERR_SHAPE
+    assert f(16, 4096, 4096, 256, 148, None, ctypes.byref(r), ctypes.byref(s)) == ERR_NULL
 
 
 def test_w4a16_record_sizes(lib):
