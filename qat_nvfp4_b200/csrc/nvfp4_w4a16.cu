@@ -1059,6 +1059,120 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------
+// Up to 8 rows of x: the CUDA cores.  With so few rows an MMA (128 weight rows x 16 of K per
+// instruction, ~50 ns to issue whatever its N) does almost no work for its cost, and the call
+// is bound by the number of MMAs; on the CUDA cores it is bound by reading the packed weight.
+//
+// One CTA per 32 weight rows (a quarter of a record row), 8 warps: warp w takes the atoms w,
+// w + 8, ... of K, each lane one weight row.  Per atom a lane reads its row's 32 code bytes
+// and scale word (a warp reads 1 KB and 128 bytes, each contiguous; the next atom's are
+// loaded before the current one is used), decodes them exactly as nvfp4_dequantize does,
+// and accumulates x[m][k] w[k] for the rows of x in fp32: a product of two bf16 values is
+// exact in fp32, and k and k + 1 go to the two halves of one packed f32x2 FMA.  The halves,
+// then the 8 warps' partial sums (in warp order) are added in shared memory, then the bias,
+// then one rounding to bf16.
+
+constexpr int kGemvWarps = 8;
+constexpr int kGemvRows = 32;
+constexpr int kGemvMaxRows = 8;  // rows of x the CUDA-core kernel takes
+
+__device__ __forceinline__ uint64_t f32x2_of_bf16x2(uint32_t v) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(v << 16), "r"(v & 0xFFFF0000u));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ void ld_nc_b128(const void* p, uint32_t (&v)[4]) {
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]) : "l"(p));
+}
+
+template <int MT>
+__global__ void __launch_bounds__(32 * kGemvWarps)
+    w4a16_gemv_kernel(const uint16_t* __restrict__ x, const LinearArgs a) {
+    static_assert(MT >= 1 && MT <= kGemvMaxRows && 32 * MT <= 32 * kGemvWarps, "rows of x");
+    __shared__ float sd_tab[256];
+    __shared__ float red[kGemvWarps][MT][kGemvRows];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    {
+        const float gs = __ldg(a.d_gs);
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) sd_tab[i] = __fdiv_rn(e4m3_to_f32((uint32_t)i), gs);
+    }
+    __syncthreads();
+    const int64_t n0 = (int64_t)blockIdx.x * kGemvRows;
+    const int64_t tn = n0 / kRecRows;
+    const int row = (int)(n0 % kRecRows) + lane;  // this lane's row of the record
+    const int kt = (int)a.kt;
+    const int mrows = (int)(a.M < MT ? a.M : MT);
+    const uint8_t* rec0 = a.tiled + tn * a.kt * kRecBytes;
+    uint64_t acc[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) acc[m] = 0ull;  // (+0.0f, +0.0f)
+    RecRow cur;
+    if (warp < kt) ld_rec_row(rec0 + (int64_t)warp * kRecBytes + row * 32, rec0 + (int64_t)warp * kRecBytes + kRecCodes + row * 4, cur);
+    for (int tk = warp; tk < kt; tk += kGemvWarps) {
+        RecRow nxt;
+        const int tn1 = tk + kGemvWarps;
+        if (tn1 < kt)
+            ld_rec_row(rec0 + (int64_t)tn1 * kRecBytes + row * 32, rec0 + (int64_t)tn1 * kRecBytes + kRecCodes + row * 4,
+                       nxt);
+        // 16-element blocks of this atom inside K (K is a multiple of 16)
+        const int64_t left = (a.K - (int64_t)tk * kBK) / kBlockElems;
+        const int nb = left < 4 ? (int)left : 4;
+#pragma unroll
+        for (int b = 0; b < kBK / kBlockElems; ++b) {
+            if (b >= nb) break;
+            const float sd = sd_tab[(cur.sc >> (8 * b)) & 0xFFu];
+            uint64_t sd2;
+            asm("mov.b64 %0, {%1, %1};" : "=l"(sd2) : "f"(sd));
+            uint64_t w2[8];  // the block's 16 weights, as (w[k], w[k + 1]) pairs
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                w2[j] = f32x2_of_bf16x2(decode_pair_x2((cur.c[2 * b] >> (8 * j)) & 0xFFu, sd2));
+                w2[4 + j] = f32x2_of_bf16x2(decode_pair_x2((cur.c[2 * b + 1] >> (8 * j)) & 0xFFu, sd2));
+            }
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                if (m >= mrows) break;
+                const uint16_t* xp = x + (int64_t)m * a.K + (int64_t)tk * kBK + b * kBlockElems;
+                uint32_t v0[4], v1[4];
+                ld_nc_b128(xp, v0);
+                ld_nc_b128(xp + 8, v1);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    acc[m] = fma_f32x2(f32x2_of_bf16x2(v0[i]), w2[i], acc[m]);
+                    acc[m] = fma_f32x2(f32x2_of_bf16x2(v1[i]), w2[4 + i], acc[m]);
+                }
+            }
+        }
+        if (tn1 < kt) cur = nxt;
+    }
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+        float lo, hi;
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(acc[m]));
+        red[warp][m][lane] = __fadd_rn(lo, hi);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32 * MT) {
+        const int m = threadIdx.x >> 5, l = threadIdx.x & 31;
+        const int64_t n = n0 + l;
+        if (m < mrows && n < a.N) {
+            float f = red[0][m][l];
+#pragma unroll
+            for (int w = 1; w < kGemvWarps; ++w) f = __fadd_rn(f, red[w][m][l]);
+            if (a.bias != nullptr) f = __fadd_rn(f, __uint_as_float((uint32_t)__ldg(a.bias + n) << 16));
+            reinterpret_cast<uint16_t*>(a.y)[(int64_t)m * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------
 // Host side.
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -1152,7 +1266,8 @@ int64_t split_workspace_bytes(int64_t M, int64_t N, int splits) {
     return partial_offset(tiles) + (int64_t)splits * tiles * 128 * 128 * 4;
 }
 
-// How a call runs.  The weight in shared memory (w4a16_linear_kernel) for up to 128 rows of
+// How a call runs.  Up to 8 rows of x: the CUDA cores (w4a16_gemv_kernel), MT = M rounded up
+// to 1, 2, 4 or 8 rows.  Otherwise the weight in shared memory (w4a16_linear_kernel) for up to 128 rows of
 // x with K split over several CTAs per tile (a weight with few output tiles, and a workspace
 // with room for the partial sums), and for up to 32 rows unsplit; everything else with the
 // weight in tensor memory (w4a16_linear_ts_kernel).  With few rows of x both kernels are
@@ -1166,12 +1281,14 @@ int64_t split_workspace_bytes(int64_t M, int64_t N, int splits) {
 // fixed cost of a stage does not shrink with the MMAs), so 128-row tiles pay only where
 // they fill SMs that would idle.
 struct Plan {
-    int ts;      // 1: weight in tensor memory, 0: in shared memory
+    int kind;    // 0: weight in shared memory, 1: in tensor memory, 2: CUDA cores
     int bt;      // rows of x per output tile
     int splits;  // CTAs per output tile over K
 };
 
-Plan make_plan(int64_t M, int64_t N, int64_t K, int64_t workspace_bytes, int sms) {
+Plan make_plan(int64_t M, int64_t N, int64_t K, int64_t workspace_bytes, int sms, bool cuda_cores = true) {
+    if (cuda_cores && M <= kGemvMaxRows && (N + kGemvRows - 1) / kGemvRows <= 0x7FFFFFFFll)
+        return Plan{2, M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8)), 1};
     int splits = M > kMmaM ? 1 : split_count(M, N, K, sms);
     if (splits > 1 && workspace_bytes < split_workspace_bytes(M, N, splits)) splits = 1;
     if (M <= kMmaM && (splits > 1 || M <= 32)) return Plan{0, kMmaM, splits};
@@ -1217,8 +1334,8 @@ NVFP4_API int64_t nvfp4_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     if (M < 0 || !weight_shape_ok(N, K)) return -1;
     int sms = 0;
     if (sm_count_w4(&sms) != NVFP4_OK) sms = 148;
-    const int splits = split_count(M, N, K, sms);
-    return splits > 1 ? split_workspace_bytes(M, N, splits) : (int64_t)sizeof(Workspace);
+    const Plan plan = make_plan(M, N, K, (int64_t)1 << 62, sms);
+    return plan.kind == 0 && plan.splits > 1 ? split_workspace_bytes(M, N, plan.splits) : (int64_t)sizeof(Workspace);
 }
 
 // The weight in tensor memory, tiles of 128 weight rows by bt rows of x (make_plan).
@@ -1279,7 +1396,7 @@ NVFP4_API nvfp4_status nvfp4_w4a16_plan(int64_t M, int64_t N, int64_t K, int64_t
     if (kernel == nullptr || rows_per_tile == nullptr || splits == nullptr) return NVFP4_ERR_NULL;
     if (sms < 1) return NVFP4_ERR_ARG;
     const Plan plan = make_plan(M, N, K, workspace_bytes, sms);
-    *kernel = plan.ts;
+    *kernel = plan.kind;
     *rows_per_tile = plan.bt;
     *splits = plan.splits;
     return NVFP4_OK;
@@ -1311,8 +1428,36 @@ static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const
     int sms = 0;
     st = sm_count_w4(&sms);
     if (st != NVFP4_OK) return st;
-    const Plan plan = make_plan(M, N, K, workspace_bytes, sms);
-    if (plan.ts)
+    // the self-test needs a kernel with barrier waits: not the CUDA-core one
+    const Plan plan = make_plan(M, N, K, workspace_bytes, sms, selftest_ns == 0);
+    if (plan.kind == 2) {
+        LinearArgs a;
+        std::memset(&a, 0, sizeof(a));
+        a.tiled = tiled;
+        a.d_gs = d_global_scale;
+        a.bias = static_cast<const uint16_t*>(bias);
+        a.y = static_cast<uint8_t*>(y);
+        a.ws = static_cast<Workspace*>(d_workspace);
+        a.M = M;
+        a.N = N;
+        a.K = K;
+        a.kt = (K + kBK - 1) / kBK;
+        a.splits = 1;
+        const unsigned grid = (unsigned)((N + kGemvRows - 1) / kGemvRows);
+        const uint16_t* xh = static_cast<const uint16_t*>(x);
+        cudaStream_t cst = reinterpret_cast<cudaStream_t>(stream);
+        if (plan.bt == 1)
+            w4a16_gemv_kernel<1><<<grid, 32 * kGemvWarps, 0, cst>>>(xh, a);
+        else if (plan.bt == 2)
+            w4a16_gemv_kernel<2><<<grid, 32 * kGemvWarps, 0, cst>>>(xh, a);
+        else if (plan.bt == 4)
+            w4a16_gemv_kernel<4><<<grid, 32 * kGemvWarps, 0, cst>>>(xh, a);
+        else
+            w4a16_gemv_kernel<8><<<grid, 32 * kGemvWarps, 0, cst>>>(xh, a);
+        note_launch();
+        return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+    }
+    if (plan.kind == 1)
         return w4a16_linear_ts(encode, x, M, K, tiled, d_global_scale, N, bias, y, d_workspace, selftest_ns, plan.bt,
                                stream);
     const int splits = plan.splits;

@@ -641,12 +641,13 @@ def nvfp4_w4a16_workspace_bytes(M: int, N: int, K: int) -> int:
 
 def nvfp4_w4a16_plan(M: int, N: int, K: int, workspace_bytes: int, sms: int) -> tuple[str, int, int]:
     """How nvfp4_w4a16_linear runs this shape with a workspace of workspace_bytes on a device
-    with `sms` SMs: where the decoded weight lives ("shared" or "tensor" memory), the rows of
-    x per output tile, and the CTAs per tile over K.  Host only, no GPU needed."""
+    with `sms` SMs: where the decoded weight lives ("shared" or "tensor" memory, or "cores":
+    registers of the CUDA-core kernel), the rows of x per output tile, and the CTAs per tile
+    over K.  Host only, no GPU needed."""
     kernel, rows, splits = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
     _check(_c_w4a16_plan(M, N, K, workspace_bytes, sms, ctypes.byref(kernel), ctypes.byref(rows),
                          ctypes.byref(splits)), "nvfp4_w4a16_plan")
-    return ("tensor" if kernel.value else "shared"), rows.value, splits.value
+    return ("shared", "tensor", "cores")[kernel.value], rows.value, splits.value
 
 
 def nvfp4_w4a16_workspace(M: int, N: int, K: int, device) -> torch.Tensor:

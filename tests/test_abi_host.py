@@ -258,6 +258,13 @@ BIG_WS = 1 << 40
 
 
 @pytest.mark.parametrize("M,N,K,ws,sms,want", [
+    # up to 8 rows of x: the CUDA cores, rows rounded up to 1, 2, 4 or 8, never split
+    (1, 4096, 4096, BIG_WS, 148, ("cores", 1, 1)),
+    (2, 14336, 4096, BIG_WS, 148, ("cores", 2, 1)),
+    (3, 4096, 4096, 256, 148, ("cores", 4, 1)),
+    (5, 13, 16, BIG_WS, 148, ("cores", 8, 1)),
+    (8, 4096, 4096, BIG_WS, 148, ("cores", 8, 1)),
+    (9, 14336, 4096, BIG_WS, 148, ("shared", 128, 1)),
     # up to 128 rows of x on a weight with few tiles: split K in shared memory when the
     # workspace has room (148 SMs / 32 tiles = 4 CTAs per tile, at least 8 atoms each) ...
     (16, 4096, 4096, BIG_WS, 148, ("shared", 128, 4)),

@@ -186,6 +186,54 @@ def test_out_parameter_and_leading_dimensions():
     _assert_within_bound(bits(y).reshape(6, 64), bits(x).reshape(6, 256), packed, scales, gs, None, "3-D x")
 
 
+@pytest.mark.parametrize("M,K,N,with_bias", [
+    (1, 4096, 4096, False),
+    (2, 1040, 200, True),     # K % 64 == 16: the last atom has one block
+    (3, 64, 300, True),       # one atom of K: seven of the eight warps have none
+    (4, 16, 13, False),       # one block of K, 13 live rows of one 32-row tile
+    (7, 4160, 1000, True),
+    (8, 1088, 128, False),
+    (8, 4096, 14336, True),   # the pages' MLP weight
+])
+def test_cuda_core_rows_match_oracle(M, K, N, with_bias):
+    """Up to 8 rows of x the call runs on the CUDA cores (decode in registers, fp32 FMAs):
+    every output within the bound, and a second call bit-identical (the partial sums are
+    added in a fixed order)."""
+    assert nv.nvfp4_w4a16_plan(M, N, K, nv.WORKSPACE_BYTES, 148)[0] == "cores"
+    rng = np.random.default_rng(M * 11 + K + N)
+    x = synthetic.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    packed, scales, gs = _weight(N, K, M + 2 * K + N)
+    bias = synthetic.to_bf16_bits(rng.standard_normal(N).astype(np.float32)) if with_bias else None
+    tiled = nv.nvfp4_w4a16_pack(packed, scales)
+    xd, bd = to_dev(x), (to_dev(bias) if with_bias else None)
+    y1 = nv.nvfp4_w4a16_linear(xd, tiled, gs, N, bias=bd)
+    y2 = nv.nvfp4_w4a16_linear(xd, tiled, gs, N, bias=bd)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    _assert_within_bound(bits(y1), x, packed, scales, gs, bias, f"CUDA cores, {M} rows")
+
+
+@pytest.mark.parametrize("K,N", [(64, 300), (1088, 200)])
+def test_cuda_core_decode_is_exact_through_one_hot_rows(K, N):
+    """8 rows of x, each a one-hot row picking one column of the weight: every output is
+    1 * w plus exact zeros, so it must be the oracle's dequantized weight bit for bit (up to
+    the sign of a zero sum), for random code and scale bytes."""
+    rng = np.random.default_rng(K + N)
+    packed = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    scales = rng.integers(0, 256, size=(N, K // 16), dtype=np.uint8)
+    scales[(scales & 0x7F) == 0x7F] = 0x3C  # NaN bytes are outside the method
+    gs = 7168.0
+    tiled = nv.nvfp4_w4a16_pack(to_dev_u8(packed), to_dev_u8(scales))
+    cols = rng.choice(K, size=8, replace=False)
+    x = np.zeros((8, K), dtype=np.float32)
+    x[np.arange(8), cols] = 1.0
+    y = bits(nv.nvfp4_w4a16_linear(to_dev(synthetic.to_bf16_bits(x)), tiled, torch.tensor([gs], device="cuda"), N))
+    want = oracle.dequantize(packed, scales, gs, N, K)[:, cols].T
+    y = np.where((y & 0x7FFF) == 0, 0, y)
+    want = np.where((want & 0x7FFF) == 0, 0, want)
+    bad = np.argwhere(y != want)
+    assert bad.size == 0, f"{len(bad)} decoded weights differ, first {bad[:3].tolist()}"
+
+
 def test_empty_rows_launch_nothing():
     packed, scales, gs = _weight(32, 64, 11)
     x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
@@ -196,9 +244,9 @@ def test_empty_rows_launch_nothing():
     assert nv.nvfp4_kernel_launch_count() == before
 
 
-@pytest.mark.parametrize("M,K", [(1, 4096), (16, 4096), (32, 4096), (33, 4096), (100, 4096), (16, 1088), (7, 4160)])
+@pytest.mark.parametrize("M,K", [(9, 4096), (16, 4096), (32, 4096), (33, 4096), (100, 4096), (16, 1088), (9, 4160)])
 def test_split_k_for_few_rows(M, K):
-    """Up to 128 rows of x on a weight with few output tiles (4096 x 4096: 32 tiles) the call
+    """9 to 128 rows of x on a weight with few output tiles (4096 x 4096: 32 tiles): the call
     splits K over several CTAs when the workspace is large enough; the result is within the
     bound, bit-identical from call to call (the partial sums are added in a fixed order),
     and the workspace can be reused.  Without the room to split, the same call runs
