@@ -313,6 +313,23 @@ def test_w4a16_plan_refusals(lib):
     assert f(16, 4096, 4096, 256, 148, None, ctypes.byref(r), ctypes.byref(s)) == ERR_NULL
 
 
+def test_w4a16_workspace_sizes(lib):
+    """Host-only (148 SMs assumed without a GPU): the status block alone unless the plan
+    splits K; with a split, the block, one counter per 128-column tile (rounded up to 256
+    bytes) and splits x tiles x 128 x 128 fp32 partial sums."""
+    f = lib.nvfp4_w4a16_workspace_bytes
+    f.restype = ctypes.c_int64
+    f.argtypes = [ctypes.c_int64] * 3
+    assert f(1, 4096, 4096) == 256          # CUDA cores: never split
+    assert f(8, 4096, 4096) == 256
+    assert f(200, 4096, 4096) == 256        # tensor memory: never split
+    assert f(16, 14336, 4096) == 256        # 112 tiles: 148 // 112 = 1 CTA per tile
+    tiles = 32                              # 4096 outputs; 148 // 32 = 4 splits, K has 64 atoms
+    assert f(16, 4096, 4096) == -(-(256 + 4 * tiles) // 256) * 256 + 4 * tiles * 128 * 128 * 4
+    assert f(16, 4096, 1088) == -(-(256 + 4 * tiles) // 256) * 256 + 2 * tiles * 128 * 128 * 4  # 17 atoms: 2
+    assert f(16, 4096, 24) == -1 and f(-1, 4096, 64) == -1
+
+
 def test_w4a16_record_sizes(lib):
     """Host-only: ceil(N / 128) * ceil(K / 64) records of 4608 bytes; refused shapes -> -1."""
     f = lib.nvfp4_w4a16_tiled_bytes
