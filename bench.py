@@ -602,7 +602,7 @@ def run_linear(args):
     hbm, hbm_src = hbm_peak()
     tc, tc_src = bf16_peak()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    ws = nv.new_workspace(dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
 
     def timed(fn, reps=15):
         for _ in range(3):
@@ -628,6 +628,8 @@ def run_linear(args):
             x = synthetic.activation_normal_device((M, K), 8 + M, dev)
             y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
             lws = nv.nvfp4_w4a16_workspace(M, N, K, dev)
+            where, tile_rows, splits = nv.nvfp4_w4a16_plan(M, N, K, lws.numel(), sms)
+            kernel = f"{where} {tile_rows}" + (f" x{splits} K" if splits > 1 else "")
             t_fused = timed(lambda: nv.nvfp4_w4a16_linear(x, tiled, gs, N, out=y, workspace=lws))
             t_pages = timed(lambda: (nv.nvfp4_dequantize(packed, scales, gs, out=wbuf), torch.matmul(x, wbuf.t(), out=y)))
             t_bf16 = timed(lambda: torch.matmul(x, w.t(), out=y))
@@ -646,18 +648,18 @@ def run_linear(args):
                          "TFLOP/s": flops / t_fused / 1e12, "GB/s": nbytes / t_fused / 1e9,
                          "bound": "tensor" if flops / (tc * 1e12) >= nbytes / (hbm * 1e9) else "hbm",
                          "frac": ideal / t_fused, "dequant_then_linear_us": t_pages * 1e6,
-                         "bf16_linear_us": t_bf16 * 1e6})
+                         "bf16_linear_us": t_bf16 * 1e6, "kernel": kernel})
             del x, y
         del w, packed, scales, tiled, wbuf
     print(f"bf16 peak {tc:.1f} TFLOP/s ({tc_src}); HBM peak {hbm:.1f} GB/s ({hbm_src})")
     print("| weight | tokens | W4A16 us | TFLOP/s | GB/s | bound | frac of roofline | dequantize + linear us "
-          "| bf16 linear (unquantized weight) us | CPU oracle us (1 thread) |")
-    print("|---|---|---|---|---|---|---|---|---|---|")
+          "| bf16 linear (unquantized weight) us | CPU oracle us (1 thread) | kernel (weight in, rows of x per tile, K split) |")
+    print("|---|---|---|---|---|---|---|---|---|---|---|")
     for r in rows:
         cpu = f"{r['oracle_cpu_us']:.0f}" if r["oracle_cpu_us"] is not None else ""
         print(f"| {r['weight'][0]}x{r['weight'][1]} | {r['tokens']} | {r['fused_us']:.1f} | {r['TFLOP/s']:.0f} | "
               f"{r['GB/s']:.0f} | {r['bound']} | {r['frac']:.2f} | {r['dequant_then_linear_us']:.1f} | "
-              f"{r['bf16_linear_us']:.1f} | {cpu} |")
+              f"{r['bf16_linear_us']:.1f} | {cpu} | {r['kernel']} |")
     with open(args.linear, "w") as f:
         json.dump({"bf16_tflops": tc, "hbm_gbs": hbm, "rows": rows}, f, indent=1)
     return 0
