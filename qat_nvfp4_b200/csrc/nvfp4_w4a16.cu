@@ -4,18 +4,21 @@
 // _float4_autocast_forward: the packed weight is unpacked for one forward and the layer's
 // own bf16 forward runs on it).
 //
-// Kernels on the sm_100a tensor cores (tcgen05, kind::f16, bf16 operands, fp32 accumulators
-// in tensor memory).  The bf16 weight is never written to HBM.  The weight is read in a
-// tile-major copy of its packed form (nvfp4_w4a16_pack: one contiguous 4608-byte record per
-// 128-row x 64-column tile, codes then scale bytes), and decoded by the kernel's own warps
-// with the same arithmetic as nvfp4_dequantize, bf16_rn(fl(LUT[code] * fl(E4M3(byte) / gs))).
+// Two kernels on the sm_100a tensor cores (tcgen05, kind::f16, bf16 operands, fp32
+// accumulators in tensor memory), and one on the CUDA cores for up to 8 rows of x
+// (w4a16_gemv_kernel, below; make_plan routes a call).  The bf16 weight is never written to
+// HBM.  The weight is read in a tile-major copy of its packed form (nvfp4_w4a16_pack: one
+// contiguous 4608-byte record per 128-row x 64-column tile, codes then scale bytes), and
+// decoded by the kernels' own warps with the same arithmetic as nvfp4_dequantize,
+// bf16_rn(fl(LUT[code] * fl(E4M3(byte) / gs))).
 //
+// The tensor-core kernels' warps:
 //   warps 0-15 decode weight rows, 32 rows per warp, then the epilogue
 //              (TMEM -> fp32 + bias -> bf16)
 //   warp 16    TMA loads of activation tiles
 //   warp 17    TMEM allocation, MMA issue (one elected thread), TMEM release
 //
-// w4a16_linear_kernel (up to 128 rows of x with K split over several CTAs per tile, and up
+// w4a16_linear_kernel (up to 128 rows of x with K split over several CTAs per tile, and 9
 // to 32 rows unsplit): x is the MMA's A operand, the decoded weight tile the B operand in
 // shared memory (128-byte swizzle, K-major), passed from the decode warps to the MMAs
 // through a ring of 2 or 3 tiles.  w4a16_linear_ts_kernel (everything else): the decoded
