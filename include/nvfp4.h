@@ -352,7 +352,7 @@ nvfp4_status nvfp4_w4a16_pack(const uint8_t* packed, const uint8_t* scales, int6
  * forward and runs the layer's bf16 forward on it.  One kernel on the tensor cores (bf16 x
  * bf16, fp32 accumulation, output rounded to bf16 once; the bias is added to the fp32 sum
  * before that rounding); the decoded weight is built tile by tile on chip (in tensor
- * memory, or in shared memory for up to 32 rows of x and whenever K is split; in registers,
+ * memory, or in shared memory for 9 to 32 rows of x and whenever K is split; in registers,
  * with fp32 FMAs on the CUDA cores, for up to 8 rows) and never written to device memory.
  * Each weight element is decoded exactly as
  * nvfp4_dequantize does; the sum is not bit-reproducible against another GEMM (the order
@@ -400,7 +400,7 @@ int64_t nvfp4_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * device with `sms` SMs (the decision that call takes with the current device's SM count).
  * Host only: launches nothing and needs no GPU.
  *   *kernel         2: the CUDA cores, no tensor cores (at most 8 rows of x); 0: the weight
- *                   decoded into shared memory (split K, or at most 32 rows of x); 1: the
+ *                   decoded into shared memory (split K, or 9 to 32 rows of x); 1: the
  *                   weight decoded into tensor memory (everything else)
  *   *rows_per_tile  rows of x per output tile: for kernel 2, M rounded up to 1, 2, 4 or 8
  *                   (tiles of 32 weight rows); 128 for kernel 0; for kernel 1, 64 or 128 up to
