@@ -198,12 +198,16 @@ nvfp4_status nvfp4_selftest_barrier_timeout(const void* x, void* y, int64_t M, i
  *     return NVFP4_ERR_ARG.
  *   - Nothing is allocated: no cudaMalloc / cudaFree, no allocating library routine.
  *   - The first call on each device looks up that device's copy of the array
- *     (cudaGetSymbolAddress, with the device current); make that first call before any
- *     stream capture.
- *   - Every call on a device shares the one array: each call clears it (a memset on
- *     `stream`) before its kernel, and calls that overlap on the GPU (different streams)
- *     race with each other.  Use nvfp4_observe_amax_ws with one workspace per stream for
- *     concurrent calls.
+ *     (cudaGetSymbolAddress, with the device current) and keeps the address for later
+ *     calls; make that first call before any stream capture.  The kept address belongs to
+ *     the device's context at that time: do not call cudaDeviceReset (or otherwise tear
+ *     down and recreate the device's primary context) in a process that has used this
+ *     call, or later calls would pass a stale address.
+ *   - Every call on a device shares the one array.  The kernel leaves it zeroed when it
+ *     completes, but calls that overlap on the GPU (different streams) race with each
+ *     other and can leave it dirty; so each call also clears it first (a memset on
+ *     `stream`), which makes the next non-overlapping call correct again.  Use
+ *     nvfp4_observe_amax_ws with one workspace per stream for concurrent calls.
  * Arguments, results and other errors are those of nvfp4_observe_amax. */
 nvfp4_status nvfp4_observe_amax_noalloc(const void* x, int64_t numel, float* d_state, nvfp4_observer kind,
                                         double decay, float* d_cur_amax, nvfp4_stream_t stream);
@@ -280,7 +284,9 @@ nvfp4_status nvfp4_fake_quant(const void* x, void* y, int64_t M, int64_t N, cons
  *   k       1 .. NVFP4_MAX_SIBLINGS
  *   d_shared_amax  fp32 out: the shared amax that was used
  * Enqueues a memset and two kernels (one amax launch and one fake-quant launch over all
- * k tensors). */
+ * k tensors).  The count k comes first on purpose, ahead of the arrays whose length it
+ * gives (a sketch of this call elsewhere puts it after the size arrays); the arguments
+ * are otherwise in the same order. */
 nvfp4_status nvfp4_fake_quant_siblings(int k, const void* const* xs, void* const* ys, const int64_t* Ms,
                                        const int64_t* Ns, float* d_shared_amax, nvfp4_stream_t stream);
 

@@ -20,7 +20,7 @@
  *             FP4 fake-quant kernel), section 2 (STE), section 4 (weight fake-quant with
  *             fusion), section 5 (activation observers).
  *
- * Readings where the pages are silent or ambiguous (each is listed in the design doc):
+ * Readings where the pages are silent or ambiguous:
  *   - the per-tensor scale 2688/amax is one IEEE division;
  *   - the E4M3 cast rounds to nearest-even and saturates to +-448 (no NaN);
  *   - fake-quant is dequantize(quantize(x)) with [FP4OPT]'s formulas;

@@ -495,7 +495,9 @@ NVFP4_API nvfp4_status nvfp4_observe_amax_noalloc(const void* x, int64_t numel, 
         }
         scratch = g_noalloc_ptr[dev];
     }
-    // The array keeps whatever the previous call left; the kernel needs it zeroed.
+    // The kernel leaves the array zeroed when it completes, but two calls that overlapped
+    // on the GPU can leave it dirty (their CTAs share the arrival counter); clearing it first
+    // makes every call that does not overlap another one correct again.
     if (cudaMemsetAsync(scratch, 0, need, cs(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
     return launch_amax_ws(L, d_cur_amax, scratch, d_state, (int)kind, keep, take, stream);
 }

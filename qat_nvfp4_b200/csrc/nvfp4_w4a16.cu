@@ -1070,8 +1070,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // w + 8, ... of K, each lane one weight row.  Per atom a lane reads its row's 32 code bytes
 // and scale word (a warp reads 1 KB and 128 bytes, each contiguous; the next atom's are
 // loaded before the current one is used), decodes them exactly as nvfp4_dequantize does,
-// and accumulates x[m][k] w[k] for the rows of x in fp32: a product of two bf16 values is
-// exact in fp32, and k and k + 1 go to the two halves of one packed f32x2 FMA.  The halves,
+// and accumulates x[m][k] w[k] for the rows of x in fp32: each step is one fused
+// multiply-add with a single rounding, and k and k + 1 go to the two halves of one packed
+// f32x2 FMA.  The halves,
 // then the 8 warps' partial sums (in warp order) are added in shared memory, then the bias,
 // then one rounding to bf16.
 

@@ -191,6 +191,8 @@ def test_out_parameter_and_leading_dimensions():
     (2, 1040, 200, True),     # K % 64 == 16: the last atom has one block
     (3, 64, 300, True),       # one atom of K: seven of the eight warps have none
     (4, 16, 13, False),       # one block of K, 13 live rows of one 32-row tile
+    (5, 1040, 333, True),     # 5 and 6 rows: the 8-row instance with 3 and 2 rows idle,
+    (6, 4112, 77, False),     # N not a multiple of 32, K % 64 != 0
     (7, 4160, 1000, True),
     (8, 1088, 128, False),
     (8, 4096, 14336, True),   # the pages' MLP weight
