@@ -1,7 +1,12 @@
 """Helpers shared by the GPU tests: moving bf16 bit patterns to and from the device and
 comparing the library's outputs with the oracle's, with a readable failure message."""
+import os
+
 import numpy as np
 import torch
+
+# Threads for the oracle's row ranges: every host core this process may run on.
+HOST_THREADS = max(1, len(os.sched_getaffinity(0)))
 
 
 def to_dev(bits: np.ndarray, device="cuda") -> torch.Tensor:
@@ -56,9 +61,10 @@ def _row_chunks(M, parts):
     return [(r, min(M, r + step)) for r in range(0, M, step)]
 
 
-def oracle_quantize_rows(x_bits, gs, threads=8, block=16):
+def oracle_quantize_rows(x_bits, gs, threads=None, block=16):
     import oracle
     from concurrent.futures import ThreadPoolExecutor
+    threads = threads or HOST_THREADS
     M, N = x_bits.shape
     B = (N + block - 1) // block  # rows are zero-padded to block * B columns
     packed = np.empty((M, block // 2 * B), dtype=np.uint8)
@@ -73,9 +79,10 @@ def oracle_quantize_rows(x_bits, gs, threads=8, block=16):
     return packed, scales
 
 
-def oracle_fake_quant_rows(x_bits, amax, threads=8, block=16):
+def oracle_fake_quant_rows(x_bits, amax, threads=None, block=16):
     import oracle
     from concurrent.futures import ThreadPoolExecutor
+    threads = threads or HOST_THREADS
     M, N = x_bits.shape
     y = np.empty((M, N), dtype=np.uint16)
 
@@ -87,9 +94,10 @@ def oracle_fake_quant_rows(x_bits, amax, threads=8, block=16):
     return y
 
 
-def oracle_dequantize_rows(packed, scales, gs, threads=8, n_cols=None, block=16):
+def oracle_dequantize_rows(packed, scales, gs, threads=None, n_cols=None, block=16):
     import oracle
     from concurrent.futures import ThreadPoolExecutor
+    threads = threads or HOST_THREADS
     M = packed.shape[0]
     N = packed.shape[1] * 2 if n_cols is None else n_cols
     y = np.empty((M, N), dtype=np.uint16)
@@ -100,10 +108,3 @@ def oracle_dequantize_rows(packed, scales, gs, threads=8, n_cols=None, block=16)
     with ThreadPoolExecutor(threads) as pool:
         list(pool.map(work, _row_chunks(M, threads * 2)))
     return y
-
-
-def sample_rows(M, n=48, seed=0):
-    rng = np.random.default_rng(seed)
-    rows = {0, M - 1, M // 2}
-    rows |= set(int(r) for r in rng.choice(M, size=min(n, M), replace=False))
-    return np.array(sorted(rows))

@@ -14,7 +14,7 @@ import torch
 import oracle
 from qat_nvfp4_b200 import synthetic
 from nvfp4_testutil import (assert_equal_bits, bits, f32_bits, oracle_dequantize_rows, oracle_fake_quant_rows,
-                            oracle_quantize_rows, sample_rows, scalar, to_dev, u8, u8_to_dev)
+                            oracle_quantize_rows, scalar, to_dev, u8, u8_to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -81,8 +81,8 @@ def test_weight_with_outliers():
 
 def test_w4a4_observers_16_steps():
     """16 steps of activations with static_minmax and EMA(0.01) observers starting unset
-    (-1); each step's fake-quant uses the updated state.  States are compared every step,
-    outputs on the whole tensor at steps 0 and 15 and on sampled rows otherwise."""
+    (-1); each step's fake-quant uses the updated state.  States and every output element
+    are compared at every step."""
     kinds = {"static_minmax": oracle.STATIC_MINMAX, "minmax": oracle.EMA}
     states_d = {k: scalar(-1.0) for k in kinds}
     states = {k: -1.0 for k in kinds}
@@ -90,23 +90,17 @@ def test_w4a4_observers_16_steps():
         x = synthetic.activation_student_t(step)
         xd = to_dev(x)
         cur = oracle.amax(x)
-        rows = slice(None) if step in (0, 15) else sample_rows(x.shape[0], 32, seed=step)
         for name, kind in kinds.items():
             cur_d = nv.nvfp4_observe_amax(xd, states_d[name], kind=name, decay=0.01)
             states[name] = oracle.observer_update(states[name], cur, kind, 0.01)
             assert f32_bits(cur_d) == f32_bits(cur), f"step {step} {name}: current amax"
             assert f32_bits(states_d[name]) == f32_bits(states[name]), f"step {step} {name}: state"
             fq = bits(nv.nvfp4_fake_quant(xd, states_d[name]))
-            want = oracle_fake_quant_rows(x[rows], states[name])
-            assert_equal_bits(fq[rows], want, f"step {step} {name}: fake-quant")
-    # the MLP weight next to the activations, with its own amax
+            want = oracle_fake_quant_rows(x, states[name])
+            assert_equal_bits(fq, want, f"step {step} {name}: fake-quant")
+    # the MLP weight next to the activations, with its own amax: every output
     w = synthetic.large_weight()
-    wd = to_dev(w)
-    a = nv.nvfp4_amax(wd)
-    assert f32_bits(a) == f32_bits(oracle.amax(w))
-    rows = sample_rows(w.shape[0], 64, seed=99)
-    assert_equal_bits(bits(nv.nvfp4_fake_quant(wd, a))[rows], oracle_fake_quant_rows(w[rows], a.item()),
-                      "14336x4096 weight fake-quant")
+    _full_check(w, what="14336x4096 MLP weight")
 
 
 def test_qkv_siblings_shared_amax():
@@ -133,26 +127,12 @@ def test_qkv_siblings_shared_amax():
 
 @pytest.mark.parametrize("size_index", range(len(synthetic.SWEEP_SHAPES)))
 def test_activation_size_sweep(size_index):
+    """Every size up to 65536 x 8192 (1 GiB): amax, global scale, every code byte, scale
+    byte, dequantized and fake-quantized element against the oracle (run over row ranges on
+    all host cores)."""
     M, N = synthetic.SWEEP_SHAPES[size_index]
     x = synthetic.activation_normal((M, N), synthetic.sweep_seed(size_index))
-    if M * N <= 4096 * 4096:
-        _full_check(x, what=f"{M}x{N}")
-        return
-    # large sizes: amax over the whole tensor, every output on sampled rows
-    xd = to_dev(x)
-    amax_d = nv.nvfp4_amax(xd)
-    a = oracle.amax(x)
-    assert f32_bits(amax_d) == f32_bits(a)
-    gs = oracle.global_scale(a)
-    rows = sample_rows(M, 64, seed=size_index)
-    packed_d, scales_d, gs_d = nv.nvfp4_quantize(xd, amax_d)
-    packed, scales = oracle_quantize_rows(x[rows], gs)
-    assert_equal_bits(u8(packed_d)[rows], packed, f"{M}x{N}: packed")
-    assert_equal_bits(u8(scales_d)[rows], scales, f"{M}x{N}: scales")
-    y = oracle_dequantize_rows(packed, scales, gs)
-    assert_equal_bits(bits(nv.nvfp4_dequantize(packed_d, scales_d, gs_d))[rows], y, f"{M}x{N}: dequantize")
-    del packed_d, scales_d
-    assert_equal_bits(bits(nv.nvfp4_fake_quant(xd, amax_d))[rows], y, f"{M}x{N}: fake-quant")
+    _full_check(x, what=f"{M}x{N}")
 
 
 # ---- adversarial inputs -----------------------------------------------------------------

@@ -20,7 +20,7 @@ import torch
 
 import oracle
 from qat_nvfp4_b200 import synthetic
-from nvfp4_testutil import bits, sample_rows, to_dev, u8
+from nvfp4_testutil import bits, to_dev, u8
 from nvfp4_testutil import u8_to_dev as to_dev_u8
 
 pytestmark = pytest.mark.gpu
@@ -157,23 +157,22 @@ def test_linear_agrees_with_a_library_gemm_on_the_dequantized_weight():
     ours = _linear(x, packed, scales, gs, bias=bias)
     w = nv.nvfp4_dequantize(packed, scales, gs)
     ref = torch.nn.functional.linear(x, w, bias)
-    rows = sample_rows(M, 32, seed=1)
-    _assert_within_bound(bits(ours)[rows], bits(x)[rows], packed, scales, gs, bits(bias), "ours")
-    _assert_within_bound(bits(ref)[rows], bits(x)[rows], packed, scales, gs, bits(bias), "cuBLAS")
+    _assert_within_bound(bits(ours), bits(x), packed, scales, gs, bits(bias), "ours")
+    _assert_within_bound(bits(ref), bits(x), packed, scales, gs, bits(bias), "cuBLAS")
     d = (ours.float() - ref.float()).abs()
     ulp = torch.finfo(torch.bfloat16).eps * ref.float().abs().clamp_min(1e-30)
     assert (d <= ulp).float().mean().item() > 0.99
 
 
-def test_mlp_weight_4096_tokens_sampled_rows():
-    """The pages' MLP weight 14336 x 4096 N(0, 0.02) under 4096 tokens of N(0, 1)."""
+def test_mlp_weight_4096_tokens():
+    """The pages' MLP weight 14336 x 4096 N(0, 0.02) under 4096 tokens of N(0, 1): every
+    output element within the bound."""
     M, K, N = 4096, 4096, 14336
     x = synthetic.activation_normal_device((M, K), 31, "cuda")
     w = synthetic.activation_normal_device((N, K), 32, "cuda") * 0.02
     packed, scales, gs = nv.nvfp4_quantize(w, nv.nvfp4_amax(w))
     y = _linear(x, packed, scales, gs)
-    rows = sample_rows(M, 24, seed=3)
-    _assert_within_bound(bits(y)[rows], bits(x)[rows], packed, scales, gs, None, "MLP 4096 tokens")
+    _assert_within_bound(bits(y), bits(x), packed, scales, gs, None, "MLP 4096 tokens")
 
 
 def test_out_parameter_and_leading_dimensions():
