@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kThreads)
     stream_blocks<unroll_for<kW>(kUnrollQ), NVFP4_PIPE_Q != 0, BlockW<kW>>(
         nblk, [&](int64_t bi, BlockW<kW>& b) { ld_block_ro(x + bi * (4 * kW), b.w); },
         [&](int64_t bi, BlockW<kW>& b) {
-            uint32_t c[kW];
+            uint32_t c[kW / 4];
             float sd;
             const uint32_t s8 = encode_block(b.w, gs, tab, c, sd);
             st_codes<kW>(packed + bi * kW, c);
@@ -93,12 +93,8 @@ __global__ void __launch_bounds__(kThreads) fake_quant_kernel(FqList L, int64_t 
             ld_block(xp, sl.w);
         },
         [&](int64_t, FqSlot<kW>& sl) {
-            uint32_t c[kW];
-            float sd;
-            encode_block(sl.w, gs, tab, c, sd);
             uint32_t o[kW];
-#pragma unroll
-            for (int i = 0; i < kW; ++i) o[i] = decode_pair(c[i], sd);
+            fake_quant_block(sl.w, gs, tab, o);
             st_block(sl.y, o);
         },
         [&] { gs = build_scale_table(tab, d_amax); });
@@ -204,12 +200,8 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads)
         stream_sched<1, kUnrollFq, false, Block32>(
             nblk, [&](int64_t bi, Block32& b) { ld_b256_hint(x + bi * kBlockBytesIn, b.w, stream_out); },
             [&](int64_t bi, Block32& b) {
-                uint32_t c[8];
-                float sd;
-                encode_block(b.w, gs, tab, c, sd);
                 uint32_t o[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
+                fake_quant_block(b.w, gs, tab, o);
                 st_b256_hint(out.y + bi * kBlockBytesIn, o, stream_out);
             });
     } else {
@@ -217,10 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads)
         stream_sched<1, kUnrollFq, false, Block32>(
             nblk, [&](int64_t bi, Block32& b) { ld_b256_hint(x + bi * kBlockBytesIn, b.w, stream_out); },
             [&](int64_t bi, Block32& b) {
-                uint32_t c[8];
+                uint32_t c[2];
                 float sd;
                 const uint32_t s8 = encode_block(b.w, gs, tab, c, sd);
-                st_b64(out.packed + bi * kBlockBytesPacked, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
+                st_b64(out.packed + bi * kBlockBytesPacked, c[0], c[1]);
                 st_u8(out.scales + bi, s8);
             });
     }

@@ -92,14 +92,41 @@ nvfp4_status occupancy(const void* fn, int* out, size_t smem = 0) {
     return NVFP4_OK;
 }
 
+// Tensors of at most `small` work items (blocks) launch at most NVFP4_GRID_SMALL times the
+// resident CTAs instead of their kernel's own multiple: below a few hundred MB an
+// oversubscribed grid is many short-lived CTAs, each paying its set-up (the scale table,
+// the first load's latency, the end-of-CTA reduction) for one or two blocks per thread.
+// The thresholds are per kernel (measured on B200 with the ncu launch list): amax,
+// quantize and fake-quant up to 512 MiB of bf16 (at 256 MiB the pipelined fake-quant is
+// 8 % slower on its oversubscribed grid), dequantize never (its one-wave grid lost 5-9 %
+// at 32-112 MiB).
+#ifndef NVFP4_SMALL_AMAX
+#define NVFP4_SMALL_AMAX (int64_t(1) << 24)
+#endif
+#ifndef NVFP4_SMALL_Q
+#define NVFP4_SMALL_Q (int64_t(1) << 24)
+#endif
+#ifndef NVFP4_SMALL_FQ
+#define NVFP4_SMALL_FQ (int64_t(1) << 24)
+#endif
+#ifndef NVFP4_SMALL_DEC
+#define NVFP4_SMALL_DEC 0
+#endif
+#ifndef NVFP4_GRID_SMALL
+#define NVFP4_GRID_SMALL 1
+#endif
+
 // Grid: min(CTAs needed for `items` work items at `per_thread` each, `mult` times the
-// CTAs resident on the whole GPU at once; mult == 0 means no cap).
-nvfp4_status grid_for(const void* fn, int64_t items, int per_thread, int mult, int* grid, size_t smem = 0) {
+// CTAs resident on the whole GPU at once; mult == 0 means no cap; NVFP4_GRID_SMALL in
+// place of mult when items <= small).
+nvfp4_status grid_for(const void* fn, int64_t items, int per_thread, int mult, int* grid, size_t smem = 0,
+                      int64_t small = 0) {
     int sms = 0, occ = 0;
     nvfp4_status st = sm_count(&sms);
     if (st != NVFP4_OK) return st;
     st = occupancy(fn, &occ, smem);
     if (st != NVFP4_OK) return st;
+    if (items <= small && mult != 0) mult = NVFP4_GRID_SMALL;
     const int64_t per_cta = (int64_t)kThreads * per_thread;
     const int64_t need = (items + per_cta - 1) / per_cta;
     const int64_t cap = mult > 0 ? (int64_t)sms * occ * mult : need;
@@ -188,7 +215,7 @@ template <int kA>
 nvfp4_status launch_quantize_rows(const void* x, const RaggedRows& H, const float* d_amax, uint8_t* packed,
                                   uint8_t* scales, float* d_gs, nvfp4_stream_t stream) {
     int grid = 1;
-    nvfp4_status st = grid_for(reinterpret_cast<const void*>(&quantize_rows_kernel<kA>), H.total, kUnrollQ,
+    nvfp4_status st = grid_for(reinterpret_cast<const void*>(&quantize_rows_kernel<kA>), H.total, kUnrollQView,
                                NVFP4_GRID_Q, &grid);
     if (st != NVFP4_OK) return st;
     quantize_rows_kernel<kA><<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), H, d_amax, packed,
@@ -243,7 +270,8 @@ nvfp4_status launch_amax(const AmaxList& L, float* d_amax, nvfp4_stream_t stream
     if (!accumulate && cudaMemsetAsync(d_amax, 0, sizeof(float), cs(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
     const int64_t units = L.full_end[L.k - 1];
     int grid = 1;
-    nvfp4_status st = grid_for(reinterpret_cast<const void*>(&amax_kernel), units, kUnrollAmax, NVFP4_GRID_AMAX, &grid);
+    nvfp4_status st = grid_for(reinterpret_cast<const void*>(&amax_kernel), units, kUnrollAmax, NVFP4_GRID_AMAX, &grid, 0,
+                                NVFP4_SMALL_AMAX);
     if (st != NVFP4_OK) return st;
     amax_kernel<<<grid, kThreads, 0, cs(stream)>>>(L, units, reinterpret_cast<unsigned*>(d_amax));
     return after_launch();
@@ -256,11 +284,13 @@ nvfp4_status launch_amax_ws(const AmaxList& L, float* d_amax, void* d_ws, float*
     Workspace* ws = static_cast<Workspace*>(d_ws);
     int grid = 1;
     if (state == nullptr) {
-        nvfp4_status st = grid_for(reinterpret_cast<const void*>(&amax_ws_kernel<false>), units, kUnrollAmax, NVFP4_GRID_AMAX, &grid);
+        nvfp4_status st = grid_for(reinterpret_cast<const void*>(&amax_ws_kernel<false>), units, kUnrollAmax, NVFP4_GRID_AMAX,
+                                   &grid, 0, NVFP4_SMALL_AMAX);
         if (st != NVFP4_OK) return st;
         amax_ws_kernel<false><<<grid, kThreads, 0, cs(stream)>>>(L, units, ws, d_amax, nullptr, 0, 0.f, 0.f);
     } else {
-        nvfp4_status st = grid_for(reinterpret_cast<const void*>(&amax_ws_kernel<true>), units, kUnrollAmax, NVFP4_GRID_AMAX, &grid);
+        nvfp4_status st = grid_for(reinterpret_cast<const void*>(&amax_ws_kernel<true>), units, kUnrollAmax, NVFP4_GRID_AMAX,
+                                   &grid, 0, NVFP4_SMALL_AMAX);
         if (st != NVFP4_OK) return st;
         amax_ws_kernel<true><<<grid, kThreads, 0, cs(stream)>>>(L, units, ws, d_amax, state, kind, keep, take);
     }
@@ -552,7 +582,8 @@ static nvfp4_status fake_quant_auto(const void* x, void* y, int64_t M, int64_t N
     F.y[0] = static_cast<uint8_t*>(y);
     F.blk_end[0] = nblk;
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<false, 8>), nblk, kUnrollFq, NVFP4_GRID_FQ, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<false, 8>), nblk, kUnrollFq, NVFP4_GRID_FQ, &grid, 0,
+                  NVFP4_SMALL_FQ);
     if (st != NVFP4_OK) return st;
     fake_quant_kernel<false, 8><<<grid, kThreads, 0, cs(stream)>>>(F, nblk, state ? state : d_amax_out);
     return after_launch();
@@ -649,7 +680,7 @@ static nvfp4_status quantize_impl(const void* x, int64_t M, int64_t N, const flo
     if (nblk == 0 && d_global_scale == nullptr) return NVFP4_OK;
     int grid = 1;
     st = grid_for(reinterpret_cast<const void*>(&quantize_kernel<kMma, kW>), nblk, unroll_for<kW>(kUnrollQ),
-                  NVFP4_GRID_Q, &grid);
+                  NVFP4_GRID_Q, &grid, 0, NVFP4_SMALL_Q);
     if (st != NVFP4_OK) return st;
     quantize_kernel<kMma, kW><<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), nblk, d_amax, packed,
                                                                  scales, d_global_scale, R.nb > 0 ? R.nb : 1, ncb);
@@ -691,7 +722,7 @@ static nvfp4_status dequantize_impl(const uint8_t* packed, const uint8_t* scales
     if (nblk == 0) return NVFP4_OK;
     int grid = 1;
     st = grid_for(reinterpret_cast<const void*>(&dequantize_kernel<kW>), nblk, unroll_for<kW>(kUnrollDecode),
-                  NVFP4_GRID_DEC, &grid);
+                  NVFP4_GRID_DEC, &grid, 0, NVFP4_SMALL_DEC);
     if (st != NVFP4_OK) return st;
     dequantize_kernel<kW><<<grid, kThreads, 0, cs(stream)>>>(packed, scales, d_global_scale, static_cast<uint8_t*>(y),
                                                              nblk);
@@ -721,7 +752,7 @@ static nvfp4_status fake_quant_impl(const void* x, void* y, int64_t M, int64_t N
     L.blk_end[0] = nblk;
     int grid = 1;
     st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<false, kW>), nblk, unroll_for<kW>(kUnrollFq),
-                  NVFP4_GRID_FQ, &grid);
+                  NVFP4_GRID_FQ, &grid, 0, NVFP4_SMALL_FQ);
     if (st != NVFP4_OK) return st;
     fake_quant_kernel<false, kW><<<grid, kThreads, 0, cs(stream)>>>(L, nblk, d_amax);
     return after_launch();
@@ -754,7 +785,8 @@ NVFP4_API nvfp4_status nvfp4_amax_strided(const void* x, int64_t M, int64_t N, i
     if (cudaMemsetAsync(d_amax, 0, sizeof(float), cs(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (S.total == 0) return NVFP4_OK;
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&amax_strided_kernel), S.total, kUnrollAmax, NVFP4_GRID_AMAX, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&amax_strided_kernel), S.total, kUnrollAmax, NVFP4_GRID_AMAX, &grid, 0,
+                  NVFP4_SMALL_AMAX);
     if (st != NVFP4_OK) return st;
     amax_strided_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), S,
                                                            reinterpret_cast<unsigned*>(d_amax));
@@ -774,7 +806,8 @@ NVFP4_API nvfp4_status nvfp4_quantize_strided(const void* x, int64_t M, int64_t 
     if (S.total > 0 && (!aligned(x, 32) || !aligned(packed, 8))) return NVFP4_ERR_ALIGN;
     if (S.total == 0 && d_global_scale == nullptr) return NVFP4_OK;
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&quantize_strided_kernel), S.total, kUnrollQ, NVFP4_GRID_Q, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&quantize_strided_kernel), S.total, kUnrollQView, NVFP4_GRID_Q, &grid, 0,
+                  NVFP4_SMALL_Q);
     if (st != NVFP4_OK) return st;
     quantize_strided_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), S, d_amax, packed,
                                                                scales, d_global_scale);
@@ -799,7 +832,8 @@ NVFP4_API nvfp4_status nvfp4_fake_quant_strided(const void* x, int64_t ldx, void
         if (px < py + (uintptr_t)(span_y * 2) && py < px + (uintptr_t)(span * 2)) return NVFP4_ERR_ARG;
     }
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&fake_quant_strided_kernel), S.total, kUnrollFq, NVFP4_GRID_FQ, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&fake_quant_strided_kernel), S.total, kUnrollFq, NVFP4_GRID_FQ, &grid, 0,
+                  NVFP4_SMALL_FQ);
     if (st != NVFP4_OK) return st;
     fake_quant_strided_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), S,
                                                                  static_cast<uint8_t*>(y), ldy * 2, d_amax);
@@ -926,7 +960,8 @@ NVFP4_API nvfp4_status nvfp4_fake_quant_siblings(int k, const void* const* xs, v
     const int64_t nblk = acc;
     if (nblk == 0) return NVFP4_OK;
     int grid = 1;
-    st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<true, 8>), nblk, kUnrollFq, NVFP4_GRID_FQ, &grid);
+    st = grid_for(reinterpret_cast<const void*>(&fake_quant_kernel<true, 8>), nblk, kUnrollFq, NVFP4_GRID_FQ, &grid, 0,
+                  NVFP4_SMALL_FQ);
     if (st != NVFP4_OK) return st;
     fake_quant_kernel<true, 8><<<grid, kThreads, 0, cs(stream)>>>(F, nblk, d_shared_amax);
     return after_launch();

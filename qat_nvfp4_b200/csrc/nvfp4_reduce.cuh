@@ -73,18 +73,22 @@ __global__ void observer_kernel(float* state, const float* cur, int kind, float 
 
 // ---------------------------------------------------------------------------------------
 // Single-launch amax (and observer step) with a workspace.  Every CTA folds its maximum
-// into ws->acc with atomicMax and then counts itself in ws->arrived; the CTA that
-// arrives last has seen every other CTA's atomicMax land (each CTA fences between its
-// two atomics), so it publishes the amax, applies the observer step if asked, and puts
-// the workspace back to zero for the next call.  No CTA ever waits for another.
-
-
+// into ws->acc with an atomic max and then counts itself in ws->arrived; the CTA that
+// arrives last has seen every other CTA's maximum land, so it publishes the amax, applies
+// the observer step if asked, and puts the workspace back to zero for the next call.  No
+// CTA ever waits for another.
+// The CTA's maximum goes out as a reduction that returns nothing; the arrival is one
+// acquire-release add, which orders that reduction before the arrival and, in the last CTA,
+// every other CTA's reduction before what it reads next (the adds on the counter form one
+// release sequence), so no separate fence is needed on either side.
 __device__ __forceinline__ bool last_to_arrive(Workspace* ws, float cta_amax) {
     __shared__ bool last;
     if (threadIdx.x == 0) {
-        atomicMax(&ws->acc, __float_as_uint(cta_amax));
-        __threadfence();
-        last = atomicAdd(&ws->arrived, 1u) == gridDim.x - 1;
+        asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(&ws->acc), "r"(__float_as_uint(cta_amax))
+                     : "memory");
+        unsigned before;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(before) : "l"(&ws->arrived) : "memory");
+        last = before == gridDim.x - 1;
     }
     __syncthreads();
     return last;
@@ -96,7 +100,6 @@ __global__ void __launch_bounds__(kThreads)
                    float take) {
     const float f = cta_max(thread_amax(L, total_units));
     if (last_to_arrive(ws, f) && threadIdx.x == 0) {
-        __threadfence();
         const float a = __uint_as_float(atomicExch(&ws->acc, 0u));
         atomicExch(&ws->arrived, 0u);
         *out = a;

@@ -24,7 +24,7 @@ namespace {
 #define NVFP4_U_FQ 2
 #endif
 #ifndef NVFP4_U_Q
-#define NVFP4_U_Q 1
+#define NVFP4_U_Q 2
 #endif
 #ifndef NVFP4_U_DEC
 #define NVFP4_U_DEC 2
@@ -44,10 +44,10 @@ namespace {
 // 1: register double buffering -- the loads of the next group of blocks are issued
 // before the current group is processed, so every thread always has loads in flight.
 #ifndef NVFP4_PIPE_FQ
-#define NVFP4_PIPE_FQ 0
+#define NVFP4_PIPE_FQ 1
 #endif
 #ifndef NVFP4_PIPE_Q
-#define NVFP4_PIPE_Q 0
+#define NVFP4_PIPE_Q 1
 #endif
 #ifndef NVFP4_PIPE_DEC
 #define NVFP4_PIPE_DEC 0
@@ -57,6 +57,15 @@ constexpr int kThreads = NVFP4_THREADS;
 constexpr int kUnrollAmax = NVFP4_U_AMAX;
 constexpr int kUnrollFq = NVFP4_U_FQ;
 constexpr int kUnrollQ = NVFP4_U_Q;
+// The row-view kernels (row-strided views, even-length rows by aligned accesses) keep their
+// own, measured shapes: quantize one block per thread per step, neither one pipelined.
+#ifndef NVFP4_U_Q_VIEW
+#define NVFP4_U_Q_VIEW 1
+#endif
+#ifndef NVFP4_PIPE_VIEW
+#define NVFP4_PIPE_VIEW 0
+#endif
+constexpr int kUnrollQView = NVFP4_U_Q_VIEW;
 constexpr int kUnrollDecode = NVFP4_U_DEC;
 static_assert(kThreads % 32 == 0 && kThreads <= 1024, "CTA size");
 
@@ -202,14 +211,13 @@ __host__ __device__ constexpr int unroll_for(int u16) {
     return kW == 8 ? u16 : (u16 / 2 > 0 ? u16 / 2 : 1);
 }
 
-// The packed codes of one block: kW bytes.
+// The packed codes of one block: kW bytes, as encode_block leaves them in kW / 4 words.
 template <int kW>
-__device__ __forceinline__ void st_codes(uint8_t* p, const uint32_t (&c)[kW]) {
+__device__ __forceinline__ void st_codes(uint8_t* p, const uint32_t (&c)[kW / 4]) {
     if constexpr (kW == 8) {
-        st_b64(p, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
+        st_b64(p, c[0], c[1]);
     } else {
-        st_b128(p, pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]), pack4(c[8], c[9], c[10], c[11]),
-                pack4(c[12], c[13], c[14], c[15]));
+        st_b128(p, c[0], c[1], c[2], c[3]);
     }
 }
 

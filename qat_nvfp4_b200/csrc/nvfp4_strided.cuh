@@ -79,10 +79,10 @@ __global__ void __launch_bounds__(kThreads)
     __shared__ float4 tab[128];
     float gs = 0.0f;
     const Div32 v = div32_of((uint32_t)S.nb);
-    stream_blocks<kUnrollQ, NVFP4_PIPE_Q != 0, Block32>(
+    stream_blocks<kUnrollQView, NVFP4_PIPE_VIEW != 0, Block32>(
         S.total, [&](int64_t g, Block32& b) { ld_block_ro(x + strided_offset(S, v, g), b.w); },
         [&](int64_t g, Block32& b) {
-            uint32_t c[8];
+            uint32_t c[2];
             float sd;
             const uint32_t s8 = encode_block(b.w, gs, tab, c, sd);
             st_codes<8>(packed + g * 8, c);
@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kThreads)
     __shared__ float4 tab[128];
     float gs = 0.0f;
     const Div32 v = div32_of((uint32_t)S.nb);
-    stream_blocks<kUnrollFq, NVFP4_PIPE_FQ != 0, FqSlot<8>>(
+    stream_blocks<kUnrollFq, NVFP4_PIPE_VIEW != 0, FqSlot<8>>(
         S.total,
         [&](int64_t g, FqSlot<8>& sl) {
             const int64_t r = strided_row(S, v, g);
@@ -110,12 +110,8 @@ __global__ void __launch_bounds__(kThreads)
             ld_block(x + r * S.ld_bytes + c, sl.w);
         },
         [&](int64_t, FqSlot<8>& sl) {
-            uint32_t c[8];
-            float sd;
-            encode_block(sl.w, gs, tab, c, sd);
             uint32_t o[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
+            fake_quant_block(sl.w, gs, tab, o);
             st_block(sl.y, o);
         },
         [&] { gs = build_scale_table(tab, d_amax); });
@@ -203,7 +199,7 @@ __global__ void __launch_bounds__(kThreads)
     __shared__ float4 tab[128];
     float gs = 0.0f;
     const Div32 v = div32_of((uint32_t)H.nb);
-    stream_blocks<kUnrollQ, NVFP4_PIPE_Q != 0, Block32>(
+    stream_blocks<kUnrollQView, NVFP4_PIPE_VIEW != 0, Block32>(
         H.total,
         [&](int64_t g, Block32& b) {
             int na;
@@ -211,7 +207,7 @@ __global__ void __launch_bounds__(kThreads)
             ld_ragged_block<kA, false>(x + r * H.ld_x + (g - r * H.nb) * kBlockBytesIn, na, b.w);
         },
         [&](int64_t g, Block32& b) {
-            uint32_t c[8];
+            uint32_t c[2];
             float sd;
             const uint32_t s8 = encode_block(b.w, gs, tab, c, sd);
             st_codes<8>(packed + g * 8, c);
@@ -230,7 +226,7 @@ __global__ void __launch_bounds__(kThreads)
     __shared__ float4 tab[128];
     float gs = 0.0f;
     const Div32 v = div32_of((uint32_t)H.nb);
-    stream_blocks<kUnrollFq, NVFP4_PIPE_FQ != 0, RaggedSlot>(
+    stream_blocks<kUnrollFq, NVFP4_PIPE_VIEW != 0, RaggedSlot>(
         H.total,
         [&](int64_t g, RaggedSlot& sl) {
             const int64_t r = ragged_row<kA>(H, v, g, sl.na);
@@ -239,12 +235,8 @@ __global__ void __launch_bounds__(kThreads)
             ld_ragged_block<kA, true>(x + r * H.ld_x + c, sl.na, sl.w);
         },
         [&](int64_t, RaggedSlot& sl) {
-            uint32_t c[8];
-            float sd;
-            encode_block(sl.w, gs, tab, c, sd);
             uint32_t o[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = decode_pair(c[i], sd);
+            fake_quant_block(sl.w, gs, tab, o);
             st_ragged_block<kA>(sl.y, sl.na, o);
         },
         [&] { gs = build_scale_table(tab, d_amax); });
