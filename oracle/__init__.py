@@ -64,6 +64,13 @@ def _lib():
         lib.oracle_dequantize_bs.restype = ctypes.c_int
         lib.oracle_fake_quant_bs.argtypes = [u16p, i64, i64, i64, f32, u16p]
         lib.oracle_fake_quant_bs.restype = ctypes.c_int
+        f32p = ctypes.POINTER(ctypes.c_float)
+        lib.oracle_quantize_f32scale.argtypes = [u16p, i64, i64, u8p, f32p]
+        lib.oracle_quantize_f32scale.restype = ctypes.c_int
+        lib.oracle_dequantize_f32scale.argtypes = [u8p, f32p, i64, i64, u16p]
+        lib.oracle_dequantize_f32scale.restype = None
+        lib.oracle_fake_quant_f32scale.argtypes = [u16p, i64, i64, u16p]
+        lib.oracle_fake_quant_f32scale.restype = ctypes.c_int
         lib.oracle_observer_update.argtypes = [f32, f32, ctypes.c_int, ctypes.c_double]
         lib.oracle_observer_update.restype = f32
         _LIB = lib
@@ -208,6 +215,42 @@ def w4a16_linear(x_bits, packed, scales, global_scale_value: float, n_out: int, 
     y = x @ w.T
     if bias_bits is not None:
         y = y + bf16_to_f64(np.asarray(bias_bits).reshape(1, n_out))
+    return y
+
+
+def quantize_f32scale(x_bits):
+    """The fp32-scale flavour with blocks of 32 (fp4_optimization.py, constants block):
+    bf16 bits [M, N] -> (packed uint8 [M, P/2], fp32 block scales [M, P/32]),
+    P = 32 ceil(N / 32)."""
+    x, xp = _u16(x_bits)
+    M, N = x.shape
+    B = padded_blocks(N, 32)
+    packed = np.empty((M, 16 * B), dtype=np.uint8)
+    scales = np.empty((M, B), dtype=np.float32)
+    rc = _lib().oracle_quantize_f32scale(xp, M, N, packed.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+                                         scales.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    if rc != 0:
+        raise MemoryError("oracle_quantize_f32scale")
+    return packed, scales
+
+
+def dequantize_f32scale(packed, scales, M: int, N: int):
+    """packed [M, P/2] + fp32 scales [M, P/32] -> bf16 bits [M, N]."""
+    p, pp = _u8(packed)
+    s = np.ascontiguousarray(scales, dtype=np.float32)
+    y = np.empty((M, N), dtype=np.uint16)
+    _lib().oracle_dequantize_f32scale(pp, s.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), M, N,
+                                      y.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)))
+    return y
+
+
+def fake_quant_f32scale(x_bits):
+    """dequantize_f32scale(quantize_f32scale(x)), bf16 bits [M, N] -> bf16 bits [M, N]."""
+    x, xp = _u16(x_bits)
+    M, N = x.shape
+    y = np.empty((M, N), dtype=np.uint16)
+    if _lib().oracle_fake_quant_f32scale(xp, M, N, y.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16))) != 0:
+        raise MemoryError("oracle_fake_quant_f32scale")
     return y
 
 

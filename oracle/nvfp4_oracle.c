@@ -285,6 +285,88 @@ ORACLE_API int oracle_fake_quant(const uint16_t* x, int64_t M, int64_t N, float 
     return oracle_fake_quant_bs(x, M, N, FLOAT4_BLOCK, amax, y);
 }
 
+/* ---- the fp32-scale flavour with blocks of 32 ------------------------------------------ */
+
+/* [FP4OPT] constants block, the FLOAT4_BLOCK_SIZE comment: NVFP4 scales 16-element blocks by
+ * an E4M3 byte plus one fp32 global scale per tensor, and blocks of 32 with an fp32 scale are
+ * the OCP MXFP4 flavour.  The pages define that flavour no further; the reading used here is
+ * quantize_weight_to_float4's steps with the scale kept in fp32 instead of being rounded to
+ * E4M3, so no per-tensor scale is needed:
+ *   block_amax  = max |x| over the 32 elements
+ *   block_scale = block_amax / 6                     (stored, fp32, one IEEE division)
+ *   divisor     = max(block_scale, 1e-12)            (the page's clamp against zero blocks)
+ *   scaled      = clamp(x / divisor, -6, 6), idx = _float4_round(|scaled|),
+ *   code        = idx + 8 if scaled < 0 else idx, packed as for NVFP4
+ * Rows are zero-padded to P = 32 ceil(N / 32) columns as the page pads them; packed is
+ * [M, P/2], scales [M, P/32] fp32.  Returns -1 if the row buffer cannot be allocated. */
+#define F32S_BLOCK 32
+
+ORACLE_API int oracle_quantize_f32scale(const uint16_t* x, int64_t M, int64_t N, uint8_t* packed, float* scales) {
+    int64_t nblk = (N + F32S_BLOCK - 1) / F32S_BLOCK;
+    int64_t P = nblk * F32S_BLOCK;
+    uint16_t* row = (uint16_t*)calloc((size_t)(P ? P : 1), sizeof(uint16_t)); /* zero padding */
+    if (!row) return -1;
+    for (int64_t r = 0; r < M; ++r) {
+        memcpy(row, x + r * N, (size_t)N * sizeof(uint16_t));
+        for (int64_t b = 0; b < nblk; ++b) {
+            const uint16_t* blk = row + b * F32S_BLOCK;
+            float block_amax = 0.0f;
+            for (int i = 0; i < F32S_BLOCK; ++i) {
+                float mag = fabsf(oracle_bf16_to_f32(blk[i]));
+                if (mag > block_amax) block_amax = mag;
+            }
+            float block_scale = block_amax / FLOAT4_MAX;
+            scales[r * nblk + b] = block_scale;
+            float divisor = block_scale < TINY_CLAMP ? TINY_CLAMP : block_scale;
+            uint8_t c32[F32S_BLOCK];
+            for (int i = 0; i < F32S_BLOCK; ++i) {
+                float q = oracle_bf16_to_f32(blk[i]) / divisor;
+                if (q < -FLOAT4_MAX) q = -FLOAT4_MAX;
+                if (q > FLOAT4_MAX) q = FLOAT4_MAX;
+                int idx = oracle_e2m1_round_index(fabsf(q));
+                c32[i] = (uint8_t)(q < 0.0f ? idx + 8 : idx);
+            }
+            uint8_t* out = packed + r * (P / 2) + b * (F32S_BLOCK / 2);
+            for (int j = 0; j < F32S_BLOCK / 2; ++j)
+                out[j] = (uint8_t)(c32[2 * j] | (c32[2 * j + 1] << 4));
+        }
+    }
+    free(row);
+    return 0;
+}
+
+/* The decode of the same flavour, as dequantize_weight_from_float4 with the stored fp32
+ * block scale in place of float(block_scale_fp8) / global_scale (no clamp on this side):
+ * bf16(LUT[code] * block_scale), cropped to the first N columns. */
+ORACLE_API void oracle_dequantize_f32scale(const uint8_t* packed, const float* scales, int64_t M, int64_t N,
+                                           uint16_t* y) {
+    int64_t nblk = (N + F32S_BLOCK - 1) / F32S_BLOCK;
+    int64_t P = nblk * F32S_BLOCK;
+    for (int64_t r = 0; r < M; ++r) {
+        for (int64_t c = 0; c < N; ++c) {
+            uint8_t byte = packed[r * (P / 2) + c / 2];
+            int nib = (c % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
+            float s32 = scales[r * nblk + c / F32S_BLOCK];
+            y[r * N + c] = oracle_f32_to_bf16(oracle_e2m1_lut(nib) * s32);
+        }
+    }
+}
+
+/* Fake-quantization in the fp32-scale flavour: dequantize(quantize(x)).  Returns -1 if the
+ * temporaries cannot be allocated, else 0. */
+ORACLE_API int oracle_fake_quant_f32scale(const uint16_t* x, int64_t M, int64_t N, uint16_t* y) {
+    int64_t nblk = (N + F32S_BLOCK - 1) / F32S_BLOCK;
+    size_t npacked = (size_t)M * (size_t)(nblk * F32S_BLOCK / 2), nscale = (size_t)M * (size_t)nblk;
+    uint8_t* packed = (uint8_t*)malloc(npacked ? npacked : 1);
+    float* scales = (float*)malloc((nscale ? nscale : 1) * sizeof(float));
+    if (!packed || !scales) { free(packed); free(scales); return -1; }
+    int rc = oracle_quantize_f32scale(x, M, N, packed, scales);
+    if (rc == 0) oracle_dequantize_f32scale(packed, scales, M, N, y);
+    free(packed);
+    free(scales);
+    return rc;
+}
+
 /* [QATLIN] section 5, one observer step given the current amax `cur` (after any
  * cross-rank MAX).  kind 0 = "static_minmax": max(state, cur); kind 1 = "minmax", an
  * exponential moving average: (1 - decay) * state + decay * cur, where both Python

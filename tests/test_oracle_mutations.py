@@ -15,6 +15,9 @@ from oracle.build import CFLAGS, SRC
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
+# Not planted: dropping the clamp of x / scale to [-6, 6] (either flavour).  The e2m1 rounding
+# saturates (any magnitude of 5 or more gives index 7; the brute-force pin checks it up to 8),
+# so clamping the quotient to 6 first changes no code: that mutant is equivalent.
 MUTATIONS = [
     ("nibble order", "pb[j] = (uint8_t)(code[2 * j] | (code[2 * j + 1] << 4));",
      "pb[j] = (uint8_t)(code[2 * j + 1] | (code[2 * j] << 4));"),
@@ -48,6 +51,18 @@ MUTATIONS = [
      "float v = oracle_bf16_to_f32(xb[i]);"),
     ("e4m3 exponent bias", "ldexp((double)(8 + m), e - 10)", "ldexp((double)(8 + m), e - 11)"),
     ("e2m1 lut sign", "return (code & 8) ? -m : m;", "return m;"),
+    ("fp32-scale nibble order", "out[j] = (uint8_t)(c32[2 * j] | (c32[2 * j + 1] << 4));",
+     "out[j] = (uint8_t)(c32[2 * j + 1] | (c32[2 * j] << 4));"),
+    ("fp32-scale block amax times 6", "float block_scale = block_amax / FLOAT4_MAX;",
+     "float block_scale = block_amax * FLOAT4_MAX;"),
+    ("fp32-scale no encode-side clamp", "float divisor = block_scale < TINY_CLAMP ? TINY_CLAMP : block_scale;",
+     "float divisor = block_scale;"),
+    ("fp32-scale clamp on the decode side too", "float s32 = scales[r * nblk + c / F32S_BLOCK];",
+     "float s32 = scales[r * nblk + c / F32S_BLOCK]; if (s32 < TINY_CLAMP) s32 = TINY_CLAMP;"),
+    ("fp32-scale signed block amax", "float mag = fabsf(oracle_bf16_to_f32(blk[i]));",
+     "float mag = oracle_bf16_to_f32(blk[i]);"),
+    ("fp32-scale sign of zero", "c32[i] = (uint8_t)(q < 0.0f ? idx + 8 : idx);",
+     "c32[i] = (uint8_t)(signbit(q) ? idx + 8 : idx);"),
     ("block size ignored", "const uint16_t* xb = row + b * B;\n            float block_amax = 0.0f;\n            for (int i = 0; i < B; ++i) {",
      "const uint16_t* xb = row + b * B;\n            float block_amax = 0.0f;\n            for (int i = 0; i < 16; ++i) {"),
 ]

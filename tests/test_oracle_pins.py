@@ -536,3 +536,101 @@ def test_linear_uses_the_dequantized_weight():
     # scaling x by a power of two scales y exactly
     x4 = _bf16_bits(oracle.bf16_to_f64(x) * 4.0)
     assert np.array_equal(oracle.w4a16_linear(x4, packed, scales, gs, n_out), 4.0 * y)
+
+
+# ---- the fp32-scale flavour with blocks of 32 (fp4_optimization.py, constants block) ---------
+#
+# The pages name this flavour and define it no further; the oracle's reading is the NVFP4
+# steps with the block scale kept as an fp32 (block_amax / 6, no E4M3 rounding, no
+# per-tensor scale).  What pins it: a block built from grid points (every code and the
+# decoded value known in advance), the all-zero block, the scale as numpy's fp32 division,
+# the codes as a brute-force nearest search on numpy's fp32 quotient, the decode as torch's
+# bf16 cast of the fp32 product, an error bound, idempotence and the zero padding.
+
+def test_f32scale_grid_block_by_construction():
+    # element 0 is 6 S with S = 2^-4, so block_amax / 6 = S exactly; the other 31 elements
+    # are grid points times S (codes by construction) or mid-points times S (ties go to the
+    # even index); every decoded value is exactly LUT * S.
+    S = 2.0 ** -4
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    ties = {0.25: 0, 0.75: 2, 1.25: 2, 1.75: 4, 2.5: 4, 3.5: 6, 5.0: 6}
+    rng = np.random.default_rng(31)
+    vals, codes = [6.0 * S], [7]
+    for _ in range(31):
+        sign = rng.integers(0, 2)
+        if rng.integers(0, 2):
+            k = int(rng.integers(0, 8))
+            m, idx = mags[k], k
+        else:
+            m, idx = list(ties.items())[int(rng.integers(0, 7))]
+        vals.append((-m if sign else m) * S)
+        codes.append(idx | (8 if sign and m > 0 else 0))
+    x = _bf16_bits(np.array(vals, dtype=np.float32)).reshape(1, 32)
+    packed, scales = oracle.quantize_f32scale(x)
+    assert scales.shape == (1, 1) and _f32_bits(scales[0, 0]) == _f32_bits(S)
+    np.testing.assert_array_equal(_unpack(packed)[0], np.array(codes))
+    y = synthetic.bf16_bits_to_f32(oracle.dequantize_f32scale(packed, scales, 1, 32))
+    want = np.array([(-1.0 if c & 8 else 1.0) * mags[c & 7] * S for c in codes], dtype=np.float32)
+    np.testing.assert_array_equal(np.abs(y[0]), np.abs(want))
+    np.testing.assert_array_equal(oracle.fake_quant_f32scale(x), oracle.dequantize_f32scale(packed, scales, 1, 32))
+
+
+def test_f32scale_zero_block_and_padding():
+    x = np.zeros((3, 70), dtype=np.uint16)                 # 70 columns: 3 blocks, 26 zeros of padding
+    x[1, 5] = _bf16_bits([1.5])[0]
+    packed, scales = oracle.quantize_f32scale(x)
+    assert packed.shape == (3, 48) and scales.shape == (3, 3)
+    assert not scales[0].any() and not packed[0].any()     # all-zero row: scale 0, codes 0
+    assert _f32_bits(scales[1, 0]) == _f32_bits(np.float32(1.5) / np.float32(6))
+    assert not scales[1, 1:].any()
+    y = oracle.fake_quant_f32scale(x)
+    assert y.shape == (3, 70) and not y[0].any() and not y[2].any()
+    assert y[1, 5] == x[1, 5]                              # the block's largest value survives
+    # a row of 70 decodes like the first 70 columns of the same row padded to 96
+    xp = np.zeros((3, 96), dtype=np.uint16)
+    xp[:, :70] = x
+    np.testing.assert_array_equal(oracle.fake_quant_f32scale(xp)[:, :70], y)
+
+
+def test_f32scale_scales_and_codes_vs_independent_rounding():
+    rng = np.random.default_rng(32)
+    x = synthetic.to_bf16_bits(rng.standard_t(3, (48, 256)).astype(np.float32))
+    x[5, :32] = 0                                          # one all-zero block
+    # one block whose scale block_amax / 6 falls below the 1e-12 clamp (the quotients use
+    # 1e-12, the decode the unclamped scale), one whose largest values are negative
+    x[6, 32:64] = synthetic.to_bf16_bits(rng.uniform(-3e-12, 3e-12, 32).astype(np.float32))
+    x[7, 64:96] = synthetic.to_bf16_bits(-np.abs(rng.standard_normal(32)).astype(np.float32))
+    packed, scales = oracle.quantize_f32scale(x)
+    xf = synthetic.bf16_bits_to_f32(x).reshape(48, 8, 32)
+    b = np.abs(xf).max(axis=2)
+    want_s = b.astype(np.float32) / np.float32(6.0)        # numpy: one IEEE fp32 division
+    np.testing.assert_array_equal(scales.view(np.uint32), want_s.view(np.uint32))
+    div = np.maximum(want_s, np.float32(1e-12))
+    q = np.clip(xf / div[..., None], np.float32(-6), np.float32(6))  # fp32 quotient, correctly rounded
+    idx = _nearest_grid_ties_even(np.abs(q).ravel()).reshape(q.shape)
+    code = np.where(q < 0, idx + 8, idx)
+    np.testing.assert_array_equal(_unpack(packed).reshape(48, 8, 32), code)
+    # decode: torch's round of the fp32 product LUT * scale to bf16
+    lut = np.array([0, .5, 1, 1.5, 2, 3, 4, 6, -0.0, -.5, -1, -1.5, -2, -3, -4, -6], dtype=np.float32)
+    prod = lut[code] * want_s[..., None]
+    want_y = torch.from_numpy(prod.reshape(48, 256)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(oracle.dequantize_f32scale(packed, scales, 48, 256), want_y)
+
+
+def test_f32scale_error_bound_and_idempotence():
+    rng = np.random.default_rng(33)
+    x = synthetic.to_bf16_bits(rng.standard_normal((64, 512)).astype(np.float32))
+    y1 = oracle.fake_quant_f32scale(x)
+    xf = synthetic.bf16_bits_to_f32(x).reshape(64, 16, 32).astype(np.float64)
+    yf = synthetic.bf16_bits_to_f32(y1).reshape(64, 16, 32).astype(np.float64)
+    s = (np.abs(xf).max(axis=2) / 6.0)[..., None]
+    scaled = np.abs(xf) / s
+    half_step = np.where(scaled <= 2.0, 0.25, np.where(scaled <= 4.0, 0.5, 1.0))
+    # half a grid step at the block's scale, plus the rounding of the output to bf16
+    assert np.all(np.abs(xf - yf) <= half_step * s * (1 + 2 ** -20) + np.abs(yf) * 2.0 ** -8)
+    # the block's largest value survives, so the scale and every code come back: fq is
+    # idempotent up to -0 -> +0 (code 8 decodes to -0, which quantizes to code 0)
+    y2 = oracle.fake_quant_f32scale(y1)
+    nz = (y1 & 0x7FFF) != 0
+    np.testing.assert_array_equal(y2[nz], y1[nz])
+    assert not y2[~nz].any()
