@@ -358,8 +358,9 @@ nvfp4_status nvfp4_w4a16_pack(const uint8_t* packed, const uint8_t* scales, int6
  * forward and runs the layer's bf16 forward on it.  One kernel on the tensor cores (bf16 x
  * bf16, fp32 accumulation, output rounded to bf16 once; the bias is added to the fp32 sum
  * before that rounding); the decoded weight is built tile by tile on chip (in tensor
- * memory, or in shared memory for 9 to 32 rows of x and whenever K is split; in registers,
- * with fp32 FMAs on the CUDA cores, for up to 8 rows) and never written to device memory.
+ * memory; in shared memory when the larger kernels split K or take 9 to 32 rows of x; in
+ * registers, with fp32 FMAs on the CUDA cores, for one row of x without room in the
+ * workspace) and never written to device memory.
  * Each weight element is decoded exactly as
  * nvfp4_dequantize does; the sum is not bit-reproducible against another GEMM (the order
  * in which the tensor cores accumulate is not sequential IEEE), the tests state the bound.
@@ -375,10 +376,12 @@ nvfp4_status nvfp4_w4a16_pack(const uint8_t* packed, const uint8_t* scales, int6
  *           wait inside the kernel that runs out records NVFP4_ERR_TIMEOUT there
  *           (nvfp4_workspace_check; zero the whole workspace before reusing it then), the
  *           kernel stops and y is unspecified.  With at least nvfp4_w4a16_workspace_bytes(M,
- *           N, K) bytes, a call with at most 128 rows of x may split K over several CTAs per
- *           output tile: each writes fp32 partial sums there and the last to finish adds them
- *           in a fixed order (so results do not depend on timing) and leaves its counter at
- *           zero again.  With less, K is not split.
+ *           N, K) bytes, a call with at most 8 rows of x runs the small kernel (the weight
+ *           cut into equal contiguous shares, two CTAs per SM) and one with at most 128 rows
+ *           may split K over several CTAs per output tile: the CTAs that share a tile write
+ *           fp32 partial sums there and the last to finish adds them in a fixed order (so
+ *           results do not depend on timing) and leaves the tile's counter at zero again.
+ *           With less, K is not split.
  * Errors: NVFP4_ERR_SHAPE (K, sizes past the 32-bit tensor-map limits), NVFP4_ERR_NULL,
  * NVFP4_ERR_ALIGN, NVFP4_ERR_ARG (tensor map rejected, workspace_bytes too small).  M == 0 or
  * N == 0 launches nothing.  Enqueues one kernel. */
@@ -397,22 +400,31 @@ nvfp4_status nvfp4_w4a16_selftest_timeout(const void* x, int64_t M, int64_t K, c
                                           const float* d_global_scale, int64_t N, void* y, void* d_workspace,
                                           int64_t workspace_bytes, uint32_t timeout_us, nvfp4_stream_t stream);
 
-/* Workspace bytes with which nvfp4_w4a16_linear may split K for this shape (at least
- * NVFP4_WORKSPACE_BYTES; -1 for a shape it refuses).  Depends on the current device's SM
- * count. */
+/* Workspace bytes with which nvfp4_w4a16_linear takes its fastest plan for this shape (room
+ * for the partial sums of the small kernel or of a split K; at least NVFP4_WORKSPACE_BYTES;
+ * -1 for a shape it refuses).  Depends on the current device's SM count.  For the small
+ * kernel: the status block, one 4-byte counter per 128 rows of W (rounded up to 256 bytes),
+ * then 2 x G x 128 x 16 fp32 partial sums (two slots per CTA), G = min(2 x SMs, ceil(N / 128)
+ * x ceil(K / 128)). */
 int64_t nvfp4_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* How nvfp4_w4a16_linear runs x [M, K] . W[N, K]^T with a workspace of workspace_bytes on a
  * device with `sms` SMs (the decision that call takes with the current device's SM count).
  * Host only: launches nothing and needs no GPU.
- *   *kernel         2: the CUDA cores, no tensor cores (at most 8 rows of x); 0: the weight
- *                   decoded into shared memory (split K, or 9 to 32 rows of x); 1: the
- *                   weight decoded into tensor memory (everything else)
- *   *rows_per_tile  rows of x per output tile: for kernel 2, M rounded up to 1, 2, 4 or 8
- *                   (tiles of 32 weight rows); 128 for kernel 0; for kernel 1, 64 or 128 up to
- *                   128 rows of x, above that 256, or 128 where 128-row tiles need no more
- *                   waves of one CTA per SM (tiles of kernels 0 and 1 cover 128 weight rows)
- *   *splits         CTAs per output tile over K (kernel 0 only; 1 otherwise)
+ *   *kernel         3: the small kernel (at most 8 rows of x and a workspace of at least
+ *                   nvfp4_w4a16_workspace_bytes: the weight's items of 128 rows x 128
+ *                   columns cut into equal contiguous shares, two CTAs per SM, the weight
+ *                   decoded into tensor memory as the MMA's 128-row operand); 2: the CUDA
+ *                   cores, no tensor cores (one row of x, workspace too small for kernel 3);
+ *                   0: the weight decoded into shared memory (split K, or 9 to 32 rows of
+ *                   x); 1: the weight decoded into tensor memory (everything else)
+ *   *rows_per_tile  rows of x per output tile: 16 for kernel 3;
+ *                   1 for kernel 2 (tiles of 32 weight rows); 128 for kernel 0; for kernel 1,
+ *                   64 or 128 up to 128 rows of x, above that 256, or 128 where 128-row tiles
+ *                   need no more waves of one CTA per SM (tiles of kernels 0 and 1 cover 128
+ *                   weight rows)
+ *   *splits         kernel 3: the CTAs that share the weight, G; kernel 0: CTAs per output
+ *                   tile over K; 1 otherwise
  * Errors: NVFP4_ERR_SHAPE as nvfp4_w4a16_linear, NVFP4_ERR_NULL (an output pointer),
  * NVFP4_ERR_ARG (sms < 1). */
 nvfp4_status nvfp4_w4a16_plan(int64_t M, int64_t N, int64_t K, int64_t workspace_bytes, int sms, int* kernel,

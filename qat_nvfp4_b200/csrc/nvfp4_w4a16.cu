@@ -154,31 +154,34 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
+// try_wait with a suspend-time hint: a thread whose phase has not completed sleeps until it
+// completes (or the hint runs out) instead of returning at once, so that a waiting warp takes
+// no issue slots from the warps that do the work.
+constexpr uint32_t kSuspendHintNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "n"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
 
 // Wait until the phase of parity `parity` of the barrier has completed.  Gives up (false)
-// after kWaitLimitNs, or early when another role has set *abort (unless ignore_abort).
+// after limit_ns, or early when another role has set *abort (unless ignore_abort); both are
+// checked each time the suspended thread wakes without the phase.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile uint32_t* abort,
                                           bool ignore_abort = false, uint64_t limit_ns = kWaitLimitNs) {
-    uint64_t t0 = 0;
-    for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 63u) {
-            if (!ignore_abort && *abort) return false;
-            const uint64_t now = global_ns();
-            if (t0 == 0) t0 = now;
-            else if (now - t0 > limit_ns) return false;
-        }
+        if (!ignore_abort && *abort) return false;
+        if (global_ns() - t0 > limit_ns) return false;
     }
 }
 
@@ -374,6 +377,13 @@ template <class Sh>
 __device__ __forceinline__ void stop_all(Sh& sh, Workspace* ws) {
     *reinterpret_cast<volatile uint32_t*>(&sh.abort) = 1u;
     atomicExch(&ws->error, (unsigned)NVFP4_ERR_TIMEOUT);
+}
+
+// One lane of a converged warp (elect.sync): the lane that issues for the warp.
+__device__ __forceinline__ bool elect_one_sync() {
+    uint32_t e;
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(e));
+    return e != 0;
 }
 
 // Wait on `bar` from every lane of a warp; true in all lanes only if every lane saw it.
@@ -800,6 +810,18 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// tmem_st32 without the wait: the caller waits (tcgen05.wait::st) before it signals the data.
+__device__ __forceinline__ void tmem_st32_nowait(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]),
+        "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]),
+        "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
 // 16 consecutive fp32 columns of this warp's 32 TMEM lanes, without waiting (the caller
 // waits once with tcgen05.wait::ld before reading v).
 __device__ __forceinline__ void tmem_ld16_issue(uint32_t taddr, uint32_t* v) {
@@ -1062,6 +1084,647 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------
+// Byte-permute decode of one 16-element block (two words of eight codes, element 2j in the
+// low nibble of byte j) into eight bf16x2 words, bit for bit bf16_rn(fl(LUT[code] * sd)):
+// the block's eight magnitudes bf16_rn(fl(m * sd)), m = 0, 0.5, 1, 1.5, 2, 3, 4, 6, are
+// formed once (four packed fp32 products, four roundings to bf16x2) and split into a table
+// of low bytes and one of high bytes; each word of codes then picks every element's two
+// bytes with byte permutes indexed by its magnitude nibbles, flips the sign bit of the high
+// byte for a negative code (fl(-m * sd) is -fl(m * sd) whatever the sign of sd, zeros
+// included), and interleaves low and high bytes into bf16 pairs.  About 2.7 instructions per weight
+// against ~4 for converting each code pair to f16, then to fp32, multiplying and rounding.
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// bf16x2 of the fp32 pair (low lane -> low half), round to nearest even
+__device__ __forceinline__ uint32_t bf16x2_of_pair(uint64_t v) {
+    uint32_t d;
+    asm("{\n\t.reg .f32 l, h;\n\tmov.b64 {l, h}, %1;\n\tcvt.rn.bf16x2.f32 %0, h, l;\n\t}" : "=r"(d) : "l"(v));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t mul_pair(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// The byte tables of one block scale sd: the low bytes (x) and high bytes (y) of
+// bf16_rn(fl(m * sd)) for the magnitudes m = 0, 0.5, 1, 1.5 and the same for 2, 3, 4, 6 (z, w).
+__device__ __forceinline__ uint4 decode_tables(float sd) {
+    uint64_t sd2;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(sd2) : "f"(sd));
+    // magnitude pairs (lane 0, lane 1) as fp32 bits: (0, 0.5), (1, 1.5), (2, 3), (4, 6)
+    const uint32_t w01 = bf16x2_of_pair(mul_pair(0x3F00000000000000ull, sd2));
+    const uint32_t w23 = bf16x2_of_pair(mul_pair(0x3FC000003F800000ull, sd2));
+    const uint32_t w45 = bf16x2_of_pair(mul_pair(0x4040000040000000ull, sd2));
+    const uint32_t w67 = bf16x2_of_pair(mul_pair(0x40C0000040800000ull, sd2));
+    return make_uint4(prmt(w01, w23, 0x6420u), prmt(w01, w23, 0x7531u), prmt(w45, w67, 0x6420u),
+                      prmt(w45, w67, 0x7531u));
+}
+
+// 16 codes (two words, element 2 i in the low nibble of byte i) -> 8 bf16 pairs, by the byte
+// tables of the block's scale (decode_tables).
+__device__ __forceinline__ void decode_block_tab(uint32_t c0, uint32_t c1, uint4 t, uint32_t* o) {
+    const uint32_t tl0 = t.x, th0 = t.y, tl1 = t.z, th1 = t.w;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t c = h ? c1 : c0;
+        const uint32_t m = c & 0x77777777u, mh = m >> 16, c4 = c << 4;
+        // sign of element k = bit 4k + 3: the top bit of byte k of {c4, c, c4, c} (elements 0..3)
+        const uint32_t l03 = prmt(tl0, tl1, m), h03 = prmt(th0, th1, m) ^ (prmt(c, c4, 0x1504u) & 0x80808080u);
+        const uint32_t l47 = prmt(tl0, tl1, mh), h47 = prmt(th0, th1, mh) ^ (prmt(c, c4, 0x3726u) & 0x80808080u);
+        o[4 * h + 0] = prmt(l03, h03, 0x5140u);
+        o[4 * h + 1] = prmt(l03, h03, 0x7362u);
+        o[4 * h + 2] = prmt(l47, h47, 0x5140u);
+        o[4 * h + 3] = prmt(l47, h47, 0x7362u);
+    }
+}
+
+__device__ __forceinline__ void decode_block_prmt(uint32_t c0, uint32_t c1, float sd, uint32_t* o) {
+    decode_block_tab(c0, c1, decode_tables(sd), o);
+}
+
+// ---------------------------------------------------------------------------------------
+// Up to 8 rows of x: w4a16_small_kernel.  With few rows the work is the packed weight
+// itself (read once, decoded once), so the kernel is laid out for the weight stream:
+//
+//   - The weight is cut into items of two 64-column atoms of one 128-row tile (two
+//     consecutive records), ordered tile by tile.  The grid is two CTAs per SM, and CTA c
+//     takes the contiguous item range [c I / G, (c + 1) I / G), so every CTA has the same
+//     share of the weight whatever the number of tiles (on the 14336 x 4096 MLP weight 112
+//     tiles would leave a third of the SMs idle).
+//   - The MMA is D[n][m] = sum_k W[n][k] x[m][k] with the decoded weight as the A operand (128
+//     weight rows, in tensor memory) and x as the B operand (BT = 16 rows of x, the MMA's N).
+//     The MMA warp runs its loop warp-uniformly and one elected lane issues, so the operands
+//     stay uniform: measured, the 8 MMAs and commits of an item then take ~130 ns (~550 ns
+//     when one lane ran the loop alone among the decode warps).
+//   - Each decode warp copies its 32 record rows of an atom (1 KB of codes as two whole
+//     512-byte halves, and the 32 scale words) from global memory into a shared-memory ring
+//     with cp.async, kRingR items ahead (issued before the barrier set-up, so that the first
+//     copies are under way at once), and each lane decodes its own row into one of the
+//     tensor-memory weight slots.  A block's 16 codes are looked up in byte tables of its
+//     scale built once per CTA for every scale byte (decode_tables).  A slot is signalled to
+//     the MMA warp one item late, so that the decode never waits for its tensor-memory store.
+//     (The records are not moved by TMA bulk copies: measured, one SM's bulk copies of 9 KB
+//     items arrived at only ~1 item per microsecond.)  One producer thread loads the x boxes
+//     of each item with TMA; one commit per item frees both the item's x stage and, kSlots
+//     items later, its weight slot; four epilogue warps read the accumulators (one per tile
+//     segment, alternating, so that a segment's epilogue overlaps the next segment's MMAs).
+//   - A tile covered by one CTA is finished in place (bias, one rounding to bf16, store).  A
+//     tile shared by several CTAs (consecutive ranges) is finished by the last of them to
+//     arrive (a counter per tile in the workspace): each writes its fp32 partial sums, and the
+//     last adds the partial sums of all of them in CTA order, whichever CTA it is, so repeated
+//     calls give identical bits.  Only a CTA's first and last tile can be shared, so a CTA
+//     has two partial-sum slots.  In a CTA's last segment both rings are idle and the last
+//     CTA stages every contributor's sums there with cp.async, all in flight at once.
+//   - Every barrier wait sleeps (try_wait with a suspend-time hint) rather than spinning.
+//
+// Measured on B200 (ncu kernel time, L2 flushed): 14336 x 4096 at 1-8 rows of x ~23-24 us,
+// 4096 x 4096 ~15 us; the kernels with x as the 128-row operand take 25 and 16-19 us there.
+// A timeline of each role shows each decode warp's item to be a chain of dependent steps (copy
+// wait, shared loads, lookups, store, slot signal) of ~650 ns even with the arithmetic taken
+// out; with four such warps per SM sub-partition and the register budget of two CTAs per SM
+// that chain, not HBM (an L2-resident copy of the weight is no faster), not the decode
+// arithmetic and not the MMAs, sets the rate.  From 16 rows up the kernels with x as the
+// 128-row operand are faster, so make_plan sends only up to 8 rows here.
+//
+// Tensor memory (256 columns per CTA): accumulators at columns 0 and BT; weight slots of 64
+// columns (two atoms of 64 bf16 pairs each, row n in lane n, the lower K in the low half, the
+// layout of the "A from tensor memory" MMA) above them: three for BT <= 32, two for BT = 64.
+
+constexpr int kSmAtoms = 2;                          // atoms of K per item
+constexpr int kSmDecodeWarps = 4 * kSmAtoms;         // lane quarter x atom
+constexpr int kSmEpiWarp = kSmDecodeWarps;           // warps 8 .. 11: epilogue
+constexpr int kSmTmaWarp = kSmEpiWarp + 4;           // warp 12: producer
+constexpr int kSmMmaWarp = kSmTmaWarp + 1;           // warp 13: TMEM allocation, MMAs
+constexpr int kSmThreads = 32 * (kSmMmaWarp + 1);    // 448
+constexpr int kSmTmemCols = 256;
+constexpr int kSmSlotCols = kSmAtoms * kBK / 2;      // 64
+constexpr int kSmRecSlotBytes = kSmAtoms * kRecBytes;  // one item's record rows: 9216 bytes
+constexpr int kSmMaxRows = 8;                        // rows of x the kernel takes (one 16-row tile)
+
+template <int BT>
+struct SmCfg {
+    static constexpr int kWCol = BT <= 32 ? 64 : 128;                      // first weight slot column
+    static constexpr int kSlots = (kSmTmemCols - kWCol) / kSmSlotCols;     // 3 or 2 weight slots
+    static constexpr int kAtomXBytes = BT * kBK * 2;                       // one x box: BT rows x 128 bytes
+    static constexpr int kStageXBytes = kSmAtoms * kAtomXBytes;
+    static constexpr int kRingX = 2 * kSlots;                              // x stages (and MMA commits) in flight
+    // record slots: what ~104 KB leaves after the x stages, at most 8 items ahead
+    static constexpr int kRingRFit = (104 * 1024 - kRingX * kStageXBytes) / kSmRecSlotBytes;
+    static constexpr int kRingR = kRingRFit < 8 ? kRingRFit : 8;
+    static constexpr int kRecOff = kRingX * kStageXBytes;                  // record ring after the x ring
+    // kind::f16 instruction descriptor: fp32 D, bf16 A and B, both K-major, N = BT, M = 128
+    static constexpr uint32_t kIdesc =
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BT >> 3) << 17) | ((uint32_t)(kMmaM >> 4) << 24);
+    struct Shared {
+        uint64_t xfull[kRingX];    // the item's x boxes landed (TMA)
+        uint64_t done[kRingX];     // the item's MMAs completed (x stage free; kSlots items on, its weight slot)
+        uint64_t w_full[kSlots];   // the decode warps wrote the weight slot
+        uint64_t acc_full[2];      // every MMA of the accumulator's tile segment completed
+        uint64_t acc_empty[2];     // the epilogue read the accumulator
+        uint64_t drain;            // used only when stopping early
+        uint64_t never;            // self-test: a barrier nothing arrives on
+        uint32_t tmem_base;
+        uint32_t abort;
+        uint32_t last;             // epilogue: this CTA finishes the shared tile
+        uint4 tab[256];            // decode byte tables (decode_tables) for every E4M3 scale byte
+    };
+    static constexpr int kSmemBytes = 1024 + kRecOff + kRingR * kSmRecSlotBytes + (int)sizeof(Shared);
+    static_assert(BT == 16 || BT == 32 || BT == 64, "MMA N");
+    static_assert(kAtomXBytes % 1024 == 0, "x boxes stay 1024-byte aligned");
+    static_assert(kRingR >= 3, "record ring depth");
+    static_assert(2 * kSmemBytes + 2 * 1024 <= 228 * 1024, "two CTAs per SM");
+    static_assert(2 * BT <= kWCol && kWCol + kSlots * kSmSlotCols == kSmTmemCols, "tensor memory columns");
+};
+
+struct SmallArgs {
+    const uint8_t* tiled;   // weight records
+    const float* d_gs;      // encode global scale of the weight
+    const uint16_t* bias;   // [N] bf16, or null
+    uint16_t* y;            // [M, N] bf16
+    Workspace* ws;
+    unsigned* counters;     // per 128-row tile: CTAs that finished their part (the last resets it)
+    float* partial;         // fp32 partial sums [2 G][128][Mp], Mp = M rounded up to 16 (rows of
+                            // x fastest): slot 2 c for CTA c's first tile, 2 c + 1 for its last
+    int64_t M, Mp, N;
+    int64_t kt;             // atoms of K (records per tile row)
+    int64_t nk;             // items per tile: ceil(kt / 2)
+    int64_t items;          // tiles x nk
+    int64_t grid;           // CTAs sharing the items
+    uint32_t box_bytes;     // bytes of one x box (rows loaded x 128)
+    uint64_t selftest_ns;   // nonzero: first wait on a barrier nothing completes, for this long
+};
+
+__device__ __forceinline__ int64_t sm_item_begin(const SmallArgs& a, int64_t c) { return c * a.items / a.grid; }
+// the CTA whose range holds item i (the largest c with begin(c) <= i; never an empty range)
+__device__ __forceinline__ int64_t sm_cta_of(const SmallArgs& a, int64_t i) { return ((i + 1) * a.grid - 1) / a.items; }
+
+// The last CTA of a shared tile adds the nc + 1 partial-sum slots (p_lo, then p0 + k stride
+// for k = 1 .. nc, CTA order) of the tile's first M rows of x, with the rings of shared memory
+// from `stage` on as a staging area: each of the 128 epilogue threads copies its own float4
+// units (row, 4 rows of x) of every contributor there (cp.async, all in flight at once), then
+// adds each unit's contributions in CTA order, adds the bias, rounds once to bf16 and stores.
+// The caller guarantees room for 4 x 128 x (nc + 1) float4 and that nothing else uses it.
+__device__ __noinline__ void small_reduce_staged(int64_t M, int64_t N, int64_t Mp, const uint16_t* bias, uint16_t* y,
+                                                 int64_t tn, uint32_t stage, const float* p_lo, const float* p0,
+                                                 int64_t stride, int nc, int mq, int tid) {
+    const int units = kRecRows * mq;
+    for (int ub = 0; ub < units; ub += 4 * 128) {
+#pragma unroll 1
+        for (int h = 0; h < 4; ++h) {
+            const int u = ub + tid + 128 * h;
+            if (u >= units) break;
+            const int ur = u / mq;
+            const int64_t off = (int64_t)ur * Mp + 4 * (u - ur * mq);
+            cp_async<16>(stage + (uint32_t)((h * 128 + tid) * 16), p_lo + off);
+            const float* src = p0 + stride + off;
+            for (int k = 1; k <= nc; ++k, src += stride)
+                cp_async<16>(stage + (uint32_t)(((k * 4 + h) * 128 + tid) * 16), src);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();  // this thread's own copies: no barrier needed
+#pragma unroll 1
+        for (int h = 0; h < 4; ++h) {
+            const int u = ub + tid + 128 * h;
+            if (u >= units) break;
+            float4 f;
+            for (int k = 0; k <= nc; ++k) {
+                float4 v;
+                asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                             : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                             : "r"(stage + (uint32_t)(((k * 4 + h) * 128 + tid) * 16)));
+                if (k == 0) {
+                    f = v;
+                } else {
+                    f.x = __fadd_rn(f.x, v.x);
+                    f.y = __fadd_rn(f.y, v.y);
+                    f.z = __fadd_rn(f.z, v.z);
+                    f.w = __fadd_rn(f.w, v.w);
+                }
+            }
+            const int ur = u / mq, m0 = 4 * (u - ur * mq);
+            const int64_t nn = tn * kRecRows + ur;
+            if (nn >= N) continue;
+            const float bb = bias != nullptr ? __uint_as_float((uint32_t)__ldg(bias + nn) << 16) : 0.f;
+            const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (m0 + e < M)
+                    y[(m0 + e) * N + nn] =
+                        __bfloat16_as_ushort(__float2bfloat16_rn(bias != nullptr ? __fadd_rn(fv[e], bb) : fv[e]));
+        }
+    }
+}
+
+__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int BT>
+__global__ void __launch_bounds__(kSmThreads, 2)
+    w4a16_small_kernel(const __grid_constant__ CUtensorMap tmap_x, const SmallArgs a) {
+    using C = SmCfg<BT>;
+    constexpr int kRingX = C::kRingX, kRingR = C::kRingR, kSlots = C::kSlots;
+    constexpr int kAtomXBytes = C::kAtomXBytes, kStageXBytes = C::kStageXBytes;
+    const int64_t cta = blockIdx.x;
+    const int64_t i0 = sm_item_begin(a, cta), i1 = sm_item_begin(a, cta + 1);
+    if (i0 >= i1) return;  // no items (fewer items than CTAs): nothing to do, no shared state touched
+    const int nitems = (int)(i1 - i0);
+
+    extern __shared__ uint8_t dsmem[];
+    const uint32_t raw = smem_u32(dsmem);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* ring = dsmem + (base - raw);
+    typename C::Shared& sh = *reinterpret_cast<typename C::Shared*>(ring + C::kRecOff + kRingR * kSmRecSlotBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kt = (int)a.kt, nk = (int)a.nk;
+    const int64_t tile_first = i0 / nk;
+
+    // Decode warp (q, t), one record row per thread: atom t of each item, weight rows 32 q ..
+    // + 31.  Its copy state is set up first and its first kRingR items' copies issued before
+    // anything else, so that they are under way while the barriers and tensor memory are
+    // prepared.  Each thread copies its own record rows into private ring slots (cp.async, one
+    // commit group per item), so no barrier guards that ring.
+    const int dq = warp & 3, dt = (warp >> 2) & 1;
+    const int drow = 32 * dq + lane;
+    const uint32_t rslot0 = base + (uint32_t)C::kRecOff + (uint32_t)(dt * kRecRows + drow) * 32u;
+    const uint32_t sslot0 =
+        base + (uint32_t)C::kRecOff + (uint32_t)(kSmAtoms * kRecCodes) + (uint32_t)(dt * kRecRows + drow) * 4u;
+    int fj = 0, fkb = (int)(i0 - tile_first * nk);  // the next item to fetch, and its item in tile
+    uint32_t fslot = 0;                              // its ring slot offset
+    // The warp copies its 32 record rows (1 KB of codes, contiguous) as two 512-byte halves, 16
+    // bytes per lane (whole sectors per instruction), and the 32 scale words; each lane then
+    // reads its own row once the warp has synchronised.
+    const uint32_t wslot0 = rslot0 - (uint32_t)lane * 16u;  // = the warp's rows + 16 lane
+    const uint8_t* frec = a.tiled + (tile_first * a.kt + kSmAtoms * fkb + dt) * kRecBytes + (32 * dq) * 32 + lane * 16;
+    const int64_t tile_skip = (a.kt - kSmAtoms * (int64_t)nk) * kRecBytes;  // 0, or -1 record for odd K atoms
+    auto fetch = [&]() {  // the next item's record rows (nothing past the range or K)
+        if (fj < nitems) {
+            if (kSmAtoms * fkb + dt < kt) {
+                cp_async<16>(wslot0 + fslot, frec);
+                cp_async<16>(wslot0 + fslot + 512, frec + 512);
+                cp_async<4>(sslot0 + fslot, frec + (kRecCodes - 896 * dq - 12 * lane));  // row 32 dq + lane's scale word
+            }
+            frec += kSmAtoms * kRecBytes;
+            if (++fkb == nk) {
+                fkb = 0;
+                frec += tile_skip;
+            }
+        }
+        ++fj;
+        fslot = fslot + (uint32_t)kSmRecSlotBytes == (uint32_t)(kRingR * kSmRecSlotBytes) ? 0u
+                                                                                          : fslot + (uint32_t)kSmRecSlotBytes;
+        cp_async_commit();
+    };
+    if (warp < kSmDecodeWarps)
+        for (int j = 0; j < kRingR; ++j) fetch();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kRingX; ++s) {
+            mbar_init(smem_u32(&sh.xfull[s]), 1);
+            mbar_init(smem_u32(&sh.done[s]), 1);
+        }
+        for (int s = 0; s < kSlots; ++s) mbar_init(smem_u32(&sh.w_full[s]), kSmDecodeWarps);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_u32(&sh.acc_full[s]), 1);
+            mbar_init(smem_u32(&sh.acc_empty[s]), 4);
+        }
+        mbar_init(smem_u32(&sh.drain), 1);
+        mbar_init(smem_u32(&sh.never), 1);
+        sh.abort = 0u;
+        sh.last = 0u;
+        fence_barrier_init();
+    }
+    {
+        const float gs = __ldg(a.d_gs);
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) sh.tab[i] = decode_tables(__fdiv_rn(e4m3_to_f32((uint32_t)i), gs));
+    }
+    if (warp == kSmMmaWarp) {
+        tmem_alloc(smem_u32(&sh.tmem_base), kSmTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+    const volatile uint32_t* abort = &sh.abort;
+
+    if (warp == kSmTmaWarp) {
+        // ---- producer: each item's x boxes (TMA), up to kRingX items ahead of the MMAs ----
+        if (lane == 0) {
+            int issued = 0;
+            int kb = (int)(i0 - tile_first * nk);  // item in its tile, advanced item by item
+            for (int j = 0; j < nitems; ++j, kb = kb + 1 == nk ? 0 : kb + 1) {
+                const int na = min(kSmAtoms, kt - kSmAtoms * kb);
+                const int s = j % kRingX;
+                if (!mbar_wait(smem_u32(&sh.done[s]), ((uint32_t)(j / kRingX) & 1u) ^ 1u, abort)) {
+                    stop_all(sh, a.ws);
+                    break;
+                }
+                const uint32_t bar = smem_u32(&sh.xfull[s]);
+                mbar_arrive_expect_tx(bar, (uint32_t)na * a.box_bytes);
+                for (int t = 0; t < na; ++t)
+                    tma_load_2d(base + (uint32_t)(s * kStageXBytes + t * kAtomXBytes), &tmap_x,
+                                (kSmAtoms * kb + t) * kBK, 0, bar);
+                ++issued;
+            }
+            // no copy lands after the CTA has left
+            for (int j = issued > kRingX ? issued - kRingX : 0; j < issued; ++j)
+                if (!mbar_wait(smem_u32(&sh.xfull[j % kRingX]), (uint32_t)(j / kRingX) & 1u, abort, true))
+                    stop_all(sh, a.ws);
+        }
+    } else if (warp == kSmMmaWarp) {
+        // ---- MMAs: per item, 4 K steps of 16 per atom into the tile segment's accumulator,
+        //      one commit per item (and one more at the end of each segment).  The whole warp
+        //      runs the loop and its waits, so that control flow and operands stay warp-uniform;
+        //      one elected lane issues the MMAs and commits ----
+        bool ok = true;
+        if (a.selftest_ns != 0 &&
+            !__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&sh.never), 0u, abort, false, a.selftest_ns))) {
+            if (lane == 0) stop_all(sh, a.ws);
+            ok = false;
+        }
+        int seg = -1;
+        bool first = true;
+        const uint64_t xdesc0 = sw128_desc(base);
+        int kb = (int)(i0 - tile_first * nk);  // item in its tile, advanced item by item
+        int s = 0, w = 0;                      // x stage and weight slot of item j, and their parities
+        uint32_t xph = 0, wph = 0;
+        for (int j = 0; ok && j < nitems; ++j) {
+            const int na = min(kSmAtoms, kt - kSmAtoms * kb);
+            if (j == 0 || kb == 0) {  // a new tile segment
+                ++seg;
+                first = true;
+                if (!warp_wait(smem_u32(&sh.acc_empty[seg & 1]), ((uint32_t)(seg >> 1) & 1u) ^ 1u, abort)) {
+                    if (lane == 0) stop_all(sh, a.ws);
+                    ok = false;
+                    break;
+                }
+            }
+            if (!warp_wait(smem_u32(&sh.xfull[s]), xph, abort) || !warp_wait(smem_u32(&sh.w_full[w]), wph, abort)) {
+                if (lane == 0) stop_all(sh, a.ws);
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem + (uint32_t)((seg & 1) * BT);
+            // B descriptors differ only in their start address field (bits 0-13, address >> 4)
+            const uint64_t bd = xdesc0 + (uint64_t)((s * kStageXBytes) >> 4);
+            const uint32_t ta = tmem + (uint32_t)(C::kWCol + w * kSmSlotCols);
+            const bool seg_end = j == nitems - 1 || kb == nk - 1;
+            if (elect_one_sync()) {
+                if (first)
+                    asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, 0;" ::"r"(d), "r"(ta), "l"(bd),
+                                 "r"(C::kIdesc)
+                                 : "memory");
+                else
+                    asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, 1;" ::"r"(d), "r"(ta), "l"(bd),
+                                 "r"(C::kIdesc)
+                                 : "memory");
+#pragma unroll
+                for (int k = 1; k < kSmAtoms * (kBK / kUmmaK); ++k) {
+                    if (k == kBK / kUmmaK && na < 2) break;
+                    // atom k / 4, K step k % 4: 8 columns of A, 32 bytes of B per step
+                    const uint32_t ak = ta + (uint32_t)((k / (kBK / kUmmaK)) * (kBK / 2) + 8 * (k % (kBK / kUmmaK)));
+                    const uint64_t bk = bd + (uint64_t)((k / (kBK / kUmmaK)) * (kAtomXBytes >> 4) + 2 * (k % (kBK / kUmmaK)));
+                    asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, 1;" ::"r"(d), "r"(ak), "l"(bk),
+                                 "r"(C::kIdesc)
+                                 : "memory");
+                }
+                umma_commit(smem_u32(&sh.done[s]));
+                if (seg_end) umma_commit(smem_u32(&sh.acc_full[seg & 1]));
+            }
+            __syncwarp();
+            first = false;
+            if (++s == kRingX) {
+                s = 0;
+                xph ^= 1u;
+            }
+            if (++w == kSlots) {
+                w = 0;
+                wph ^= 1u;
+            }
+            kb = kb + 1 == nk ? 0 : kb + 1;
+        }
+        if (!ok) {
+            if (elect_one_sync()) umma_commit(smem_u32(&sh.drain));
+            __syncwarp();
+            mbar_wait(smem_u32(&sh.drain), 0u, abort, true);
+        }
+        __syncwarp();
+    } else if (warp < kSmDecodeWarps) {
+        // ---- decode: warp (q, t) decodes atom t of each item into the tensor memory lanes
+        //      32 q .. + 31 (the lanes its tcgen05.st may write); copies as set up above ----
+        const int t = dt;
+        const uint32_t tw = tmem + ((uint32_t)(32 * dq) << 16) + (uint32_t)(C::kWCol + t * (kBK / 2));
+        int kb = (int)(i0 - tile_first * nk);  // the item being decoded, in its tile
+        uint32_t rs = 0;                       // its ring slot offset
+        int w = 0;                             // its weight slot
+        int ds = 0;                            // the done barrier of item j - kSlots, and its parity
+        uint32_t dph = 0;
+        for (int j = 0; j < nitems; ++j) {
+            const bool live = kSmAtoms * kb + t < kt;  // an atom past K is neither written nor multiplied
+            uint32_t o[32];
+            cp_async_wait<kRingR - 1>();  // item j's group has landed
+            __syncwarp();                 // ... and the other lanes' (each lane reads its own row)
+            if (live) {
+                uint32_t c[8], sc;
+                asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+                             : "r"(rslot0 + rs));
+                asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(c[4]), "=r"(c[5]), "=r"(c[6]), "=r"(c[7])
+                             : "r"(rslot0 + rs + 16));
+                asm volatile("ld.shared.b32 %0, [%1];" : "=r"(sc) : "r"(sslot0 + rs));
+#pragma unroll
+                for (int b = 0; b < kBK / kBlockElems; ++b)  // block b: columns 8 b .. 8 b + 7
+                    decode_block_tab(c[2 * b], c[2 * b + 1], sh.tab[(sc >> (8 * b)) & 0xFFu], o + 8 * b);
+            }
+            fetch();  // item j + kRingR into the slot just read (its bytes were used above)
+            // the weight slot is free once the MMAs of the item kSlots before have completed
+            if (j >= kSlots) {
+                if (!warp_wait(smem_u32(&sh.done[ds]), dph, abort)) {
+                    if (lane == 0) stop_all(sh, a.ws);
+                    break;
+                }
+                if (++ds == kRingX) {
+                    ds = 0;
+                    dph ^= 1u;
+                }
+            }
+            // The previous item's store has had this item's decode to complete: wait for it,
+            // then signal that item's weight slot (one item late, so that the decode never
+            // waits on the store; the slot ring has room for the delay).
+            if (j > 0) {
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&sh.w_full[w == 0 ? kSlots - 1 : w - 1]));
+            }
+            if (live) {
+                tc_fence_after();
+                tmem_st32_nowait(tw + (uint32_t)(w * kSmSlotCols), o);
+            }
+            w = w + 1 == kSlots ? 0 : w + 1;
+            rs = rs + (uint32_t)kSmRecSlotBytes == (uint32_t)(kRingR * kSmRecSlotBytes) ? 0u : rs + (uint32_t)kSmRecSlotBytes;
+            kb = kb + 1 == nk ? 0 : kb + 1;
+            if (j == nitems - 1) {  // the last item's store and signal
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&sh.w_full[w == 0 ? kSlots - 1 : w - 1]));
+            }
+        }
+        cp_async_wait<0>();  // no copy of this thread lands after it leaves the loop
+    } else {
+        // ---- epilogue: warp q reads accumulator lanes 32 q .. + 31 (weight rows n), columns m
+        //      (rows of x) in chunks of 16; a whole tile is finished here, a shared one goes
+        //      through the partial sums and the tile's counter ----
+        const int q = warp - kSmEpiWarp;
+        const int row = 32 * q + lane;
+        const int tid = threadIdx.x - 32 * kSmEpiWarp;  // 0 .. 127
+        bool ok = true;
+        int seg = 0;
+        for (int64_t tn = tile_first; tn * nk < i1; ++tn, ++seg) {
+            const int64_t s0 = tn * nk > i0 ? tn * nk : i0, s1 = (tn + 1) * nk < i1 ? (tn + 1) * nk : i1;
+            const bool whole = s0 == tn * nk && s1 == (tn + 1) * nk;
+            const int64_t n = tn * kRecRows + row;
+            const bool live_n = n < a.N;
+            const float bias = (a.bias != nullptr && live_n) ? __uint_as_float((uint32_t)__ldg(a.bias + n) << 16) : 0.f;
+            const int which = tn == tile_first ? 0 : 1;
+            float* mine = a.partial + ((2 * cta + which) * kRecRows + row) * a.Mp;
+            if (ok && !warp_wait(smem_u32(&sh.acc_full[seg & 1]), (uint32_t)(seg >> 1) & 1u, abort)) {
+                if (lane == 0) stop_all(sh, a.ws);
+                ok = false;
+            }
+            if (ok) {
+                tc_fence_after();
+                const uint32_t tacc = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((seg & 1) * BT);
+#pragma unroll 1
+                for (int c = 0; c < BT / 16 && 16 * c < a.M; ++c) {
+                    uint32_t v[16];
+                    tmem_ld16(tacc + 16u * c, v);
+                    if (whole) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int64_t m = 16 * c + e;
+                            if (m < a.M && live_n) {
+                                const float f = __uint_as_float(v[e]);
+                                a.y[m * a.N + n] = __bfloat16_as_ushort(
+                                    __float2bfloat16_rn(a.bias != nullptr ? __fadd_rn(f, bias) : f));
+                            }
+                        }
+                    } else {  // 16 partial sums of this row: four 16-byte stores (rows of x fastest)
+#pragma unroll
+                        for (int e = 0; e < 16; e += 4)
+                            asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(mine + 16 * c + e), "r"(v[e]),
+                                         "r"(v[e + 1]), "r"(v[e + 2]), "r"(v[e + 3])
+                                         : "memory");
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&sh.acc_empty[seg & 1]));
+            }
+            if (whole) continue;
+            // a shared tile: every CTA of it counts itself (also after a failed wait, so that
+            // the counter always returns to zero) with one acquire-release add after the four
+            // warps' partial sums (the add releases them, and in the last CTA acquires everyone
+            // else's); the last one adds all partial sums in CTA order
+            const int64_t c_lo = sm_cta_of(a, tn * nk), c_hi = sm_cta_of(a, (tn + 1) * nk - 1);
+            epi_bar_sync();
+            if (tid == 0) {
+                unsigned prev;
+                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(a.counters + tn) : "memory");
+                const bool last = prev == (unsigned)(c_hi - c_lo);
+                if (last) atomicExch(a.counters + tn, 0u);
+                sh.last = last ? 1u : 0u;
+            }
+            epi_bar_sync();
+            const bool last = sh.last != 0u;
+            epi_bar_sync();  // everyone has read sh.last before the next tile rewrites it
+            if (last && ok && !*abort) {
+                // float4 units (row, 4 rows of x) of the slots, added strictly in CTA order
+                const int64_t stride = 2 * kRecRows * a.Mp;  // floats from one CTA's slots to the next
+                const float* p0 = a.partial + 2 * c_lo * kRecRows * a.Mp;
+                const float* p_lo = sm_item_begin(a, c_lo) >= tn * nk ? p0 : p0 + kRecRows * a.Mp;
+                const int nc = (int)(c_hi - c_lo);
+                const int mq = (int)((a.M + 3) / 4);  // float4 units per row that hold rows of x
+                const int units = kRecRows * mq;
+                auto finish_unit = [&](int u, float4 f) {  // bias, one rounding to bf16, store
+                    const int ur = u / mq, m0 = 4 * (u - ur * mq);
+                    const int64_t nn = tn * kRecRows + ur;
+                    if (nn >= a.N) return;
+                    const float bb = a.bias != nullptr ? __uint_as_float((uint32_t)__ldg(a.bias + nn) << 16) : 0.f;
+                    const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (m0 + e < a.M)
+                            a.y[(m0 + e) * a.N + nn] =
+                                __bfloat16_as_ushort(__float2bfloat16_rn(a.bias != nullptr ? __fadd_rn(fv[e], bb) : fv[e]));
+                };
+                auto unit_src = [&](int k, int u) {  // contributor k's float4 of unit u
+                    const int ur = u / mq, um = u - ur * mq;
+                    return (k == 0 ? p_lo : p0 + k * stride) + (int64_t)ur * a.Mp + 4 * um;
+                };
+                constexpr int kStage = (C::kRecOff + kRingR * kSmRecSlotBytes) / (4 * 128 * 16);  // contributors that fit
+                static_assert(kStage >= 2, "staging room");
+                if ((tn + 1) * nk >= i1 && nc < kStage) {
+                    // This CTA's last segment: its MMAs have all completed, so every x box and
+                    // record copy has landed and been read, and both rings are idle
+                    small_reduce_staged(a.M, a.N, a.Mp, a.bias, a.y, tn, base, p_lo, p0, stride, nc, mq, tid);
+                } else
+                // two units per thread at a time with two contributors' loads in flight
+                for (int u0 = tid; u0 < units; u0 += 2 * 128) {
+                    float4 f[2];
+                    int64_t off[2];
+                    bool have[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int u = u0 + 128 * h;
+                        have[h] = u < units;
+                        const int ur = have[h] ? u / mq : 0, um = have[h] ? u - ur * mq : 0;
+                        off[h] = (int64_t)ur * a.Mp + 4 * um;
+                        f[h] = have[h] ? __ldcg(reinterpret_cast<const float4*>(p_lo + off[h])) : make_float4(0, 0, 0, 0);
+                    }
+                    for (int k0 = 1; k0 <= nc; k0 += 2) {
+                        float4 v[2][2];
+#pragma unroll
+                        for (int k = 0; k < 2; ++k)
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+                                if (have[h] && k0 + k <= nc)
+                                    v[h][k] = __ldcg(reinterpret_cast<const float4*>(p0 + (k0 + k) * stride + off[h]));
+#pragma unroll
+                        for (int k = 0; k < 2; ++k)
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+                                if (have[h] && k0 + k <= nc) {
+                                    f[h].x = __fadd_rn(f[h].x, v[h][k].x);
+                                    f[h].y = __fadd_rn(f[h].y, v[h][k].y);
+                                    f[h].z = __fadd_rn(f[h].z, v[h][k].z);
+                                    f[h].w = __fadd_rn(f[h].w, v[h][k].w);
+                                }
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        if (have[h]) finish_unit(u0 + 128 * h, f[h]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kSmMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kSmTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
 // Up to 8 rows of x: the CUDA cores.  With so few rows an MMA (128 weight rows x 16 of K per
 // instruction, ~50 ns to issue whatever its N) does almost no work for its cost, and the call
 // is bound by the number of MMAs; on the CUDA cores it is bound by reading the packed weight.
@@ -1219,7 +1882,12 @@ nvfp4_status gemm_smem_optin() {
             cudaFuncSetAttribute(w4a16_linear_ts_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  TsCfg<128>::kSmemBytes) != cudaSuccess ||
             cudaFuncSetAttribute(w4a16_linear_ts_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 TsCfg<64>::kSmemBytes) != cudaSuccess)
+                                 TsCfg<64>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(w4a16_small_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SmCfg<16>::kSmemBytes) != cudaSuccess ||
+            // all of the SM's configurable memory as shared memory, so that two CTAs fit
+            cudaFuncSetAttribute(w4a16_small_kernel<16>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         g_smem_set[dev] = true;
     }
@@ -1270,13 +1938,25 @@ int64_t split_workspace_bytes(int64_t M, int64_t N, int splits) {
     return partial_offset(tiles) + (int64_t)splits * tiles * 128 * 128 * 4;
 }
 
-// How a call runs.  Up to 8 rows of x: the CUDA cores (w4a16_gemv_kernel), MT = M rounded up
-// to 1, 2, 4 or 8 rows.  Otherwise the weight in shared memory (w4a16_linear_kernel) for up to 128 rows of
-// x with K split over several CTAs per tile (a weight with few output tiles, and a workspace
-// with room for the partial sums), and for up to 32 rows unsplit; everything else with the
-// weight in tensor memory (w4a16_linear_ts_kernel).  With few rows of x both kernels are
-// bound by the rate at which one thread issues MMAs (~50 ns per 128 x N x 16 step, whatever
-// N), so they only differ in fixed costs: measured, the shared-memory kernel is ~0.8 us
+// The small kernel's grid (two CTAs per SM, never more CTAs than items) and workspace: the
+// status block, one counter per 128-row tile, then two fp32 partial-sum slots of 128 x Mp per
+// CTA (Mp = M rounded up to 16).
+int64_t small_grid(int64_t N, int64_t K, int sms) {
+    const int64_t items = ((N + kRecRows - 1) / kRecRows) * (((K + kBK - 1) / kBK + kSmAtoms - 1) / kSmAtoms);
+    return items < 2 * (int64_t)sms ? items : 2 * (int64_t)sms;
+}
+int64_t small_workspace_bytes(int64_t M, int64_t N, int64_t K, int sms) {
+    return partial_offset((N + 127) / 128) + 2 * small_grid(N, K, sms) * ((M + 15) / 16 * 16) * kRecRows * 4;
+}
+
+// How a call runs.  Up to 8 rows of x with a workspace that holds the partial sums: the
+// small kernel (w4a16_small_kernel), BT = 16.  Otherwise one row
+// of x takes the CUDA cores (w4a16_gemv_kernel); up to 128 rows the weight in shared memory
+// (w4a16_linear_kernel) with K split over several CTAs per tile (a weight with few output
+// tiles, and a workspace with room for the partial sums), and up to 32 rows unsplit;
+// everything else the weight in tensor memory (w4a16_linear_ts_kernel).  With few rows of x
+// the last two are bound by the rate at which one thread issues MMAs with x as the 128-row
+// operand, so they only differ in fixed costs: measured, the shared-memory kernel is ~0.8 us
 // faster up to 32 rows, the tensor-memory one ~4 us faster at 128.
 //
 // Tensor-memory tiles are 128 weight rows by bt rows of x.  Up to 128 rows of x, bt is M
@@ -1285,14 +1965,15 @@ int64_t split_workspace_bytes(int64_t M, int64_t N, int splits) {
 // fixed cost of a stage does not shrink with the MMAs), so 128-row tiles pay only where
 // they fill SMs that would idle.
 struct Plan {
-    int kind;    // 0: weight in shared memory, 1: in tensor memory, 2: CUDA cores
+    int kind;    // 0: weight in shared memory, 1: in tensor memory, 2: CUDA cores, 3: small kernel
     int bt;      // rows of x per output tile
-    int splits;  // CTAs per output tile over K
+    int splits;  // CTAs per output tile over K; for the small kernel, the CTAs sharing the weight
 };
 
 Plan make_plan(int64_t M, int64_t N, int64_t K, int64_t workspace_bytes, int sms, bool cuda_cores = true) {
-    if (cuda_cores && M <= kGemvMaxRows && (N + kGemvRows - 1) / kGemvRows <= 0x7FFFFFFFll)
-        return Plan{2, M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8)), 1};
+    if (M <= kSmMaxRows && workspace_bytes >= small_workspace_bytes(M, N, K, sms))
+        return Plan{3, 16, (int)small_grid(N, K, sms)};
+    if (cuda_cores && M <= 1 && (N + kGemvRows - 1) / kGemvRows <= 0x7FFFFFFFll) return Plan{2, 1, 1};
     int splits = M > kMmaM ? 1 : split_count(M, N, K, sms);
     if (splits > 1 && workspace_bytes < split_workspace_bytes(M, N, splits)) splits = 1;
     if (M <= kMmaM && (splits > 1 || M <= 32)) return Plan{0, kMmaM, splits};
@@ -1339,6 +2020,7 @@ NVFP4_API int64_t nvfp4_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     int sms = 0;
     if (sm_count_w4(&sms) != NVFP4_OK) sms = 148;
     const Plan plan = make_plan(M, N, K, (int64_t)1 << 62, sms);
+    if (plan.kind == 3) return small_workspace_bytes(M, N, K, sms);
     return plan.kind == 0 && plan.splits > 1 ? split_workspace_bytes(M, N, plan.splits) : (int64_t)sizeof(Workspace);
 }
 
@@ -1393,6 +2075,54 @@ static nvfp4_status w4a16_linear_ts(EncodeTiledFn encode, const void* x, int64_t
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// Up to 8 rows of x: the small kernel over the whole weight (make_plan, small_grid).
+static nvfp4_status w4a16_linear_small(EncodeTiledFn encode, const void* x, int64_t M, int64_t K, const uint8_t* tiled,
+                                       const float* d_global_scale, int64_t N, const void* bias, void* y,
+                                       void* d_workspace, uint64_t selftest_ns, int bt, int64_t grid,
+                                       nvfp4_stream_t stream) {
+    const int64_t tiles_n = (N + kRecRows - 1) / kRecRows;
+    // x as a [M, K] bf16 tensor, boxes of M rounded up to 8 rows (at most bt) x 64 columns,
+    // 128-byte swizzle, zero fill past the end of K: the rows of a stage's box past it are
+    // never written, and the accumulator columns they feed are rows of y past M, not stored.
+    CUtensorMap map;
+    std::memset(&map, 0, sizeof(map));
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const int box_rows = (int)((M + 7) / 8 * 8) < bt ? (int)((M + 7) / 8 * 8) : bt;
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return NVFP4_ERR_ARG;
+    SmallArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.tiled = tiled;
+    a.d_gs = d_global_scale;
+    a.bias = static_cast<const uint16_t*>(bias);
+    a.y = static_cast<uint16_t*>(y);
+    a.ws = static_cast<Workspace*>(d_workspace);
+    a.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(d_workspace) + counters_offset());
+    a.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(d_workspace) + partial_offset(tiles_n));
+    a.M = M;
+    a.Mp = (M + 15) / 16 * 16;
+    a.N = N;
+    a.kt = (K + kBK - 1) / kBK;
+    a.nk = (a.kt + kSmAtoms - 1) / kSmAtoms;
+    a.items = tiles_n * a.nk;
+    a.grid = grid;
+    a.box_bytes = (uint32_t)box_rows * kBK * 2;
+    a.selftest_ns = selftest_ns;
+    // No CTA waits for another (a shared tile is finished by whichever of its CTAs arrives
+    // last), so the grid needs no co-residency and takes a plain launch.
+    const dim3 g((unsigned)grid), b(kSmThreads);
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (bt != 16) return NVFP4_ERR_ARG;
+    w4a16_small_kernel<16><<<g, b, SmCfg<16>::kSmemBytes, st>>>(map, a);
+    note_launch();
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
 NVFP4_API nvfp4_status nvfp4_w4a16_plan(int64_t M, int64_t N, int64_t K, int64_t workspace_bytes, int sms,
                                         int* kernel, int* rows_per_tile, int* splits) {
     if (M < 0 || !weight_shape_ok(N, K) || M > 0x7FFFFF00ll) return NVFP4_ERR_SHAPE;
@@ -1434,6 +2164,9 @@ static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const
     if (st != NVFP4_OK) return st;
     // the self-test needs a kernel with barrier waits: not the CUDA-core one
     const Plan plan = make_plan(M, N, K, workspace_bytes, sms, selftest_ns == 0);
+    if (plan.kind == 3)
+        return w4a16_linear_small(encode, x, M, K, tiled, d_global_scale, N, bias, y, d_workspace, selftest_ns, plan.bt,
+                                  plan.splits, stream);
     if (plan.kind == 2) {
         LinearArgs a;
         std::memset(&a, 0, sizeof(a));
@@ -1450,14 +2183,7 @@ static nvfp4_status w4a16_linear_impl(const void* x, int64_t M, int64_t K, const
         const unsigned grid = (unsigned)((N + kGemvRows - 1) / kGemvRows);
         const uint16_t* xh = static_cast<const uint16_t*>(x);
         cudaStream_t cst = reinterpret_cast<cudaStream_t>(stream);
-        if (plan.bt == 1)
-            w4a16_gemv_kernel<1><<<grid, 32 * kGemvWarps, 0, cst>>>(xh, a);
-        else if (plan.bt == 2)
-            w4a16_gemv_kernel<2><<<grid, 32 * kGemvWarps, 0, cst>>>(xh, a);
-        else if (plan.bt == 4)
-            w4a16_gemv_kernel<4><<<grid, 32 * kGemvWarps, 0, cst>>>(xh, a);
-        else
-            w4a16_gemv_kernel<8><<<grid, 32 * kGemvWarps, 0, cst>>>(xh, a);
+        w4a16_gemv_kernel<1><<<grid, 32 * kGemvWarps, 0, cst>>>(xh, a);
         note_launch();
         return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
     }

@@ -634,20 +634,22 @@ def nvfp4_w4a16_selftest_timeout(x: torch.Tensor, tiled: torch.Tensor, global_sc
 
 
 def nvfp4_w4a16_workspace_bytes(M: int, N: int, K: int) -> int:
-    """Workspace bytes with which nvfp4_w4a16_linear may split K on this shape (current
-    device), at least WORKSPACE_BYTES; -1 if the shape is refused."""
+    """Workspace bytes with which nvfp4_w4a16_linear takes its fastest plan on this shape
+    (current device: room for the partial sums of a split K or of the small kernel), at least
+    WORKSPACE_BYTES; -1 if the shape is refused."""
     return int(_c_w4a16_workspace_bytes(M, N, K))
 
 
 def nvfp4_w4a16_plan(M: int, N: int, K: int, workspace_bytes: int, sms: int) -> tuple[str, int, int]:
     """How nvfp4_w4a16_linear runs this shape with a workspace of workspace_bytes on a device
-    with `sms` SMs: where the decoded weight lives ("shared" or "tensor" memory, or "cores":
-    registers of the CUDA-core kernel), the rows of x per output tile, and the CTAs per tile
-    over K.  Host only, no GPU needed."""
+    with `sms` SMs: which kernel ("small": up to 8 rows of x, the weight shared evenly by two
+    CTAs per SM; "shared" or "tensor": where the larger kernels keep the decoded weight;
+    "cores": the CUDA-core kernel for one row), the rows of x per output tile, and the CTAs
+    per tile over K (for "small": the CTAs that share the weight).  Host only, no GPU needed."""
     kernel, rows, splits = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
     _check(_c_w4a16_plan(M, N, K, workspace_bytes, sms, ctypes.byref(kernel), ctypes.byref(rows),
                          ctypes.byref(splits)), "nvfp4_w4a16_plan")
-    return ("shared", "tensor", "cores")[kernel.value], rows.value, splits.value
+    return ("shared", "tensor", "cores", "small")[kernel.value], rows.value, splits.value
 
 
 def nvfp4_w4a16_workspace(M: int, N: int, K: int, device) -> torch.Tensor:

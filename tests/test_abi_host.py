@@ -258,29 +258,40 @@ BIG_WS = 1 << 40
 
 
 @pytest.mark.parametrize("M,N,K,ws,sms,want", [
-    # up to 8 rows of x: the CUDA cores, rows rounded up to 1, 2, 4 or 8, never split
-    (1, 4096, 4096, BIG_WS, 148, ("cores", 1, 1)),
-    (2, 14336, 4096, BIG_WS, 148, ("cores", 2, 1)),
-    (3, 4096, 4096, 256, 148, ("cores", 4, 1)),
-    (5, 13, 16, BIG_WS, 148, ("cores", 8, 1)),
-    (8, 4096, 4096, BIG_WS, 148, ("cores", 8, 1)),
-    (9, 14336, 4096, BIG_WS, 148, ("shared", 128, 1)),
-    # up to 128 rows of x on a weight with few tiles: split K in shared memory when the
-    # workspace has room (148 SMs / 32 tiles = 4 CTAs per tile, at least 8 atoms each) ...
+    # up to 8 rows of x with room for the partial sums: the small kernel, 16-row tiles of x,
+    # shared by min(2 x SMs, items) CTAs (items: 128 weight rows x 128 of K)
+    (1, 4096, 4096, BIG_WS, 148, ("small", 16, 296)),        # 32 x 32 items
+    (2, 14336, 4096, BIG_WS, 148, ("small", 16, 296)),
+    (8, 4096, 4096, BIG_WS, 148, ("small", 16, 296)),
+    (8, 4096, 4096, BIG_WS, 132, ("small", 16, 264)),
+    (8, 4096, 512, BIG_WS, 148, ("small", 16, 128)),         # 32 x 4 items: one CTA each
+    (5, 13, 16, BIG_WS, 148, ("small", 16, 1)),              # one item
+    # from 9 rows on the kernels with x as the 128-row operand (below), with the same room
+    (9, 13, 16, BIG_WS, 148, ("shared", 128, 1)),
     (16, 4096, 4096, BIG_WS, 148, ("shared", 128, 4)),
-    (100, 4096, 4096, BIG_WS, 148, ("shared", 128, 4)),
     (16, 4096, 4096, BIG_WS, 132, ("shared", 128, 4)),
-    # ... and without room, or with too little K to split (8 atoms): shared memory up to 32
-    # rows, tensor memory above, tiles of 64 or 128 rows of x
-    (16, 4096, 4096, 256, 148, ("shared", 128, 1)),
-    (100, 4096, 4096, 256, 148, ("tensor", 128, 1)),
-    (16, 4096, 512, BIG_WS, 148, ("shared", 128, 1)),
-    (100, 4096, 512, BIG_WS, 148, ("tensor", 128, 1)),
-    # a weight with 112 tiles is never split (148 / 112 = 1)
-    (16, 14336, 4096, BIG_WS, 148, ("shared", 128, 1)),
+    (17, 14336, 4096, BIG_WS, 148, ("shared", 128, 1)),
     (32, 14336, 4096, BIG_WS, 148, ("shared", 128, 1)),
     (33, 14336, 4096, BIG_WS, 148, ("tensor", 64, 1)),
     (64, 14336, 4096, BIG_WS, 148, ("tensor", 64, 1)),
+    # without that room: one row of x takes the CUDA cores, never split ...
+    (1, 4096, 4096, 256, 148, ("cores", 1, 1)),
+    (1, 14336, 4096, 256, 148, ("cores", 1, 1)),
+    # ... more rows shared memory up to 32 rows (K split only with room for it), tensor
+    # memory above, tiles of 64 or 128 rows of x
+    (2, 4096, 4096, 256, 148, ("shared", 128, 1)),
+    (3, 4096, 4096, 256, 148, ("shared", 128, 1)),
+    (16, 4096, 4096, 256, 148, ("shared", 128, 1)),
+    (16, 14336, 4096, 256, 148, ("shared", 128, 1)),
+    (33, 14336, 4096, 256, 148, ("tensor", 64, 1)),
+    (64, 14336, 4096, 256, 148, ("tensor", 64, 1)),
+    (100, 4096, 4096, 256, 148, ("tensor", 128, 1)),
+    # 65 to 128 rows of x on a weight with few tiles: split K in shared memory when the
+    # workspace has room (148 SMs / 32 tiles = 4 CTAs per tile, at least 8 atoms each) ...
+    (100, 4096, 4096, BIG_WS, 148, ("shared", 128, 4)),
+    (100, 4096, 4096, BIG_WS, 132, ("shared", 128, 4)),
+    # ... not with too little K to split (8 atoms), nor on a weight with 112 tiles (148 / 112 = 1)
+    (100, 4096, 512, BIG_WS, 148, ("tensor", 128, 1)),
     (65, 14336, 4096, BIG_WS, 148, ("tensor", 128, 1)),
     (128, 14336, 4096, BIG_WS, 148, ("tensor", 128, 1)),
     # more rows: 256-row tiles unless 128-row tiles need no more waves of one CTA per SM
@@ -314,19 +325,28 @@ def test_w4a16_plan_refusals(lib):
 
 
 def test_w4a16_workspace_sizes(lib):
-    """Host-only (148 SMs assumed without a GPU): the status block alone unless the plan
-    splits K; with a split, the block, one counter per 128-column tile (rounded up to 256
-    bytes) and splits x tiles x 128 x 128 fp32 partial sums."""
+    """Host-only (148 SMs assumed without a GPU): for the small kernel (up to 8 rows of x)
+    the status block, one counter per 128-row tile (rounded up to 256 bytes) and 2 x G x 128 x
+    16 fp32 partial sums (two slots per CTA), G = min(296, items); for a split K (65 to 128
+    rows) the block, the counters and splits x tiles x 128 x 128 fp32 partial sums; otherwise
+    the block alone."""
     f = lib.nvfp4_w4a16_workspace_bytes
     f.restype = ctypes.c_int64
     f.argtypes = [ctypes.c_int64] * 3
-    assert f(1, 4096, 4096) == 256          # CUDA cores: never split
-    assert f(8, 4096, 4096) == 256
+
+    def head(tiles):
+        return -(-(256 + 4 * tiles) // 256) * 256
+
+    assert f(1, 4096, 4096) == head(32) + 2 * 296 * 128 * 16 * 4
+    assert f(8, 4096, 4096) == head(32) + 2 * 296 * 128 * 16 * 4
+    assert f(2, 14336, 4096) == head(112) + 2 * 296 * 128 * 16 * 4
+    assert f(8, 4096, 512) == head(32) + 2 * 128 * 128 * 16 * 4   # 128 items: 128 CTAs
+    assert f(17, 14336, 4096) == 256       # 112 tiles: not split
+    assert f(16, 4096, 4096) == head(32) + 4 * 32 * 128 * 128 * 4     # split K, 4 CTAs per tile
     assert f(200, 4096, 4096) == 256        # tensor memory: never split
-    assert f(16, 14336, 4096) == 256        # 112 tiles: 148 // 112 = 1 CTA per tile
-    tiles = 32                              # 4096 outputs; 148 // 32 = 4 splits, K has 64 atoms
-    assert f(16, 4096, 4096) == -(-(256 + 4 * tiles) // 256) * 256 + 4 * tiles * 128 * 128 * 4
-    assert f(16, 4096, 1088) == -(-(256 + 4 * tiles) // 256) * 256 + 2 * tiles * 128 * 128 * 4  # 17 atoms: 2
+    assert f(100, 14336, 4096) == 256       # 112 tiles: 148 // 112 = 1 CTA per tile
+    assert f(100, 4096, 4096) == head(32) + 4 * 32 * 128 * 128 * 4    # 4 splits, K has 64 atoms
+    assert f(100, 4096, 1088) == head(32) + 2 * 32 * 128 * 128 * 4    # 17 atoms: 2
     assert f(16, 4096, 24) == -1 and f(-1, 4096, 64) == -1
 
 

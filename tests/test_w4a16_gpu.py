@@ -185,39 +185,91 @@ def test_out_parameter_and_leading_dimensions():
     _assert_within_bound(bits(y).reshape(6, 64), bits(x).reshape(6, 256), packed, scales, gs, None, "3-D x")
 
 
-@pytest.mark.parametrize("M,K,N,with_bias", [
-    (1, 4096, 4096, False),
-    (2, 1040, 200, True),     # K % 64 == 16: the last atom has one block
-    (3, 64, 300, True),       # one atom of K: seven of the eight warps have none
-    (4, 16, 13, False),       # one block of K, 13 live rows of one 32-row tile
-    (5, 1040, 333, True),     # 5 and 6 rows: the 8-row instance with 3 and 2 rows idle,
-    (6, 4112, 77, False),     # N not a multiple of 32, K % 64 != 0
-    (7, 4160, 1000, True),
-    (8, 1088, 128, False),
-    (8, 4096, 14336, True),   # the pages' MLP weight
+@pytest.mark.parametrize("K,N,with_bias", [
+    (4096, 4096, False),
+    (1040, 200, True),      # K % 64 == 16: the last atom has one block
+    (64, 300, True),        # one atom of K: seven of the eight warps have none
+    (16, 13, False),        # one block of K, 13 live rows of one 32-row tile
+    (4160, 1000, True),
+    (4096, 14336, True),    # the pages' MLP weight
 ])
-def test_cuda_core_rows_match_oracle(M, K, N, with_bias):
-    """Up to 8 rows of x the call runs on the CUDA cores (decode in registers, fp32 FMAs):
-    every output within the bound, and a second call bit-identical (the partial sums are
-    added in a fixed order)."""
-    assert nv.nvfp4_w4a16_plan(M, N, K, nv.WORKSPACE_BYTES, 148)[0] == "cores"
-    rng = np.random.default_rng(M * 11 + K + N)
-    x = synthetic.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
-    packed, scales, gs = _weight(N, K, M + 2 * K + N)
+def test_cuda_core_row_matches_oracle(K, N, with_bias):
+    """One row of x with a workspace too small for the small kernel runs on the CUDA cores
+    (decode in registers, fp32 FMAs): every output within the bound, and a second call
+    bit-identical (the partial sums are added in a fixed order)."""
+    assert nv.nvfp4_w4a16_plan(1, N, K, nv.WORKSPACE_BYTES, 148)[0] == "cores"
+    rng = np.random.default_rng(K + N)
+    x = synthetic.to_bf16_bits(rng.standard_normal((1, K)).astype(np.float32))
+    packed, scales, gs = _weight(N, K, 2 * K + N)
     bias = synthetic.to_bf16_bits(rng.standard_normal(N).astype(np.float32)) if with_bias else None
     tiled = nv.nvfp4_w4a16_pack(packed, scales)
     xd, bd = to_dev(x), (to_dev(bias) if with_bias else None)
-    y1 = nv.nvfp4_w4a16_linear(xd, tiled, gs, N, bias=bd)
-    y2 = nv.nvfp4_w4a16_linear(xd, tiled, gs, N, bias=bd)
+    ws = nv.new_workspace("cuda")
+    y1 = nv.nvfp4_w4a16_linear(xd, tiled, gs, N, bias=bd, workspace=ws)
+    y2 = nv.nvfp4_w4a16_linear(xd, tiled, gs, N, bias=bd, workspace=ws)
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
-    _assert_within_bound(bits(y1), x, packed, scales, gs, bias, f"CUDA cores, {M} rows")
+    _assert_within_bound(bits(y1), x, packed, scales, gs, bias, "CUDA cores, 1 row")
+
+
+@pytest.mark.parametrize("M,K,N,with_bias", [
+    (1, 4096, 4096, False),
+    (1, 4096, 14336, True),     # the pages' MLP weight at one token
+    (2, 1040, 200, True),       # 17 atoms of K: each tile's last item has one atom; N ragged
+    (5, 64, 300, True),         # one atom of K: every item has one atom
+    (6, 4112, 77, False),       # K % 64 == 16, 3 CTAs ... on one 77-row tile
+    (7, 4160, 1000, False),
+    (8, 1088, 128, True),
+    (7, 16, 13, False),         # one item (one block of K), 13 live rows: one CTA
+    (8, 4096, 14336, True),
+    (8, 128, 18944, True),      # 148 tiles of one item: every tile whole in one CTA
+    (8, 8192, 256, True),       # 2 tiles of 64 items on 128 CTAs: each tile shared by 64 CTAs
+    (3, 256, 128000, False),    # 1000 tiles of 2 items on 296 CTAs: ranges of ~6.8 items span a
+                                # shared first tile, whole middle tiles and a shared last tile
+    (8, 128, 40000, True),      # 313 tiles of one item on 296 CTAs: ranges of 1 or 2 whole tiles
+    # from 9 rows on: the kernels with x as the 128-row operand, the same workspace
+    (9, 8192, 256, True),
+    (13, 16, 13, False),
+    (16, 4096, 14336, True),
+    (17, 2048, 1000, True),
+    (31, 704, 384, False),
+    (32, 4096, 4096, True),
+    (33, 1040, 200, True),
+    (48, 4096, 14336, False),
+    (64, 4096, 4096, True),
+    (64, 128, 18944, True),
+    (16, 128, 40000, True),
+])
+def test_full_workspace_matches_oracle(M, K, N, with_bias):
+    """A full workspace: up to 8 rows of x the small kernel (the weight's items shared evenly
+    by two CTAs per SM; a tile shared by several CTAs is finished by the last from the fp32
+    partial sums in CTA order), more rows the kernels with x as the 128-row operand (K split
+    where the plan says so).  Every output within the bound, a second call on the same
+    workspace bit-identical, and every tile counter back at zero."""
+    plan = nv.nvfp4_w4a16_plan(M, N, K, 1 << 40, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert (plan[0] == "small") == (M <= 8)
+    rng = np.random.default_rng(M * 13 + K + N)
+    x = synthetic.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    packed, scales, gs = _weight(N, K, M + 3 * K + N)
+    bias = synthetic.to_bf16_bits(rng.standard_normal(N).astype(np.float32)) if with_bias else None
+    tiled = nv.nvfp4_w4a16_pack(packed, scales)
+    xd, bd = to_dev(x), (to_dev(bias) if with_bias else None)
+    ws = nv.nvfp4_w4a16_workspace(M, N, K, "cuda")
+    y1 = nv.nvfp4_w4a16_linear(xd, tiled, gs, N, bias=bd, workspace=ws)
+    y2 = nv.nvfp4_w4a16_linear(xd, tiled, gs, N, bias=bd, workspace=ws)
+    torch.cuda.synchronize()
+    assert nv.nvfp4_workspace_check(ws[:nv.WORKSPACE_BYTES]) == 0
+    tiles = -(-N // 128)
+    assert not ws[nv.WORKSPACE_BYTES:nv.WORKSPACE_BYTES + 4 * tiles].any().item(), "tile counters left non-zero"
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    _assert_within_bound(bits(y1), x, packed, scales, gs, bias, f"{plan[0]} kernel, {M}x{K} . {N}x{K}^T")
 
 
 @pytest.mark.parametrize("K,N", [(64, 300), (1088, 200)])
-def test_cuda_core_decode_is_exact_through_one_hot_rows(K, N):
-    """8 rows of x, each a one-hot row picking one column of the weight: every output is
-    1 * w plus exact zeros, so it must be the oracle's dequantized weight bit for bit (up to
-    the sign of a zero sum), for random code and scale bytes."""
+def test_small_and_cuda_core_decode_is_exact_through_one_hot_rows(K, N):
+    """8 rows of x (the small kernel), each a one-hot row picking one column of the weight:
+    every output is 1 * w plus exact zeros, so it must be the oracle's dequantized weight bit
+    for bit (up to the sign of a zero sum), for random code and scale bytes.  The same rows
+    one at a time with a minimal workspace go through the CUDA-core kernel."""
     rng = np.random.default_rng(K + N)
     packed = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
     scales = rng.integers(0, 256, size=(N, K // 16), dtype=np.uint8)
@@ -227,12 +279,17 @@ def test_cuda_core_decode_is_exact_through_one_hot_rows(K, N):
     cols = rng.choice(K, size=8, replace=False)
     x = np.zeros((8, K), dtype=np.float32)
     x[np.arange(8), cols] = 1.0
-    y = bits(nv.nvfp4_w4a16_linear(to_dev(synthetic.to_bf16_bits(x)), tiled, torch.tensor([gs], device="cuda"), N))
+    g = torch.tensor([gs], device="cuda")
+    xd = to_dev(synthetic.to_bf16_bits(x))
     want = oracle.dequantize(packed, scales, gs, N, K)[:, cols].T
-    y = np.where((y & 0x7FFF) == 0, 0, y)
     want = np.where((want & 0x7FFF) == 0, 0, want)
-    bad = np.argwhere(y != want)
-    assert bad.size == 0, f"{len(bad)} decoded weights differ, first {bad[:3].tolist()}"
+    ws = nv.new_workspace("cuda")
+    for name, y in (("small kernel", bits(nv.nvfp4_w4a16_linear(xd, tiled, g, N))),
+                    ("CUDA cores", np.concatenate([bits(nv.nvfp4_w4a16_linear(xd[r:r + 1], tiled, g, N, workspace=ws))
+                                                   for r in range(8)]))):
+        y = np.where((y & 0x7FFF) == 0, 0, y)
+        bad = np.argwhere(y != want)
+        assert bad.size == 0, f"{name}: {len(bad)} decoded weights differ, first {bad[:3].tolist()}"
 
 
 def test_empty_rows_launch_nothing():
@@ -245,9 +302,9 @@ def test_empty_rows_launch_nothing():
     assert nv.nvfp4_kernel_launch_count() == before
 
 
-@pytest.mark.parametrize("M,K", [(9, 4096), (16, 4096), (32, 4096), (33, 4096), (100, 4096), (16, 1088), (9, 4160)])
+@pytest.mark.parametrize("M,K", [(65, 4096), (100, 4096), (128, 4096), (100, 1088), (65, 4160)])
 def test_split_k_for_few_rows(M, K):
-    """9 to 128 rows of x on a weight with few output tiles (4096 x 4096: 32 tiles): the call
+    """65 to 128 rows of x on a weight with few output tiles (4096 x 4096: 32 tiles): the call
     splits K over several CTAs when the workspace is large enough; the result is within the
     bound, bit-identical from call to call (the partial sums are added in a fixed order),
     and the workspace can be reused.  Without the room to split, the same call runs
@@ -272,13 +329,13 @@ def test_split_k_for_few_rows(M, K):
     _assert_within_bound(bits(y3), x, packed, scales, gs, bias, f"unsplit, {M} rows")
 
 
-@pytest.mark.parametrize("M,N", [(16, 4096), (700, 512), (4096, 2560)])
+@pytest.mark.parametrize("M,N", [(8, 4096), (100, 4096), (700, 512), (4096, 2560)])
 def test_bounded_wait_reports_a_timeout_and_the_context_recovers(M, N):
     """A wait on a barrier that nothing completes (2 ms limit) runs out: the call reports
     NVFP4_ERR_TIMEOUT through the workspace instead of hanging, every role stops, and the
-    next call on the same context and workspace is correct.  16 rows take the split-K
-    path, 700 rows the tensor-memory weight with 128-row tiles of x, 4096 rows on 2560
-    outputs its 256-row tiles."""
+    next call on the same context and workspace is correct.  8 rows take the small kernel,
+    100 rows the split-K path, 700 rows the tensor-memory weight with 128-row tiles of x,
+    4096 rows on 2560 outputs its 256-row tiles."""
     K = 1024
     rng = np.random.default_rng(M + N)
     x = synthetic.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
