@@ -535,6 +535,7 @@ def run_sweep(args):
         y = torch.empty_like(x)
         packed, scales, gs = nv.nvfp4_quantize(x, amax)
         packed32, scales32, _ = nv.nvfp4_quantize(x, amax, block=32)
+        packed_f, scales_f = nv.nvfp4_quantize_f32scale(x)
         scales_mma = torch.empty(nv.mma_scale_bytes(M, N), dtype=torch.uint8, device=dev)
         t = {
             "amax": (2.0, timed(lambda: nv.nvfp4_amax(x, out=amax, workspace=ws))),
@@ -551,12 +552,16 @@ def run_sweep(args):
             "quantize_b32": (2.53125, timed(lambda: nv.nvfp4_quantize(x, amax, packed32, scales32, gs, block=32))),
             "dequantize_b32": (2.53125, timed(lambda: nv.nvfp4_dequantize(packed32, scales32, gs, out=y,
                                                                           block=32))),
+            # the fp32-scale flavour: blocks of 32, a 4-byte scale per block (1/8 byte per element)
+            "fake_quant_f32s": (4.0, timed(lambda: nv.nvfp4_fake_quant_f32scale(x, out=y))),
+            "quantize_f32s": (2.625, timed(lambda: nv.nvfp4_quantize_f32scale(x, packed_f, scales_f))),
+            "dequantize_f32s": (2.625, timed(lambda: nv.nvfp4_dequantize_f32scale(packed_f, scales_f, out=y))),
         }
         rec = {"workload": name, "shape": [M, N], "bytes": 2 * n}
         for k, (bpe, sec) in t.items():
             rec[k] = {"us": sec * 1e6, "GB/s": n * bpe / sec / 1e9, "frac": n * bpe / sec / 1e9 / peak}
         rows.append(rec)
-        del x, y, packed, scales, scales_mma, packed32, scales32
+        del x, y, packed, scales, scales_mma, packed32, scales32, packed_f, scales_f
     # the q/k/v siblings: shared amax + fake-quant of all three in one call
     qkv = [synthetic.activation_normal_device(s, 98, dev) for s in ((4096, 4096), (1024, 4096), (1024, 4096))]
     outs = [torch.empty_like(t) for t in qkv]
@@ -568,7 +573,8 @@ def run_sweep(args):
                                                "frac": n * 6.0 / sec / 1e9 / peak}})
 
     cols = ["amax", "fake_quant", "fake_quant_with_own_amax", "quantize", "quantize_with_own_amax", "quantize_mma",
-            "dequantize", "fake_quant_b32", "quantize_b32", "dequantize_b32"]
+            "dequantize", "fake_quant_b32", "quantize_b32", "dequantize_b32", "fake_quant_f32s", "quantize_f32s",
+            "dequantize_f32s"]
     print(f"peak {peak:.1f} GB/s ({peak_src}); GB/s of algorithmic bytes (frac of peak); L2 flushed by a read")
     print("| workload | shape | " + " | ".join(cols) + " |")
     print("|---|---|" + "---|" * len(cols))

@@ -331,6 +331,34 @@ nvfp4_status nvfp4_dequantize_bs(const uint8_t* packed, const uint8_t* scales, c
 nvfp4_status nvfp4_fake_quant_bs(const void* x, void* y, int64_t M, int64_t N, int block, const float* d_amax,
                                  nvfp4_stream_t stream);
 
+/* ---- the fp32-scale flavour: blocks of 32, one fp32 scale each ---------------------- */
+
+/* [FP4OPT] constants block (the FLOAT4_BLOCK_SIZE comment): 32-element blocks with an fp32
+ * scale are the OCP MXFP4 flavour of the same quantizer.  The page defines it no further;
+ * these calls read it as quantize_weight_to_float4's steps (block_size = 32) with the block
+ * scale kept in fp32 instead of being rounded to E4M3, so there is no per-tensor scale:
+ *   scale   = fl(block_amax / 6)           block_amax = max |x| over 32 consecutive elements
+ *   divisor = max(scale, 1e-12)            (the page's clamp against a zero block)
+ *   code    = E2M1 index of fl(x / divisor) (nearest, ties to even, saturating at 6) + 8 if
+ *             fl(x / divisor) < 0
+ *   y       = bf16_rn(fl(LUT[code] * scale))   (decode: the stored scale, no clamp)
+ * Layouts: x / y bf16 [M, N] row-major, contiguous, 32-byte aligned; rows padded with zeros
+ * to P = 32 ceil(N / 32) columns; packed uint8 [M, P/2] (16-byte aligned; byte j of a row:
+ * element 2j in the low nibble), scales fp32 [M, P/32] (4-byte aligned), both written for
+ * the padded layout, y only for the N real columns.  All pointers are device memory owned
+ * by the caller.  One pass, no workspace: nothing outside the outputs is written.
+ * Errors: NVFP4_ERR_SHAPE (M or N < 0, sizes past the element limit), NVFP4_ERR_NULL,
+ * NVFP4_ERR_ALIGN, NVFP4_ERR_ARG (fake-quant: x and y overlap without being the same
+ * buffer; y == x fake-quantizes in place).  M == 0 or N == 0 launches nothing.  Enqueue
+ * one kernel each. */
+nvfp4_status nvfp4_quantize_f32scale(const void* x, int64_t M, int64_t N, uint8_t* packed, float* scales,
+                                     nvfp4_stream_t stream);
+
+nvfp4_status nvfp4_dequantize_f32scale(const uint8_t* packed, const float* scales, int64_t M, int64_t N, void* y,
+                                       nvfp4_stream_t stream);
+
+nvfp4_status nvfp4_fake_quant_f32scale(const void* x, void* y, int64_t M, int64_t N, nvfp4_stream_t stream);
+
 /* ---- forward of a Linear layer on a packed weight (W4A16) ---------------------------- */
 
 /* The weight's operand form: the packed weight cut into 128-row x 64-column tiles, one

@@ -17,7 +17,7 @@ LIB = os.path.join(PKG, "libnvfp4.so")
 SOURCES = [os.path.join(CSRC, "nvfp4_kernels.cu"), os.path.join(CSRC, "nvfp4_w4a16.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("nvfp4_device.cuh", "nvfp4_runtime.h", "nvfp4_stream.cuh",
                                                   "nvfp4_reduce.cuh", "nvfp4_encode.cuh", "nvfp4_ragged.cuh",
-                                                  "nvfp4_strided.cuh")]
+                                                  "nvfp4_strided.cuh", "nvfp4_f32scale.cuh")]
 DEPS += [os.path.join(INCLUDE, "nvfp4.h")]
 
 NVCC_FLAGS = [

@@ -39,6 +39,7 @@
 #include "nvfp4_encode.cuh"
 #include "nvfp4_ragged.cuh"
 #include "nvfp4_strided.cuh"
+#include "nvfp4_f32scale.cuh"
 
 namespace nvfp4 {
 namespace {
@@ -917,6 +918,99 @@ NVFP4_API nvfp4_status nvfp4_fake_quant_bs(const void* x, void* y, int64_t M, in
         case 16: return fake_quant_impl<16>(x, y, M, N, d_amax, stream);
         default: return NVFP4_ERR_ARG;
     }
+}
+
+// ---------------------------------------------------------------------------------------
+// The fp32-scale flavour (blocks of 32, one fp32 scale per block, no global scale):
+// nvfp4_f32scale.cuh.  One pass each; whole-block rows stream, other rows are staged.
+
+NVFP4_API nvfp4_status nvfp4_quantize_f32scale(const void* x, int64_t M, int64_t N, uint8_t* packed, float* scales,
+                                               nvfp4_stream_t stream) {
+    constexpr int kE = 2 * kF32sW;
+    int64_t numel = 0;
+    nvfp4_status st = check_matrix(M, N, &numel, kE);
+    if (st != NVFP4_OK) return st;
+    if (numel > 0 && (x == nullptr || packed == nullptr || scales == nullptr)) return NVFP4_ERR_NULL;
+    if (numel > 0 && (!aligned(x, 32) || !aligned(packed, 16) || !aligned(scales, 4))) return NVFP4_ERR_ALIGN;
+    if (numel == 0) return NVFP4_OK;
+    int grid = 1;
+    if (N % kE != 0) {
+        const Ragged R = ragged_of(M, N, kE);
+        st = ragged_smem_optin(quantize_f32s_ragged_kernel, kStageBytes);
+        if (st != NVFP4_OK) return st;
+        st = grid_for(reinterpret_cast<const void*>(&quantize_f32s_ragged_kernel), R.total, ragged_u<kF32sW>(),
+                      NVFP4_GRID_Q, &grid, kStageBytes);
+        if (st != NVFP4_OK) return st;
+        quantize_f32s_ragged_kernel<<<grid, kThreads, kStageBytes, cs(stream)>>>(static_cast<const uint8_t*>(x), R,
+                                                                               packed, scales);
+        return after_launch();
+    }
+    const int64_t nblk = numel / kE;
+    st = grid_for(reinterpret_cast<const void*>(&quantize_f32s_kernel), nblk, unroll_for<kF32sW>(kUnrollQ),
+                  NVFP4_GRID_Q, &grid, 0, NVFP4_SMALL_Q);
+    if (st != NVFP4_OK) return st;
+    quantize_f32s_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x), nblk, packed, scales);
+    return after_launch();
+}
+
+NVFP4_API nvfp4_status nvfp4_dequantize_f32scale(const uint8_t* packed, const float* scales, int64_t M, int64_t N,
+                                                 void* y, nvfp4_stream_t stream) {
+    constexpr int kE = 2 * kF32sW;
+    int64_t numel = 0;
+    nvfp4_status st = check_matrix(M, N, &numel, kE);
+    if (st != NVFP4_OK) return st;
+    if (numel > 0 && (packed == nullptr || scales == nullptr || y == nullptr)) return NVFP4_ERR_NULL;
+    if (numel > 0 && (!aligned(packed, 16) || !aligned(scales, 4) || !aligned(y, 32))) return NVFP4_ERR_ALIGN;
+    if (numel == 0) return NVFP4_OK;
+    int grid = 1;
+    if (N % kE != 0) {
+        const Ragged R = ragged_of(M, N, kE);
+        st = ragged_smem_optin(dequantize_f32s_ragged_kernel, kStageBytes);
+        if (st != NVFP4_OK) return st;
+        st = grid_for(reinterpret_cast<const void*>(&dequantize_f32s_ragged_kernel), R.total, ragged_u<kF32sW>(),
+                      NVFP4_GRID_DEC, &grid, kStageBytes);
+        if (st != NVFP4_OK) return st;
+        dequantize_f32s_ragged_kernel<<<grid, kThreads, kStageBytes, cs(stream)>>>(packed, scales,
+                                                                                 static_cast<uint8_t*>(y), R);
+        return after_launch();
+    }
+    const int64_t nblk = numel / kE;
+    st = grid_for(reinterpret_cast<const void*>(&dequantize_f32s_kernel), nblk, unroll_for<kF32sW>(kUnrollDecode),
+                  NVFP4_GRID_DEC, &grid, 0, NVFP4_SMALL_DEC);
+    if (st != NVFP4_OK) return st;
+    dequantize_f32s_kernel<<<grid, kThreads, 0, cs(stream)>>>(packed, scales, static_cast<uint8_t*>(y), nblk);
+    return after_launch();
+}
+
+NVFP4_API nvfp4_status nvfp4_fake_quant_f32scale(const void* x, void* y, int64_t M, int64_t N,
+                                                 nvfp4_stream_t stream) {
+    constexpr int kE = 2 * kF32sW;
+    int64_t numel = 0;
+    nvfp4_status st = check_matrix(M, N, &numel, kE);
+    if (st != NVFP4_OK) return st;
+    if (numel > 0 && (x == nullptr || y == nullptr)) return NVFP4_ERR_NULL;
+    if (numel > 0 && (!aligned(x, 32) || !aligned(y, 32))) return NVFP4_ERR_ALIGN;
+    if (x != y && numel > 0 && overlap(x, y, numel * 2)) return NVFP4_ERR_ARG;
+    if (numel == 0) return NVFP4_OK;
+    int grid = 1;
+    if (N % kE != 0) {
+        const Ragged R = ragged_of(M, N, kE);
+        st = ragged_smem_optin(fake_quant_f32s_ragged_kernel, kStageBytes);
+        if (st != NVFP4_OK) return st;
+        st = grid_for(reinterpret_cast<const void*>(&fake_quant_f32s_ragged_kernel), R.total, ragged_u<kF32sW>(),
+                      NVFP4_GRID_FQ, &grid, kStageBytes);
+        if (st != NVFP4_OK) return st;
+        fake_quant_f32s_ragged_kernel<<<grid, kThreads, kStageBytes, cs(stream)>>>(static_cast<const uint8_t*>(x),
+                                                                                 static_cast<uint8_t*>(y), R);
+        return after_launch();
+    }
+    const int64_t nblk = numel / kE;
+    st = grid_for(reinterpret_cast<const void*>(&fake_quant_f32s_kernel), nblk, unroll_for<kF32sW>(kUnrollFq),
+                  NVFP4_GRID_FQ, &grid, 0, NVFP4_SMALL_FQ);
+    if (st != NVFP4_OK) return st;
+    fake_quant_f32s_kernel<<<grid, kThreads, 0, cs(stream)>>>(static_cast<const uint8_t*>(x),
+                                                              static_cast<uint8_t*>(y), nblk);
+    return after_launch();
 }
 
 NVFP4_API nvfp4_status nvfp4_fake_quant_siblings(int k, const void* const* xs, void* const* ys, const int64_t* Ms,

@@ -70,6 +70,9 @@ _c_fake_quant_strided = _sig("nvfp4_fake_quant_strided", [_vp, _i64, _vp, _i64, 
 _c_quantize_bs = _sig("nvfp4_quantize_bs", [_vp, _i64, _i64, ctypes.c_int, _vp, _vp, _vp, _vp, _vp])
 _c_dequantize_bs = _sig("nvfp4_dequantize_bs", [_vp, _vp, _vp, _i64, _i64, ctypes.c_int, _vp, _vp])
 _c_fake_quant_bs = _sig("nvfp4_fake_quant_bs", [_vp, _vp, _i64, _i64, ctypes.c_int, _vp, _vp])
+_c_quantize_f32scale = _sig("nvfp4_quantize_f32scale", [_vp, _i64, _i64, _vp, _vp, _vp])
+_c_dequantize_f32scale = _sig("nvfp4_dequantize_f32scale", [_vp, _vp, _i64, _i64, _vp, _vp])
+_c_fake_quant_f32scale = _sig("nvfp4_fake_quant_f32scale", [_vp, _vp, _i64, _i64, _vp])
 _c_fake_quant_siblings = _sig("nvfp4_fake_quant_siblings",
                               [ctypes.c_int, ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_i64),
                                ctypes.POINTER(_i64), _vp, _vp])
@@ -440,6 +443,68 @@ def nvfp4_fake_quant(x: torch.Tensor, amax: torch.Tensor, out: torch.Tensor | No
         else:
             st = _c_fake_quant_bs(x.data_ptr(), out.data_ptr(), M, N, block, amax.data_ptr(), _stream(x.device))
         _check(st, "nvfp4_fake_quant")
+    return out
+
+
+# ---- the fp32-scale flavour (blocks of 32, one fp32 scale each, no global scale) ----
+
+def nvfp4_quantize_f32scale(x: torch.Tensor, packed: torch.Tensor | None = None,
+                            scales: torch.Tensor | None = None):
+    """bf16 [..., N] -> (packed uint8 [..., P/2], fp32 block scales [..., P/32]),
+    P = 32 * ceil(N / 32): blocks of 32 with scale = block amax / 6 kept in fp32 (the
+    fp32-scale flavour of quantize_weight_to_float4; no per-tensor scale)."""
+    M, N = _matrix(x)
+    B = padded_blocks(N, 32)
+    lead = tuple(x.shape[:-1])
+    if packed is None:
+        packed = torch.empty(lead + (16 * B,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(lead + (B,), dtype=torch.float32, device=x.device)
+    _cuda(packed, "packed", torch.uint8)
+    _cuda(scales, "scales", torch.float32)
+    if packed.numel() != M * 16 * B or scales.numel() != M * B:
+        raise RuntimeError("packed / scales have the wrong number of elements")
+    with torch.cuda.device(x.device):
+        _check(_c_quantize_f32scale(x.data_ptr(), M, N, packed.data_ptr(), scales.data_ptr(), _stream(x.device)),
+               "nvfp4_quantize_f32scale")
+    return packed, scales
+
+
+def nvfp4_dequantize_f32scale(packed: torch.Tensor, scales: torch.Tensor, n_cols: int | None = None,
+                              out: torch.Tensor | None = None) -> torch.Tensor:
+    """(packed [..., P/2], fp32 scales [..., P/32]) -> bf16 [..., n_cols]: bf16(LUT * scale),
+    cropped to n_cols (default P)."""
+    _cuda(packed, "packed", torch.uint8)
+    _cuda(scales, "scales", torch.float32)
+    P = packed.shape[-1] * 2
+    N = P if n_cols is None else int(n_cols)
+    if padded_blocks(N, 32) * 32 != P:
+        raise RuntimeError(f"n_cols={N} does not match packed rows of {P // 2} bytes")
+    M = math.prod(packed.shape[:-1])
+    if scales.numel() != M * (P // 32):
+        raise RuntimeError("scales has the wrong number of elements")
+    if out is None:
+        out = torch.empty(tuple(packed.shape[:-1]) + (N,), dtype=torch.bfloat16, device=packed.device)
+    _cuda(out, "out", torch.bfloat16)
+    if out.numel() != M * N:
+        raise RuntimeError("out has the wrong number of elements")
+    with torch.cuda.device(packed.device):
+        _check(_c_dequantize_f32scale(packed.data_ptr(), scales.data_ptr(), M, N, out.data_ptr(),
+                                      _stream(packed.device)), "nvfp4_dequantize_f32scale")
+    return out
+
+
+def nvfp4_fake_quant_f32scale(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 -> bf16: dequantize_f32scale(quantize_f32scale(x)) in one pass; ``out`` may be x."""
+    M, N = _matrix(x)
+    if out is None:
+        out = torch.empty(x.shape, dtype=x.dtype, device=x.device)
+    _cuda(out, "out", torch.bfloat16)
+    if out.numel() != x.numel():
+        raise RuntimeError("out has the wrong number of elements")
+    with torch.cuda.device(x.device):
+        _check(_c_fake_quant_f32scale(x.data_ptr(), out.data_ptr(), M, N, _stream(x.device)),
+               "nvfp4_fake_quant_f32scale")
     return out
 
 

@@ -108,3 +108,36 @@ def oracle_dequantize_rows(packed, scales, gs, threads=None, n_cols=None, block=
     with ThreadPoolExecutor(threads) as pool:
         list(pool.map(work, _row_chunks(M, threads * 2)))
     return y
+
+
+def oracle_quantize_f32s_rows(x_bits, threads=None):
+    """oracle.quantize_f32scale on row ranges from several threads (rows are independent)."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    threads = threads or HOST_THREADS
+    M, N = x_bits.shape
+    B = (N + 31) // 32
+    packed = np.empty((M, 16 * B), dtype=np.uint8)
+    scales = np.empty((M, B), dtype=np.float32)
+
+    def work(rr):
+        r0, r1 = rr
+        packed[r0:r1], scales[r0:r1] = oracle.quantize_f32scale(x_bits[r0:r1])
+    with ThreadPoolExecutor(threads) as pool:
+        list(pool.map(work, _row_chunks(M, threads * 2)))
+    return packed, scales
+
+
+def oracle_dequantize_f32s_rows(packed, scales, n_cols, threads=None):
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    threads = threads or HOST_THREADS
+    M = packed.shape[0]
+    y = np.empty((M, n_cols), dtype=np.uint16)
+
+    def work(rr):
+        r0, r1 = rr
+        y[r0:r1] = oracle.dequantize_f32scale(packed[r0:r1], scales[r0:r1], r1 - r0, n_cols)
+    with ThreadPoolExecutor(threads) as pool:
+        list(pool.map(work, _row_chunks(M, threads * 2)))
+    return y

@@ -35,7 +35,8 @@ def test_header_declares_the_entry_points():
                      "nvfp4_w4a16_pack", "nvfp4_w4a16_tiled_bytes", "nvfp4_quantize_fused",
                      "nvfp4_amax_accumulate", "nvfp4_w4a16_workspace_bytes", "nvfp4_amax_strided",
                      "nvfp4_quantize_strided", "nvfp4_fake_quant_strided", "nvfp4_w4a16_plan",
-                     "nvfp4_status_string", "nvfp4_kernel_launch_count"]:
+                     "nvfp4_status_string", "nvfp4_kernel_launch_count", "nvfp4_quantize_f32scale",
+                     "nvfp4_dequantize_f32scale", "nvfp4_fake_quant_f32scale"]:
         assert required in names
 
 
@@ -145,6 +146,24 @@ def test_validation_errors_launch_nothing(lib):
         (ERR_SHAPE, "nvfp4_quantize_bs", _p(A32), _i(1 << 56), _i(33), _c(32), amax, _p(A32), _p(A32), gs, S),
         (ERR_SHAPE, "nvfp4_fake_quant_bs", _p(A32), _p(A32 + 4096), _i(2), _i(-32), _c(32), amax, S),
         (ERR_NULL, "nvfp4_fake_quant_bs", _p(A32), _p(A32 + 4096), _i(2), _i(64), _c(32), _p(0), S),
+        # fp32-scale flavour: quantize(x, M, N, packed, scales), dequantize(packed, scales, M, N, y),
+        # fake_quant(x, y, M, N); codes 16-byte aligned, scales 4, bf16 tensors 32
+        (ERR_NULL, "nvfp4_quantize_f32scale", _p(A32), _i(2), _i(64), _p(A32), _p(0), S),
+        (ERR_ALIGN, "nvfp4_quantize_f32scale", _p(A32), _i(2), _i(64), _p(A8), _p(A32), S),
+        (ERR_ALIGN, "nvfp4_quantize_f32scale", _p(A32), _i(2), _i(64), _p(A32), _p(A32 + 2), S),
+        (ERR_ALIGN, "nvfp4_quantize_f32scale", _p(A32 + 16), _i(2), _i(64), _p(A32), _p(A32), S),
+        (ERR_SHAPE, "nvfp4_quantize_f32scale", _p(A32), _i(-1), _i(64), _p(A32), _p(A32), S),
+        (ERR_SHAPE, "nvfp4_quantize_f32scale", _p(A32), _i(1 << 56), _i(33), _p(A32), _p(A32), S),
+        (NVFP4_OK, "nvfp4_quantize_f32scale", _p(0), _i(0), _i(64), _p(0), _p(0), S),
+        (ERR_NULL, "nvfp4_dequantize_f32scale", _p(A32), _p(A32), _i(2), _i(64), _p(0), S),
+        (ERR_ALIGN, "nvfp4_dequantize_f32scale", _p(A32), _p(A32), _i(2), _i(64), _p(A8), S),
+        (ERR_ALIGN, "nvfp4_dequantize_f32scale", _p(A32), _p(A32 + 1), _i(2), _i(64), _p(A32), S),
+        (ERR_SHAPE, "nvfp4_dequantize_f32scale", _p(A32), _p(A32), _i(2), _i(-64), _p(A32), S),
+        (NVFP4_OK, "nvfp4_dequantize_f32scale", _p(0), _p(0), _i(3), _i(0), _p(0), S),
+        (ERR_ARG, "nvfp4_fake_quant_f32scale", _p(A32), _p(A32 + 64), _i(2), _i(64), S),   # y inside x's span
+        (ERR_NULL, "nvfp4_fake_quant_f32scale", _p(0), _p(A32), _i(2), _i(64), S),
+        (ERR_ALIGN, "nvfp4_fake_quant_f32scale", _p(A32), _p(A8), _i(2), _i(64), S),
+        (ERR_SHAPE, "nvfp4_fake_quant_f32scale", _p(A32), _p(A32), _i(-2), _i(64), S),
         # W4A16: linear(x, M, K, tiled, gs, N, bias, y, workspace), pack(packed, scales, N, K, tiled)
         (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(24), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), _i(256), S),
         (ERR_SHAPE, "nvfp4_w4a16_linear", _p(A32), _i(4), _i(0), _p(A32), gs, _i(8), _p(0), _p(A32), _p(A32), _i(256), S),
