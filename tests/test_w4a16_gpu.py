@@ -8,11 +8,12 @@ mag = sum_k |x_k| |w_k| (+ |bias|):
 
     |y - exact| <= 2^-8 |exact| + (1 + 2^-8) K 2^-23 mag
 
-(every bf16 x bf16 product is exact in fp32; an fp32 sum of K terms in any order, rounded
-or truncated, is within K 2^-23 mag of the exact sum; rounding the result to bf16 adds at
-most half an ulp, 2^-8 relative.)  Shapes span several tiles in both dimensions with
-ragged edges in M, N and K, the single-tile and single-row cases, and the pages' MLP
-weight (14336 x 4096) under 4096 tokens on sampled rows.
+(every bf16 x bf16 product is exact in fp32 within the normal fp32 range, which these
+inputs stay in; an fp32 sum of K terms in any order, rounded or truncated, is within
+K 2^-23 mag of the exact sum; rounding the result to bf16 adds at most half an ulp, 2^-8
+relative.)  Shapes span several tiles in both dimensions with ragged edges in M, N and K,
+the single-tile and single-row cases, and the pages' MLP weight (14336 x 4096) under 4096
+tokens, every output element.
 """
 import numpy as np
 import pytest
