@@ -494,23 +494,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     stop_all(sh, a.ws);
         }
     } else if (warp == kMmaWarp) {
-        if (lane == 0) {
-            bool ok = true;
-            // self-test of the bounded waits: the limit runs out, every role stops
-            if (a.selftest_ns != 0 && !mbar_wait(smem_u32(&sh.never), 0u, abort, false, a.selftest_ns)) {
-                stop_all(sh, a.ws);
+        // The whole warp runs the loop and its waits (warp-uniform control flow and operands);
+        // one elected lane issues the MMAs and the commits that track them.
+        bool ok = true;
+        // self-test of the bounded waits: the limit runs out, every role stops
+        if (a.selftest_ns != 0 &&
+            !__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&sh.never), 0u, abort, false, a.selftest_ns))) {
+            if (lane == 0) stop_all(sh, a.ws);
+            ok = false;
+        }
+        for (int kb = 0; ok && kb < nk; ++kb) {
+            const int sa = kb % kRingA, sb = kb % kRingB;
+            if (!warp_wait(smem_u32(&sh.a_full[sa]), (uint32_t)(kb / kRingA) & 1u, abort) ||
+                !warp_wait(smem_u32(&sh.b_full[sb]), (uint32_t)(kb / kRingB) & 1u, abort)) {
+                if (lane == 0) stop_all(sh, a.ws);
                 ok = false;
+                break;
             }
-            for (int kb = 0; ok && kb < nk; ++kb) {
-                const int sa = kb % kRingA, sb = kb % kRingB;
-                if (!mbar_wait(smem_u32(&sh.a_full[sa]), (uint32_t)(kb / kRingA) & 1u, abort) ||
-                    !mbar_wait(smem_u32(&sh.b_full[sb]), (uint32_t)(kb / kRingB) & 1u, abort)) {
-                    stop_all(sh, a.ws);
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const int na = min(kAtoms, (int)(a.kt - (int64_t)(kb0 + kb) * kAtoms));
+            tc_fence_after();
+            const int na = min(kAtoms, (int)(a.kt - (int64_t)(kb0 + kb) * kAtoms));
+            if (elect_one_sync()) {
 #pragma unroll
                 for (int t = 0; t < kAtoms; ++t) {
                     if (t >= na) break;
@@ -527,12 +530,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 umma_commit(smem_u32(&sh.a_empty[sa]));
                 umma_commit(smem_u32(&sh.b_empty[sb]));
             }
-            if (ok) {
-                umma_commit(smem_u32(&sh.accum));
-            } else {  // let the MMAs already issued finish before tensor memory is released
-                umma_commit(smem_u32(&sh.drain));
-                mbar_wait(smem_u32(&sh.drain), 0u, abort, true);
-            }
+            __syncwarp();
+        }
+        if (ok) {
+            if (elect_one_sync()) umma_commit(smem_u32(&sh.accum));
+        } else {  // let the MMAs already issued finish before tensor memory is released
+            if (elect_one_sync()) umma_commit(smem_u32(&sh.drain));
+            __syncwarp();
+            mbar_wait(smem_u32(&sh.drain), 0u, abort, true);
         }
         __syncwarp();
     } else {
@@ -920,38 +925,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     stop_all(sh, a.ws);
         }
     } else if (warp == kMmaWarp) {
-        if (lane == 0) {
+        // Up to 128 rows of x the whole warp runs the loop and its waits (warp-uniform control
+        // flow and operands) and one elected lane issues, as in the kernel above; measured on
+        // one box, 14336 x 4096 at 128 tokens 26.5 -> 24.3 us.  With 256-row tiles each stage's
+        // MMAs are long and the stage hand-off is on the critical path: there lane 0 alone runs
+        // the loop (the warp-wide waits and syncs measured 3-4 % slower at 1024-8192 tokens).
+        constexpr bool kUniform = BT <= 128;
+        auto wait_on = [&](uint32_t bar, uint32_t parity) {
+            return kUniform ? warp_wait(bar, parity, abort) : mbar_wait(bar, parity, abort);
+        };
+        if (kUniform || lane == 0) {
             bool ok = true;
-            if (a.selftest_ns != 0 && !mbar_wait(smem_u32(&sh.never), 0u, abort, false, a.selftest_ns)) {
-                stop_all(sh, a.ws);
+            if (a.selftest_ns != 0 &&
+                !(kUniform ? __all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&sh.never), 0u, abort, false, a.selftest_ns))
+                           : mbar_wait(smem_u32(&sh.never), 0u, abort, false, a.selftest_ns))) {
+                if (lane == 0) stop_all(sh, a.ws);
                 ok = false;
             }
             for (int kb = 0; ok && kb < nk; ++kb) {
                 const int sa = kb % kRingA, st = kb % kTsRingT;
-                if (!mbar_wait(smem_u32(&sh.a_full[sa]), (uint32_t)(kb / kRingA) & 1u, abort) ||
-                    !mbar_wait(smem_u32(&sh.w_full[st]), (uint32_t)(kb / kTsRingT) & 1u, abort)) {
-                    stop_all(sh, a.ws);
+                if (!wait_on(smem_u32(&sh.a_full[sa]), (uint32_t)(kb / kRingA) & 1u) ||
+                    !wait_on(smem_u32(&sh.w_full[st]), (uint32_t)(kb / kTsRingT) & 1u)) {
+                    if (lane == 0) stop_all(sh, a.ws);
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const int na = min(kTsAtoms, kt - kb * kTsAtoms);
+                if (!kUniform || elect_one_sync()) {
 #pragma unroll
-                for (int t = 0; t < kTsAtoms; ++t) {
-                    if (t >= na) break;
-                    const uint64_t bd = sw128_desc(sA0 + sa * kStageABytes + t * kAtomABytes);
-                    const uint32_t ta = tmem + (uint32_t)(kTsWCol + st * kTsSlotCols + t * (kBK / 2));
+                    for (int t = 0; t < kTsAtoms; ++t) {
+                        if (t >= na) break;
+                        const uint64_t bd = sw128_desc(sA0 + sa * kStageABytes + t * kAtomABytes);
+                        const uint32_t ta = tmem + (uint32_t)(kTsWCol + st * kTsSlotCols + t * (kBK / 2));
 #pragma unroll
-                    for (int j = 0; j < kBK / kUmmaK; ++j)  // 16 of K: 8 columns of A, 32 bytes of B
-                        umma_f16_ts(tmem, ta + 8u * j, bd + 2u * j, kIdesc, (kb | t | j) != 0 ? 1u : 0u);
+                        for (int j = 0; j < kBK / kUmmaK; ++j)  // 16 of K: 8 columns of A, 32 bytes of B
+                            umma_f16_ts(tmem, ta + 8u * j, bd + 2u * j, kIdesc, (kb | t | j) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(smem_u32(&sh.a_empty[sa]));
+                    umma_commit(smem_u32(&sh.w_empty[st]));
                 }
-                umma_commit(smem_u32(&sh.a_empty[sa]));
-                umma_commit(smem_u32(&sh.w_empty[st]));
+                if (kUniform) __syncwarp();
             }
             if (ok) {
-                umma_commit(smem_u32(&sh.accum));
+                if (!kUniform || elect_one_sync()) umma_commit(smem_u32(&sh.accum));
             } else {
-                umma_commit(smem_u32(&sh.drain));
+                if (!kUniform || elect_one_sync()) umma_commit(smem_u32(&sh.drain));
+                if (kUniform) __syncwarp();
                 mbar_wait(smem_u32(&sh.drain), 0u, abort, true);
             }
         }
@@ -1143,10 +1163,6 @@ __device__ __forceinline__ void decode_block_tab(uint32_t c0, uint32_t c1, uint4
         o[4 * h + 2] = prmt(l47, h47, 0x5140u);
         o[4 * h + 3] = prmt(l47, h47, 0x7362u);
     }
-}
-
-__device__ __forceinline__ void decode_block_prmt(uint32_t c0, uint32_t c1, float sd, uint32_t* o) {
-    decode_block_tab(c0, c1, decode_tables(sd), o);
 }
 
 // ---------------------------------------------------------------------------------------
