@@ -403,13 +403,14 @@ nvfp4_status nvfp4_w4a16_pack(const uint8_t* packed, const uint8_t* scales, int6
  *           workspace.  Its first NVFP4_WORKSPACE_BYTES are a workspace as above: a bounded
  *           wait inside the kernel that runs out records NVFP4_ERR_TIMEOUT there
  *           (nvfp4_workspace_check; zero the whole workspace before reusing it then), the
- *           kernel stops and y is unspecified.  With at least nvfp4_w4a16_workspace_bytes(M,
- *           N, K) bytes, a call with at most 8 rows of x runs the small kernel (the weight
- *           cut into equal contiguous shares, two CTAs per SM) and one with at most 128 rows
- *           may split K over several CTAs per output tile: the CTAs that share a tile write
- *           fp32 partial sums there and the last to finish adds them in a fixed order (so
- *           results do not depend on timing) and leaves the tile's counter at zero again.
- *           With less, K is not split.
+ *           kernel stops and y is unspecified.  On a weight with at most one 128-row output
+ *           tile per two SMs and with at least nvfp4_w4a16_workspace_bytes(M, N, K) bytes, a
+ *           call with at most 8 rows of x runs the small kernel (the weight cut into equal
+ *           contiguous shares, two CTAs per SM) and one with at most 128 rows may split K
+ *           over several CTAs per output tile: the CTAs that share a tile write fp32 partial
+ *           sums there and the last to finish adds them in a fixed order (so results do not
+ *           depend on timing) and leaves the tile's counter at zero again.  With less, K is
+ *           not split.  (nvfp4_w4a16_plan states every rule.)
  * Errors: NVFP4_ERR_SHAPE (K, sizes past the 32-bit tensor-map limits), NVFP4_ERR_NULL,
  * NVFP4_ERR_ALIGN, NVFP4_ERR_ARG (tensor map rejected, workspace_bytes too small).  M == 0 or
  * N == 0 launches nothing.  Enqueues one kernel. */
@@ -439,18 +440,21 @@ int64_t nvfp4_w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
 /* How nvfp4_w4a16_linear runs x [M, K] . W[N, K]^T with a workspace of workspace_bytes on a
  * device with `sms` SMs (the decision that call takes with the current device's SM count).
  * Host only: launches nothing and needs no GPU.
- *   *kernel         3: the small kernel (at most 8 rows of x and a workspace of at least
- *                   nvfp4_w4a16_workspace_bytes: the weight's items of 128 rows x 128
- *                   columns cut into equal contiguous shares, two CTAs per SM, the weight
- *                   decoded into tensor memory as the MMA's 128-row operand); 2: the CUDA
- *                   cores, no tensor cores (one row of x, workspace too small for kernel 3);
- *                   0: the weight decoded into shared memory (split K, or 9 to 32 rows of
- *                   x); 1: the weight decoded into tensor memory (everything else)
+ *   *kernel         On a weight with at most one 128-row output tile per two SMs
+ *                   (2 ceil(N / 128) <= sms): 3, the small kernel, for at most 8 rows of x
+ *                   and a workspace of at least nvfp4_w4a16_workspace_bytes (the weight's
+ *                   items of 128 rows x 128 columns cut into equal contiguous shares, two
+ *                   CTAs per SM, the weight decoded into tensor memory as the MMA's 128-row
+ *                   operand); else 2, the CUDA cores without tensor cores, for one row of x.
+ *                   On a weight with more tiles: 1, the weight decoded into tensor memory,
+ *                   for at most 64 rows of x.  Otherwise 0, the weight decoded into shared
+ *                   memory, for up to 128 rows with K split or up to 32 rows unsplit; 1 for
+ *                   everything else.
  *   *rows_per_tile  rows of x per output tile: 16 for kernel 3;
  *                   1 for kernel 2 (tiles of 32 weight rows); 128 for kernel 0; for kernel 1,
- *                   64 or 128 up to 128 rows of x, above that 256, or 128 where 128-row tiles
- *                   need no more waves of one CTA per SM (tiles of kernels 0 and 1 cover 128
- *                   weight rows)
+ *                   64 up to 64 rows of x, 128 up to 128, above that 256, or 128 where
+ *                   128-row tiles need no more waves of one CTA per SM (tiles of kernels 0
+ *                   and 1 cover 128 weight rows)
  *   *splits         kernel 3: the CTAs that share the weight, G; kernel 0: CTAs per output
  *                   tile over K; 1 otherwise
  * Errors: NVFP4_ERR_SHAPE as nvfp4_w4a16_linear, NVFP4_ERR_NULL (an output pointer),

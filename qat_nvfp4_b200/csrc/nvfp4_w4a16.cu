@@ -1965,15 +1965,19 @@ int64_t small_workspace_bytes(int64_t M, int64_t N, int64_t K, int sms) {
     return partial_offset((N + 127) / 128) + 2 * small_grid(N, K, sms) * ((M + 15) / 16 * 16) * kRecRows * 4;
 }
 
-// How a call runs.  Up to 8 rows of x with a workspace that holds the partial sums: the
-// small kernel (w4a16_small_kernel), BT = 16.  Otherwise one row
-// of x takes the CUDA cores (w4a16_gemv_kernel); up to 128 rows the weight in shared memory
-// (w4a16_linear_kernel) with K split over several CTAs per tile (a weight with few output
-// tiles, and a workspace with room for the partial sums), and up to 32 rows unsplit;
-// everything else the weight in tensor memory (w4a16_linear_ts_kernel).  With few rows of x
-// the last two are bound by the rate at which one thread issues MMAs with x as the 128-row
-// operand, so they only differ in fixed costs: measured, the shared-memory kernel is ~0.8 us
-// faster up to 32 rows, the tensor-memory one ~4 us faster at 128.
+// How a call runs.  On a weight with few 128-row output tiles (at most one per two SMs, such
+// as 4096 x 4096's 32), up to 8 rows of x with a workspace that holds the partial sums take
+// the small kernel (w4a16_small_kernel, BT = 16: the weight spread evenly over two CTAs per
+// SM), one row without that room the CUDA cores (w4a16_gemv_kernel), and up to 128 rows the
+// weight in shared memory (w4a16_linear_kernel) with K split over several CTAs per tile when
+// the workspace has room for the partial sums.  On a weight with more tiles (14336 x 4096:
+// 112), up to 64 rows take the weight in tensor memory (w4a16_linear_ts_kernel) with 64-row
+// tiles of x.  Otherwise up to 32 rows the shared-memory kernel unsplit, everything else the
+// tensor-memory one.  Measured (ncu kernel time, one box): 14336 x 4096 at 1-32 tokens
+// 21.8-22.2 us with 64-row tensor-memory tiles against 22.5-23.0 in shared memory, 22.9-23.6
+// on the small kernel and 22.9 on the CUDA cores at one token; 4096 x 4096 at 1-4 tokens
+// 14.2-15.0 us on the small kernel against 15.9-18.6 otherwise (21 on tensor-memory tiles,
+// which cannot fill the SMs there without splitting K).
 //
 // Tensor-memory tiles are 128 weight rows by bt rows of x.  Up to 128 rows of x, bt is M
 // rounded up to 64 or 128.  Above that, bt = 256 unless 128-row tiles need no more waves of
@@ -1987,13 +1991,19 @@ struct Plan {
 };
 
 Plan make_plan(int64_t M, int64_t N, int64_t K, int64_t workspace_bytes, int sms, bool cuda_cores = true) {
-    if (M <= kSmMaxRows && workspace_bytes >= small_workspace_bytes(M, N, K, sms))
-        return Plan{3, 16, (int)small_grid(N, K, sms)};
-    if (cuda_cores && M <= 1 && (N + kGemvRows - 1) / kGemvRows <= 0x7FFFFFFFll) return Plan{2, 1, 1};
+    const int64_t tiles_n = (N + kRecRows - 1) / kRecRows;
+    if (2 * tiles_n <= sms) {
+        // few output tiles (at most one per two SMs): spread the weight itself
+        if (M <= kSmMaxRows && workspace_bytes >= small_workspace_bytes(M, N, K, sms))
+            return Plan{3, 16, (int)small_grid(N, K, sms)};
+        if (cuda_cores && M <= 1 && (N + kGemvRows - 1) / kGemvRows <= 0x7FFFFFFFll) return Plan{2, 1, 1};
+    } else if (M <= 64) {
+        // enough output tiles for the SMs: the weight in tensor memory, 64-row tiles of x
+        return Plan{1, 64, 1};
+    }
     int splits = M > kMmaM ? 1 : split_count(M, N, K, sms);
     if (splits > 1 && workspace_bytes < split_workspace_bytes(M, N, splits)) splits = 1;
     if (M <= kMmaM && (splits > 1 || M <= 32)) return Plan{0, kMmaM, splits};
-    const int64_t tiles_n = (N + kRecRows - 1) / kRecRows;
     int bt = M <= 64 ? 64 : 128;
     if (M > kMmaM) {
         const int64_t w256 = (tiles_n * ((M + 255) / 256) + sms - 1) / sms;

@@ -707,10 +707,11 @@ def nvfp4_w4a16_workspace_bytes(M: int, N: int, K: int) -> int:
 
 def nvfp4_w4a16_plan(M: int, N: int, K: int, workspace_bytes: int, sms: int) -> tuple[str, int, int]:
     """How nvfp4_w4a16_linear runs this shape with a workspace of workspace_bytes on a device
-    with `sms` SMs: which kernel ("small": up to 8 rows of x, the weight shared evenly by two
-    CTAs per SM; "shared" or "tensor": where the larger kernels keep the decoded weight;
-    "cores": the CUDA-core kernel for one row), the rows of x per output tile, and the CTAs
-    per tile over K (for "small": the CTAs that share the weight).  Host only, no GPU needed."""
+    with `sms` SMs: which kernel ("small": up to 8 rows of x on a weight with at most one
+    output tile per two SMs, the weight shared evenly by two CTAs per SM; "shared" or
+    "tensor": where the larger kernels keep the decoded weight; "cores": the CUDA-core kernel
+    for one row), the rows of x per output tile, and the CTAs per tile over K (for "small":
+    the CTAs that share the weight).  Host only, no GPU needed."""
     kernel, rows, splits = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
     _check(_c_w4a16_plan(M, N, K, workspace_bytes, sms, ctypes.byref(kernel), ctypes.byref(rows),
                          ctypes.byref(splits)), "nvfp4_w4a16_plan")

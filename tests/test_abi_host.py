@@ -277,34 +277,38 @@ BIG_WS = 1 << 40
 
 
 @pytest.mark.parametrize("M,N,K,ws,sms,want", [
-    # up to 8 rows of x with room for the partial sums: the small kernel, 16-row tiles of x,
-    # shared by min(2 x SMs, items) CTAs (items: 128 weight rows x 128 of K)
+    # a weight with at most one 128-row output tile per two SMs: up to 8 rows of x with room
+    # for the partial sums take the small kernel, 16-row tiles of x, shared by
+    # min(2 x SMs, items) CTAs (items: 128 weight rows x 128 of K) ...
     (1, 4096, 4096, BIG_WS, 148, ("small", 16, 296)),        # 32 x 32 items
-    (2, 14336, 4096, BIG_WS, 148, ("small", 16, 296)),
     (8, 4096, 4096, BIG_WS, 148, ("small", 16, 296)),
     (8, 4096, 4096, BIG_WS, 132, ("small", 16, 264)),
     (8, 4096, 512, BIG_WS, 148, ("small", 16, 128)),         # 32 x 4 items: one CTA each
     (5, 13, 16, BIG_WS, 148, ("small", 16, 1)),              # one item
-    # from 9 rows on the kernels with x as the 128-row operand (below), with the same room
+    (4, 9472, 4096, BIG_WS, 148, ("small", 16, 296)),        # 74 tiles: still one per two SMs
+    # ... one row without that room the CUDA cores ...
+    (1, 4096, 4096, 256, 148, ("cores", 1, 1)),
+    (1, 4096, 14336, 256, 148, ("cores", 1, 1)),
+    # ... and more rows the shared-memory weight, K split when the workspace has room
+    # (148 SMs / 32 tiles = 4 CTAs per tile, at least 8 atoms each), up to 32 rows unsplit
     (9, 13, 16, BIG_WS, 148, ("shared", 128, 1)),
     (16, 4096, 4096, BIG_WS, 148, ("shared", 128, 4)),
     (16, 4096, 4096, BIG_WS, 132, ("shared", 128, 4)),
-    (17, 14336, 4096, BIG_WS, 148, ("shared", 128, 1)),
-    (32, 14336, 4096, BIG_WS, 148, ("shared", 128, 1)),
-    (33, 14336, 4096, BIG_WS, 148, ("tensor", 64, 1)),
-    (64, 14336, 4096, BIG_WS, 148, ("tensor", 64, 1)),
-    # without that room: one row of x takes the CUDA cores, never split ...
-    (1, 4096, 4096, 256, 148, ("cores", 1, 1)),
-    (1, 14336, 4096, 256, 148, ("cores", 1, 1)),
-    # ... more rows shared memory up to 32 rows (K split only with room for it), tensor
-    # memory above, tiles of 64 or 128 rows of x
     (2, 4096, 4096, 256, 148, ("shared", 128, 1)),
     (3, 4096, 4096, 256, 148, ("shared", 128, 1)),
     (16, 4096, 4096, 256, 148, ("shared", 128, 1)),
-    (16, 14336, 4096, 256, 148, ("shared", 128, 1)),
-    (33, 14336, 4096, 256, 148, ("tensor", 64, 1)),
-    (64, 14336, 4096, 256, 148, ("tensor", 64, 1)),
+    (33, 4096, 4096, 256, 148, ("tensor", 64, 1)),
     (100, 4096, 4096, 256, 148, ("tensor", 128, 1)),
+    # a weight with more tiles (14336 x 4096: 112, 9600 x 4096: 75): up to 64 rows of x the
+    # tensor-memory weight with 64-row tiles, whatever the workspace
+    (1, 14336, 4096, BIG_WS, 148, ("tensor", 64, 1)),
+    (1, 14336, 4096, 256, 148, ("tensor", 64, 1)),
+    (2, 14336, 4096, BIG_WS, 148, ("tensor", 64, 1)),
+    (8, 9600, 4096, BIG_WS, 148, ("tensor", 64, 1)),
+    (17, 14336, 4096, BIG_WS, 148, ("tensor", 64, 1)),
+    (32, 14336, 4096, BIG_WS, 148, ("tensor", 64, 1)),
+    (64, 14336, 4096, 256, 148, ("tensor", 64, 1)),
+    (8, 14336, 4096, BIG_WS, 264, ("small", 16, 528)),       # 112 tiles on 264 SMs: few
     # 65 to 128 rows of x on a weight with few tiles: split K in shared memory when the
     # workspace has room (148 SMs / 32 tiles = 4 CTAs per tile, at least 8 atoms each) ...
     (100, 4096, 4096, BIG_WS, 148, ("shared", 128, 4)),
@@ -344,9 +348,10 @@ def test_w4a16_plan_refusals(lib):
 
 
 def test_w4a16_workspace_sizes(lib):
-    """Host-only (148 SMs assumed without a GPU): for the small kernel (up to 8 rows of x)
-    the status block, one counter per 128-row tile (rounded up to 256 bytes) and 2 x G x 128 x
-    16 fp32 partial sums (two slots per CTA), G = min(296, items); for a split K (65 to 128
+    """Host-only (148 SMs assumed without a GPU): for the small kernel (up to 8 rows of x on a
+    weight with at most 74 output tiles) the status block, one counter per 128-row tile
+    (rounded up to 256 bytes) and 2 x G x 128 x 16 fp32 partial sums (two slots per CTA),
+    G = min(296, items); for a split K (65 to 128
     rows) the block, the counters and splits x tiles x 128 x 128 fp32 partial sums; otherwise
     the block alone."""
     f = lib.nvfp4_w4a16_workspace_bytes
@@ -358,7 +363,8 @@ def test_w4a16_workspace_sizes(lib):
 
     assert f(1, 4096, 4096) == head(32) + 2 * 296 * 128 * 16 * 4
     assert f(8, 4096, 4096) == head(32) + 2 * 296 * 128 * 16 * 4
-    assert f(2, 14336, 4096) == head(112) + 2 * 296 * 128 * 16 * 4
+    assert f(2, 14336, 4096) == 256        # 112 tiles: the tensor-memory weight, nothing to split
+    assert f(4, 4096, 14336) == head(32) + 2 * 296 * 128 * 16 * 4  # the down-projection: 32 tiles
     assert f(8, 4096, 512) == head(32) + 2 * 128 * 128 * 16 * 4   # 128 items: 128 CTAs
     assert f(17, 14336, 4096) == 256       # 112 tiles: not split
     assert f(16, 4096, 4096) == head(32) + 4 * 32 * 128 * 128 * 4     # split K, 4 CTAs per tile

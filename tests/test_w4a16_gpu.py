@@ -192,12 +192,12 @@ def test_out_parameter_and_leading_dimensions():
     (64, 300, True),        # one atom of K: seven of the eight warps have none
     (16, 13, False),        # one block of K, 13 live rows of one 32-row tile
     (4160, 1000, True),
-    (4096, 14336, True),    # the pages' MLP weight
+    (14336, 4096, True),    # the pages' MLP down-projection (32 output tiles)
 ])
 def test_cuda_core_row_matches_oracle(K, N, with_bias):
-    """One row of x with a workspace too small for the small kernel runs on the CUDA cores
-    (decode in registers, fp32 FMAs): every output within the bound, and a second call
-    bit-identical (the partial sums are added in a fixed order)."""
+    """One row of x on a weight with few output tiles and a workspace too small for the small
+    kernel runs on the CUDA cores (decode in registers, fp32 FMAs): every output within the
+    bound, and a second call bit-identical (the partial sums are added in a fixed order)."""
     assert nv.nvfp4_w4a16_plan(1, N, K, nv.WORKSPACE_BYTES, 148)[0] == "cores"
     rng = np.random.default_rng(K + N)
     x = synthetic.to_bf16_bits(rng.standard_normal((1, K)).astype(np.float32))
@@ -213,21 +213,26 @@ def test_cuda_core_row_matches_oracle(K, N, with_bias):
 
 
 @pytest.mark.parametrize("M,K,N,with_bias", [
+    # weights with few output tiles (at most one per two SMs): the small kernel up to 8 rows
     (1, 4096, 4096, False),
-    (1, 4096, 14336, True),     # the pages' MLP weight at one token
+    (4, 14336, 4096, True),     # the pages' MLP down-projection at 4 tokens
     (2, 1040, 200, True),       # 17 atoms of K: each tile's last item has one atom; N ragged
     (5, 64, 300, True),         # one atom of K: every item has one atom
     (6, 4112, 77, False),       # K % 64 == 16, 3 CTAs ... on one 77-row tile
     (7, 4160, 1000, False),
     (8, 1088, 128, True),
     (7, 16, 13, False),         # one item (one block of K), 13 live rows: one CTA
-    (8, 4096, 14336, True),
-    (8, 128, 18944, True),      # 148 tiles of one item: every tile whole in one CTA
     (8, 8192, 256, True),       # 2 tiles of 64 items on 128 CTAs: each tile shared by 64 CTAs
-    (3, 256, 128000, False),    # 1000 tiles of 2 items on 296 CTAs: ranges of ~6.8 items span a
-                                # shared first tile, whole middle tiles and a shared last tile
-    (8, 128, 40000, True),      # 313 tiles of one item on 296 CTAs: ranges of 1 or 2 whole tiles
-    # from 9 rows on: the kernels with x as the 128-row operand, the same workspace
+    (8, 128, 9472, True),       # 74 tiles of one item on 74 CTAs: every tile whole in one CTA
+    (3, 4096, 9472, False),     # 74 tiles of 32 items on 296 CTAs: every tile shared
+    # more rows, or weights with many tiles (more than one per two SMs): the kernels with x as
+    # the 128-row operand; up to 64 rows on many tiles, the weight in tensor memory with
+    # 64-row tiles of x (boxes cut to the rows of x)
+    (1, 4096, 14336, True),     # the pages' MLP weight at one token
+    (8, 4096, 14336, True),
+    (3, 256, 128000, False),    # 1000 tiles of 2 atoms each
+    (8, 128, 40000, True),      # 313 tiles of one item, K of one stage
+    (5, 1040, 9728, True),      # 76 tiles, 17 atoms of K (the last stage half full)
     (9, 8192, 256, True),
     (13, 16, 13, False),
     (16, 4096, 14336, True),
@@ -241,13 +246,15 @@ def test_cuda_core_row_matches_oracle(K, N, with_bias):
     (16, 128, 40000, True),
 ])
 def test_full_workspace_matches_oracle(M, K, N, with_bias):
-    """A full workspace: up to 8 rows of x the small kernel (the weight's items shared evenly
-    by two CTAs per SM; a tile shared by several CTAs is finished by the last from the fp32
-    partial sums in CTA order), more rows the kernels with x as the 128-row operand (K split
-    where the plan says so).  Every output within the bound, a second call on the same
-    workspace bit-identical, and every tile counter back at zero."""
-    plan = nv.nvfp4_w4a16_plan(M, N, K, 1 << 40, torch.cuda.get_device_properties(0).multi_processor_count)
-    assert (plan[0] == "small") == (M <= 8)
+    """A full workspace: on a weight with at most one output tile per two SMs, up to 8 rows
+    of x take the small kernel (the weight's items shared evenly by two CTAs per SM; a tile
+    shared by several CTAs is finished by the last from the fp32 partial sums in CTA order);
+    everything else the kernels with x as the 128-row operand (K split where the plan says
+    so).  Every output within the bound, a second call on the same workspace bit-identical,
+    and every tile counter back at zero."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    plan = nv.nvfp4_w4a16_plan(M, N, K, 1 << 40, sms)
+    assert (plan[0] == "small") == (M <= 8 and 2 * (-(-N // 128)) <= sms)
     rng = np.random.default_rng(M * 13 + K + N)
     x = synthetic.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
     packed, scales, gs = _weight(N, K, M + 3 * K + N)
